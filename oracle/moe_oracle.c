@@ -1,0 +1,478 @@
+/*
+ * CPU oracle for the 4-bit routed-expert MoE layer of Step-5-Preview.
+ *
+ * TEST INFRASTRUCTURE ONLY.  This file is the plain, slow reference that the
+ * CUDA library is checked against.  Only the test suite, the smoke check and the
+ * CPU-baseline leg of the benchmark may load it.  It shares no code, header,
+ * table or constant with the CUDA library, and the library never calls it.
+ *
+ * Sources (web pages, by title and section):
+ *   [Int4]  "Step-5-Preview-Int4-g128": Recipe (RTN + clip search over 17 ratios
+ *           in [0.60, 1.00], search in bf16 = storage precision of the scale);
+ *           Tensor layout (experts fused as [352, out, in]).
+ *   [NVFP4] "Step-5-Preview-NVFP4-Local": Modifications item 2 (E2M1 pairs
+ *           U8 [352, R, K/2], weight_scale_2 F32 [352], BF16 activations);
+ *           Format (one E4M3 byte per 16 weights, [E, R, C]; dequant =
+ *           E2M1 value x E4M3 block scale x weight_scale_2; nibble order
+ *           "low nibble first" stated there for the CSF codes).
+ *   [Spark] "Step-5-Preview-Spark": At a glance (hidden 4096, 352 routed
+ *           experts, top-8, sigmoid router, 1 shared expert).
+ *   [Art]   "Step 5 Preview: 92 narrow layers, and a sparse indexer that scores
+ *           blocks of 8": The shape (8 routed experts per token plus one shared
+ *           expert, each a SwiGLU of width 1536).
+ *
+ * Readings where the pages are silent (each listed in the design notes):
+ *   - int4: divisor 7 with clamp [-8, 7]; ratios r_i = (24 + i) / 40, i = 0..16;
+ *     candidate scale bf16_rne((r_i * amax) / 7) in fp32; rounding error
+ *     sum (q*s - w)^2 accumulated in fp32 in index order; ties keep the larger
+ *     ratio; offset-binary nibbles u = q + 8, element 8c+j in bits 4j..4j+3
+ *     of word c.
+ *   - NVFP4: global g = amax / (6 * 448) per expert matrix (fp32);
+ *     block scale sb = e4m3_rne_sat(amax_b / (6 * g)); code =
+ *     e2m1_rne_sat(w / (e4m3(sb) * g)); even element in the low nibble.
+ *   - Router: l = sum_h x*Wr (fp32, index order) + bias; s = 1/(1+exp(-l))
+ *     (fp32); top-k by s, ties to the lower expert id, listed by descending s;
+ *     weights s / sum(selected s) (fp32).
+ *   - Layer: no routed scaling factor, no shared-expert gate, SwiGLU limit off.
+ *
+ * Floating point: quantiser decisions are taken in fp32 (the precision the
+ * CUDA library's own quantiser uses, so codes agree bit for bit); dequantised
+ * weights are exact in fp32; the layer forward accumulates in fp64.
+ *
+ * Parity pins: every function here is pinned by tests against facts the pages
+ * or mathematics fix (exhaustive code tables, library conversions, the pages'
+ * error table, closed forms, brute force).  The absolute layer output has no
+ * printed example on the pages; it is pinned only through those invariants and
+ * the brute-force dense mixture.
+ */
+#include <math.h>
+#include <stdint.h>
+#include <stdlib.h>
+#include <string.h>
+
+/* ------------------------------------------------------------------------ */
+/* bf16 <-> fp32                                                             */
+/* ------------------------------------------------------------------------ */
+
+float oracle_bf16_to_f32(uint16_t b) {
+    uint32_t u = ((uint32_t)b) << 16;
+    float f;
+    memcpy(&f, &u, 4);
+    return f;
+}
+
+/* Round-to-nearest-even to bf16 (finite inputs). */
+uint16_t oracle_f32_to_bf16(float f) {
+    uint32_t u;
+    memcpy(&u, &f, 4);
+    if ((u & 0x7f800000u) == 0x7f800000u) {            /* inf / nan: truncate */
+        return (uint16_t)((u >> 16) | ((u & 0xffffu) ? 0x40u : 0u));
+    }
+    uint32_t lsb = (u >> 16) & 1u;
+    u += 0x7fffu + lsb;
+    return (uint16_t)(u >> 16);
+}
+
+/* ------------------------------------------------------------------------ */
+/* E2M1 and E4M3 (the two NVFP4 element types)                               */
+/* ------------------------------------------------------------------------ */
+
+/* E2M1: 1 sign, 2 exponent (bias 1), 1 mantissa bit; no inf/nan.
+ * Magnitudes for codes 0..7: 0, 0.5, 1, 1.5, 2, 3, 4, 6. */
+float oracle_e2m1_decode(uint8_t code) {
+    int s = (code >> 3) & 1;
+    int e = (code >> 1) & 3;
+    int m = code & 1;
+    float mag;
+    if (e == 0) mag = 0.5f * (float)m;                         /* subnormal */
+    else        mag = ldexpf(1.0f + 0.5f * (float)m, e - 1);
+    return s ? -mag : mag;
+}
+
+/* Nearest E2M1 code, ties to the code with an even (zero) mantissa bit,
+ * saturating at 6.  Negative inputs keep the sign bit even when the magnitude
+ * rounds to zero (IEEE behaviour). */
+uint8_t oracle_e2m1_encode(float v) {
+    uint8_t sign = 0;
+    float a = v;
+    if (v < 0.0f) { sign = 8; a = -v; }
+    if (a >= 6.0f) return (uint8_t)(sign | 7);       /* saturate at the largest magnitude */
+    uint8_t best = 0;
+    float best_d = INFINITY;
+    for (uint8_t c = 0; c < 8; c++) {
+        float d = fabsf(oracle_e2m1_decode(c) - a);
+        if (d < best_d || (d == best_d && (c & 1) == 0)) { best = c; best_d = d; }
+    }
+    return (uint8_t)(sign | best);
+}
+
+/* E4M3 "FN": 1 sign, 4 exponent (bias 7), 3 mantissa bits, subnormals,
+ * S.1111.111 is NaN, no infinity; largest finite 448. */
+float oracle_e4m3_decode(uint8_t b) {
+    int s = (b >> 7) & 1;
+    int e = (b >> 3) & 15;
+    int m = b & 7;
+    float mag;
+    if (e == 15 && m == 7) return NAN;
+    if (e == 0) mag = ldexpf((float)m, -9);                    /* m/8 * 2^(1-7) */
+    else        mag = ldexpf(1.0f + (float)m / 8.0f, e - 7);
+    return s ? -mag : mag;
+}
+
+/* Nearest non-negative E4M3 byte for v >= 0, ties to an even mantissa,
+ * saturating at 448.  Codes 0x00..0x7E decode to strictly increasing values,
+ * so a binary search finds the bracketing pair. */
+uint8_t oracle_e4m3_encode_nonneg(float v) {
+    if (!(v > 0.0f)) return 0;
+    if (v >= 448.0f) return 0x7E;
+    int lo = 0, hi = 0x7E;                       /* decode(lo) <= v < decode(hi) */
+    while (hi - lo > 1) {
+        int mid = (lo + hi) / 2;
+        if (oracle_e4m3_decode((uint8_t)mid) <= v) lo = mid; else hi = mid;
+    }
+    float dl = v - oracle_e4m3_decode((uint8_t)lo);
+    float dh = oracle_e4m3_decode((uint8_t)hi) - v;
+    if (dl < dh) return (uint8_t)lo;
+    if (dh < dl) return (uint8_t)hi;
+    return (uint8_t)(((lo & 1) == 0) ? lo : hi);
+}
+
+/* ------------------------------------------------------------------------ */
+/* int4 symmetric g128 with clip search  [Int4] Recipe                       */
+/* ------------------------------------------------------------------------ */
+
+#define I4_GROUP 128
+#define I4_NRATIO 17
+
+/* The 17 evenly spaced clip ratios in [0.60, 1.00]: (24 + i) / 40. */
+static float clip_ratio(int i) { return (float)(24 + i) / 40.0f; }
+
+static int32_t rne_clamp_q(float w, float s) {
+    /* Division in double is exact enough that rint() sees the true
+     * rounding of w/s (w and s carry 8 significant bits each). */
+    double q = rint((double)w / (double)s);
+    if (q < -8.0) q = -8.0;
+    if (q > 7.0) q = 7.0;
+    return (int32_t)q;
+}
+
+/* One group of n <= 128 bf16 weights -> scale (bf16 bits) and codes q.
+ * Candidates are ratios first_ratio..16; first_ratio = 16 is the plain
+ * max-abs scale (the page's "max-abs scale" row), 0 the full clip search. */
+static void quant_int4_group(const uint16_t* w, int n, int first_ratio,
+                             uint16_t* scale_out, int8_t* q_out, int* ratio_out) {
+    float wf[I4_GROUP];
+    float amax = 0.0f;
+    for (int i = 0; i < n; i++) {
+        wf[i] = oracle_bf16_to_f32(w[i]);
+        float a = fabsf(wf[i]);
+        if (a > amax) amax = a;
+    }
+    if (amax == 0.0f) {
+        *scale_out = 0;
+        for (int i = 0; i < n; i++) q_out[i] = 0;
+        if (ratio_out) *ratio_out = I4_NRATIO - 1;
+        return;
+    }
+    float best_err = INFINITY;
+    uint16_t best_s = 0;
+    int best_i = I4_NRATIO - 1;
+    /* Larger ratios first; a later candidate must be strictly better. */
+    for (int i = I4_NRATIO - 1; i >= first_ratio; i--) {
+        float t = clip_ratio(i) * amax;
+        float sf = t / 7.0f;
+        uint16_t sb = oracle_f32_to_bf16(sf);
+        float s = oracle_bf16_to_f32(sb);
+        if (s == 0.0f) continue;
+        float err = 0.0f;
+        for (int j = 0; j < n; j++) {
+            int32_t q = rne_clamp_q(wf[j], s);
+            float d = (float)q * s - wf[j];
+            err = err + d * d;
+        }
+        if (err < best_err) { best_err = err; best_s = sb; best_i = i; }
+    }
+    float s = oracle_bf16_to_f32(best_s);
+    for (int j = 0; j < n; j++) q_out[j] = (int8_t)(s == 0.0f ? 0 : rne_clamp_q(wf[j], s));
+    *scale_out = best_s;
+    if (ratio_out) *ratio_out = best_i;
+}
+
+/* Quantise a bf16 matrix [rows, cols] (cols % 128 == 0).
+ * packed: int32 [rows, cols/8]; scales: bf16 bits [rows, cols/128];
+ * q (optional): int8 [rows, cols]; ratio_idx (optional): int32 [rows, cols/128].
+ * first_ratio: 0 for the clip search of the recipe, 16 for max-abs only. */
+void oracle_quant_int4_g128(const uint16_t* w, int64_t rows, int64_t cols,
+                            int32_t* packed, uint16_t* scales, int8_t* q,
+                            int32_t* ratio_idx, int first_ratio) {
+    int64_t ng = cols / I4_GROUP;
+    #pragma omp parallel for schedule(static)
+    for (int64_t r = 0; r < rows; r++) {
+        int8_t qg[I4_GROUP];
+        for (int64_t g = 0; g < ng; g++) {
+            int ri;
+            quant_int4_group(w + r * cols + g * I4_GROUP, I4_GROUP, first_ratio,
+                             &scales[r * ng + g], qg, &ri);
+            if (ratio_idx) ratio_idx[r * ng + g] = ri;
+            for (int c = 0; c < I4_GROUP / 8; c++) {
+                uint32_t word = 0;
+                for (int j = 0; j < 8; j++) {
+                    uint32_t u = (uint32_t)(qg[c * 8 + j] + 8) & 0xFu;
+                    word |= u << (4 * j);
+                }
+                packed[r * (cols / 8) + g * (I4_GROUP / 8) + c] = (int32_t)word;
+            }
+            if (q) memcpy(q + r * cols + g * I4_GROUP, qg, I4_GROUP);
+        }
+    }
+}
+
+/* Exact dequantisation: fp32(q) * fp32(s). */
+void oracle_dequant_int4_g128(const int32_t* packed, const uint16_t* scales,
+                              int64_t rows, int64_t cols, float* out) {
+    int64_t ng = cols / I4_GROUP;
+    #pragma omp parallel for schedule(static)
+    for (int64_t r = 0; r < rows; r++) {
+        for (int64_t c = 0; c < cols; c++) {
+            uint32_t word = (uint32_t)packed[r * (cols / 8) + c / 8];
+            int32_t q = (int32_t)((word >> (4 * (c % 8))) & 0xFu) - 8;
+            float s = oracle_bf16_to_f32(scales[r * ng + c / I4_GROUP]);
+            out[r * cols + c] = (float)q * s;
+        }
+    }
+}
+
+/* ------------------------------------------------------------------------ */
+/* NVFP4 (W4A16)  [NVFP4] Modifications item 2, Format                       */
+/* ------------------------------------------------------------------------ */
+
+#define FP4_BLOCK 16
+
+/* Quantise one expert matrix [rows, cols] (cols % 16 == 0).
+ * packed: uint8 [rows, cols/2]; scales: uint8 E4M3 [rows, cols/16];
+ * *global: fp32 weight_scale_2. */
+void oracle_quant_nvfp4(const uint16_t* w, int64_t rows, int64_t cols,
+                        uint8_t* packed, uint8_t* scales, float* global) {
+    float amax = 0.0f;
+    for (int64_t i = 0; i < rows * cols; i++) {
+        float a = fabsf(oracle_bf16_to_f32(w[i]));
+        if (a > amax) amax = a;
+    }
+    float g = amax / (6.0f * 448.0f);
+    *global = g;
+    int64_t nb = cols / FP4_BLOCK;
+    #pragma omp parallel for schedule(static)
+    for (int64_t r = 0; r < rows; r++) {
+        for (int64_t b = 0; b < nb; b++) {
+            const uint16_t* wb = w + r * cols + b * FP4_BLOCK;
+            float wf[FP4_BLOCK];
+            float amax_b = 0.0f;
+            for (int j = 0; j < FP4_BLOCK; j++) {
+                wf[j] = oracle_bf16_to_f32(wb[j]);
+                float a = fabsf(wf[j]);
+                if (a > amax_b) amax_b = a;
+            }
+            uint8_t sb = 0;
+            if (g > 0.0f) sb = oracle_e4m3_encode_nonneg(amax_b / (6.0f * g));
+            scales[r * nb + b] = sb;
+            float eff = oracle_e4m3_decode(sb) * g;
+            uint8_t codes[FP4_BLOCK];
+            for (int j = 0; j < FP4_BLOCK; j++)
+                codes[j] = (eff > 0.0f) ? oracle_e2m1_encode(wf[j] / eff) : 0;
+            for (int j = 0; j < FP4_BLOCK / 2; j++)
+                packed[r * (cols / 2) + b * (FP4_BLOCK / 2) + j] =
+                    (uint8_t)(codes[2 * j] | (codes[2 * j + 1] << 4));
+        }
+    }
+}
+
+/* Exact dequantisation in fp32: (E2M1 value x E4M3 scale) x global.  The
+ * first product is exact (at most 5 significant bits); one rounding follows. */
+void oracle_dequant_nvfp4(const uint8_t* packed, const uint8_t* scales, float global,
+                          int64_t rows, int64_t cols, float* out) {
+    int64_t nb = cols / FP4_BLOCK;
+    #pragma omp parallel for schedule(static)
+    for (int64_t r = 0; r < rows; r++) {
+        for (int64_t c = 0; c < cols; c++) {
+            uint8_t byte = packed[r * (cols / 2) + c / 2];
+            uint8_t code = (c % 2 == 0) ? (byte & 0xF) : (byte >> 4);
+            float sb = oracle_e4m3_decode(scales[r * nb + c / FP4_BLOCK]);
+            out[r * cols + c] = (oracle_e2m1_decode(code) * sb) * global;
+        }
+    }
+}
+
+/* ------------------------------------------------------------------------ */
+/* Expert banks (fused [E, out, in], [Int4] Tensor layout / [NVFP4] Format)  */
+/* ------------------------------------------------------------------------ */
+
+typedef struct {
+    int32_t fmt;            /* 0 int4 g128, 1 nvfp4, 2 bf16 */
+    int32_t E, out, in;
+    const void* packed;     /* int4: int32 [E,out,in/8]; nvfp4: u8 [E,out,in/2]; bf16: u16 [E,out,in] */
+    const void* scales;     /* int4: bf16 bits [E,out,in/128]; nvfp4: u8 [E,out,in/16]; bf16: NULL */
+    const float* global_scale; /* nvfp4: [E]; else NULL */
+} oracle_bank;
+
+/* Dequantise expert e of a bank into fp32 [out, in]. */
+void oracle_dequant_expert(const oracle_bank* b, int e, float* w) {
+    int64_t rows = b->out, cols = b->in;
+    if (b->fmt == 0) {
+        oracle_dequant_int4_g128((const int32_t*)b->packed + (int64_t)e * rows * (cols / 8),
+                                 (const uint16_t*)b->scales + (int64_t)e * rows * (cols / I4_GROUP),
+                                 rows, cols, w);
+    } else if (b->fmt == 1) {
+        oracle_dequant_nvfp4((const uint8_t*)b->packed + (int64_t)e * rows * (cols / 2),
+                             (const uint8_t*)b->scales + (int64_t)e * rows * (cols / FP4_BLOCK),
+                             b->global_scale[e], rows, cols, w);
+    } else {
+        const uint16_t* src = (const uint16_t*)b->packed + (int64_t)e * rows * cols;
+        for (int64_t i = 0; i < rows * cols; i++) w[i] = oracle_bf16_to_f32(src[i]);
+    }
+}
+
+/* ------------------------------------------------------------------------ */
+/* Router  [Spark] At a glance: sigmoid router, top-8                        */
+/* ------------------------------------------------------------------------ */
+
+/* x: bf16 bits [T,H]; Wr: fp32 [E,H]; bias: fp32 [E] or NULL.
+ * ids: int32 [T,k]; w: fp32 [T,k]; scores (optional): fp32 [T,E] sigmoids. */
+void oracle_route(const uint16_t* x, int64_t T, int64_t H, const float* Wr,
+                  const float* bias, int64_t E, int k, int32_t* ids, float* w,
+                  float* scores) {
+    #pragma omp parallel for schedule(dynamic, 1)
+    for (int64_t t = 0; t < T; t++) {
+        float* s = (float*)malloc(sizeof(float) * E);
+        char* taken = (char*)calloc(E, 1);
+        for (int64_t e = 0; e < E; e++) {
+            float l = 0.0f;
+            for (int64_t h = 0; h < H; h++)
+                l = l + oracle_bf16_to_f32(x[t * H + h]) * Wr[e * H + h];
+            if (bias) l = l + bias[e];
+            s[e] = 1.0f / (1.0f + expf(-l));
+            if (scores) scores[t * E + e] = s[e];
+        }
+        float sum = 0.0f;
+        for (int j = 0; j < k; j++) {
+            int64_t best = -1;
+            for (int64_t e = 0; e < E; e++) {
+                if (taken[e]) continue;
+                if (best < 0 || s[e] > s[best]) best = e;   /* strict: lower id wins ties */
+            }
+            taken[best] = 1;
+            ids[t * k + j] = (int32_t)best;
+            w[t * k + j] = s[best];
+            sum = sum + s[best];
+        }
+        for (int j = 0; j < k; j++) w[t * k + j] = w[t * k + j] / sum;
+        free(s);
+        free(taken);
+    }
+}
+
+/* ------------------------------------------------------------------------ */
+/* Token -> expert bucketing                                                 */
+/* ------------------------------------------------------------------------ */
+
+/* Stable counting sort of the R = T*k slots (slot = t*k + j) by expert id.
+ * offsets: [E+1]; row_slot[r] = slot at permuted row r; slot_row = inverse.
+ * Returns 0, or -1 if an id is out of range. */
+int oracle_permute(const int32_t* ids, int64_t T, int k, int64_t E,
+                   int32_t* offsets, int32_t* row_slot, int32_t* slot_row) {
+    int64_t R = T * k;
+    int64_t* count = (int64_t*)calloc(E, sizeof(int64_t));
+    for (int64_t s = 0; s < R; s++) {
+        if (ids[s] < 0 || ids[s] >= E) { free(count); return -1; }
+        count[ids[s]]++;
+    }
+    offsets[0] = 0;
+    for (int64_t e = 0; e < E; e++) offsets[e + 1] = offsets[e] + (int32_t)count[e];
+    memset(count, 0, sizeof(int64_t) * E);
+    for (int64_t s = 0; s < R; s++) {
+        int64_t e = ids[s];
+        int64_t r = offsets[e] + count[e]++;
+        row_slot[r] = (int32_t)s;
+        slot_row[s] = (int32_t)r;
+    }
+    free(count);
+    return 0;
+}
+
+/* ------------------------------------------------------------------------ */
+/* Layer forward  [Art] The shape: 8 routed SwiGLU experts + 1 shared        */
+/* ------------------------------------------------------------------------ */
+
+static double silu(double v) { return v / (1.0 + exp(-v)); }
+
+/* y[i,:] for tokens tok[i], i < n:
+ *   y = FFN_shared(x) + sum_j w[t,j] * FFN_{ids[t,j]}(x),
+ *   FFN(x) = Wd (silu(Wg x) * (Wu x)),
+ * with fp32-exact dequantised weights and fp64 accumulation.  Experts are
+ * visited one at a time (each dequantised once); each expert serves the
+ * (token, slot) pairs that selected it.  sh_* may be NULL (no shared expert).
+ * Returns 0, or -1 on an out-of-range id. */
+int oracle_moe_forward(const uint16_t* x, int64_t T, int64_t H, int64_t F, int k,
+                       const int32_t* ids, const float* topk_w,
+                       const oracle_bank* gate, const oracle_bank* up,
+                       const oracle_bank* down, const oracle_bank* sh_gate,
+                       const oracle_bank* sh_up, const oracle_bank* sh_down,
+                       const int32_t* tok, int64_t n, double* y) {
+    int64_t E = gate->E;
+    for (int64_t i = 0; i < n; i++)
+        for (int64_t j = 0; j < k; j++) {
+            int32_t e = ids[tok[i] * k + j];
+            if (e < 0 || e >= E) return -1;
+        }
+    double* xd = (double*)malloc(sizeof(double) * n * H);
+    for (int64_t i = 0; i < n; i++)
+        for (int64_t h = 0; h < H; h++)
+            xd[i * H + h] = (double)oracle_bf16_to_f32(x[tok[i] * H + h]);
+    memset(y, 0, sizeof(double) * n * H);
+
+    float* wg = (float*)malloc(sizeof(float) * F * H);
+    float* wu = (float*)malloc(sizeof(float) * F * H);
+    float* wd = (float*)malloc(sizeof(float) * H * F);
+    double* hbuf = (double*)malloc(sizeof(double) * F);
+    int64_t* who = (int64_t*)malloc(sizeof(int64_t) * n * k);
+
+    int64_t nexp = E + (sh_gate ? 1 : 0);
+    for (int64_t e = 0; e < nexp; e++) {
+        int shared = (e == E);
+        int64_t m = 0;                           /* (token index i, weight slot) pairs */
+        if (shared) {
+            for (int64_t i = 0; i < n; i++) who[m++] = -1 - i;  /* negative: shared, weight 1 */
+        } else {
+            for (int64_t i = 0; i < n; i++)
+                for (int64_t j = 0; j < k; j++)
+                    if (ids[tok[i] * k + j] == e) who[m++] = i * k + j;
+        }
+        if (m == 0) continue;
+        oracle_dequant_expert(shared ? sh_gate : gate, shared ? 0 : (int)e, wg);
+        oracle_dequant_expert(shared ? sh_up : up, shared ? 0 : (int)e, wu);
+        oracle_dequant_expert(shared ? sh_down : down, shared ? 0 : (int)e, wd);
+        for (int64_t p = 0; p < m; p++) {
+            int64_t i, slot;
+            double wt;
+            if (who[p] < 0) { i = -1 - who[p]; slot = -1; wt = 1.0; }
+            else { i = who[p] / k; slot = who[p] % k; wt = (double)topk_w[tok[i] * k + slot]; }
+            const double* xi = xd + i * H;
+            #pragma omp parallel for schedule(static)
+            for (int64_t f = 0; f < F; f++) {
+                double g = 0.0, u = 0.0;
+                for (int64_t h = 0; h < H; h++) {
+                    g += (double)wg[f * H + h] * xi[h];
+                    u += (double)wu[f * H + h] * xi[h];
+                }
+                hbuf[f] = silu(g) * u;
+            }
+            #pragma omp parallel for schedule(static)
+            for (int64_t h = 0; h < H; h++) {
+                double acc = 0.0;
+                for (int64_t f = 0; f < F; f++) acc += (double)wd[h * F + f] * hbuf[f];
+                y[i * H + h] += wt * acc;
+            }
+        }
+    }
+    free(xd); free(wg); free(wu); free(wd); free(hbuf); free(who);
+    return 0;
+}
