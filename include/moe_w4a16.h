@@ -1,0 +1,219 @@
+/*
+ * moe_w4a16.h -- C ABI of libmoe: the routed-expert MoE layer of Step-5-Preview
+ * run directly on 4-bit weights, on one NVIDIA B200 (sm_100a).
+ *
+ * The layer ("Step-5-Preview-Spark", At a glance; "Step 5 Preview: 92 narrow
+ * layers, and a sparse indexer that scores blocks of 8", The shape): hidden
+ * size H = 4096, E = 352 routed experts chosen top-8 by a sigmoid router, each
+ * a SwiGLU of width F = 1536, plus one shared SwiGLU expert of the same width:
+ *
+ *     y[t] = FFN_shared(x[t]) + sum_{j<k} w[t,j] * FFN_{e[t,j]}(x[t]),
+ *     FFN(x) = W_down (silu(W_gate x) * (W_up x)).
+ *
+ * Routed expert weights come in the pages' fused layout [E, out, in] in one of
+ * two 4-bit formats:
+ *   MOE_FMT_INT4_G128 -- "Step-5-Preview-Int4-g128", Recipe / Tensor layout:
+ *       int4 symmetric, group 128 along `in`, one bf16 scale per group.
+ *       packed: int32 [E, out, in/8]; element in = 8c + j is bits 4j..4j+3 of
+ *       word c, stored offset-binary (nibble u = q + 8, q in [-8, 7]).
+ *       scales: bf16 [E, out, in/128].  w = q * scale.
+ *   MOE_FMT_NVFP4 -- "Step-5-Preview-NVFP4-Local", Modifications item 2 and
+ *       Format (W4A16_NVFP4, activations stay bf16): packed: uint8
+ *       [E, out, in/2], two E2M1 codes per byte, even element in the low nibble;
+ *       scales: uint8 E4M3 [E, out, in/16]; global_scale: fp32 [E]
+ *       (weight_scale_2).  w = e2m1(code) * e4m3(scale) * global_scale[e].
+ *   MOE_FMT_BF16 -- plain bf16 [E, out, in] (used for the shared expert).
+ *
+ * Conventions for every entry point:
+ *   - All tensor pointers are caller-owned DEVICE memory on the current device.
+ *     The library never allocates, frees, or synchronises the stream, except
+ *     moe_read_status(), which synchronises to read the status word.
+ *   - Calls are asynchronous and stream-ordered on `stream` (a cudaStream_t;
+ *     NULL = legacy default stream).
+ *   - The return value reports argument and launch errors only (moe_status).
+ *     On an argument error nothing is launched.  Conditions found on the device
+ *     (an expert id out of range, a bounded wait that ran out) are recorded in
+ *     the status word at the start of the workspace; read it with
+ *     moe_read_status().
+ *   - Weight, activation and output pointers must be 16-byte aligned.
+ *     H, F must be multiples of 128; 1 <= top_k <= 8; 1 <= E <= 1024.
+ *     Other shapes return MOE_ERR_UNSUPPORTED.  T = 0 is a no-op (MOE_OK).
+ *   - bf16 tensors are passed as `void*` (2 bytes per element, IEEE bfloat16).
+ *   - Intermediates: h_perm is bf16 [rows, F]; y_perm is bf16 [rows, H].
+ *   - The workspace `ws` (ws_bytes bytes, 256-byte aligned) must be zero-filled
+ *     once before first use (moe_workspace_init); kernels leave their counters
+ *     at zero again when they finish.  Its first 256 bytes hold the status
+ *     word; the step calls use the bytes after them as scratch (sizes below),
+ *     the layer entries the whole of moe_workspace_bytes().  A workspace of
+ *     moe_workspace_bytes(T, H, E, F, top_k) bytes serves every call at those
+ *     sizes.  Calls that share a workspace must not run concurrently.
+ */
+#ifndef MOE_W4A16_H
+#define MOE_W4A16_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef struct CUstream_st* moe_stream_t; /* same type as cudaStream_t */
+
+typedef enum {
+    MOE_OK = 0,
+    MOE_ERR_INVALID_ARG = -1, /* null pointer, negative size, misalignment   */
+    MOE_ERR_UNSUPPORTED = -2, /* valid but unsupported shape / format         */
+    MOE_ERR_CUDA = -3,        /* a CUDA call or kernel launch failed          */
+    MOE_ERR_TIMEOUT = -4,     /* device status: a bounded wait ran out        */
+    MOE_ERR_WORKSPACE = -5,   /* workspace missing or too small               */
+    MOE_ERR_DEVICE_INDEX = -6 /* device status: an index was out of range     */
+} moe_status;
+
+typedef enum { MOE_FMT_INT4_G128 = 0, MOE_FMT_NVFP4 = 1, MOE_FMT_BF16 = 2 } moe_wfmt;
+
+/* One projection bank in the pages' fused layout [num_experts, out_dim, in_dim]. */
+typedef struct {
+    int32_t fmt;              /* moe_wfmt                                          */
+    int32_t num_experts;      /* E (1 for the shared expert)                      */
+    int32_t out_dim;          /* rows: F for gate/up, H for down                  */
+    int32_t in_dim;           /* reduction length: H for gate/up, F for down      */
+    const void* packed;       /* INT4: int32[E,out,in/8]; NVFP4: u8[E,out,in/2]; BF16: bf16[E,out,in] */
+    const void* scales;       /* INT4: bf16[E,out,in/128]; NVFP4: u8 E4M3[E,out,in/16]; BF16: NULL   */
+    const float* global_scale;/* NVFP4: fp32[E]; otherwise NULL                    */
+} moe_qweight;
+
+/* A whole MoE layer.  sh_gate/sh_up/sh_down: MOE_FMT_BF16 banks with
+ * num_experts = 1, or all three with packed = NULL for no shared expert.
+ * router_w: fp32 [E, H]; router_bias: fp32 [E] added to the logits before
+ * the sigmoid, or NULL.  swiglu_limit must be 0 (the pages give no value or
+ * definition for a SwiGLU limit, so none is applied). */
+typedef struct {
+    moe_qweight gate, up, down;
+    moe_qweight sh_gate, sh_up, sh_down;
+    const float* router_w;
+    const float* router_bias;
+    int32_t E, H, F, top_k;
+    float swiglu_limit;
+} moe_layer;
+
+/* ---------------------------------------------------------------------- */
+/* Workspace and status                                                    */
+/* ---------------------------------------------------------------------- */
+
+/* Bytes of workspace sufficient for every entry point below at these sizes
+ * (T tokens), including the intermediates of moe_layer_decode and
+ * moe_layer_forward.  Returns 0 for invalid sizes. */
+size_t moe_workspace_bytes(int T, int H, int E, int F, int top_k);
+
+/* Zero-fill a workspace (cudaMemsetAsync on `stream`). */
+int moe_workspace_init(void* ws, size_t ws_bytes, moe_stream_t stream);
+
+/* Synchronise `stream`, copy the workspace's device status word to
+ * *status_out (MOE_OK or a negative moe_status), and clear it. */
+int moe_read_status(void* ws, moe_stream_t stream, int32_t* status_out);
+
+/* Static description of a status code. */
+const char* moe_status_string(int status);
+
+/* ---------------------------------------------------------------------- */
+/* Hot-path steps                                                          */
+/* ---------------------------------------------------------------------- */
+
+/* Router ("Step-5-Preview-Spark", At a glance: sigmoid router, top-8).
+ *   l[t,e] = sum_h x[t,h] * router_w[e,h] (+ router_bias[e]), fp32;
+ *   s = 1 / (1 + exp(-l)), fp32; the top_k largest s per token, ties to the
+ *   lower expert id, listed by descending s; topk_w = s / sum(selected s).
+ * x: bf16 [T, H]; router_w: fp32 [E, H]; router_bias: fp32 [E] or NULL;
+ * topk_ids: int32 [T, top_k] (out); topk_w: fp32 [T, top_k] (out).
+ * ws: at least 256 + 4*T*E bytes. */
+int moe_route_topk(const void* x, int T, int H, const float* router_w,
+                   const float* router_bias, int E, int top_k, int32_t* topk_ids,
+                   float* topk_w, void* ws, size_t ws_bytes, moe_stream_t stream);
+
+/* Token -> expert bucketing: a stable counting sort of the R = T*top_k slots
+ * (slot = t*top_k + j) by expert id.
+ * topk_ids: int32 [T, top_k], each in [0, E) (an id outside sets the device
+ * status MOE_ERR_DEVICE_INDEX and is dropped);
+ * expert_offsets: int32 [E+1] (out), exclusive prefix sum of per-expert counts;
+ * row_slot: int32 [R] (out), the slot placed at permuted row r;
+ * slot_row: int32 [R] (out), its inverse.
+ * Rows of one expert are ordered by slot (token, then rank j).
+ * ws: at least 256 + 4*E*ceil(T*top_k / 4096) bytes. */
+int moe_permute(const int32_t* topk_ids, int T, int top_k, int E,
+                int32_t* expert_offsets, int32_t* row_slot, int32_t* slot_row,
+                void* ws, size_t ws_bytes, moe_stream_t stream);
+
+/* Grouped gate/up projection with fused SwiGLU, weights dequantised in-kernel:
+ * for each expert e and row r in [expert_offsets[e], expert_offsets[e+1]),
+ * with token t = row_slot[r] / top_k:
+ *     h_perm[r, f] = bf16( silu(g) * u ),  g = x[t] . Wg[e,f,:],  u = x[t] . Wu[e,f,:]
+ * (fp32 accumulation).  x: bf16 [T, H]; gate/up: banks [E, F, H] of the same
+ * format; h_perm: bf16 [T*top_k, F] (out).  swiglu_limit must be 0.
+ * For the shared expert pass BF16 banks with E = 1, expert_offsets = {0, T}
+ * and row_slot[i] = i * top_k.  Decode-sized calls (T*top_k <= 256) stream
+ * the weights with a GEMV; larger calls run a tcgen05 grouped GEMM.
+ * ws: at least 256 + 16*(E+2) bytes. */
+int moe_grouped_w4a16_swiglu(const void* x, int T, int H,
+                             const int32_t* expert_offsets, const int32_t* row_slot,
+                             int top_k, const moe_qweight* gate, const moe_qweight* up,
+                             float swiglu_limit, void* h_perm,
+                             void* ws, size_t ws_bytes, moe_stream_t stream);
+
+/* Grouped down projection with the routing weight fused:
+ *     y_perm[r, :] = bf16( topk_w[row_slot[r]] * (h_perm[r] . Wd[e]^T) )
+ * for rows r of expert e (fp32 accumulation).  h_perm: bf16 [rows, F];
+ * topk_w: fp32 [rows] indexed by slot, or NULL for weight 1;
+ * down: bank [E, H, F]; y_perm: bf16 [rows, H] (out).
+ * ws: at least 256 + 16*(E+2) bytes. */
+int moe_grouped_w4a16_down(const void* h_perm, const int32_t* expert_offsets,
+                           const int32_t* row_slot, const float* topk_w, int rows,
+                           const moe_qweight* down, void* y_perm,
+                           void* ws, size_t ws_bytes, moe_stream_t stream);
+
+/* Unpermute and combine:
+ *     y[t, :] = bf16( shared_out[t, :] + sum_{j<top_k} y_perm[slot_row[t*top_k + j], :] )
+ * summed in fp32 in the order shared, j = 0..top_k-1.  y_perm: bf16 [T*top_k, H];
+ * shared_out: bf16 [T, H] or NULL; y: bf16 [T, H] (out). */
+int moe_unpermute_combine(const void* y_perm, const int32_t* slot_row, int T,
+                          int top_k, int H, const void* shared_out, void* y,
+                          moe_stream_t stream);
+
+/* The whole layer for decode-sized batches (1 <= T <= 64): router, bucketing,
+ * gate/up + SwiGLU, down with routing weights, shared expert and combine, on
+ * device with no host synchronisation.  x: bf16 [T, H]; y: bf16 [T, H] (out). */
+int moe_layer_decode(const void* x, int T, const moe_layer* L, void* y,
+                     void* ws, size_t ws_bytes, moe_stream_t stream);
+
+/* The whole layer for any T >= 1 (prefill-sized batches use the tcgen05
+ * grouped GEMM).  Same arguments and result as moe_layer_decode. */
+int moe_layer_forward(const void* x, int T, const moe_layer* L, void* y,
+                      void* ws, size_t ws_bytes, moe_stream_t stream);
+
+/* ---------------------------------------------------------------------- */
+/* Weight conversion (offline step, not on the hot path)                   */
+/* ---------------------------------------------------------------------- */
+
+/* int4 symmetric g128 quantiser ("Step-5-Preview-Int4-g128", Recipe): per row
+ * and group of 128, the scale is bf16((r * amax) / 7) for the clip ratio r in
+ * {24/40, 25/40, ..., 40/40} that minimises sum (q*s - w)^2 (fp32, index
+ * order; ties keep the larger ratio); q = clamp(rint(w / s), -8, 7).
+ * w: bf16 [rows, cols] (cols % 128 == 0); packed: int32 [rows, cols/8] (out);
+ * scales: bf16 [rows, cols/128] (out). */
+int moe_quantize_int4_g128(const void* w, int64_t rows, int64_t cols, int32_t* packed,
+                           void* scales, moe_stream_t stream);
+
+/* NVFP4 quantiser ("Step-5-Preview-NVFP4-Local", Format): per matrix,
+ * global = amax / (6 * 448) (fp32); per block of 16 along cols,
+ * scale = e4m3_rne(amax_block / (6 * global)); code = e2m1_rne(w / (e4m3(scale) * global)).
+ * w: bf16 [rows, cols] (one expert matrix, cols % 16 == 0); packed: uint8
+ * [rows, cols/2] (out); scales: uint8 [rows, cols/16] (out); global_scale:
+ * fp32 [1] (out).  ws: at least 256 bytes of zero-filled workspace. */
+int moe_quantize_nvfp4(const void* w, int64_t rows, int64_t cols, uint8_t* packed,
+                       uint8_t* scales, float* global_scale, void* ws, size_t ws_bytes,
+                       moe_stream_t stream);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* MOE_W4A16_H */

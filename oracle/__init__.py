@@ -55,6 +55,12 @@ def lib():
         L.oracle_permute.restype = I
         L.oracle_moe_forward.argtypes = [P, I64, I64, I64, I, P, P, P, P, P, P, P, P, P, I64, P]
         L.oracle_moe_forward.restype = I
+        L.oracle_grouped_swiglu.argtypes = [P, I64, I64, I, P, P, P, P, P, I64, P]
+        L.oracle_grouped_swiglu.restype = None
+        L.oracle_grouped_down.argtypes = [P, I64, I64, P, P, P, P, P, I64, P]
+        L.oracle_grouped_down.restype = None
+        L.oracle_combine.argtypes = [P, P, I64, I, I64, P, P]
+        L.oracle_combine.restype = None
         _lib = L
     return _lib
 
@@ -239,4 +245,40 @@ def moe_forward(x_bits, ids, topk_w, gate, up, down, shared=None, tokens=None):
     rc = lib().oracle_moe_forward(_p(x), T, H, F, k, _p(ids), _p(w), *refs, _p(tok), n, _p(y))
     if rc != 0:
         raise ValueError("expert id out of range")
+    return y
+
+
+def grouped_swiglu(x_bits, offsets, row_slot, k, gate, up, rows):
+    """h[i, :] for permuted rows `rows` (fp64 [n, F])."""
+    x = _c(x_bits, np.uint16)
+    H = x.shape[1]
+    F = gate.out
+    rows = _c(rows, np.int32)
+    h = np.empty((rows.shape[0], F), np.float64)
+    g, u = gate._struct(), up._struct()
+    lib().oracle_grouped_swiglu(_p(x), H, F, k, _p(_c(offsets, np.int32)), _p(_c(row_slot, np.int32)),
+                                ctypes.addressof(g), ctypes.addressof(u), _p(rows), rows.shape[0], _p(h))
+    return h
+
+
+def grouped_down(h_bits, offsets, row_slot, topk_w, down, rows):
+    """y[i, :] for permuted rows `rows` (fp64 [n, H]); topk_w indexed by slot or None."""
+    hb = _c(h_bits, np.uint16)
+    F = hb.shape[1]
+    H = down.out
+    rows = _c(rows, np.int32)
+    y = np.empty((rows.shape[0], H), np.float64)
+    d = down._struct()
+    tw = None if topk_w is None else _c(topk_w, np.float32)
+    lib().oracle_grouped_down(_p(hb), F, H, _p(_c(offsets, np.int32)), _p(_c(row_slot, np.int32)), _p(tw),
+                              ctypes.addressof(d), _p(rows), rows.shape[0], _p(y))
+    return y
+
+
+def combine(y_perm_bits, slot_row, T, k, shared_bits=None):
+    yp = _c(y_perm_bits, np.uint16)
+    H = yp.shape[1]
+    y = np.empty((T, H), np.float64)
+    sh = None if shared_bits is None else _c(shared_bits, np.uint16)
+    lib().oracle_combine(_p(yp), _p(_c(slot_row, np.int32)), T, k, H, _p(sh), _p(y))
     return y

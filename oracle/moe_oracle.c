@@ -476,3 +476,91 @@ int oracle_moe_forward(const uint16_t* x, int64_t T, int64_t H, int64_t F, int k
     free(xd); free(wg); free(wu); free(wd); free(hbuf); free(who);
     return 0;
 }
+
+/* ------------------------------------------------------------------------ */
+/* Per-step definitions (one per library call), fp64 accumulation           */
+/* ------------------------------------------------------------------------ */
+
+/* Gate/up + SwiGLU over bucketed rows: for expert e and row r in
+ * [offsets[e], offsets[e+1]), token t = row_slot[r] / k:
+ *   h[r, f] = silu(x[t] . Wg[e,f,:]) * (x[t] . Wu[e,f,:]).
+ * Rows listed in `rows` (n of them) are computed; h is [n, F]. */
+void oracle_grouped_swiglu(const uint16_t* x, int64_t H, int64_t F, int k,
+                           const int32_t* offsets, const int32_t* row_slot,
+                           const oracle_bank* gate, const oracle_bank* up,
+                           const int32_t* rows, int64_t n, double* h) {
+    int64_t E = gate->E;
+    float* wg = (float*)malloc(sizeof(float) * F * H);
+    float* wu = (float*)malloc(sizeof(float) * F * H);
+    for (int64_t e = 0; e < E; e++) {
+        int any = 0;
+        for (int64_t i = 0; i < n; i++)
+            if (rows[i] >= offsets[e] && rows[i] < offsets[e + 1]) any = 1;
+        if (!any) continue;
+        oracle_dequant_expert(gate, (int)e, wg);
+        oracle_dequant_expert(up, (int)e, wu);
+        for (int64_t i = 0; i < n; i++) {
+            int32_t r = rows[i];
+            if (r < offsets[e] || r >= offsets[e + 1]) continue;
+            int64_t t = row_slot[r] / k;
+            #pragma omp parallel for schedule(static)
+            for (int64_t f = 0; f < F; f++) {
+                double g = 0.0, u = 0.0;
+                for (int64_t hh = 0; hh < H; hh++) {
+                    double xv = (double)oracle_bf16_to_f32(x[t * H + hh]);
+                    g += (double)wg[f * H + hh] * xv;
+                    u += (double)wu[f * H + hh] * xv;
+                }
+                h[i * F + f] = silu(g) * u;
+            }
+        }
+    }
+    free(wg);
+    free(wu);
+}
+
+/* Down projection with the routing weight: for row r of expert e,
+ *   y[r, :] = w[row_slot[r]] * (Wd[e] h_in[r])     (w = 1 if topk_w is NULL).
+ * h_in: bf16 bits [R, F]; rows listed in `rows`; y is [n, H]. */
+void oracle_grouped_down(const uint16_t* h_in, int64_t F, int64_t H,
+                         const int32_t* offsets, const int32_t* row_slot,
+                         const float* topk_w, const oracle_bank* down,
+                         const int32_t* rows, int64_t n, double* y) {
+    int64_t E = down->E;
+    float* wd = (float*)malloc(sizeof(float) * H * F);
+    for (int64_t e = 0; e < E; e++) {
+        int any = 0;
+        for (int64_t i = 0; i < n; i++)
+            if (rows[i] >= offsets[e] && rows[i] < offsets[e + 1]) any = 1;
+        if (!any) continue;
+        oracle_dequant_expert(down, (int)e, wd);
+        for (int64_t i = 0; i < n; i++) {
+            int32_t r = rows[i];
+            if (r < offsets[e] || r >= offsets[e + 1]) continue;
+            double wt = topk_w ? (double)topk_w[row_slot[r]] : 1.0;
+            #pragma omp parallel for schedule(static)
+            for (int64_t hh = 0; hh < H; hh++) {
+                double acc = 0.0;
+                for (int64_t f = 0; f < F; f++)
+                    acc += (double)wd[hh * F + f] * (double)oracle_bf16_to_f32(h_in[(int64_t)r * F + f]);
+                y[i * H + hh] = wt * acc;
+            }
+        }
+    }
+    free(wd);
+}
+
+/* Combine: y[t] = shared[t] + sum_j y_perm[slot_row[t*k + j]] (fp64).
+ * y_perm: bf16 bits [T*k, H]; shared: bf16 bits [T, H] or NULL. */
+void oracle_combine(const uint16_t* y_perm, const int32_t* slot_row, int64_t T, int k,
+                    int64_t H, const uint16_t* shared, double* y) {
+    for (int64_t t = 0; t < T; t++)
+        for (int64_t hh = 0; hh < H; hh++) {
+            double acc = shared ? (double)oracle_bf16_to_f32(shared[t * H + hh]) : 0.0;
+            for (int j = 0; j < k; j++) {
+                int32_t r = slot_row[t * k + j];
+                acc += (double)oracle_bf16_to_f32(y_perm[(int64_t)r * H + hh]);
+            }
+            y[t * H + hh] = acc;
+        }
+}

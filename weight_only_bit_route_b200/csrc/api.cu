@@ -1,0 +1,302 @@
+// C ABI entry points of libmoe (declared in include/moe_w4a16.h): argument
+// validation, workspace carving and kernel composition.  Nothing here touches
+// the data; every step runs in the kernels of this library.
+#include <algorithm>
+
+#include "moe_internal.cuh"
+
+using namespace moe;
+
+namespace {
+
+inline bool al16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+inline cudaStream_t cs(moe_stream_t s) { return reinterpret_cast<cudaStream_t>(s); }
+
+template <typename T>
+inline T* at(void* ws, size_t off) {
+    return reinterpret_cast<T*>(reinterpret_cast<uint8_t*>(ws) + off);
+}
+
+int check_dims(int T, int H, int E, int F, int k) {
+    if (T < 0 || H <= 0 || E <= 0 || F <= 0 || k <= 0) return MOE_ERR_INVALID_ARG;
+    if (H % 128 || F % 128 || k > kMaxTopK || E > kMaxE || k > E) return MOE_ERR_UNSUPPORTED;
+    return MOE_OK;
+}
+
+int check_bank(const moe_qweight* b, int E, int out, int in) {
+    if (!b) return MOE_ERR_INVALID_ARG;
+    if (b->fmt != MOE_FMT_INT4_G128 && b->fmt != MOE_FMT_NVFP4 && b->fmt != MOE_FMT_BF16)
+        return MOE_ERR_UNSUPPORTED;
+    if (b->num_experts != E || b->out_dim != out || b->in_dim != in) return MOE_ERR_INVALID_ARG;
+    if (in % 128 || out <= 0) return MOE_ERR_UNSUPPORTED;
+    if (!b->packed || !al16(b->packed)) return MOE_ERR_INVALID_ARG;
+    if (b->fmt != MOE_FMT_BF16 && !b->scales) return MOE_ERR_INVALID_ARG;
+    if (b->fmt == MOE_FMT_NVFP4 && !b->global_scale) return MOE_ERR_INVALID_ARG;
+    return MOE_OK;
+}
+
+int check_ws(void* ws, size_t ws_bytes, size_t need) {
+    if (!ws || (reinterpret_cast<uintptr_t>(ws) & 255u)) return MOE_ERR_WORKSPACE;
+    if (ws_bytes < need) return MOE_ERR_WORKSPACE;
+    return MOE_OK;
+}
+
+#define MOE_TRY(x)                     \
+    do {                               \
+        int _rc = (x);                 \
+        if (_rc != MOE_OK) return _rc; \
+    } while (0)
+
+// decode-sized calls stream weights with the GEMV; larger ones use the GEMM
+constexpr int kGemvMaxRows = 256;
+
+// rows_total: rows present over all experts; max_touched: bound on the number
+// of experts holding at least one row (sizes the persistent grid).
+int run_grouped(const GemvProblem& p, bool gateup, int rows_total, int max_touched,
+                int32_t* tile_ws, cudaStream_t s) {
+    if (rows_total <= kGemvMaxRows) return launch_grouped_gemv(p, gateup, max_touched, s);
+    return launch_grouped_gemm(p, gateup, rows_total, max_touched, tile_ws, s);
+}
+
+int layer_checks(const void* x, int T, const moe_layer* L, void* y, void* ws, size_t ws_bytes) {
+    if (!L) return MOE_ERR_INVALID_ARG;
+    MOE_TRY(check_dims(T, L->H, L->E, L->F, L->top_k));
+    if (T == 0) return MOE_OK;
+    if (!x || !y) return MOE_ERR_INVALID_ARG;
+    if (!al16(x) || !al16(y) || !L->router_w || !al16(L->router_w)) return MOE_ERR_INVALID_ARG;
+    if (L->swiglu_limit != 0.0f) return MOE_ERR_UNSUPPORTED;
+    MOE_TRY(check_bank(&L->gate, L->E, L->F, L->H));
+    MOE_TRY(check_bank(&L->up, L->E, L->F, L->H));
+    MOE_TRY(check_bank(&L->down, L->E, L->H, L->F));
+    if (L->gate.fmt == MOE_FMT_BF16 || L->gate.fmt != L->up.fmt || L->gate.fmt != L->down.fmt)
+        return MOE_ERR_UNSUPPORTED;
+    const bool has_sh = L->sh_gate.packed || L->sh_up.packed || L->sh_down.packed;
+    if (has_sh) {
+        MOE_TRY(check_bank(&L->sh_gate, 1, L->F, L->H));
+        MOE_TRY(check_bank(&L->sh_up, 1, L->F, L->H));
+        MOE_TRY(check_bank(&L->sh_down, 1, L->H, L->F));
+        if (L->sh_gate.fmt != MOE_FMT_BF16 || L->sh_up.fmt != MOE_FMT_BF16 || L->sh_down.fmt != MOE_FMT_BF16)
+            return MOE_ERR_UNSUPPORTED;
+    }
+    return check_ws(ws, ws_bytes, ws_layout(T, L->H, L->E, L->F, L->top_k).total);
+}
+
+int layer_run(const void* x, int T, const moe_layer* L, void* y, void* ws, cudaStream_t s) {
+    const int H = L->H, E = L->E, F = L->F, k = L->top_k;
+    const WsLayout W = ws_layout(T, H, E, F, k);
+    const int R = T * k;
+    int32_t* status = at<int32_t>(ws, W.ctrl);
+    int32_t* ids = at<int32_t>(ws, W.ids);
+    float* tw = at<float>(ws, W.tw);
+    int32_t* offsets = at<int32_t>(ws, W.offsets);
+    int32_t* row_slot = at<int32_t>(ws, W.row_slot);
+    int32_t* slot_row = at<int32_t>(ws, W.slot_row);
+    __nv_bfloat16* h_perm = at<__nv_bfloat16>(ws, W.h_perm);
+    __nv_bfloat16* y_perm = at<__nv_bfloat16>(ws, W.y_perm);
+    __nv_bfloat16* ys = at<__nv_bfloat16>(ws, W.ys);
+    int32_t* tiles = at<int32_t>(ws, W.tiles);
+    const __nv_bfloat16* xb = reinterpret_cast<const __nv_bfloat16*>(x);
+
+    MOE_TRY(launch_route(xb, T, H, L->router_w, L->router_bias, E, k, ids, tw,
+                         at<float>(ws, W.logits), status, s));
+    MOE_TRY(launch_permute(ids, T, k, E, offsets, row_slot, slot_row, at<int32_t>(ws, W.hist), status, s));
+
+    GemvProblem gu{};
+    gu.act = xb; gu.act_by_token = 1; gu.top_k = k; gu.offsets = offsets; gu.row_slot = row_slot;
+    gu.E = E; gu.topk_w = nullptr; gu.fmt = L->gate.fmt; gu.out_dim = F; gu.in_dim = H;
+    gu.p0 = L->gate.packed; gu.s0 = L->gate.scales; gu.g0 = L->gate.global_scale;
+    gu.p1 = L->up.packed; gu.s1 = L->up.scales; gu.g1 = L->up.global_scale;
+    gu.out = h_perm; gu.status = status;
+    MOE_TRY(run_grouped(gu, true, R, std::min(E, R), tiles, s));
+
+    GemvProblem dn{};
+    dn.act = h_perm; dn.act_by_token = 0; dn.top_k = k; dn.offsets = offsets; dn.row_slot = row_slot;
+    dn.E = E; dn.topk_w = tw; dn.fmt = L->down.fmt; dn.out_dim = H; dn.in_dim = F;
+    dn.p0 = L->down.packed; dn.s0 = L->down.scales; dn.g0 = L->down.global_scale;
+    dn.out = y_perm; dn.status = status;
+    MOE_TRY(run_grouped(dn, false, R, std::min(E, R), tiles, s));
+
+    const bool has_sh = L->sh_gate.packed != nullptr;
+    if (has_sh) {
+        int32_t* sh_off = at<int32_t>(ws, W.sh_offsets);
+        int32_t* sh_rs = at<int32_t>(ws, W.sh_rowslot);
+        __nv_bfloat16* h_sh = h_perm + size_t(R) * F;
+        MOE_TRY(launch_shared_routing(T, k, sh_off, sh_rs, s));
+        GemvProblem sg{};
+        sg.act = xb; sg.act_by_token = 1; sg.top_k = k; sg.offsets = sh_off; sg.row_slot = sh_rs;
+        sg.E = 1; sg.fmt = MOE_FMT_BF16; sg.out_dim = F; sg.in_dim = H;
+        sg.p0 = L->sh_gate.packed; sg.p1 = L->sh_up.packed; sg.out = h_sh; sg.status = status;
+        MOE_TRY(run_grouped(sg, true, T, 1, tiles, s));
+        GemvProblem sd{};
+        sd.act = h_sh; sd.act_by_token = 0; sd.top_k = k; sd.offsets = sh_off; sd.row_slot = sh_rs;
+        sd.E = 1; sd.fmt = MOE_FMT_BF16; sd.out_dim = H; sd.in_dim = F;
+        sd.p0 = L->sh_down.packed; sd.out = ys; sd.status = status;
+        MOE_TRY(run_grouped(sd, false, T, 1, tiles, s));
+    }
+    return launch_combine(y_perm, slot_row, T, k, H, has_sh ? ys : nullptr,
+                          reinterpret_cast<__nv_bfloat16*>(y), s);
+}
+
+}  // namespace
+
+extern "C" {
+
+size_t moe_workspace_bytes(int T, int H, int E, int F, int top_k) {
+    if (check_dims(T, H, E, F, top_k) != MOE_OK) return 0;
+    return ws_layout(std::max(T, 1), H, E, F, top_k).total;
+}
+
+int moe_workspace_init(void* ws, size_t ws_bytes, moe_stream_t stream) {
+    if (!ws) return MOE_ERR_INVALID_ARG;
+    return cudaMemsetAsync(ws, 0, ws_bytes, cs(stream)) == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
+}
+
+int moe_read_status(void* ws, moe_stream_t stream, int32_t* status_out) {
+    if (!ws || !status_out) return MOE_ERR_INVALID_ARG;
+    int32_t v = 0;
+    if (cudaMemcpyAsync(&v, ws, 4, cudaMemcpyDeviceToHost, cs(stream)) != cudaSuccess) return MOE_ERR_CUDA;
+    if (cudaStreamSynchronize(cs(stream)) != cudaSuccess) return MOE_ERR_CUDA;
+    *status_out = v;
+    if (v != 0 && cudaMemsetAsync(ws, 0, 4, cs(stream)) != cudaSuccess) return MOE_ERR_CUDA;
+    return MOE_OK;
+}
+
+const char* moe_status_string(int status) {
+    switch (status) {
+        case MOE_OK: return "ok";
+        case MOE_ERR_INVALID_ARG: return "invalid argument";
+        case MOE_ERR_UNSUPPORTED: return "unsupported shape or format";
+        case MOE_ERR_CUDA: return "CUDA error";
+        case MOE_ERR_TIMEOUT: return "device wait timed out";
+        case MOE_ERR_WORKSPACE: return "workspace missing, misaligned or too small";
+        case MOE_ERR_DEVICE_INDEX: return "index out of range on device";
+    }
+    return "unknown status";
+}
+
+int moe_route_topk(const void* x, int T, int H, const float* router_w, const float* router_bias,
+                   int E, int top_k, int32_t* topk_ids, float* topk_w, void* ws, size_t ws_bytes,
+                   moe_stream_t stream) {
+    if (T < 0 || H <= 0 || E <= 0 || top_k <= 0) return MOE_ERR_INVALID_ARG;
+    if (H % 128 || E > kMaxE || top_k > kMaxTopK || top_k > E) return MOE_ERR_UNSUPPORTED;
+    if (T == 0) return MOE_OK;
+    if (!x || !router_w || !topk_ids || !topk_w || !al16(x) || !al16(router_w)) return MOE_ERR_INVALID_ARG;
+    MOE_TRY(check_ws(ws, ws_bytes, kStepScratch + route_scratch(T, E)));
+    return launch_route(reinterpret_cast<const __nv_bfloat16*>(x), T, H, router_w, router_bias, E,
+                        top_k, topk_ids, topk_w, at<float>(ws, kStepScratch), at<int32_t>(ws, 0),
+                        cs(stream));
+}
+
+int moe_permute(const int32_t* topk_ids, int T, int top_k, int E, int32_t* expert_offsets,
+                int32_t* row_slot, int32_t* slot_row, void* ws, size_t ws_bytes, moe_stream_t stream) {
+    if (T < 0 || top_k <= 0 || E <= 0) return MOE_ERR_INVALID_ARG;
+    if (E > kMaxE || top_k > kMaxTopK) return MOE_ERR_UNSUPPORTED;
+    if (!expert_offsets) return MOE_ERR_INVALID_ARG;
+    if (T == 0) {
+        return cudaMemsetAsync(expert_offsets, 0, size_t(E + 1) * 4, cs(stream)) == cudaSuccess
+                   ? MOE_OK : MOE_ERR_CUDA;
+    }
+    if (!topk_ids || !row_slot || !slot_row) return MOE_ERR_INVALID_ARG;
+    MOE_TRY(check_ws(ws, ws_bytes, kStepScratch + permute_scratch(T, top_k, E)));
+    return launch_permute(topk_ids, T, top_k, E, expert_offsets, row_slot, slot_row,
+                          at<int32_t>(ws, kStepScratch), at<int32_t>(ws, 0), cs(stream));
+}
+
+int moe_grouped_w4a16_swiglu(const void* x, int T, int H, const int32_t* expert_offsets,
+                             const int32_t* row_slot, int top_k, const moe_qweight* gate,
+                             const moe_qweight* up, float swiglu_limit, void* h_perm, void* ws,
+                             size_t ws_bytes, moe_stream_t stream) {
+    if (T < 0 || H <= 0 || top_k <= 0 || !gate || !up) return MOE_ERR_INVALID_ARG;
+    if (swiglu_limit != 0.0f) return MOE_ERR_UNSUPPORTED;
+    if (top_k > kMaxTopK || H % 128) return MOE_ERR_UNSUPPORTED;
+    const int E = gate->num_experts, F = gate->out_dim;
+    if (E <= 0 || E > kMaxE) return MOE_ERR_UNSUPPORTED;
+    MOE_TRY(check_bank(gate, E, F, H));
+    MOE_TRY(check_bank(up, E, F, H));
+    if (gate->fmt != up->fmt || F % 128) return MOE_ERR_UNSUPPORTED;
+    if (T == 0) return MOE_OK;
+    if (!x || !al16(x) || !expert_offsets || !row_slot || !h_perm || !al16(h_perm)) return MOE_ERR_INVALID_ARG;
+    MOE_TRY(check_ws(ws, ws_bytes, kStepScratch + grouped_scratch(E)));
+    // rows present: T * top_k routed slots, or T for a single shared expert
+    const int rows = (E == 1) ? T : T * top_k;
+    GemvProblem p{};
+    p.act = reinterpret_cast<const __nv_bfloat16*>(x); p.act_by_token = 1; p.top_k = top_k;
+    p.offsets = expert_offsets; p.row_slot = row_slot; p.E = E; p.fmt = gate->fmt;
+    p.out_dim = F; p.in_dim = H;
+    p.p0 = gate->packed; p.s0 = gate->scales; p.g0 = gate->global_scale;
+    p.p1 = up->packed; p.s1 = up->scales; p.g1 = up->global_scale;
+    p.out = reinterpret_cast<__nv_bfloat16*>(h_perm); p.status = at<int32_t>(ws, 0);
+    return run_grouped(p, true, rows, std::min(E, rows), at<int32_t>(ws, kStepScratch), cs(stream));
+}
+
+int moe_grouped_w4a16_down(const void* h_perm, const int32_t* expert_offsets, const int32_t* row_slot,
+                           const float* topk_w, int rows, const moe_qweight* down, void* y_perm,
+                           void* ws, size_t ws_bytes, moe_stream_t stream) {
+    if (rows < 0 || !down) return MOE_ERR_INVALID_ARG;
+    const int E = down->num_experts, H = down->out_dim, F = down->in_dim;
+    if (E <= 0 || E > kMaxE) return MOE_ERR_UNSUPPORTED;
+    MOE_TRY(check_bank(down, E, H, F));
+    if (H % 128) return MOE_ERR_UNSUPPORTED;
+    if (rows == 0) return MOE_OK;
+    if (!h_perm || !al16(h_perm) || !expert_offsets || !row_slot || !y_perm || !al16(y_perm))
+        return MOE_ERR_INVALID_ARG;
+    MOE_TRY(check_ws(ws, ws_bytes, kStepScratch + grouped_scratch(E)));
+    GemvProblem p{};
+    p.act = reinterpret_cast<const __nv_bfloat16*>(h_perm); p.act_by_token = 0; p.top_k = 1;
+    p.offsets = expert_offsets; p.row_slot = row_slot; p.E = E; p.topk_w = topk_w;
+    p.fmt = down->fmt; p.out_dim = H; p.in_dim = F;
+    p.p0 = down->packed; p.s0 = down->scales; p.g0 = down->global_scale;
+    p.out = reinterpret_cast<__nv_bfloat16*>(y_perm); p.status = at<int32_t>(ws, 0);
+    return run_grouped(p, false, rows, std::min(E, rows), at<int32_t>(ws, kStepScratch), cs(stream));
+}
+
+int moe_unpermute_combine(const void* y_perm, const int32_t* slot_row, int T, int top_k, int H,
+                          const void* shared_out, void* y, moe_stream_t stream) {
+    if (T < 0 || top_k <= 0 || H <= 0) return MOE_ERR_INVALID_ARG;
+    if (H % 128 || top_k > kMaxTopK) return MOE_ERR_UNSUPPORTED;
+    if (T == 0) return MOE_OK;
+    if (!y_perm || !slot_row || !y || !al16(y_perm) || !al16(y) || (shared_out && !al16(shared_out)))
+        return MOE_ERR_INVALID_ARG;
+    return launch_combine(reinterpret_cast<const __nv_bfloat16*>(y_perm), slot_row, T, top_k, H,
+                          reinterpret_cast<const __nv_bfloat16*>(shared_out),
+                          reinterpret_cast<__nv_bfloat16*>(y), cs(stream));
+}
+
+int moe_layer_decode(const void* x, int T, const moe_layer* L, void* y, void* ws, size_t ws_bytes,
+                     moe_stream_t stream) {
+    MOE_TRY(layer_checks(x, T, L, y, ws, ws_bytes));
+    if (T > kMaxDecodeT) return MOE_ERR_UNSUPPORTED;
+    if (T == 0) return MOE_OK;
+    return layer_run(x, T, L, y, ws, cs(stream));
+}
+
+int moe_layer_forward(const void* x, int T, const moe_layer* L, void* y, void* ws, size_t ws_bytes,
+                      moe_stream_t stream) {
+    MOE_TRY(layer_checks(x, T, L, y, ws, ws_bytes));
+    if (T == 0) return MOE_OK;
+    return layer_run(x, T, L, y, ws, cs(stream));
+}
+
+int moe_quantize_int4_g128(const void* w, int64_t rows, int64_t cols, int32_t* packed, void* scales,
+                           moe_stream_t stream) {
+    if (rows < 0 || cols < 0) return MOE_ERR_INVALID_ARG;
+    if (cols % 128) return MOE_ERR_UNSUPPORTED;
+    if (rows == 0 || cols == 0) return MOE_OK;
+    if (!w || !packed || !scales || !al16(w) || !al16(packed)) return MOE_ERR_INVALID_ARG;
+    return launch_quant_int4(reinterpret_cast<const __nv_bfloat16*>(w), rows, cols, packed,
+                             reinterpret_cast<__nv_bfloat16*>(scales), cs(stream));
+}
+
+int moe_quantize_nvfp4(const void* w, int64_t rows, int64_t cols, uint8_t* packed, uint8_t* scales,
+                       float* global_scale, void* ws, size_t ws_bytes, moe_stream_t stream) {
+    if (rows < 0 || cols < 0) return MOE_ERR_INVALID_ARG;
+    if (cols % 16) return MOE_ERR_UNSUPPORTED;
+    if (rows == 0 || cols == 0) return MOE_OK;
+    if (!w || !packed || !scales || !global_scale || !al16(w)) return MOE_ERR_INVALID_ARG;
+    MOE_TRY(check_ws(ws, ws_bytes, 256));
+    return launch_quant_nvfp4(reinterpret_cast<const __nv_bfloat16*>(w), rows, cols, packed, scales,
+                              global_scale, at<uint32_t>(ws, 8), cs(stream));
+}
+
+}  // extern "C"

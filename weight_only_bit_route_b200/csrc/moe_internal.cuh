@@ -1,0 +1,124 @@
+// Internal declarations of libmoe (sm_100a).  Kernels and host helpers share
+// this header; the public boundary is include/moe_w4a16.h.
+#pragma once
+
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "../../include/moe_w4a16.h"
+
+namespace moe {
+
+constexpr int kMaxE = 1024;
+constexpr int kMaxTopK = 8;
+constexpr int kMaxDecodeT = 64;
+
+// ---------------------------------------------------------------------------
+// Workspace layout.  Every region starts on a 256-byte boundary.
+// ctrl (256 B): [0] status word, [1] router arrival counter, [2] quantiser
+//               amax (float bits), [3..] reserved.
+// ---------------------------------------------------------------------------
+struct WsLayout {
+    size_t ctrl, logits, hist, offsets, row_slot, slot_row, ids, tw;
+    size_t sh_offsets, sh_rowslot, h_perm, y_perm, ys, tiles, total;
+};
+
+constexpr int kPermChunk = 4096;   // slots handled by one bucketing block
+
+inline size_t align256(size_t v) { return (v + 255) & ~size_t(255); }
+
+// Step-level calls use the workspace as [ctrl 256 B][their own scratch].
+constexpr size_t kStepScratch = 256;
+inline size_t route_scratch(int T, int E) { return size_t(T) * E * 4; }
+inline size_t permute_scratch(int T, int k, int E) {
+    size_t R = size_t(T) * k;
+    size_t nb = (R + kPermChunk - 1) / kPermChunk;
+    return (nb ? nb : 1) * E * 4;
+}
+inline size_t grouped_scratch(int E) { return size_t(E + 2) * 16; }
+
+inline WsLayout ws_layout(int T, int H, int E, int F, int k) {
+    WsLayout L{};
+    size_t R = size_t(T) * k;
+    size_t nb = (R + kPermChunk - 1) / kPermChunk;
+    if (nb == 0) nb = 1;
+    size_t o = 0;
+    L.ctrl = o;       o = align256(o + 256);
+    L.logits = o;     o = align256(o + size_t(T) * E * 4);
+    L.hist = o;       o = align256(o + nb * E * 4);
+    L.offsets = o;    o = align256(o + size_t(E + 1) * 4);
+    L.row_slot = o;   o = align256(o + R * 4);
+    L.slot_row = o;   o = align256(o + R * 4);
+    L.ids = o;        o = align256(o + R * 4);
+    L.tw = o;         o = align256(o + R * 4);
+    L.sh_offsets = o; o = align256(o + 2 * 4);
+    L.sh_rowslot = o; o = align256(o + size_t(T) * 4);
+    L.h_perm = o;     o = align256(o + (R + T) * size_t(F) * 2);
+    L.y_perm = o;     o = align256(o + R * size_t(H) * 2);
+    L.ys = o;         o = align256(o + size_t(T) * H * 2);
+    L.tiles = o;      o = align256(o + size_t(E + 2) * 4 * 4);
+    L.total = o;
+    return L;
+}
+
+// ---------------------------------------------------------------------------
+// Device status word: the first error recorded wins.
+// ---------------------------------------------------------------------------
+__device__ __forceinline__ void set_status(int32_t* status, int32_t code) {
+    if (status) atomicCAS(status, 0, code);
+}
+
+__device__ __forceinline__ float bf16_lo(uint32_t v) { return __uint_as_float(v << 16); }
+__device__ __forceinline__ float bf16_hi(uint32_t v) { return __uint_as_float(v & 0xffff0000u); }
+
+__device__ __forceinline__ float warp_sum(float v, int width) {
+    for (int o = width / 2; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+    return v;
+}
+
+// ---------------------------------------------------------------------------
+// Host-side launchers (defined in the .cu files).
+// ---------------------------------------------------------------------------
+int launch_route(const __nv_bfloat16* x, int T, int H, const float* Wr, const float* bias,
+                 int E, int k, int32_t* ids, float* w, float* logits, int32_t* status,
+                 cudaStream_t s);
+
+int launch_permute(const int32_t* ids, int T, int k, int E, int32_t* offsets,
+                   int32_t* row_slot, int32_t* slot_row, int32_t* hist, int32_t* status,
+                   cudaStream_t s);
+
+struct GemvProblem {
+    const __nv_bfloat16* act;  // gate/up: x [T, in]; down: h_perm [rows, in]
+    int act_by_token;          // 1: activation row = row_slot[r] / top_k; 0: row r
+    int top_k;
+    const int32_t* offsets;    // [E+1]
+    const int32_t* row_slot;   // [rows]
+    int E;
+    const float* topk_w;       // down only: weight by slot (nullable)
+    int fmt, out_dim, in_dim;
+    const void* p0; const void* s0; const float* g0;   // gate (or down)
+    const void* p1; const void* s1; const float* g1;   // up (gate/up only)
+    __nv_bfloat16* out;        // [rows, out_dim]
+    int32_t* status;
+};
+
+int launch_grouped_gemv(const GemvProblem& p, bool gateup, int max_touched,
+                        cudaStream_t s);
+
+int launch_combine(const __nv_bfloat16* y_perm, const int32_t* slot_row, int T, int k, int H,
+                   const __nv_bfloat16* shared_out, __nv_bfloat16* y, cudaStream_t s);
+
+int launch_quant_int4(const __nv_bfloat16* w, int64_t rows, int64_t cols, int32_t* packed,
+                      __nv_bfloat16* scales, cudaStream_t s);
+int launch_quant_nvfp4(const __nv_bfloat16* w, int64_t rows, int64_t cols, uint8_t* packed,
+                       uint8_t* scales, float* global, uint32_t* amax_slot, cudaStream_t s);
+
+int launch_shared_routing(int T, int k, int32_t* sh_offsets, int32_t* sh_rowslot,
+                          cudaStream_t s);
+
+struct GemmProblem;   // tcgen05 grouped GEMM (prefill), see gemm_tc.cu
+int launch_grouped_gemm(const GemvProblem& p, bool gateup, int rows_total, int max_touched,
+                        int32_t* tile_ws, cudaStream_t s);
+
+}  // namespace moe
