@@ -51,12 +51,12 @@ int check_ws(void* ws, size_t ws_bytes, size_t need) {
 // decode-sized calls stream weights with the GEMV; larger ones use the GEMM
 constexpr int kGemvMaxRows = 256;
 
-// rows_total: rows present over all experts; max_touched: bound on the number
-// of experts holding at least one row (sizes the persistent grid).
-int run_grouped(const GemvProblem& p, bool gateup, int rows_total, int max_touched,
-                int32_t* tile_ws, cudaStream_t s) {
-    if (rows_total <= kGemvMaxRows) return launch_grouped_gemv(p, gateup, max_touched, s);
-    return launch_grouped_gemm(p, gateup, rows_total, max_touched, tile_ws, s);
+// rows_total: rows present over all experts of the routed problem; act_rows:
+// its activation rows (T for gate/up, rows for down).
+int run_grouped(const GemvProblem& p, const GemvProblem* shared, bool gateup, int rows_total, int act_rows,
+                void* prep_ws, int32_t* tile_ws, cudaStream_t s) {
+    if (rows_total <= kGemvMaxRows) return launch_stream_gemv(p, shared, gateup, act_rows, prep_ws, s, false);
+    return launch_grouped_gemm(p, shared, gateup, act_rows, prep_ws, tile_ws, s);
 }
 
 int layer_checks(const void* x, int T, const moe_layer* L, void* y, void* ws, size_t ws_bytes) {
@@ -98,9 +98,27 @@ int layer_run(const void* x, int T, const moe_layer* L, void* y, void* ws, cudaS
     int32_t* tiles = at<int32_t>(ws, W.tiles);
     const __nv_bfloat16* xb = reinterpret_cast<const __nv_bfloat16*>(x);
 
-    MOE_TRY(launch_route(xb, T, H, L->router_w, L->router_bias, E, k, ids, tw,
-                         at<float>(ws, W.logits), status, s));
-    MOE_TRY(launch_permute(ids, T, k, E, offsets, row_slot, slot_row, at<int32_t>(ws, W.hist), status, s));
+    const bool has_sh = L->sh_gate.packed != nullptr;
+    int32_t* sh_off = at<int32_t>(ws, W.sh_offsets);
+    int32_t* sh_rs = at<int32_t>(ws, W.sh_rowslot);
+    int32_t* counter = status + 1;
+    if (T <= kRouterDecodeMaxT) {
+        // router, top-k, bucketing and shared routing in one launch
+        RouterDecodeArgs ra{};
+        ra.x = xb; ra.T = T; ra.H = H; ra.Wr = L->router_w; ra.bias = L->router_bias; ra.E = E; ra.k = k;
+        ra.logits = at<float>(ws, W.logits); ra.ids = ids; ra.w = tw; ra.counter = counter; ra.status = status;
+        ra.offsets = offsets; ra.row_slot = row_slot; ra.slot_row = slot_row;
+        ra.sh_offsets = has_sh ? sh_off : nullptr; ra.sh_rowslot = has_sh ? sh_rs : nullptr;
+        MOE_TRY(launch_route_decode(ra, s));
+    } else {
+        MOE_TRY(launch_route(xb, T, H, L->router_w, L->router_bias, E, k, ids, tw, at<float>(ws, W.logits),
+                             status, counter, s));
+        MOE_TRY(launch_permute(ids, T, k, E, offsets, row_slot, slot_row, at<int32_t>(ws, W.hist), status, s));
+        if (has_sh) MOE_TRY(launch_shared_routing(T, k, sh_off, sh_rs, s));
+    }
+
+    void* prep = at<void>(ws, W.prep);
+    __nv_bfloat16* h_sh = h_perm + size_t(R) * F;
 
     GemvProblem gu{};
     gu.act = xb; gu.act_by_token = 1; gu.top_k = k; gu.offsets = offsets; gu.row_slot = row_slot;
@@ -108,32 +126,23 @@ int layer_run(const void* x, int T, const moe_layer* L, void* y, void* ws, cudaS
     gu.p0 = L->gate.packed; gu.s0 = L->gate.scales; gu.g0 = L->gate.global_scale;
     gu.p1 = L->up.packed; gu.s1 = L->up.scales; gu.g1 = L->up.global_scale;
     gu.out = h_perm; gu.status = status;
-    MOE_TRY(run_grouped(gu, true, R, std::min(E, R), tiles, s));
+    GemvProblem sg{};
+    sg.act = xb; sg.act_by_token = 1; sg.top_k = k; sg.offsets = sh_off; sg.row_slot = sh_rs;
+    sg.E = 1; sg.fmt = MOE_FMT_BF16; sg.out_dim = F; sg.in_dim = H;
+    sg.p0 = L->sh_gate.packed; sg.p1 = L->sh_up.packed; sg.out = h_sh; sg.status = status;
+    MOE_TRY(run_grouped(gu, has_sh ? &sg : nullptr, true, R, T, prep, tiles, s));
 
     GemvProblem dn{};
     dn.act = h_perm; dn.act_by_token = 0; dn.top_k = k; dn.offsets = offsets; dn.row_slot = row_slot;
     dn.E = E; dn.topk_w = tw; dn.fmt = L->down.fmt; dn.out_dim = H; dn.in_dim = F;
     dn.p0 = L->down.packed; dn.s0 = L->down.scales; dn.g0 = L->down.global_scale;
     dn.out = y_perm; dn.status = status;
-    MOE_TRY(run_grouped(dn, false, R, std::min(E, R), tiles, s));
+    GemvProblem sd{};
+    sd.act = h_sh; sd.act_by_token = 0; sd.top_k = k; sd.offsets = sh_off; sd.row_slot = sh_rs;
+    sd.E = 1; sd.fmt = MOE_FMT_BF16; sd.out_dim = H; sd.in_dim = F;
+    sd.p0 = L->sh_down.packed; sd.out = ys; sd.status = status;
+    MOE_TRY(run_grouped(dn, has_sh ? &sd : nullptr, false, R, R, prep, tiles, s));
 
-    const bool has_sh = L->sh_gate.packed != nullptr;
-    if (has_sh) {
-        int32_t* sh_off = at<int32_t>(ws, W.sh_offsets);
-        int32_t* sh_rs = at<int32_t>(ws, W.sh_rowslot);
-        __nv_bfloat16* h_sh = h_perm + size_t(R) * F;
-        MOE_TRY(launch_shared_routing(T, k, sh_off, sh_rs, s));
-        GemvProblem sg{};
-        sg.act = xb; sg.act_by_token = 1; sg.top_k = k; sg.offsets = sh_off; sg.row_slot = sh_rs;
-        sg.E = 1; sg.fmt = MOE_FMT_BF16; sg.out_dim = F; sg.in_dim = H;
-        sg.p0 = L->sh_gate.packed; sg.p1 = L->sh_up.packed; sg.out = h_sh; sg.status = status;
-        MOE_TRY(run_grouped(sg, true, T, 1, tiles, s));
-        GemvProblem sd{};
-        sd.act = h_sh; sd.act_by_token = 0; sd.top_k = k; sd.offsets = sh_off; sd.row_slot = sh_rs;
-        sd.E = 1; sd.fmt = MOE_FMT_BF16; sd.out_dim = H; sd.in_dim = F;
-        sd.p0 = L->sh_down.packed; sd.out = ys; sd.status = status;
-        MOE_TRY(run_grouped(sd, false, T, 1, tiles, s));
-    }
     return launch_combine(y_perm, slot_row, T, k, H, has_sh ? ys : nullptr,
                           reinterpret_cast<__nv_bfloat16*>(y), s);
 }
@@ -185,7 +194,7 @@ int moe_route_topk(const void* x, int T, int H, const float* router_w, const flo
     MOE_TRY(check_ws(ws, ws_bytes, kStepScratch + route_scratch(T, E)));
     return launch_route(reinterpret_cast<const __nv_bfloat16*>(x), T, H, router_w, router_bias, E,
                         top_k, topk_ids, topk_w, at<float>(ws, kStepScratch), at<int32_t>(ws, 0),
-                        cs(stream));
+                        at<int32_t>(ws, 4), cs(stream));
 }
 
 int moe_permute(const int32_t* topk_ids, int T, int top_k, int E, int32_t* expert_offsets,
@@ -217,7 +226,7 @@ int moe_grouped_w4a16_swiglu(const void* x, int T, int H, const int32_t* expert_
     if (gate->fmt != up->fmt || F % 128) return MOE_ERR_UNSUPPORTED;
     if (T == 0) return MOE_OK;
     if (!x || !al16(x) || !expert_offsets || !row_slot || !h_perm || !al16(h_perm)) return MOE_ERR_INVALID_ARG;
-    MOE_TRY(check_ws(ws, ws_bytes, kStepScratch + grouped_scratch(E)));
+    MOE_TRY(check_ws(ws, ws_bytes, kStepScratch + grouped_scratch(E, T, H)));
     // rows present: T * top_k routed slots, or T for a single shared expert
     const int rows = (E == 1) ? T : T * top_k;
     GemvProblem p{};
@@ -227,7 +236,8 @@ int moe_grouped_w4a16_swiglu(const void* x, int T, int H, const int32_t* expert_
     p.p0 = gate->packed; p.s0 = gate->scales; p.g0 = gate->global_scale;
     p.p1 = up->packed; p.s1 = up->scales; p.g1 = up->global_scale;
     p.out = reinterpret_cast<__nv_bfloat16*>(h_perm); p.status = at<int32_t>(ws, 0);
-    return run_grouped(p, true, rows, std::min(E, rows), at<int32_t>(ws, kStepScratch), cs(stream));
+    return run_grouped(p, nullptr, true, rows, T, at<void>(ws, kStepScratch + align256(size_t(E + 2) * 16)),
+                       at<int32_t>(ws, kStepScratch), cs(stream));
 }
 
 int moe_grouped_w4a16_down(const void* h_perm, const int32_t* expert_offsets, const int32_t* row_slot,
@@ -241,14 +251,15 @@ int moe_grouped_w4a16_down(const void* h_perm, const int32_t* expert_offsets, co
     if (rows == 0) return MOE_OK;
     if (!h_perm || !al16(h_perm) || !expert_offsets || !row_slot || !y_perm || !al16(y_perm))
         return MOE_ERR_INVALID_ARG;
-    MOE_TRY(check_ws(ws, ws_bytes, kStepScratch + grouped_scratch(E)));
+    MOE_TRY(check_ws(ws, ws_bytes, kStepScratch + grouped_scratch(E, rows, F)));
     GemvProblem p{};
     p.act = reinterpret_cast<const __nv_bfloat16*>(h_perm); p.act_by_token = 0; p.top_k = 1;
     p.offsets = expert_offsets; p.row_slot = row_slot; p.E = E; p.topk_w = topk_w;
     p.fmt = down->fmt; p.out_dim = H; p.in_dim = F;
     p.p0 = down->packed; p.s0 = down->scales; p.g0 = down->global_scale;
     p.out = reinterpret_cast<__nv_bfloat16*>(y_perm); p.status = at<int32_t>(ws, 0);
-    return run_grouped(p, false, rows, std::min(E, rows), at<int32_t>(ws, kStepScratch), cs(stream));
+    return run_grouped(p, nullptr, false, rows, rows, at<void>(ws, kStepScratch + align256(size_t(E + 2) * 16)),
+                       at<int32_t>(ws, kStepScratch), cs(stream));
 }
 
 int moe_unpermute_combine(const void* y_perm, const int32_t* slot_row, int T, int top_k, int H,

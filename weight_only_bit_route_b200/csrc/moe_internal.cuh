@@ -6,6 +6,8 @@
 #include <cuda_runtime.h>
 #include <stdint.h>
 
+#include <algorithm>
+
 #include "../../include/moe_w4a16.h"
 
 namespace moe {
@@ -21,12 +23,27 @@ constexpr int kMaxDecodeT = 64;
 // ---------------------------------------------------------------------------
 struct WsLayout {
     size_t ctrl, logits, hist, offsets, row_slot, slot_row, ids, tw;
-    size_t sh_offsets, sh_rowslot, h_perm, y_perm, ys, tiles, total;
+    size_t sh_offsets, sh_rowslot, h_perm, y_perm, ys, tiles, prep, total;
 };
 
 constexpr int kPermChunk = 4096;   // slots handled by one bucketing block
 
 inline size_t align256(size_t v) { return (v + 255) & ~size_t(255); }
+
+// ---------------------------------------------------------------------------
+// Device status word: the first error recorded wins.
+// ---------------------------------------------------------------------------
+__device__ __forceinline__ void set_status(int32_t* status, int32_t code) {
+    if (status) atomicCAS(status, 0, code);
+}
+
+__device__ __forceinline__ float bf16_lo(uint32_t v) { return __uint_as_float(v << 16); }
+__device__ __forceinline__ float bf16_hi(uint32_t v) { return __uint_as_float(v & 0xffff0000u); }
+
+__device__ __forceinline__ float warp_sum(float v, int width) {
+    for (int o = width / 2; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+    return v;
+}
 
 // Step-level calls use the workspace as [ctrl 256 B][their own scratch].
 constexpr size_t kStepScratch = 256;
@@ -36,7 +53,14 @@ inline size_t permute_scratch(int T, int k, int E) {
     size_t nb = (R + kPermChunk - 1) / kPermChunk;
     return (nb ? nb : 1) * E * 4;
 }
-inline size_t grouped_scratch(int E) { return size_t(E + 2) * 16; }
+// Activation pre-pass output of the streaming GEMV (largest over formats):
+// int4 chunk sums [rows, in/32] fp32 + a reordered bf16 copy [rows, in].
+inline size_t prep_scratch(int rows, int in_dim) {
+    return align256(size_t(rows) * (in_dim / 32) * 4) + align256(size_t(rows) * in_dim * 2);
+}
+inline size_t grouped_scratch(int E, int act_rows, int in_dim) {
+    return align256(size_t(E + 2) * 16) + prep_scratch(act_rows, in_dim);
+}
 
 inline WsLayout ws_layout(int T, int H, int E, int F, int k) {
     WsLayout L{};
@@ -58,31 +82,31 @@ inline WsLayout ws_layout(int T, int H, int E, int F, int k) {
     L.y_perm = o;     o = align256(o + R * size_t(H) * 2);
     L.ys = o;         o = align256(o + size_t(T) * H * 2);
     L.tiles = o;      o = align256(o + size_t(E + 2) * 4 * 4);
+    L.prep = o;       o = align256(o + std::max(prep_scratch(T, H), prep_scratch(int(R), F)));
     L.total = o;
     return L;
 }
 
 // ---------------------------------------------------------------------------
-// Device status word: the first error recorded wins.
-// ---------------------------------------------------------------------------
-__device__ __forceinline__ void set_status(int32_t* status, int32_t code) {
-    if (status) atomicCAS(status, 0, code);
-}
-
-__device__ __forceinline__ float bf16_lo(uint32_t v) { return __uint_as_float(v << 16); }
-__device__ __forceinline__ float bf16_hi(uint32_t v) { return __uint_as_float(v & 0xffff0000u); }
-
-__device__ __forceinline__ float warp_sum(float v, int width) {
-    for (int o = width / 2; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
-    return v;
-}
-
-// ---------------------------------------------------------------------------
 // Host-side launchers (defined in the .cu files).
 // ---------------------------------------------------------------------------
+constexpr int kRouterDecodeMaxT = 16;
+
+// Router: logits + sigmoid top-k.  counter: a zeroed int in the workspace
+// (enables the fused decode router for T <= kRouterDecodeMaxT), or null.
 int launch_route(const __nv_bfloat16* x, int T, int H, const float* Wr, const float* bias,
                  int E, int k, int32_t* ids, float* w, float* logits, int32_t* status,
-                 cudaStream_t s);
+                 int32_t* counter, cudaStream_t s);
+
+struct RouterDecodeArgs {
+    const __nv_bfloat16* x; int T, H; const float* Wr; const float* bias; int E, k;
+    float* logits; int32_t* ids; float* w;
+    int32_t* counter; int32_t* status;
+    int32_t* offsets; int32_t* row_slot; int32_t* slot_row;     // bucketing (nullable: skip)
+    int32_t* sh_offsets; int32_t* sh_rowslot;                   // shared routing (nullable: skip)
+};
+// Fused decode router: logits, top-k, bucketing and shared routing in one launch.
+int launch_route_decode(const RouterDecodeArgs& a, cudaStream_t s);
 
 int launch_permute(const int32_t* ids, int T, int k, int E, int32_t* offsets,
                    int32_t* row_slot, int32_t* slot_row, int32_t* hist, int32_t* status,
@@ -103,8 +127,11 @@ struct GemvProblem {
     int32_t* status;
 };
 
-int launch_grouped_gemv(const GemvProblem& p, bool gateup, int max_touched,
-                        cudaStream_t s);
+// Streaming grouped GEMV (decode): routed bank plus an optional BF16 shared
+// bank in one launch.  act_rows: activation rows of the routed problem (T for
+// gate/up, rows for down); prep_ws: prep_scratch(act_rows, in_dim) bytes.
+int launch_stream_gemv(const GemvProblem& routed, const GemvProblem* shared, bool gateup, int act_rows,
+                       void* prep_ws, cudaStream_t s, bool pdl);
 
 int launch_combine(const __nv_bfloat16* y_perm, const int32_t* slot_row, int T, int k, int H,
                    const __nv_bfloat16* shared_out, __nv_bfloat16* y, cudaStream_t s);
@@ -117,8 +144,8 @@ int launch_quant_nvfp4(const __nv_bfloat16* w, int64_t rows, int64_t cols, uint8
 int launch_shared_routing(int T, int k, int32_t* sh_offsets, int32_t* sh_rowslot,
                           cudaStream_t s);
 
-struct GemmProblem;   // tcgen05 grouped GEMM (prefill), see gemm_tc.cu
-int launch_grouped_gemm(const GemvProblem& p, bool gateup, int rows_total, int max_touched,
-                        int32_t* tile_ws, cudaStream_t s);
+// Prefill-shaped grouped GEMM (tcgen05), same contract as launch_stream_gemv.
+int launch_grouped_gemm(const GemvProblem& routed, const GemvProblem* shared, bool gateup, int act_rows,
+                        void* prep_ws, int32_t* tile_ws, cudaStream_t s);
 
 }  // namespace moe

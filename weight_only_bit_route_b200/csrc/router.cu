@@ -6,11 +6,12 @@
 //   ids    = top_k of s, ties to the lower expert id, by descending s
 //   w      = s_sel / sum(s_sel)                     fp32
 //
-// Two logit kernels: for few tokens (decode) one warp streams one router row
-// (16 KB at H = 4096) against every token, so the 5.8 MB of router weights
-// are read once across ~100 CTAs; for many tokens a register-tiled fp32 SIMT
-// GEMM.  A warp-per-token kernel then does the sigmoid, selection and
+// Decode (T <= 16): one fused kernel, see router_decode below.  Otherwise two
+// logit kernels (warp per router row for T <= 32, a register-tiled fp32 SIMT
+// GEMM above) and a warp-per-token kernel for the sigmoid, selection and
 // renormalisation.
+#include <algorithm>
+
 #include "moe_internal.cuh"
 
 namespace moe {
@@ -115,66 +116,245 @@ __global__ void __launch_bounds__(256) router_logits_tiled(
 }
 
 // ---------------------------------------------------------------------------
-// Sigmoid + top-k + renormalisation: warp per token.
+// Sigmoid + top-k + renormalisation for one token, by one warp.  PER is the
+// number of experts each lane holds (ceil(E / 32) rounded to a supported size).
 // ---------------------------------------------------------------------------
+template <int PER>
+__device__ __forceinline__ void topk_warp(const float* __restrict__ lrow, const float* __restrict__ bias, int E,
+                                          int k, int32_t* __restrict__ ids, float* __restrict__ wout, int lane) {
+    float s[PER];
+#pragma unroll
+    for (int i = 0; i < PER; i++) {
+        const int e = lane + 32 * i;
+        float v = -INFINITY;
+        if (e < E) {
+            float l = __ldcg(lrow + e);       // written by other CTAs of the fused router
+            if (bias) l = l + bias[e];
+            v = 1.0f / (1.0f + expf(-l));
+        }
+        s[i] = v;
+    }
+    float sum = 0.f, my_s = 0.f;
+    int my_id = 0;
+    for (int j = 0; j < k; j++) {
+        // largest s, lowest id on ties (ids grow with i)
+        float bv = -INFINITY;
+        int bi = 0x7fffffff;
+#pragma unroll
+        for (int i = 0; i < PER; i++) {
+            const int e = lane + 32 * i;
+            if (e < E && (s[i] > bv || (s[i] == bv && e < bi))) { bv = s[i]; bi = e; }
+        }
+        for (int o = 16; o > 0; o >>= 1) {
+            const float ov = __shfl_xor_sync(0xffffffffu, bv, o);
+            const int oi = __shfl_xor_sync(0xffffffffu, bi, o);
+            if (ov > bv || (ov == bv && oi < bi)) { bv = ov; bi = oi; }
+        }
+        if ((bi & 31) == lane) {
+#pragma unroll
+            for (int i = 0; i < PER; i++)
+                if (lane + 32 * i == bi) s[i] = -INFINITY;
+        }
+        if (lane == j) { my_s = bv; my_id = bi; }
+        sum = sum + bv;
+    }
+    if (lane < k) {
+        ids[lane] = my_id;
+        wout[lane] = my_s / sum;
+    }
+}
+
 __global__ void __launch_bounds__(256) router_topk(
         const float* __restrict__ logits, const float* __restrict__ bias, int T, int E, int k,
         int32_t* __restrict__ ids, float* __restrict__ wout) {
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int t = blockIdx.x * (blockDim.x >> 5) + warp;
     if (t >= T) return;
-    constexpr int PER = kMaxE / 32;
-    float s[PER];
-#pragma unroll
-    for (int i = 0; i < PER; i++) {
-        int e = lane + 32 * i;
-        float v = -INFINITY;
-        if (e < E) {
-            float l = logits[size_t(t) * E + e];
-            if (bias) l = l + bias[e];
-            v = 1.0f / (1.0f + expf(-l));
-        }
-        s[i] = v;
+    if (E <= 384) topk_warp<12>(logits + size_t(t) * E, bias, E, k, ids + size_t(t) * k, wout + size_t(t) * k, lane);
+    else topk_warp<kMaxE / 32>(logits + size_t(t) * E, bias, E, k, ids + size_t(t) * k, wout + size_t(t) * k, lane);
+}
+
+// ---------------------------------------------------------------------------
+// Fused decode router (T <= 16): logits, then the last CTA to finish does the
+// top-k of every token, the stable bucketing of the T*k slots and the shared
+// expert's routing.  Each warp owns one router row (16 KB at H = 4096) and
+// multiplies it with every token's activations, staged once per CTA in shared
+// memory; the router weights are read once in total across ~90 CTAs.  The
+// last CTA is found with an arrival counter in the workspace (no waiting);
+// it leaves the counter at zero for the next call.
+// ---------------------------------------------------------------------------
+constexpr int RD_WARPS = 4;
+constexpr int RD_TG = 8;            // tokens per staging pass
+
+
+
+__global__ void __launch_bounds__(RD_WARPS * 32) router_decode(RouterDecodeArgs a) {
+    extern __shared__ __align__(16) uint8_t rsm[];
+    __shared__ int s_last;
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int e = blockIdx.x * RD_WARPS + warp;
+    __nv_bfloat16* xs = reinterpret_cast<__nv_bfloat16*>(rsm);
+    __shared__ __align__(8) uint64_t bar;
+    const uint32_t bar_a = static_cast<uint32_t>(__cvta_generic_to_shared(&bar));
+    const uint32_t xs_a = static_cast<uint32_t>(__cvta_generic_to_shared(xs));
+    if (threadIdx.x == 0) {
+        asm volatile("mbarrier.init.shared::cta.b64 [%0], 1;" ::"r"(bar_a));
+        asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
     }
-    float sel[kMaxTopK];
-    int sel_id[kMaxTopK];
-    float sum = 0.f;
-    for (int j = 0; j < k; j++) {
-        // local best: largest s, lowest id on ties (ids grow with i)
-        float bv = -INFINITY;
-        int bi = 0x7fffffff;
+    __syncthreads();
+    int phase = 0;
+    for (int t0 = 0; t0 < a.T; t0 += RD_TG, phase ^= 1) {
+        const int nt = min(RD_TG, a.T - t0);
+        __syncthreads();                                 // previous pass done with xs
+        if (threadIdx.x == 0) {                          // one bulk copy of nt token rows
+            const uint32_t bytes = uint32_t(nt) * a.H * 2;
+            asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(bar_a), "r"(bytes) : "memory");
+            asm volatile("cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];"
+                         ::"r"(xs_a), "l"(a.x + size_t(t0) * a.H), "r"(bytes), "r"(bar_a) : "memory");
+        }
+        // router row of this warp, 4 floats per lane per step, 8 steps in flight
+        float acc[RD_TG];
 #pragma unroll
-        for (int i = 0; i < PER; i++) {
-            int e = lane + 32 * i;
-            if (e < E && (s[i] > bv || (s[i] == bv && e < bi))) { bv = s[i]; bi = e; }
-        }
-        for (int o = 16; o > 0; o >>= 1) {
-            float ov = __shfl_xor_sync(0xffffffffu, bv, o);
-            int oi = __shfl_xor_sync(0xffffffffu, bi, o);
-            if (ov > bv || (ov == bv && oi < bi)) { bv = ov; bi = oi; }
-        }
-        // the owner removes the winner from its candidates
-        if ((bi & 31) == lane) {
+        for (int t = 0; t < RD_TG; t++) acc[t] = 0.f;
+        const float* wrow = a.Wr + size_t(e < a.E ? e : 0) * a.H;
+        bool ready = false;
+        for (int h0 = 0; h0 < a.H; h0 += 8 * 128) {
+            float4 wv[8];
 #pragma unroll
-            for (int i = 0; i < PER; i++)
-                if (lane + 32 * i == bi) s[i] = -INFINITY;
+            for (int q = 0; q < 8; q++) {
+                const int h = h0 + q * 128 + lane * 4;
+                wv[q] = (h < a.H) ? __ldg(reinterpret_cast<const float4*>(wrow + h)) : make_float4(0, 0, 0, 0);
+            }
+            if (!ready) {                                  // activations landed (bounded wait)
+                uint32_t ok = 0;
+                unsigned long long t_start, t_now;
+                asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t_start));
+                while (!ok) {
+                    asm volatile("{ .reg .pred p; mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2; selp.u32 %0, 1, 0, p; }"
+                                 : "=r"(ok) : "r"(bar_a), "r"(phase) : "memory");
+                    asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t_now));
+                    if (!ok && t_now - t_start > 2000000000ull) { set_status(a.status, MOE_ERR_TIMEOUT); break; }
+                }
+                ready = true;
+            }
+#pragma unroll
+            for (int q = 0; q < 8; q++) {
+                const int h = h0 + q * 128 + lane * 4;
+                if (h < a.H) {
+#pragma unroll
+                    for (int t = 0; t < RD_TG; t++) {
+                        if (t < nt) {
+                            const uint2 xv = *reinterpret_cast<const uint2*>(xs + t * a.H + h);
+                            float v = acc[t];
+                            v = fmaf(bf16_lo(xv.x), wv[q].x, v); v = fmaf(bf16_hi(xv.x), wv[q].y, v);
+                            v = fmaf(bf16_lo(xv.y), wv[q].z, v); v = fmaf(bf16_hi(xv.y), wv[q].w, v);
+                            acc[t] = v;
+                        }
+                    }
+                }
+            }
         }
-        sel[j] = bv;
-        sel_id[j] = bi;
-        sum = sum + bv;
+#pragma unroll
+        for (int t = 0; t < RD_TG; t++) {
+            const float v = warp_sum(acc[t], 32);
+            if (lane == 0 && t < nt && e < a.E) a.logits[size_t(t0 + t) * a.E + e] = v;
+        }
     }
-    if (lane == 0) {
-        for (int j = 0; j < k; j++) {
-            ids[size_t(t) * k + j] = sel_id[j];
-            wout[size_t(t) * k + j] = sel[j] / sum;
+    // last CTA to arrive continues
+    __threadfence();
+    __syncthreads();
+    if (threadIdx.x == 0) s_last = (atomicAdd(a.counter, 1) == int(gridDim.x) - 1);
+    __syncthreads();
+    if (!s_last) return;
+    __threadfence();
+    for (int t = warp; t < a.T; t += RD_WARPS) {
+        if (a.E <= 384) topk_warp<12>(a.logits + size_t(t) * a.E, a.bias, a.E, a.k, a.ids + size_t(t) * a.k, a.w + size_t(t) * a.k, lane);
+        else topk_warp<kMaxE / 32>(a.logits + size_t(t) * a.E, a.bias, a.E, a.k, a.ids + size_t(t) * a.k, a.w + size_t(t) * a.k, lane);
+    }
+    if (threadIdx.x == 0) *a.counter = 0;
+    if (a.sh_offsets) {
+        if (threadIdx.x == 0) { a.sh_offsets[0] = 0; a.sh_offsets[1] = a.T; }
+        for (int i = threadIdx.x; i < a.T; i += blockDim.x) a.sh_rowslot[i] = i * a.k;
+    }
+    if (!a.offsets) return;
+    __syncthreads();                       // ids of every token written (by this CTA)
+    // stable counting sort of the R <= 128 slots by expert id
+    int32_t* cnt = reinterpret_cast<int32_t*>(rsm);          // [E] (x staging is no longer needed)
+    __shared__ int s_wsum[RD_WARPS];
+    const int R = a.T * a.k;
+    for (int i = threadIdx.x; i < a.E; i += blockDim.x) cnt[i] = 0;
+    __syncthreads();
+    for (int sl = threadIdx.x; sl < R; sl += blockDim.x) {
+        const int id = a.ids[sl];
+        if (id >= 0 && id < a.E) atomicAdd(&cnt[id], 1);
+        else set_status(a.status, MOE_ERR_DEVICE_INDEX);
+    }
+    __syncthreads();
+    // exclusive scan of cnt over E: each thread a contiguous run of experts
+    const int per = (a.E + blockDim.x - 1) / blockDim.x;
+    const int b0 = threadIdx.x * per, b1 = min(a.E, b0 + per);
+    int local = 0;
+    for (int i = b0; i < b1; i++) local += cnt[i];
+    int v = local;
+    for (int o = 1; o < 32; o <<= 1) {
+        const int n = __shfl_up_sync(0xffffffffu, v, o);
+        if (lane >= o) v += n;
+    }
+    if (lane == 31) s_wsum[warp] = v;
+    __syncthreads();
+    int base = 0;
+    for (int q = 0; q < warp; q++) base += s_wsum[q];
+    int run = base + v - local;
+    for (int i = b0; i < b1; i++) {
+        const int c = cnt[i];
+        a.offsets[i] = run;
+        cnt[i] = run;                        // becomes the next free row of expert i
+        run += c;
+    }
+    if (threadIdx.x == blockDim.x - 1) a.offsets[a.E] = base + v;
+    __syncthreads();
+    if (warp == 0) {
+        const unsigned lt = (1u << lane) - 1u;
+        for (int s0 = 0; s0 < R; s0 += 32) {
+            const int sl = s0 + lane;
+            const int id = (sl < R) ? a.ids[sl] : -1;
+            const bool ok = id >= 0 && id < a.E;
+            const unsigned act = __ballot_sync(0xffffffffu, ok);
+            const unsigned peers = __match_any_sync(0xffffffffu, ok ? id : -1) & act;
+            int pos = 0;
+            if (ok) pos = cnt[id] + __popc(peers & lt);
+            __syncwarp();
+            if (ok && (__ffs(peers) - 1) == lane) cnt[id] += __popc(peers);
+            __syncwarp();
+            if (sl < R) {
+                if (ok) { a.row_slot[pos] = sl; a.slot_row[sl] = pos; }
+                else a.slot_row[sl] = -1;
+            }
         }
     }
 }
 
+int launch_route_decode(const RouterDecodeArgs& a, cudaStream_t s) {
+    const size_t smem = std::max<size_t>(size_t(RD_TG) * a.H * 2, size_t(a.E) * 4);
+    static size_t smem_set = 0;
+    if (smem > 48 * 1024 && smem > smem_set) {
+        if (cudaFuncSetAttribute(router_decode, cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem)) != cudaSuccess)
+            return MOE_ERR_UNSUPPORTED;
+        smem_set = smem;
+    }
+    router_decode<<<(a.E + RD_WARPS - 1) / RD_WARPS, RD_WARPS * 32, smem, s>>>(a);
+    return cudaGetLastError() == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
+}
+
 int launch_route(const __nv_bfloat16* x, int T, int H, const float* Wr, const float* bias,
                  int E, int k, int32_t* ids, float* w, float* logits, int32_t* status,
-                 cudaStream_t s) {
-    (void)status;
+                 int32_t* counter, cudaStream_t s) {
+    if (T <= kRouterDecodeMaxT && counter) {
+        RouterDecodeArgs a{};
+        a.x = x; a.T = T; a.H = H; a.Wr = Wr; a.bias = bias; a.E = E; a.k = k;
+        a.logits = logits; a.ids = ids; a.w = w; a.counter = counter; a.status = status;
+        return launch_route_decode(a, s);
+    }
     if (T <= 32) {
         dim3 block(256);
         int epb = 8;
