@@ -163,10 +163,15 @@ def test_permute_reports_bad_id():
 # grouped gate/up + SwiGLU, grouped down, combine (per step)
 # ---------------------------------------------------------------------------
 
-@pytest.mark.parametrize("fmt", ["int4", "nvfp4"])
-def test_grouped_swiglu(fmt):
-    wl = syn.WORKLOADS[0] if fmt == "int4" else syn.Workload("tiny_nvfp4", 16, 1024, 32, 256, 8, "nvfp4", False,
-                                                                1 / 32.0, False)
+def _tiny(fmt, T):
+    base = syn.WORKLOADS[0]
+    return syn.Workload(f"tiny_{fmt}_T{T}", T, base.H, base.E, base.F, base.k, fmt, False, base.router_std, False)
+
+
+# T = 16 gives 128 rows (streaming GEMV); T = 96 gives 768 rows (tcgen05 GEMM)
+@pytest.mark.parametrize("fmt,T", [("int4", 16), ("nvfp4", 16), ("int4", 96), ("nvfp4", 96)])
+def test_grouped_swiglu(fmt, T):
+    wl = _tiny(fmt, T)
     P = build(wl, "quantised")
     off, rs, sr = oracle.permute(P.ids, wl.E)
     R = wl.T * wl.k
@@ -181,10 +186,9 @@ def test_grouped_swiglu(fmt):
     assert moe.read_status(ws) == 0
 
 
-@pytest.mark.parametrize("fmt", ["int4", "nvfp4"])
-def test_grouped_down(fmt):
-    wl = syn.WORKLOADS[0] if fmt == "int4" else syn.Workload("tiny_nvfp4", 16, 1024, 32, 256, 8, "nvfp4", False,
-                                                                1 / 32.0, False)
+@pytest.mark.parametrize("fmt,T", [("int4", 16), ("nvfp4", 16), ("int4", 96), ("nvfp4", 96)])
+def test_grouped_down(fmt, T):
+    wl = _tiny(fmt, T)
     P = build(wl, "quantised")
     off, rs, sr = oracle.permute(P.ids, wl.E)
     R = wl.T * wl.k
@@ -200,9 +204,9 @@ def test_grouped_down(fmt):
     assert np.all(np.abs(gf - ref) <= layer_tolerance(ref))
 
 
-def test_shared_expert_bf16_steps():
+@pytest.mark.parametrize("T", [5, 300])
+def test_shared_expert_bf16_steps(T):
     wl = syn.WORKLOADS[1]
-    T = 5
     x = syn.gen_x(wl, T=T)
     sg, su, sd = (oracle.Bank(oracle.FMT_BF16, syn.gen_shared(wl, w)[None]) for w in ("gate", "up", "down"))
     off = np.array([0, T], np.int32)
