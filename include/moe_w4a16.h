@@ -144,6 +144,25 @@ int moe_permute(const int32_t* topk_ids, int T, int top_k, int E,
                 int32_t* expert_offsets, int32_t* row_slot, int32_t* slot_row,
                 void* ws, size_t ws_bytes, moe_stream_t stream);
 
+/* Bucketing for callers that cannot allocate device memory.  Some callers run
+ * inside another runtime's fixed memory plan (an engine that reserves the GPU's
+ * memory up front and hands out no extra buffers), or cannot afford the
+ * device-wide synchronisation that an allocation can cause in the middle of a
+ * step; they cannot supply the workspace moe_permute needs.  This call computes exactly what moe_permute
+ * computes (same arguments and outputs, minus the workspace) and allocates
+ * nothing: its scratch is a file-scope device array of about 64 KB that every
+ * GPU loading the library keeps until the process exits.
+ * Limits: T*top_k <= 65536 and E <= 1024; larger sizes return
+ * MOE_ERR_UNSUPPORTED.  The first call on a device looks up the array's device
+ * address (cudaGetSymbolAddress), so make one call on each device before any
+ * stream capture.  All calls share the array and each call overwrites it:
+ * calls that may overlap on the GPU (different streams with no ordering
+ * between them) race.  An expert id outside [0, E) is dropped and its slot_row
+ * entry is -1.  The paper has no counterpart to this call. */
+int moe_permute_noalloc(const int32_t* topk_ids, int T, int top_k, int E,
+                        int32_t* expert_offsets, int32_t* row_slot, int32_t* slot_row,
+                        moe_stream_t stream);
+
 /* Grouped gate/up projection with fused SwiGLU, weights dequantised in-kernel:
  * for each expert e and row r in [expert_offsets[e], expert_offsets[e+1]),
  * with token t = row_slot[r] / top_k:

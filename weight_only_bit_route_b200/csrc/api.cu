@@ -212,6 +212,19 @@ int moe_permute(const int32_t* topk_ids, int T, int top_k, int E, int32_t* exper
                           at<int32_t>(ws, kStepScratch), at<int32_t>(ws, 0), cs(stream));
 }
 
+int moe_permute_noalloc(const int32_t* topk_ids, int T, int top_k, int E, int32_t* expert_offsets,
+                        int32_t* row_slot, int32_t* slot_row, moe_stream_t stream) {
+    if (T < 0 || top_k <= 0 || E <= 0) return MOE_ERR_INVALID_ARG;
+    if (E > kMaxE || top_k > kMaxTopK) return MOE_ERR_UNSUPPORTED;
+    if (!expert_offsets) return MOE_ERR_INVALID_ARG;
+    if (T == 0) {
+        return cudaMemsetAsync(expert_offsets, 0, size_t(E + 1) * 4, cs(stream)) == cudaSuccess
+                   ? MOE_OK : MOE_ERR_CUDA;
+    }
+    if (!topk_ids || !row_slot || !slot_row) return MOE_ERR_INVALID_ARG;
+    return launch_permute_noalloc(topk_ids, T, top_k, E, expert_offsets, row_slot, slot_row, cs(stream));
+}
+
 int moe_grouped_w4a16_swiglu(const void* x, int T, int H, const int32_t* expert_offsets,
                              const int32_t* row_slot, int top_k, const moe_qweight* gate,
                              const moe_qweight* up, float swiglu_limit, void* h_perm, void* ws,

@@ -111,6 +111,8 @@ int launch_route_decode(const RouterDecodeArgs& a, cudaStream_t s);
 int launch_permute(const int32_t* ids, int T, int k, int E, int32_t* offsets,
                    int32_t* row_slot, int32_t* slot_row, int32_t* hist, int32_t* status,
                    cudaStream_t s);
+int launch_permute_noalloc(const int32_t* ids, int T, int k, int E, int32_t* offsets, int32_t* row_slot,
+                           int32_t* slot_row, cudaStream_t s);
 
 struct GemvProblem {
     const __nv_bfloat16* act;  // gate/up: x [T, in]; down: h_perm [rows, in]

@@ -11,6 +11,8 @@
 //               __match_any_sync groups equal ids inside a 32-slot step, so the
 //               rank of a slot among equal ids is its popcount of lower lanes.
 // No global atomics decide a position, so the permutation is deterministic.
+#include <mutex>
+
 #include "moe_internal.cuh"
 
 namespace moe {
@@ -139,6 +141,51 @@ int launch_permute(const int32_t* ids, int T, int k, int E, int32_t* offsets,
     const size_t smem = size_t(kPermWarps) * E * sizeof(int32_t);
     perm_scatter<<<nb, kPermThreads, smem, s>>>(ids, R, E, hist, row_slot, slot_row);
     return cudaGetLastError() == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
+}
+
+// ---------------------------------------------------------------------------
+// Bucketing without caller-provided workspace, for callers that cannot
+// allocate: code running inside a fixed memory plan that has no spare buffer to
+// give, or a step that must not stall on the device-wide synchronisation an
+// allocation can cause.  Its scratch (a status word and the per-block expert
+// histograms) is a file-scope device array, so the call allocates nothing;
+// every GPU that loads this library holds the array (about 64 KB) until the
+// process exits.  Calls that overlap on the GPU share the array and race.
+// ---------------------------------------------------------------------------
+constexpr int kNoAllocMaxSlots = 65536;                       // T * top_k
+constexpr int kNoAllocBlocks = kNoAllocMaxSlots / kPermChunk;
+constexpr int kNoAllocHeader = 64;                            // status word + padding (ints)
+static __device__ __align__(256) int32_t g_noalloc_scratch[kNoAllocHeader + kNoAllocBlocks * kMaxE];
+
+// Device address of the scratch array on the current device.  In host code
+// the array's name is only a host-side stand-in, so the address is resolved
+// with cudaGetSymbolAddress the first time a device is used and cached.
+static int noalloc_scratch(int32_t** out) {
+    constexpr int kMaxDevices = 64;
+    static int32_t* addr[kMaxDevices] = {};
+    static std::mutex mu;
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess) return MOE_ERR_CUDA;
+    if (dev < 0 || dev >= kMaxDevices) return MOE_ERR_UNSUPPORTED;
+    std::lock_guard<std::mutex> lock(mu);
+    if (!addr[dev]) {
+        void* p = nullptr;
+        if (cudaGetSymbolAddress(&p, g_noalloc_scratch) != cudaSuccess || !p) return MOE_ERR_CUDA;
+        addr[dev] = static_cast<int32_t*>(p);
+    }
+    *out = addr[dev];
+    return MOE_OK;
+}
+
+int launch_permute_noalloc(const int32_t* ids, int T, int k, int E, int32_t* offsets, int32_t* row_slot,
+                           int32_t* slot_row, cudaStream_t s) {
+    if (size_t(T) * k > size_t(kNoAllocMaxSlots) || E > kMaxE) return MOE_ERR_UNSUPPORTED;
+    int32_t* scratch = nullptr;
+    const int rc = noalloc_scratch(&scratch);
+    if (rc != MOE_OK) return rc;
+    // the status word must start at zero; the histograms are fully rewritten
+    if (cudaMemsetAsync(scratch, 0, sizeof(int32_t), s) != cudaSuccess) return MOE_ERR_CUDA;
+    return launch_permute(ids, T, k, E, offsets, row_slot, slot_row, scratch + kNoAllocHeader, scratch, s);
 }
 
 }  // namespace moe

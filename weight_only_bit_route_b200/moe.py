@@ -57,6 +57,7 @@ _sig("moe_read_status", _I, [_P, _P, ctypes.POINTER(ctypes.c_int32)])
 _sig("moe_status_string", ctypes.c_char_p, [_I])
 _sig("moe_route_topk", _I, [_P, _I, _I, _P, _P, _I, _I, _P, _P, _P, _SZ, _P])
 _sig("moe_permute", _I, [_P, _I, _I, _I, _P, _P, _P, _P, _SZ, _P])
+_sig("moe_permute_noalloc", _I, [_P, _I, _I, _I, _P, _P, _P, _P])
 _sig("moe_grouped_w4a16_swiglu", _I, [_P, _I, _I, _P, _P, _I, _P, _P, _F, _P, _P, _SZ, _P])
 _sig("moe_grouped_w4a16_down", _I, [_P, _P, _P, _P, _I, _P, _P, _P, _SZ, _P])
 _sig("moe_unpermute_combine", _I, [_P, _P, _I, _I, _I, _P, _P, _P])
@@ -171,6 +172,17 @@ def permute(ids, E, ws):
     sr = torch.empty(T * k, dtype=torch.int32, device=ids.device)
     _check("moe_permute", lib.moe_permute(_ptr(ids), T, k, E, _ptr(off), _ptr(rs), _ptr(sr),
                                           _ptr(ws), ws.numel(), _stream()))
+    return off, rs, sr
+
+
+def permute_noalloc(ids, E):
+    """moe_permute without a workspace (scratch in a static device array)."""
+    T, k = ids.shape
+    off = torch.empty(E + 1, dtype=torch.int32, device=ids.device)
+    rs = torch.empty(T * k, dtype=torch.int32, device=ids.device)
+    sr = torch.empty(T * k, dtype=torch.int32, device=ids.device)
+    _check("moe_permute_noalloc", lib.moe_permute_noalloc(_ptr(ids), T, k, E, _ptr(off), _ptr(rs), _ptr(sr),
+                                                          _stream()))
     return off, rs, sr
 
 
