@@ -170,9 +170,12 @@ int moe_permute_noalloc(const int32_t* topk_ids, int T, int top_k, int E,
  * (fp32 accumulation).  x: bf16 [T, H]; gate/up: banks [E, F, H] of the same
  * format; h_perm: bf16 [T*top_k, F] (out).  swiglu_limit must be 0.
  * For the shared expert pass BF16 banks with E = 1, expert_offsets = {0, T}
- * and row_slot[i] = i * top_k.  Decode-sized calls (T*top_k <= 256) stream
- * the weights with a GEMV; larger calls run a tcgen05 grouped GEMM.
- * ws: at least 256 + 16*(E+2) bytes. */
+ * and row_slot[i] = i * top_k.  Decode-sized calls (rows <= 256, rows =
+ * T*top_k, or T for E = 1) stream the weights with a GEMV; larger calls run a
+ * tcgen05 grouped GEMM, which needs H to be a multiple of 256.
+ * ws (256-byte aligned): at least 256 + a(16*(E+2)) + a(rows*H/8) + a(2*rows*H)
+ * bytes, a() rounding up to a multiple of 256; moe_workspace_bytes(T, H, E, F,
+ * top_k) is always enough. */
 int moe_grouped_w4a16_swiglu(const void* x, int T, int H,
                              const int32_t* expert_offsets, const int32_t* row_slot,
                              int top_k, const moe_qweight* gate, const moe_qweight* up,
@@ -183,8 +186,11 @@ int moe_grouped_w4a16_swiglu(const void* x, int T, int H,
  *     y_perm[r, :] = bf16( topk_w[row_slot[r]] * (h_perm[r] . Wd[e]^T) )
  * for rows r of expert e (fp32 accumulation).  h_perm: bf16 [rows, F];
  * topk_w: fp32 [rows] indexed by slot, or NULL for weight 1;
- * down: bank [E, H, F]; y_perm: bf16 [rows, H] (out).
- * ws: at least 256 + 16*(E+2) bytes. */
+ * down: bank [E, H, F]; y_perm: bf16 [rows, H] (out).  More than 256 rows
+ * run the tcgen05 GEMM, which needs F to be a multiple of 256.
+ * ws (256-byte aligned): at least 256 + a(16*(E+2)) + a(rows*F/8) + a(2*rows*F)
+ * bytes, a() rounding up to a multiple of 256; moe_workspace_bytes(T, H, E, F,
+ * top_k) with rows = T*top_k is always enough. */
 int moe_grouped_w4a16_down(const void* h_perm, const int32_t* expert_offsets,
                            const int32_t* row_slot, const float* topk_w, int rows,
                            const moe_qweight* down, void* y_perm,

@@ -292,6 +292,25 @@ def test_layer_forward_sampled(cfg):
     print(f"cfg {cfg}: near-tie {n_nt}, flipped {n_flip}, max rel err {rel:.2e}")
 
 
+@pytest.mark.parametrize("fmt", ["int4", "nvfp4"])
+def test_layer_forward_gemm_path_all_tokens(fmt):
+    """100 tokens give 800 routed rows, so both projections run on the tcgen05
+    GEMM (int4 h passes between them in the pair order); every token is
+    compared with the oracle, shared expert included."""
+    wl = _tiny(fmt, 100)
+    P = build(wl, "quantised", shared=True)
+    L = device_layer(moe, P)
+    ws = _ws(P.T, wl)
+    x = dev_bf16(P.x)
+    y = moe.layer_forward(x, L, ws)
+    ids, _ = moe.route_topk(x, L.router_w, L.router_bias, wl.k, ws)
+    torch.cuda.synchronize()
+    assert moe.read_status(ws) == 0
+    tokens = np.arange(P.T, dtype=np.int32)
+    n_nt, n_flip, rel = _layer_check(P, bf16_bits(y), tokens, ids.cpu().numpy())
+    print(f"{fmt}: near-tie {n_nt}, flipped {n_flip}, max rel err {rel:.2e}")
+
+
 def test_layer_zero_input_is_zero():
     P = build(0, "quantised", shared=True)
     L = device_layer(moe, P)

@@ -51,14 +51,20 @@ int check_ws(void* ws, size_t ws_bytes, size_t need) {
 // decode-sized calls stream weights with the GEMV; larger ones use the GEMM
 constexpr int kGemvMaxRows = 256;
 
-// rows_total: rows present over all experts of the routed problem; act_rows:
-// its activation rows (T for gate/up, rows for down).
-int run_grouped(const GemvProblem& p, const GemvProblem* shared, bool gateup, int rows_total, int act_rows,
-                void* prep_ws, int32_t* tile_ws, cudaStream_t s) {
-    if (rows_total <= kGemvMaxRows) return launch_stream_gemv(p, shared, gateup, act_rows, prep_ws, s, false);
-    return launch_grouped_gemm(p, shared, gateup, act_rows, prep_ws, tile_ws, s);
+// The tcgen05 GEMM of one problem of a step-level call: its activation
+// pre-pass goes to prep ([rows] fp32 scales, then [rows, in] 16-bit rows).
+GemmBuffers step_buffers(void* prep, int rows, bool act_ready) {
+    GemmBuffers b{};
+    b.scale_buf = reinterpret_cast<float*>(prep);
+    b.act_buf = reinterpret_cast<uint8_t*>(prep) + align256(size_t(rows) * 4);
+    b.act_ready = act_ready;
+    b.perm_out = 0;
+    return b;
 }
 
+// Step-level scratch after the 256-byte control block: room for the GEMV
+// pre-pass of act_rows rows or the GEMM pre-pass of rows rows.
+size_t step_scratch(int E, int rows, int in_dim) { return grouped_scratch(E, rows, in_dim); }
 int layer_checks(const void* x, int T, const moe_layer* L, void* y, void* ws, size_t ws_bytes) {
     if (!L) return MOE_ERR_INVALID_ARG;
     MOE_TRY(check_dims(T, L->H, L->E, L->F, L->top_k));
@@ -95,7 +101,6 @@ int layer_run(const void* x, int T, const moe_layer* L, void* y, void* ws, cudaS
     __nv_bfloat16* h_perm = at<__nv_bfloat16>(ws, W.h_perm);
     __nv_bfloat16* y_perm = at<__nv_bfloat16>(ws, W.y_perm);
     __nv_bfloat16* ys = at<__nv_bfloat16>(ws, W.ys);
-    int32_t* tiles = at<int32_t>(ws, W.tiles);
     const __nv_bfloat16* xb = reinterpret_cast<const __nv_bfloat16*>(x);
 
     const bool has_sh = L->sh_gate.packed != nullptr;
@@ -119,6 +124,8 @@ int layer_run(const void* x, int T, const moe_layer* L, void* y, void* ws, cudaS
 
     void* prep = at<void>(ws, W.prep);
     __nv_bfloat16* h_sh = h_perm + size_t(R) * F;
+    const bool gemv = R <= kGemvMaxRows;
+    const bool int4 = L->gate.fmt == MOE_FMT_INT4_G128;
 
     GemvProblem gu{};
     gu.act = xb; gu.act_by_token = 1; gu.top_k = k; gu.offsets = offsets; gu.row_slot = row_slot;
@@ -130,7 +137,6 @@ int layer_run(const void* x, int T, const moe_layer* L, void* y, void* ws, cudaS
     sg.act = xb; sg.act_by_token = 1; sg.top_k = k; sg.offsets = sh_off; sg.row_slot = sh_rs;
     sg.E = 1; sg.fmt = MOE_FMT_BF16; sg.out_dim = F; sg.in_dim = H;
     sg.p0 = L->sh_gate.packed; sg.p1 = L->sh_up.packed; sg.out = h_sh; sg.status = status;
-    MOE_TRY(run_grouped(gu, has_sh ? &sg : nullptr, true, R, T, prep, tiles, s));
 
     GemvProblem dn{};
     dn.act = h_perm; dn.act_by_token = 0; dn.top_k = k; dn.offsets = offsets; dn.row_slot = row_slot;
@@ -141,7 +147,28 @@ int layer_run(const void* x, int T, const moe_layer* L, void* y, void* ws, cudaS
     sd.act = h_sh; sd.act_by_token = 0; sd.top_k = k; sd.offsets = sh_off; sd.row_slot = sh_rs;
     sd.E = 1; sd.fmt = MOE_FMT_BF16; sd.out_dim = H; sd.in_dim = F;
     sd.p0 = L->sh_down.packed; sd.out = ys; sd.status = status;
-    MOE_TRY(run_grouped(dn, has_sh ? &sd : nullptr, false, R, R, prep, tiles, s));
+
+    if (gemv) {
+        MOE_TRY(launch_stream_gemv(gu, has_sh ? &sg : nullptr, true, T, prep, s, false));
+        MOE_TRY(launch_stream_gemv(dn, has_sh ? &sd : nullptr, false, R, prep, s, false));
+    } else {
+        // gate/up: the routed activation rows are gathered into the y_perm
+        // region (free until the down projection writes it); int4 writes h in
+        // the pair order the down GEMM reads.  The shared expert reads x and
+        // its own h directly (identity routing, natural order).
+        GemmBuffers gb{};
+        gb.act_buf = y_perm; gb.scale_buf = reinterpret_cast<float*>(prep); gb.act_ready = 0; gb.perm_out = int4;
+        MOE_TRY(launch_grouped_gemm(gu, true, R, gb, s));
+        GemmBuffers direct{};
+        direct.act_ready = 1;
+        if (has_sh) MOE_TRY(launch_grouped_gemm(sg, true, T, direct, s));
+        GemmBuffers db{};
+        db.scale_buf = reinterpret_cast<float*>(prep);
+        db.act_buf = reinterpret_cast<uint8_t*>(prep) + align256(size_t(R) * 4);
+        db.act_ready = int4;
+        MOE_TRY(launch_grouped_gemm(dn, false, R, db, s));
+        if (has_sh) MOE_TRY(launch_grouped_gemm(sd, false, T, direct, s));
+    }
 
     return launch_combine(y_perm, slot_row, T, k, H, has_sh ? ys : nullptr,
                           reinterpret_cast<__nv_bfloat16*>(y), s);
@@ -239,9 +266,9 @@ int moe_grouped_w4a16_swiglu(const void* x, int T, int H, const int32_t* expert_
     if (gate->fmt != up->fmt || F % 128) return MOE_ERR_UNSUPPORTED;
     if (T == 0) return MOE_OK;
     if (!x || !al16(x) || !expert_offsets || !row_slot || !h_perm || !al16(h_perm)) return MOE_ERR_INVALID_ARG;
-    MOE_TRY(check_ws(ws, ws_bytes, kStepScratch + grouped_scratch(E, T, H)));
     // rows present: T * top_k routed slots, or T for a single shared expert
     const int rows = (E == 1) ? T : T * top_k;
+    MOE_TRY(check_ws(ws, ws_bytes, kStepScratch + step_scratch(E, rows, H)));
     GemvProblem p{};
     p.act = reinterpret_cast<const __nv_bfloat16*>(x); p.act_by_token = 1; p.top_k = top_k;
     p.offsets = expert_offsets; p.row_slot = row_slot; p.E = E; p.fmt = gate->fmt;
@@ -249,8 +276,9 @@ int moe_grouped_w4a16_swiglu(const void* x, int T, int H, const int32_t* expert_
     p.p0 = gate->packed; p.s0 = gate->scales; p.g0 = gate->global_scale;
     p.p1 = up->packed; p.s1 = up->scales; p.g1 = up->global_scale;
     p.out = reinterpret_cast<__nv_bfloat16*>(h_perm); p.status = at<int32_t>(ws, 0);
-    return run_grouped(p, nullptr, true, rows, T, at<void>(ws, kStepScratch + align256(size_t(E + 2) * 16)),
-                       at<int32_t>(ws, kStepScratch), cs(stream));
+    void* prep = at<void>(ws, kStepScratch + align256(size_t(E + 2) * 16));
+    if (rows <= kGemvMaxRows) return launch_stream_gemv(p, nullptr, true, T, prep, cs(stream), false);
+    return launch_grouped_gemm(p, true, rows, step_buffers(prep, rows, false), cs(stream));
 }
 
 int moe_grouped_w4a16_down(const void* h_perm, const int32_t* expert_offsets, const int32_t* row_slot,
@@ -264,15 +292,17 @@ int moe_grouped_w4a16_down(const void* h_perm, const int32_t* expert_offsets, co
     if (rows == 0) return MOE_OK;
     if (!h_perm || !al16(h_perm) || !expert_offsets || !row_slot || !y_perm || !al16(y_perm))
         return MOE_ERR_INVALID_ARG;
-    MOE_TRY(check_ws(ws, ws_bytes, kStepScratch + grouped_scratch(E, rows, F)));
+    MOE_TRY(check_ws(ws, ws_bytes, kStepScratch + step_scratch(E, rows, F)));
     GemvProblem p{};
     p.act = reinterpret_cast<const __nv_bfloat16*>(h_perm); p.act_by_token = 0; p.top_k = 1;
     p.offsets = expert_offsets; p.row_slot = row_slot; p.E = E; p.topk_w = topk_w;
     p.fmt = down->fmt; p.out_dim = H; p.in_dim = F;
     p.p0 = down->packed; p.s0 = down->scales; p.g0 = down->global_scale;
     p.out = reinterpret_cast<__nv_bfloat16*>(y_perm); p.status = at<int32_t>(ws, 0);
-    return run_grouped(p, nullptr, false, rows, rows, at<void>(ws, kStepScratch + align256(size_t(E + 2) * 16)),
-                       at<int32_t>(ws, kStepScratch), cs(stream));
+    void* prep = at<void>(ws, kStepScratch + align256(size_t(E + 2) * 16));
+    if (rows <= kGemvMaxRows) return launch_stream_gemv(p, nullptr, false, rows, prep, cs(stream), false);
+    // BF16 rows are read in place (row r is activation row r)
+    return launch_grouped_gemm(p, false, rows, step_buffers(prep, rows, down->fmt == MOE_FMT_BF16), cs(stream));
 }
 
 int moe_unpermute_combine(const void* y_perm, const int32_t* slot_row, int T, int top_k, int H,

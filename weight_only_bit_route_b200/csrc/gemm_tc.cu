@@ -7,222 +7,310 @@
 // with the 4-bit weights dequantised inside the kernel
 // ("Step-5-Preview-Int4-g128", Recipe; "Step-5-Preview-NVFP4-Local", Format).
 //
-// Tiles are swapped (weights are the M = 128 operand, tokens the N operand),
-// because an expert sees few tokens (about 47 at 2048 tokens): a tile is
-// (expert, n-tile of up to 256 rows, m-tile of 128 weight rows).  A persistent
-// CTA per SM walks the tile list (built on the device from expert_offsets).
-// For each 64-wide K block all eight warps
-//   - dequantise the 128 x 64 weight tile(s) into bf16 (int4: q*s rounded
-//     once; NVFP4: e2m1 * e4m3 exactly, in f16 with f16 activations) laid out
-//     K-major with the 128-byte swizzle the MMA descriptors expect, and
-//   - gather the tile's activation rows into the same layout,
-// then one thread issues tcgen05.mma (M = 128, N = tile rows, K = 16, fp32
-// accumulation in tensor memory; gate and up are two accumulators sharing the
-// activation operand) and tcgen05.commit arrives on the stage's mbarrier.  A
-// ring of three stages lets the next blocks be produced while the MMAs run.
-// The epilogue reads the accumulators with tcgen05.ld and fuses SwiGLU (gate/up)
-// or the routing weight (down); NVFP4 global and activation row scales are
-// applied there too.  Waits are bounded (about 2 s) and report MOE_ERR_TIMEOUT.
+// Tiles are swapped: weights are the M = 128 operand and tokens the N operand,
+// because an expert sees few tokens (about 47 at 2048 tokens).  A tile is
+// (expert, m-tile of 128 weight rows, n-tile of up to 128 (gate/up) or 256
+// (down) rows).  The n-tiles of one m-tile are adjacent in the tile order, so
+// CTAs running side by side share the weight tile through L2.  A persistent
+// CTA per SM walks the tile list, which it builds on the device from
+// expert_offsets.
+//
+// Warp roles inside a CTA (16 warps):
+//   warp 0      TMA producer of the weight stream: per stage, one 2D tensor
+//               copy of 128 rows x 128 bytes of packed weights (K = 256 for
+//               4-bit formats, K = 64 for BF16) per matrix, 128-byte
+//               swizzled, plus the NVFP4 block scales of those rows.  int4
+//               scales are one bulk copy per tile, since all groups of the
+//               tile's rows are contiguous.
+//   warp 1      TMA producer of the activation operand: 16-row boxes of the
+//               tile's rows (K = 64 per stage), 128-byte swizzled.  That is
+//               the K-major layout the MMA descriptors read.
+//   warp 2      allocates tensor memory and issues tcgen05.mma from one thread.
+//   warps 4-7   epilogue: tcgen05.ld of the accumulators, SwiGLU or the
+//               routing weight, bf16 stores.  Warp w reads TMEM lanes
+//               32*(w%4) to 32*(w%4)+31.
+//   warps 8-15  dequantisation (4-bit formats).  Each thread owns one weight
+//               row of the tile.  It turns packed weights into bf16 pairs
+//               (int4: q*s rounded once) or f16 pairs (NVFP4: e2m1 * e4m3,
+//               exact) in registers and writes them to tensor memory with
+//               tcgen05.st; the MMA reads its A operand from there.  The
+//               dequantised weights never pass through shared memory.
+// BF16 weights (the shared expert) need no dequantisation: the MMA reads the
+// TMA-staged weight tile from shared memory directly.
+//
+// Tensor memory (512 columns): accumulators in [0, 256) (for gate/up, gate at
+// 0 and up at 128), A stages in [256, 512).
+//
+// int4 pairs: one mask turns the nibbles (j, j+4) of a packed word into one
+// bf16 pair, so the A operand holds the K elements of each group of 8 in the
+// order 0,4,1,5,2,6,3,7.  The activation operand is stored in the same order,
+// by a pre-pass or by the gate/up epilogue writing h that way.  A dot product
+// does not depend on the order of its terms.
+//
+// Every wait is bounded (about 2 s).  On expiry the kernel records
+// MOE_ERR_TIMEOUT and stops issuing work.  It then waits, again bounded, for
+// the copies and MMAs it has in flight, frees its tensor memory and returns.
+#include <cuda.h>
+#include <cudaTypedefs.h>
 #include <cuda_fp16.h>
 
-#include <algorithm>
+#include <cstring>
+#include <mutex>
 #include <type_traits>
 
 #include "moe_internal.cuh"
 
 namespace moe {
 
-constexpr int TC_BM = 128;
-constexpr int TC_BK = 64;
-constexpr int TC_BN_MAX = 256;
-constexpr int TC_STAGES = 3;
-constexpr int TC_THREADS = 256;
-constexpr int TC_A_BYTES = TC_BM * TC_BK * 2;          // 16 KB per weight matrix
-constexpr int TC_B_BYTES = TC_BN_MAX * TC_BK * 2;      // 32 KB
-constexpr int TC_STAGE_BYTES = 2 * TC_A_BYTES + TC_B_BYTES;
-constexpr unsigned long long TC_WAIT_NS = 2000000000ull;
+constexpr int G_BM = 128;
+constexpr int G_BK = 64;
+constexpr int G_THREADS = 512;
+constexpr int G_DQ_WARPS = 8;
+constexpr int G_EPI_WARPS = 4;
+constexpr unsigned long long G_WAIT_NS = 2000000000ull;
 
-struct TcArgs {
-    int fmt, gateup, E, out_dim, in_dim, top_k, act_by_token;
-    const uint8_t* p0; const uint8_t* s0; const float* g0;
-    const uint8_t* p1; const uint8_t* s1; const float* g1;
+template <int FMT, bool GU>
+struct GCfg {
+    static constexpr bool kTmemA = FMT != MOE_FMT_BF16;
+    static constexpr int kNMat = GU ? 2 : 1;
+    static constexpr int kNMax = GU ? 64 : 128;                    // token rows per tile
+    static constexpr int kUpCol = 64;                               // up accumulator within a buffer
+    static constexpr int kPkK = kTmemA ? 256 : 64;                  // K per weight stage
+    static constexpr int kPkX = kTmemA ? 128 : 64;                  // its width in tensor-map elements
+    static constexpr int kMatBytes = G_BM * 128;                    // one matrix per stage: 16 KB
+    static constexpr int kNvScBytes = FMT == MOE_FMT_NVFP4 ? G_BM * 16 : 0;
+    static constexpr int kPkStageBytes = kNMat * (kMatBytes + kNvScBytes);
+    static constexpr int kPkStages = (GU && FMT == MOE_FMT_INT4_G128) ? 3 : 4;
+    static constexpr int kBStages = GU ? 8 : 6;
+    static constexpr int kBStageBytes = kNMax * 128;
+    static constexpr int kAStageCols = kNMat * 32;                  // K = 64 as 16-bit pairs, per matrix
+    static constexpr int kAStages = 256 / kAStageCols;
+    // gate/up: every dequantisation warp writes its matrix of every A stage;
+    // down: the four warps of one parity write the stages of their K blocks
+    static constexpr int kAFullCount = GU ? G_DQ_WARPS : G_DQ_WARPS / 2;
+    static constexpr bool kMmaF16 = FMT == MOE_FMT_NVFP4;
+};
+
+struct GArgs {
+    CUtensorMap tm_p0, tm_p1;        // packed (or BF16) weights of gate (or down) and up
+    CUtensorMap tm_s0, tm_s1;        // NVFP4 block scales
+    CUtensorMap tm_b;                // activation operand rows
+    const uint8_t* sc0;              // int4 scales (bf16), bulk-copied per tile
+    const uint8_t* sc1;
+    const float* g0;                 // NVFP4 per-expert global scales
+    const float* g1;
     const int32_t* offsets;
     const int32_t* row_slot;
-    const float* topk_w;        // down: routing weight by slot (nullable)
-    const uint8_t* act;         // bf16 rows (int4, bf16) or f16 rows (NVFP4, pre-scaled)
-    const float* act_scale;     // NVFP4: activation row scale [act rows]
+    const float* topk_w;             // down: routing weight by slot (nullable)
+    const float* act_scale;          // NVFP4: activation row scale, by GEMM row
     __nv_bfloat16* out;
     int32_t* status;
+    int E, out_dim, in_dim, perm_out;
 };
 
 // ---------------------------------------------------------------------------
 // PTX helpers
 // ---------------------------------------------------------------------------
-__device__ __forceinline__ uint32_t tc_smem(const void* p) { return static_cast<uint32_t>(__cvta_generic_to_shared(p)); }
-__device__ __forceinline__ unsigned long long tc_timer() {
+__device__ __forceinline__ uint32_t g_smem(const void* p) { return static_cast<uint32_t>(__cvta_generic_to_shared(p)); }
+__device__ __forceinline__ unsigned long long g_timer() {
     unsigned long long t;
     asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
     return t;
 }
-__device__ __forceinline__ bool tc_wait(uint32_t bar, uint32_t parity) {
-    uint32_t ok = 0;
-    const unsigned long long t0 = tc_timer();
+__device__ __forceinline__ bool g_try(uint32_t bar, uint32_t parity) {
+    uint32_t ok;
+    asm volatile("{ .reg .pred p; mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2; selp.u32 %0, 1, 0, p; }"
+                 : "=r"(ok) : "r"(bar), "r"(parity) : "memory");
+    return ok != 0;
+}
+// Bounded wait: false after about 2 s, or as soon as another role has aborted.
+// Roles off the critical path back off with a short sleep between polls so
+// that they leave issue slots to the dequantisation warps.
+__device__ __forceinline__ bool g_wait(uint32_t bar, uint32_t parity, volatile int* abort_flag, int sleep_ns = 0) {
+    if (g_try(bar, parity)) return true;
+    const unsigned long long t0 = g_timer();
     while (true) {
-        asm volatile("{ .reg .pred p; mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2; selp.u32 %0, 1, 0, p; }"
-                     : "=r"(ok) : "r"(bar), "r"(parity) : "memory");
-        if (ok) return true;
-        if (tc_timer() - t0 > TC_WAIT_NS) return false;
+        if (sleep_ns) __nanosleep(sleep_ns);
+        if (g_try(bar, parity)) return true;
+        if (*abort_flag || g_timer() - t0 > G_WAIT_NS) return false;
     }
 }
+// Bounded wait that ignores the abort flag (draining work already in flight).
+__device__ __forceinline__ void g_drain_wait(uint32_t bar, uint32_t parity) {
+    const unsigned long long t0 = g_timer();
+    while (!g_try(bar, parity) && g_timer() - t0 < G_WAIT_NS) {
+    }
+}
+__device__ __forceinline__ void g_arrive(uint32_t bar) {
+    asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(bar) : "memory");
+}
+__device__ __forceinline__ void g_expect(uint32_t bar, uint32_t bytes) {
+    asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(bar), "r"(bytes) : "memory");
+}
+__device__ __forceinline__ void g_tma2d(uint32_t dst, const CUtensorMap* map, int x, int y, uint32_t bar) {
+    asm volatile(
+        "cp.async.bulk.tensor.2d.shared::cluster.global.tile.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3}], [%4];"
+        ::"r"(dst), "l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(y), "r"(bar) : "memory");
+}
+__device__ __forceinline__ void g_bulk(uint32_t dst, const void* src, uint32_t bytes, uint32_t bar) {
+    asm volatile("cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];"
+                 ::"r"(dst), "l"(src), "r"(bytes), "r"(bar) : "memory");
+}
 // K-major operand, 128-byte swizzle, 8-row groups 1024 bytes apart
-__device__ __forceinline__ uint64_t tc_desc(uint32_t saddr) {
+__device__ __forceinline__ uint64_t g_desc(uint32_t saddr) {
     return uint64_t((saddr >> 4) & 0x3FFF) | (uint64_t(1) << 16) | (uint64_t(64) << 32) | (uint64_t(1) << 46) |
            (uint64_t(2) << 61);
 }
-// kind::f16 instruction descriptor: fp32 accumulate, A/B bf16 (or f16), K-major, M = 128
-__device__ __forceinline__ uint32_t tc_idesc(int n, bool f16) {
+// kind::f16 instruction descriptor: fp32 accumulate, A/B bf16 (or f16), both K-major, M = 128
+__device__ __forceinline__ uint32_t g_idesc(int n, bool f16) {
     const uint32_t ab = f16 ? 0u : 1u;
-    return (1u << 4) | (ab << 7) | (ab << 10) | (uint32_t(n >> 3) << 17) | (uint32_t(TC_BM >> 4) << 24);
+    return (1u << 4) | (ab << 7) | (ab << 10) | (uint32_t(n >> 3) << 17) | (uint32_t(G_BM >> 4) << 24);
 }
-__device__ __forceinline__ void tc_mma(uint32_t tmem_d, uint64_t a, uint64_t b, uint32_t idesc, uint32_t acc) {
+__device__ __forceinline__ void g_mma_ss(uint32_t d, uint64_t a, uint64_t b, uint32_t idesc, uint32_t acc) {
     asm volatile("{ .reg .pred p; setp.ne.b32 p, %4, 0; tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p; }"
-                 ::"r"(tmem_d), "l"(a), "l"(b), "r"(idesc), "r"(acc) : "memory");
+                 ::"r"(d), "l"(a), "l"(b), "r"(idesc), "r"(acc) : "memory");
 }
-__device__ __forceinline__ void tc_commit(uint32_t bar) {
+__device__ __forceinline__ void g_mma_ts(uint32_t d, uint32_t a_tmem, uint64_t b, uint32_t idesc, uint32_t acc) {
+    asm volatile("{ .reg .pred p; setp.ne.b32 p, %4, 0; tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p; }"
+                 ::"r"(d), "r"(a_tmem), "l"(b), "r"(idesc), "r"(acc) : "memory");
+}
+__device__ __forceinline__ void g_commit(uint32_t bar) {
     asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(bar) : "memory");
 }
-__device__ __forceinline__ void tc_fence_before() { asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory"); }
-__device__ __forceinline__ void tc_fence_after() { asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory"); }
-__device__ __forceinline__ void tc_ld16(uint32_t taddr, uint32_t (&r)[16]) {
+__device__ __forceinline__ void g_fence_before() { asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory"); }
+__device__ __forceinline__ void g_fence_after() { asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory"); }
+__device__ __forceinline__ void g_ld16(uint32_t taddr, uint32_t (&r)[16]) {
     asm volatile("tcgen05.ld.sync.aligned.32x32b.x16.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15}, [%16];"
                  : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]),
                    "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15])
                  : "r"(taddr));
 }
-__device__ __forceinline__ void tc_ld_wait() { asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory"); }
-__device__ __forceinline__ uint32_t tc_e2m1x2_f16x2(uint32_t byte) {
+__device__ __forceinline__ void g_ld_wait() { asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory"); }
+__device__ __forceinline__ void g_st16(uint32_t taddr, const uint32_t (&v)[16]) {
+    asm volatile("tcgen05.st.sync.aligned.32x32b.x16.b32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16};"
+                 ::"r"(taddr), "r"(v[0]), "r"(v[1]), "r"(v[2]), "r"(v[3]), "r"(v[4]), "r"(v[5]), "r"(v[6]), "r"(v[7]),
+                   "r"(v[8]), "r"(v[9]), "r"(v[10]), "r"(v[11]), "r"(v[12]), "r"(v[13]), "r"(v[14]), "r"(v[15])
+                 : "memory");
+}
+__device__ __forceinline__ void g_st_wait() { asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory"); }
+__device__ __forceinline__ uint32_t g_e2m1x2_f16x2(uint32_t byte) {
     uint32_t h;
     asm("{ .reg .b8 t; cvt.u8.u32 t, %1; cvt.rn.f16x2.e2m1x2 %0, t; }" : "=r"(h) : "r"(byte));
     return h;
 }
-__device__ __forceinline__ uint32_t tc_e4m3_f16x2(uint32_t byte) {          // {s, s} in f16
+__device__ __forceinline__ uint32_t g_e4m3_f16x2(uint32_t byte) {          // {s, s} in f16
     uint32_t h;
     asm("{ .reg .b16 t; cvt.u16.u32 t, %1; cvt.rn.f16x2.e4m3x2 %0, t; }" : "=r"(h) : "r"(byte | (byte << 8)));
     return h;
 }
+// byte offset of 16-byte chunk c of row r in a 128-byte-swizzled tile (1024-byte aligned)
+__device__ __forceinline__ uint32_t g_swz(int r, int c) { return uint32_t(r * 128 + ((c ^ (r & 7)) << 4)); }
 
-// byte offset of 16-byte chunk c of row r inside a K-major, 128B-swizzled tile
-__device__ __forceinline__ uint32_t tc_swz(int r, int c) {
-    return uint32_t((r >> 3) * 1024 + (r & 7) * 128 + ((c ^ (r & 7)) << 4));
+// ---------------------------------------------------------------------------
+// Dequantisation of one 16-byte chunk of packed weights (32 weights) into 16
+// bf16/f16 pairs.  int4: pair order within each 8, sc = bf16 scale bits.
+// NVFP4: natural order, sc = two E4M3 bytes (K 0-15, K 16-31 of the chunk).
+// ---------------------------------------------------------------------------
+__device__ __forceinline__ void g_dq_int4(const uint4 w, uint32_t sc, uint32_t (&o)[16]) {
+    const __nv_bfloat162 s2 = __bfloat162bfloat162(__ushort_as_bfloat16(static_cast<unsigned short>(sc)));
+    const __nv_bfloat162 off = __floats2bfloat162_rn(136.f, 136.f);
+    const uint32_t ws[4] = {w.x, w.y, w.z, w.w};
+#pragma unroll
+    for (int j = 0; j < 4; j++) {
+#pragma unroll
+        for (int p = 0; p < 4; p++) {
+            // nibbles (p, p+4) -> bf16 {128+u}; minus 136 gives q exactly; times s rounds once
+            uint32_t v = ((ws[j] >> (4 * p)) & 0x000F000Fu) | 0x43004300u;
+            __nv_bfloat162 h = *reinterpret_cast<__nv_bfloat162*>(&v);
+            h = __hmul2(__hsub2(h, off), s2);
+            o[j * 4 + p] = *reinterpret_cast<uint32_t*>(&h);
+        }
+    }
 }
-
-// ---------------------------------------------------------------------------
-// Weight unit: 32 consecutive K elements of one row of one matrix -> 4 chunks
-// ---------------------------------------------------------------------------
-struct TcWUnit { uint4 w[4]; uint32_t sc; };     // packed weights (int4/NVFP4 use w[0]) and scale bits
-
-template <int FMT>
-__device__ __forceinline__ void tc_load_wunit(const TcArgs& a, int mi, size_t wrow, int k, TcWUnit& u) {
-    const uint8_t* p = mi ? a.p1 : a.p0;
-    const uint8_t* sp = mi ? a.s1 : a.s0;
-    if (FMT == MOE_FMT_INT4_G128) {
-        u.w[0] = __ldg(reinterpret_cast<const uint4*>(p + wrow * (a.in_dim / 2) + k / 2));
-        u.sc = __ldg(reinterpret_cast<const uint16_t*>(sp) + wrow * (a.in_dim / 128) + k / 128);
-    } else if (FMT == MOE_FMT_NVFP4) {
-        u.w[0] = __ldg(reinterpret_cast<const uint4*>(p + wrow * (a.in_dim / 2) + k / 2));
-        u.sc = __ldg(reinterpret_cast<const uint16_t*>(sp + wrow * (a.in_dim / 16) + k / 16));   // two E4M3 bytes
-    } else {
-        const uint4* q = reinterpret_cast<const uint4*>(p + (wrow * a.in_dim + k) * 2);
-        u.w[0] = __ldg(q); u.w[1] = __ldg(q + 1); u.w[2] = __ldg(q + 2); u.w[3] = __ldg(q + 3);
+__device__ __forceinline__ void g_dq_nvfp4(const uint4 w, uint32_t sc2, uint32_t (&o)[16]) {
+    const uint32_t ws[4] = {w.x, w.y, w.z, w.w};
+#pragma unroll
+    for (int j = 0; j < 4; j++) {
+        uint32_t sv = g_e4m3_f16x2((sc2 >> (8 * (j >> 1))) & 0xffu);
+        const __half2 s2 = *reinterpret_cast<__half2*>(&sv);
+#pragma unroll
+        for (int b = 0; b < 4; b++) {
+            uint32_t hv = g_e2m1x2_f16x2((ws[j] >> (8 * b)) & 0xffu);
+            __half2 h = __hmul2(*reinterpret_cast<__half2*>(&hv), s2);       // exact
+            o[j * 4 + b] = *reinterpret_cast<uint32_t*>(&h);
+        }
     }
 }
 
-// Dequantise a unit and store its 4 chunks (row r, chunks c0..c0+3) into a swizzled tile.
-template <int FMT>
-__device__ __forceinline__ void tc_store_wunit(uint8_t* tile, int r, int c0, const TcWUnit& u) {
-    if (FMT == MOE_FMT_INT4_G128) {
-        const __nv_bfloat162 s2 = __bfloat162bfloat162(__ushort_as_bfloat16(static_cast<unsigned short>(u.sc)));
-        const __nv_bfloat162 off = __floats2bfloat162_rn(136.f, 136.f);
-        const uint32_t ws[4] = {u.w[0].x, u.w[0].y, u.w[0].z, u.w[0].w};
-#pragma unroll
-        for (int j = 0; j < 4; j++) {
-            const uint32_t w = ws[j];
-            uint32_t pr[4];
-#pragma unroll
-            for (int p = 0; p < 4; p++) {
-                // nibbles (p, p+4) -> bf16 {128+u}; minus 136 -> q exactly; times s (one rounding)
-                uint32_t v = ((w >> (4 * p)) & 0x000F000Fu) | 0x43004300u;
-                __nv_bfloat162 h = *reinterpret_cast<__nv_bfloat162*>(&v);
-                h = __hmul2(__hsub2(h, off), s2);
-                pr[p] = *reinterpret_cast<uint32_t*>(&h);
-            }
-            uint4 o;   // natural order: (x0,x1) (x2,x3) (x4,x5) (x6,x7)
-            o.x = __byte_perm(pr[0], pr[1], 0x5410);
-            o.y = __byte_perm(pr[2], pr[3], 0x5410);
-            o.z = __byte_perm(pr[0], pr[1], 0x7632);
-            o.w = __byte_perm(pr[2], pr[3], 0x7632);
-            *reinterpret_cast<uint4*>(tile + tc_swz(r, c0 + j)) = o;
-        }
-    } else if (FMT == MOE_FMT_NVFP4) {
-        const uint32_t ws[4] = {u.w[0].x, u.w[0].y, u.w[0].z, u.w[0].w};
-#pragma unroll
-        for (int j = 0; j < 4; j++) {
-            uint32_t sv = tc_e4m3_f16x2((u.sc >> (8 * (j >> 1))) & 0xffu);
-            const __half2 s2 = *reinterpret_cast<__half2*>(&sv);
-            const uint32_t w = ws[j];
-            uint32_t o[4];
-#pragma unroll
-            for (int b = 0; b < 4; b++) {
-                uint32_t hv = tc_e2m1x2_f16x2((w >> (8 * b)) & 0xffu);
-                __half2 h = __hmul2(*reinterpret_cast<__half2*>(&hv), s2);       // exact
-                o[b] = *reinterpret_cast<uint32_t*>(&h);
-            }
-            *reinterpret_cast<uint4*>(tile + tc_swz(r, c0 + j)) = make_uint4(o[0], o[1], o[2], o[3]);
-        }
-    } else {
-#pragma unroll
-        for (int j = 0; j < 4; j++) *reinterpret_cast<uint4*>(tile + tc_swz(r, c0 + j)) = u.w[j];
-    }
-}
+struct GTile { int e, m0, n0, nval, bn, ebase; };
 
 // ---------------------------------------------------------------------------
 // Kernel
 // ---------------------------------------------------------------------------
-template <int FMT>
-__global__ void __launch_bounds__(TC_THREADS, 1) tc_grouped_gemm(TcArgs a) {
+template <int FMT, bool GU>
+__global__ void __launch_bounds__(G_THREADS, 1) tc_grouped_gemm(const __grid_constant__ GArgs a) {
+    using C = GCfg<FMT, GU>;
     extern __shared__ __align__(1024) uint8_t smem[];
-    __shared__ __align__(8) uint64_t bars[TC_STAGES];
+    __shared__ __align__(8) uint64_t pk_full[C::kPkStages], pk_empty[C::kPkStages];
+    __shared__ __align__(8) uint64_t b_full[C::kBStages], b_empty[C::kBStages];
+    __shared__ __align__(8) uint64_t a_full[C::kAStages], a_empty[C::kAStages];
+    __shared__ __align__(8) uint64_t sc_full[2], sc_empty[2];
+    __shared__ __align__(8) uint64_t acc_full[2], acc_empty[2], drain;
     __shared__ uint32_t s_tmem;
     __shared__ int s_active[kMaxE];
     __shared__ int s_prefix[kMaxE];
-    __shared__ int s_wsum[TC_THREADS / 32];
-    __shared__ int s_nact, s_total, s_abort;
+    __shared__ int s_wsum[G_THREADS / 32], s_wt[G_THREADS / 32];
+    __shared__ int s_nact, s_total;
+    __shared__ volatile int s_abort;
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-    const int MT = a.out_dim / TC_BM;
-    const int KB = a.in_dim / TC_BK;
+    const int MT = a.out_dim / G_BM;
+    const int in_dim = a.in_dim;
+    const int KB = in_dim / G_BK;
+    const int NPS = in_dim / C::kPkK;
+    const int ngroups = in_dim / 128;
+    const uint32_t sc_mat_bytes = uint32_t(G_BM * ngroups * 2);
 
     if (tid == 0) {
-        for (int s = 0; s < TC_STAGES; s++) asm volatile("mbarrier.init.shared::cta.b64 [%0], 1;" ::"r"(tc_smem(&bars[s])));
+        for (int s = 0; s < C::kPkStages; s++) {
+            asm volatile("mbarrier.init.shared::cta.b64 [%0], 1;" ::"r"(g_smem(&pk_full[s])));
+            asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(g_smem(&pk_empty[s])),
+                         "r"(C::kTmemA ? G_DQ_WARPS : 1));
+        }
+        for (int s = 0; s < C::kBStages; s++) {
+            asm volatile("mbarrier.init.shared::cta.b64 [%0], 1;" ::"r"(g_smem(&b_full[s])));
+            asm volatile("mbarrier.init.shared::cta.b64 [%0], 1;" ::"r"(g_smem(&b_empty[s])));
+        }
+        for (int s = 0; s < C::kAStages; s++) {
+            asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(g_smem(&a_full[s])), "r"(C::kAFullCount));
+            asm volatile("mbarrier.init.shared::cta.b64 [%0], 1;" ::"r"(g_smem(&a_empty[s])));
+        }
+        for (int s = 0; s < 2; s++) {
+            asm volatile("mbarrier.init.shared::cta.b64 [%0], 1;" ::"r"(g_smem(&sc_full[s])));
+            asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(g_smem(&sc_empty[s])), "r"(G_DQ_WARPS));
+            asm volatile("mbarrier.init.shared::cta.b64 [%0], 1;" ::"r"(g_smem(&acc_full[s])));
+            asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(g_smem(&acc_empty[s])), "r"(G_EPI_WARPS));
+        }
+        asm volatile("mbarrier.init.shared::cta.b64 [%0], 1;" ::"r"(g_smem(&drain)));
         asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
         s_abort = 0;
     }
-    if (warp == 0) {   // 512 TMEM columns: gate accumulator at 0, up at 256
-        asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], 512;" ::"r"(tc_smem(&s_tmem)));
+    if (warp == 2) {
+        asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], 512;" ::"r"(g_smem(&s_tmem)));
         asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;");
     }
     asm volatile("griddepcontrol.wait;" ::: "memory");
 
-    // tile list: active experts, tiles per expert = ceil(n / 256) * MT
+    // tile list: active experts and the prefix sum of their tile counts
     {
-        constexpr int PER = kMaxE / TC_THREADS;
+        constexpr int PER = kMaxE / G_THREADS;
         int cnt[PER], nt[PER], local = 0, ltiles = 0;
 #pragma unroll
         for (int i = 0; i < PER; i++) {
             const int e = tid * PER + i;
             const int n = (e < a.E) ? a.offsets[e + 1] - a.offsets[e] : 0;
             cnt[i] = n > 0;
-            nt[i] = n > 0 ? ((n + TC_BN_MAX - 1) / TC_BN_MAX) * MT : 0;
+            nt[i] = n > 0 ? ((n + C::kNMax - 1) / C::kNMax) * MT : 0;
             local += cnt[i];
             ltiles += nt[i];
         }
@@ -231,13 +319,12 @@ __global__ void __launch_bounds__(TC_THREADS, 1) tc_grouped_gemm(TcArgs a) {
             const int n1 = __shfl_up_sync(0xffffffffu, v, o), n2 = __shfl_up_sync(0xffffffffu, w, o);
             if (lane >= o) { v += n1; w += n2; }
         }
-        __shared__ int s_wt[TC_THREADS / 32];
         if (lane == 31) { s_wsum[warp] = v; s_wt[warp] = w; }
-        tc_fence_before();
+        g_fence_before();
         __syncthreads();
-        tc_fence_after();
+        g_fence_after();
         int base = 0, tbase = 0, tot = 0, ttot = 0;
-        for (int q = 0; q < TC_THREADS / 32; q++) {
+        for (int q = 0; q < G_THREADS / 32; q++) {
             if (q < warp) { base += s_wsum[q]; tbase += s_wt[q]; }
             tot += s_wsum[q];
             ttot += s_wt[q];
@@ -250,234 +337,478 @@ __global__ void __launch_bounds__(TC_THREADS, 1) tc_grouped_gemm(TcArgs a) {
         __syncthreads();
     }
     asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
-    const uint32_t tmem = s_tmem;
-    const int ntiles = s_total;
-    // stage ring on a 1024-byte boundary (128B-swizzle atoms)
-    uint8_t* ring = smem + ((1024u - (tc_smem(smem) & 1023u)) & 1023u);
-    uint32_t kcount = 0;            // K blocks issued by this CTA (stage / phase counter)
 
-    for (int tile = blockIdx.x; tile < ntiles && !s_abort; tile += gridDim.x) {
-        // tile -> (expert, n-tile, m-tile)
-        int lo = 0, hi = s_nact - 1;
+    const uint32_t tmem = s_tmem;
+    const int ntiles = s_total, nact = s_nact;
+    uint8_t* pk = smem + ((1024u - (g_smem(smem) & 1023u)) & 1023u);
+    uint8_t* bring = pk + C::kPkStages * C::kPkStageBytes;
+    uint8_t* scbuf = bring + C::kBStages * C::kBStageBytes;         // int4: 2 buffers x kNMat x sc_mat_bytes
+
+    auto tile_of = [&](int tile) {
+        int lo = 0, hi = nact - 1;
         while (lo < hi) {
             const int mid = (lo + hi + 1) >> 1;
             if (s_prefix[mid] <= tile) lo = mid; else hi = mid - 1;
         }
-        const int e = s_active[lo];
+        GTile t;
+        t.e = s_active[lo];
         const int local = tile - s_prefix[lo];
-        const int nti = local / MT, m0 = (local % MT) * TC_BM;
-        const int ebase = a.offsets[e], n_e = a.offsets[e + 1] - ebase;
-        const int ntile = (n_e + TC_BN_MAX - 1) / TC_BN_MAX;
-        const int per = (n_e + ntile - 1) / ntile;                 // balanced rows per n-tile
-        const int n0 = nti * per;
-        const int nval = min(per, n_e - n0);
-        const int bn = (nval + 15) & ~15;                            // MMA N: multiple of 16
-        const uint32_t idesc = tc_idesc(bn, FMT == MOE_FMT_NVFP4);
+        t.ebase = a.offsets[t.e];
+        const int n_e = a.offsets[t.e + 1] - t.ebase;
+        const int ntile = (n_e + C::kNMax - 1) / C::kNMax;
+        const int per = (n_e + ntile - 1) / ntile;                  // balanced rows per n-tile
+        t.m0 = (local / ntile) * G_BM;
+        t.n0 = (local % ntile) * per;
+        t.nval = min(per, n_e - t.n0);
+        t.bn = (t.nval + 15) & ~15;
+        return t;
+    };
+    auto fail = [&]() {
+        set_status(a.status, MOE_ERR_TIMEOUT);
+        s_abort = 1;
+    };
 
-        // Register double buffer: the global loads of block kb+1 are issued
-        // before block kb is dequantised and stored.  Per thread: up to 2
-        // weight units and up to 8 activation chunks per block.
-        const int nunits = (a.gateup ? 2 : 1) * TC_BM * 2;
-        const int nchunks = bn * 8;
-        TcWUnit wu[2][2];
-        uint4 xv[2][8];
-        auto load_block = [&](int kb, auto bufc) {
-            constexpr int buf = decltype(bufc)::value;
-            const int k0 = kb * TC_BK;
-#pragma unroll
-            for (int q = 0; q < 2; q++) {
-                const int uidx = tid + q * TC_THREADS;
-                if (uidx < nunits) {
-                    const int mi = uidx / (TC_BM * 2), rr = (uidx / 2) % TC_BM, half = uidx & 1;
-                    tc_load_wunit<FMT>(a, mi, size_t(e) * a.out_dim + m0 + rr, k0 + half * 32, wu[buf][q]);
+    if (warp == 0) {
+        // ---------------- weight producer ----------------
+        if (lane == 0) {
+            uint32_t pc = 0;
+            int t = 0;
+            for (int tile = blockIdx.x; tile < ntiles && !s_abort; tile += gridDim.x) {
+                const GTile T = tile_of(tile);
+                const int row0 = T.e * a.out_dim + T.m0;
+                if (FMT == MOE_FMT_INT4_G128) {
+                    const int b = t & 1;
+                    if (t >= 2 && !g_wait(g_smem(&sc_empty[b]), ((t >> 1) - 1) & 1, &s_abort, 64)) { fail(); break; }
+                    const uint32_t bar = g_smem(&sc_full[b]);
+                    uint8_t* dst = scbuf + b * C::kNMat * sc_mat_bytes;
+                    g_expect(bar, sc_mat_bytes * C::kNMat);
+                    g_bulk(g_smem(dst), a.sc0 + size_t(row0) * ngroups * 2, sc_mat_bytes, bar);
+                    if (GU) g_bulk(g_smem(dst + sc_mat_bytes), a.sc1 + size_t(row0) * ngroups * 2, sc_mat_bytes, bar);
                 }
-            }
-#pragma unroll
-            for (int q = 0; q < 8; q++) {
-                const int cidx = tid + q * TC_THREADS;
-                uint4 v = make_uint4(0, 0, 0, 0);
-                if (cidx < nchunks) {
-                    const int n = cidx >> 3, c = cidx & 7;
-                    if (n < nval) {
-                        const int r = ebase + n0 + n;
-                        const int arow = a.act_by_token ? a.row_slot[r] / a.top_k : r;
-                        v = __ldg(reinterpret_cast<const uint4*>(a.act + (size_t(arow) * a.in_dim + k0 + c * 8) * 2));
+                t++;
+                bool ok = true;
+                for (int ps = 0; ps < NPS; ps++, pc++) {
+                    const int s = pc % C::kPkStages;
+                    if (pc >= uint32_t(C::kPkStages) &&
+                        !g_wait(g_smem(&pk_empty[s]), ((pc / C::kPkStages) - 1) & 1, &s_abort, 32)) {
+                        ok = false;
+                        break;
+                    }
+                    const uint32_t bar = g_smem(&pk_full[s]);
+                    uint8_t* st = pk + s * C::kPkStageBytes;
+                    g_expect(bar, C::kPkStageBytes);
+                    g_tma2d(g_smem(st), &a.tm_p0, ps * C::kPkX, row0, bar);
+                    if (GU) g_tma2d(g_smem(st + C::kMatBytes), &a.tm_p1, ps * C::kPkX, row0, bar);
+                    if (FMT == MOE_FMT_NVFP4) {
+                        uint8_t* ss = st + C::kNMat * C::kMatBytes;
+                        g_tma2d(g_smem(ss), &a.tm_s0, ps * 16, row0, bar);
+                        if (GU) g_tma2d(g_smem(ss + C::kNvScBytes), &a.tm_s1, ps * 16, row0, bar);
                     }
                 }
-                xv[buf][q] = v;
+                if (!ok) { fail(); break; }
             }
-        };
-        load_block(0, std::integral_constant<int, 0>{});
-        auto step = [&](int kb, auto bufc) {
-            constexpr int buf = decltype(bufc)::value;
-            const int s = kcount % TC_STAGES;
-            uint8_t* A0 = ring + s * TC_STAGE_BYTES;
-            uint8_t* A1 = A0 + TC_A_BYTES;
-            uint8_t* B = A0 + 2 * TC_A_BYTES;
-            if (kb + 1 < KB) load_block(kb + 1, std::integral_constant<int, buf ^ 1>{});
-            if (kcount >= TC_STAGES && !s_abort) {                  // the MMAs that read this stage are done
-                if (!tc_wait(tc_smem(&bars[s]), ((kcount / TC_STAGES) - 1) & 1)) {
-                    set_status(a.status, MOE_ERR_TIMEOUT);
-                    s_abort = 1;
-                }
-            }
-#pragma unroll
-            for (int q = 0; q < 2; q++) {
-                const int uidx = tid + q * TC_THREADS;
-                if (uidx < nunits) {
-                    const int mi = uidx / (TC_BM * 2), rr = (uidx / 2) % TC_BM, half = uidx & 1;
-                    tc_store_wunit<FMT>(mi ? A1 : A0, rr, half * 4, wu[buf][q]);
-                }
-            }
-#pragma unroll
-            for (int q = 0; q < 8; q++) {
-                const int cidx = tid + q * TC_THREADS;
-                if (cidx < nchunks) *reinterpret_cast<uint4*>(B + tc_swz(cidx >> 3, cidx & 7)) = xv[buf][q];
-            }
-            asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
-            __syncthreads();
-            if (tid == 0 && !s_abort) {
-                tc_fence_after();
-                const uint32_t a0 = tc_smem(A0), a1 = tc_smem(A1), b0 = tc_smem(B);
-#pragma unroll
-                for (int ks = 0; ks < TC_BK / 16; ks++) {
-                    const uint32_t acc = (kb > 0 || ks > 0) ? 1u : 0u;
-                    tc_mma(tmem, tc_desc(a0 + ks * 32), tc_desc(b0 + ks * 32), idesc, acc);
-                    if (a.gateup) tc_mma(tmem + 256, tc_desc(a1 + ks * 32), tc_desc(b0 + ks * 32), idesc, acc);
-                }
-                tc_commit(tc_smem(&bars[s]));
-            }
-            kcount++;
-        };
-        for (int kb = 0; kb < KB; kb += 2) {
-            step(kb, std::integral_constant<int, 0>{});
-            if (kb + 1 < KB) step(kb + 1, std::integral_constant<int, 1>{});
+            // drain: every copy issued has landed before the CTA exits
+            const uint32_t first = pc > uint32_t(C::kPkStages) ? pc - C::kPkStages : 0;
+            for (uint32_t n = first; n < pc; n++) g_drain_wait(g_smem(&pk_full[n % C::kPkStages]), (n / C::kPkStages) & 1);
+            if (FMT == MOE_FMT_INT4_G128)
+                for (int n = t > 2 ? t - 2 : 0; n < t; n++) g_drain_wait(g_smem(&sc_full[n & 1]), (n >> 1) & 1);
         }
-        // epilogue: wait for the tile's last commit, read the accumulators
-        {
-            const uint32_t last = kcount - 1;
-            if (!s_abort && !tc_wait(tc_smem(&bars[last % TC_STAGES]), (last / TC_STAGES) & 1)) {
-                set_status(a.status, MOE_ERR_TIMEOUT);
-                s_abort = 1;
+    } else if (warp == 1) {
+        // ---------------- activation producer ----------------
+        if (lane == 0) {
+            uint32_t bc = 0;
+            for (int tile = blockIdx.x; tile < ntiles && !s_abort; tile += gridDim.x) {
+                const GTile T = tile_of(tile);
+                const int row0 = T.ebase + T.n0;
+                const int nbox = T.bn / 16;
+                bool ok = true;
+                for (int kb = 0; kb < KB; kb++, bc++) {
+                    const int s = bc % C::kBStages;
+                    if (bc >= uint32_t(C::kBStages) &&
+                        !g_wait(g_smem(&b_empty[s]), ((bc / C::kBStages) - 1) & 1, &s_abort, 32)) {
+                        ok = false;
+                        break;
+                    }
+                    const uint32_t bar = g_smem(&b_full[s]);
+                    uint8_t* st = bring + s * C::kBStageBytes;
+                    g_expect(bar, uint32_t(nbox) * 2048u);
+                    for (int j = 0; j < nbox; j++) g_tma2d(g_smem(st + j * 2048), &a.tm_b, kb * G_BK, row0 + 16 * j, bar);
+                }
+                if (!ok) { fail(); break; }
             }
-            tc_fence_after();
-            const int quarter = warp & 3, chalf = warp >> 2;
-            const int f = m0 + quarter * 32 + lane;            // output feature of this thread
-            const uint32_t lane_addr = uint32_t(quarter * 32) << 16;
+            const uint32_t first = bc > uint32_t(C::kBStages) ? bc - C::kBStages : 0;
+            for (uint32_t n = first; n < bc; n++) g_drain_wait(g_smem(&b_full[n % C::kBStages]), (n / C::kBStages) & 1);
+        }
+    } else if (warp == 2) {
+        // ---------------- MMA issuer ----------------
+        if (lane == 0) {
+            uint32_t bc = 0, ac = 0, pc = 0;
+            int t = 0;
+            for (int tile = blockIdx.x; tile < ntiles && !s_abort; tile += gridDim.x, t++) {
+                const GTile T = tile_of(tile);
+                const uint32_t idesc = g_idesc(T.bn, C::kMmaF16);
+                const int buf = t & 1;
+                const uint32_t d = tmem + buf * 128;
+                if (t >= 2 && !g_wait(g_smem(&acc_empty[buf]), ((t >> 1) - 1) & 1, &s_abort)) { fail(); break; }
+                g_fence_after();
+                bool ok = true;
+                for (int kb = 0; kb < KB; kb++) {
+                    const int sb = bc % C::kBStages;
+                    if (!g_wait(g_smem(&b_full[sb]), (bc / C::kBStages) & 1, &s_abort)) { ok = false; break; }
+                    int sa = 0, sp = 0;
+                    if (C::kTmemA) {
+                        sa = ac % C::kAStages;
+                        if (!g_wait(g_smem(&a_full[sa]), (ac / C::kAStages) & 1, &s_abort)) { ok = false; break; }
+                    } else {
+                        sp = pc % C::kPkStages;
+                        if (!g_wait(g_smem(&pk_full[sp]), (pc / C::kPkStages) & 1, &s_abort)) { ok = false; break; }
+                    }
+                    g_fence_after();
+                    const uint32_t b0 = g_smem(bring + sb * C::kBStageBytes);
+#pragma unroll
+                    for (int ks = 0; ks < G_BK / 16; ks++) {
+                        const uint32_t acc = (kb > 0 || ks > 0) ? 1u : 0u;
+                        const uint64_t bd = g_desc(b0 + ks * 32);
+                        if (C::kTmemA) {
+                            const uint32_t at = tmem + 256 + sa * C::kAStageCols + ks * 8;
+                            g_mma_ts(d, at, bd, idesc, acc);
+                            if (GU) g_mma_ts(d + C::kUpCol, at + 32, bd, idesc, acc);
+                        } else {
+                            const uint32_t a0 = g_smem(pk + sp * C::kPkStageBytes);
+                            g_mma_ss(d, g_desc(a0 + ks * 32), bd, idesc, acc);
+                            if (GU) g_mma_ss(d + C::kUpCol, g_desc(a0 + C::kMatBytes + ks * 32), bd, idesc, acc);
+                        }
+                    }
+                    g_commit(g_smem(&b_empty[sb]));
+                    if (C::kTmemA) g_commit(g_smem(&a_empty[sa]));
+                    else g_commit(g_smem(&pk_empty[sp]));
+                    bc++;
+                    if (C::kTmemA) ac++; else pc++;
+                }
+                if (!ok) { fail(); break; }
+                g_commit(g_smem(&acc_full[buf]));
+            }
+            // drain: every MMA this thread issued has completed
+            g_commit(g_smem(&drain));
+            g_drain_wait(g_smem(&drain), 0);
+        }
+    } else if (warp >= 4 && warp < 8) {
+        // ---------------- epilogue ----------------
+        const int q = warp & 3;
+        const uint32_t lane_addr = uint32_t(q * 32) << 16;
+        int t = 0;
+        for (int tile = blockIdx.x; tile < ntiles && !s_abort; tile += gridDim.x, t++) {
+            const GTile T = tile_of(tile);
+            const int buf = t & 1;
+            if (!g_wait(g_smem(&acc_full[buf]), (t >> 1) & 1, &s_abort, 128)) { fail(); break; }
+            g_fence_after();
+            const int f = T.m0 + q * 32 + lane;
+            const int fo = a.perm_out ? ((f & ~7) | ((f & 7) < 4 ? 2 * (f & 7) : 2 * (f & 7) - 7)) : f;
             float gsc = 1.f, usc = 1.f;
-            if (FMT == MOE_FMT_NVFP4) { gsc = a.g0[e]; usc = a.gateup ? a.g1[e] : 1.f; }
-            for (int cc = chalf; cc * 16 < bn; cc += 2) {
-                uint32_t g[16], uvals[16];
-                tc_ld16(tmem + lane_addr + cc * 16, g);
-                if (a.gateup) tc_ld16(tmem + 256 + lane_addr + cc * 16, uvals);
-                tc_ld_wait();
+            if (FMT == MOE_FMT_NVFP4) { gsc = a.g0[T.e]; if (GU) usc = a.g1[T.e]; }
+            const uint32_t acc0 = tmem + lane_addr + buf * 128;
+            const int rbase = T.ebase + T.n0;
+            for (int c = 0; c < T.bn; c += 16) {
+                // the factor of row c + j (activation row scale, routing weight) sits in lane j
+                float rowf = 1.f;
+                const int nn = c + (lane & 15);
+                if (nn < T.nval) {
+                    if (FMT == MOE_FMT_NVFP4) rowf = a.act_scale[rbase + nn];
+                    if (!GU && a.topk_w) rowf *= a.topk_w[a.row_slot[rbase + nn]];
+                }
+                uint32_t g[16], u[16];
+                g_ld16(acc0 + c, g);
+                if (GU) g_ld16(acc0 + C::kUpCol + c, u);
+                g_ld_wait();
 #pragma unroll
                 for (int j = 0; j < 16; j++) {
-                    const int n = cc * 16 + j;
-                    if (n >= nval) break;
-                    const int r = ebase + n0 + n;
-                    float rs = 1.f;
-                    if (FMT == MOE_FMT_NVFP4) rs = a.act_scale[a.act_by_token ? a.row_slot[r] / a.top_k : r];
-                    float v;
-                    if (a.gateup) {
-                        const float gg = __uint_as_float(g[j]) * gsc * rs, uu = __uint_as_float(uvals[j]) * usc * rs;
-                        v = gg / (1.0f + expf(-gg)) * uu;
-                    } else {
-                        const float wt = a.topk_w ? a.topk_w[a.row_slot[r]] : 1.f;
-                        v = wt * (__uint_as_float(g[j]) * gsc * rs);
+                    const float fj = __shfl_sync(0xffffffffu, rowf, j);
+                    if (c + j < T.nval) {
+                        float v;
+                        if (GU) {
+                            const float gg = __uint_as_float(g[j]) * gsc * fj;
+                            const float uu = __uint_as_float(u[j]) * usc * fj;
+                            v = gg / (1.0f + expf(-gg)) * uu;
+                        } else {
+                            v = __uint_as_float(g[j]) * gsc * fj;
+                        }
+                        a.out[size_t(rbase + c + j) * a.out_dim + fo] = __float2bfloat16_rn(v);
                     }
-                    a.out[size_t(r) * a.out_dim + f] = __float2bfloat16_rn(v);
                 }
             }
-            tc_fence_before();
-            __syncthreads();          // accumulators free for the next tile
+            g_fence_before();
+            __syncwarp();
+            if (lane == 0) g_arrive(g_smem(&acc_empty[buf]));
         }
+    } else if (warp >= 8 && C::kTmemA) {
+        // ---------------- dequantisation ----------------
+        // gate/up: this warp fills matrix hsel of every A stage (all four K
+        // blocks of a weight stage); down: it fills the K blocks of parity
+        // hsel.  Each K block is two 16-byte chunks of this thread's row.
+        // The next K block is dequantised while the tensor-memory store of
+        // the current one completes.
+        constexpr int kMine = GU ? 4 : 2;
+        const int q = warp & 3, hsel = (warp - 8) >> 2;
+        const int r = q * 32 + lane;                                 // weight row within the tile
+        const uint32_t lane_addr = uint32_t(q * 32) << 16;
+        uint32_t pc = 0;
+        int t = 0;
+        bool ok = true;
+        for (int tile = blockIdx.x; tile < ntiles && ok && !s_abort; tile += gridDim.x, t++) {
+            const uint8_t* scrow = nullptr;
+            if (FMT == MOE_FMT_INT4_G128) {
+                const int b = t & 1;
+                if (!g_wait(g_smem(&sc_full[b]), (t >> 1) & 1, &s_abort)) { ok = false; break; }
+                scrow = scbuf + b * C::kNMat * sc_mat_bytes + (GU ? hsel * sc_mat_bytes : 0) + r * ngroups * 2;
+            }
+            for (int ps = 0; ps < NPS && ok; ps++, pc++) {
+                const int s = pc % C::kPkStages;
+                if (!g_wait(g_smem(&pk_full[s]), (pc / C::kPkStages) & 1, &s_abort)) { ok = false; break; }
+                const uint8_t* st = pk + s * C::kPkStageBytes;
+                const uint8_t* wt = st + (GU ? hsel * C::kMatBytes : 0);
+                uint32_t scw = 0;                      // int4: bf16 scales of groups 2ps (low) and 2ps+1 (high)
+                uint4 nsc = make_uint4(0, 0, 0, 0);    // NVFP4: the 16 E4M3 scales of this row and stage
+                if (FMT == MOE_FMT_INT4_G128) scw = *reinterpret_cast<const uint32_t*>(scrow + ps * 4);
+                else if (FMT == MOE_FMT_NVFP4)
+                    nsc = *reinterpret_cast<const uint4*>(st + C::kNMat * C::kMatBytes + (GU ? hsel * C::kNvScBytes : 0) +
+                                                          r * 16);
+                const uint32_t nscw[4] = {nsc.x, nsc.y, nsc.z, nsc.w};
+                uint32_t o[2][2][16];
+                // dequantise my i-th K block of this stage into o[buf]
+                auto produce = [&](auto ic, auto bc) {
+                    constexpr int i = decltype(ic)::value, buf = decltype(bc)::value;
+                    const int sub = GU ? i : hsel + 2 * i;
+#pragma unroll
+                    for (int h = 0; h < 2; h++) {
+                        const uint4 w = *reinterpret_cast<const uint4*>(wt + g_swz(r, 2 * sub + h));
+                        if (FMT == MOE_FMT_INT4_G128) {
+                            g_dq_int4(w, scw >> (16 * (GU ? (i >> 1) : i)), o[buf][h]);
+                        } else {
+                            const uint32_t sw = GU ? nscw[i] : (hsel ? nscw[2 * i + 1] : nscw[2 * i]);
+                            g_dq_nvfp4(w, sw >> (16 * h), o[buf][h]);
+                        }
+                    }
+                };
+                auto publish = [&](auto ic, auto bc) {
+                    constexpr int i = decltype(ic)::value, buf = decltype(bc)::value;
+                    const int sub = GU ? i : hsel + 2 * i;
+                    const uint32_t kbg = pc * 4 + sub;                  // K block index in this CTA's stream
+                    const int sa = kbg % C::kAStages;
+                    if (kbg >= uint32_t(C::kAStages) &&
+                        !g_wait(g_smem(&a_empty[sa]), ((kbg / C::kAStages) - 1) & 1, &s_abort)) {
+                        ok = false;
+                        return;
+                    }
+                    g_fence_after();
+                    const uint32_t col = 256 + sa * C::kAStageCols + (GU ? hsel * 32 : 0);
+                    g_st16(tmem + lane_addr + col, o[buf][0]);
+                    g_st16(tmem + lane_addr + col + 16, o[buf][1]);
+                    if constexpr (i + 1 < kMine) produce(std::integral_constant<int, i + 1>{},
+                                                         std::integral_constant<int, buf ^ 1>{});
+                    g_st_wait();
+                    g_fence_before();
+                    __syncwarp();
+                    if (lane == 0) g_arrive(g_smem(&a_full[sa]));
+                };
+                produce(std::integral_constant<int, 0>{}, std::integral_constant<int, 0>{});
+                publish(std::integral_constant<int, 0>{}, std::integral_constant<int, 0>{});
+                if (ok) publish(std::integral_constant<int, 1>{}, std::integral_constant<int, 1>{});
+                if constexpr (kMine == 4) {
+                    if (ok) publish(std::integral_constant<int, 2>{}, std::integral_constant<int, 0>{});
+                    if (ok) publish(std::integral_constant<int, 3>{}, std::integral_constant<int, 1>{});
+                }
+                __syncwarp();
+                if (lane == 0) g_arrive(g_smem(&pk_empty[s]));
+            }
+            if (!ok) break;
+            if (FMT == MOE_FMT_INT4_G128) {
+                __syncwarp();
+                if (lane == 0) g_arrive(g_smem(&sc_empty[t & 1]));
+            }
+        }
+        if (!ok) fail();
     }
+
+    g_fence_before();
     __syncthreads();
-    tc_fence_after();
-    if (warp == 0) asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, 512;" ::"r"(tmem));
+    g_fence_after();
+    if (warp == 2) asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, 512;" ::"r"(tmem));
 }
 
-// NVFP4: activations as f16 rows times 2^-e (e >= 0 least with |x| * 2^-e <= 16384), scale 2^e.
-__global__ void __launch_bounds__(256) tc_act_f16(const __nv_bfloat16* __restrict__ act, int rows, int in_dim,
-                                                  __half* __restrict__ out, float* __restrict__ scale) {
+// ---------------------------------------------------------------------------
+// Activation pre-pass: gather the GEMM's rows (row r reads activation row
+// row_slot[r] / top_k when by_token, else row r) into the operand order:
+//   mode 0: bf16 copy;  mode 1: bf16, pair order 0,4,1,5,2,6,3,7 in every 8;
+//   mode 2: f16 times 2^-e (e >= 0 least with |x| * 2^-e <= 16384), row scale 2^e.
+// One warp per row.
+// ---------------------------------------------------------------------------
+__global__ void __launch_bounds__(256) g_prep(const __nv_bfloat16* __restrict__ src, int in_dim,
+                                              const int32_t* __restrict__ row_slot, int top_k, int by_token,
+                                              int rows, int mode, uint16_t* __restrict__ dst,
+                                              float* __restrict__ scale) {
     asm volatile("griddepcontrol.wait;" ::: "memory");
-    const int warp = (blockIdx.x * blockDim.x + threadIdx.x) >> 5, lane = threadIdx.x & 31;
-    if (warp >= rows) return;
-    const __nv_bfloat16* row = act + size_t(warp) * in_dim;
-    float amax = 0.f;
-    for (int i = lane * 8; i < in_dim; i += 256) {
-        const uint4 v = *reinterpret_cast<const uint4*>(row + i);
-        amax = fmaxf(amax, fmaxf(fmaxf(fabsf(bf16_lo(v.x)), fabsf(bf16_hi(v.x))), fmaxf(fabsf(bf16_lo(v.y)), fabsf(bf16_hi(v.y)))));
-        amax = fmaxf(amax, fmaxf(fmaxf(fabsf(bf16_lo(v.z)), fabsf(bf16_hi(v.z))), fmaxf(fabsf(bf16_lo(v.w)), fabsf(bf16_hi(v.w)))));
+    const int row = (blockIdx.x * blockDim.x + threadIdx.x) >> 5, lane = threadIdx.x & 31;
+    if (row >= rows) return;
+    const int srow = by_token ? row_slot[row] / top_k : row;
+    const uint4* s = reinterpret_cast<const uint4*>(src + size_t(srow) * in_dim);
+    uint4* d = reinterpret_cast<uint4*>(dst + size_t(row) * in_dim);
+    const int n16 = in_dim / 8;
+    if (mode == 0) {
+        for (int i = lane; i < n16; i += 32) d[i] = s[i];
+    } else if (mode == 1) {
+        for (int i = lane; i < n16; i += 32) {
+            const uint4 v = s[i];
+            uint4 o;
+            o.x = __byte_perm(v.x, v.z, 0x5410);   // (x0, x4)
+            o.y = __byte_perm(v.x, v.z, 0x7632);   // (x1, x5)
+            o.z = __byte_perm(v.y, v.w, 0x5410);   // (x2, x6)
+            o.w = __byte_perm(v.y, v.w, 0x7632);   // (x3, x7)
+            d[i] = o;
+        }
+    } else {
+        float amax = 0.f;
+        for (int i = lane; i < n16; i += 32) {
+            const uint4 v = s[i];
+            amax = fmaxf(amax, fmaxf(fmaxf(fabsf(bf16_lo(v.x)), fabsf(bf16_hi(v.x))), fmaxf(fabsf(bf16_lo(v.y)), fabsf(bf16_hi(v.y)))));
+            amax = fmaxf(amax, fmaxf(fmaxf(fabsf(bf16_lo(v.z)), fabsf(bf16_hi(v.z))), fmaxf(fabsf(bf16_lo(v.w)), fabsf(bf16_hi(v.w)))));
+        }
+        for (int o = 16; o > 0; o >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, o));
+        int e = 0;
+        while (e < 126 && ldexpf(amax, -e) > 16384.f) e++;
+        const float down = ldexpf(1.f, -e);
+        for (int i = lane; i < n16; i += 32) {
+            const uint4 v = s[i];
+            __half2 h[4];
+            h[0] = __floats2half2_rn(bf16_lo(v.x) * down, bf16_hi(v.x) * down);
+            h[1] = __floats2half2_rn(bf16_lo(v.y) * down, bf16_hi(v.y) * down);
+            h[2] = __floats2half2_rn(bf16_lo(v.z) * down, bf16_hi(v.z) * down);
+            h[3] = __floats2half2_rn(bf16_lo(v.w) * down, bf16_hi(v.w) * down);
+            d[i] = *reinterpret_cast<uint4*>(h);
+        }
+        if (lane == 0) scale[row] = ldexpf(1.f, e);
     }
-    for (int o = 16; o > 0; o >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, o));
-    int e = 0;
-    while (e < 126 && ldexpf(amax, -e) > 16384.f) e++;
-    const float down = ldexpf(1.f, -e);
-    for (int i = lane * 8; i < in_dim; i += 256) {
-        const uint4 v = *reinterpret_cast<const uint4*>(row + i);
-        __half2 h[4];
-        h[0] = __floats2half2_rn(bf16_lo(v.x) * down, bf16_hi(v.x) * down);
-        h[1] = __floats2half2_rn(bf16_lo(v.y) * down, bf16_hi(v.y) * down);
-        h[2] = __floats2half2_rn(bf16_lo(v.z) * down, bf16_hi(v.z) * down);
-        h[3] = __floats2half2_rn(bf16_lo(v.w) * down, bf16_hi(v.w) * down);
-        *reinterpret_cast<uint4*>(out + size_t(warp) * in_dim + i) = *reinterpret_cast<uint4*>(h);
-    }
-    if (lane == 0) scale[warp] = ldexpf(1.f, e);
 }
 
-template <int FMT>
-static cudaError_t tc_launch(const TcArgs& a, cudaStream_t s) {
-    static int sms = 0;
-    static bool attr = false;
-    auto k = tc_grouped_gemm<FMT>;
-    if (sms == 0) {
-        int dev = 0;
-        cudaGetDevice(&dev);
-        cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
-    }
-    const int smem = TC_STAGES * TC_STAGE_BYTES + 1024;
-    if (!attr) {
-        cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
-        if (e != cudaSuccess) return e;
-        attr = true;
-    }
-    k<<<sms, TC_THREADS, smem, s>>>(a);
-    return cudaGetLastError();
+// ---------------------------------------------------------------------------
+// Host side
+// ---------------------------------------------------------------------------
+static PFN_cuTensorMapEncodeTiled g_encode_fn = nullptr;
+
+static int g_encoder() {
+    static std::once_flag once;
+    std::call_once(once, [] {
+        void* fn = nullptr;
+        cudaDriverEntryPointQueryResult q{};
+        if (cudaGetDriverEntryPointByVersion("cuTensorMapEncodeTiled", &fn, 12000, cudaEnableDefault, &q) ==
+                cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            g_encode_fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled>(fn);
+    });
+    return g_encode_fn ? MOE_OK : MOE_ERR_CUDA;
 }
 
-static int tc_run(const GemvProblem& p, bool gateup, int act_rows, void* prep_ws, cudaStream_t s) {
-    if (p.out_dim % TC_BM || p.in_dim % TC_BK) return MOE_ERR_UNSUPPORTED;
-    TcArgs a{};
-    a.fmt = p.fmt; a.gateup = gateup; a.E = p.E; a.out_dim = p.out_dim; a.in_dim = p.in_dim;
-    a.top_k = p.top_k; a.act_by_token = p.act_by_token;
-    a.p0 = reinterpret_cast<const uint8_t*>(p.p0); a.s0 = reinterpret_cast<const uint8_t*>(p.s0); a.g0 = p.g0;
-    a.p1 = reinterpret_cast<const uint8_t*>(p.p1); a.s1 = reinterpret_cast<const uint8_t*>(p.s1); a.g1 = p.g1;
-    a.offsets = p.offsets; a.row_slot = p.row_slot; a.topk_w = p.topk_w; a.out = p.out; a.status = p.status;
-    a.act = reinterpret_cast<const uint8_t*>(p.act);
-    if (p.fmt == MOE_FMT_NVFP4) {
-        float* scale = reinterpret_cast<float*>(prep_ws);
-        __half* act16 = reinterpret_cast<__half*>(reinterpret_cast<uint8_t*>(prep_ws) + align256(size_t(act_rows) * 4));
-        tc_act_f16<<<(act_rows * 32 + 255) / 256, 256, 0, s>>>(p.act, act_rows, p.in_dim, act16, scale);
-        a.act = reinterpret_cast<const uint8_t*>(act16);
-        a.act_scale = scale;
-    }
-    cudaError_t e;
-    if (p.fmt == MOE_FMT_INT4_G128) e = tc_launch<MOE_FMT_INT4_G128>(a, s);
-    else if (p.fmt == MOE_FMT_NVFP4) e = tc_launch<MOE_FMT_NVFP4>(a, s);
-    else e = tc_launch<MOE_FMT_BF16>(a, s);
-    return e == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
+// 2D map over [outer rows][inner elements] of 1- or 2-byte elements; pitch in bytes.
+static int g_map(CUtensorMap* m, bool two_byte, const void* base, uint64_t inner, uint64_t outer, uint64_t pitch,
+                 uint32_t box_in, uint32_t box_out, bool swz) {
+    if ((reinterpret_cast<uintptr_t>(base) & 15u) || (pitch & 15u)) return MOE_ERR_INVALID_ARG;
+    cuuint64_t dims[2] = {inner, outer};
+    cuuint64_t strides[1] = {pitch};
+    cuuint32_t box[2] = {box_in, box_out};
+    cuuint32_t es[2] = {1, 1};
+    const CUresult r = g_encode_fn(m, two_byte ? CU_TENSOR_MAP_DATA_TYPE_UINT16 : CU_TENSOR_MAP_DATA_TYPE_UINT8, 2,
+                                   const_cast<void*>(base), dims, strides, box, es, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                                   swz ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_NONE,
+                                   CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS ? MOE_OK : MOE_ERR_CUDA;
 }
 
-int launch_grouped_gemm(const GemvProblem& routed, const GemvProblem* shared, bool gateup, int act_rows,
-                        void* prep_ws, int32_t* tile_ws, cudaStream_t s) {
-    (void)tile_ws;
-    int rc = tc_run(routed, gateup, act_rows, prep_ws, s);
-    if (rc != MOE_OK || !shared) return rc;
-    const int sh_rows = act_rows;   // the shared expert sees every token (gate/up) or every shared row (down)
-    (void)sh_rows;
-    return tc_run(*shared, gateup, 0, nullptr, s);
+template <int FMT, bool GU>
+static size_t g_smem_bytes(int in_dim) {
+    using C = GCfg<FMT, GU>;
+    size_t b = size_t(C::kPkStages) * C::kPkStageBytes + size_t(C::kBStages) * C::kBStageBytes + 1024;
+    if (FMT == MOE_FMT_INT4_G128) b += 2 * size_t(C::kNMat) * G_BM * (in_dim / 128) * 2;
+    return b;
+}
+
+template <int FMT, bool GU>
+static int g_launch(const GArgs& a, cudaStream_t s) {
+    auto k = tc_grouped_gemm<FMT, GU>;
+    const size_t smem = g_smem_bytes<FMT, GU>(a.in_dim);
+    int dev = 0, sms = 0, optin = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess) return MOE_ERR_CUDA;
+    if (cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) return MOE_ERR_CUDA;
+    if (cudaDeviceGetAttribute(&optin, cudaDevAttrMaxSharedMemoryPerBlockOptin, dev) != cudaSuccess) return MOE_ERR_CUDA;
+    cudaFuncAttributes fa{};
+    if (cudaFuncGetAttributes(&fa, k) != cudaSuccess) return MOE_ERR_CUDA;
+    if (smem + fa.sharedSizeBytes > size_t(optin)) return MOE_ERR_UNSUPPORTED;
+    if (cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem)) != cudaSuccess)
+        return MOE_ERR_CUDA;
+    k<<<sms, G_THREADS, smem, s>>>(a);
+    return cudaGetLastError() == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
+}
+
+#define G_TRY(x)                       \
+    do {                               \
+        int _rc = (x);                 \
+        if (_rc != MOE_OK) return _rc; \
+    } while (0)
+
+int launch_grouped_gemm(const GemvProblem& p, bool gateup, int rows, const GemmBuffers& buf, cudaStream_t s) {
+    if (p.out_dim % G_BM || p.in_dim % 256 || p.E > kMaxE) return MOE_ERR_UNSUPPORTED;
+    if (p.fmt == MOE_FMT_INT4_G128 &&
+        ((reinterpret_cast<uintptr_t>(p.s0) & 15u) || (gateup && (reinterpret_cast<uintptr_t>(p.s1) & 15u))))
+        return MOE_ERR_INVALID_ARG;
+    if (rows <= 0) return MOE_OK;
+    G_TRY(g_encoder());
+
+    const int in = p.in_dim, out = p.out_dim, E = p.E;
+    const bool nv = p.fmt == MOE_FMT_NVFP4, i4 = p.fmt == MOE_FMT_INT4_G128;
+    // activation operand rows [rows, in]: bf16 (f16 for NVFP4) in the kernel's order
+    const void* bsrc = p.act;
+    const float* ascale = nullptr;
+    if (!buf.act_ready || nv) {
+        if (!buf.act_buf || (nv && !buf.scale_buf)) return MOE_ERR_WORKSPACE;
+        const int mode = nv ? 2 : (i4 ? 1 : 0);
+        g_prep<<<(rows * 32 + 255) / 256, 256, 0, s>>>(p.act, in, p.row_slot, p.top_k, p.act_by_token, rows, mode,
+                                                       reinterpret_cast<uint16_t*>(buf.act_buf), buf.scale_buf);
+        if (cudaGetLastError() != cudaSuccess) return MOE_ERR_CUDA;
+        bsrc = buf.act_buf;
+        ascale = buf.scale_buf;
+    }
+
+    GArgs a;
+    memset(&a, 0, sizeof(a));
+    const uint64_t wrows = uint64_t(E) * out;
+    if (p.fmt == MOE_FMT_BF16) {
+        G_TRY(g_map(&a.tm_p0, true, p.p0, in, wrows, uint64_t(in) * 2, 64, 128, true));
+        if (gateup) G_TRY(g_map(&a.tm_p1, true, p.p1, in, wrows, uint64_t(in) * 2, 64, 128, true));
+    } else {
+        G_TRY(g_map(&a.tm_p0, false, p.p0, in / 2, wrows, uint64_t(in) / 2, 128, 128, true));
+        if (gateup) G_TRY(g_map(&a.tm_p1, false, p.p1, in / 2, wrows, uint64_t(in) / 2, 128, 128, true));
+    }
+    if (nv) {
+        G_TRY(g_map(&a.tm_s0, false, p.s0, in / 16, wrows, uint64_t(in) / 16, 16, 128, false));
+        if (gateup) G_TRY(g_map(&a.tm_s1, false, p.s1, in / 16, wrows, uint64_t(in) / 16, 16, 128, false));
+    }
+    G_TRY(g_map(&a.tm_b, true, bsrc, in, uint64_t(rows), uint64_t(in) * 2, 64, 16, true));
+    a.sc0 = reinterpret_cast<const uint8_t*>(p.s0);
+    a.sc1 = reinterpret_cast<const uint8_t*>(p.s1);
+    a.g0 = p.g0;
+    a.g1 = p.g1;
+    a.offsets = p.offsets;
+    a.row_slot = p.row_slot;
+    a.topk_w = p.topk_w;
+    a.act_scale = ascale;
+    a.out = p.out;
+    a.status = p.status;
+    a.E = E;
+    a.out_dim = out;
+    a.in_dim = in;
+    a.perm_out = buf.perm_out;
+
+    if (i4) return gateup ? g_launch<MOE_FMT_INT4_G128, true>(a, s) : g_launch<MOE_FMT_INT4_G128, false>(a, s);
+    if (nv) return gateup ? g_launch<MOE_FMT_NVFP4, true>(a, s) : g_launch<MOE_FMT_NVFP4, false>(a, s);
+    return gateup ? g_launch<MOE_FMT_BF16, true>(a, s) : g_launch<MOE_FMT_BF16, false>(a, s);
 }
 
 }  // namespace moe

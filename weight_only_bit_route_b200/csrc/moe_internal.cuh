@@ -146,8 +146,24 @@ int launch_quant_nvfp4(const __nv_bfloat16* w, int64_t rows, int64_t cols, uint8
 int launch_shared_routing(int T, int k, int32_t* sh_offsets, int32_t* sh_rowslot,
                           cudaStream_t s);
 
-// Prefill-shaped grouped GEMM (tcgen05), same contract as launch_stream_gemv.
-int launch_grouped_gemm(const GemvProblem& routed, const GemvProblem* shared, bool gateup, int act_rows,
-                        void* prep_ws, int32_t* tile_ws, cudaStream_t s);
+// Activation operand of the tcgen05 grouped GEMM.  Unless act_ready, a
+// pre-pass gathers the problem's rows (row r reads activation row
+// row_slot[r] / top_k when act_by_token, else row r) into act_buf
+// ([rows, in] 16-bit) in the kernel's operand order: bf16 pairs reordered
+// 0,4,1,5,2,6,3,7 in every 8 for int4, f16 with a power-of-two row scale
+// (scale_buf, [rows] fp32) for NVFP4, a plain copy for BF16.  act_ready: the
+// activation rows are already in that order (row r is row r; int4 h written
+// with perm_out, or BF16 rows that need no gather); NVFP4 always runs the
+// pre-pass.  perm_out (gate/up): write h columns in the int4 pair order.
+struct GemmBuffers {
+    void* act_buf;
+    float* scale_buf;
+    int act_ready;
+    int perm_out;
+};
+
+// Prefill-shaped grouped GEMM (tcgen05) for one problem; rows: activation
+// (and output) rows of the problem.
+int launch_grouped_gemm(const GemvProblem& p, bool gateup, int rows, const GemmBuffers& buf, cudaStream_t s);
 
 }  // namespace moe
