@@ -80,8 +80,11 @@ struct GCfg {
     static constexpr int kMatBytes = G_BM * 128;                    // one matrix per stage: 16 KB
     static constexpr int kNvScBytes = FMT == MOE_FMT_NVFP4 ? G_BM * 16 : 0;
     static constexpr int kPkStageBytes = kNMat * (kMatBytes + kNvScBytes);
-    static constexpr int kPkStages = (GU && FMT == MOE_FMT_INT4_G128) ? 3 : 4;
-    static constexpr int kBStages = GU ? 8 : 6;
+    static constexpr int kPkStages = 4;
+    static constexpr int kAStagesT = 256 / (kNMat * 32);
+    // 4-bit formats: the activation ring runs in step with the A ring, so one
+    // commit per K block frees both; BF16 keeps its own deeper ring.
+    static constexpr int kBStages = kTmemA ? kAStagesT : (GU ? 8 : 6);
     static constexpr int kBStageBytes = kNMax * 128;
     static constexpr int kAStageCols = kNMat * 32;                  // K = 64 as 16-bit pairs, per matrix
     static constexpr int kAStages = 256 / kAStageCols;
@@ -135,11 +138,25 @@ __device__ __forceinline__ bool g_wait(uint32_t bar, uint32_t parity, volatile i
         if (*abort_flag || g_timer() - t0 > G_WAIT_NS) return false;
     }
 }
+// Warp-wide bounded wait: every lane observes the phase (so whichever lane
+// is elected to issue has acquired it); the outcome is warp-uniform.
+__device__ __forceinline__ bool g_wait_w(uint32_t bar, uint32_t parity, volatile int* abort_flag, int sleep_ns = 0) {
+    const bool ok = g_wait(bar, parity, abort_flag, sleep_ns);
+    return __all_sync(0xffffffffu, ok);
+}
 // Bounded wait that ignores the abort flag (draining work already in flight).
 __device__ __forceinline__ void g_drain_wait(uint32_t bar, uint32_t parity) {
     const unsigned long long t0 = g_timer();
     while (!g_try(bar, parity) && g_timer() - t0 < G_WAIT_NS) {
     }
+}
+// One lane of a converged warp (warp-uniform code keeps the operands of the
+// tcgen05 and TMA instructions in uniform registers; issuing from inside a
+// lane-0 branch costs tens of cycles per instruction).
+__device__ __forceinline__ bool g_elect() {
+    uint32_t pred = 0;
+    asm volatile("{ .reg .pred p; elect.sync _|p, 0xffffffff; selp.u32 %0, 1, 0, p; }" : "=r"(pred));
+    return pred != 0;
 }
 __device__ __forceinline__ void g_arrive(uint32_t bar) {
     asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(bar) : "memory");
@@ -368,130 +385,149 @@ __global__ void __launch_bounds__(G_THREADS, 1) tc_grouped_gemm(const __grid_con
         s_abort = 1;
     };
 
+    static_assert(!C::kTmemA || C::kBStages == C::kAStages, "A and B rings must step together");
     if (warp == 0) {
-        // ---------------- weight producer ----------------
-        if (lane == 0) {
-            uint32_t pc = 0;
-            int t = 0;
-            for (int tile = blockIdx.x; tile < ntiles && !s_abort; tile += gridDim.x) {
-                const GTile T = tile_of(tile);
-                const int row0 = T.e * a.out_dim + T.m0;
-                if (FMT == MOE_FMT_INT4_G128) {
-                    const int b = t & 1;
-                    if (t >= 2 && !g_wait(g_smem(&sc_empty[b]), ((t >> 1) - 1) & 1, &s_abort, 64)) { fail(); break; }
-                    const uint32_t bar = g_smem(&sc_full[b]);
-                    uint8_t* dst = scbuf + b * C::kNMat * sc_mat_bytes;
+        // ---------------- weight producer (whole warp, one lane issues) ----------------
+        uint32_t pc = 0;
+        int t = 0;
+        for (int tile = blockIdx.x; tile < ntiles && !s_abort; tile += gridDim.x) {
+            const GTile T = tile_of(tile);
+            const int row0 = T.e * a.out_dim + T.m0;
+            if (FMT == MOE_FMT_INT4_G128) {
+                const int b = t & 1;
+                if (t >= 2 && !g_wait_w(g_smem(&sc_empty[b]), ((t >> 1) - 1) & 1, &s_abort, 64)) { fail(); break; }
+                const uint32_t bar = g_smem(&sc_full[b]);
+                uint8_t* dst = scbuf + b * C::kNMat * sc_mat_bytes;
+                if (g_elect()) {
                     g_expect(bar, sc_mat_bytes * C::kNMat);
                     g_bulk(g_smem(dst), a.sc0 + size_t(row0) * ngroups * 2, sc_mat_bytes, bar);
                     if (GU) g_bulk(g_smem(dst + sc_mat_bytes), a.sc1 + size_t(row0) * ngroups * 2, sc_mat_bytes, bar);
                 }
-                t++;
-                bool ok = true;
-                for (int ps = 0; ps < NPS; ps++, pc++) {
-                    const int s = pc % C::kPkStages;
-                    if (pc >= uint32_t(C::kPkStages) &&
-                        !g_wait(g_smem(&pk_empty[s]), ((pc / C::kPkStages) - 1) & 1, &s_abort, 32)) {
-                        ok = false;
-                        break;
-                    }
-                    const uint32_t bar = g_smem(&pk_full[s]);
-                    uint8_t* st = pk + s * C::kPkStageBytes;
+                __syncwarp();
+            }
+            t++;
+            bool ok = true;
+            for (int ps = 0; ps < NPS; ps++, pc++) {
+                const int s = pc % C::kPkStages;
+                if (pc >= uint32_t(C::kPkStages) &&
+                    !g_wait_w(g_smem(&pk_empty[s]), ((pc / C::kPkStages) - 1) & 1, &s_abort, 32)) {
+                    ok = false;
+                    break;
+                }
+                const uint32_t bar = g_smem(&pk_full[s]);
+                const uint32_t st = g_smem(pk + s * C::kPkStageBytes);
+                if (g_elect()) {
                     g_expect(bar, C::kPkStageBytes);
-                    g_tma2d(g_smem(st), &a.tm_p0, ps * C::kPkX, row0, bar);
-                    if (GU) g_tma2d(g_smem(st + C::kMatBytes), &a.tm_p1, ps * C::kPkX, row0, bar);
+                    g_tma2d(st, &a.tm_p0, ps * C::kPkX, row0, bar);
+                    if (GU) g_tma2d(st + C::kMatBytes, &a.tm_p1, ps * C::kPkX, row0, bar);
                     if (FMT == MOE_FMT_NVFP4) {
-                        uint8_t* ss = st + C::kNMat * C::kMatBytes;
-                        g_tma2d(g_smem(ss), &a.tm_s0, ps * 16, row0, bar);
-                        if (GU) g_tma2d(g_smem(ss + C::kNvScBytes), &a.tm_s1, ps * 16, row0, bar);
+                        const uint32_t ss = st + C::kNMat * C::kMatBytes;
+                        g_tma2d(ss, &a.tm_s0, ps * 16, row0, bar);
+                        if (GU) g_tma2d(ss + C::kNvScBytes, &a.tm_s1, ps * 16, row0, bar);
                     }
                 }
-                if (!ok) { fail(); break; }
+                __syncwarp();
             }
-            // drain: every copy issued has landed before the CTA exits
+            if (!ok) { fail(); break; }
+        }
+        // drain: every copy issued has landed before the CTA exits
+        if (lane == 0) {
             const uint32_t first = pc > uint32_t(C::kPkStages) ? pc - C::kPkStages : 0;
             for (uint32_t n = first; n < pc; n++) g_drain_wait(g_smem(&pk_full[n % C::kPkStages]), (n / C::kPkStages) & 1);
             if (FMT == MOE_FMT_INT4_G128)
                 for (int n = t > 2 ? t - 2 : 0; n < t; n++) g_drain_wait(g_smem(&sc_full[n & 1]), (n >> 1) & 1);
         }
+        __syncwarp();
     } else if (warp == 1) {
-        // ---------------- activation producer ----------------
-        if (lane == 0) {
-            uint32_t bc = 0;
-            for (int tile = blockIdx.x; tile < ntiles && !s_abort; tile += gridDim.x) {
-                const GTile T = tile_of(tile);
-                const int row0 = T.ebase + T.n0;
-                const int nbox = T.bn / 16;
-                bool ok = true;
-                for (int kb = 0; kb < KB; kb++, bc++) {
-                    const int s = bc % C::kBStages;
-                    if (bc >= uint32_t(C::kBStages) &&
-                        !g_wait(g_smem(&b_empty[s]), ((bc / C::kBStages) - 1) & 1, &s_abort, 32)) {
-                        ok = false;
-                        break;
-                    }
-                    const uint32_t bar = g_smem(&b_full[s]);
-                    uint8_t* st = bring + s * C::kBStageBytes;
-                    g_expect(bar, uint32_t(nbox) * 2048u);
-                    for (int j = 0; j < nbox; j++) g_tma2d(g_smem(st + j * 2048), &a.tm_b, kb * G_BK, row0 + 16 * j, bar);
+        // ---------------- activation producer (whole warp, one lane issues) ----------------
+        // 4-bit formats: a B stage is free once the MMAs of its K block are done,
+        // which the A-ring "empty" barrier of the same index records.
+        uint32_t bc = 0;
+        for (int tile = blockIdx.x; tile < ntiles && !s_abort; tile += gridDim.x) {
+            const GTile T = tile_of(tile);
+            const int row0 = T.ebase + T.n0;
+            const int nbox = T.bn / 16;
+            bool ok = true;
+            for (int kb = 0; kb < KB; kb++, bc++) {
+                const int s = bc % C::kBStages;
+                const uint32_t empty = C::kTmemA ? g_smem(&a_empty[s]) : g_smem(&b_empty[s]);
+                if (bc >= uint32_t(C::kBStages) && !g_wait_w(empty, ((bc / C::kBStages) - 1) & 1, &s_abort, 32)) {
+                    ok = false;
+                    break;
                 }
-                if (!ok) { fail(); break; }
+                const uint32_t bar = g_smem(&b_full[s]);
+                const uint32_t st = g_smem(bring + s * C::kBStageBytes);
+                if (g_elect()) {
+                    g_expect(bar, uint32_t(nbox) * 2048u);
+                    for (int j = 0; j < nbox; j++) g_tma2d(st + j * 2048, &a.tm_b, kb * G_BK, row0 + 16 * j, bar);
+                }
+                __syncwarp();
             }
+            if (!ok) { fail(); break; }
+        }
+        if (lane == 0) {
             const uint32_t first = bc > uint32_t(C::kBStages) ? bc - C::kBStages : 0;
             for (uint32_t n = first; n < bc; n++) g_drain_wait(g_smem(&b_full[n % C::kBStages]), (n / C::kBStages) & 1);
         }
+        __syncwarp();
     } else if (warp == 2) {
-        // ---------------- MMA issuer ----------------
-        if (lane == 0) {
-            uint32_t bc = 0, ac = 0, pc = 0;
-            int t = 0;
-            for (int tile = blockIdx.x; tile < ntiles && !s_abort; tile += gridDim.x, t++) {
-                const GTile T = tile_of(tile);
-                const uint32_t idesc = g_idesc(T.bn, C::kMmaF16);
-                const int buf = t & 1;
-                const uint32_t d = tmem + buf * 128;
-                if (t >= 2 && !g_wait(g_smem(&acc_empty[buf]), ((t >> 1) - 1) & 1, &s_abort)) { fail(); break; }
+        // ---------------- MMA issuer (whole warp, one lane issues) ----------------
+        uint32_t bc = 0, pc = 0;
+        int t = 0;
+        for (int tile = blockIdx.x; tile < ntiles && !s_abort; tile += gridDim.x, t++) {
+            const GTile T = tile_of(tile);
+            const uint32_t idesc = g_idesc(T.bn, C::kMmaF16);
+            const int buf = t & 1;
+            const uint32_t d = tmem + buf * 128;
+            if (t >= 2 && !g_wait_w(g_smem(&acc_empty[buf]), ((t >> 1) - 1) & 1, &s_abort)) { fail(); break; }
+            g_fence_after();
+            bool ok = true;
+            for (int kb = 0; kb < KB; kb++) {
+                const int sb = bc % C::kBStages;           // 4-bit formats: also the A stage
+                if (!g_wait_w(g_smem(&b_full[sb]), (bc / C::kBStages) & 1, &s_abort)) { ok = false; break; }
+                const int sp = pc % C::kPkStages;
+                if (C::kTmemA) {
+                    if (!g_wait_w(g_smem(&a_full[sb]), (bc / C::kAStages) & 1, &s_abort)) { ok = false; break; }
+                } else {
+                    if (!g_wait_w(g_smem(&pk_full[sp]), (pc / C::kPkStages) & 1, &s_abort)) { ok = false; break; }
+                }
                 g_fence_after();
-                bool ok = true;
-                for (int kb = 0; kb < KB; kb++) {
-                    const int sb = bc % C::kBStages;
-                    if (!g_wait(g_smem(&b_full[sb]), (bc / C::kBStages) & 1, &s_abort)) { ok = false; break; }
-                    int sa = 0, sp = 0;
-                    if (C::kTmemA) {
-                        sa = ac % C::kAStages;
-                        if (!g_wait(g_smem(&a_full[sa]), (ac / C::kAStages) & 1, &s_abort)) { ok = false; break; }
-                    } else {
-                        sp = pc % C::kPkStages;
-                        if (!g_wait(g_smem(&pk_full[sp]), (pc / C::kPkStages) & 1, &s_abort)) { ok = false; break; }
-                    }
-                    g_fence_after();
-                    const uint32_t b0 = g_smem(bring + sb * C::kBStageBytes);
+                const uint32_t b0 = g_smem(bring + sb * C::kBStageBytes);
+                const uint32_t at = tmem + 256 + sb * C::kAStageCols;
+                const uint32_t a0 = g_smem(pk + sp * C::kPkStageBytes);
+                if (g_elect()) {
 #pragma unroll
                     for (int ks = 0; ks < G_BK / 16; ks++) {
                         const uint32_t acc = (kb > 0 || ks > 0) ? 1u : 0u;
                         const uint64_t bd = g_desc(b0 + ks * 32);
                         if (C::kTmemA) {
-                            const uint32_t at = tmem + 256 + sa * C::kAStageCols + ks * 8;
-                            g_mma_ts(d, at, bd, idesc, acc);
-                            if (GU) g_mma_ts(d + C::kUpCol, at + 32, bd, idesc, acc);
+                            g_mma_ts(d, at + ks * 8, bd, idesc, acc);
+                            if (GU) g_mma_ts(d + C::kUpCol, at + 32 + ks * 8, bd, idesc, acc);
                         } else {
-                            const uint32_t a0 = g_smem(pk + sp * C::kPkStageBytes);
                             g_mma_ss(d, g_desc(a0 + ks * 32), bd, idesc, acc);
                             if (GU) g_mma_ss(d + C::kUpCol, g_desc(a0 + C::kMatBytes + ks * 32), bd, idesc, acc);
                         }
                     }
-                    g_commit(g_smem(&b_empty[sb]));
-                    if (C::kTmemA) g_commit(g_smem(&a_empty[sa]));
-                    else g_commit(g_smem(&pk_empty[sp]));
-                    bc++;
-                    if (C::kTmemA) ac++; else pc++;
+                    if (C::kTmemA) {
+                        g_commit(g_smem(&a_empty[sb]));            // frees A stage sb and B stage sb
+                    } else {
+                        g_commit(g_smem(&b_empty[sb]));
+                        g_commit(g_smem(&pk_empty[sp]));
+                    }
                 }
-                if (!ok) { fail(); break; }
-                g_commit(g_smem(&acc_full[buf]));
+                __syncwarp();
+                bc++;
+                if (!C::kTmemA) pc++;
             }
-            // drain: every MMA this thread issued has completed
-            g_commit(g_smem(&drain));
-            g_drain_wait(g_smem(&drain), 0);
+            if (!ok) { fail(); break; }
+            if (g_elect()) g_commit(g_smem(&acc_full[buf]));
+            __syncwarp();
         }
+        // drain: every MMA issued has completed
+        if (g_elect()) g_commit(g_smem(&drain));
+        __syncwarp();
+        if (lane == 0) g_drain_wait(g_smem(&drain), 0);
+        __syncwarp();
     } else if (warp >= 4 && warp < 8) {
         // ---------------- epilogue ----------------
         const int q = warp & 3;
