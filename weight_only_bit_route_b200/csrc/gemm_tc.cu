@@ -16,16 +16,21 @@
 // expert_offsets.
 //
 // Warp roles inside a CTA (16 warps):
-//   warp 0      TMA producer of the weight stream: per stage, one 2D tensor
-//               copy of 128 rows x 128 bytes of packed weights (K = 256 for
-//               4-bit formats, K = 64 for BF16) per matrix, 128-byte
-//               swizzled, plus the NVFP4 block scales of those rows.  int4
-//               scales are one bulk copy per tile, since all groups of the
-//               tile's rows are contiguous.
-//   warp 1      TMA producer of the activation operand: 16-row boxes of the
-//               tile's rows (K = 64 per stage), 128-byte swizzled.  That is
-//               the K-major layout the MMA descriptors read.
-//   warp 2      allocates tensor memory and issues tcgen05.mma from one thread.
+//   warp 0      TMA producer of the weight stream: per stage, 2D tensor
+//               copies of 128 rows x 128 bytes (K = 256 of packed 4-bit
+//               weights, or K = 64 of BF16) per matrix, 128-byte swizzled,
+//               plus the NVFP4 block scales of those rows.  int4 scales are
+//               one bulk copy per tile, since all groups of the tile's rows
+//               are contiguous.
+//   warp 1      TMA producer of the activation operand: per K = 128 stage, two
+//               boxes of the tile's rows x 64 elements, 128-byte swizzled (the
+//               K-major layout the MMA descriptors read); the box height comes
+//               from one of several tensor maps, matching the tile's rows.
+//   warp 2      allocates tensor memory and issues tcgen05.mma from one lane.
+// The three single-issue roles run warp-uniform loops and elect one lane to
+// issue, which keeps the instruction operands in uniform registers.  The MMA
+// pipeline steps in K = 128: a tcgen05.commit costs about as much issue time
+// as several MMAs, so it is paid once per 16 (gate/up) or 8 (down) MMAs.
 //   warps 4-7   epilogue: tcgen05.ld of the accumulators, SwiGLU or the
 //               routing weight, bf16 stores.  Warp w reads TMEM lanes
 //               32*(w%4) to 32*(w%4)+31.
@@ -38,8 +43,9 @@
 // BF16 weights (the shared expert) need no dequantisation: the MMA reads the
 // TMA-staged weight tile from shared memory directly.
 //
-// Tensor memory (512 columns): accumulators in [0, 256) (for gate/up, gate at
-// 0 and up at 128), A stages in [256, 512).
+// Tensor memory (512 columns): two accumulator buffers in [0, 256), so the
+// epilogue of one tile overlaps the main loop of the next (buffer b at
+// 128*b; gate/up keeps gate at +0 and up at +64), A stages in [256, 512).
 //
 // int4 pairs: one mask turns the nibbles (j, j+4) of a packed word into one
 // bf16 pair, so the A operand holds the K elements of each group of 8 in the
@@ -63,7 +69,6 @@
 namespace moe {
 
 constexpr int G_BM = 128;
-constexpr int G_BK = 64;
 constexpr int G_THREADS = 512;
 constexpr int G_DQ_WARPS = 8;
 constexpr int G_EPI_WARPS = 4;
@@ -75,29 +80,26 @@ struct GCfg {
     static constexpr int kNMat = GU ? 2 : 1;
     static constexpr int kNMax = GU ? 64 : 128;                    // token rows per tile
     static constexpr int kUpCol = 64;                               // up accumulator within a buffer
-    static constexpr int kPkK = kTmemA ? 256 : 64;                  // K per weight stage
-    static constexpr int kPkX = kTmemA ? 128 : 64;                  // its width in tensor-map elements
-    static constexpr int kMatBytes = G_BM * 128;                    // one matrix per stage: 16 KB
+    static constexpr int kSK = 128;                                 // K per MMA stage
+    static constexpr int kPkK = kTmemA ? 256 : 128;                 // K per weight stage
+    static constexpr int kMatBytes = kTmemA ? G_BM * 128 : G_BM * 256;   // one matrix of a weight stage
     static constexpr int kNvScBytes = FMT == MOE_FMT_NVFP4 ? G_BM * 16 : 0;
     static constexpr int kPkStageBytes = kNMat * (kMatBytes + kNvScBytes);
-    static constexpr int kPkStages = 4;
-    static constexpr int kAStagesT = 256 / (kNMat * 32);
-    // 4-bit formats: the activation ring runs in step with the A ring, so one
-    // commit per K block frees both; BF16 keeps its own deeper ring.
-    static constexpr int kBStages = kTmemA ? kAStagesT : (GU ? 8 : 6);
-    static constexpr int kBStageBytes = kNMax * 128;
-    static constexpr int kAStageCols = kNMat * 32;                  // K = 64 as 16-bit pairs, per matrix
+    static constexpr int kPkStages = kTmemA ? ((GU && FMT == MOE_FMT_INT4_G128) ? 3 : 4) : 2;
+    static constexpr int kBAtom = kNMax * 128;                      // one 64-wide K half of a B stage
+    static constexpr int kBStageBytes = 2 * kBAtom;
+    static constexpr int kBStages = 4;
+    static constexpr int kAStageCols = kNMat * 64;                  // K = 128 as 16-bit pairs, per matrix
     static constexpr int kAStages = 256 / kAStageCols;
-    // gate/up: every dequantisation warp writes its matrix of every A stage;
-    // down: the four warps of one parity write the stages of their K blocks
-    static constexpr int kAFullCount = GU ? G_DQ_WARPS : G_DQ_WARPS / 2;
     static constexpr bool kMmaF16 = FMT == MOE_FMT_NVFP4;
 };
+
+constexpr int G_NB_MAPS = 8;                                        // box heights 16, 32, ..., 128
 
 struct GArgs {
     CUtensorMap tm_p0, tm_p1;        // packed (or BF16) weights of gate (or down) and up
     CUtensorMap tm_s0, tm_s1;        // NVFP4 block scales
-    CUtensorMap tm_b;                // activation operand rows
+    CUtensorMap tm_b[G_NB_MAPS];     // activation operand rows, box height 16*(i+1)
     const uint8_t* sc0;              // int4 scales (bf16), bulk-copied per tile
     const uint8_t* sc1;
     const float* g0;                 // NVFP4 per-expert global scales
@@ -264,6 +266,14 @@ struct GTile { int e, m0, n0, nval, bn, ebase; };
 // ---------------------------------------------------------------------------
 // Kernel
 // ---------------------------------------------------------------------------
+template <int I, int N, class F>
+__device__ __forceinline__ void g_static_for(F&& f) {
+    if constexpr (I < N) {
+        f(std::integral_constant<int, I>{});
+        g_static_for<I + 1, N>(f);
+    }
+}
+
 template <int FMT, bool GU>
 __global__ void __launch_bounds__(G_THREADS, 1) tc_grouped_gemm(const __grid_constant__ GArgs a) {
     using C = GCfg<FMT, GU>;
@@ -283,8 +293,8 @@ __global__ void __launch_bounds__(G_THREADS, 1) tc_grouped_gemm(const __grid_con
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int MT = a.out_dim / G_BM;
     const int in_dim = a.in_dim;
-    const int KB = in_dim / G_BK;
-    const int NPS = in_dim / C::kPkK;
+    const int KS = in_dim / C::kSK;                                 // MMA stages per tile
+    const int NPS = in_dim / C::kPkK;                               // weight stages per tile
     const int ngroups = in_dim / 128;
     const uint32_t sc_mat_bytes = uint32_t(G_BM * ngroups * 2);
 
@@ -299,7 +309,7 @@ __global__ void __launch_bounds__(G_THREADS, 1) tc_grouped_gemm(const __grid_con
             asm volatile("mbarrier.init.shared::cta.b64 [%0], 1;" ::"r"(g_smem(&b_empty[s])));
         }
         for (int s = 0; s < C::kAStages; s++) {
-            asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(g_smem(&a_full[s])), "r"(C::kAFullCount));
+            asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(g_smem(&a_full[s])), "r"(G_DQ_WARPS));
             asm volatile("mbarrier.init.shared::cta.b64 [%0], 1;" ::"r"(g_smem(&a_empty[s])));
         }
         for (int s = 0; s < 2; s++) {
@@ -385,7 +395,6 @@ __global__ void __launch_bounds__(G_THREADS, 1) tc_grouped_gemm(const __grid_con
         s_abort = 1;
     };
 
-    static_assert(!C::kTmemA || C::kBStages == C::kAStages, "A and B rings must step together");
     if (warp == 0) {
         // ---------------- weight producer (whole warp, one lane issues) ----------------
         uint32_t pc = 0;
@@ -418,12 +427,22 @@ __global__ void __launch_bounds__(G_THREADS, 1) tc_grouped_gemm(const __grid_con
                 const uint32_t st = g_smem(pk + s * C::kPkStageBytes);
                 if (g_elect()) {
                     g_expect(bar, C::kPkStageBytes);
-                    g_tma2d(st, &a.tm_p0, ps * C::kPkX, row0, bar);
-                    if (GU) g_tma2d(st + C::kMatBytes, &a.tm_p1, ps * C::kPkX, row0, bar);
-                    if (FMT == MOE_FMT_NVFP4) {
-                        const uint32_t ss = st + C::kNMat * C::kMatBytes;
-                        g_tma2d(ss, &a.tm_s0, ps * 16, row0, bar);
-                        if (GU) g_tma2d(ss + C::kNvScBytes, &a.tm_s1, ps * 16, row0, bar);
+                    if (C::kTmemA) {
+                        // 4-bit: 128 bytes of each row = K 256
+                        g_tma2d(st, &a.tm_p0, ps * 128, row0, bar);
+                        if (GU) g_tma2d(st + C::kMatBytes, &a.tm_p1, ps * 128, row0, bar);
+                        if (FMT == MOE_FMT_NVFP4) {
+                            const uint32_t ss = st + C::kNMat * C::kMatBytes;
+                            g_tma2d(ss, &a.tm_s0, ps * 16, row0, bar);
+                            if (GU) g_tma2d(ss + C::kNvScBytes, &a.tm_s1, ps * 16, row0, bar);
+                        }
+                    } else {
+                        // BF16: two 64-element halves of K 128 per matrix
+#pragma unroll
+                        for (int h = 0; h < 2; h++) {
+                            g_tma2d(st + h * (G_BM * 128), &a.tm_p0, ps * 128 + h * 64, row0, bar);
+                            if (GU) g_tma2d(st + C::kMatBytes + h * (G_BM * 128), &a.tm_p1, ps * 128 + h * 64, row0, bar);
+                        }
                     }
                 }
                 __syncwarp();
@@ -440,26 +459,25 @@ __global__ void __launch_bounds__(G_THREADS, 1) tc_grouped_gemm(const __grid_con
         __syncwarp();
     } else if (warp == 1) {
         // ---------------- activation producer (whole warp, one lane issues) ----------------
-        // 4-bit formats: a B stage is free once the MMAs of its K block are done,
-        // which the A-ring "empty" barrier of the same index records.
         uint32_t bc = 0;
         for (int tile = blockIdx.x; tile < ntiles && !s_abort; tile += gridDim.x) {
             const GTile T = tile_of(tile);
             const int row0 = T.ebase + T.n0;
-            const int nbox = T.bn / 16;
+            const CUtensorMap* map = &a.tm_b[T.bn / 16 - 1];
             bool ok = true;
-            for (int kb = 0; kb < KB; kb++, bc++) {
+            for (int ks = 0; ks < KS; ks++, bc++) {
                 const int s = bc % C::kBStages;
-                const uint32_t empty = C::kTmemA ? g_smem(&a_empty[s]) : g_smem(&b_empty[s]);
-                if (bc >= uint32_t(C::kBStages) && !g_wait_w(empty, ((bc / C::kBStages) - 1) & 1, &s_abort, 32)) {
+                if (bc >= uint32_t(C::kBStages) &&
+                    !g_wait_w(g_smem(&b_empty[s]), ((bc / C::kBStages) - 1) & 1, &s_abort, 32)) {
                     ok = false;
                     break;
                 }
                 const uint32_t bar = g_smem(&b_full[s]);
                 const uint32_t st = g_smem(bring + s * C::kBStageBytes);
                 if (g_elect()) {
-                    g_expect(bar, uint32_t(nbox) * 2048u);
-                    for (int j = 0; j < nbox; j++) g_tma2d(st + j * 2048, &a.tm_b, kb * G_BK, row0 + 16 * j, bar);
+                    g_expect(bar, uint32_t(T.bn) * 256u);
+                    g_tma2d(st, map, ks * C::kSK, row0, bar);
+                    g_tma2d(st + C::kBAtom, map, ks * C::kSK + 64, row0, bar);
                 }
                 __syncwarp();
             }
@@ -472,7 +490,7 @@ __global__ void __launch_bounds__(G_THREADS, 1) tc_grouped_gemm(const __grid_con
         __syncwarp();
     } else if (warp == 2) {
         // ---------------- MMA issuer (whole warp, one lane issues) ----------------
-        uint32_t bc = 0, pc = 0;
+        uint32_t bc = 0, ac = 0, pc = 0;
         int t = 0;
         for (int tile = blockIdx.x; tile < ntiles && !s_abort; tile += gridDim.x, t++) {
             const GTile T = tile_of(tile);
@@ -482,42 +500,38 @@ __global__ void __launch_bounds__(G_THREADS, 1) tc_grouped_gemm(const __grid_con
             if (t >= 2 && !g_wait_w(g_smem(&acc_empty[buf]), ((t >> 1) - 1) & 1, &s_abort)) { fail(); break; }
             g_fence_after();
             bool ok = true;
-            for (int kb = 0; kb < KB; kb++) {
-                const int sb = bc % C::kBStages;           // 4-bit formats: also the A stage
+            for (int ks = 0; ks < KS; ks++) {
+                const int sb = bc % C::kBStages, sa = ac % C::kAStages, sp = pc % C::kPkStages;
                 if (!g_wait_w(g_smem(&b_full[sb]), (bc / C::kBStages) & 1, &s_abort)) { ok = false; break; }
-                const int sp = pc % C::kPkStages;
                 if (C::kTmemA) {
-                    if (!g_wait_w(g_smem(&a_full[sb]), (bc / C::kAStages) & 1, &s_abort)) { ok = false; break; }
+                    if (!g_wait_w(g_smem(&a_full[sa]), (ac / C::kAStages) & 1, &s_abort)) { ok = false; break; }
                 } else {
                     if (!g_wait_w(g_smem(&pk_full[sp]), (pc / C::kPkStages) & 1, &s_abort)) { ok = false; break; }
                 }
                 g_fence_after();
                 const uint32_t b0 = g_smem(bring + sb * C::kBStageBytes);
-                const uint32_t at = tmem + 256 + sb * C::kAStageCols;
+                const uint32_t at = tmem + 256 + sa * C::kAStageCols;
                 const uint32_t a0 = g_smem(pk + sp * C::kPkStageBytes);
                 if (g_elect()) {
 #pragma unroll
-                    for (int ks = 0; ks < G_BK / 16; ks++) {
-                        const uint32_t acc = (kb > 0 || ks > 0) ? 1u : 0u;
-                        const uint64_t bd = g_desc(b0 + ks * 32);
+                    for (int k = 0; k < C::kSK / 16; k++) {
+                        const uint32_t acc = (ks > 0 || k > 0) ? 1u : 0u;
+                        const uint64_t bd = g_desc(b0 + (k >> 2) * C::kBAtom + (k & 3) * 32);
                         if (C::kTmemA) {
-                            g_mma_ts(d, at + ks * 8, bd, idesc, acc);
-                            if (GU) g_mma_ts(d + C::kUpCol, at + 32 + ks * 8, bd, idesc, acc);
+                            g_mma_ts(d, at + k * 8, bd, idesc, acc);
+                            if (GU) g_mma_ts(d + C::kUpCol, at + 64 + k * 8, bd, idesc, acc);
                         } else {
-                            g_mma_ss(d, g_desc(a0 + ks * 32), bd, idesc, acc);
-                            if (GU) g_mma_ss(d + C::kUpCol, g_desc(a0 + C::kMatBytes + ks * 32), bd, idesc, acc);
+                            const uint32_t ak = a0 + (k >> 2) * (G_BM * 128) + (k & 3) * 32;
+                            g_mma_ss(d, g_desc(ak), bd, idesc, acc);
+                            if (GU) g_mma_ss(d + C::kUpCol, g_desc(ak + C::kMatBytes), bd, idesc, acc);
                         }
                     }
-                    if (C::kTmemA) {
-                        g_commit(g_smem(&a_empty[sb]));            // frees A stage sb and B stage sb
-                    } else {
-                        g_commit(g_smem(&b_empty[sb]));
-                        g_commit(g_smem(&pk_empty[sp]));
-                    }
+                    g_commit(g_smem(&b_empty[sb]));
+                    g_commit(C::kTmemA ? g_smem(&a_empty[sa]) : g_smem(&pk_empty[sp]));
                 }
                 __syncwarp();
                 bc++;
-                if (!C::kTmemA) pc++;
+                if (C::kTmemA) ac++; else pc++;
             }
             if (!ok) { fail(); break; }
             if (g_elect()) g_commit(g_smem(&acc_full[buf]));
@@ -578,15 +592,17 @@ __global__ void __launch_bounds__(G_THREADS, 1) tc_grouped_gemm(const __grid_con
         }
     } else if (warp >= 8 && C::kTmemA) {
         // ---------------- dequantisation ----------------
-        // gate/up: this warp fills matrix hsel of every A stage (all four K
-        // blocks of a weight stage); down: it fills the K blocks of parity
-        // hsel.  Each K block is two 16-byte chunks of this thread's row.
-        // The next K block is dequantised while the tensor-memory store of
-        // the current one completes.
-        constexpr int kMine = GU ? 4 : 2;
+        // A weight stage (K = 256) holds two A stages (K = 128).  gate/up: this
+        // warp writes matrix hsel of both (4 chunks of 16 bytes per A stage);
+        // down: it writes K half hsel of both (2 chunks per A stage).  Chunks
+        // are software-pipelined: the next one is dequantised while the
+        // tensor-memory store of the current one is in flight.
+        constexpr int kPer = GU ? 4 : 2;               // my chunks per A stage
+        constexpr int kChunks = 2 * kPer;              // per weight stage
         const int q = warp & 3, hsel = (warp - 8) >> 2;
-        const int r = q * 32 + lane;                                 // weight row within the tile
+        const int r = q * 32 + lane;                   // weight row within the tile
         const uint32_t lane_addr = uint32_t(q * 32) << 16;
+        const uint32_t colw = 256 + (GU ? hsel * 64 : hsel * 32);
         uint32_t pc = 0;
         int t = 0;
         bool ok = true;
@@ -605,54 +621,47 @@ __global__ void __launch_bounds__(G_THREADS, 1) tc_grouped_gemm(const __grid_con
                 uint32_t scw = 0;                      // int4: bf16 scales of groups 2ps (low) and 2ps+1 (high)
                 uint4 nsc = make_uint4(0, 0, 0, 0);    // NVFP4: the 16 E4M3 scales of this row and stage
                 if (FMT == MOE_FMT_INT4_G128) scw = *reinterpret_cast<const uint32_t*>(scrow + ps * 4);
-                else if (FMT == MOE_FMT_NVFP4)
-                    nsc = *reinterpret_cast<const uint4*>(st + C::kNMat * C::kMatBytes + (GU ? hsel * C::kNvScBytes : 0) +
-                                                          r * 16);
+                else nsc = *reinterpret_cast<const uint4*>(st + C::kNMat * C::kMatBytes + (GU ? hsel * C::kNvScBytes : 0) +
+                                                           r * 16);
                 const uint32_t nscw[4] = {nsc.x, nsc.y, nsc.z, nsc.w};
-                uint32_t o[2][2][16];
-                // dequantise my i-th K block of this stage into o[buf]
-                auto produce = [&](auto ic, auto bc) {
-                    constexpr int i = decltype(ic)::value, buf = decltype(bc)::value;
-                    const int sub = GU ? i : hsel + 2 * i;
-#pragma unroll
-                    for (int h = 0; h < 2; h++) {
-                        const uint4 w = *reinterpret_cast<const uint4*>(wt + g_swz(r, 2 * sub + h));
-                        if (FMT == MOE_FMT_INT4_G128) {
-                            g_dq_int4(w, scw >> (16 * (GU ? (i >> 1) : i)), o[buf][h]);
-                        } else {
-                            const uint32_t sw = GU ? nscw[i] : (hsel ? nscw[2 * i + 1] : nscw[2 * i]);
-                            g_dq_nvfp4(w, sw >> (16 * h), o[buf][h]);
+                uint32_t o[2][16];
+                // chunk index (16 bytes of this row in the weight stage) of my i-th chunk
+                auto dq = [&](auto ic) {
+                    constexpr int i = decltype(ic)::value, j = i / kPer, l = i % kPer;
+                    const int c = 4 * j + (GU ? l : 2 * hsel + l);
+                    const uint4 w = *reinterpret_cast<const uint4*>(wt + g_swz(r, c));
+                    if (FMT == MOE_FMT_INT4_G128) {
+                        g_dq_int4(w, scw >> (16 * j), o[i & 1]);
+                    } else {
+                        // the two E4M3 scales of chunk c are bytes 2c and 2c+1
+                        const uint32_t sw = GU ? nscw[2 * j + (l >> 1)] : (hsel ? nscw[2 * j + 1] : nscw[2 * j]);
+                        g_dq_nvfp4(w, sw >> (16 * (GU ? (l & 1) : l)), o[i & 1]);
+                    }
+                };
+                int sa = 0;
+                dq(std::integral_constant<int, 0>{});
+                g_static_for<0, kChunks>([&](auto ic) {
+                    constexpr int i = decltype(ic)::value, j = i / kPer, l = i % kPer;
+                    if (!ok) return;
+                    if (l == 0) {
+                        const uint32_t acn = pc * 2 + j;             // A stage index in this CTA's stream
+                        sa = acn % C::kAStages;
+                        if (acn >= uint32_t(C::kAStages) &&
+                            !g_wait(g_smem(&a_empty[sa]), ((acn / C::kAStages) - 1) & 1, &s_abort)) {
+                            ok = false;
+                            return;
                         }
+                        g_fence_after();
                     }
-                };
-                auto publish = [&](auto ic, auto bc) {
-                    constexpr int i = decltype(ic)::value, buf = decltype(bc)::value;
-                    const int sub = GU ? i : hsel + 2 * i;
-                    const uint32_t kbg = pc * 4 + sub;                  // K block index in this CTA's stream
-                    const int sa = kbg % C::kAStages;
-                    if (kbg >= uint32_t(C::kAStages) &&
-                        !g_wait(g_smem(&a_empty[sa]), ((kbg / C::kAStages) - 1) & 1, &s_abort)) {
-                        ok = false;
-                        return;
+                    g_st16(tmem + lane_addr + colw + sa * C::kAStageCols + l * 16, o[i & 1]);
+                    if constexpr (i + 1 < kChunks) dq(std::integral_constant<int, i + 1>{});
+                    if (l == kPer - 1) {
+                        g_st_wait();
+                        g_fence_before();
+                        __syncwarp();
+                        if (lane == 0) g_arrive(g_smem(&a_full[sa]));
                     }
-                    g_fence_after();
-                    const uint32_t col = 256 + sa * C::kAStageCols + (GU ? hsel * 32 : 0);
-                    g_st16(tmem + lane_addr + col, o[buf][0]);
-                    g_st16(tmem + lane_addr + col + 16, o[buf][1]);
-                    if constexpr (i + 1 < kMine) produce(std::integral_constant<int, i + 1>{},
-                                                         std::integral_constant<int, buf ^ 1>{});
-                    g_st_wait();
-                    g_fence_before();
-                    __syncwarp();
-                    if (lane == 0) g_arrive(g_smem(&a_full[sa]));
-                };
-                produce(std::integral_constant<int, 0>{}, std::integral_constant<int, 0>{});
-                publish(std::integral_constant<int, 0>{}, std::integral_constant<int, 0>{});
-                if (ok) publish(std::integral_constant<int, 1>{}, std::integral_constant<int, 1>{});
-                if constexpr (kMine == 4) {
-                    if (ok) publish(std::integral_constant<int, 2>{}, std::integral_constant<int, 0>{});
-                    if (ok) publish(std::integral_constant<int, 3>{}, std::integral_constant<int, 1>{});
-                }
+                });
                 __syncwarp();
                 if (lane == 0) g_arrive(g_smem(&pk_empty[s]));
             }
@@ -826,7 +835,8 @@ int launch_grouped_gemm(const GemvProblem& p, bool gateup, int rows, const GemmB
         G_TRY(g_map(&a.tm_s0, false, p.s0, in / 16, wrows, uint64_t(in) / 16, 16, 128, false));
         if (gateup) G_TRY(g_map(&a.tm_s1, false, p.s1, in / 16, wrows, uint64_t(in) / 16, 16, 128, false));
     }
-    G_TRY(g_map(&a.tm_b, true, bsrc, in, uint64_t(rows), uint64_t(in) * 2, 64, 16, true));
+    for (int i = 0; i < G_NB_MAPS; i++)
+        G_TRY(g_map(&a.tm_b[i], true, bsrc, in, uint64_t(rows), uint64_t(in) * 2, 64, uint32_t(16 * (i + 1)), true));
     a.sc0 = reinterpret_cast<const uint8_t*>(p.s0);
     a.sc1 = reinterpret_cast<const uint8_t*>(p.s1);
     a.g0 = p.g0;
