@@ -126,7 +126,11 @@ const char* moe_status_string(int status);
  *   lower expert id, listed by descending s; topk_w = s / sum(selected s).
  * x: bf16 [T, H]; router_w: fp32 [E, H]; router_bias: fp32 [E] or NULL;
  * topk_ids: int32 [T, top_k] (out); topk_w: fp32 [T, top_k] (out).
- * ws: at least 256 + 4*T*E bytes. */
+ * From 64 tokens the logits run on the tensor cores: router_w is split into
+ * three bf16 planes (hi + mid + lo) whose bf16 x bf16 products are exact in
+ * fp32, accumulated in fp32.
+ * ws (256-byte aligned): at least 256 + a(4*T*E) + a(6*E*H) bytes, a()
+ * rounding up to a multiple of 256. */
 int moe_route_topk(const void* x, int T, int H, const float* router_w,
                    const float* router_bias, int E, int top_k, int32_t* topk_ids,
                    float* topk_w, void* ws, size_t ws_bytes, moe_stream_t stream);

@@ -99,7 +99,7 @@ def test_quantize_nvfp4_golden_block():
 # router
 # ---------------------------------------------------------------------------
 
-@pytest.mark.parametrize("cfg,T", [(0, 16), (1, 8), (1, 1), (0, 37), (4, 300)])
+@pytest.mark.parametrize("cfg,T", [(0, 16), (1, 8), (1, 1), (0, 37), (0, 100), (4, 300), (3, 2048)])
 def test_route_topk(cfg, T):
     wl = syn.WORKLOADS[cfg]
     x = syn.gen_x(wl, T=T)
@@ -168,7 +168,8 @@ def _tiny(fmt, T):
     return syn.Workload(f"tiny_{fmt}_T{T}", T, base.H, base.E, base.F, base.k, fmt, False, base.router_std, False)
 
 
-# T = 16 gives 128 rows (streaming GEMV); T = 96 gives 768 rows (tcgen05 GEMM)
+# T = 16 gives 128 rows (streaming GEMV); T = 96 gives 768 rows (tcgen05 GEMM).
+# The router takes the tensor-core path from 64 tokens (T = 100, 300, 2048 above).
 @pytest.mark.parametrize("fmt,T", [("int4", 16), ("nvfp4", 16), ("int4", 96), ("nvfp4", 96)])
 def test_grouped_swiglu(fmt, T):
     wl = _tiny(fmt, T)

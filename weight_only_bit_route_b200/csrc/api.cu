@@ -117,7 +117,7 @@ int layer_run(const void* x, int T, const moe_layer* L, void* y, void* ws, cudaS
         MOE_TRY(launch_route_decode(ra, s));
     } else {
         MOE_TRY(launch_route(xb, T, H, L->router_w, L->router_bias, E, k, ids, tw, at<float>(ws, W.logits),
-                             status, counter, s));
+                             at<__nv_bfloat16>(ws, W.wsplit), status, counter, s));
         MOE_TRY(launch_permute(ids, T, k, E, offsets, row_slot, slot_row, at<int32_t>(ws, W.hist), status, s));
         if (has_sh) MOE_TRY(launch_shared_routing(T, k, sh_off, sh_rs, s));
     }
@@ -218,9 +218,10 @@ int moe_route_topk(const void* x, int T, int H, const float* router_w, const flo
     if (H % 128 || E > kMaxE || top_k > kMaxTopK || top_k > E) return MOE_ERR_UNSUPPORTED;
     if (T == 0) return MOE_OK;
     if (!x || !router_w || !topk_ids || !topk_w || !al16(x) || !al16(router_w)) return MOE_ERR_INVALID_ARG;
-    MOE_TRY(check_ws(ws, ws_bytes, kStepScratch + route_scratch(T, E)));
+    MOE_TRY(check_ws(ws, ws_bytes, kStepScratch + route_scratch(T, E, H)));
     return launch_route(reinterpret_cast<const __nv_bfloat16*>(x), T, H, router_w, router_bias, E,
-                        top_k, topk_ids, topk_w, at<float>(ws, kStepScratch), at<int32_t>(ws, 0),
+                        top_k, topk_ids, topk_w, at<float>(ws, kStepScratch),
+                        at<__nv_bfloat16>(ws, kStepScratch + align256(size_t(T) * E * 4)), at<int32_t>(ws, 0),
                         at<int32_t>(ws, 4), cs(stream));
 }
 

@@ -22,7 +22,7 @@ constexpr int kMaxDecodeT = 64;
 //               amax (float bits), [3..] reserved.
 // ---------------------------------------------------------------------------
 struct WsLayout {
-    size_t ctrl, logits, hist, offsets, row_slot, slot_row, ids, tw;
+    size_t ctrl, logits, wsplit, hist, offsets, row_slot, slot_row, ids, tw;
     size_t sh_offsets, sh_rowslot, h_perm, y_perm, ys, tiles, prep, total;
 };
 
@@ -47,7 +47,9 @@ __device__ __forceinline__ float warp_sum(float v, int width) {
 
 // Step-level calls use the workspace as [ctrl 256 B][their own scratch].
 constexpr size_t kStepScratch = 256;
-inline size_t route_scratch(int T, int E) { return size_t(T) * E * 4; }
+// router: logits [T, E] fp32, then the three bf16 planes of the router weights
+// used by the tensor-core path (3 * E * H bf16)
+inline size_t route_scratch(int T, int E, int H) { return align256(size_t(T) * E * 4) + align256(size_t(E) * H * 6); }
 inline size_t permute_scratch(int T, int k, int E) {
     size_t R = size_t(T) * k;
     size_t nb = (R + kPermChunk - 1) / kPermChunk;
@@ -70,6 +72,7 @@ inline WsLayout ws_layout(int T, int H, int E, int F, int k) {
     size_t o = 0;
     L.ctrl = o;       o = align256(o + 256);
     L.logits = o;     o = align256(o + size_t(T) * E * 4);
+    L.wsplit = o;     o = align256(o + size_t(E) * H * 6);
     L.hist = o;       o = align256(o + nb * E * 4);
     L.offsets = o;    o = align256(o + size_t(E + 1) * 4);
     L.row_slot = o;   o = align256(o + R * 4);
@@ -91,12 +94,17 @@ inline WsLayout ws_layout(int T, int H, int E, int F, int k) {
 // Host-side launchers (defined in the .cu files).
 // ---------------------------------------------------------------------------
 constexpr int kRouterDecodeMaxT = 16;
+constexpr int kRouterTcMinT = 64;      // from this many tokens the router logits run on the tensor cores
 
 // Router: logits + sigmoid top-k.  counter: a zeroed int in the workspace
 // (enables the fused decode router for T <= kRouterDecodeMaxT), or null.
+// planes: 3 * E * H bf16 of scratch for the tensor-core logits (used when T >= 64).
 int launch_route(const __nv_bfloat16* x, int T, int H, const float* Wr, const float* bias,
-                 int E, int k, int32_t* ids, float* w, float* logits, int32_t* status,
-                 int32_t* counter, cudaStream_t s);
+                 int E, int k, int32_t* ids, float* w, float* logits, __nv_bfloat16* planes,
+                 int32_t* status, int32_t* counter, cudaStream_t s);
+// Router logits l = x Wr^T (fp32) on the tensor cores (Wr split into three bf16 planes).
+int launch_router_logits_tc(const __nv_bfloat16* x, int T, int H, const float* Wr, int E, float* logits,
+                            __nv_bfloat16* planes, int32_t* status, cudaStream_t s);
 
 struct RouterDecodeArgs {
     const __nv_bfloat16* x; int T, H; const float* Wr; const float* bias; int E, k;

@@ -347,8 +347,8 @@ int launch_route_decode(const RouterDecodeArgs& a, cudaStream_t s) {
 }
 
 int launch_route(const __nv_bfloat16* x, int T, int H, const float* Wr, const float* bias,
-                 int E, int k, int32_t* ids, float* w, float* logits, int32_t* status,
-                 int32_t* counter, cudaStream_t s) {
+                 int E, int k, int32_t* ids, float* w, float* logits, __nv_bfloat16* planes,
+                 int32_t* status, int32_t* counter, cudaStream_t s) {
     if (T <= kRouterDecodeMaxT && counter) {
         RouterDecodeArgs a{};
         a.x = x; a.T = T; a.H = H; a.Wr = Wr; a.bias = bias; a.E = E; a.k = k;
@@ -365,6 +365,9 @@ int launch_route(const __nv_bfloat16* x, int T, int H, const float* Wr, const fl
             dim3 grid((E + epb - 1) / epb, (T + 7) / 8);
             router_logits_rows<8><<<grid, block, 0, s>>>(x, T, H, Wr, E, logits);
         }
+    } else if (T >= kRouterTcMinT && planes) {
+        const int rc = launch_router_logits_tc(x, T, H, Wr, E, logits, planes, status, s);
+        if (rc != MOE_OK) return rc;
     } else {
         dim3 grid((E + RT_BN - 1) / RT_BN, (T + RT_BM - 1) / RT_BM);
         router_logits_tiled<<<grid, 256, 0, s>>>(x, T, H, Wr, E, logits);
