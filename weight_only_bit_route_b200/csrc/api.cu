@@ -149,8 +149,8 @@ int layer_run(const void* x, int T, const moe_layer* L, void* y, void* ws, cudaS
     sd.p0 = L->sh_down.packed; sd.out = ys; sd.status = status;
 
     if (gemv) {
-        MOE_TRY(launch_stream_gemv(gu, has_sh ? &sg : nullptr, true, T, prep, s, false));
-        MOE_TRY(launch_stream_gemv(dn, has_sh ? &sd : nullptr, false, R, prep, s, false));
+        MOE_TRY(launch_stream_gemv(gu, has_sh ? &sg : nullptr, true, T, prep, s, true));
+        MOE_TRY(launch_stream_gemv(dn, has_sh ? &sd : nullptr, false, R, prep, s, true));
     } else {
         // gate/up: the routed activation rows are gathered into the y_perm
         // region (free until the down projection writes it); int4 writes h in

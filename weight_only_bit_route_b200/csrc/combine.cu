@@ -10,6 +10,7 @@ namespace moe {
 __global__ void __launch_bounds__(256) combine_kernel(
         const __nv_bfloat16* __restrict__ y_perm, const int32_t* __restrict__ slot_row, int T,
         int k, int H, const __nv_bfloat16* __restrict__ shared_out, __nv_bfloat16* __restrict__ y) {
+    asm volatile("griddepcontrol.wait;" ::: "memory");   // y_perm / shared_out of the previous kernels
     const int per_row = H / 8;
     const long long idx = (long long)blockIdx.x * blockDim.x + threadIdx.x;
     if (idx >= (long long)T * per_row) return;
@@ -43,7 +44,8 @@ int launch_combine(const __nv_bfloat16* y_perm, const int32_t* slot_row, int T, 
                    const __nv_bfloat16* shared_out, __nv_bfloat16* y, cudaStream_t s) {
     const long long n = (long long)T * (H / 8);
     const int blocks = int((n + 255) / 256);
-    combine_kernel<<<blocks, 256, 0, s>>>(y_perm, slot_row, T, k, H, shared_out, y);
+    if (launch_pdl(combine_kernel, dim3(blocks), dim3(256), 0, s, y_perm, slot_row, T, k, H, shared_out, y) != cudaSuccess)
+        return MOE_ERR_CUDA;
     return cudaGetLastError() == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
 }
 

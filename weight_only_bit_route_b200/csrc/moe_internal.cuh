@@ -90,6 +90,24 @@ inline WsLayout ws_layout(int T, int H, int E, int F, int k) {
     return L;
 }
 
+// Launch with programmatic dependent launch allowed: the kernel may start
+// while the previous kernel on the stream finishes, and must execute
+// griddepcontrol.wait before it reads anything that kernel wrote.
+template <typename K, typename... Args>
+inline cudaError_t launch_pdl(K kern, dim3 grid, dim3 block, size_t smem, cudaStream_t s, Args... args) {
+    cudaLaunchConfig_t cfg{};
+    cfg.gridDim = grid;
+    cfg.blockDim = block;
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = s;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    return cudaLaunchKernelEx(&cfg, kern, args...);
+}
+
 // ---------------------------------------------------------------------------
 // Host-side launchers (defined in the .cu files).
 // ---------------------------------------------------------------------------

@@ -183,16 +183,18 @@ __global__ void __launch_bounds__(256) router_topk(
 // last CTA is found with an arrival counter in the workspace (no waiting);
 // it leaves the counter at zero for the next call.
 // ---------------------------------------------------------------------------
-constexpr int RD_WARPS = 4;
-constexpr int RD_TG = 8;            // tokens per staging pass
-
-
+constexpr int RD_WARPS = 8;          // 2 experts x 4 quarters of H per CTA
+constexpr int RD_EPC = 2;            // experts per CTA
+constexpr int RD_TMAX = 16;          // tokens (kRouterDecodeMaxT)
 
 __global__ void __launch_bounds__(RD_WARPS * 32) router_decode(RouterDecodeArgs a) {
     extern __shared__ __align__(16) uint8_t rsm[];
     __shared__ int s_last;
+    __shared__ float s_part[RD_EPC][4][RD_TMAX];
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const int e = blockIdx.x * RD_WARPS + warp;
+    const int el = warp >> 2, kq = warp & 3;                 // expert of the CTA, quarter of H
+    const int e = blockIdx.x * RD_EPC + el;
+    const int hq = a.H / 4;                                  // elements per quarter (a multiple of 32)
     __nv_bfloat16* xs = reinterpret_cast<__nv_bfloat16*>(rsm);
     __shared__ __align__(8) uint64_t bar;
     const uint32_t bar_a = static_cast<uint32_t>(__cvta_generic_to_shared(&bar));
@@ -201,64 +203,78 @@ __global__ void __launch_bounds__(RD_WARPS * 32) router_decode(RouterDecodeArgs 
         asm volatile("mbarrier.init.shared::cta.b64 [%0], 1;" ::"r"(bar_a));
         asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
     }
+    asm volatile("griddepcontrol.wait;" ::: "memory");      // x may come from the previous kernel
+    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
     __syncthreads();
-    int phase = 0;
-    for (int t0 = 0; t0 < a.T; t0 += RD_TG, phase ^= 1) {
-        const int nt = min(RD_TG, a.T - t0);
-        __syncthreads();                                 // previous pass done with xs
-        if (threadIdx.x == 0) {                          // one bulk copy of nt token rows
-            const uint32_t bytes = uint32_t(nt) * a.H * 2;
-            asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(bar_a), "r"(bytes) : "memory");
-            asm volatile("cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];"
-                         ::"r"(xs_a), "l"(a.x + size_t(t0) * a.H), "r"(bytes), "r"(bar_a) : "memory");
+    if (threadIdx.x == 0) {                                  // all token rows, one bulk copy
+        const uint32_t bytes = uint32_t(a.T) * a.H * 2;
+        asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(bar_a), "r"(bytes) : "memory");
+        asm volatile("cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];"
+                     ::"r"(xs_a), "l"(a.x), "r"(bytes), "r"(bar_a) : "memory");
+    }
+    // this warp's quarter of its router row: every load issued before any math
+    const float* wq = a.Wr + size_t(e < a.E ? e : 0) * a.H + kq * hq;
+    float4 wv[8];
+    const int nq = hq / 128;                                 // float4 steps of the warp (8 at H = 4096)
+#pragma unroll
+    for (int q = 0; q < 8; q++)
+        wv[q] = (q < nq) ? __ldg(reinterpret_cast<const float4*>(wq + q * 128 + lane * 4)) : make_float4(0, 0, 0, 0);
+    {   // activations landed (bounded wait)
+        uint32_t ok = 0;
+        unsigned long long t_start, t_now;
+        asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t_start));
+        while (!ok) {
+            asm volatile("{ .reg .pred p; mbarrier.try_wait.parity.shared::cta.b64 p, [%1], 0; selp.u32 %0, 1, 0, p; }"
+                         : "=r"(ok) : "r"(bar_a) : "memory");
+            asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t_now));
+            if (!ok && t_now - t_start > 2000000000ull) { set_status(a.status, MOE_ERR_TIMEOUT); break; }
         }
-        // router row of this warp, 4 floats per lane per step, 8 steps in flight
-        float acc[RD_TG];
+    }
+    float acc[RD_TMAX];
 #pragma unroll
-        for (int t = 0; t < RD_TG; t++) acc[t] = 0.f;
-        const float* wrow = a.Wr + size_t(e < a.E ? e : 0) * a.H;
-        bool ready = false;
-        for (int h0 = 0; h0 < a.H; h0 += 8 * 128) {
-            float4 wv[8];
+    for (int t = 0; t < RD_TMAX; t++) acc[t] = 0.f;
 #pragma unroll
-            for (int q = 0; q < 8; q++) {
-                const int h = h0 + q * 128 + lane * 4;
-                wv[q] = (h < a.H) ? __ldg(reinterpret_cast<const float4*>(wrow + h)) : make_float4(0, 0, 0, 0);
-            }
-            if (!ready) {                                  // activations landed (bounded wait)
-                uint32_t ok = 0;
-                unsigned long long t_start, t_now;
-                asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t_start));
-                while (!ok) {
-                    asm volatile("{ .reg .pred p; mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2; selp.u32 %0, 1, 0, p; }"
-                                 : "=r"(ok) : "r"(bar_a), "r"(phase) : "memory");
-                    asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t_now));
-                    if (!ok && t_now - t_start > 2000000000ull) { set_status(a.status, MOE_ERR_TIMEOUT); break; }
-                }
-                ready = true;
-            }
+    for (int q = 0; q < 8; q++) {
+        if (q < nq) {
+            const int h = kq * hq + q * 128 + lane * 4;
 #pragma unroll
-            for (int q = 0; q < 8; q++) {
-                const int h = h0 + q * 128 + lane * 4;
-                if (h < a.H) {
-#pragma unroll
-                    for (int t = 0; t < RD_TG; t++) {
-                        if (t < nt) {
-                            const uint2 xv = *reinterpret_cast<const uint2*>(xs + t * a.H + h);
-                            float v = acc[t];
-                            v = fmaf(bf16_lo(xv.x), wv[q].x, v); v = fmaf(bf16_hi(xv.x), wv[q].y, v);
-                            v = fmaf(bf16_lo(xv.y), wv[q].z, v); v = fmaf(bf16_hi(xv.y), wv[q].w, v);
-                            acc[t] = v;
-                        }
-                    }
+            for (int t = 0; t < RD_TMAX; t++) {
+                if (t < a.T) {
+                    const uint2 xv = *reinterpret_cast<const uint2*>(xs + t * a.H + h);
+                    float v = acc[t];
+                    v = fmaf(bf16_lo(xv.x), wv[q].x, v); v = fmaf(bf16_hi(xv.x), wv[q].y, v);
+                    v = fmaf(bf16_lo(xv.y), wv[q].z, v); v = fmaf(bf16_hi(xv.y), wv[q].w, v);
+                    acc[t] = v;
                 }
             }
         }
+    }
+    // larger H: the rest of the quarter, 4 floats per lane per step
+    for (int h0 = 8 * 128; h0 < hq; h0 += 128) {
+        const float4 w4 = __ldg(reinterpret_cast<const float4*>(wq + h0 + lane * 4));
+        const int h = kq * hq + h0 + lane * 4;
 #pragma unroll
-        for (int t = 0; t < RD_TG; t++) {
-            const float v = warp_sum(acc[t], 32);
-            if (lane == 0 && t < nt && e < a.E) a.logits[size_t(t0 + t) * a.E + e] = v;
+        for (int t = 0; t < RD_TMAX; t++) {
+            if (t < a.T) {
+                const uint2 xv = *reinterpret_cast<const uint2*>(xs + t * a.H + h);
+                float v = acc[t];
+                v = fmaf(bf16_lo(xv.x), w4.x, v); v = fmaf(bf16_hi(xv.x), w4.y, v);
+                v = fmaf(bf16_lo(xv.y), w4.z, v); v = fmaf(bf16_hi(xv.y), w4.w, v);
+                acc[t] = v;
+            }
         }
+    }
+#pragma unroll
+    for (int t = 0; t < RD_TMAX; t++) {
+        const float v = warp_sum(acc[t], 32);
+        if (lane == 0 && t < a.T) s_part[el][kq][t] = v;
+    }
+    __syncthreads();
+    // quarters in a fixed order
+    for (int i = threadIdx.x; i < RD_EPC * a.T; i += blockDim.x) {
+        const int ee = i / a.T, t = i % a.T, eg = blockIdx.x * RD_EPC + ee;
+        if (eg < a.E)
+            a.logits[size_t(t) * a.E + eg] = ((s_part[ee][0][t] + s_part[ee][1][t]) + s_part[ee][2][t]) + s_part[ee][3][t];
     }
     // last CTA to arrive continues
     __threadfence();
@@ -335,15 +351,16 @@ __global__ void __launch_bounds__(RD_WARPS * 32) router_decode(RouterDecodeArgs 
 }
 
 int launch_route_decode(const RouterDecodeArgs& a, cudaStream_t s) {
-    const size_t smem = std::max<size_t>(size_t(RD_TG) * a.H * 2, size_t(a.E) * 4);
+    const size_t smem = std::max<size_t>(size_t(a.T) * a.H * 2, size_t(a.E) * 4);
     static size_t smem_set = 0;
     if (smem > 48 * 1024 && smem > smem_set) {
         if (cudaFuncSetAttribute(router_decode, cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem)) != cudaSuccess)
             return MOE_ERR_UNSUPPORTED;
         smem_set = smem;
     }
-    router_decode<<<(a.E + RD_WARPS - 1) / RD_WARPS, RD_WARPS * 32, smem, s>>>(a);
-    return cudaGetLastError() == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
+    if (a.T > RD_TMAX || a.H % 512) return MOE_ERR_UNSUPPORTED;
+    return launch_pdl(router_decode, dim3((a.E + RD_EPC - 1) / RD_EPC), dim3(RD_WARPS * 32), smem, s, a) == cudaSuccess
+               ? MOE_OK : MOE_ERR_CUDA;
 }
 
 int launch_route(const __nv_bfloat16* x, int T, int H, const float* Wr, const float* bias,
