@@ -168,7 +168,7 @@ def _tiny(fmt, T):
     return syn.Workload(f"tiny_{fmt}_T{T}", T, base.H, base.E, base.F, base.k, fmt, False, base.router_std, False)
 
 
-# T = 16 gives 128 rows (streaming GEMV); T = 96 gives 768 rows (tcgen05 GEMM).
+# Routed experts take the tcgen05 GEMM at every batch size (T = 16: 128 rows; T = 96: 768 rows).
 # The router takes the tensor-core path from 64 tokens (T = 100, 300, 2048 above).
 @pytest.mark.parametrize("fmt,T", [("int4", 16), ("nvfp4", 16), ("int4", 96), ("nvfp4", 96)])
 def test_grouped_swiglu(fmt, T):
@@ -203,6 +203,49 @@ def test_grouped_down(fmt, T):
     torch.cuda.synchronize()
     gf = oracle.bf16_to_f32(bf16_bits(y)).astype(np.float64)
     assert np.all(np.abs(gf - ref) <= layer_tolerance(ref))
+
+
+def _odd(fmt, T):
+    # F = 384 is a multiple of 128 but not of 256: the tcgen05 GEMM does not
+    # take the down projection (K = F), so a layer streams both routed
+    # projections through the GEMV, and so does a down step call
+    base = syn.WORKLOADS[0]
+    return syn.Workload(f"odd_{fmt}_T{T}", T, 1024, 16, 384, base.k, fmt, False, base.router_std, False)
+
+
+@pytest.mark.parametrize("fmt", ["int4", "nvfp4"])
+def test_grouped_steps_streaming_gemv(fmt):
+    wl = _odd(fmt, 12)
+    P = build(wl, "quantised")
+    off, rs, sr = oracle.permute(P.ids, wl.E)
+    R = wl.T * wl.k
+    ws = _ws(wl.T, wl)
+    g, u, d = (device_bank(moe, P.banks[w]) for w in ("gate", "up", "down"))
+    ref_h = oracle.grouped_swiglu(P.x, off, rs, wl.k, P.banks["gate"], P.banks["up"], np.arange(R))
+    h = moe.grouped_swiglu(dev_bf16(P.x), dev(off), dev(rs), wl.k, g, u, R, ws)
+    torch.cuda.synchronize()
+    hb = bf16_bits(h)
+    assert np.all(np.abs(oracle.bf16_to_f32(hb).astype(np.float64) - ref_h) <= layer_tolerance(ref_h))
+    tw = P.w.ravel()
+    ref_y = oracle.grouped_down(hb, off, rs, tw, P.banks["down"], np.arange(R))
+    y = moe.grouped_down(h, dev(off), dev(rs), dev(tw), d, ws)
+    torch.cuda.synchronize()
+    assert np.all(np.abs(oracle.bf16_to_f32(bf16_bits(y)).astype(np.float64) - ref_y) <= layer_tolerance(ref_y))
+    assert moe.read_status(ws) == 0
+
+
+@pytest.mark.parametrize("fmt", ["int4", "nvfp4"])
+def test_layer_streaming_gemv_path(fmt):
+    wl = _odd(fmt, 12)
+    P = build(wl, "quantised", shared=True)
+    L = device_layer(moe, P)
+    ws = _ws(P.T, wl)
+    x = dev_bf16(P.x)
+    y = moe.layer_decode(x, L, ws)
+    ids, _ = moe.route_topk(x, L.router_w, L.router_bias, wl.k, ws)
+    torch.cuda.synchronize()
+    assert moe.read_status(ws) == 0
+    _layer_check(P, bf16_bits(y), np.arange(P.T, dtype=np.int32), ids.cpu().numpy())
 
 
 @pytest.mark.parametrize("T", [5, 300])

@@ -48,8 +48,22 @@ int check_ws(void* ws, size_t ws_bytes, size_t need) {
         if (_rc != MOE_OK) return _rc; \
     } while (0)
 
-// decode-sized calls stream weights with the GEMV; larger ones use the GEMM
-constexpr int kGemvMaxRows = 256;
+// Routed experts run on the tcgen05 grouped GEMM whenever its shape rules
+// hold (in and out dimensions multiples of 256 and 128), at any batch size;
+// other shapes take the streaming GEMV.  The BF16 shared expert sees every
+// token, so at small T its GEMM has only a few tiles: up to kSharedGemvMaxT
+// tokens it streams through the GEMV instead.
+constexpr int kSharedGemvMaxT = 16;
+
+bool gemm_shape_ok(int in_dim, int out_dim) { return in_dim % 256 == 0 && out_dim % 128 == 0; }
+
+// The problem p (rows activation rows) on the path the rules above choose.
+int run_problem(const GemvProblem& p, bool gateup, int rows, int act_rows, void* prep, const GemmBuffers& gb,
+                cudaStream_t s) {
+    const bool shared_small = p.E == 1 && p.fmt == MOE_FMT_BF16 && rows <= kSharedGemvMaxT;
+    if (!shared_small && gemm_shape_ok(p.in_dim, p.out_dim)) return launch_grouped_gemm(p, gateup, rows, gb, s);
+    return launch_stream_gemv(p, nullptr, gateup, act_rows, prep, s, true);
+}
 
 // The tcgen05 GEMM of one problem of a step-level call: its activation
 // pre-pass goes to prep ([rows] fp32 scales, then [rows, in] 16-bit rows).
@@ -107,7 +121,7 @@ int layer_run(const void* x, int T, const moe_layer* L, void* y, void* ws, cudaS
     int32_t* sh_off = at<int32_t>(ws, W.sh_offsets);
     int32_t* sh_rs = at<int32_t>(ws, W.sh_rowslot);
     int32_t* counter = status + 1;
-    if (T <= kRouterDecodeMaxT) {
+    if (T <= kRouterDecodeMaxT && router_decode_ok(H)) {
         // router, top-k, bucketing and shared routing in one launch
         RouterDecodeArgs ra{};
         ra.x = xb; ra.T = T; ra.H = H; ra.Wr = L->router_w; ra.bias = L->router_bias; ra.E = E; ra.k = k;
@@ -124,7 +138,7 @@ int layer_run(const void* x, int T, const moe_layer* L, void* y, void* ws, cudaS
 
     void* prep = at<void>(ws, W.prep);
     __nv_bfloat16* h_sh = h_perm + size_t(R) * F;
-    const bool gemv = R <= kGemvMaxRows;
+    const bool routed_gemm = gemm_shape_ok(H, F) && gemm_shape_ok(F, H);
     const bool int4 = L->gate.fmt == MOE_FMT_INT4_G128;
 
     GemvProblem gu{};
@@ -148,27 +162,31 @@ int layer_run(const void* x, int T, const moe_layer* L, void* y, void* ws, cudaS
     sd.E = 1; sd.fmt = MOE_FMT_BF16; sd.out_dim = H; sd.in_dim = F;
     sd.p0 = L->sh_down.packed; sd.out = ys; sd.status = status;
 
-    if (gemv) {
-        MOE_TRY(launch_stream_gemv(gu, has_sh ? &sg : nullptr, true, T, prep, s, true));
-        MOE_TRY(launch_stream_gemv(dn, has_sh ? &sd : nullptr, false, R, prep, s, true));
-    } else {
-        // gate/up: the routed activation rows are gathered into the y_perm
-        // region (free until the down projection writes it); int4 writes h in
-        // the pair order the down GEMM reads.  The shared expert reads x and
-        // its own h directly (identity routing, natural order).
+    // routed experts: both projections on one path (the int4 GEMM hands h to
+    // the down GEMM in its pair order)
+    if (routed_gemm) {
+        // the gate/up activation rows are gathered into the y_perm region,
+        // free until the down projection writes it
         GemmBuffers gb{};
         gb.act_buf = y_perm; gb.scale_buf = reinterpret_cast<float*>(prep); gb.act_ready = 0; gb.perm_out = int4;
         MOE_TRY(launch_grouped_gemm(gu, true, R, gb, s));
-        GemmBuffers direct{};
-        direct.act_ready = 1;
-        if (has_sh) MOE_TRY(launch_grouped_gemm(sg, true, T, direct, s));
+    } else {
+        MOE_TRY(launch_stream_gemv(gu, nullptr, true, T, prep, s, true));
+    }
+    // the shared expert reads x and its own h directly (identity routing, natural order)
+    GemmBuffers direct{};
+    direct.act_ready = 1;
+    if (has_sh) MOE_TRY(run_problem(sg, true, T, T, nullptr, direct, s));
+    if (routed_gemm) {
         GemmBuffers db{};
         db.scale_buf = reinterpret_cast<float*>(prep);
         db.act_buf = reinterpret_cast<uint8_t*>(prep) + align256(size_t(R) * 4);
         db.act_ready = int4;
         MOE_TRY(launch_grouped_gemm(dn, false, R, db, s));
-        if (has_sh) MOE_TRY(launch_grouped_gemm(sd, false, T, direct, s));
+    } else {
+        MOE_TRY(launch_stream_gemv(dn, nullptr, false, R, prep, s, true));
     }
+    if (has_sh) MOE_TRY(run_problem(sd, false, T, T, nullptr, direct, s));
 
     return launch_combine(y_perm, slot_row, T, k, H, has_sh ? ys : nullptr,
                           reinterpret_cast<__nv_bfloat16*>(y), s);
@@ -278,8 +296,7 @@ int moe_grouped_w4a16_swiglu(const void* x, int T, int H, const int32_t* expert_
     p.p1 = up->packed; p.s1 = up->scales; p.g1 = up->global_scale;
     p.out = reinterpret_cast<__nv_bfloat16*>(h_perm); p.status = at<int32_t>(ws, 0);
     void* prep = at<void>(ws, kStepScratch + align256(size_t(E + 2) * 16));
-    if (rows <= kGemvMaxRows) return launch_stream_gemv(p, nullptr, true, T, prep, cs(stream), false);
-    return launch_grouped_gemm(p, true, rows, step_buffers(prep, rows, false), cs(stream));
+    return run_problem(p, true, rows, T, prep, step_buffers(prep, rows, false), cs(stream));
 }
 
 int moe_grouped_w4a16_down(const void* h_perm, const int32_t* expert_offsets, const int32_t* row_slot,
@@ -301,9 +318,8 @@ int moe_grouped_w4a16_down(const void* h_perm, const int32_t* expert_offsets, co
     p.p0 = down->packed; p.s0 = down->scales; p.g0 = down->global_scale;
     p.out = reinterpret_cast<__nv_bfloat16*>(y_perm); p.status = at<int32_t>(ws, 0);
     void* prep = at<void>(ws, kStepScratch + align256(size_t(E + 2) * 16));
-    if (rows <= kGemvMaxRows) return launch_stream_gemv(p, nullptr, false, rows, prep, cs(stream), false);
     // BF16 rows are read in place (row r is activation row r)
-    return launch_grouped_gemm(p, false, rows, step_buffers(prep, rows, down->fmt == MOE_FMT_BF16), cs(stream));
+    return run_problem(p, false, rows, rows, prep, step_buffers(prep, rows, down->fmt == MOE_FMT_BF16), cs(stream));
 }
 
 int moe_unpermute_combine(const void* y_perm, const int32_t* slot_row, int T, int top_k, int H,

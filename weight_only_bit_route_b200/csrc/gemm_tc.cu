@@ -647,8 +647,7 @@ static int g_launch(const GArgs& a, cudaStream_t s) {
     if (smem + fa.sharedSizeBytes > size_t(optin)) return MOE_ERR_UNSUPPORTED;
     if (cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem)) != cudaSuccess)
         return MOE_ERR_CUDA;
-    k<<<sms, G_THREADS, smem, s>>>(a);
-    return cudaGetLastError() == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
+    return launch_pdl(k, dim3(sms), dim3(G_THREADS), smem, s, a) == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
 }
 
 #define G_TRY(x)                       \
@@ -673,9 +672,9 @@ int launch_grouped_gemm(const GemvProblem& p, bool gateup, int rows, const GemmB
     if (!buf.act_ready || nv) {
         if (!buf.act_buf || (nv && !buf.scale_buf)) return MOE_ERR_WORKSPACE;
         const int mode = nv ? 2 : (i4 ? 1 : 0);
-        g_prep<<<(rows * 32 + 255) / 256, 256, 0, s>>>(p.act, in, p.row_slot, p.top_k, p.act_by_token, rows, mode,
-                                                       reinterpret_cast<uint16_t*>(buf.act_buf), buf.scale_buf);
-        if (cudaGetLastError() != cudaSuccess) return MOE_ERR_CUDA;
+        if (launch_pdl(g_prep, dim3((rows * 32 + 255) / 256), dim3(256), 0, s, p.act, in, p.row_slot, p.top_k,
+                       p.act_by_token, rows, mode, reinterpret_cast<uint16_t*>(buf.act_buf), buf.scale_buf) != cudaSuccess)
+            return MOE_ERR_CUDA;
         bsrc = buf.act_buf;
         ascale = buf.scale_buf;
     }

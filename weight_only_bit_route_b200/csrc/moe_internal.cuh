@@ -112,6 +112,8 @@ inline cudaError_t launch_pdl(K kern, dim3 grid, dim3 block, size_t smem, cudaSt
 // Host-side launchers (defined in the .cu files).
 // ---------------------------------------------------------------------------
 constexpr int kRouterDecodeMaxT = 16;
+// the fused decode router splits H into four quarters of whole 128-wide steps
+inline bool router_decode_ok(int H) { return H % 512 == 0; }
 constexpr int kRouterTcMinT = 64;      // from this many tokens the router logits run on the tensor cores
 
 // Router: logits + sigmoid top-k.  counter: a zeroed int in the workspace

@@ -366,7 +366,7 @@ int launch_route_decode(const RouterDecodeArgs& a, cudaStream_t s) {
 int launch_route(const __nv_bfloat16* x, int T, int H, const float* Wr, const float* bias,
                  int E, int k, int32_t* ids, float* w, float* logits, __nv_bfloat16* planes,
                  int32_t* status, int32_t* counter, cudaStream_t s) {
-    if (T <= kRouterDecodeMaxT && counter) {
+    if (T <= kRouterDecodeMaxT && counter && router_decode_ok(H)) {
         RouterDecodeArgs a{};
         a.x = x; a.T = T; a.H = H; a.Wr = Wr; a.bias = bias; a.E = E; a.k = k;
         a.logits = logits; a.ids = ids; a.w = w; a.counter = counter; a.status = status;

@@ -206,8 +206,7 @@ static int rt_launch(const RtArgs& a, cudaStream_t s) {
     if (cudaFuncSetAttribute(router_tc, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess)
         return MOE_ERR_CUDA;
     dim3 grid((a.E + RT_M - 1) / RT_M, (a.T + RT_BN - 1) / RT_BN);
-    router_tc<<<grid, RT_THREADS, smem, s>>>(a);
-    return cudaGetLastError() == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
+    return launch_pdl(router_tc, grid, dim3(RT_THREADS), size_t(smem), s, a) == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
 }
 
 int launch_router_logits_tc(const __nv_bfloat16* x, int T, int H, const float* Wr, int E, float* logits,
