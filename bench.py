@@ -345,12 +345,15 @@ def main():
     torch.cuda.synchronize()
     k_ms = float(np.mean([a.elapsed_time(b) for a, b in kev]))
     pk, pk_kind = peaks()
+    # DRAM bytes (read + write) of one gate/up tcgen05_grouped_gemm launch, from the ncu captures summarised
+    # under profiles/ for the current kernel; workloads without a capture report null
+    traffic = {"decode_int4_T8": 394335232, "prefill_int4_T2048": 2484627008}.get(wl.name)
     decode = T <= 64
     if decode:
         kbytes = touched * gateup_bytes_per_expert(wl) + T * wl.H * 2
         achieved = kbytes / (k_ms * 1e-3) / 1e9
         roof = {"bound": "hbm", "achieved": round(achieved, 1), "peak": pk["hbm_gbs"], "unit": "GB/s",
-                "frac": round(achieved / pk["hbm_gbs"], 4), "traffic": None,
+                "frac": round(achieved / pk["hbm_gbs"], 4), "traffic": traffic,
                 "kernel": "tc_grouped_gemm gate/up+SwiGLU (with its activation gather)", "algorithmic_bytes": kbytes,
                 "kernel_ms": round(k_ms, 5), "peak_source": f"{pk_kind} hbm_gbs"}
     else:
@@ -358,7 +361,7 @@ def main():
         achieved = kflops / (k_ms * 1e-3) / 1e12
         peak = pk["bf16_tflops"]
         roof = {"bound": "tensor", "achieved": round(achieved, 1), "peak": peak, "unit": "TFLOP/s",
-                "frac": round(achieved / peak, 4), "traffic": None,
+                "frac": round(achieved / peak, 4), "traffic": traffic,
                 "kernel": "tc_grouped_gemm gate/up+SwiGLU (with its activation gather)",
                 "algorithmic_flops": kflops, "kernel_ms": round(k_ms, 5), "peak_source": f"{pk_kind} bf16_tflops"}
 
