@@ -49,24 +49,23 @@ int check_ws(void* ws, size_t ws_bytes, size_t need) {
     } while (0)
 
 // Routed experts run on the tcgen05 grouped GEMM whenever its shape rules
-// hold (in and out dimensions multiples of 256 and 128), at any batch size;
-// other shapes take the streaming GEMV.  The BF16 shared expert sees every
-// token, so at small T its GEMM has only a few tiles: up to kSharedGemvMaxT
-// tokens it streams through the GEMV instead.
-constexpr int kSharedGemvMaxT = 16;
-
+// hold (input dimension a multiple of 256, output a multiple of 128), at any
+// batch size; other shapes take the streaming GEMV.  The BF16 shared expert at
+// a small batch splits K across tiles (shared_ksplit) so that its weight
+// stream spreads over the GPU; partial is split_bytes() of scratch for that.
 bool gemm_shape_ok(int in_dim, int out_dim) { return in_dim % 256 == 0 && out_dim % 128 == 0; }
 
-// The problem p (rows activation rows) on the path the rules above choose.
 int run_problem(const GemvProblem& p, bool gateup, int rows, int act_rows, void* prep, const GemmBuffers& gb,
-                cudaStream_t s) {
-    const bool shared_small = p.E == 1 && p.fmt == MOE_FMT_BF16 && rows <= kSharedGemvMaxT;
-    if (!shared_small && gemm_shape_ok(p.in_dim, p.out_dim)) return launch_grouped_gemm(p, gateup, rows, gb, s);
-    return launch_stream_gemv(p, nullptr, gateup, act_rows, prep, s, true);
+                float* partial, cudaStream_t s) {
+    if (!gemm_shape_ok(p.in_dim, p.out_dim)) return launch_stream_gemv(p, nullptr, gateup, act_rows, prep, s, true);
+    GemmBuffers b = gb;
+    b.ksplit = shared_ksplit(p.E, p.fmt, gateup, rows, p.in_dim);
+    b.partial = partial;
+    return launch_grouped_gemm(p, gateup, rows, b, s);
 }
 
-// The tcgen05 GEMM of one problem of a step-level call: its activation
-// pre-pass goes to prep ([rows] fp32 scales, then [rows, in] 16-bit rows).
+// The step-level calls' scratch: the GEMV or GEMM pre-pass of rows rows, then
+// the shared expert's split-K partial sums.
 GemmBuffers step_buffers(void* prep, int rows, bool act_ready) {
     GemmBuffers b{};
     b.scale_buf = reinterpret_cast<float*>(prep);
@@ -75,10 +74,13 @@ GemmBuffers step_buffers(void* prep, int rows, bool act_ready) {
     b.perm_out = 0;
     return b;
 }
+size_t step_scratch(int E, int fmt, bool gateup, int rows, int in_dim, int out_dim) {
+    return grouped_scratch(E, rows, in_dim) + split_bytes(shared_ksplit(E, fmt, gateup, rows, in_dim), gateup, rows, out_dim);
+}
+float* step_partial(void* ws, int E, int rows, int in_dim) {
+    return at<float>(ws, kStepScratch + grouped_scratch(E, rows, in_dim));
+}
 
-// Step-level scratch after the 256-byte control block: room for the GEMV
-// pre-pass of act_rows rows or the GEMM pre-pass of rows rows.
-size_t step_scratch(int E, int rows, int in_dim) { return grouped_scratch(E, rows, in_dim); }
 int layer_checks(const void* x, int T, const moe_layer* L, void* y, void* ws, size_t ws_bytes) {
     if (!L) return MOE_ERR_INVALID_ARG;
     MOE_TRY(check_dims(T, L->H, L->E, L->F, L->top_k));
@@ -176,7 +178,8 @@ int layer_run(const void* x, int T, const moe_layer* L, void* y, void* ws, cudaS
     // the shared expert reads x and its own h directly (identity routing, natural order)
     GemmBuffers direct{};
     direct.act_ready = 1;
-    if (has_sh) MOE_TRY(run_problem(sg, true, T, T, nullptr, direct, s));
+    float* shpart = at<float>(ws, W.shpart);
+    if (has_sh) MOE_TRY(run_problem(sg, true, T, T, nullptr, direct, shpart, s));
     if (routed_gemm) {
         GemmBuffers db{};
         db.scale_buf = reinterpret_cast<float*>(prep);
@@ -186,7 +189,7 @@ int layer_run(const void* x, int T, const moe_layer* L, void* y, void* ws, cudaS
     } else {
         MOE_TRY(launch_stream_gemv(dn, nullptr, false, R, prep, s, true));
     }
-    if (has_sh) MOE_TRY(run_problem(sd, false, T, T, nullptr, direct, s));
+    if (has_sh) MOE_TRY(run_problem(sd, false, T, T, nullptr, direct, shpart, s));
 
     return launch_combine(y_perm, slot_row, T, k, H, has_sh ? ys : nullptr,
                           reinterpret_cast<__nv_bfloat16*>(y), s);
@@ -287,7 +290,7 @@ int moe_grouped_w4a16_swiglu(const void* x, int T, int H, const int32_t* expert_
     if (!x || !al16(x) || !expert_offsets || !row_slot || !h_perm || !al16(h_perm)) return MOE_ERR_INVALID_ARG;
     // rows present: T * top_k routed slots, or T for a single shared expert
     const int rows = (E == 1) ? T : T * top_k;
-    MOE_TRY(check_ws(ws, ws_bytes, kStepScratch + step_scratch(E, rows, H)));
+    MOE_TRY(check_ws(ws, ws_bytes, kStepScratch + step_scratch(E, gate->fmt, true, rows, H, F)));
     GemvProblem p{};
     p.act = reinterpret_cast<const __nv_bfloat16*>(x); p.act_by_token = 1; p.top_k = top_k;
     p.offsets = expert_offsets; p.row_slot = row_slot; p.E = E; p.fmt = gate->fmt;
@@ -296,7 +299,8 @@ int moe_grouped_w4a16_swiglu(const void* x, int T, int H, const int32_t* expert_
     p.p1 = up->packed; p.s1 = up->scales; p.g1 = up->global_scale;
     p.out = reinterpret_cast<__nv_bfloat16*>(h_perm); p.status = at<int32_t>(ws, 0);
     void* prep = at<void>(ws, kStepScratch + align256(size_t(E + 2) * 16));
-    return run_problem(p, true, rows, T, prep, step_buffers(prep, rows, false), cs(stream));
+    return run_problem(p, true, rows, T, prep, step_buffers(prep, rows, false), step_partial(ws, E, rows, H),
+                       cs(stream));
 }
 
 int moe_grouped_w4a16_down(const void* h_perm, const int32_t* expert_offsets, const int32_t* row_slot,
@@ -310,7 +314,7 @@ int moe_grouped_w4a16_down(const void* h_perm, const int32_t* expert_offsets, co
     if (rows == 0) return MOE_OK;
     if (!h_perm || !al16(h_perm) || !expert_offsets || !row_slot || !y_perm || !al16(y_perm))
         return MOE_ERR_INVALID_ARG;
-    MOE_TRY(check_ws(ws, ws_bytes, kStepScratch + step_scratch(E, rows, F)));
+    MOE_TRY(check_ws(ws, ws_bytes, kStepScratch + step_scratch(E, down->fmt, false, rows, F, H)));
     GemvProblem p{};
     p.act = reinterpret_cast<const __nv_bfloat16*>(h_perm); p.act_by_token = 0; p.top_k = 1;
     p.offsets = expert_offsets; p.row_slot = row_slot; p.E = E; p.topk_w = topk_w;
@@ -319,7 +323,8 @@ int moe_grouped_w4a16_down(const void* h_perm, const int32_t* expert_offsets, co
     p.out = reinterpret_cast<__nv_bfloat16*>(y_perm); p.status = at<int32_t>(ws, 0);
     void* prep = at<void>(ws, kStepScratch + align256(size_t(E + 2) * 16));
     // BF16 rows are read in place (row r is activation row r)
-    return run_problem(p, false, rows, rows, prep, step_buffers(prep, rows, down->fmt == MOE_FMT_BF16), cs(stream));
+    return run_problem(p, false, rows, rows, prep, step_buffers(prep, rows, down->fmt == MOE_FMT_BF16),
+                       step_partial(ws, E, rows, F), cs(stream));
 }
 
 int moe_unpermute_combine(const void* y_perm, const int32_t* slot_row, int T, int top_k, int H,

@@ -58,6 +58,7 @@
 // the copies and MMAs it has in flight, frees its tensor memory and returns.
 #include <cuda_fp16.h>
 
+#include <algorithm>
 #include <cstring>
 #include <type_traits>
 
@@ -107,7 +108,9 @@ struct GArgs {
     const float* act_scale;          // NVFP4: activation row scale, by GEMM row
     __nv_bfloat16* out;
     int32_t* status;
+    float* partial;                  // split-K: fp32 partial sums [ksplit][nmat][rows][out_dim]
     int E, out_dim, in_dim, perm_out;
+    int ksplit, rows;                // K slices per (m-tile, n-tile); activation rows of the problem
 };
 
 // ---------------------------------------------------------------------------
@@ -146,7 +149,7 @@ __device__ __forceinline__ void g_dq_nvfp4(const uint4 w, uint32_t sc2, uint32_t
     }
 }
 
-struct GTile { int e, m0, n0, nval, bn, ebase; };
+struct GTile { int e, m0, n0, nval, bn, ebase, ks, kbase; };
 
 // ---------------------------------------------------------------------------
 // Kernel
@@ -178,8 +181,10 @@ __global__ void __launch_bounds__(G_THREADS, 1) tc_grouped_gemm(const __grid_con
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int MT = a.out_dim / G_BM;
     const int in_dim = a.in_dim;
-    const int KS = in_dim / C::kSK;                                 // MMA stages per tile
-    const int NPS = in_dim / C::kPkK;                               // weight stages per tile
+    const int ksplit = a.ksplit;                                    // K slices (BF16 split-K), else 1
+    const int kc = in_dim / ksplit;                                 // K of one tile
+    const int KS = kc / C::kSK;                                     // MMA stages per tile
+    const int NPS = kc / C::kPkK;                                   // weight stages per tile
     const int ngroups = in_dim / 128;
     const uint32_t sc_mat_bytes = uint32_t(G_BM * ngroups * 2);
 
@@ -222,7 +227,7 @@ __global__ void __launch_bounds__(G_THREADS, 1) tc_grouped_gemm(const __grid_con
             const int e = tid * PER + i;
             const int n = (e < a.E) ? a.offsets[e + 1] - a.offsets[e] : 0;
             cnt[i] = n > 0;
-            nt[i] = n > 0 ? ((n + C::kNMax - 1) / C::kNMax) * MT : 0;
+            nt[i] = n > 0 ? ((n + C::kNMax - 1) / C::kNMax) * MT * ksplit : 0;
             local += cnt[i];
             ltiles += nt[i];
         }
@@ -269,8 +274,11 @@ __global__ void __launch_bounds__(G_THREADS, 1) tc_grouped_gemm(const __grid_con
         const int n_e = a.offsets[t.e + 1] - t.ebase;
         const int ntile = (n_e + C::kNMax - 1) / C::kNMax;
         const int per = (n_e + ntile - 1) / ntile;                  // balanced rows per n-tile
-        t.m0 = (local / ntile) * G_BM;
-        t.n0 = (local % ntile) * per;
+        t.ks = local % ksplit;                                      // K slice fastest
+        t.kbase = t.ks * kc;
+        const int mn = local / ksplit;
+        t.m0 = (mn / ntile) * G_BM;
+        t.n0 = (mn % ntile) * per;
         t.nval = min(per, n_e - t.n0);
         t.bn = (t.nval + 15) & ~15;
         return t;
@@ -314,19 +322,20 @@ __global__ void __launch_bounds__(G_THREADS, 1) tc_grouped_gemm(const __grid_con
                     g_expect(bar, C::kPkStageBytes);
                     if (C::kTmemA) {
                         // 4-bit: 128 bytes of each row = K 256
-                        g_tma2d(st, &a.tm_p0, ps * 128, row0, bar);
-                        if (GU) g_tma2d(st + C::kMatBytes, &a.tm_p1, ps * 128, row0, bar);
+                        g_tma2d(st, &a.tm_p0, T.kbase / 2 + ps * 128, row0, bar);
+                        if (GU) g_tma2d(st + C::kMatBytes, &a.tm_p1, T.kbase / 2 + ps * 128, row0, bar);
                         if (FMT == MOE_FMT_NVFP4) {
                             const uint32_t ss = st + C::kNMat * C::kMatBytes;
-                            g_tma2d(ss, &a.tm_s0, ps * 16, row0, bar);
-                            if (GU) g_tma2d(ss + C::kNvScBytes, &a.tm_s1, ps * 16, row0, bar);
+                            g_tma2d(ss, &a.tm_s0, T.kbase / 16 + ps * 16, row0, bar);
+                            if (GU) g_tma2d(ss + C::kNvScBytes, &a.tm_s1, T.kbase / 16 + ps * 16, row0, bar);
                         }
                     } else {
                         // BF16: two 64-element halves of K 128 per matrix
 #pragma unroll
                         for (int h = 0; h < 2; h++) {
-                            g_tma2d(st + h * (G_BM * 128), &a.tm_p0, ps * 128 + h * 64, row0, bar);
-                            if (GU) g_tma2d(st + C::kMatBytes + h * (G_BM * 128), &a.tm_p1, ps * 128 + h * 64, row0, bar);
+                            const int x = T.kbase + ps * 128 + h * 64;
+                            g_tma2d(st + h * (G_BM * 128), &a.tm_p0, x, row0, bar);
+                            if (GU) g_tma2d(st + C::kMatBytes + h * (G_BM * 128), &a.tm_p1, x, row0, bar);
                         }
                     }
                 }
@@ -361,8 +370,8 @@ __global__ void __launch_bounds__(G_THREADS, 1) tc_grouped_gemm(const __grid_con
                 const uint32_t st = g_smem(bring + s * C::kBStageBytes);
                 if (g_elect()) {
                     g_expect(bar, uint32_t(T.bn) * 256u);
-                    g_tma2d(st, map, ks * C::kSK, row0, bar);
-                    g_tma2d(st + C::kBAtom, map, ks * C::kSK + 64, row0, bar);
+                    g_tma2d(st, map, T.kbase + ks * C::kSK, row0, bar);
+                    g_tma2d(st + C::kBAtom, map, T.kbase + ks * C::kSK + 64, row0, bar);
                 }
                 __syncwarp();
             }
@@ -455,6 +464,19 @@ __global__ void __launch_bounds__(G_THREADS, 1) tc_grouped_gemm(const __grid_con
                 g_ld16(acc0 + c, g);
                 if (GU) g_ld16(acc0 + C::kUpCol + c, u);
                 g_ld_wait();
+                if (ksplit > 1) {
+                    // split-K: raw fp32 sums of this K slice; a reduction kernel finishes the rows
+#pragma unroll
+                    for (int j = 0; j < 16; j++) {
+                        if (c + j < T.nval) {
+                            const size_t r = size_t(rbase + c + j);
+                            a.partial[((size_t(T.ks) * C::kNMat) * a.rows + r) * a.out_dim + f] = __uint_as_float(g[j]);
+                            if (GU)
+                                a.partial[((size_t(T.ks) * C::kNMat + 1) * a.rows + r) * a.out_dim + f] = __uint_as_float(u[j]);
+                        }
+                    }
+                    continue;
+                }
 #pragma unroll
                 for (int j = 0; j < 16; j++) {
                     const float fj = __shfl_sync(0xffffffffu, rowf, j);
@@ -624,6 +646,47 @@ __global__ void __launch_bounds__(256) g_prep(const __nv_bfloat16* __restrict__ 
 }
 
 // ---------------------------------------------------------------------------
+// Split-K finish: sums the K slices of every (row, feature) in slice order,
+// then h = bf16(silu(g) * u) (gate/up) or y = bf16(w * d) (down, w the routing
+// weight of the row's slot, 1 without routing weights).  Four features per thread.
+// ---------------------------------------------------------------------------
+__global__ void __launch_bounds__(256) g_splitk_finish(const float* __restrict__ part, int ksplit, int nmat, int rows,
+                                                       int out_dim, const float* __restrict__ topk_w,
+                                                       const int32_t* __restrict__ row_slot,
+                                                       __nv_bfloat16* __restrict__ out) {
+    asm volatile("griddepcontrol.wait;" ::: "memory");
+    const size_t n4 = size_t(rows) * out_dim / 4;
+    const size_t plane = size_t(rows) * out_dim;
+    for (size_t i = size_t(blockIdx.x) * blockDim.x + threadIdx.x; i < n4; i += size_t(gridDim.x) * blockDim.x) {
+        float4 g = make_float4(0.f, 0.f, 0.f, 0.f), u = g;
+        for (int k = 0; k < ksplit; k++) {
+            const float4 a = reinterpret_cast<const float4*>(part + (size_t(k) * nmat) * plane)[i];
+            g.x += a.x; g.y += a.y; g.z += a.z; g.w += a.w;
+            if (nmat == 2) {
+                const float4 b = reinterpret_cast<const float4*>(part + (size_t(k) * nmat + 1) * plane)[i];
+                u.x += b.x; u.y += b.y; u.z += b.z; u.w += b.w;
+            }
+        }
+        float v[4];
+        if (nmat == 2) {
+            v[0] = g.x / (1.0f + expf(-g.x)) * u.x;
+            v[1] = g.y / (1.0f + expf(-g.y)) * u.y;
+            v[2] = g.z / (1.0f + expf(-g.z)) * u.z;
+            v[3] = g.w / (1.0f + expf(-g.w)) * u.w;
+        } else {
+            const int r = int((i * 4) / out_dim);
+            const float w = topk_w ? topk_w[row_slot[r]] : 1.f;
+            v[0] = w * g.x; v[1] = w * g.y; v[2] = w * g.z; v[3] = w * g.w;
+        }
+        __nv_bfloat162 lo = __floats2bfloat162_rn(v[0], v[1]), hi = __floats2bfloat162_rn(v[2], v[3]);
+        uint2 o;
+        o.x = *reinterpret_cast<uint32_t*>(&lo);
+        o.y = *reinterpret_cast<uint32_t*>(&hi);
+        reinterpret_cast<uint2*>(out)[i] = o;
+    }
+}
+
+// ---------------------------------------------------------------------------
 // Host side
 // ---------------------------------------------------------------------------
 template <int FMT, bool GU>
@@ -658,6 +721,10 @@ static int g_launch(const GArgs& a, cudaStream_t s) {
 
 int launch_grouped_gemm(const GemvProblem& p, bool gateup, int rows, const GemmBuffers& buf, cudaStream_t s) {
     if (p.out_dim % G_BM || p.in_dim % 256 || p.E > kMaxE) return MOE_ERR_UNSUPPORTED;
+    const int ksplit = buf.ksplit > 1 ? buf.ksplit : 1;
+    if (ksplit > 1 && (p.fmt != MOE_FMT_BF16 || p.E != 1 || p.in_dim % (ksplit * 128) || !buf.partial ||
+                       p.out_dim % 4))
+        return MOE_ERR_UNSUPPORTED;
     if (p.fmt == MOE_FMT_INT4_G128 &&
         ((reinterpret_cast<uintptr_t>(p.s0) & 15u) || (gateup && (reinterpret_cast<uintptr_t>(p.s1) & 15u))))
         return MOE_ERR_INVALID_ARG;
@@ -709,10 +776,22 @@ int launch_grouped_gemm(const GemvProblem& p, bool gateup, int rows, const GemmB
     a.out_dim = out;
     a.in_dim = in;
     a.perm_out = buf.perm_out;
+    a.ksplit = ksplit;
+    a.partial = buf.partial;
+    a.rows = rows;
 
     if (i4) return gateup ? g_launch<MOE_FMT_INT4_G128, true>(a, s) : g_launch<MOE_FMT_INT4_G128, false>(a, s);
     if (nv) return gateup ? g_launch<MOE_FMT_NVFP4, true>(a, s) : g_launch<MOE_FMT_NVFP4, false>(a, s);
-    return gateup ? g_launch<MOE_FMT_BF16, true>(a, s) : g_launch<MOE_FMT_BF16, false>(a, s);
+    const int rc = gateup ? g_launch<MOE_FMT_BF16, true>(a, s) : g_launch<MOE_FMT_BF16, false>(a, s);
+    if (rc != MOE_OK) return rc;
+    if (ksplit > 1) {
+        const size_t n4 = size_t(rows) * out / 4;
+        const int blocks = int(std::min<size_t>((n4 + 255) / 256, 148 * 8));
+        if (launch_pdl(g_splitk_finish, dim3(blocks), dim3(256), 0, s, static_cast<const float*>(buf.partial), ksplit,
+                       gateup ? 2 : 1, rows, out, p.topk_w, p.row_slot, p.out) != cudaSuccess)
+            return MOE_ERR_CUDA;
+    }
+    return MOE_OK;
 }
 
 }  // namespace moe

@@ -23,7 +23,7 @@ constexpr int kMaxDecodeT = 64;
 // ---------------------------------------------------------------------------
 struct WsLayout {
     size_t ctrl, logits, wsplit, hist, offsets, row_slot, slot_row, ids, tw;
-    size_t sh_offsets, sh_rowslot, h_perm, y_perm, ys, tiles, prep, total;
+    size_t sh_offsets, sh_rowslot, h_perm, y_perm, ys, tiles, prep, shpart, total;
 };
 
 constexpr int kPermChunk = 4096;   // slots handled by one bucketing block
@@ -64,6 +64,18 @@ inline size_t grouped_scratch(int E, int act_rows, int in_dim) {
     return align256(size_t(E + 2) * 16) + prep_scratch(act_rows, in_dim);
 }
 
+// The BF16 shared expert at a small batch has few (m, n) tiles (12 for gate/up,
+// 32 for down); split K so that the weight stream spreads over the GPU.
+inline int shared_ksplit(int E, int fmt, bool gateup, int rows, int in_dim) {
+    if (E != 1 || fmt != MOE_FMT_BF16 || rows > 64) return 1;
+    int ks = gateup ? 8 : 4;
+    while (ks > 1 && in_dim % (ks * 128)) ks >>= 1;
+    return ks;
+}
+inline size_t split_bytes(int ksplit, bool gateup, int rows, int out_dim) {
+    return ksplit > 1 ? align256(size_t(ksplit) * (gateup ? 2 : 1) * rows * out_dim * 4) : 0;
+}
+
 inline WsLayout ws_layout(int T, int H, int E, int F, int k) {
     WsLayout L{};
     size_t R = size_t(T) * k;
@@ -86,6 +98,8 @@ inline WsLayout ws_layout(int T, int H, int E, int F, int k) {
     L.ys = o;         o = align256(o + size_t(T) * H * 2);
     L.tiles = o;      o = align256(o + size_t(E + 2) * 4 * 4);
     L.prep = o;       o = align256(o + std::max(prep_scratch(T, H), prep_scratch(int(R), F)));
+    L.shpart = o;     o = align256(o + std::max(split_bytes(shared_ksplit(1, MOE_FMT_BF16, true, T, H), true, T, F),
+                                                split_bytes(shared_ksplit(1, MOE_FMT_BF16, false, T, F), false, T, H)));
     L.total = o;
     return L;
 }
@@ -188,7 +202,10 @@ struct GemmBuffers {
     float* scale_buf;
     int act_ready;
     int perm_out;
+    int ksplit;          // > 1: split K into this many slices (BF16 only); fp32 partial sums go to partial
+    float* partial;      // split_bytes(...) bytes
 };
+
 
 // Prefill-shaped grouped GEMM (tcgen05) for one problem; rows: activation
 // (and output) rows of the problem.
