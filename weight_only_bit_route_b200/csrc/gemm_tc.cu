@@ -72,24 +72,38 @@ constexpr int G_THREADS = 512;
 constexpr int G_DQ_WARPS = 8;
 constexpr int G_EPI_WARPS = 4;
 
+// int4 with small token tiles ("fast int4"): the dequantisation makes f16
+// values 1024 + u (even nibbles) or 1024 + 16u (odd nibbles) with bit masks
+// only; the activations are stored as f16 x * 2^-e, divided by 16 at the odd
+// positions, so each product is u * x * 2^-e plus a constant times x.  Each
+// K = 128 stage (one scale group) accumulates from zero, and the epilogue warps
+// fold scale * (stage sum - Z) into fp32 totals, Z being the per-token, per-
+// group constant the pre-pass computes.  The group scale and the -8 offset
+// leave the per-weight work.  Internal format value.
+constexpr int FMT_INT4_FAST = 3;
+
 template <int FMT, bool GU>
 struct GCfg {
+    static constexpr bool kFast = FMT == FMT_INT4_FAST;
+    static constexpr bool kInt4 = FMT == MOE_FMT_INT4_G128 || kFast;
     static constexpr bool kTmemA = FMT != MOE_FMT_BF16;
     static constexpr int kNMat = GU ? 2 : 1;
-    static constexpr int kNMax = GU ? 64 : 128;                    // token rows per tile
-    static constexpr int kUpCol = 64;                               // up accumulator within a buffer
+    static constexpr int kNMax = kFast ? 16 : (GU ? 64 : 128);     // token rows per tile
+    static constexpr int kUpCol = kFast ? 16 : 64;                  // up accumulator within a buffer
+    static constexpr int kAccCols = kFast ? kNMat * 16 : 128;       // one accumulator buffer
     static constexpr int kSK = 128;                                 // K per MMA stage
     static constexpr int kPkK = kTmemA ? 256 : 128;                 // K per weight stage
     static constexpr int kMatBytes = kTmemA ? G_BM * 128 : G_BM * 256;   // one matrix of a weight stage
     static constexpr int kNvScBytes = FMT == MOE_FMT_NVFP4 ? G_BM * 16 : 0;
     static constexpr int kPkStageBytes = kNMat * (kMatBytes + kNvScBytes);
     static constexpr int kPkStages = kTmemA ? ((GU && FMT == MOE_FMT_INT4_G128) ? 3 : 4) : 2;
+    static constexpr int kScStages = kFast ? G_EPI_WARPS : G_DQ_WARPS;   // readers of the int4 scale buffer
     static constexpr int kBAtom = kNMax * 128;                      // one 64-wide K half of a B stage
     static constexpr int kBStageBytes = 2 * kBAtom;
     static constexpr int kBStages = 4;
     static constexpr int kAStageCols = kNMat * 64;                  // K = 128 as 16-bit pairs, per matrix
     static constexpr int kAStages = 256 / kAStageCols;
-    static constexpr bool kMmaF16 = FMT == MOE_FMT_NVFP4;
+    static constexpr bool kMmaF16 = FMT == MOE_FMT_NVFP4 || kFast;
 };
 
 constexpr int G_NB_MAPS = 8;                                        // box heights 16, 32, ..., 128
@@ -109,6 +123,7 @@ struct GArgs {
     __nv_bfloat16* out;
     int32_t* status;
     float* partial;                  // split-K: fp32 partial sums [ksplit][nmat][rows][out_dim]
+    const float* zsum;               // fast int4: per-row, per-group constant [rows][in / 128]
     int E, out_dim, in_dim, perm_out;
     int ksplit, rows;                // K slices per (m-tile, n-tile); activation rows of the problem
 };
@@ -146,6 +161,20 @@ __device__ __forceinline__ void g_dq_nvfp4(const uint4 w, uint32_t sc2, uint32_t
             __half2 h = __hmul2(*reinterpret_cast<__half2*>(&hv), s2);       // exact
             o[j * 4 + b] = *reinterpret_cast<uint32_t*>(&h);
         }
+    }
+}
+
+// fast int4: nibble pairs (p, p+4) of each word as f16 {1024 + u} (p = 0, 2)
+// or {1024 + 16u} (p = 1, 3); four logic ops and one shift per word.
+__device__ __forceinline__ void g_dq_int4_fast(const uint4 w, uint32_t (&o)[16]) {
+    const uint32_t ws[4] = {w.x, w.y, w.z, w.w};
+#pragma unroll
+    for (int j = 0; j < 4; j++) {
+        const uint32_t hi = ws[j] >> 8;
+        o[j * 4 + 0] = (ws[j] & 0x000F000Fu) | 0x64006400u;
+        o[j * 4 + 1] = (ws[j] & 0x00F000F0u) | 0x64006400u;
+        o[j * 4 + 2] = (hi & 0x000F000Fu) | 0x64006400u;
+        o[j * 4 + 3] = (hi & 0x00F000F0u) | 0x64006400u;
     }
 }
 
@@ -204,7 +233,7 @@ __global__ void __launch_bounds__(G_THREADS, 1) tc_grouped_gemm(const __grid_con
         }
         for (int s = 0; s < 2; s++) {
             asm volatile("mbarrier.init.shared::cta.b64 [%0], 1;" ::"r"(g_smem(&sc_full[s])));
-            asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(g_smem(&sc_empty[s])), "r"(G_DQ_WARPS));
+            asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(g_smem(&sc_empty[s])), "r"(C::kScStages));
             asm volatile("mbarrier.init.shared::cta.b64 [%0], 1;" ::"r"(g_smem(&acc_full[s])));
             asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(g_smem(&acc_empty[s])), "r"(G_EPI_WARPS));
         }
@@ -295,7 +324,7 @@ __global__ void __launch_bounds__(G_THREADS, 1) tc_grouped_gemm(const __grid_con
         for (int tile = blockIdx.x; tile < ntiles && !s_abort; tile += gridDim.x) {
             const GTile T = tile_of(tile);
             const int row0 = T.e * a.out_dim + T.m0;
-            if (FMT == MOE_FMT_INT4_G128) {
+            if (C::kInt4) {
                 const int b = t & 1;
                 if (t >= 2 && !g_wait_w(g_smem(&sc_empty[b]), ((t >> 1) - 1) & 1, &s_abort, 64)) { fail(); break; }
                 const uint32_t bar = g_smem(&sc_full[b]);
@@ -347,7 +376,7 @@ __global__ void __launch_bounds__(G_THREADS, 1) tc_grouped_gemm(const __grid_con
         if (lane == 0) {
             const uint32_t first = pc > uint32_t(C::kPkStages) ? pc - C::kPkStages : 0;
             for (uint32_t n = first; n < pc; n++) g_drain_wait(g_smem(&pk_full[n % C::kPkStages]), (n / C::kPkStages) & 1);
-            if (FMT == MOE_FMT_INT4_G128)
+            if (C::kInt4)
                 for (int n = t > 2 ? t - 2 : 0; n < t; n++) g_drain_wait(g_smem(&sc_full[n & 1]), (n >> 1) & 1);
         }
         __syncwarp();
@@ -390,8 +419,11 @@ __global__ void __launch_bounds__(G_THREADS, 1) tc_grouped_gemm(const __grid_con
             const GTile T = tile_of(tile);
             const uint32_t idesc = g_idesc(T.bn, C::kMmaF16);
             const int buf = t & 1;
-            const uint32_t d = tmem + buf * 128;
-            if (t >= 2 && !g_wait_w(g_smem(&acc_empty[buf]), ((t >> 1) - 1) & 1, &s_abort)) { fail(); break; }
+            uint32_t d = tmem + buf * 128;
+            if (!C::kFast && t >= 2 && !g_wait_w(g_smem(&acc_empty[buf]), ((t >> 1) - 1) & 1, &s_abort)) {
+                fail();
+                break;
+            }
             g_fence_after();
             bool ok = true;
             for (int ks = 0; ks < KS; ks++) {
@@ -402,6 +434,12 @@ __global__ void __launch_bounds__(G_THREADS, 1) tc_grouped_gemm(const __grid_con
                 } else {
                     if (!g_wait_w(g_smem(&pk_full[sp]), (pc / C::kPkStages) & 1, &s_abort)) { ok = false; break; }
                 }
+                if (C::kFast) {
+                    // every stage into a fresh buffer of the two; the epilogue frees it
+                    const int bi = ac & 1;
+                    if (ac >= 2 && !g_wait_w(g_smem(&acc_empty[bi]), ((ac >> 1) - 1) & 1, &s_abort)) { ok = false; break; }
+                    d = tmem + bi * C::kAccCols;
+                }
                 g_fence_after();
                 const uint32_t b0 = g_smem(bring + sb * C::kBStageBytes);
                 const uint32_t at = tmem + 256 + sa * C::kAStageCols;
@@ -409,7 +447,7 @@ __global__ void __launch_bounds__(G_THREADS, 1) tc_grouped_gemm(const __grid_con
                 if (g_elect()) {
 #pragma unroll
                     for (int k = 0; k < C::kSK / 16; k++) {
-                        const uint32_t acc = (ks > 0 || k > 0) ? 1u : 0u;
+                        const uint32_t acc = (k > 0 || (!C::kFast && ks > 0)) ? 1u : 0u;
                         const uint64_t bd = g_desc(b0 + (k >> 2) * C::kBAtom + (k & 3) * 32);
                         if (C::kTmemA) {
                             g_mma_ts(d, at + k * 8, bd, idesc, acc);
@@ -428,7 +466,7 @@ __global__ void __launch_bounds__(G_THREADS, 1) tc_grouped_gemm(const __grid_con
                 if (C::kTmemA) ac++; else pc++;
             }
             if (!ok) { fail(); break; }
-            if (g_elect()) g_commit(g_smem(&acc_full[buf]));
+            if (!C::kFast && g_elect()) g_commit(g_smem(&acc_full[buf]));
             __syncwarp();
         }
         // drain: every MMA issued has completed
@@ -436,6 +474,76 @@ __global__ void __launch_bounds__(G_THREADS, 1) tc_grouped_gemm(const __grid_con
         __syncwarp();
         if (lane == 0) g_drain_wait(g_smem(&drain), 0);
         __syncwarp();
+    } else if (warp >= 4 && warp < 8 && C::kFast) {
+        // ---------------- fast int4 epilogue: fold every K = 128 stage ----------------
+        // Thread (warp w, lane l) owns weight row 32*(w%4) + l of the tile; lane
+        // j < 16 also holds token row j's group constant and row factor.
+        const int q = warp & 3;
+        const uint32_t lane_addr = uint32_t(q * 32) << 16;
+        const int r = q * 32 + lane;
+        const int nj = lane & 15;
+        uint32_t ac = 0;
+        int t = 0;
+        bool ok = true;
+        for (int tile = blockIdx.x; tile < ntiles && ok && !s_abort; tile += gridDim.x, t++) {
+            const GTile T = tile_of(tile);
+            const int f = T.m0 + r;
+            const int rbase = T.ebase + T.n0;
+            const bool live = nj < T.nval;
+            const int b = t & 1;
+            if (!g_wait(g_smem(&sc_full[b]), (t >> 1) & 1, &s_abort, 64)) { ok = false; break; }
+            const __nv_bfloat16* sc0 = reinterpret_cast<const __nv_bfloat16*>(scbuf + b * C::kNMat * sc_mat_bytes) + r * ngroups;
+            const __nv_bfloat16* sc1 = sc0 + G_BM * ngroups;
+            const float* zrow = a.zsum + size_t(rbase + (live ? nj : 0)) * ngroups;
+            float tg[16], tu[16];
+#pragma unroll
+            for (int j = 0; j < 16; j++) tg[j] = tu[j] = 0.f;
+            for (int ks = 0; ks < KS; ks++, ac++) {
+                const int sa = ac % C::kAStages, bi = ac & 1;
+                if (!g_wait(g_smem(&a_empty[sa]), (ac / C::kAStages) & 1, &s_abort)) { ok = false; break; }
+                g_fence_after();
+                uint32_t g[16], u[16];
+                g_ld16(tmem + lane_addr + bi * C::kAccCols, g);
+                if (GU) g_ld16(tmem + lane_addr + bi * C::kAccCols + C::kUpCol, u);
+                g_ld_wait();
+                g_fence_before();
+                __syncwarp();
+                if (lane == 0) g_arrive(g_smem(&acc_empty[bi]));      // the buffer takes stage ac + 2
+                const int grp = T.kbase / 128 + ks;
+                const float z = live ? zrow[grp] : 0.f;
+                const float s0 = __bfloat162float(sc0[grp]);
+                const float s1 = GU ? __bfloat162float(sc1[grp]) : 0.f;
+#pragma unroll
+                for (int j = 0; j < 16; j++) {
+                    const float zj = __shfl_sync(0xffffffffu, z, j);
+                    tg[j] = fmaf(s0, __uint_as_float(g[j]) - zj, tg[j]);
+                    if (GU) tu[j] = fmaf(s1, __uint_as_float(u[j]) - zj, tu[j]);
+                }
+            }
+            if (!ok) break;
+            __syncwarp();
+            if (lane == 0) g_arrive(g_smem(&sc_empty[b]));
+            float rowf = 1.f;
+            if (live) {
+                rowf = a.act_scale[rbase + nj];
+                if (!GU && a.topk_w) rowf *= a.topk_w[a.row_slot[rbase + nj]];
+            }
+#pragma unroll
+            for (int j = 0; j < 16; j++) {
+                const float fj = __shfl_sync(0xffffffffu, rowf, j);
+                if (j < T.nval) {
+                    float v;
+                    if (GU) {
+                        const float gg = tg[j] * fj, uu = tu[j] * fj;
+                        v = gg / (1.0f + expf(-gg)) * uu;
+                    } else {
+                        v = tg[j] * fj;
+                    }
+                    a.out[size_t(rbase + j) * a.out_dim + f] = __float2bfloat16_rn(v);
+                }
+            }
+        }
+        if (!ok) fail();
     } else if (warp >= 4 && warp < 8) {
         // ---------------- epilogue ----------------
         const int q = warp & 3;
@@ -529,8 +637,9 @@ __global__ void __launch_bounds__(G_THREADS, 1) tc_grouped_gemm(const __grid_con
                 uint32_t scw = 0;                      // int4: bf16 scales of groups 2ps (low) and 2ps+1 (high)
                 uint4 nsc = make_uint4(0, 0, 0, 0);    // NVFP4: the 16 E4M3 scales of this row and stage
                 if (FMT == MOE_FMT_INT4_G128) scw = *reinterpret_cast<const uint32_t*>(scrow + ps * 4);
-                else nsc = *reinterpret_cast<const uint4*>(st + C::kNMat * C::kMatBytes + (GU ? hsel * C::kNvScBytes : 0) +
-                                                           r * 16);
+                else if (FMT == MOE_FMT_NVFP4)
+                    nsc = *reinterpret_cast<const uint4*>(st + C::kNMat * C::kMatBytes + (GU ? hsel * C::kNvScBytes : 0) +
+                                                          r * 16);
                 const uint32_t nscw[4] = {nsc.x, nsc.y, nsc.z, nsc.w};
                 // Four register buffers in rotation: a buffer is rewritten three
                 // chunks after its tensor-memory store was issued, so the store
@@ -541,7 +650,9 @@ __global__ void __launch_bounds__(G_THREADS, 1) tc_grouped_gemm(const __grid_con
                     constexpr int i = decltype(ic)::value, j = i / kPer, l = i % kPer;
                     const int c = 4 * j + (GU ? l : 2 * hsel + l);
                     const uint4 w = *reinterpret_cast<const uint4*>(wt + g_swz(r, c));
-                    if (FMT == MOE_FMT_INT4_G128) {
+                    if (FMT == FMT_INT4_FAST) {
+                        g_dq_int4_fast(w, o[i % kNBuf]);
+                    } else if (FMT == MOE_FMT_INT4_G128) {
                         g_dq_int4(w, scw >> (16 * j), o[i % kNBuf]);
                     } else {
                         // the two E4M3 scales of chunk c are bytes 2c and 2c+1
@@ -598,10 +709,15 @@ __global__ void __launch_bounds__(G_THREADS, 1) tc_grouped_gemm(const __grid_con
 //   mode 2: f16 times 2^-e (e >= 0 least with |x| * 2^-e <= 16384), row scale 2^e.
 // One warp per row.
 // ---------------------------------------------------------------------------
+//   mode 3 (fast int4): f16 in the pair order, times 2^-e, with the elements
+//          paired with odd nibbles (x1, x5, x3, x7 of every 8) divided by 16;
+//          zsum[row][g] = sum over group g of (1024 + 8c) * value, c = 16 at
+//          the divided positions and 1 elsewhere: the part of the MMA sum
+//          that is not q * x * 2^-e.
 __global__ void __launch_bounds__(256) g_prep(const __nv_bfloat16* __restrict__ src, int in_dim,
                                               const int32_t* __restrict__ row_slot, int top_k, int by_token,
                                               int rows, int mode, uint16_t* __restrict__ dst,
-                                              float* __restrict__ scale) {
+                                              float* __restrict__ scale, float* __restrict__ zsum) {
     asm volatile("griddepcontrol.wait;" ::: "memory");
     const int row = (blockIdx.x * blockDim.x + threadIdx.x) >> 5, lane = threadIdx.x & 31;
     if (row >= rows) return;
@@ -621,6 +737,37 @@ __global__ void __launch_bounds__(256) g_prep(const __nv_bfloat16* __restrict__ 
             o.w = __byte_perm(v.y, v.w, 0x7632);   // (x3, x7)
             d[i] = o;
         }
+    } else if (mode == 3) {
+        float amax = 0.f;
+        for (int i = lane; i < n16; i += 32) {
+            const uint4 v = s[i];
+            amax = fmaxf(amax, fmaxf(fmaxf(fabsf(bf16_lo(v.x)), fabsf(bf16_hi(v.x))), fmaxf(fabsf(bf16_lo(v.y)), fabsf(bf16_hi(v.y)))));
+            amax = fmaxf(amax, fmaxf(fmaxf(fabsf(bf16_lo(v.z)), fabsf(bf16_hi(v.z))), fmaxf(fabsf(bf16_lo(v.w)), fabsf(bf16_hi(v.w)))));
+        }
+        for (int o = 16; o > 0; o >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, o));
+        int e = 0;
+        while (e < 126 && ldexpf(amax, -e) > 16384.f) e++;
+        const float down = ldexpf(1.f, -e), down16 = down * 0.0625f;
+        // 16 pieces of 8 make a group of 128: lanes 0-15 and 16-31 take one group each per pass
+        for (int i0 = 0; i0 < n16; i0 += 32) {
+            const int i = i0 + lane;
+            float z = 0.f;
+            if (i < n16) {
+                const uint4 v = s[i];
+                __half2 h[4];
+                h[0] = __floats2half2_rn(bf16_lo(v.x) * down, bf16_lo(v.z) * down);       // (x0, x4)
+                h[1] = __floats2half2_rn(bf16_hi(v.x) * down16, bf16_hi(v.z) * down16);   // (x1, x5) / 16
+                h[2] = __floats2half2_rn(bf16_lo(v.y) * down, bf16_lo(v.w) * down);       // (x2, x6)
+                h[3] = __floats2half2_rn(bf16_hi(v.y) * down16, bf16_hi(v.w) * down16);   // (x3, x7) / 16
+                d[i] = *reinterpret_cast<uint4*>(h);
+                const float2 a0 = __half22float2(h[0]), a1 = __half22float2(h[1]);
+                const float2 a2 = __half22float2(h[2]), a3 = __half22float2(h[3]);
+                z = 1032.f * (a0.x + a0.y + a2.x + a2.y) + 1152.f * (a1.x + a1.y + a3.x + a3.y);
+            }
+            for (int o = 8; o > 0; o >>= 1) z += __shfl_xor_sync(0xffffffffu, z, o);
+            if ((lane & 15) == 0 && i < n16) zsum[size_t(row) * (in_dim / 128) + i / 16] = z;
+        }
+        if (lane == 0) scale[row] = ldexpf(1.f, e);
     } else {
         float amax = 0.f;
         for (int i = lane; i < n16; i += 32) {
@@ -693,7 +840,7 @@ template <int FMT, bool GU>
 static size_t g_smem_bytes(int in_dim) {
     using C = GCfg<FMT, GU>;
     size_t b = size_t(C::kPkStages) * C::kPkStageBytes + size_t(C::kBStages) * C::kBStageBytes + 1024;
-    if (FMT == MOE_FMT_INT4_G128) b += 2 * size_t(C::kNMat) * G_BM * (in_dim / 128) * 2;
+    if (C::kInt4) b += 2 * size_t(C::kNMat) * G_BM * (in_dim / 128) * 2;
     return b;
 }
 
@@ -733,14 +880,17 @@ int launch_grouped_gemm(const GemvProblem& p, bool gateup, int rows, const GemmB
 
     const int in = p.in_dim, out = p.out_dim, E = p.E;
     const bool nv = p.fmt == MOE_FMT_NVFP4, i4 = p.fmt == MOE_FMT_INT4_G128;
+    const bool fast = i4 && buf.fast;
+    if (fast && (!buf.zbuf || !buf.scale_buf || !buf.act_buf || buf.perm_out || ksplit > 1)) return MOE_ERR_UNSUPPORTED;
     // activation operand rows [rows, in]: bf16 (f16 for NVFP4) in the kernel's order
     const void* bsrc = p.act;
     const float* ascale = nullptr;
-    if (!buf.act_ready || nv) {
+    if (!buf.act_ready || nv || fast) {
         if (!buf.act_buf || (nv && !buf.scale_buf)) return MOE_ERR_WORKSPACE;
-        const int mode = nv ? 2 : (i4 ? 1 : 0);
+        const int mode = fast ? 3 : nv ? 2 : (i4 ? 1 : 0);
         if (launch_pdl(g_prep, dim3((rows * 32 + 255) / 256), dim3(256), 0, s, p.act, in, p.row_slot, p.top_k,
-                       p.act_by_token, rows, mode, reinterpret_cast<uint16_t*>(buf.act_buf), buf.scale_buf) != cudaSuccess)
+                       p.act_by_token, rows, mode, reinterpret_cast<uint16_t*>(buf.act_buf), buf.scale_buf,
+                       buf.zbuf) != cudaSuccess)
             return MOE_ERR_CUDA;
         bsrc = buf.act_buf;
         ascale = buf.scale_buf;
@@ -779,7 +929,9 @@ int launch_grouped_gemm(const GemvProblem& p, bool gateup, int rows, const GemmB
     a.ksplit = ksplit;
     a.partial = buf.partial;
     a.rows = rows;
+    a.zsum = buf.zbuf;
 
+    if (fast) return gateup ? g_launch<FMT_INT4_FAST, true>(a, s) : g_launch<FMT_INT4_FAST, false>(a, s);
     if (i4) return gateup ? g_launch<MOE_FMT_INT4_G128, true>(a, s) : g_launch<MOE_FMT_INT4_G128, false>(a, s);
     if (nv) return gateup ? g_launch<MOE_FMT_NVFP4, true>(a, s) : g_launch<MOE_FMT_NVFP4, false>(a, s);
     const int rc = gateup ? g_launch<MOE_FMT_BF16, true>(a, s) : g_launch<MOE_FMT_BF16, false>(a, s);
