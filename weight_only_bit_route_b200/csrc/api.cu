@@ -66,9 +66,9 @@ int run_problem(const GemvProblem& p, bool gateup, int rows, int act_rows, void*
 
 // The step-level calls' scratch: the GEMV or GEMM pre-pass of rows rows, then
 // the shared expert's split-K partial sums.
-// GEMM pre-pass layout in a scratch region: row scales [rows], per-group
-// constants [rows][in / 128] (fast int4), gathered rows [rows][in].
-GemmBuffers gemm_buffers(void* base, int rows, int in_dim, bool act_ready, bool fast) {
+// GEMM pre-pass layout in a scratch region of gemm_prep_bytes(rows, in_dim):
+// row scales [rows], group sums [rows][in / 128] (8-bit int4), gathered rows.
+GemmBuffers gemm_buffers(void* base, int rows, int in_dim, bool act_ready, bool i8) {
     uint8_t* p = reinterpret_cast<uint8_t*>(base);
     GemmBuffers b{};
     b.scale_buf = reinterpret_cast<float*>(p);
@@ -76,14 +76,11 @@ GemmBuffers gemm_buffers(void* base, int rows, int in_dim, bool act_ready, bool 
     b.act_buf = p + align256(size_t(rows) * 4) + align256(size_t(rows) * (in_dim / 128) * 4);
     b.act_ready = act_ready;
     b.perm_out = 0;
-    b.fast = fast;
+    b.i8 = i8;
     return b;
 }
-bool fast_int4(const GemvProblem& p, int rows) {
-    return p.fmt == MOE_FMT_INT4_G128 && p.E > 1 && rows <= kFastInt4MaxRows;
-}
-GemmBuffers step_buffers(void* prep, int rows, int in_dim, bool act_ready, bool fast) {
-    return gemm_buffers(prep, rows, in_dim, act_ready, fast);
+bool i8_int4(const GemvProblem& p, int rows) {
+    return p.fmt == MOE_FMT_INT4_G128 && p.E > 1 && rows <= kI8Int4MaxRows;
 }
 size_t step_scratch(int E, int fmt, bool gateup, int rows, int in_dim, int out_dim) {
     return grouped_scratch(E, rows, in_dim) + split_bytes(shared_ksplit(E, fmt, gateup, rows, in_dim), gateup, rows, out_dim);
@@ -177,13 +174,13 @@ int layer_run(const void* x, int T, const moe_layer* L, void* y, void* ws, cudaS
 
     // routed experts: both projections on one path (the int4 GEMM hands h to
     // the down GEMM in its pair order)
-    const bool fast = routed_gemm && fast_int4(gu, R);
+    const bool i8 = routed_gemm && i8_int4(gu, R);
     if (routed_gemm) {
-        // the gate/up activation rows are gathered into the y_perm region,
+        // 16-bit gate/up activation rows are gathered into the y_perm region,
         // free until the down projection writes it
-        GemmBuffers gb = gemm_buffers(prep, R, H, false, fast);
-        gb.act_buf = y_perm;
-        gb.perm_out = int4 && !fast;
+        GemmBuffers gb = gemm_buffers(prep, R, H, false, i8);
+        if (!i8) gb.act_buf = y_perm;
+        gb.perm_out = int4 && !i8;
         MOE_TRY(launch_grouped_gemm(gu, true, R, gb, s));
     } else {
         MOE_TRY(launch_stream_gemv(gu, nullptr, true, T, prep, s, true));
@@ -194,8 +191,8 @@ int layer_run(const void* x, int T, const moe_layer* L, void* y, void* ws, cudaS
     float* shpart = at<float>(ws, W.shpart);
     if (has_sh) MOE_TRY(run_problem(sg, true, T, T, nullptr, direct, shpart, s));
     if (routed_gemm) {
-        // int4 h is already in the pair order unless the fast path made it
-        GemmBuffers db = gemm_buffers(prep, R, F, int4 && !fast, fast);
+        // int4 h is already in the pair order unless the 8-bit path made it
+        GemmBuffers db = gemm_buffers(prep, R, F, int4 && !i8, i8);
         MOE_TRY(launch_grouped_gemm(dn, false, R, db, s));
     } else {
         MOE_TRY(launch_stream_gemv(dn, nullptr, false, R, prep, s, true));
@@ -310,7 +307,7 @@ int moe_grouped_w4a16_swiglu(const void* x, int T, int H, const int32_t* expert_
     p.p1 = up->packed; p.s1 = up->scales; p.g1 = up->global_scale;
     p.out = reinterpret_cast<__nv_bfloat16*>(h_perm); p.status = at<int32_t>(ws, 0);
     void* prep = at<void>(ws, kStepScratch + align256(size_t(E + 2) * 16));
-    return run_problem(p, true, rows, T, prep, step_buffers(prep, rows, H, false, fast_int4(p, rows)),
+    return run_problem(p, true, rows, T, prep, gemm_buffers(prep, rows, H, false, i8_int4(p, rows)),
                        step_partial(ws, E, rows, H), cs(stream));
 }
 
@@ -335,7 +332,7 @@ int moe_grouped_w4a16_down(const void* h_perm, const int32_t* expert_offsets, co
     void* prep = at<void>(ws, kStepScratch + align256(size_t(E + 2) * 16));
     // BF16 rows are read in place (row r is activation row r)
     return run_problem(p, false, rows, rows, prep,
-                       step_buffers(prep, rows, F, down->fmt == MOE_FMT_BF16, fast_int4(p, rows)),
+                       gemm_buffers(prep, rows, F, down->fmt == MOE_FMT_BF16, i8_int4(p, rows)),
                        step_partial(ws, E, rows, F), cs(stream));
 }
 

@@ -29,8 +29,12 @@
 //   warp 2      allocates tensor memory and issues tcgen05.mma from one lane.
 // The three single-issue roles run warp-uniform loops and elect one lane to
 // issue, which keeps the instruction operands in uniform registers.  The MMA
-// pipeline steps in K = 128: a tcgen05.commit costs about as much issue time
-// as several MMAs, so it is paid once per 16 (gate/up) or 8 (down) MMAs.
+// pipeline steps in K = 128 and commits once per step, to one barrier of a
+// ring of 16 ("stage done"): a tcgen05.commit costs as much issue time as
+// several MMAs, so every role that waits for a step to finish (the activation
+// producer, the dequantisation warps, the BF16 weight producer, the small-
+// batch epilogue) waits on that one barrier.  No waiter can fall 16 steps
+// behind, which keeps the ring's phases unambiguous.
 //   warps 4-7   epilogue: tcgen05.ld of the accumulators, SwiGLU or the
 //               routing weight, bf16 stores.  Warp w reads TMEM lanes
 //               32*(w%4) to 32*(w%4)+31.
@@ -72,39 +76,49 @@ constexpr int G_THREADS = 512;
 constexpr int G_DQ_WARPS = 8;
 constexpr int G_EPI_WARPS = 4;
 
-// int4 with small token tiles ("fast int4"): the dequantisation makes f16
-// values 1024 + u (even nibbles) or 1024 + 16u (odd nibbles) with bit masks
-// only; the activations are stored as f16 x * 2^-e, divided by 16 at the odd
-// positions, so each product is u * x * 2^-e plus a constant times x.  Each
-// K = 128 stage (one scale group) accumulates from zero, and the epilogue warps
-// fold scale * (stage sum - Z) into fp32 totals, Z being the per-token, per-
-// group constant the pre-pass computes.  The group scale and the -8 offset
-// leave the per-weight work.  Internal format value.
-constexpr int FMT_INT4_FAST = 3;
+// int4 with small token tiles (8-bit MMA): the dequantisation only unpacks
+// each nibble u into a byte (two logic ops per 4 weights) and the tensor
+// cores run kind::i8 (u8 weights x s8 activations, exact s32 sums, K = 32 per
+// instruction).  The pre-pass writes each activation row as a 24-bit fixed
+// point X = x * 2^c (c per row, |X| < 2^22) in three signed 8-bit digits,
+// X = 65536 d2 + 256 d1 + d0, one B operand row per digit (token j's digits
+// are rows 3j, 3j+1, 3j+2 of the tile: five tokens fill N = 16).  Each K = 128
+// step (one scale group) accumulates from zero; the epilogue warps combine
+// the digit sums, subtract 8 * sum(X) over the group (the u - 8 offset) and
+// fold scale * value into fp32 totals.  The group scale and the offset leave
+// the per-weight work, and the accumulation itself is exact.  Internal
+// format value.
+constexpr int FMT_INT4_I8 = 3;
 
 template <int FMT, bool GU>
 struct GCfg {
-    static constexpr bool kFast = FMT == FMT_INT4_FAST;
-    static constexpr bool kInt4 = FMT == MOE_FMT_INT4_G128 || kFast;
+    static constexpr bool kI8 = FMT == FMT_INT4_I8;
+    static constexpr bool kInt4 = FMT == MOE_FMT_INT4_G128 || kI8;
     static constexpr bool kTmemA = FMT != MOE_FMT_BF16;
     static constexpr int kNMat = GU ? 2 : 1;
-    static constexpr int kNMax = kFast ? 16 : (GU ? 64 : 128);     // token rows per tile
-    static constexpr int kUpCol = kFast ? 16 : 64;                  // up accumulator within a buffer
-    static constexpr int kAccCols = kFast ? kNMat * 16 : 128;       // one accumulator buffer
+    static constexpr int kNMax = kI8 ? 5 : (GU ? 64 : 128);        // token rows per tile
+    static constexpr int kUpCol = kI8 ? 16 : 64;                    // up accumulator within a buffer
+    static constexpr int kAccCols = kI8 ? kNMat * 16 : 128;         // one accumulator buffer
+    static constexpr int kAccBufs = kI8 ? 4 : 2;                    // accumulator buffers in [0, 256)
     static constexpr int kSK = 128;                                 // K per MMA stage
+    static constexpr int kMmaK = kI8 ? 32 : 16;                     // K per MMA instruction
     static constexpr int kPkK = kTmemA ? 256 : 128;                 // K per weight stage
     static constexpr int kMatBytes = kTmemA ? G_BM * 128 : G_BM * 256;   // one matrix of a weight stage
     static constexpr int kNvScBytes = FMT == MOE_FMT_NVFP4 ? G_BM * 16 : 0;
     static constexpr int kPkStageBytes = kNMat * (kMatBytes + kNvScBytes);
-    static constexpr int kPkStages = kTmemA ? ((GU && FMT == MOE_FMT_INT4_G128) ? 3 : 4) : 2;
-    static constexpr int kScStages = kFast ? G_EPI_WARPS : G_DQ_WARPS;   // readers of the int4 scale buffer
-    static constexpr int kBAtom = kNMax * 128;                      // one 64-wide K half of a B stage
-    static constexpr int kBStageBytes = 2 * kBAtom;
+    static constexpr int kPkMax = 12;                               // weight stages: as many as fit, up to this
+    static constexpr int kScStages = kI8 ? G_EPI_WARPS : G_DQ_WARPS;     // readers of the int4 scale buffer
+    static constexpr int kBAtom = (kI8 ? 16 : kNMax) * 128;         // 128 bytes of K for every B row
+    static constexpr int kBStageBytes = (kI8 ? 1 : 2) * kBAtom;     // K = 128 of 8-bit (i8) or 16-bit operands
     static constexpr int kBStages = 4;
-    static constexpr int kAStageCols = kNMat * 64;                  // K = 128 as 16-bit pairs, per matrix
+    static constexpr int kAColsK = kI8 ? 32 : 64;                   // TMEM columns of K = 128, one matrix
+    static constexpr int kAStageCols = kNMat * kAColsK;
     static constexpr int kAStages = 256 / kAStageCols;
-    static constexpr bool kMmaF16 = FMT == MOE_FMT_NVFP4 || kFast;
+    static constexpr int kChunkCols = kI8 ? 8 : 16;                 // TMEM columns of one 16-byte packed chunk
+    static constexpr bool kMmaF16 = FMT == MOE_FMT_NVFP4;
 };
+
+constexpr int G_DONE = 16;                                          // "stage done" barrier ring
 
 constexpr int G_NB_MAPS = 8;                                        // box heights 16, 32, ..., 128
 
@@ -123,9 +137,10 @@ struct GArgs {
     __nv_bfloat16* out;
     int32_t* status;
     float* partial;                  // split-K: fp32 partial sums [ksplit][nmat][rows][out_dim]
-    const float* zsum;               // fast int4: per-row, per-group constant [rows][in / 128]
+    const float* zsum;               // 8-bit int4: 8 * sum of the row's fixed-point values per group [rows][in / 128]
     int E, out_dim, in_dim, perm_out;
     int ksplit, rows;                // K slices per (m-tile, n-tile); activation rows of the problem
+    int npk;                         // weight stages in the shared-memory ring (2 .. kPkMax)
 };
 
 // ---------------------------------------------------------------------------
@@ -164,17 +179,14 @@ __device__ __forceinline__ void g_dq_nvfp4(const uint4 w, uint32_t sc2, uint32_t
     }
 }
 
-// fast int4: nibble pairs (p, p+4) of each word as f16 {1024 + u} (p = 0, 2)
-// or {1024 + 16u} (p = 1, 3); four logic ops and one shift per word.
-__device__ __forceinline__ void g_dq_int4_fast(const uint4 w, uint32_t (&o)[16]) {
+// 8-bit int4: the nibbles of each word as bytes, even nibbles first: the K
+// order within every 8 weights becomes 0, 2, 4, 6, 1, 3, 5, 7.
+__device__ __forceinline__ void g_dq_int4_i8(const uint4 w, uint32_t (&o)[16]) {
     const uint32_t ws[4] = {w.x, w.y, w.z, w.w};
 #pragma unroll
     for (int j = 0; j < 4; j++) {
-        const uint32_t hi = ws[j] >> 8;
-        o[j * 4 + 0] = (ws[j] & 0x000F000Fu) | 0x64006400u;
-        o[j * 4 + 1] = (ws[j] & 0x00F000F0u) | 0x64006400u;
-        o[j * 4 + 2] = (hi & 0x000F000Fu) | 0x64006400u;
-        o[j * 4 + 3] = (hi & 0x00F000F0u) | 0x64006400u;
+        o[2 * j] = ws[j] & 0x0F0F0F0Fu;
+        o[2 * j + 1] = (ws[j] >> 4) & 0x0F0F0F0Fu;
     }
 }
 
@@ -195,11 +207,10 @@ template <int FMT, bool GU>
 __global__ void __launch_bounds__(G_THREADS, 1) tc_grouped_gemm(const __grid_constant__ GArgs a) {
     using C = GCfg<FMT, GU>;
     extern __shared__ __align__(1024) uint8_t smem[];
-    __shared__ __align__(8) uint64_t pk_full[C::kPkStages], pk_empty[C::kPkStages];
-    __shared__ __align__(8) uint64_t b_full[C::kBStages], b_empty[C::kBStages];
-    __shared__ __align__(8) uint64_t a_full[C::kAStages], a_empty[C::kAStages];
+    __shared__ __align__(8) uint64_t pk_full[C::kPkMax], pk_empty[C::kPkMax];
+    __shared__ __align__(8) uint64_t b_full[C::kBStages], a_full[C::kAStages], done[G_DONE];
     __shared__ __align__(8) uint64_t sc_full[2], sc_empty[2];
-    __shared__ __align__(8) uint64_t acc_full[2], acc_empty[2], drain;
+    __shared__ __align__(8) uint64_t acc_full[2], acc_empty[C::kAccBufs], drain;
     __shared__ uint32_t s_tmem;
     __shared__ int s_active[kMaxE];
     __shared__ int s_prefix[kMaxE];
@@ -216,27 +227,27 @@ __global__ void __launch_bounds__(G_THREADS, 1) tc_grouped_gemm(const __grid_con
     const int NPS = kc / C::kPkK;                                   // weight stages per tile
     const int ngroups = in_dim / 128;
     const uint32_t sc_mat_bytes = uint32_t(G_BM * ngroups * 2);
+    const uint32_t NPK = uint32_t(a.npk);                          // weight stages in the ring
 
     if (tid == 0) {
-        for (int s = 0; s < C::kPkStages; s++) {
+        for (int s = 0; s < a.npk; s++) {
             asm volatile("mbarrier.init.shared::cta.b64 [%0], 1;" ::"r"(g_smem(&pk_full[s])));
-            asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(g_smem(&pk_empty[s])),
-                         "r"(C::kTmemA ? G_DQ_WARPS : 1));
+            if (C::kTmemA)     // BF16 weight stages are freed through the "stage done" ring
+                asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(g_smem(&pk_empty[s])), "r"(G_DQ_WARPS));
         }
-        for (int s = 0; s < C::kBStages; s++) {
+        for (int s = 0; s < C::kBStages; s++)
             asm volatile("mbarrier.init.shared::cta.b64 [%0], 1;" ::"r"(g_smem(&b_full[s])));
-            asm volatile("mbarrier.init.shared::cta.b64 [%0], 1;" ::"r"(g_smem(&b_empty[s])));
-        }
-        for (int s = 0; s < C::kAStages; s++) {
+        for (int s = 0; s < C::kAStages; s++)
             asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(g_smem(&a_full[s])), "r"(G_DQ_WARPS));
-            asm volatile("mbarrier.init.shared::cta.b64 [%0], 1;" ::"r"(g_smem(&a_empty[s])));
-        }
+        for (int s = 0; s < G_DONE; s++)
+            asm volatile("mbarrier.init.shared::cta.b64 [%0], 1;" ::"r"(g_smem(&done[s])));
         for (int s = 0; s < 2; s++) {
             asm volatile("mbarrier.init.shared::cta.b64 [%0], 1;" ::"r"(g_smem(&sc_full[s])));
             asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(g_smem(&sc_empty[s])), "r"(C::kScStages));
             asm volatile("mbarrier.init.shared::cta.b64 [%0], 1;" ::"r"(g_smem(&acc_full[s])));
-            asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(g_smem(&acc_empty[s])), "r"(G_EPI_WARPS));
         }
+        for (int s = 0; s < C::kAccBufs; s++)
+            asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(g_smem(&acc_empty[s])), "r"(G_EPI_WARPS));
         asm volatile("mbarrier.init.shared::cta.b64 [%0], 1;" ::"r"(g_smem(&drain)));
         asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
         s_abort = 0;
@@ -287,7 +298,7 @@ __global__ void __launch_bounds__(G_THREADS, 1) tc_grouped_gemm(const __grid_con
     const uint32_t tmem = s_tmem;
     const int ntiles = s_total, nact = s_nact;
     uint8_t* pk = smem + ((1024u - (g_smem(smem) & 1023u)) & 1023u);
-    uint8_t* bring = pk + C::kPkStages * C::kPkStageBytes;
+    uint8_t* bring = pk + NPK * C::kPkStageBytes;
     uint8_t* scbuf = bring + C::kBStages * C::kBStageBytes;         // int4: 2 buffers x kNMat x sc_mat_bytes
 
     auto tile_of = [&](int tile) {
@@ -339,9 +350,11 @@ __global__ void __launch_bounds__(G_THREADS, 1) tc_grouped_gemm(const __grid_con
             t++;
             bool ok = true;
             for (int ps = 0; ps < NPS; ps++, pc++) {
-                const int s = pc % C::kPkStages;
-                if (pc >= uint32_t(C::kPkStages) &&
-                    !g_wait_w(g_smem(&pk_empty[s]), ((pc / C::kPkStages) - 1) & 1, &s_abort, 32)) {
+                const int s = pc % NPK;
+                // 4-bit stages are freed by the dequantisation warps, BF16 ones by the MMA step
+                if (pc >= NPK && !(C::kTmemA ? g_wait_w(g_smem(&pk_empty[s]), ((pc / NPK) - 1) & 1, &s_abort, 32)
+                                             : g_wait_w(g_smem(&done[(pc - NPK) % G_DONE]), ((pc - NPK) / G_DONE) & 1,
+                                                        &s_abort, 32))) {
                     ok = false;
                     break;
                 }
@@ -374,8 +387,8 @@ __global__ void __launch_bounds__(G_THREADS, 1) tc_grouped_gemm(const __grid_con
         }
         // drain: every copy issued has landed before the CTA exits
         if (lane == 0) {
-            const uint32_t first = pc > uint32_t(C::kPkStages) ? pc - C::kPkStages : 0;
-            for (uint32_t n = first; n < pc; n++) g_drain_wait(g_smem(&pk_full[n % C::kPkStages]), (n / C::kPkStages) & 1);
+            const uint32_t first = pc > NPK ? pc - NPK : 0;
+            for (uint32_t n = first; n < pc; n++) g_drain_wait(g_smem(&pk_full[n % NPK]), (n / NPK) & 1);
             if (C::kInt4)
                 for (int n = t > 2 ? t - 2 : 0; n < t; n++) g_drain_wait(g_smem(&sc_full[n & 1]), (n >> 1) & 1);
         }
@@ -385,22 +398,27 @@ __global__ void __launch_bounds__(G_THREADS, 1) tc_grouped_gemm(const __grid_con
         uint32_t bc = 0;
         for (int tile = blockIdx.x; tile < ntiles && !s_abort; tile += gridDim.x) {
             const GTile T = tile_of(tile);
-            const int row0 = T.ebase + T.n0;
-            const CUtensorMap* map = &a.tm_b[T.bn / 16 - 1];
+            const int row0 = (C::kI8 ? 3 : 1) * (T.ebase + T.n0);      // i8: three digit rows per token
+            const CUtensorMap* map = &a.tm_b[C::kI8 ? 0 : T.bn / 16 - 1];
             bool ok = true;
             for (int ks = 0; ks < KS; ks++, bc++) {
                 const int s = bc % C::kBStages;
-                if (bc >= uint32_t(C::kBStages) &&
-                    !g_wait_w(g_smem(&b_empty[s]), ((bc / C::kBStages) - 1) & 1, &s_abort, 32)) {
+                if (bc >= uint32_t(C::kBStages) && !g_wait_w(g_smem(&done[(bc - C::kBStages) % G_DONE]),
+                                                             ((bc - C::kBStages) / G_DONE) & 1, &s_abort, 32)) {
                     ok = false;
                     break;
                 }
                 const uint32_t bar = g_smem(&b_full[s]);
                 const uint32_t st = g_smem(bring + s * C::kBStageBytes);
                 if (g_elect()) {
-                    g_expect(bar, uint32_t(T.bn) * 256u);
-                    g_tma2d(st, map, T.kbase + ks * C::kSK, row0, bar);
-                    g_tma2d(st + C::kBAtom, map, T.kbase + ks * C::kSK + 64, row0, bar);
+                    if (C::kI8) {
+                        g_expect(bar, uint32_t(C::kBAtom));
+                        g_tma2d(st, map, T.kbase + ks * C::kSK, row0, bar);
+                    } else {
+                        g_expect(bar, uint32_t(T.bn) * 256u);
+                        g_tma2d(st, map, T.kbase + ks * C::kSK, row0, bar);
+                        g_tma2d(st + C::kBAtom, map, T.kbase + ks * C::kSK + 64, row0, bar);
+                    }
                 }
                 __syncwarp();
             }
@@ -417,27 +435,28 @@ __global__ void __launch_bounds__(G_THREADS, 1) tc_grouped_gemm(const __grid_con
         int t = 0;
         for (int tile = blockIdx.x; tile < ntiles && !s_abort; tile += gridDim.x, t++) {
             const GTile T = tile_of(tile);
-            const uint32_t idesc = g_idesc(T.bn, C::kMmaF16);
+            const uint32_t idesc = C::kI8 ? g_idesc_i8(T.bn) : g_idesc(T.bn, C::kMmaF16);
             const int buf = t & 1;
             uint32_t d = tmem + buf * 128;
-            if (!C::kFast && t >= 2 && !g_wait_w(g_smem(&acc_empty[buf]), ((t >> 1) - 1) & 1, &s_abort)) {
+            if (!C::kI8 && t >= 2 && !g_wait_w(g_smem(&acc_empty[buf]), ((t >> 1) - 1) & 1, &s_abort)) {
                 fail();
                 break;
             }
             g_fence_after();
             bool ok = true;
             for (int ks = 0; ks < KS; ks++) {
-                const int sb = bc % C::kBStages, sa = ac % C::kAStages, sp = pc % C::kPkStages;
+                const int sb = bc % C::kBStages, sa = ac % C::kAStages, sp = pc % NPK;
                 if (!g_wait_w(g_smem(&b_full[sb]), (bc / C::kBStages) & 1, &s_abort)) { ok = false; break; }
                 if (C::kTmemA) {
                     if (!g_wait_w(g_smem(&a_full[sa]), (ac / C::kAStages) & 1, &s_abort)) { ok = false; break; }
                 } else {
-                    if (!g_wait_w(g_smem(&pk_full[sp]), (pc / C::kPkStages) & 1, &s_abort)) { ok = false; break; }
+                    if (!g_wait_w(g_smem(&pk_full[sp]), (pc / NPK) & 1, &s_abort)) { ok = false; break; }
                 }
-                if (C::kFast) {
-                    // every stage into a fresh buffer of the two; the epilogue frees it
-                    const int bi = ac & 1;
-                    if (ac >= 2 && !g_wait_w(g_smem(&acc_empty[bi]), ((ac >> 1) - 1) & 1, &s_abort)) { ok = false; break; }
+                if (C::kI8) {
+                    // every step into the next accumulator buffer; the epilogue frees it
+                    const int bi = bc % C::kAccBufs;
+                    if (bc >= uint32_t(C::kAccBufs) &&
+                        !g_wait_w(g_smem(&acc_empty[bi]), ((bc / C::kAccBufs) - 1) & 1, &s_abort)) { ok = false; break; }
                     d = tmem + bi * C::kAccCols;
                 }
                 g_fence_after();
@@ -446,27 +465,29 @@ __global__ void __launch_bounds__(G_THREADS, 1) tc_grouped_gemm(const __grid_con
                 const uint32_t a0 = g_smem(pk + sp * C::kPkStageBytes);
                 if (g_elect()) {
 #pragma unroll
-                    for (int k = 0; k < C::kSK / 16; k++) {
-                        const uint32_t acc = (k > 0 || (!C::kFast && ks > 0)) ? 1u : 0u;
+                    for (int k = 0; k < C::kSK / C::kMmaK; k++) {
+                        const uint32_t acc = (k > 0 || (!C::kI8 && ks > 0)) ? 1u : 0u;
                         const uint64_t bd = g_desc(b0 + (k >> 2) * C::kBAtom + (k & 3) * 32);
-                        if (C::kTmemA) {
+                        if (C::kI8) {
+                            g_mma_ts_i8(d, at + k * 8, bd, idesc, acc);
+                            if (GU) g_mma_ts_i8(d + C::kUpCol, at + C::kAColsK + k * 8, bd, idesc, acc);
+                        } else if (C::kTmemA) {
                             g_mma_ts(d, at + k * 8, bd, idesc, acc);
-                            if (GU) g_mma_ts(d + C::kUpCol, at + 64 + k * 8, bd, idesc, acc);
+                            if (GU) g_mma_ts(d + C::kUpCol, at + C::kAColsK + k * 8, bd, idesc, acc);
                         } else {
                             const uint32_t ak = a0 + (k >> 2) * (G_BM * 128) + (k & 3) * 32;
                             g_mma_ss(d, g_desc(ak), bd, idesc, acc);
                             if (GU) g_mma_ss(d + C::kUpCol, g_desc(ak + C::kMatBytes), bd, idesc, acc);
                         }
                     }
-                    g_commit(g_smem(&b_empty[sb]));
-                    g_commit(C::kTmemA ? g_smem(&a_empty[sa]) : g_smem(&pk_empty[sp]));
+                    g_commit(g_smem(&done[bc % G_DONE]));
                 }
                 __syncwarp();
                 bc++;
                 if (C::kTmemA) ac++; else pc++;
             }
             if (!ok) { fail(); break; }
-            if (!C::kFast && g_elect()) g_commit(g_smem(&acc_full[buf]));
+            if (!C::kI8 && g_elect()) g_commit(g_smem(&acc_full[buf]));
             __syncwarp();
         }
         // drain: every MMA issued has completed
@@ -474,14 +495,14 @@ __global__ void __launch_bounds__(G_THREADS, 1) tc_grouped_gemm(const __grid_con
         __syncwarp();
         if (lane == 0) g_drain_wait(g_smem(&drain), 0);
         __syncwarp();
-    } else if (warp >= 4 && warp < 8 && C::kFast) {
-        // ---------------- fast int4 epilogue: fold every K = 128 stage ----------------
+    } else if (warp >= 4 && warp < 8 && C::kI8) {
+        // ---------------- 8-bit int4 epilogue: fold every K = 128 step ----------------
         // Thread (warp w, lane l) owns weight row 32*(w%4) + l of the tile; lane
-        // j < 16 also holds token row j's group constant and row factor.
+        // j < kNMax also holds token j's group term and row factor.  Token j's
+        // digit sums are accumulator columns 3j (d2), 3j+1 (d1), 3j+2 (d0).
         const int q = warp & 3;
         const uint32_t lane_addr = uint32_t(q * 32) << 16;
         const int r = q * 32 + lane;
-        const int nj = lane & 15;
         uint32_t ac = 0;
         int t = 0;
         bool ok = true;
@@ -489,18 +510,18 @@ __global__ void __launch_bounds__(G_THREADS, 1) tc_grouped_gemm(const __grid_con
             const GTile T = tile_of(tile);
             const int f = T.m0 + r;
             const int rbase = T.ebase + T.n0;
-            const bool live = nj < T.nval;
+            const bool live = lane < T.nval;
             const int b = t & 1;
             if (!g_wait(g_smem(&sc_full[b]), (t >> 1) & 1, &s_abort, 64)) { ok = false; break; }
             const __nv_bfloat16* sc0 = reinterpret_cast<const __nv_bfloat16*>(scbuf + b * C::kNMat * sc_mat_bytes) + r * ngroups;
             const __nv_bfloat16* sc1 = sc0 + G_BM * ngroups;
-            const float* zrow = a.zsum + size_t(rbase + (live ? nj : 0)) * ngroups;
-            float tg[16], tu[16];
+            const float* zrow = a.zsum + size_t(rbase + (live ? lane : 0)) * ngroups;
+            float tg[C::kNMax], tu[C::kNMax];
 #pragma unroll
-            for (int j = 0; j < 16; j++) tg[j] = tu[j] = 0.f;
+            for (int j = 0; j < C::kNMax; j++) tg[j] = tu[j] = 0.f;
             for (int ks = 0; ks < KS; ks++, ac++) {
-                const int sa = ac % C::kAStages, bi = ac & 1;
-                if (!g_wait(g_smem(&a_empty[sa]), (ac / C::kAStages) & 1, &s_abort)) { ok = false; break; }
+                const int bi = ac % C::kAccBufs;
+                if (!g_wait(g_smem(&done[ac % G_DONE]), (ac / G_DONE) & 1, &s_abort)) { ok = false; break; }
                 g_fence_after();
                 uint32_t g[16], u[16];
                 g_ld16(tmem + lane_addr + bi * C::kAccCols, g);
@@ -508,16 +529,22 @@ __global__ void __launch_bounds__(G_THREADS, 1) tc_grouped_gemm(const __grid_con
                 g_ld_wait();
                 g_fence_before();
                 __syncwarp();
-                if (lane == 0) g_arrive(g_smem(&acc_empty[bi]));      // the buffer takes stage ac + 2
+                if (lane == 0) g_arrive(g_smem(&acc_empty[bi]));
                 const int grp = T.kbase / 128 + ks;
                 const float z = live ? zrow[grp] : 0.f;
                 const float s0 = __bfloat162float(sc0[grp]);
                 const float s1 = GU ? __bfloat162float(sc1[grp]) : 0.f;
 #pragma unroll
-                for (int j = 0; j < 16; j++) {
+                for (int j = 0; j < C::kNMax; j++) {
                     const float zj = __shfl_sync(0xffffffffu, z, j);
-                    tg[j] = fmaf(s0, __uint_as_float(g[j]) - zj, tg[j]);
-                    if (GU) tu[j] = fmaf(s1, __uint_as_float(u[j]) - zj, tu[j]);
+                    const float vg = fmaf(float(int(g[3 * j])), 65536.f,
+                                          fmaf(float(int(g[3 * j + 1])), 256.f, float(int(g[3 * j + 2])))) - zj;
+                    tg[j] = fmaf(s0, vg, tg[j]);
+                    if (GU) {
+                        const float vu = fmaf(float(int(u[3 * j])), 65536.f,
+                                              fmaf(float(int(u[3 * j + 1])), 256.f, float(int(u[3 * j + 2])))) - zj;
+                        tu[j] = fmaf(s1, vu, tu[j]);
+                    }
                 }
             }
             if (!ok) break;
@@ -525,11 +552,11 @@ __global__ void __launch_bounds__(G_THREADS, 1) tc_grouped_gemm(const __grid_con
             if (lane == 0) g_arrive(g_smem(&sc_empty[b]));
             float rowf = 1.f;
             if (live) {
-                rowf = a.act_scale[rbase + nj];
-                if (!GU && a.topk_w) rowf *= a.topk_w[a.row_slot[rbase + nj]];
+                rowf = a.act_scale[rbase + lane];
+                if (!GU && a.topk_w) rowf *= a.topk_w[a.row_slot[rbase + lane]];
             }
 #pragma unroll
-            for (int j = 0; j < 16; j++) {
+            for (int j = 0; j < C::kNMax; j++) {
                 const float fj = __shfl_sync(0xffffffffu, rowf, j);
                 if (j < T.nval) {
                     float v;
@@ -618,7 +645,7 @@ __global__ void __launch_bounds__(G_THREADS, 1) tc_grouped_gemm(const __grid_con
         const int q = warp & 3, hsel = (warp - 8) >> 2;
         const int r = q * 32 + lane;                   // weight row within the tile
         const uint32_t lane_addr = uint32_t(q * 32) << 16;
-        const uint32_t colw = 256 + (GU ? hsel * 64 : hsel * 32);
+        const uint32_t colw = 256 + (GU ? hsel * C::kAColsK : hsel * (C::kAColsK / 2));
         uint32_t pc = 0;
         int t = 0;
         bool ok = true;
@@ -630,8 +657,8 @@ __global__ void __launch_bounds__(G_THREADS, 1) tc_grouped_gemm(const __grid_con
                 scrow = scbuf + b * C::kNMat * sc_mat_bytes + (GU ? hsel * sc_mat_bytes : 0) + r * ngroups * 2;
             }
             for (int ps = 0; ps < NPS && ok; ps++, pc++) {
-                const int s = pc % C::kPkStages;
-                if (!g_wait(g_smem(&pk_full[s]), (pc / C::kPkStages) & 1, &s_abort)) { ok = false; break; }
+                const int s = pc % NPK;
+                if (!g_wait(g_smem(&pk_full[s]), (pc / NPK) & 1, &s_abort)) { ok = false; break; }
                 const uint8_t* st = pk + s * C::kPkStageBytes;
                 const uint8_t* wt = st + (GU ? hsel * C::kMatBytes : 0);
                 uint32_t scw = 0;                      // int4: bf16 scales of groups 2ps (low) and 2ps+1 (high)
@@ -650,8 +677,8 @@ __global__ void __launch_bounds__(G_THREADS, 1) tc_grouped_gemm(const __grid_con
                     constexpr int i = decltype(ic)::value, j = i / kPer, l = i % kPer;
                     const int c = 4 * j + (GU ? l : 2 * hsel + l);
                     const uint4 w = *reinterpret_cast<const uint4*>(wt + g_swz(r, c));
-                    if (FMT == FMT_INT4_FAST) {
-                        g_dq_int4_fast(w, o[i % kNBuf]);
+                    if (FMT == FMT_INT4_I8) {
+                        g_dq_int4_i8(w, o[i % kNBuf]);
                     } else if (FMT == MOE_FMT_INT4_G128) {
                         g_dq_int4(w, scw >> (16 * j), o[i % kNBuf]);
                     } else {
@@ -668,14 +695,15 @@ __global__ void __launch_bounds__(G_THREADS, 1) tc_grouped_gemm(const __grid_con
                     if (l == 0) {
                         const uint32_t acn = pc * 2 + j;             // A stage index in this CTA's stream
                         sa = acn % C::kAStages;
-                        if (acn >= uint32_t(C::kAStages) &&
-                            !g_wait(g_smem(&a_empty[sa]), ((acn / C::kAStages) - 1) & 1, &s_abort)) {
+                        if (acn >= uint32_t(C::kAStages) && !g_wait(g_smem(&done[(acn - C::kAStages) % G_DONE]),
+                                                                    ((acn - C::kAStages) / G_DONE) & 1, &s_abort)) {
                             ok = false;
                             return;
                         }
                         g_fence_after();
                     }
-                    g_st16(tmem + lane_addr + colw + sa * C::kAStageCols + l * 16, o[i % kNBuf]);
+                    if constexpr (C::kI8) g_st8(tmem + lane_addr + colw + sa * C::kAStageCols + l * C::kChunkCols, o[i % kNBuf]);
+                    else g_st16(tmem + lane_addr + colw + sa * C::kAStageCols + l * C::kChunkCols, o[i % kNBuf]);
                     if constexpr (i + 1 < kChunks) dq(std::integral_constant<int, i + 1>{});
                     if (l == kPer - 1) {
                         g_st_wait();
@@ -709,11 +737,11 @@ __global__ void __launch_bounds__(G_THREADS, 1) tc_grouped_gemm(const __grid_con
 //   mode 2: f16 times 2^-e (e >= 0 least with |x| * 2^-e <= 16384), row scale 2^e.
 // One warp per row.
 // ---------------------------------------------------------------------------
-//   mode 3 (fast int4): f16 in the pair order, times 2^-e, with the elements
-//          paired with odd nibbles (x1, x5, x3, x7 of every 8) divided by 16;
-//          zsum[row][g] = sum over group g of (1024 + 8c) * value, c = 16 at
-//          the divided positions and 1 elsewhere: the part of the MMA sum
-//          that is not q * x * 2^-e.
+//   mode 3 (8-bit int4): X = rint(x * 2^c), c the row's exponent that puts
+//          max |X| in [2^21, 2^22), as signed digits X = 65536 d2 + 256 d1 + d0
+//          in rows 3 row (d2), 3 row + 1 (d1), 3 row + 2 (d0) of int8 dst, in
+//          the K order 0, 2, 4, 6, 1, 3, 5, 7 of every 8; scale[row] = 2^-c;
+//          zsum[row][g] = 8 * sum of X over group g (the u - 8 offset).
 __global__ void __launch_bounds__(256) g_prep(const __nv_bfloat16* __restrict__ src, int in_dim,
                                               const int32_t* __restrict__ row_slot, int top_k, int by_token,
                                               int rows, int mode, uint16_t* __restrict__ dst,
@@ -745,29 +773,40 @@ __global__ void __launch_bounds__(256) g_prep(const __nv_bfloat16* __restrict__ 
             amax = fmaxf(amax, fmaxf(fmaxf(fabsf(bf16_lo(v.z)), fabsf(bf16_hi(v.z))), fmaxf(fabsf(bf16_lo(v.w)), fabsf(bf16_hi(v.w)))));
         }
         for (int o = 16; o > 0; o >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, o));
-        int e = 0;
-        while (e < 126 && ldexpf(amax, -e) > 16384.f) e++;
-        const float down = ldexpf(1.f, -e), down16 = down * 0.0625f;
+        int ex = 0;
+        frexpf(amax, &ex);                                  // amax < 2^ex
+        const int c = amax > 0.f ? min(22 - ex, 126) : 0;   // |x| 2^c < 2^22
+        uint8_t* d8 = reinterpret_cast<uint8_t*>(dst) + size_t(row) * 3 * in_dim;
         // 16 pieces of 8 make a group of 128: lanes 0-15 and 16-31 take one group each per pass
         for (int i0 = 0; i0 < n16; i0 += 32) {
             const int i = i0 + lane;
-            float z = 0.f;
+            int zs = 0;
             if (i < n16) {
                 const uint4 v = s[i];
-                __half2 h[4];
-                h[0] = __floats2half2_rn(bf16_lo(v.x) * down, bf16_lo(v.z) * down);       // (x0, x4)
-                h[1] = __floats2half2_rn(bf16_hi(v.x) * down16, bf16_hi(v.z) * down16);   // (x1, x5) / 16
-                h[2] = __floats2half2_rn(bf16_lo(v.y) * down, bf16_lo(v.w) * down);       // (x2, x6)
-                h[3] = __floats2half2_rn(bf16_hi(v.y) * down16, bf16_hi(v.w) * down16);   // (x3, x7) / 16
-                d[i] = *reinterpret_cast<uint4*>(h);
-                const float2 a0 = __half22float2(h[0]), a1 = __half22float2(h[1]);
-                const float2 a2 = __half22float2(h[2]), a3 = __half22float2(h[3]);
-                z = 1032.f * (a0.x + a0.y + a2.x + a2.y) + 1152.f * (a1.x + a1.y + a3.x + a3.y);
+                // the K order of the weight bytes: 0, 2, 4, 6, 1, 3, 5, 7
+                const float xs[8] = {bf16_lo(v.x), bf16_lo(v.y), bf16_lo(v.z), bf16_lo(v.w),
+                                     bf16_hi(v.x), bf16_hi(v.y), bf16_hi(v.z), bf16_hi(v.w)};
+                uint32_t p2[2] = {0u, 0u}, p1[2] = {0u, 0u}, p0[2] = {0u, 0u};
+#pragma unroll
+                for (int e = 0; e < 8; e++) {
+                    const int X = __float2int_rn(ldexpf(xs[e], c));
+                    zs += X;
+                    const int d0 = ((X + 128) & 255) - 128;          // signed digits in [-128, 127]
+                    const int X1 = (X - d0) >> 8;
+                    const int d1 = ((X1 + 128) & 255) - 128;
+                    const int d2 = (X1 - d1) >> 8;
+                    p0[e >> 2] |= uint32_t(d0 & 255) << (8 * (e & 3));
+                    p1[e >> 2] |= uint32_t(d1 & 255) << (8 * (e & 3));
+                    p2[e >> 2] |= uint32_t(d2 & 255) << (8 * (e & 3));
+                }
+                *reinterpret_cast<uint2*>(d8 + size_t(i) * 8) = make_uint2(p2[0], p2[1]);
+                *reinterpret_cast<uint2*>(d8 + in_dim + size_t(i) * 8) = make_uint2(p1[0], p1[1]);
+                *reinterpret_cast<uint2*>(d8 + 2 * size_t(in_dim) + size_t(i) * 8) = make_uint2(p0[0], p0[1]);
             }
-            for (int o = 8; o > 0; o >>= 1) z += __shfl_xor_sync(0xffffffffu, z, o);
-            if ((lane & 15) == 0 && i < n16) zsum[size_t(row) * (in_dim / 128) + i / 16] = z;
+            for (int o = 8; o > 0; o >>= 1) zs += __shfl_xor_sync(0xffffffffu, zs, o);
+            if ((lane & 15) == 0 && i < n16) zsum[size_t(row) * (in_dim / 128) + i / 16] = 8.f * float(zs);
         }
-        if (lane == 0) scale[row] = ldexpf(1.f, e);
+        if (lane == 0) scale[row] = ldexpf(1.f, -c);
     } else {
         float amax = 0.f;
         for (int i = lane; i < n16; i += 32) {
@@ -837,27 +876,34 @@ __global__ void __launch_bounds__(256) g_splitk_finish(const float* __restrict__
 // Host side
 // ---------------------------------------------------------------------------
 template <int FMT, bool GU>
-static size_t g_smem_bytes(int in_dim) {
+static size_t g_smem_bytes(int in_dim, int npk) {
     using C = GCfg<FMT, GU>;
-    size_t b = size_t(C::kPkStages) * C::kPkStageBytes + size_t(C::kBStages) * C::kBStageBytes + 1024;
+    size_t b = size_t(npk) * C::kPkStageBytes + size_t(C::kBStages) * C::kBStageBytes + 1024;
     if (C::kInt4) b += 2 * size_t(C::kNMat) * G_BM * (in_dim / 128) * 2;
     return b;
 }
 
 template <int FMT, bool GU>
 static int g_launch(const GArgs& a, cudaStream_t s) {
+    using C = GCfg<FMT, GU>;
     auto k = tc_grouped_gemm<FMT, GU>;
-    const size_t smem = g_smem_bytes<FMT, GU>(a.in_dim);
     int dev = 0, sms = 0, optin = 0;
     if (cudaGetDevice(&dev) != cudaSuccess) return MOE_ERR_CUDA;
     if (cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) return MOE_ERR_CUDA;
     if (cudaDeviceGetAttribute(&optin, cudaDevAttrMaxSharedMemoryPerBlockOptin, dev) != cudaSuccess) return MOE_ERR_CUDA;
     cudaFuncAttributes fa{};
     if (cudaFuncGetAttributes(&fa, k) != cudaSuccess) return MOE_ERR_CUDA;
-    if (smem + fa.sharedSizeBytes > size_t(optin)) return MOE_ERR_UNSUPPORTED;
+    // the weight stream wants as many bytes in flight as shared memory holds
+    const size_t room = size_t(optin) - std::min(size_t(optin), fa.sharedSizeBytes);
+    const size_t fixed = g_smem_bytes<FMT, GU>(a.in_dim, 0);
+    const int npk = fixed < room ? int(std::min<size_t>(C::kPkMax, (room - fixed) / C::kPkStageBytes)) : 0;
+    if (npk < 2) return MOE_ERR_UNSUPPORTED;
+    GArgs args = a;
+    args.npk = npk;
+    const size_t smem = g_smem_bytes<FMT, GU>(a.in_dim, npk);
     if (cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem)) != cudaSuccess)
         return MOE_ERR_CUDA;
-    return launch_pdl(k, dim3(sms), dim3(G_THREADS), smem, s, a) == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
+    return launch_pdl(k, dim3(sms), dim3(G_THREADS), smem, s, args) == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
 }
 
 #define G_TRY(x)                       \
@@ -880,14 +926,15 @@ int launch_grouped_gemm(const GemvProblem& p, bool gateup, int rows, const GemmB
 
     const int in = p.in_dim, out = p.out_dim, E = p.E;
     const bool nv = p.fmt == MOE_FMT_NVFP4, i4 = p.fmt == MOE_FMT_INT4_G128;
-    const bool fast = i4 && buf.fast;
-    if (fast && (!buf.zbuf || !buf.scale_buf || !buf.act_buf || buf.perm_out || ksplit > 1)) return MOE_ERR_UNSUPPORTED;
-    // activation operand rows [rows, in]: bf16 (f16 for NVFP4) in the kernel's order
+    const bool i8 = i4 && buf.i8;
+    if (i8 && (!buf.zbuf || !buf.scale_buf || !buf.act_buf || buf.perm_out || ksplit > 1)) return MOE_ERR_UNSUPPORTED;
+    // activation operand rows [rows, in]: bf16 (f16 for NVFP4) in the kernel's order; 8-bit int4: three
+    // int8 digit rows per row
     const void* bsrc = p.act;
     const float* ascale = nullptr;
-    if (!buf.act_ready || nv || fast) {
+    if (!buf.act_ready || nv || i8) {
         if (!buf.act_buf || (nv && !buf.scale_buf)) return MOE_ERR_WORKSPACE;
-        const int mode = fast ? 3 : nv ? 2 : (i4 ? 1 : 0);
+        const int mode = i8 ? 3 : nv ? 2 : (i4 ? 1 : 0);
         if (launch_pdl(g_prep, dim3((rows * 32 + 255) / 256), dim3(256), 0, s, p.act, in, p.row_slot, p.top_k,
                        p.act_by_token, rows, mode, reinterpret_cast<uint16_t*>(buf.act_buf), buf.scale_buf,
                        buf.zbuf) != cudaSuccess)
@@ -910,8 +957,11 @@ int launch_grouped_gemm(const GemvProblem& p, bool gateup, int rows, const GemmB
         G_TRY(g_map(&a.tm_s0, false, p.s0, in / 16, wrows, uint64_t(in) / 16, 16, 128, false));
         if (gateup) G_TRY(g_map(&a.tm_s1, false, p.s1, in / 16, wrows, uint64_t(in) / 16, 16, 128, false));
     }
-    for (int i = 0; i < G_NB_MAPS; i++)
-        G_TRY(g_map(&a.tm_b[i], true, bsrc, in, uint64_t(rows), uint64_t(in) * 2, 64, uint32_t(16 * (i + 1)), true));
+    if (i8)
+        G_TRY(g_map(&a.tm_b[0], false, bsrc, in, uint64_t(rows) * 3, uint64_t(in), 128, 16, true));
+    else
+        for (int i = 0; i < G_NB_MAPS; i++)
+            G_TRY(g_map(&a.tm_b[i], true, bsrc, in, uint64_t(rows), uint64_t(in) * 2, 64, uint32_t(16 * (i + 1)), true));
     a.sc0 = reinterpret_cast<const uint8_t*>(p.s0);
     a.sc1 = reinterpret_cast<const uint8_t*>(p.s1);
     a.g0 = p.g0;
@@ -931,7 +981,7 @@ int launch_grouped_gemm(const GemvProblem& p, bool gateup, int rows, const GemmB
     a.rows = rows;
     a.zsum = buf.zbuf;
 
-    if (fast) return gateup ? g_launch<FMT_INT4_FAST, true>(a, s) : g_launch<FMT_INT4_FAST, false>(a, s);
+    if (i8) return gateup ? g_launch<FMT_INT4_I8, true>(a, s) : g_launch<FMT_INT4_I8, false>(a, s);
     if (i4) return gateup ? g_launch<MOE_FMT_INT4_G128, true>(a, s) : g_launch<MOE_FMT_INT4_G128, false>(a, s);
     if (nv) return gateup ? g_launch<MOE_FMT_NVFP4, true>(a, s) : g_launch<MOE_FMT_NVFP4, false>(a, s);
     const int rc = gateup ? g_launch<MOE_FMT_BF16, true>(a, s) : g_launch<MOE_FMT_BF16, false>(a, s);

@@ -60,12 +60,19 @@ inline size_t permute_scratch(int T, int k, int E) {
 inline size_t prep_scratch(int rows, int in_dim) {
     return align256(size_t(rows) * (in_dim / 32) * 4) + align256(size_t(rows) * in_dim * 2);
 }
+// int4 routed problems with at most this many rows take the 8-bit int4 GEMM
+constexpr int kI8Int4MaxRows = 512;
+// GEMM pre-pass output: row scales [rows] fp32, group sums [rows][in/128] fp32,
+// then the gathered rows: 16-bit [rows][in], or three int8 digit rows per row
+// when the 8-bit int4 GEMM can take the problem.
+inline size_t gemm_prep_bytes(int rows, int in_dim) {
+    return align256(size_t(rows) * 4) + align256(size_t(rows) * (in_dim / 128) * 4) +
+           align256(size_t(rows) * in_dim * (rows <= kI8Int4MaxRows ? 3 : 2));
+}
 // Step-level scratch of a grouped call: tile metadata, then the pre-pass of
-// act_rows rows (GEMV), or row scales, per-group constants and the gathered
-// rows (GEMM).
+// act_rows rows (GEMV or GEMM).
 inline size_t grouped_scratch(int E, int act_rows, int in_dim) {
-    return align256(size_t(E + 2) * 16) + prep_scratch(act_rows, in_dim) + align256(size_t(act_rows) * (in_dim / 128) * 4) +
-           1024;
+    return align256(size_t(E + 2) * 16) + std::max(prep_scratch(act_rows, in_dim), gemm_prep_bytes(act_rows, in_dim));
 }
 
 // The BF16 shared expert at a small batch has few (m, n) tiles (12 for gate/up,
@@ -101,8 +108,8 @@ inline WsLayout ws_layout(int T, int H, int E, int F, int k) {
     L.y_perm = o;     o = align256(o + R * size_t(H) * 2);
     L.ys = o;         o = align256(o + size_t(T) * H * 2);
     L.tiles = o;      o = align256(o + size_t(E + 2) * 4 * 4);
-    L.prep = o;       o = align256(o + std::max(prep_scratch(T, H), prep_scratch(int(R), F)) +
-                               align256(R * size_t(std::max(H, F) / 128) * 4) + 1024);
+    L.prep = o;       o = align256(o + std::max(std::max(prep_scratch(T, H), prep_scratch(int(R), F)),
+                                            std::max(gemm_prep_bytes(int(R), H), gemm_prep_bytes(int(R), F))));
     L.shpart = o;     o = align256(o + std::max(split_bytes(shared_ksplit(1, MOE_FMT_BF16, true, T, H), true, T, F),
                                                 split_bytes(shared_ksplit(1, MOE_FMT_BF16, false, T, F), false, T, H)));
     L.total = o;
@@ -209,12 +216,9 @@ struct GemmBuffers {
     int perm_out;
     int ksplit;          // > 1: split K into this many slices (BF16 only); fp32 partial sums go to partial
     float* partial;      // split_bytes(...) bytes
-    int fast;            // int4 with 16-row token tiles and per-group accumulation (small batches)
-    float* zbuf;         // fast: per-row, per-group constants [rows][in / 128]
+    int i8;              // int4 on the 8-bit MMA with per-group accumulation (small batches)
+    float* zbuf;         // i8: 8 * group sums of the fixed-point rows [rows][in / 128]
 };
-
-// int4 routed problems with at most this many rows take the fast int4 GEMM
-constexpr int kFastInt4MaxRows = 512;
 
 
 // Prefill-shaped grouped GEMM (tcgen05) for one problem; rows: activation
