@@ -82,10 +82,11 @@ constexpr int G_EPI_WARPS = 4;
 // instruction).  The pre-pass writes each activation row as a 24-bit fixed
 // point X = x * 2^c (c per row, |X| < 2^22) in three signed 8-bit digits,
 // X = 65536 d2 + 256 d1 + d0, one B operand row per digit (token j's digits
-// are rows 3j, 3j+1, 3j+2 of the tile: five tokens fill N = 16).  Each K = 128
-// step (one scale group) accumulates from zero; the epilogue warps combine
-// the digit sums, subtract 8 * sum(X) over the group (the u - 8 offset) and
-// fold scale * value into fp32 totals.  The group scale and the offset leave
+// are rows 3j, 3j+1, 3j+2 of the tile: five tokens fill N = 16).  An MMA step
+// covers K = 256; each of its two scale groups accumulates from zero into its
+// own columns.  The epilogue warps combine the digit sums, subtract
+// 8 * sum(X) over the group (the u - 8 offset) and fold scale * value into
+// fp32 totals.  The group scale and the offset leave
 // the per-weight work, and the accumulation itself is exact.  Internal
 // format value.
 constexpr int FMT_INT4_I8 = 3;
@@ -97,10 +98,11 @@ struct GCfg {
     static constexpr bool kTmemA = FMT != MOE_FMT_BF16;
     static constexpr int kNMat = GU ? 2 : 1;
     static constexpr int kNMax = kI8 ? 5 : (GU ? 64 : 128);        // token rows per tile
-    static constexpr int kUpCol = kI8 ? 16 : 64;                    // up accumulator within a buffer
-    static constexpr int kAccCols = kI8 ? kNMat * 16 : 128;         // one accumulator buffer
-    static constexpr int kAccBufs = kI8 ? 4 : 2;                    // accumulator buffers in [0, 256)
-    static constexpr int kSK = 128;                                 // K per MMA stage
+    static constexpr int kUpCol = 64;                               // 16-bit paths: up accumulator within a buffer
+    static constexpr int kSK = kI8 ? 256 : 128;                     // K per MMA stage
+    static constexpr int kGroups = kSK / 128;                       // i8: scale groups per MMA stage
+    static constexpr int kAccCols = kI8 ? kGroups * kNMat * 16 : 128;   // one accumulator buffer
+    static constexpr int kAccBufs = 256 / kAccCols;                 // accumulator buffers in [0, 256)
     static constexpr int kMmaK = kI8 ? 32 : 16;                     // K per MMA instruction
     static constexpr int kPkK = kTmemA ? 256 : 128;                 // K per weight stage
     static constexpr int kMatBytes = kTmemA ? G_BM * 128 : G_BM * 256;   // one matrix of a weight stage
@@ -109,16 +111,18 @@ struct GCfg {
     static constexpr int kPkMax = 12;                               // weight stages: as many as fit, up to this
     static constexpr int kScStages = kI8 ? G_EPI_WARPS : G_DQ_WARPS;     // readers of the int4 scale buffer
     static constexpr int kBAtom = (kI8 ? 16 : kNMax) * 128;         // 128 bytes of K for every B row
-    static constexpr int kBStageBytes = (kI8 ? 1 : 2) * kBAtom;     // K = 128 of 8-bit (i8) or 16-bit operands
-    static constexpr int kBStages = 4;
-    static constexpr int kAColsK = kI8 ? 32 : 64;                   // TMEM columns of K = 128, one matrix
+    static constexpr int kBStageBytes = 2 * kBAtom;                 // K = 256 of 8-bit (i8) or 128 of 16-bit operands
+    static constexpr int kBStages = kI8 ? 6 : 4;                    // i8 stages are small; cover the copy latency
+    static constexpr int kAColsK = 64;                              // TMEM columns of one matrix's A stage
     static constexpr int kAStageCols = kNMat * kAColsK;
     static constexpr int kAStages = 256 / kAStageCols;
+    static constexpr int kAPerPk = kPkK / kSK;                      // A stages per weight stage (2, or 1 for i8)
     static constexpr int kChunkCols = kI8 ? 8 : 16;                 // TMEM columns of one 16-byte packed chunk
     static constexpr bool kMmaF16 = FMT == MOE_FMT_NVFP4;
 };
 
 constexpr int G_DONE = 16;                                          // "stage done" barrier ring
+constexpr int G_SC_MAX = 8;                                         // int4 scale buffers (one tile each)
 
 constexpr int G_NB_MAPS = 8;                                        // box heights 16, 32, ..., 128
 
@@ -137,10 +141,11 @@ struct GArgs {
     __nv_bfloat16* out;
     int32_t* status;
     float* partial;                  // split-K: fp32 partial sums [ksplit][nmat][rows][out_dim]
-    const float* zsum;               // 8-bit int4: 8 * sum of the row's fixed-point values per group [rows][in / 128]
+    const float* zsum;               // 8-bit int4: 8 * sum of the row's fixed-point values per group [rows][zst]
     int E, out_dim, in_dim, perm_out;
     int ksplit, rows;                // K slices per (m-tile, n-tile); activation rows of the problem
     int npk;                         // weight stages in the shared-memory ring (2 .. kPkMax)
+    int nsc;                         // int4 scale buffers (2 .. G_SC_MAX)
 };
 
 // ---------------------------------------------------------------------------
@@ -209,7 +214,7 @@ __global__ void __launch_bounds__(G_THREADS, 1) tc_grouped_gemm(const __grid_con
     extern __shared__ __align__(1024) uint8_t smem[];
     __shared__ __align__(8) uint64_t pk_full[C::kPkMax], pk_empty[C::kPkMax];
     __shared__ __align__(8) uint64_t b_full[C::kBStages], a_full[C::kAStages], done[G_DONE];
-    __shared__ __align__(8) uint64_t sc_full[2], sc_empty[2];
+    __shared__ __align__(8) uint64_t sc_full[G_SC_MAX], sc_empty[G_SC_MAX];
     __shared__ __align__(8) uint64_t acc_full[2], acc_empty[C::kAccBufs], drain;
     __shared__ uint32_t s_tmem;
     __shared__ int s_active[kMaxE];
@@ -227,7 +232,12 @@ __global__ void __launch_bounds__(G_THREADS, 1) tc_grouped_gemm(const __grid_con
     const int NPS = kc / C::kPkK;                                   // weight stages per tile
     const int ngroups = in_dim / 128;
     const uint32_t sc_mat_bytes = uint32_t(G_BM * ngroups * 2);
+    const int zst = ((ngroups + 3) & ~3);                           // i8: group-sum row stride
+    // one scale buffer: the int4 scales of the tile's rows (per matrix), then
+    // (i8) the group sums of the tile's tokens
+    const uint32_t sc_buf_bytes = C::kNMat * sc_mat_bytes + (C::kI8 ? uint32_t(C::kNMax * zst * 4) : 0u);
     const uint32_t NPK = uint32_t(a.npk);                          // weight stages in the ring
+    const int NSC = a.nsc;                                          // int4 scale buffers, one tile each
 
     if (tid == 0) {
         for (int s = 0; s < a.npk; s++) {
@@ -241,11 +251,12 @@ __global__ void __launch_bounds__(G_THREADS, 1) tc_grouped_gemm(const __grid_con
             asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(g_smem(&a_full[s])), "r"(G_DQ_WARPS));
         for (int s = 0; s < G_DONE; s++)
             asm volatile("mbarrier.init.shared::cta.b64 [%0], 1;" ::"r"(g_smem(&done[s])));
-        for (int s = 0; s < 2; s++) {
+        for (int s = 0; s < a.nsc; s++) {
             asm volatile("mbarrier.init.shared::cta.b64 [%0], 1;" ::"r"(g_smem(&sc_full[s])));
             asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(g_smem(&sc_empty[s])), "r"(C::kScStages));
-            asm volatile("mbarrier.init.shared::cta.b64 [%0], 1;" ::"r"(g_smem(&acc_full[s])));
         }
+        for (int s = 0; s < 2; s++)
+            asm volatile("mbarrier.init.shared::cta.b64 [%0], 1;" ::"r"(g_smem(&acc_full[s])));
         for (int s = 0; s < C::kAccBufs; s++)
             asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(g_smem(&acc_empty[s])), "r"(G_EPI_WARPS));
         asm volatile("mbarrier.init.shared::cta.b64 [%0], 1;" ::"r"(g_smem(&drain)));
@@ -299,7 +310,7 @@ __global__ void __launch_bounds__(G_THREADS, 1) tc_grouped_gemm(const __grid_con
     const int ntiles = s_total, nact = s_nact;
     uint8_t* pk = smem + ((1024u - (g_smem(smem) & 1023u)) & 1023u);
     uint8_t* bring = pk + NPK * C::kPkStageBytes;
-    uint8_t* scbuf = bring + C::kBStages * C::kBStageBytes;         // int4: 2 buffers x kNMat x sc_mat_bytes
+    uint8_t* scbuf = bring + C::kBStages * C::kBStageBytes;         // int4: NSC buffers of sc_buf_bytes
 
     auto tile_of = [&](int tile) {
         int lo = 0, hi = nact - 1;
@@ -336,14 +347,17 @@ __global__ void __launch_bounds__(G_THREADS, 1) tc_grouped_gemm(const __grid_con
             const GTile T = tile_of(tile);
             const int row0 = T.e * a.out_dim + T.m0;
             if (C::kInt4) {
-                const int b = t & 1;
-                if (t >= 2 && !g_wait_w(g_smem(&sc_empty[b]), ((t >> 1) - 1) & 1, &s_abort, 64)) { fail(); break; }
+                const int b = t % NSC;
+                if (t >= NSC && !g_wait_w(g_smem(&sc_empty[b]), ((t / NSC) - 1) & 1, &s_abort, 64)) { fail(); break; }
                 const uint32_t bar = g_smem(&sc_full[b]);
-                uint8_t* dst = scbuf + b * C::kNMat * sc_mat_bytes;
+                uint8_t* dst = scbuf + b * sc_buf_bytes;
+                const uint32_t zbytes = C::kI8 ? uint32_t(T.nval * zst * 4) : 0u;
                 if (g_elect()) {
-                    g_expect(bar, sc_mat_bytes * C::kNMat);
+                    g_expect(bar, sc_mat_bytes * C::kNMat + zbytes);
                     g_bulk(g_smem(dst), a.sc0 + size_t(row0) * ngroups * 2, sc_mat_bytes, bar);
                     if (GU) g_bulk(g_smem(dst + sc_mat_bytes), a.sc1 + size_t(row0) * ngroups * 2, sc_mat_bytes, bar);
+                    if (C::kI8)
+                        g_bulk(g_smem(dst + C::kNMat * sc_mat_bytes), a.zsum + size_t(T.ebase + T.n0) * zst, zbytes, bar);
                 }
                 __syncwarp();
             }
@@ -390,7 +404,7 @@ __global__ void __launch_bounds__(G_THREADS, 1) tc_grouped_gemm(const __grid_con
             const uint32_t first = pc > NPK ? pc - NPK : 0;
             for (uint32_t n = first; n < pc; n++) g_drain_wait(g_smem(&pk_full[n % NPK]), (n / NPK) & 1);
             if (C::kInt4)
-                for (int n = t > 2 ? t - 2 : 0; n < t; n++) g_drain_wait(g_smem(&sc_full[n & 1]), (n >> 1) & 1);
+                for (int n = t > NSC ? t - NSC : 0; n < t; n++) g_drain_wait(g_smem(&sc_full[n % NSC]), (n / NSC) & 1);
         }
         __syncwarp();
     } else if (warp == 1) {
@@ -412,8 +426,10 @@ __global__ void __launch_bounds__(G_THREADS, 1) tc_grouped_gemm(const __grid_con
                 const uint32_t st = g_smem(bring + s * C::kBStageBytes);
                 if (g_elect()) {
                     if (C::kI8) {
-                        g_expect(bar, uint32_t(C::kBAtom));
+                        // K = 256 as two 128-byte boxes of the tile's 16 digit rows
+                        g_expect(bar, uint32_t(C::kBStageBytes));
                         g_tma2d(st, map, T.kbase + ks * C::kSK, row0, bar);
+                        g_tma2d(st + C::kBAtom, map, T.kbase + ks * C::kSK + 128, row0, bar);
                     } else {
                         g_expect(bar, uint32_t(T.bn) * 256u);
                         g_tma2d(st, map, T.kbase + ks * C::kSK, row0, bar);
@@ -445,36 +461,44 @@ __global__ void __launch_bounds__(G_THREADS, 1) tc_grouped_gemm(const __grid_con
             g_fence_after();
             bool ok = true;
             for (int ks = 0; ks < KS; ks++) {
-                const int sb = bc % C::kBStages, sa = ac % C::kAStages, sp = pc % NPK;
+                const int sb = bc % C::kBStages, sa = ac % C::kAStages;
                 if (!g_wait_w(g_smem(&b_full[sb]), (bc / C::kBStages) & 1, &s_abort)) { ok = false; break; }
                 if (C::kTmemA) {
                     if (!g_wait_w(g_smem(&a_full[sa]), (ac / C::kAStages) & 1, &s_abort)) { ok = false; break; }
                 } else {
-                    if (!g_wait_w(g_smem(&pk_full[sp]), (pc / NPK) & 1, &s_abort)) { ok = false; break; }
+                    if (!g_wait_w(g_smem(&pk_full[pc % NPK]), (pc / NPK) & 1, &s_abort)) { ok = false; break; }
                 }
                 if (C::kI8) {
-                    // every step into the next accumulator buffer; the epilogue frees it
+                    // every step into the next accumulator buffer.  The epilogue frees
+                    // them in order, so one wait per half ring covers the next kAccBufs / 2 steps.
+                    constexpr int kHalf = C::kAccBufs / 2;
                     const int bi = bc % C::kAccBufs;
-                    if (bc >= uint32_t(C::kAccBufs) &&
-                        !g_wait_w(g_smem(&acc_empty[bi]), ((bc / C::kAccBufs) - 1) & 1, &s_abort)) { ok = false; break; }
+                    if (bc >= uint32_t(C::kAccBufs) && bc % kHalf == 0) {
+                        const uint32_t y = bc - C::kAccBufs + kHalf - 1;      // last earlier user of these buffers
+                        if (!g_wait_w(g_smem(&acc_empty[y % C::kAccBufs]), (y / C::kAccBufs) & 1, &s_abort)) { ok = false; break; }
+                    }
                     d = tmem + bi * C::kAccCols;
                 }
                 g_fence_after();
                 const uint32_t b0 = g_smem(bring + sb * C::kBStageBytes);
                 const uint32_t at = tmem + 256 + sa * C::kAStageCols;
-                const uint32_t a0 = g_smem(pk + sp * C::kPkStageBytes);
+                const uint32_t a0 = g_smem(pk + (pc % NPK) * C::kPkStageBytes);
                 if (g_elect()) {
 #pragma unroll
                     for (int k = 0; k < C::kSK / C::kMmaK; k++) {
-                        const uint32_t acc = (k > 0 || (!C::kI8 && ks > 0)) ? 1u : 0u;
                         const uint64_t bd = g_desc(b0 + (k >> 2) * C::kBAtom + (k & 3) * 32);
                         if (C::kI8) {
-                            g_mma_ts_i8(d, at + k * 8, bd, idesc, acc);
-                            if (GU) g_mma_ts_i8(d + C::kUpCol, at + C::kAColsK + k * 8, bd, idesc, acc);
+                            // group k / 4 of the step into its own accumulator: gate at 16 g, up at 16 (kGroups + g)
+                            const uint32_t acc = (k & 3) ? 1u : 0u;
+                            const uint32_t dg = d + (k >> 2) * 16;
+                            g_mma_ts_i8(dg, at + k * 8, bd, idesc, acc);
+                            if (GU) g_mma_ts_i8(dg + C::kGroups * 16, at + C::kAColsK + k * 8, bd, idesc, acc);
                         } else if (C::kTmemA) {
+                            const uint32_t acc = (k > 0 || ks > 0) ? 1u : 0u;
                             g_mma_ts(d, at + k * 8, bd, idesc, acc);
                             if (GU) g_mma_ts(d + C::kUpCol, at + C::kAColsK + k * 8, bd, idesc, acc);
                         } else {
+                            const uint32_t acc = (k > 0 || ks > 0) ? 1u : 0u;
                             const uint32_t ak = a0 + (k >> 2) * (G_BM * 128) + (k & 3) * 32;
                             g_mma_ss(d, g_desc(ak), bd, idesc, acc);
                             if (GU) g_mma_ss(d + C::kUpCol, g_desc(ak + C::kMatBytes), bd, idesc, acc);
@@ -498,8 +522,9 @@ __global__ void __launch_bounds__(G_THREADS, 1) tc_grouped_gemm(const __grid_con
     } else if (warp >= 4 && warp < 8 && C::kI8) {
         // ---------------- 8-bit int4 epilogue: fold every K = 128 step ----------------
         // Thread (warp w, lane l) owns weight row 32*(w%4) + l of the tile; lane
-        // j < kNMax also holds token j's group term and row factor.  Token j's
-        // digit sums are accumulator columns 3j (d2), 3j+1 (d1), 3j+2 (d0).
+        // j < kNMax also holds token j's row factor.  A step holds kGroups scale
+        // groups, each in its own 16 accumulator columns (gate, then up); token
+        // j's digit sums are columns 3j (d2), 3j+1 (d1), 3j+2 (d0) of a group.
         const int q = warp & 3;
         const uint32_t lane_addr = uint32_t(q * 32) << 16;
         const int r = q * 32 + lane;
@@ -511,11 +536,17 @@ __global__ void __launch_bounds__(G_THREADS, 1) tc_grouped_gemm(const __grid_con
             const int f = T.m0 + r;
             const int rbase = T.ebase + T.n0;
             const bool live = lane < T.nval;
-            const int b = t & 1;
-            if (!g_wait(g_smem(&sc_full[b]), (t >> 1) & 1, &s_abort, 64)) { ok = false; break; }
-            const __nv_bfloat16* sc0 = reinterpret_cast<const __nv_bfloat16*>(scbuf + b * C::kNMat * sc_mat_bytes) + r * ngroups;
+            const int b = t % NSC;
+            // the row factors are needed after the last step: issue their loads now
+            float rowf = 1.f;
+            if (live) {
+                rowf = a.act_scale[rbase + lane];
+                if (!GU && a.topk_w) rowf *= a.topk_w[a.row_slot[rbase + lane]];
+            }
+            if (!g_wait(g_smem(&sc_full[b]), (t / NSC) & 1, &s_abort, 64)) { ok = false; break; }
+            const __nv_bfloat16* sc0 = reinterpret_cast<const __nv_bfloat16*>(scbuf + b * sc_buf_bytes) + r * ngroups;
             const __nv_bfloat16* sc1 = sc0 + G_BM * ngroups;
-            const float* zrow = a.zsum + size_t(rbase + (live ? lane : 0)) * ngroups;
+            const float* zs = reinterpret_cast<const float*>(scbuf + b * sc_buf_bytes + C::kNMat * sc_mat_bytes);
             float tg[C::kNMax], tu[C::kNMax];
 #pragma unroll
             for (int j = 0; j < C::kNMax; j++) tg[j] = tu[j] = 0.f;
@@ -523,38 +554,39 @@ __global__ void __launch_bounds__(G_THREADS, 1) tc_grouped_gemm(const __grid_con
                 const int bi = ac % C::kAccBufs;
                 if (!g_wait(g_smem(&done[ac % G_DONE]), (ac / G_DONE) & 1, &s_abort)) { ok = false; break; }
                 g_fence_after();
-                uint32_t g[16], u[16];
-                g_ld16(tmem + lane_addr + bi * C::kAccCols, g);
-                if (GU) g_ld16(tmem + lane_addr + bi * C::kAccCols + C::kUpCol, u);
+                uint32_t g[C::kGroups][16], u[C::kGroups][16];
+                const uint32_t ab = tmem + lane_addr + bi * C::kAccCols;
+#pragma unroll
+                for (int gi = 0; gi < C::kGroups; gi++) {
+                    g_ld16(ab + gi * 16, g[gi]);
+                    if (GU) g_ld16(ab + (C::kGroups + gi) * 16, u[gi]);
+                }
                 g_ld_wait();
                 g_fence_before();
                 __syncwarp();
                 if (lane == 0) g_arrive(g_smem(&acc_empty[bi]));
-                const int grp = T.kbase / 128 + ks;
-                const float z = live ? zrow[grp] : 0.f;
-                const float s0 = __bfloat162float(sc0[grp]);
-                const float s1 = GU ? __bfloat162float(sc1[grp]) : 0.f;
 #pragma unroll
-                for (int j = 0; j < C::kNMax; j++) {
-                    const float zj = __shfl_sync(0xffffffffu, z, j);
-                    const float vg = fmaf(float(int(g[3 * j])), 65536.f,
-                                          fmaf(float(int(g[3 * j + 1])), 256.f, float(int(g[3 * j + 2])))) - zj;
-                    tg[j] = fmaf(s0, vg, tg[j]);
-                    if (GU) {
-                        const float vu = fmaf(float(int(u[3 * j])), 65536.f,
-                                              fmaf(float(int(u[3 * j + 1])), 256.f, float(int(u[3 * j + 2])))) - zj;
-                        tu[j] = fmaf(s1, vu, tu[j]);
+                for (int gi = 0; gi < C::kGroups; gi++) {
+                    const int grp = T.kbase / 128 + ks * C::kGroups + gi;
+                    const float s0 = __bfloat162float(sc0[grp]);
+                    const float s1 = GU ? __bfloat162float(sc1[grp]) : 0.f;
+#pragma unroll
+                    for (int j = 0; j < C::kNMax; j++) {
+                        const float zj = j < T.nval ? zs[j * zst + grp] : 0.f;
+                        const float vg = fmaf(float(int(g[gi][3 * j])), 65536.f,
+                                              fmaf(float(int(g[gi][3 * j + 1])), 256.f, float(int(g[gi][3 * j + 2])))) - zj;
+                        tg[j] = fmaf(s0, vg, tg[j]);
+                        if (GU) {
+                            const float vu = fmaf(float(int(u[gi][3 * j])), 65536.f,
+                                                  fmaf(float(int(u[gi][3 * j + 1])), 256.f, float(int(u[gi][3 * j + 2])))) - zj;
+                            tu[j] = fmaf(s1, vu, tu[j]);
+                        }
                     }
                 }
             }
             if (!ok) break;
             __syncwarp();
             if (lane == 0) g_arrive(g_smem(&sc_empty[b]));
-            float rowf = 1.f;
-            if (live) {
-                rowf = a.act_scale[rbase + lane];
-                if (!GU && a.topk_w) rowf *= a.topk_w[a.row_slot[rbase + lane]];
-            }
 #pragma unroll
             for (int j = 0; j < C::kNMax; j++) {
                 const float fj = __shfl_sync(0xffffffffu, rowf, j);
@@ -579,22 +611,28 @@ __global__ void __launch_bounds__(G_THREADS, 1) tc_grouped_gemm(const __grid_con
         for (int tile = blockIdx.x; tile < ntiles && !s_abort; tile += gridDim.x, t++) {
             const GTile T = tile_of(tile);
             const int buf = t & 1;
+            const int rbase = T.ebase + T.n0;
+            // the factor of row c + j (activation row scale, routing weight) sits in lane j;
+            // the loads of the first 16 rows' factors and of the global scales go out before the wait
+            auto row_factor = [&](int c) {
+                float v = 1.f;
+                const int nn = c + (lane & 15);
+                if (nn < T.nval) {
+                    if (FMT == MOE_FMT_NVFP4) v = a.act_scale[rbase + nn];
+                    if (!GU && a.topk_w) v *= a.topk_w[a.row_slot[rbase + nn]];
+                }
+                return v;
+            };
+            float rowf0 = row_factor(0);
+            float gsc = 1.f, usc = 1.f;
+            if (FMT == MOE_FMT_NVFP4) { gsc = a.g0[T.e]; if (GU) usc = a.g1[T.e]; }
             if (!g_wait(g_smem(&acc_full[buf]), (t >> 1) & 1, &s_abort, 128)) { fail(); break; }
             g_fence_after();
             const int f = T.m0 + q * 32 + lane;
             const int fo = a.perm_out ? ((f & ~7) | ((f & 7) < 4 ? 2 * (f & 7) : 2 * (f & 7) - 7)) : f;
-            float gsc = 1.f, usc = 1.f;
-            if (FMT == MOE_FMT_NVFP4) { gsc = a.g0[T.e]; if (GU) usc = a.g1[T.e]; }
             const uint32_t acc0 = tmem + lane_addr + buf * 128;
-            const int rbase = T.ebase + T.n0;
             for (int c = 0; c < T.bn; c += 16) {
-                // the factor of row c + j (activation row scale, routing weight) sits in lane j
-                float rowf = 1.f;
-                const int nn = c + (lane & 15);
-                if (nn < T.nval) {
-                    if (FMT == MOE_FMT_NVFP4) rowf = a.act_scale[rbase + nn];
-                    if (!GU && a.topk_w) rowf *= a.topk_w[a.row_slot[rbase + nn]];
-                }
+                const float rowf = c == 0 ? rowf0 : row_factor(c);
                 uint32_t g[16], u[16];
                 g_ld16(acc0 + c, g);
                 if (GU) g_ld16(acc0 + C::kUpCol + c, u);
@@ -634,31 +672,31 @@ __global__ void __launch_bounds__(G_THREADS, 1) tc_grouped_gemm(const __grid_con
         }
     } else if (warp >= 8 && C::kTmemA) {
         // ---------------- dequantisation ----------------
-        // A weight stage (K = 256) holds two A stages (K = 128).  gate/up: this
-        // warp writes matrix hsel of both (4 chunks of 16 bytes per A stage);
-        // down: it writes K half hsel of both (2 chunks per A stage).  Chunks
-        // are software-pipelined: the next one is dequantised while the
-        // tensor-memory store of the current one is in flight.
-        constexpr int kPer = GU ? 4 : 2;               // my chunks per A stage
-        constexpr int kChunks = 2 * kPer;              // per weight stage
+        // A weight stage (K = 256, 8 chunks of 16 bytes per row) holds kAPerPk
+        // A stages.  gate/up: this warp writes matrix hsel (all chunks of its
+        // rows); down: it writes K half hsel of every A stage.  Chunks are
+        // software-pipelined: the next one is dequantised while the tensor-
+        // memory store of the current one is in flight.
+        constexpr int kPer = (GU ? 8 : 4) / C::kAPerPk;    // my chunks per A stage
+        constexpr int kChunks = C::kAPerPk * kPer;         // per weight stage
         constexpr int kNBuf = 4;
         const int q = warp & 3, hsel = (warp - 8) >> 2;
         const int r = q * 32 + lane;                   // weight row within the tile
         const uint32_t lane_addr = uint32_t(q * 32) << 16;
-        const uint32_t colw = 256 + (GU ? hsel * C::kAColsK : hsel * (C::kAColsK / 2));
+        const uint32_t colw = 256 + (GU ? hsel * C::kAColsK : hsel * kPer * C::kChunkCols);
         uint32_t pc = 0;
         int t = 0;
         bool ok = true;
         for (int tile = blockIdx.x; tile < ntiles && ok && !s_abort; tile += gridDim.x, t++) {
             const uint8_t* scrow = nullptr;
             if (FMT == MOE_FMT_INT4_G128) {
-                const int b = t & 1;
-                if (!g_wait(g_smem(&sc_full[b]), (t >> 1) & 1, &s_abort)) { ok = false; break; }
-                scrow = scbuf + b * C::kNMat * sc_mat_bytes + (GU ? hsel * sc_mat_bytes : 0) + r * ngroups * 2;
+                const int b = t % NSC;
+                if (!g_wait(g_smem(&sc_full[b]), (t / NSC) & 1, &s_abort)) { ok = false; break; }
+                scrow = scbuf + b * sc_buf_bytes + (GU ? hsel * sc_mat_bytes : 0) + r * ngroups * 2;
             }
             for (int ps = 0; ps < NPS && ok; ps++, pc++) {
                 const int s = pc % NPK;
-                if (!g_wait(g_smem(&pk_full[s]), (pc / NPK) & 1, &s_abort)) { ok = false; break; }
+                if (!g_wait_w(g_smem(&pk_full[s]), (pc / NPK) & 1, &s_abort)) { ok = false; break; }
                 const uint8_t* st = pk + s * C::kPkStageBytes;
                 const uint8_t* wt = st + (GU ? hsel * C::kMatBytes : 0);
                 uint32_t scw = 0;                      // int4: bf16 scales of groups 2ps (low) and 2ps+1 (high)
@@ -675,7 +713,7 @@ __global__ void __launch_bounds__(G_THREADS, 1) tc_grouped_gemm(const __grid_con
                 // chunk index (16 bytes of this row in the weight stage) of my i-th chunk
                 auto dq = [&](auto ic) {
                     constexpr int i = decltype(ic)::value, j = i / kPer, l = i % kPer;
-                    const int c = 4 * j + (GU ? l : 2 * hsel + l);
+                    const int c = (8 / C::kAPerPk) * j + (GU ? l : kPer * hsel + l);
                     const uint4 w = *reinterpret_cast<const uint4*>(wt + g_swz(r, c));
                     if (FMT == FMT_INT4_I8) {
                         g_dq_int4_i8(w, o[i % kNBuf]);
@@ -693,10 +731,10 @@ __global__ void __launch_bounds__(G_THREADS, 1) tc_grouped_gemm(const __grid_con
                     constexpr int i = decltype(ic)::value, j = i / kPer, l = i % kPer;
                     if (!ok) return;
                     if (l == 0) {
-                        const uint32_t acn = pc * 2 + j;             // A stage index in this CTA's stream
+                        const uint32_t acn = pc * C::kAPerPk + j;    // A stage index in this CTA's stream
                         sa = acn % C::kAStages;
-                        if (acn >= uint32_t(C::kAStages) && !g_wait(g_smem(&done[(acn - C::kAStages) % G_DONE]),
-                                                                    ((acn - C::kAStages) / G_DONE) & 1, &s_abort)) {
+                        if (acn >= uint32_t(C::kAStages) && !g_wait_w(g_smem(&done[(acn - C::kAStages) % G_DONE]),
+                                                                      ((acn - C::kAStages) / G_DONE) & 1, &s_abort)) {
                             ok = false;
                             return;
                         }
@@ -718,7 +756,7 @@ __global__ void __launch_bounds__(G_THREADS, 1) tc_grouped_gemm(const __grid_con
             if (!ok) break;
             if (FMT == MOE_FMT_INT4_G128) {
                 __syncwarp();
-                if (lane == 0) g_arrive(g_smem(&sc_empty[t & 1]));
+                if (lane == 0) g_arrive(g_smem(&sc_empty[t % NSC]));
             }
         }
         if (!ok) fail();
@@ -737,15 +775,10 @@ __global__ void __launch_bounds__(G_THREADS, 1) tc_grouped_gemm(const __grid_con
 //   mode 2: f16 times 2^-e (e >= 0 least with |x| * 2^-e <= 16384), row scale 2^e.
 // One warp per row.
 // ---------------------------------------------------------------------------
-//   mode 3 (8-bit int4): X = rint(x * 2^c), c the row's exponent that puts
-//          max |X| in [2^21, 2^22), as signed digits X = 65536 d2 + 256 d1 + d0
-//          in rows 3 row (d2), 3 row + 1 (d1), 3 row + 2 (d0) of int8 dst, in
-//          the K order 0, 2, 4, 6, 1, 3, 5, 7 of every 8; scale[row] = 2^-c;
-//          zsum[row][g] = 8 * sum of X over group g (the u - 8 offset).
 __global__ void __launch_bounds__(256) g_prep(const __nv_bfloat16* __restrict__ src, int in_dim,
                                               const int32_t* __restrict__ row_slot, int top_k, int by_token,
                                               int rows, int mode, uint16_t* __restrict__ dst,
-                                              float* __restrict__ scale, float* __restrict__ zsum) {
+                                              float* __restrict__ scale) {
     asm volatile("griddepcontrol.wait;" ::: "memory");
     const int row = (blockIdx.x * blockDim.x + threadIdx.x) >> 5, lane = threadIdx.x & 31;
     if (row >= rows) return;
@@ -765,48 +798,6 @@ __global__ void __launch_bounds__(256) g_prep(const __nv_bfloat16* __restrict__ 
             o.w = __byte_perm(v.y, v.w, 0x7632);   // (x3, x7)
             d[i] = o;
         }
-    } else if (mode == 3) {
-        float amax = 0.f;
-        for (int i = lane; i < n16; i += 32) {
-            const uint4 v = s[i];
-            amax = fmaxf(amax, fmaxf(fmaxf(fabsf(bf16_lo(v.x)), fabsf(bf16_hi(v.x))), fmaxf(fabsf(bf16_lo(v.y)), fabsf(bf16_hi(v.y)))));
-            amax = fmaxf(amax, fmaxf(fmaxf(fabsf(bf16_lo(v.z)), fabsf(bf16_hi(v.z))), fmaxf(fabsf(bf16_lo(v.w)), fabsf(bf16_hi(v.w)))));
-        }
-        for (int o = 16; o > 0; o >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, o));
-        int ex = 0;
-        frexpf(amax, &ex);                                  // amax < 2^ex
-        const int c = amax > 0.f ? min(22 - ex, 126) : 0;   // |x| 2^c < 2^22
-        uint8_t* d8 = reinterpret_cast<uint8_t*>(dst) + size_t(row) * 3 * in_dim;
-        // 16 pieces of 8 make a group of 128: lanes 0-15 and 16-31 take one group each per pass
-        for (int i0 = 0; i0 < n16; i0 += 32) {
-            const int i = i0 + lane;
-            int zs = 0;
-            if (i < n16) {
-                const uint4 v = s[i];
-                // the K order of the weight bytes: 0, 2, 4, 6, 1, 3, 5, 7
-                const float xs[8] = {bf16_lo(v.x), bf16_lo(v.y), bf16_lo(v.z), bf16_lo(v.w),
-                                     bf16_hi(v.x), bf16_hi(v.y), bf16_hi(v.z), bf16_hi(v.w)};
-                uint32_t p2[2] = {0u, 0u}, p1[2] = {0u, 0u}, p0[2] = {0u, 0u};
-#pragma unroll
-                for (int e = 0; e < 8; e++) {
-                    const int X = __float2int_rn(ldexpf(xs[e], c));
-                    zs += X;
-                    const int d0 = ((X + 128) & 255) - 128;          // signed digits in [-128, 127]
-                    const int X1 = (X - d0) >> 8;
-                    const int d1 = ((X1 + 128) & 255) - 128;
-                    const int d2 = (X1 - d1) >> 8;
-                    p0[e >> 2] |= uint32_t(d0 & 255) << (8 * (e & 3));
-                    p1[e >> 2] |= uint32_t(d1 & 255) << (8 * (e & 3));
-                    p2[e >> 2] |= uint32_t(d2 & 255) << (8 * (e & 3));
-                }
-                *reinterpret_cast<uint2*>(d8 + size_t(i) * 8) = make_uint2(p2[0], p2[1]);
-                *reinterpret_cast<uint2*>(d8 + in_dim + size_t(i) * 8) = make_uint2(p1[0], p1[1]);
-                *reinterpret_cast<uint2*>(d8 + 2 * size_t(in_dim) + size_t(i) * 8) = make_uint2(p0[0], p0[1]);
-            }
-            for (int o = 8; o > 0; o >>= 1) zs += __shfl_xor_sync(0xffffffffu, zs, o);
-            if ((lane & 15) == 0 && i < n16) zsum[size_t(row) * (in_dim / 128) + i / 16] = 8.f * float(zs);
-        }
-        if (lane == 0) scale[row] = ldexpf(1.f, -c);
     } else {
         float amax = 0.f;
         for (int i = lane; i < n16; i += 32) {
@@ -829,6 +820,70 @@ __global__ void __launch_bounds__(256) g_prep(const __nv_bfloat16* __restrict__ 
         }
         if (lane == 0) scale[row] = ldexpf(1.f, e);
     }
+}
+
+// 8-bit int4 pre-pass: one CTA of 128 threads per GEMM row (gathered like
+// g_prep).  X = rint(x * 2^c), c the row's exponent that puts max |X| in
+// [2^21, 2^22), written as signed digits X = 65536 d2 + 256 d1 + d0 in int8
+// rows 3 row (d2), 3 row + 1 (d1), 3 row + 2 (d0) of dst, in the K order
+// 0, 2, 4, 6, 1, 3, 5, 7 of every 8 (the order of the unpacked weight bytes);
+// scale[row] = 2^-c; zsum[row][g] (row stride zst) = 8 * sum of X over group
+// g, the u - 8 offset of the weights.
+constexpr int G_PREP_I8_THREADS = 128;
+__global__ void __launch_bounds__(G_PREP_I8_THREADS) g_prep_i8(const __nv_bfloat16* __restrict__ src, int in_dim,
+                                                               const int32_t* __restrict__ row_slot, int top_k,
+                                                               int by_token, uint8_t* __restrict__ dst,
+                                                               float* __restrict__ scale, float* __restrict__ zsum) {
+    __shared__ float s_max[G_PREP_I8_THREADS / 32];
+    asm volatile("griddepcontrol.wait;" ::: "memory");
+    const int row = blockIdx.x, tid = threadIdx.x, lane = tid & 31;
+    const int srow = by_token ? row_slot[row] / top_k : row;
+    const uint4* s = reinterpret_cast<const uint4*>(src + size_t(srow) * in_dim);
+    const int n16 = in_dim / 8, zst = ((in_dim / 128) + 3) & ~3;
+    float amax = 0.f;
+    for (int i = tid; i < n16; i += G_PREP_I8_THREADS) {
+        const uint4 v = s[i];
+        amax = fmaxf(amax, fmaxf(fmaxf(fabsf(bf16_lo(v.x)), fabsf(bf16_hi(v.x))), fmaxf(fabsf(bf16_lo(v.y)), fabsf(bf16_hi(v.y)))));
+        amax = fmaxf(amax, fmaxf(fmaxf(fabsf(bf16_lo(v.z)), fabsf(bf16_hi(v.z))), fmaxf(fabsf(bf16_lo(v.w)), fabsf(bf16_hi(v.w)))));
+    }
+    for (int o = 16; o > 0; o >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, o));
+    if (lane == 0) s_max[tid >> 5] = amax;
+    __syncthreads();
+    amax = fmaxf(fmaxf(s_max[0], s_max[1]), fmaxf(s_max[2], s_max[3]));
+    int ex = 0;
+    frexpf(amax, &ex);                                  // amax < 2^ex
+    const int c = amax > 0.f ? min(22 - ex, 126) : 0;   // |x| 2^c < 2^22
+    const float fc = ldexpf(1.f, c);                    // a power of two: x * fc is exact
+    uint8_t* d8 = dst + size_t(row) * 3 * in_dim;
+    // 16 pieces of 8 make a group of 128: lanes 0-15 and 16-31 hold one group each
+    for (int i0 = 0; i0 < n16; i0 += G_PREP_I8_THREADS) {
+        const int i = i0 + tid;
+        int zs = 0;
+        if (i < n16) {
+            const uint4 v = s[i];
+            const float xs[8] = {bf16_lo(v.x), bf16_lo(v.y), bf16_lo(v.z), bf16_lo(v.w),
+                                 bf16_hi(v.x), bf16_hi(v.y), bf16_hi(v.z), bf16_hi(v.w)};
+            uint32_t p2[2] = {0u, 0u}, p1[2] = {0u, 0u}, p0[2] = {0u, 0u};
+#pragma unroll
+            for (int e = 0; e < 8; e++) {
+                const int X = __float2int_rn(xs[e] * fc);
+                zs += X;
+                const int d0 = ((X + 128) & 255) - 128;          // signed digits in [-128, 127]
+                const int X1 = (X - d0) >> 8;
+                const int d1 = ((X1 + 128) & 255) - 128;
+                const int d2 = (X1 - d1) >> 8;
+                p0[e >> 2] |= uint32_t(d0 & 255) << (8 * (e & 3));
+                p1[e >> 2] |= uint32_t(d1 & 255) << (8 * (e & 3));
+                p2[e >> 2] |= uint32_t(d2 & 255) << (8 * (e & 3));
+            }
+            *reinterpret_cast<uint2*>(d8 + size_t(i) * 8) = make_uint2(p2[0], p2[1]);
+            *reinterpret_cast<uint2*>(d8 + in_dim + size_t(i) * 8) = make_uint2(p1[0], p1[1]);
+            *reinterpret_cast<uint2*>(d8 + 2 * size_t(in_dim) + size_t(i) * 8) = make_uint2(p0[0], p0[1]);
+        }
+        for (int o = 8; o > 0; o >>= 1) zs += __shfl_xor_sync(0xffffffffu, zs, o);
+        if ((lane & 15) == 0 && i < n16) zsum[size_t(row) * zst + i / 16] = 8.f * float(zs);
+    }
+    if (tid == 0) scale[row] = 1.f / fc;
 }
 
 // ---------------------------------------------------------------------------
@@ -876,10 +931,10 @@ __global__ void __launch_bounds__(256) g_splitk_finish(const float* __restrict__
 // Host side
 // ---------------------------------------------------------------------------
 template <int FMT, bool GU>
-static size_t g_smem_bytes(int in_dim, int npk) {
+static size_t g_smem_bytes(int in_dim, int npk, int nsc) {
     using C = GCfg<FMT, GU>;
     size_t b = size_t(npk) * C::kPkStageBytes + size_t(C::kBStages) * C::kBStageBytes + 1024;
-    if (C::kInt4) b += 2 * size_t(C::kNMat) * G_BM * (in_dim / 128) * 2;
+    if (C::kInt4) b += size_t(nsc) * (C::kNMat * G_BM * (in_dim / 128) * 2 + (C::kI8 ? C::kNMax * (((in_dim / 128) + 3) & ~3) * 4 : 0));
     return b;
 }
 
@@ -893,14 +948,22 @@ static int g_launch(const GArgs& a, cudaStream_t s) {
     if (cudaDeviceGetAttribute(&optin, cudaDevAttrMaxSharedMemoryPerBlockOptin, dev) != cudaSuccess) return MOE_ERR_CUDA;
     cudaFuncAttributes fa{};
     if (cudaFuncGetAttributes(&fa, k) != cudaSuccess) return MOE_ERR_CUDA;
-    // the weight stream wants as many bytes in flight as shared memory holds
+    // The weight stream wants as many bytes in flight as shared memory holds.
+    // The producer runs ahead by whole tiles only as far as free int4 scale
+    // buffers allow, so those cover the ring's reach: one per tile it spans,
+    // plus the tile being consumed.
     const size_t room = size_t(optin) - std::min(size_t(optin), fa.sharedSizeBytes);
-    const size_t fixed = g_smem_bytes<FMT, GU>(a.in_dim, 0);
-    const int npk = fixed < room ? int(std::min<size_t>(C::kPkMax, (room - fixed) / C::kPkStageBytes)) : 0;
+    const int nps = std::max(1, (a.in_dim / a.ksplit) / C::kPkK);            // weight stages per tile
+    int npk = C::kPkMax, nsc = 2;
+    for (; npk >= 2; npk--) {
+        nsc = C::kInt4 ? std::min(G_SC_MAX, std::max(2, (npk + nps - 1) / nps + 1)) : 2;
+        if (g_smem_bytes<FMT, GU>(a.in_dim, npk, nsc) <= room) break;
+    }
     if (npk < 2) return MOE_ERR_UNSUPPORTED;
     GArgs args = a;
     args.npk = npk;
-    const size_t smem = g_smem_bytes<FMT, GU>(a.in_dim, npk);
+    args.nsc = nsc;
+    const size_t smem = g_smem_bytes<FMT, GU>(a.in_dim, npk, nsc);
     if (cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem)) != cudaSuccess)
         return MOE_ERR_CUDA;
     return launch_pdl(k, dim3(sms), dim3(G_THREADS), smem, s, args) == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
@@ -934,11 +997,17 @@ int launch_grouped_gemm(const GemvProblem& p, bool gateup, int rows, const GemmB
     const float* ascale = nullptr;
     if (!buf.act_ready || nv || i8) {
         if (!buf.act_buf || (nv && !buf.scale_buf)) return MOE_ERR_WORKSPACE;
-        const int mode = i8 ? 3 : nv ? 2 : (i4 ? 1 : 0);
-        if (launch_pdl(g_prep, dim3((rows * 32 + 255) / 256), dim3(256), 0, s, p.act, in, p.row_slot, p.top_k,
-                       p.act_by_token, rows, mode, reinterpret_cast<uint16_t*>(buf.act_buf), buf.scale_buf,
-                       buf.zbuf) != cudaSuccess)
-            return MOE_ERR_CUDA;
+        if (i8) {
+            if (launch_pdl(g_prep_i8, dim3(rows), dim3(G_PREP_I8_THREADS), 0, s, p.act, in, p.row_slot, p.top_k,
+                           p.act_by_token, reinterpret_cast<uint8_t*>(buf.act_buf), buf.scale_buf, buf.zbuf) != cudaSuccess)
+                return MOE_ERR_CUDA;
+        } else {
+            const int mode = nv ? 2 : (i4 ? 1 : 0);
+            if (launch_pdl(g_prep, dim3((rows * 32 + 255) / 256), dim3(256), 0, s, p.act, in, p.row_slot, p.top_k,
+                           p.act_by_token, rows, mode, reinterpret_cast<uint16_t*>(buf.act_buf), buf.scale_buf) !=
+                cudaSuccess)
+                return MOE_ERR_CUDA;
+        }
         bsrc = buf.act_buf;
         ascale = buf.scale_buf;
     }

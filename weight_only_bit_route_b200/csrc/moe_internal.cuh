@@ -62,11 +62,14 @@ inline size_t prep_scratch(int rows, int in_dim) {
 }
 // int4 routed problems with at most this many rows take the 8-bit int4 GEMM
 constexpr int kI8Int4MaxRows = 512;
-// GEMM pre-pass output: row scales [rows] fp32, group sums [rows][in/128] fp32,
+// Row stride (floats) of the 8-bit int4 group sums: in/128 rounded up to a
+// multiple of 4, so that a tile's rows are one 16-byte aligned block.
+inline int zsum_stride(int in_dim) { return ((in_dim / 128) + 3) & ~3; }
+// GEMM pre-pass output: row scales [rows] fp32, group sums [rows][zsum_stride] fp32,
 // then the gathered rows: 16-bit [rows][in], or three int8 digit rows per row
 // when the 8-bit int4 GEMM can take the problem.
 inline size_t gemm_prep_bytes(int rows, int in_dim) {
-    return align256(size_t(rows) * 4) + align256(size_t(rows) * (in_dim / 128) * 4) +
+    return align256(size_t(rows) * 4) + align256(size_t(rows) * zsum_stride(in_dim) * 4) +
            align256(size_t(rows) * in_dim * (rows <= kI8Int4MaxRows ? 3 : 2));
 }
 // Step-level scratch of a grouped call: tile metadata, then the pre-pass of
@@ -217,7 +220,7 @@ struct GemmBuffers {
     int ksplit;          // > 1: split K into this many slices (BF16 only); fp32 partial sums go to partial
     float* partial;      // split_bytes(...) bytes
     int i8;              // int4 on the 8-bit MMA with per-group accumulation (small batches)
-    float* zbuf;         // i8: 8 * group sums of the fixed-point rows [rows][in / 128]
+    float* zbuf;         // i8: 8 * group sums of the fixed-point rows [rows][zsum_stride(in)]
 };
 
 
