@@ -22,11 +22,15 @@
 //               plus the NVFP4 block scales of those rows.  int4 scales are
 //               one bulk copy per tile, since all groups of the tile's rows
 //               are contiguous.
-//   warp 1      TMA producer of the activation operand: per K = 128 stage, two
-//               boxes of the tile's rows x 64 elements, 128-byte swizzled (the
+//   warp 1      producer of the activation operand: per K = 128 stage, two
+//               TMA boxes of the tile's rows x 64 elements, 128-byte swizzled (the
 //               K-major layout the MMA descriptors read); the box height comes
-//               from one of several tensor maps, matching the tile's rows.
-//   warp 2      allocates tensor memory and issues tcgen05.mma from one lane.
+//               from one of several tensor maps, matching the tile's rows.  The
+//               8-bit int4 path copies its small stages (16 rows x 256 bytes)
+//               with per-lane 16-byte asynchronous copies instead, which do not
+//               queue behind the weight stream in the tensor-copy engine.
+//   warp 2      allocates tensor memory and issues tcgen05.mma from one lane
+//               (8-bit int4: warps 2 and 3 take alternate steps).
 // The three single-issue roles run warp-uniform loops and elect one lane to
 // issue, which keeps the instruction operands in uniform registers.  The MMA
 // pipeline steps in K = 128 and commits once per step, to one barrier of a
@@ -50,6 +54,8 @@
 // Tensor memory (512 columns): two accumulator buffers in [0, 256), so the
 // epilogue of one tile overlaps the main loop of the next (buffer b at
 // 128*b; gate/up keeps gate at +0 and up at +64), A stages in [256, 512).
+// The 8-bit path accumulates per step: its small accumulator buffers take
+// [0, 128) and the A stages [128, 512).
 //
 // int4 pairs: one mask turns the nibbles (j, j+4) of a packed word into one
 // bf16 pair, so the A operand holds the K elements of each group of 8 in the
@@ -102,7 +108,11 @@ struct GCfg {
     static constexpr int kSK = kI8 ? 256 : 128;                     // K per MMA stage
     static constexpr int kGroups = kSK / 128;                       // i8: scale groups per MMA stage
     static constexpr int kAccCols = kI8 ? kGroups * kNMat * 16 : 128;   // one accumulator buffer
-    static constexpr int kAccBufs = 256 / kAccCols;                 // accumulator buffers in [0, 256)
+    // Tensor memory: accumulators in [0, kABase), A stages in [kABase, 512).  The
+    // 8-bit path keeps few small accumulators and gives the A ring the room
+    // (its dequantise -> MMA -> free cycle is long against a step).
+    static constexpr int kAccBufs = kI8 ? 128 / kAccCols : 256 / kAccCols;
+    static constexpr int kABase = kAccBufs * kAccCols;
     static constexpr int kMmaK = kI8 ? 32 : 16;                     // K per MMA instruction
     static constexpr int kPkK = kTmemA ? 256 : 128;                 // K per weight stage
     static constexpr int kMatBytes = kTmemA ? G_BM * 128 : G_BM * 256;   // one matrix of a weight stage
@@ -115,9 +125,10 @@ struct GCfg {
     static constexpr int kBStages = kI8 ? 6 : 4;                    // i8 stages are small; cover the copy latency
     static constexpr int kAColsK = 64;                              // TMEM columns of one matrix's A stage
     static constexpr int kAStageCols = kNMat * kAColsK;
-    static constexpr int kAStages = 256 / kAStageCols;
+    static constexpr int kAStages = (512 - kABase) / kAStageCols;
     static constexpr int kAPerPk = kPkK / kSK;                      // A stages per weight stage (2, or 1 for i8)
-    static constexpr int kChunkCols = kI8 ? 8 : 16;                 // TMEM columns of one 16-byte packed chunk
+    static constexpr int kChunkCols = 16;                           // 16-bit paths: TMEM columns of one packed chunk
+    static constexpr int kDqArrivals = kI8 ? G_DQ_WARPS / 2 : G_DQ_WARPS;  // warps that fill one stage
     static constexpr bool kMmaF16 = FMT == MOE_FMT_NVFP4;
 };
 
@@ -142,6 +153,7 @@ struct GArgs {
     int32_t* status;
     float* partial;                  // split-K: fp32 partial sums [ksplit][nmat][rows][out_dim]
     const float* zsum;               // 8-bit int4: 8 * sum of the row's fixed-point values per group [rows][zst]
+    const uint8_t* bdig;             // 8-bit int4: the digit rows [3 rows][in]
     int E, out_dim, in_dim, perm_out;
     int ksplit, rows;                // K slices per (m-tile, n-tile); activation rows of the problem
     int npk;                         // weight stages in the shared-memory ring (2 .. kPkMax)
@@ -185,13 +197,15 @@ __device__ __forceinline__ void g_dq_nvfp4(const uint4 w, uint32_t sc2, uint32_t
 }
 
 // 8-bit int4: the nibbles of each word as bytes, even nibbles first: the K
-// order within every 8 weights becomes 0, 2, 4, 6, 1, 3, 5, 7.
+// order within every 8 weights becomes 0, 2, 4, 6, 1, 3, 5, 7.  One 16-byte
+// chunk gives 8 words, at o[OFF .. OFF + 7].
+template <int OFF>
 __device__ __forceinline__ void g_dq_int4_i8(const uint4 w, uint32_t (&o)[16]) {
     const uint32_t ws[4] = {w.x, w.y, w.z, w.w};
 #pragma unroll
     for (int j = 0; j < 4; j++) {
-        o[2 * j] = ws[j] & 0x0F0F0F0Fu;
-        o[2 * j + 1] = (ws[j] >> 4) & 0x0F0F0F0Fu;
+        o[OFF + 2 * j] = ws[j] & 0x0F0F0F0Fu;
+        o[OFF + 2 * j + 1] = (ws[j] >> 4) & 0x0F0F0F0Fu;
     }
 }
 
@@ -243,12 +257,12 @@ __global__ void __launch_bounds__(G_THREADS, 1) tc_grouped_gemm(const __grid_con
         for (int s = 0; s < a.npk; s++) {
             asm volatile("mbarrier.init.shared::cta.b64 [%0], 1;" ::"r"(g_smem(&pk_full[s])));
             if (C::kTmemA)     // BF16 weight stages are freed through the "stage done" ring
-                asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(g_smem(&pk_empty[s])), "r"(G_DQ_WARPS));
+                asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(g_smem(&pk_empty[s])), "r"(C::kDqArrivals));
         }
-        for (int s = 0; s < C::kBStages; s++)
-            asm volatile("mbarrier.init.shared::cta.b64 [%0], 1;" ::"r"(g_smem(&b_full[s])));
+        for (int s = 0; s < C::kBStages; s++)   // i8: one asynchronous arrival per lane of the copying warp
+            asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(g_smem(&b_full[s])), "r"(C::kI8 ? 32 : 1));
         for (int s = 0; s < C::kAStages; s++)
-            asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(g_smem(&a_full[s])), "r"(G_DQ_WARPS));
+            asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(g_smem(&a_full[s])), "r"(C::kDqArrivals));
         for (int s = 0; s < G_DONE; s++)
             asm volatile("mbarrier.init.shared::cta.b64 [%0], 1;" ::"r"(g_smem(&done[s])));
         for (int s = 0; s < a.nsc; s++) {
@@ -259,7 +273,7 @@ __global__ void __launch_bounds__(G_THREADS, 1) tc_grouped_gemm(const __grid_con
             asm volatile("mbarrier.init.shared::cta.b64 [%0], 1;" ::"r"(g_smem(&acc_full[s])));
         for (int s = 0; s < C::kAccBufs; s++)
             asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(g_smem(&acc_empty[s])), "r"(G_EPI_WARPS));
-        asm volatile("mbarrier.init.shared::cta.b64 [%0], 1;" ::"r"(g_smem(&drain)));
+        asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(g_smem(&drain)), "r"(C::kI8 ? 2 : 1));
         asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
         s_abort = 0;
     }
@@ -424,17 +438,23 @@ __global__ void __launch_bounds__(G_THREADS, 1) tc_grouped_gemm(const __grid_con
                 }
                 const uint32_t bar = g_smem(&b_full[s]);
                 const uint32_t st = g_smem(bring + s * C::kBStageBytes);
+                if (C::kI8) {
+                    // lane: digit row n = lane / 2 of the tile, 128-byte K half h = lane % 2, as eight
+                    // 16-byte chunks at their 128-byte-swizzled places; rows past the end read as zero
+                    const int n = lane >> 1, h = lane & 1;
+                    const int grow = row0 + n;
+                    const bool in_rows = grow < 3 * a.rows;
+                    const uint8_t* src = a.bdig + size_t(in_rows ? grow : 0) * in_dim + T.kbase + ks * C::kSK + h * 128;
+                    const uint32_t dst = st + h * C::kBAtom + n * 128;
+#pragma unroll
+                    for (int c = 0; c < 8; c++) g_cp16(dst + ((c ^ (n & 7)) << 4), src + c * 16, in_rows ? 16u : 0u);
+                    g_cp_arrive(bar);
+                    continue;
+                }
                 if (g_elect()) {
-                    if (C::kI8) {
-                        // K = 256 as two 128-byte boxes of the tile's 16 digit rows
-                        g_expect(bar, uint32_t(C::kBStageBytes));
-                        g_tma2d(st, map, T.kbase + ks * C::kSK, row0, bar);
-                        g_tma2d(st + C::kBAtom, map, T.kbase + ks * C::kSK + 128, row0, bar);
-                    } else {
-                        g_expect(bar, uint32_t(T.bn) * 256u);
-                        g_tma2d(st, map, T.kbase + ks * C::kSK, row0, bar);
-                        g_tma2d(st + C::kBAtom, map, T.kbase + ks * C::kSK + 64, row0, bar);
-                    }
+                    g_expect(bar, uint32_t(T.bn) * 256u);
+                    g_tma2d(st, map, T.kbase + ks * C::kSK, row0, bar);
+                    g_tma2d(st + C::kBAtom, map, T.kbase + ks * C::kSK + 64, row0, bar);
                 }
                 __syncwarp();
             }
@@ -445,8 +465,13 @@ __global__ void __launch_bounds__(G_THREADS, 1) tc_grouped_gemm(const __grid_con
             for (uint32_t n = first; n < bc; n++) g_drain_wait(g_smem(&b_full[n % C::kBStages]), (n / C::kBStages) & 1);
         }
         __syncwarp();
-    } else if (warp == 2) {
+    } else if (warp == 2 || (C::kI8 && warp == 3)) {
         // ---------------- MMA issuer (whole warp, one lane issues) ----------------
+        // The 8-bit path has two issuers, warps 2 and 3, taking the even and odd
+        // steps: its steps share no accumulator, and one issuing warp alone
+        // cannot keep up with the weight stream (each step costs it about a
+        // thousand cycles of serial work around eight or sixteen MMAs).
+        const uint32_t n_iss = C::kI8 ? 2u : 1u, iss = uint32_t(warp - 2);
         uint32_t bc = 0, ac = 0, pc = 0;
         int t = 0;
         for (int tile = blockIdx.x; tile < ntiles && !s_abort; tile += gridDim.x, t++) {
@@ -461,27 +486,29 @@ __global__ void __launch_bounds__(G_THREADS, 1) tc_grouped_gemm(const __grid_con
             g_fence_after();
             bool ok = true;
             for (int ks = 0; ks < KS; ks++) {
+                if (C::kI8 && bc % n_iss != iss) {      // the other issuer's step
+                    bc++;
+                    ac++;
+                    continue;
+                }
                 const int sb = bc % C::kBStages, sa = ac % C::kAStages;
                 if (!g_wait_w(g_smem(&b_full[sb]), (bc / C::kBStages) & 1, &s_abort)) { ok = false; break; }
+                if (C::kI8) g_fence_proxy_async();      // B was written through the generic proxy
                 if (C::kTmemA) {
                     if (!g_wait_w(g_smem(&a_full[sa]), (ac / C::kAStages) & 1, &s_abort)) { ok = false; break; }
                 } else {
                     if (!g_wait_w(g_smem(&pk_full[pc % NPK]), (pc / NPK) & 1, &s_abort)) { ok = false; break; }
                 }
                 if (C::kI8) {
-                    // every step into the next accumulator buffer.  The epilogue frees
-                    // them in order, so one wait per half ring covers the next kAccBufs / 2 steps.
-                    constexpr int kHalf = C::kAccBufs / 2;
+                    // every step into the next accumulator buffer, freed by the epilogue
                     const int bi = bc % C::kAccBufs;
-                    if (bc >= uint32_t(C::kAccBufs) && bc % kHalf == 0) {
-                        const uint32_t y = bc - C::kAccBufs + kHalf - 1;      // last earlier user of these buffers
-                        if (!g_wait_w(g_smem(&acc_empty[y % C::kAccBufs]), (y / C::kAccBufs) & 1, &s_abort)) { ok = false; break; }
-                    }
+                    if (bc >= uint32_t(C::kAccBufs) &&
+                        !g_wait_w(g_smem(&acc_empty[bi]), ((bc / C::kAccBufs) - 1) & 1, &s_abort)) { ok = false; break; }
                     d = tmem + bi * C::kAccCols;
                 }
                 g_fence_after();
                 const uint32_t b0 = g_smem(bring + sb * C::kBStageBytes);
-                const uint32_t at = tmem + 256 + sa * C::kAStageCols;
+                const uint32_t at = tmem + C::kABase + sa * C::kAStageCols;
                 const uint32_t a0 = g_smem(pk + (pc % NPK) * C::kPkStageBytes);
                 if (g_elect()) {
 #pragma unroll
@@ -670,6 +697,61 @@ __global__ void __launch_bounds__(G_THREADS, 1) tc_grouped_gemm(const __grid_con
             __syncwarp();
             if (lane == 0) g_arrive(g_smem(&acc_empty[buf]));
         }
+    } else if (warp >= 8 && C::kI8) {
+        // ---------------- 8-bit int4 unpacking ----------------
+        // Two groups of four warps take alternate weight stages; a warp unpacks
+        // its 32 rows of every matrix of the stage.  A warp learns that its
+        // tensor-memory stores have landed only by waiting for all of them, so
+        // one group's wait overlaps the other group's stage.  Pieces of 32
+        // bytes of a row (two chunks, 16 TMEM columns) are software-pipelined:
+        // the next piece is unpacked while the store of the current one is in
+        // flight.
+        constexpr int kPieces = C::kNMat * 4;          // per row and weight stage (K = 256 of each matrix)
+        constexpr int kNBuf = 4;
+        const int q = warp & 3, grp = (warp - 8) >> 2;
+        const int r = q * 32 + lane;
+        const uint32_t lane_addr = uint32_t(q * 32) << 16;
+        uint32_t pc = 0;
+        bool ok = true;
+        for (int tile = blockIdx.x; tile < ntiles && ok && !s_abort; tile += gridDim.x) {
+            for (int ps = 0; ps < NPS; ps++, pc++) {
+                if (int(pc & 1) != grp) continue;
+                const int s = pc % NPK;
+                if (!g_wait_w(g_smem(&pk_full[s]), (pc / NPK) & 1, &s_abort)) { ok = false; break; }
+                const uint8_t* st = pk + s * C::kPkStageBytes;
+                uint32_t o[kNBuf][16];
+                auto unpack = [&](auto uc) {
+                    constexpr int u = decltype(uc)::value, m = u / 4, c0 = 2 * (u % 4);
+                    const uint8_t* wt = st + m * C::kMatBytes;
+                    const uint4 w0 = *reinterpret_cast<const uint4*>(wt + g_swz(r, c0));
+                    const uint4 w1 = *reinterpret_cast<const uint4*>(wt + g_swz(r, c0 + 1));
+                    g_dq_int4_i8<0>(w0, o[u % kNBuf]);
+                    g_dq_int4_i8<8>(w1, o[u % kNBuf]);
+                };
+                unpack(std::integral_constant<int, 0>{});
+                const int sa = pc % C::kAStages;
+                if (pc >= uint32_t(C::kAStages) && !g_wait_w(g_smem(&done[(pc - C::kAStages) % G_DONE]),
+                                                             ((pc - C::kAStages) / G_DONE) & 1, &s_abort)) {
+                    ok = false;
+                    break;
+                }
+                g_fence_after();
+                const uint32_t a0 = tmem + lane_addr + C::kABase + sa * C::kAStageCols;
+                g_static_for<0, kPieces>([&](auto uc) {
+                    constexpr int u = decltype(uc)::value;
+                    g_st16(a0 + (u / 4) * C::kAColsK + (u % 4) * 16, o[u % kNBuf]);
+                    if constexpr (u + 1 < kPieces) unpack(std::integral_constant<int, u + 1>{});
+                });
+                g_st_wait();
+                g_fence_before();
+                __syncwarp();
+                if (lane == 0) {
+                    g_arrive(g_smem(&a_full[sa]));
+                    g_arrive(g_smem(&pk_empty[s]));
+                }
+            }
+        }
+        if (!ok) fail();
     } else if (warp >= 8 && C::kTmemA) {
         // ---------------- dequantisation ----------------
         // A weight stage (K = 256, 8 chunks of 16 bytes per row) holds kAPerPk
@@ -683,7 +765,7 @@ __global__ void __launch_bounds__(G_THREADS, 1) tc_grouped_gemm(const __grid_con
         const int q = warp & 3, hsel = (warp - 8) >> 2;
         const int r = q * 32 + lane;                   // weight row within the tile
         const uint32_t lane_addr = uint32_t(q * 32) << 16;
-        const uint32_t colw = 256 + (GU ? hsel * C::kAColsK : hsel * kPer * C::kChunkCols);
+        const uint32_t colw = C::kABase + (GU ? hsel * C::kAColsK : hsel * kPer * C::kChunkCols);
         uint32_t pc = 0;
         int t = 0;
         bool ok = true;
@@ -715,9 +797,7 @@ __global__ void __launch_bounds__(G_THREADS, 1) tc_grouped_gemm(const __grid_con
                     constexpr int i = decltype(ic)::value, j = i / kPer, l = i % kPer;
                     const int c = (8 / C::kAPerPk) * j + (GU ? l : kPer * hsel + l);
                     const uint4 w = *reinterpret_cast<const uint4*>(wt + g_swz(r, c));
-                    if (FMT == FMT_INT4_I8) {
-                        g_dq_int4_i8(w, o[i % kNBuf]);
-                    } else if (FMT == MOE_FMT_INT4_G128) {
+                    if (FMT == MOE_FMT_INT4_G128) {
                         g_dq_int4(w, scw >> (16 * j), o[i % kNBuf]);
                     } else {
                         // the two E4M3 scales of chunk c are bytes 2c and 2c+1
@@ -740,8 +820,7 @@ __global__ void __launch_bounds__(G_THREADS, 1) tc_grouped_gemm(const __grid_con
                         }
                         g_fence_after();
                     }
-                    if constexpr (C::kI8) g_st8(tmem + lane_addr + colw + sa * C::kAStageCols + l * C::kChunkCols, o[i % kNBuf]);
-                    else g_st16(tmem + lane_addr + colw + sa * C::kAStageCols + l * C::kChunkCols, o[i % kNBuf]);
+                    g_st16(tmem + lane_addr + colw + sa * C::kAStageCols + l * C::kChunkCols, o[i % kNBuf]);
                     if constexpr (i + 1 < kChunks) dq(std::integral_constant<int, i + 1>{});
                     if (l == kPer - 1) {
                         g_st_wait();
@@ -1027,7 +1106,7 @@ int launch_grouped_gemm(const GemvProblem& p, bool gateup, int rows, const GemmB
         if (gateup) G_TRY(g_map(&a.tm_s1, false, p.s1, in / 16, wrows, uint64_t(in) / 16, 16, 128, false));
     }
     if (i8)
-        G_TRY(g_map(&a.tm_b[0], false, bsrc, in, uint64_t(rows) * 3, uint64_t(in), 128, 16, true));
+        a.bdig = static_cast<const uint8_t*>(bsrc);
     else
         for (int i = 0; i < G_NB_MAPS; i++)
             G_TRY(g_map(&a.tm_b[i], true, bsrc, in, uint64_t(rows), uint64_t(in) * 2, 64, uint32_t(16 * (i + 1)), true));

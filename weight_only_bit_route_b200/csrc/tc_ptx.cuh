@@ -23,10 +23,14 @@ __device__ __forceinline__ unsigned long long g_timer() {
     asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
     return t;
 }
+// One poll of an mbarrier phase.  A thread whose phase is not complete yet is
+// suspended until it completes or for at most G_SUSPEND_NS, so waiting warps
+// take no issue slots from the warps that work.
+constexpr uint32_t G_SUSPEND_NS = 200000;
 __device__ __forceinline__ bool g_try(uint32_t bar, uint32_t parity) {
     uint32_t ok;
-    asm volatile("{ .reg .pred p; mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2; selp.u32 %0, 1, 0, p; }"
-                 : "=r"(ok) : "r"(bar), "r"(parity) : "memory");
+    asm volatile("{ .reg .pred p; mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3; selp.u32 %0, 1, 0, p; }"
+                 : "=r"(ok) : "r"(bar), "r"(parity), "r"(G_SUSPEND_NS) : "memory");
     return ok != 0;
 }
 // Bounded wait: false after about 2 s, or as soon as another role has aborted.
@@ -120,11 +124,16 @@ __device__ __forceinline__ void g_st16(uint32_t taddr, const uint32_t (&v)[16]) 
                    "r"(v[8]), "r"(v[9]), "r"(v[10]), "r"(v[11]), "r"(v[12]), "r"(v[13]), "r"(v[14]), "r"(v[15])
                  : "memory");
 }
-__device__ __forceinline__ void g_st8(uint32_t taddr, const uint32_t* v) {
-    asm volatile("tcgen05.st.sync.aligned.32x32b.x8.b32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8};"
-                 ::"r"(taddr), "r"(v[0]), "r"(v[1]), "r"(v[2]), "r"(v[3]), "r"(v[4]), "r"(v[5]), "r"(v[6]), "r"(v[7])
-                 : "memory");
+// 16-byte global -> shared copy outside the tensor-copy engine (zero fill past
+// src_size), and an mbarrier arrival (counted against the expected arrivals)
+// once every such copy of the calling thread has landed.
+__device__ __forceinline__ void g_cp16(uint32_t dst, const void* src, uint32_t src_size) {
+    asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(dst), "l"(src), "r"(src_size) : "memory");
 }
+__device__ __forceinline__ void g_cp_arrive(uint32_t bar) {
+    asm volatile("cp.async.mbarrier.arrive.noinc.shared::cta.b64 [%0];" ::"r"(bar) : "memory");
+}
+__device__ __forceinline__ void g_fence_proxy_async() { asm volatile("fence.proxy.async.shared::cta;" ::: "memory"); }
 __device__ __forceinline__ void g_st_wait() { asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory"); }
 __device__ __forceinline__ uint32_t g_e2m1x2_f16x2(uint32_t byte) {
     uint32_t h;
