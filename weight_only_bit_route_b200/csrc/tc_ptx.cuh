@@ -23,14 +23,10 @@ __device__ __forceinline__ unsigned long long g_timer() {
     asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
     return t;
 }
-// One poll of an mbarrier phase.  A thread whose phase is not complete yet is
-// suspended until it completes or for at most G_SUSPEND_NS, so waiting warps
-// take no issue slots from the warps that work.
-constexpr uint32_t G_SUSPEND_NS = 200000;
 __device__ __forceinline__ bool g_try(uint32_t bar, uint32_t parity) {
     uint32_t ok;
-    asm volatile("{ .reg .pred p; mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3; selp.u32 %0, 1, 0, p; }"
-                 : "=r"(ok) : "r"(bar), "r"(parity), "r"(G_SUSPEND_NS) : "memory");
+    asm volatile("{ .reg .pred p; mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2; selp.u32 %0, 1, 0, p; }"
+                 : "=r"(ok) : "r"(bar), "r"(parity) : "memory");
     return ok != 0;
 }
 // Bounded wait: false after about 2 s, or as soon as another role has aborted.
