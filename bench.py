@@ -126,14 +126,6 @@ def build_layer(moe, wl, seed=0, device="cuda"):
     return x, layer
 
 
-def launches_per_step(wl):
-    """Kernel launches of one layer call (fixed by the composition in the C ABI)."""
-    n = 2 + 3 + 1 + 1 + 1      # router (logits, top-k), bucketing (3), gate/up, down, combine
-    if wl.shared:
-        n += 3                  # shared routing, shared gate/up, shared down
-    return n
-
-
 # ---------------------------------------------------------------------------
 # clocks during the timed region
 # ---------------------------------------------------------------------------
@@ -313,6 +305,7 @@ def main():
     if dist:
         dist.barrier()
     torch.cuda.synchronize()
+    launches0 = moe.launch_count()
     with ClockSampler(local_rank) as clk:
         for i in range(args.steps):
             flush.zero_()
@@ -320,6 +313,7 @@ def main():
             step()
             evs[i][1].record(stream)
         torch.cuda.synchronize()
+    launches = moe.launch_count() - launches0      # the library's own kernels in the timed region
     if dist:
         dist.barrier()
     step_ms = [a.elapsed_time(b) for a, b in evs]
@@ -402,7 +396,7 @@ def main():
         "roofline": roof,
         "e2e": {"value": round(world * T / (e_ms * 1e-3), 1), "unit": UNIT,
                 "h2d_bytes_per_step": int(x.numel() * 2), "d2h_bytes_per_step": int(y.numel() * 2)},
-        "gpu_launches": launches_per_step(wl) * args.steps,
+        "gpu_launches": launches,
         "clocks": clk.summary(),
     }
     if rank == 0 and world == 1 and not args.no_cpu_baseline:

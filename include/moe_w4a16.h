@@ -42,8 +42,9 @@
  *   - Intermediates: h_perm is bf16 [rows, F]; y_perm is bf16 [rows, H].
  *   - The workspace `ws` (ws_bytes bytes, 256-byte aligned) must be zero-filled
  *     once before first use (moe_workspace_init); kernels leave their counters
- *     at zero again when they finish.  Its first 256 bytes hold the status
- *     word; the step calls use the bytes after them as scratch (sizes below),
+ *     at zero again when they finish.  Its first 1024 bytes hold the status
+ *     word and those counters; the step calls use the bytes after them as
+ *     scratch (sizes below),
  *     the layer entries the whole of moe_workspace_bytes().  A workspace of
  *     moe_workspace_bytes(T, H, E, F, top_k) bytes serves every call at those
  *     sizes.  Calls that share a workspace must not run concurrently.
@@ -116,6 +117,11 @@ int moe_read_status(void* ws, moe_stream_t stream, int32_t* status_out);
 /* Static description of a status code. */
 const char* moe_status_string(int status);
 
+/* Number of kernels this library has launched in this process since it was
+ * loaded (a host-side count of successful launch calls, over every stream
+ * and device).  For measurement; no part of the layer's arithmetic. */
+uint64_t moe_launch_count(void);
+
 /* ---------------------------------------------------------------------- */
 /* Hot-path steps                                                          */
 /* ---------------------------------------------------------------------- */
@@ -129,7 +135,7 @@ const char* moe_status_string(int status);
  * From 64 tokens the logits run on the tensor cores: router_w is split into
  * three bf16 planes (hi + mid + lo) whose bf16 x bf16 products are exact in
  * fp32, accumulated in fp32.
- * ws (256-byte aligned): at least 256 + a(4*T*E) + a(6*E*H) bytes, a()
+ * ws (256-byte aligned): at least 1024 + a(4*T*E) + a(6*E*H) bytes, a()
  * rounding up to a multiple of 256. */
 int moe_route_topk(const void* x, int T, int H, const float* router_w,
                    const float* router_bias, int E, int top_k, int32_t* topk_ids,
@@ -143,7 +149,7 @@ int moe_route_topk(const void* x, int T, int H, const float* router_w,
  * row_slot: int32 [R] (out), the slot placed at permuted row r;
  * slot_row: int32 [R] (out), its inverse.
  * Rows of one expert are ordered by slot (token, then rank j).
- * ws: at least 256 + 4*E*ceil(T*top_k / 4096) bytes. */
+ * ws: at least 1024 + 4*E*ceil(T*top_k / 4096) bytes. */
 int moe_permute(const int32_t* topk_ids, int T, int top_k, int E,
                 int32_t* expert_offsets, int32_t* row_slot, int32_t* slot_row,
                 void* ws, size_t ws_bytes, moe_stream_t stream);
@@ -180,7 +186,7 @@ int moe_permute_noalloc(const int32_t* topk_ids, int T, int top_k, int E,
  * 8-bit digits of a per-row 24-bit fixed point, exact integer sums per scale
  * group), everything else on the 16-bit one; other shapes stream the weights
  * with a GEMV.
- * ws (256-byte aligned): at least 256 + a(16*(E+2)) + max(a(rows*H/8) +
+ * ws (256-byte aligned): at least 1024 + a(16*(E+2)) + max(a(rows*H/8) +
  * a(2*rows*H), a(4*rows) + a(rows*H/32) + a(c*rows*H)) bytes, c = 3 for
  * rows <= 512 and 2 above, plus a(8*k*rows*F) for a BF16 bank with E = 1 and
  * rows <= 64 (split-K partial sums, k = 8 halved while H is not a multiple of
@@ -199,7 +205,7 @@ int moe_grouped_w4a16_swiglu(const void* x, int T, int H,
  * down: bank [E, H, F]; y_perm: bf16 [rows, H] (out).  The path follows the
  * gate/up call's rule with the roles of H and F exchanged (F a multiple of
  * 256, H of 128 for the GEMM).
- * ws (256-byte aligned): at least 256 + a(16*(E+2)) + max(a(rows*F/8) +
+ * ws (256-byte aligned): at least 1024 + a(16*(E+2)) + max(a(rows*F/8) +
  * a(2*rows*F), a(4*rows) + a(rows*F/32) + a(c*rows*F)) bytes, c = 3 for
  * rows <= 512 and 2 above, plus a(4*k*rows*H) for a BF16 bank with E = 1 and
  * rows <= 64 (k = 4 halved while F is not a multiple of 128*k); a() rounds up

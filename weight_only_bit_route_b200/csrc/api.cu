@@ -2,6 +2,7 @@
 // validation, workspace carving and kernel composition.  Nothing here touches
 // the data; every step runs in the kernels of this library.
 #include <algorithm>
+#include <atomic>
 
 #include "moe_internal.cuh"
 
@@ -61,6 +62,7 @@ int run_problem(const GemvProblem& p, bool gateup, int rows, int act_rows, void*
     GemmBuffers b = gb;
     b.ksplit = shared_ksplit(p.E, p.fmt, gateup, rows, p.in_dim);
     b.partial = partial;
+    b.tile_cnt = p.status + 16;            // the control block's split-K counters
     return launch_grouped_gemm(p, gateup, rows, b, s);
 }
 
@@ -205,6 +207,13 @@ int layer_run(const void* x, int T, const moe_layer* L, void* y, void* ws, cudaS
 
 }  // namespace
 
+namespace moe {
+namespace {
+std::atomic<uint64_t> g_launches{0};
+}
+void count_launch() { g_launches.fetch_add(1, std::memory_order_relaxed); }
+}  // namespace moe
+
 extern "C" {
 
 size_t moe_workspace_bytes(int T, int H, int E, int F, int top_k) {
@@ -226,6 +235,8 @@ int moe_read_status(void* ws, moe_stream_t stream, int32_t* status_out) {
     if (v != 0 && cudaMemsetAsync(ws, 0, 4, cs(stream)) != cudaSuccess) return MOE_ERR_CUDA;
     return MOE_OK;
 }
+
+uint64_t moe_launch_count(void) { return moe::g_launches.load(std::memory_order_relaxed); }
 
 const char* moe_status_string(int status) {
     switch (status) {
@@ -379,7 +390,7 @@ int moe_quantize_nvfp4(const void* w, int64_t rows, int64_t cols, uint8_t* packe
     if (cols % 16) return MOE_ERR_UNSUPPORTED;
     if (rows == 0 || cols == 0) return MOE_OK;
     if (!w || !packed || !scales || !global_scale || !al16(w)) return MOE_ERR_INVALID_ARG;
-    MOE_TRY(check_ws(ws, ws_bytes, 256));
+    MOE_TRY(check_ws(ws, ws_bytes, 256));                 // uses only the control block's amax word
     return launch_quant_nvfp4(reinterpret_cast<const __nv_bfloat16*>(w), rows, cols, packed, scales,
                               global_scale, at<uint32_t>(ws, 8), cs(stream));
 }

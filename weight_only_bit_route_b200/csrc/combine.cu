@@ -59,6 +59,7 @@ __global__ void shared_routing_kernel(int T, int k, int32_t* sh_offsets, int32_t
 
 int launch_shared_routing(int T, int k, int32_t* sh_offsets, int32_t* sh_rowslot, cudaStream_t s) {
     shared_routing_kernel<<<(T + 255) / 256, 256, 0, s>>>(T, k, sh_offsets, sh_rowslot);
+    count_launch();
     return cudaGetLastError() == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
 }
 

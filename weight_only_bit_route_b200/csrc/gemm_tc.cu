@@ -134,6 +134,7 @@ struct GCfg {
 
 constexpr int G_DONE = 16;                                          // "stage done" barrier ring
 constexpr int G_SC_MAX = 8;                                         // int4 scale buffers (one tile each)
+constexpr int G_KSPLIT_MAX = 8;                                     // split-K slices summed inside the GEMM
 
 constexpr int G_NB_MAPS = 8;                                        // box heights 16, 32, ..., 128
 
@@ -156,6 +157,8 @@ struct GArgs {
     const uint8_t* bdig;             // 8-bit int4: the digit rows [3 rows][in]
     int E, out_dim, in_dim, perm_out;
     int ksplit, rows;                // K slices per (m-tile, n-tile); activation rows of the problem
+    int* tile_cnt;                   // split-K: zeroed arrival counters, four per (m-tile, n-tile); the last
+                                     // epilogue warp of each quarter sums the slices (else a kernel does)
     int npk;                         // weight stages in the shared-memory ring (2 .. kPkMax)
     int nsc;                         // int4 scale buffers (2 .. G_SC_MAX)
 };
@@ -209,7 +212,7 @@ __device__ __forceinline__ void g_dq_int4_i8(const uint4 w, uint32_t (&o)[16]) {
     }
 }
 
-struct GTile { int e, m0, n0, nval, bn, ebase, ks, kbase; };
+struct GTile { int e, m0, n0, nval, bn, ebase, ks, kbase, mn; };
 
 // ---------------------------------------------------------------------------
 // Kernel
@@ -342,6 +345,7 @@ __global__ void __launch_bounds__(G_THREADS, 1) tc_grouped_gemm(const __grid_con
         t.ks = local % ksplit;                                      // K slice fastest
         t.kbase = t.ks * kc;
         const int mn = local / ksplit;
+        t.mn = mn;
         t.m0 = (mn / ntile) * G_BM;
         t.n0 = (mn % ntile) * per;
         t.nval = min(per, n_e - t.n0);
@@ -665,7 +669,7 @@ __global__ void __launch_bounds__(G_THREADS, 1) tc_grouped_gemm(const __grid_con
                 if (GU) g_ld16(acc0 + C::kUpCol + c, u);
                 g_ld_wait();
                 if (ksplit > 1) {
-                    // split-K: raw fp32 sums of this K slice; a reduction kernel finishes the rows
+                    // split-K: raw fp32 sums of this K slice; the tile's last slice (or a kernel) finishes the rows
 #pragma unroll
                     for (int j = 0; j < 16; j++) {
                         if (c + j < T.nval) {
@@ -696,6 +700,47 @@ __global__ void __launch_bounds__(G_THREADS, 1) tc_grouped_gemm(const __grid_con
             g_fence_before();
             __syncwarp();
             if (lane == 0) g_arrive(g_smem(&acc_empty[buf]));
+            if (ksplit > 1 && a.tile_cnt) {
+                // Per (tile, quarter of its rows): the epilogue warp that writes the last K slice of
+                // its 32 rows sums all slices in slice order and writes the bf16 rows (E = 1: no
+                // routing weight on gate/up, the slot weight on down).  Warps count separately, so
+                // no warp ever waits for another here.
+                __threadfence();
+                __syncwarp();
+                int last = 0;
+                if (lane == 0) last = atomicAdd(&a.tile_cnt[T.mn * 4 + q], 1) == ksplit - 1;
+                if (__shfl_sync(0xffffffffu, last, 0)) {
+                    __threadfence();
+                    const size_t plane = size_t(a.rows) * a.out_dim;
+                    for (int j = 0; j < T.nval; j++) {
+                        const size_t o = size_t(rbase + j) * a.out_dim + f;
+                        // all slices' loads first (ksplit <= G_KSPLIT_MAX), then the sums in slice order
+                        float pg[G_KSPLIT_MAX], pu[G_KSPLIT_MAX];
+#pragma unroll
+                        for (int k = 0; k < G_KSPLIT_MAX; k++) {
+                            pg[k] = k < ksplit ? a.partial[(size_t(k) * C::kNMat) * plane + o] : 0.f;
+                            pu[k] = (GU && k < ksplit) ? a.partial[(size_t(k) * C::kNMat + 1) * plane + o] : 0.f;
+                        }
+                        float gs = 0.f, us = 0.f;
+#pragma unroll
+                        for (int k = 0; k < G_KSPLIT_MAX; k++) {
+                            if (k < ksplit) {
+                                gs += pg[k];
+                                us += pu[k];
+                            }
+                        }
+                        float v;
+                        if (GU) {
+                            v = gs / (1.0f + expf(-gs)) * us;
+                        } else {
+                            const float w = a.topk_w ? a.topk_w[a.row_slot[rbase + j]] : 1.f;
+                            v = w * gs;
+                        }
+                        a.out[o] = __float2bfloat16_rn(v);
+                    }
+                    if (lane == 0) a.tile_cnt[T.mn * 4 + q] = 0;          // ready for the next call
+                }
+            }
         }
     } else if (warp >= 8 && C::kI8) {
         // ---------------- 8-bit int4 unpacking ----------------
@@ -1128,13 +1173,17 @@ int launch_grouped_gemm(const GemvProblem& p, bool gateup, int rows, const GemmB
     a.partial = buf.partial;
     a.rows = rows;
     a.zsum = buf.zbuf;
+    // split-K tiles finish in the GEMM when their counters fit the workspace's control block
+    const int ntile_max = (rows + (gateup ? 63 : 127)) / (gateup ? 64 : 128);
+    if (ksplit > 1 && ksplit <= G_KSPLIT_MAX && buf.tile_cnt && 4 * (out / G_BM) * ntile_max <= kTileCounters)
+        a.tile_cnt = buf.tile_cnt;
 
     if (i8) return gateup ? g_launch<FMT_INT4_I8, true>(a, s) : g_launch<FMT_INT4_I8, false>(a, s);
     if (i4) return gateup ? g_launch<MOE_FMT_INT4_G128, true>(a, s) : g_launch<MOE_FMT_INT4_G128, false>(a, s);
     if (nv) return gateup ? g_launch<MOE_FMT_NVFP4, true>(a, s) : g_launch<MOE_FMT_NVFP4, false>(a, s);
     const int rc = gateup ? g_launch<MOE_FMT_BF16, true>(a, s) : g_launch<MOE_FMT_BF16, false>(a, s);
     if (rc != MOE_OK) return rc;
-    if (ksplit > 1) {
+    if (ksplit > 1 && !a.tile_cnt) {
         const size_t n4 = size_t(rows) * out / 4;
         const int blocks = int(std::min<size_t>((n4 + 255) / 256, 148 * 8));
         if (launch_pdl(g_splitk_finish, dim3(blocks), dim3(256), 0, s, static_cast<const float*>(buf.partial), ksplit,

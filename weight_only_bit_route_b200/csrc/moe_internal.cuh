@@ -18,8 +18,9 @@ constexpr int kMaxDecodeT = 64;
 
 // ---------------------------------------------------------------------------
 // Workspace layout.  Every region starts on a 256-byte boundary.
-// ctrl (256 B): [0] status word, [1] router arrival counter, [2] quantiser
-//               amax (float bits), [3..] reserved.
+// ctrl (1 KB): [0] status word, [1] router arrival counter, [2] quantiser
+//              amax (float bits), [3..15] reserved, [16..255] split-K tile
+//              arrival counters (left at zero by every call).
 // ---------------------------------------------------------------------------
 struct WsLayout {
     size_t ctrl, logits, wsplit, hist, offsets, row_slot, slot_row, ids, tw;
@@ -45,8 +46,8 @@ __device__ __forceinline__ float warp_sum(float v, int width) {
     return v;
 }
 
-// Step-level calls use the workspace as [ctrl 256 B][their own scratch].
-constexpr size_t kStepScratch = 256;
+// Step-level calls use the workspace as [ctrl 1 KB][their own scratch].
+constexpr size_t kStepScratch = 1024;
 // router: logits [T, E] fp32, then the three bf16 planes of the router weights
 // used by the tensor-core path (3 * E * H bf16)
 inline size_t route_scratch(int T, int E, int H) { return align256(size_t(T) * E * 4) + align256(size_t(E) * H * 6); }
@@ -96,7 +97,7 @@ inline WsLayout ws_layout(int T, int H, int E, int F, int k) {
     size_t nb = (R + kPermChunk - 1) / kPermChunk;
     if (nb == 0) nb = 1;
     size_t o = 0;
-    L.ctrl = o;       o = align256(o + 256);
+    L.ctrl = o;       o = align256(o + kStepScratch);
     L.logits = o;     o = align256(o + size_t(T) * E * 4);
     L.wsplit = o;     o = align256(o + size_t(E) * H * 6);
     L.hist = o;       o = align256(o + nb * E * 4);
@@ -119,6 +120,9 @@ inline WsLayout ws_layout(int T, int H, int E, int F, int k) {
     return L;
 }
 
+// Host-side count of successful kernel launches (moe_launch_count).
+void count_launch();
+
 // Launch with programmatic dependent launch allowed: the kernel may start
 // while the previous kernel on the stream finishes, and must execute
 // griddepcontrol.wait before it reads anything that kernel wrote.
@@ -134,7 +138,9 @@ inline cudaError_t launch_pdl(K kern, dim3 grid, dim3 block, size_t smem, cudaSt
     attr[0].val.programmaticStreamSerializationAllowed = 1;
     cfg.attrs = attr;
     cfg.numAttrs = 1;
-    return cudaLaunchKernelEx(&cfg, kern, args...);
+    const cudaError_t e = cudaLaunchKernelEx(&cfg, kern, args...);
+    if (e == cudaSuccess) count_launch();
+    return e;
 }
 
 // ---------------------------------------------------------------------------
@@ -221,7 +227,9 @@ struct GemmBuffers {
     float* partial;      // split_bytes(...) bytes
     int i8;              // int4 on the 8-bit MMA with per-group accumulation (small batches)
     float* zbuf;         // i8: 8 * group sums of the fixed-point rows [rows][zsum_stride(in)]
+    int* tile_cnt;       // split-K: kTileCounters zeroed ints (the control block's [16..255])
 };
+constexpr int kTileCounters = 240;
 
 
 // Prefill-shaped grouped GEMM (tcgen05) for one problem; rows: activation

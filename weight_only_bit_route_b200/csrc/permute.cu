@@ -137,9 +137,12 @@ int launch_permute(const int32_t* ids, int T, int k, int E, int32_t* offsets,
     const int R = T * k;
     const int nb = (R + kPermChunk - 1) / kPermChunk;
     perm_count<<<nb, kPermThreads, 0, s>>>(ids, R, E, hist, status);
+    count_launch();
     perm_scan<<<1, 1024, 0, s>>>(hist, nb, E, offsets);
+    count_launch();
     const size_t smem = size_t(kPermWarps) * E * sizeof(int32_t);
     perm_scatter<<<nb, kPermThreads, smem, s>>>(ids, R, E, hist, row_slot, slot_row);
+    count_launch();
     return cudaGetLastError() == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
 }
 

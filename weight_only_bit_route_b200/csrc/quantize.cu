@@ -128,6 +128,7 @@ int launch_quant_int4(const __nv_bfloat16* w, int64_t rows, int64_t cols, int32_
                       __nv_bfloat16* scales, cudaStream_t s) {
     const long long n = rows * (cols / 128);
     quant_int4_kernel<<<int((n + 127) / 128), 128, 0, s>>>(w, rows, cols, packed, scales);
+    count_launch();
     return cudaGetLastError() == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
 }
 
@@ -137,8 +138,10 @@ int launch_quant_nvfp4(const __nv_bfloat16* w, int64_t rows, int64_t cols, uint8
     const long long n = rows * cols;
     int blocks = int(std::min<long long>((n + 255) / 256, 148 * 8));
     amax_kernel<<<blocks, 256, 0, s>>>(w, n, amax_slot);
+    count_launch();
     const long long nb = rows * (cols / 16);
     quant_nvfp4_kernel<<<int((nb + 255) / 256), 256, 0, s>>>(w, rows, cols, amax_slot, packed, scales, global);
+    count_launch();
     return cudaGetLastError() == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
 }
 

@@ -378,9 +378,11 @@ int launch_route(const __nv_bfloat16* x, int T, int H, const float* Wr, const fl
         if (T <= 8) {
             dim3 grid((E + epb - 1) / epb, 1);
             router_logits_rows<8><<<grid, block, 0, s>>>(x, T, H, Wr, E, logits);
+            count_launch();
         } else {
             dim3 grid((E + epb - 1) / epb, (T + 7) / 8);
             router_logits_rows<8><<<grid, block, 0, s>>>(x, T, H, Wr, E, logits);
+            count_launch();
         }
     } else if (T >= kRouterTcMinT && planes) {
         const int rc = launch_router_logits_tc(x, T, H, Wr, E, logits, planes, status, s);
@@ -388,8 +390,10 @@ int launch_route(const __nv_bfloat16* x, int T, int H, const float* Wr, const fl
     } else {
         dim3 grid((E + RT_BN - 1) / RT_BN, (T + RT_BM - 1) / RT_BM);
         router_logits_tiled<<<grid, 256, 0, s>>>(x, T, H, Wr, E, logits);
+        count_launch();
     }
     router_topk<<<(T + 7) / 8, 256, 0, s>>>(logits, bias, T, E, k, ids, w);
+    count_launch();
     return cudaGetLastError() == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
 }
 

@@ -216,6 +216,7 @@ int launch_router_logits_tc(const __nv_bfloat16* x, int T, int H, const float* W
     const size_t n = size_t(E) * H;
     router_split<<<std::min<size_t>((n / 4 + 255) / 256, 148 * 8), 256, 0, s>>>(
         reinterpret_cast<const float4*>(Wr), n / 4, planes);
+    count_launch();
     if (cudaGetLastError() != cudaSuccess) return MOE_ERR_CUDA;
     RtArgs a;
     memset(&a, 0, sizeof(a));

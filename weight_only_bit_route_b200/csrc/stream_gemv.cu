@@ -841,7 +841,9 @@ static cudaError_t launch_ex(K kern, dim3 grid, dim3 block, size_t smem, cudaStr
     attr[0].val.programmaticStreamSerializationAllowed = 1;
     cfg.attrs = attr;
     cfg.numAttrs = pdl ? 1 : 0;
-    return cudaLaunchKernelEx(&cfg, kern, args...);
+    const cudaError_t e = cudaLaunchKernelEx(&cfg, kern, args...);
+    if (e == cudaSuccess) count_launch();
+    return e;
 }
 
 template <int FMT>

@@ -55,6 +55,7 @@ _sig("moe_workspace_bytes", _SZ, [_I, _I, _I, _I, _I])
 _sig("moe_workspace_init", _I, [_P, _SZ, _P])
 _sig("moe_read_status", _I, [_P, _P, ctypes.POINTER(ctypes.c_int32)])
 _sig("moe_status_string", ctypes.c_char_p, [_I])
+_sig("moe_launch_count", ctypes.c_uint64, [])
 _sig("moe_route_topk", _I, [_P, _I, _I, _P, _P, _I, _I, _P, _P, _P, _SZ, _P])
 _sig("moe_permute", _I, [_P, _I, _I, _I, _P, _P, _P, _P, _SZ, _P])
 _sig("moe_permute_noalloc", _I, [_P, _I, _I, _I, _P, _P, _P, _P])
@@ -71,7 +72,7 @@ def declared_functions():
     """Names of the functions declared in the public header."""
     text = open(HEADER_PATH).read()
     text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
-    return sorted(set(re.findall(r"^\s*(?:int|size_t|const char\*)\s+(moe_\w+)\s*\(", text, flags=re.M)))
+    return sorted(set(re.findall(r"^\s*(?:int|size_t|uint64_t|const char\*)\s+(moe_\w+)\s*\(", text, flags=re.M)))
 
 
 class MoEError(RuntimeError):
@@ -147,6 +148,11 @@ def workspace(T, H, E, F, top_k, device="cuda"):
     ws = torch.empty(n, dtype=torch.uint8, device=device)
     _check("moe_workspace_init", lib.moe_workspace_init(_ptr(ws), n, _stream()))
     return ws
+
+
+def launch_count():
+    """Kernels the library has launched in this process so far."""
+    return int(lib.moe_launch_count())
 
 
 def read_status(ws):
