@@ -248,6 +248,28 @@ def test_layer_streaming_gemv_path(fmt):
     _layer_check(P, bf16_bits(y), np.arange(P.T, dtype=np.int32), ids.cpu().numpy())
 
 
+def _mid(fmt, T):
+    # F = 768 is a multiple of 256 but not of 512: int4 gate/up runs the 8-bit
+    # GEMM (K = H = 1024) while the down GEMM (K = F) takes the 16-bit int4 path,
+    # gathering the natural-order h the 8-bit gate/up wrote
+    base = syn.WORKLOADS[0]
+    return syn.Workload(f"mid_{fmt}_T{T}", T, 1024, 16, 768, base.k, fmt, False, base.router_std, False)
+
+
+@pytest.mark.parametrize("fmt", ["int4", "nvfp4"])
+def test_layer_down_width_not_multiple_of_512(fmt):
+    wl = _mid(fmt, 12)
+    P = build(wl, "quantised", shared=True)
+    L = device_layer(moe, P)
+    ws = _ws(P.T, wl)
+    x = dev_bf16(P.x)
+    y = moe.layer_decode(x, L, ws)
+    ids, _ = moe.route_topk(x, L.router_w, L.router_bias, wl.k, ws)
+    torch.cuda.synchronize()
+    assert moe.read_status(ws) == 0
+    _layer_check(P, bf16_bits(y), np.arange(P.T, dtype=np.int32), ids.cpu().numpy())
+
+
 @pytest.mark.parametrize("T", [5, 300])
 def test_shared_expert_bf16_steps(T):
     wl = syn.WORKLOADS[1]

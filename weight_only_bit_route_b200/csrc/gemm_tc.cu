@@ -105,7 +105,9 @@ struct GCfg {
     static constexpr int kNMat = GU ? 2 : 1;
     static constexpr int kNMax = kI8 ? 5 : (GU ? 64 : 128);        // token rows per tile
     static constexpr int kUpCol = 64;                               // 16-bit paths: up accumulator within a buffer
-    static constexpr int kSK = kI8 ? 256 : 128;                     // K per MMA stage
+    // K per MMA step: 8-bit down steps are K = 512, so that the per-step fixed cost of the
+    // issuer and the unpack warps covers 32 KB of weights, as a gate/up step does
+    static constexpr int kSK = kI8 ? (GU ? 256 : 512) : 128;
     static constexpr int kGroups = kSK / 128;                       // i8: scale groups per MMA stage
     static constexpr int kAccCols = kI8 ? kGroups * kNMat * 16 : 128;   // one accumulator buffer
     // Tensor memory: accumulators in [0, kABase), A stages in [kABase, 512).  The
@@ -114,16 +116,18 @@ struct GCfg {
     static constexpr int kAccBufs = kI8 ? 128 / kAccCols : 256 / kAccCols;
     static constexpr int kABase = kAccBufs * kAccCols;
     static constexpr int kMmaK = kI8 ? 32 : 16;                     // K per MMA instruction
-    static constexpr int kPkK = kTmemA ? 256 : 128;                 // K per weight stage
-    static constexpr int kMatBytes = kTmemA ? G_BM * 128 : G_BM * 256;   // one matrix of a weight stage
+    static constexpr int kPkK = kTmemA ? (kI8 ? kSK : 256) : 128;   // K per weight stage
+    static constexpr int kBoxes = kTmemA ? kPkK / 256 : 2;          // 128-byte-wide TMA boxes per matrix and stage
+    static constexpr int kMatBytes = kTmemA ? G_BM * kPkK / 2 : G_BM * 256;   // one matrix of a weight stage
     static constexpr int kNvScBytes = FMT == MOE_FMT_NVFP4 ? G_BM * 16 : 0;
     static constexpr int kPkStageBytes = kNMat * (kMatBytes + kNvScBytes);
     static constexpr int kPkMax = 12;                               // weight stages: as many as fit, up to this
     static constexpr int kScStages = kI8 ? G_EPI_WARPS : G_DQ_WARPS;     // readers of the int4 scale buffer
     static constexpr int kBAtom = (kI8 ? 16 : kNMax) * 128;         // 128 bytes of K for every B row
-    static constexpr int kBStageBytes = 2 * kBAtom;                 // K = 256 of 8-bit (i8) or 128 of 16-bit operands
-    static constexpr int kBStages = kI8 ? 6 : 4;                    // i8 stages are small; cover the copy latency
-    static constexpr int kAColsK = 64;                              // TMEM columns of one matrix's A stage
+    static constexpr int kBAtoms = kI8 ? kSK / 128 : 2;             // 128-byte K slices per B stage
+    static constexpr int kBStageBytes = kBAtoms * kBAtom;
+    static constexpr int kBStages = kI8 ? (GU ? 6 : 4) : 4;         // i8 stages are small; cover the copy latency
+    static constexpr int kAColsK = kI8 ? kSK / 4 : 64;              // TMEM columns of one matrix's A stage
     static constexpr int kAStageCols = kNMat * kAColsK;
     static constexpr int kAStages = (512 - kABase) / kAStageCols;
     static constexpr int kAPerPk = kPkK / kSK;                      // A stages per weight stage (2, or 1 for i8)
@@ -395,9 +399,13 @@ __global__ void __launch_bounds__(G_THREADS, 1) tc_grouped_gemm(const __grid_con
                 if (g_elect()) {
                     g_expect(bar, C::kPkStageBytes);
                     if (C::kTmemA) {
-                        // 4-bit: 128 bytes of each row = K 256
-                        g_tma2d(st, &a.tm_p0, T.kbase / 2 + ps * 128, row0, bar);
-                        if (GU) g_tma2d(st + C::kMatBytes, &a.tm_p1, T.kbase / 2 + ps * 128, row0, bar);
+                        // 4-bit: 128 bytes of each row = K 256 per box, kBoxes boxes side by side
+#pragma unroll
+                        for (int h = 0; h < C::kBoxes; h++) {
+                            const int x = T.kbase / 2 + ps * (C::kPkK / 2) + h * 128;
+                            g_tma2d(st + h * (G_BM * 128), &a.tm_p0, x, row0, bar);
+                            if (GU) g_tma2d(st + C::kMatBytes + h * (G_BM * 128), &a.tm_p1, x, row0, bar);
+                        }
                         if (FMT == MOE_FMT_NVFP4) {
                             const uint32_t ss = st + C::kNMat * C::kMatBytes;
                             g_tma2d(ss, &a.tm_s0, T.kbase / 16 + ps * 16, row0, bar);
@@ -443,15 +451,20 @@ __global__ void __launch_bounds__(G_THREADS, 1) tc_grouped_gemm(const __grid_con
                 const uint32_t bar = g_smem(&b_full[s]);
                 const uint32_t st = g_smem(bring + s * C::kBStageBytes);
                 if (C::kI8) {
-                    // lane: digit row n = lane / 2 of the tile, 128-byte K half h = lane % 2, as eight
-                    // 16-byte chunks at their 128-byte-swizzled places; rows past the end read as zero
-                    const int n = lane >> 1, h = lane & 1;
+                    // lane: digit row n = lane / 2 of the tile and the 128-byte K slices h, h + 2, ... of the
+                    // stage, each as eight 16-byte chunks at their 128-byte-swizzled places; rows past the end
+                    // read as zero
+                    const int n = lane >> 1;
                     const int grow = row0 + n;
                     const bool in_rows = grow < 3 * a.rows;
-                    const uint8_t* src = a.bdig + size_t(in_rows ? grow : 0) * in_dim + T.kbase + ks * C::kSK + h * 128;
-                    const uint32_t dst = st + h * C::kBAtom + n * 128;
+                    const uint8_t* src = a.bdig + size_t(in_rows ? grow : 0) * in_dim + T.kbase + ks * C::kSK;
 #pragma unroll
-                    for (int c = 0; c < 8; c++) g_cp16(dst + ((c ^ (n & 7)) << 4), src + c * 16, in_rows ? 16u : 0u);
+                    for (int h = lane & 1; h < C::kBAtoms; h += 2) {
+                        const uint32_t dst = st + h * C::kBAtom + n * 128;
+#pragma unroll
+                        for (int c = 0; c < 8; c++)
+                            g_cp16(dst + ((c ^ (n & 7)) << 4), src + h * 128 + c * 16, in_rows ? 16u : 0u);
+                    }
                     g_cp_arrive(bar);
                     continue;
                 }
@@ -751,7 +764,8 @@ __global__ void __launch_bounds__(G_THREADS, 1) tc_grouped_gemm(const __grid_con
         // bytes of a row (two chunks, 16 TMEM columns) are software-pipelined:
         // the next piece is unpacked while the store of the current one is in
         // flight.
-        constexpr int kPieces = C::kNMat * 4;          // per row and weight stage (K = 256 of each matrix)
+        constexpr int kPpm = C::kPkK / 64;             // 32-byte pieces of a row per matrix and stage
+        constexpr int kPieces = C::kNMat * kPpm;
         constexpr int kNBuf = 4;
         const int q = warp & 3, grp = (warp - 8) >> 2;
         const int r = q * 32 + lane;
@@ -766,10 +780,11 @@ __global__ void __launch_bounds__(G_THREADS, 1) tc_grouped_gemm(const __grid_con
                 const uint8_t* st = pk + s * C::kPkStageBytes;
                 uint32_t o[kNBuf][16];
                 auto unpack = [&](auto uc) {
-                    constexpr int u = decltype(uc)::value, m = u / 4, c0 = 2 * (u % 4);
-                    const uint8_t* wt = st + m * C::kMatBytes;
-                    const uint4 w0 = *reinterpret_cast<const uint4*>(wt + g_swz(r, c0));
-                    const uint4 w1 = *reinterpret_cast<const uint4*>(wt + g_swz(r, c0 + 1));
+                    // piece u: matrix m, 16-byte chunks c0 and c0 + 1 of the row, in TMA box c0 / 8
+                    constexpr int u = decltype(uc)::value, m = u / kPpm, c0 = 2 * (u % kPpm);
+                    const uint8_t* wt = st + m * C::kMatBytes + (c0 / 8) * (G_BM * 128);
+                    const uint4 w0 = *reinterpret_cast<const uint4*>(wt + g_swz(r, c0 % 8));
+                    const uint4 w1 = *reinterpret_cast<const uint4*>(wt + g_swz(r, c0 % 8 + 1));
                     g_dq_int4_i8<0>(w0, o[u % kNBuf]);
                     g_dq_int4_i8<8>(w1, o[u % kNBuf]);
                 };
@@ -784,7 +799,7 @@ __global__ void __launch_bounds__(G_THREADS, 1) tc_grouped_gemm(const __grid_con
                 const uint32_t a0 = tmem + lane_addr + C::kABase + sa * C::kAStageCols;
                 g_static_for<0, kPieces>([&](auto uc) {
                     constexpr int u = decltype(uc)::value;
-                    g_st16(a0 + (u / 4) * C::kAColsK + (u % 4) * 16, o[u % kNBuf]);
+                    g_st16(a0 + (u / kPpm) * C::kAColsK + (u % kPpm) * 16, o[u % kNBuf]);
                     if constexpr (u + 1 < kPieces) unpack(std::integral_constant<int, u + 1>{});
                 });
                 g_st_wait();
@@ -1113,7 +1128,8 @@ int launch_grouped_gemm(const GemvProblem& p, bool gateup, int rows, const GemmB
 
     const int in = p.in_dim, out = p.out_dim, E = p.E;
     const bool nv = p.fmt == MOE_FMT_NVFP4, i4 = p.fmt == MOE_FMT_INT4_G128;
-    const bool i8 = i4 && buf.i8;
+    // the 8-bit down GEMM steps in K = 512; other widths take the 16-bit int4 path
+    const bool i8 = i4 && buf.i8 && (gateup || in % 512 == 0);
     if (i8 && (!buf.zbuf || !buf.scale_buf || !buf.act_buf || buf.perm_out || ksplit > 1)) return MOE_ERR_UNSUPPORTED;
     // activation operand rows [rows, in]: bf16 (f16 for NVFP4) in the kernel's order; 8-bit int4: three
     // int8 digit rows per row
