@@ -838,7 +838,7 @@ __global__ void __launch_bounds__(G_THREADS, 1) tc_grouped_gemm(const __grid_con
             }
             for (int ps = 0; ps < NPS && ok; ps++, pc++) {
                 const int s = pc % NPK;
-                if (!g_wait_w(g_smem(&pk_full[s]), (pc / NPK) & 1, &s_abort)) { ok = false; break; }
+                if (!g_wait(g_smem(&pk_full[s]), (pc / NPK) & 1, &s_abort)) { ok = false; break; }
                 const uint8_t* st = pk + s * C::kPkStageBytes;
                 const uint8_t* wt = st + (GU ? hsel * C::kMatBytes : 0);
                 uint32_t scw = 0;                      // int4: bf16 scales of groups 2ps (low) and 2ps+1 (high)
@@ -873,7 +873,7 @@ __global__ void __launch_bounds__(G_THREADS, 1) tc_grouped_gemm(const __grid_con
                     if (l == 0) {
                         const uint32_t acn = pc * C::kAPerPk + j;    // A stage index in this CTA's stream
                         sa = acn % C::kAStages;
-                        if (acn >= uint32_t(C::kAStages) && !g_wait_w(g_smem(&done[(acn - C::kAStages) % G_DONE]),
+                        if (acn >= uint32_t(C::kAStages) && !g_wait(g_smem(&done[(acn - C::kAStages) % G_DONE]),
                                                                       ((acn - C::kAStages) / G_DONE) & 1, &s_abort)) {
                             ok = false;
                             return;
