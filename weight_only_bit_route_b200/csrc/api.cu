@@ -3,6 +3,7 @@
 // the data; every step runs in the kernels of this library.
 #include <algorithm>
 #include <atomic>
+#include <mutex>
 
 #include "moe_internal.cuh"
 
@@ -114,6 +115,28 @@ int layer_checks(const void* x, int T, const moe_layer* L, void* y, void* ws, si
     return check_ws(ws, ws_bytes, ws_layout(T, L->H, L->E, L->F, L->top_k).total);
 }
 
+// A non-blocking stream per device for the shared expert, with fork/join
+// events, created on first use.
+struct SideStream {
+    cudaStream_t s = nullptr;
+    cudaEvent_t fork = nullptr, join = nullptr;
+};
+int side_stream(SideStream** out) {
+    static std::mutex mu;
+    static SideStream per_dev[64];
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return MOE_ERR_CUDA;
+    std::lock_guard<std::mutex> lock(mu);
+    SideStream& st = per_dev[dev];
+    if (!st.s) {
+        if (cudaStreamCreateWithFlags(&st.s, cudaStreamNonBlocking) != cudaSuccess) return MOE_ERR_CUDA;
+        if (cudaEventCreateWithFlags(&st.fork, cudaEventDisableTiming) != cudaSuccess) return MOE_ERR_CUDA;
+        if (cudaEventCreateWithFlags(&st.join, cudaEventDisableTiming) != cudaSuccess) return MOE_ERR_CUDA;
+    }
+    *out = &st;
+    return MOE_OK;
+}
+
 int layer_run(const void* x, int T, const moe_layer* L, void* y, void* ws, cudaStream_t s) {
     const int H = L->H, E = L->E, F = L->F, k = L->top_k;
     const WsLayout W = ws_layout(T, H, E, F, k);
@@ -133,23 +156,49 @@ int layer_run(const void* x, int T, const moe_layer* L, void* y, void* ws, cudaS
     int32_t* sh_off = at<int32_t>(ws, W.sh_offsets);
     int32_t* sh_rs = at<int32_t>(ws, W.sh_rowslot);
     int32_t* counter = status + 1;
+    void* prep = at<void>(ws, W.prep);
+    __nv_bfloat16* h_sh = h_perm + size_t(R) * F;
+
+    // The shared expert needs x only: it runs on a side stream while the
+    // router, the bucketing and the routed experts run on `s`, and `s` waits
+    // for it before the combine.  Its own routing (offsets {0, T}, row i at
+    // slot i * top_k) comes first on that stream.
+    SideStream* side = nullptr;
+    if (has_sh) {
+        MOE_TRY(side_stream(&side));
+        if (cudaEventRecord(side->fork, s) != cudaSuccess || cudaStreamWaitEvent(side->s, side->fork, 0) != cudaSuccess)
+            return MOE_ERR_CUDA;
+        GemvProblem sg{};
+        sg.act = xb; sg.act_by_token = 1; sg.top_k = k; sg.offsets = sh_off; sg.row_slot = sh_rs;
+        sg.E = 1; sg.fmt = MOE_FMT_BF16; sg.out_dim = F; sg.in_dim = H;
+        sg.p0 = L->sh_gate.packed; sg.p1 = L->sh_up.packed; sg.out = h_sh; sg.status = status;
+        GemvProblem sd{};
+        sd.act = h_sh; sd.act_by_token = 0; sd.top_k = k; sd.offsets = sh_off; sd.row_slot = sh_rs;
+        sd.E = 1; sd.fmt = MOE_FMT_BF16; sd.out_dim = H; sd.in_dim = F;
+        sd.p0 = L->sh_down.packed; sd.out = ys; sd.status = status;
+        // the shared expert reads x and its own h directly (identity routing, natural order)
+        GemmBuffers direct{};
+        direct.act_ready = 1;
+        float* shpart = at<float>(ws, W.shpart);
+        MOE_TRY(launch_shared_routing(T, k, sh_off, sh_rs, side->s));
+        MOE_TRY(run_problem(sg, true, T, T, nullptr, direct, shpart, side->s));
+        MOE_TRY(run_problem(sd, false, T, T, nullptr, direct, shpart, side->s));
+        if (cudaEventRecord(side->join, side->s) != cudaSuccess) return MOE_ERR_CUDA;
+    }
+
     if (T <= kRouterDecodeMaxT && router_decode_ok(H)) {
-        // router, top-k, bucketing and shared routing in one launch
+        // router, top-k and bucketing in one launch
         RouterDecodeArgs ra{};
         ra.x = xb; ra.T = T; ra.H = H; ra.Wr = L->router_w; ra.bias = L->router_bias; ra.E = E; ra.k = k;
         ra.logits = at<float>(ws, W.logits); ra.ids = ids; ra.w = tw; ra.counter = counter; ra.status = status;
         ra.offsets = offsets; ra.row_slot = row_slot; ra.slot_row = slot_row;
-        ra.sh_offsets = has_sh ? sh_off : nullptr; ra.sh_rowslot = has_sh ? sh_rs : nullptr;
+        ra.sh_offsets = nullptr; ra.sh_rowslot = nullptr;
         MOE_TRY(launch_route_decode(ra, s));
     } else {
         MOE_TRY(launch_route(xb, T, H, L->router_w, L->router_bias, E, k, ids, tw, at<float>(ws, W.logits),
                              at<__nv_bfloat16>(ws, W.wsplit), status, counter, s));
         MOE_TRY(launch_permute(ids, T, k, E, offsets, row_slot, slot_row, at<int32_t>(ws, W.hist), status, s));
-        if (has_sh) MOE_TRY(launch_shared_routing(T, k, sh_off, sh_rs, s));
     }
-
-    void* prep = at<void>(ws, W.prep);
-    __nv_bfloat16* h_sh = h_perm + size_t(R) * F;
     const bool routed_gemm = gemm_shape_ok(H, F) && gemm_shape_ok(F, H);
     const bool int4 = L->gate.fmt == MOE_FMT_INT4_G128;
 
@@ -159,21 +208,11 @@ int layer_run(const void* x, int T, const moe_layer* L, void* y, void* ws, cudaS
     gu.p0 = L->gate.packed; gu.s0 = L->gate.scales; gu.g0 = L->gate.global_scale;
     gu.p1 = L->up.packed; gu.s1 = L->up.scales; gu.g1 = L->up.global_scale;
     gu.out = h_perm; gu.status = status;
-    GemvProblem sg{};
-    sg.act = xb; sg.act_by_token = 1; sg.top_k = k; sg.offsets = sh_off; sg.row_slot = sh_rs;
-    sg.E = 1; sg.fmt = MOE_FMT_BF16; sg.out_dim = F; sg.in_dim = H;
-    sg.p0 = L->sh_gate.packed; sg.p1 = L->sh_up.packed; sg.out = h_sh; sg.status = status;
-
     GemvProblem dn{};
     dn.act = h_perm; dn.act_by_token = 0; dn.top_k = k; dn.offsets = offsets; dn.row_slot = row_slot;
     dn.E = E; dn.topk_w = tw; dn.fmt = L->down.fmt; dn.out_dim = H; dn.in_dim = F;
     dn.p0 = L->down.packed; dn.s0 = L->down.scales; dn.g0 = L->down.global_scale;
     dn.out = y_perm; dn.status = status;
-    GemvProblem sd{};
-    sd.act = h_sh; sd.act_by_token = 0; sd.top_k = k; sd.offsets = sh_off; sd.row_slot = sh_rs;
-    sd.E = 1; sd.fmt = MOE_FMT_BF16; sd.out_dim = H; sd.in_dim = F;
-    sd.p0 = L->sh_down.packed; sd.out = ys; sd.status = status;
-
     // routed experts: both projections on one path (the int4 GEMM hands h to
     // the down GEMM in its pair order)
     const bool i8 = routed_gemm && i8_int4(gu, R);
@@ -187,11 +226,6 @@ int layer_run(const void* x, int T, const moe_layer* L, void* y, void* ws, cudaS
     } else {
         MOE_TRY(launch_stream_gemv(gu, nullptr, true, T, prep, s, true));
     }
-    // the shared expert reads x and its own h directly (identity routing, natural order)
-    GemmBuffers direct{};
-    direct.act_ready = 1;
-    float* shpart = at<float>(ws, W.shpart);
-    if (has_sh) MOE_TRY(run_problem(sg, true, T, T, nullptr, direct, shpart, s));
     if (routed_gemm) {
         // int4 h is already in the pair order unless the 8-bit path made it
         GemmBuffers db = gemm_buffers(prep, R, F, int4 && !i8, i8);
@@ -199,10 +233,12 @@ int layer_run(const void* x, int T, const moe_layer* L, void* y, void* ws, cudaS
     } else {
         MOE_TRY(launch_stream_gemv(dn, nullptr, false, R, prep, s, true));
     }
-    if (has_sh) MOE_TRY(run_problem(sd, false, T, T, nullptr, direct, shpart, s));
+    if (has_sh && cudaStreamWaitEvent(s, side->join, 0) != cudaSuccess) return MOE_ERR_CUDA;
 
+    // after a join with the side stream the combine starts only when both inputs are complete (no
+    // early launch of a dependent grid across an event wait)
     return launch_combine(y_perm, slot_row, T, k, H, has_sh ? ys : nullptr,
-                          reinterpret_cast<__nv_bfloat16*>(y), s);
+                          reinterpret_cast<__nv_bfloat16*>(y), s, !has_sh);
 }
 
 }  // namespace

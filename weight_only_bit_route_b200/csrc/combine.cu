@@ -41,11 +41,17 @@ __global__ void __launch_bounds__(256) combine_kernel(
 }
 
 int launch_combine(const __nv_bfloat16* y_perm, const int32_t* slot_row, int T, int k, int H,
-                   const __nv_bfloat16* shared_out, __nv_bfloat16* y, cudaStream_t s) {
+                   const __nv_bfloat16* shared_out, __nv_bfloat16* y, cudaStream_t s, bool pdl) {
     const long long n = (long long)T * (H / 8);
     const int blocks = int((n + 255) / 256);
-    if (launch_pdl(combine_kernel, dim3(blocks), dim3(256), 0, s, y_perm, slot_row, T, k, H, shared_out, y) != cudaSuccess)
-        return MOE_ERR_CUDA;
+    if (pdl) {
+        if (launch_pdl(combine_kernel, dim3(blocks), dim3(256), 0, s, y_perm, slot_row, T, k, H, shared_out, y) !=
+            cudaSuccess)
+            return MOE_ERR_CUDA;
+    } else {
+        combine_kernel<<<blocks, 256, 0, s>>>(y_perm, slot_row, T, k, H, shared_out, y);
+        count_launch();
+    }
     return cudaGetLastError() == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
 }
 

@@ -199,7 +199,7 @@ int launch_stream_gemv(const GemvProblem& routed, const GemvProblem* shared, boo
                        void* prep_ws, cudaStream_t s, bool pdl);
 
 int launch_combine(const __nv_bfloat16* y_perm, const int32_t* slot_row, int T, int k, int H,
-                   const __nv_bfloat16* shared_out, __nv_bfloat16* y, cudaStream_t s);
+                   const __nv_bfloat16* shared_out, __nv_bfloat16* y, cudaStream_t s, bool pdl = true);
 
 int launch_quant_int4(const __nv_bfloat16* w, int64_t rows, int64_t cols, int32_t* packed,
                       __nv_bfloat16* scales, cudaStream_t s);
