@@ -118,42 +118,48 @@ __global__ void __launch_bounds__(256) router_logits_tiled(
 // ---------------------------------------------------------------------------
 // Sigmoid + top-k + renormalisation for one token, by one warp.  PER is the
 // number of experts each lane holds (ceil(E / 32) rounded to a supported size).
+// Each expert is a 64-bit key: the score's bits (s >= 0, so they order like the
+// score) above the complement of its id (so equal scores prefer the lower id);
+// 0 marks an empty or taken slot.  A lane keeps the largest of its keys; a pick
+// is one warp-wide maximum, after which only the lane that owned the winner
+// rescans its keys.
 // ---------------------------------------------------------------------------
 template <int PER>
 __device__ __forceinline__ void topk_warp(const float* __restrict__ lrow, const float* __restrict__ bias, int E,
                                           int k, int32_t* __restrict__ ids, float* __restrict__ wout, int lane) {
-    float s[PER];
+    unsigned long long key[PER];
 #pragma unroll
     for (int i = 0; i < PER; i++) {
         const int e = lane + 32 * i;
-        float v = -INFINITY;
+        key[i] = 0ull;
         if (e < E) {
             float l = __ldcg(lrow + e);       // written by other CTAs of the fused router
             if (bias) l = l + bias[e];
-            v = 1.0f / (1.0f + expf(-l));
+            const float v = 1.0f / (1.0f + expf(-l));
+            key[i] = (static_cast<unsigned long long>(__float_as_uint(v)) << 32) | static_cast<uint32_t>(~e);
         }
-        s[i] = v;
     }
+    unsigned long long lmax = 0ull;
+#pragma unroll
+    for (int i = 0; i < PER; i++) lmax = key[i] > lmax ? key[i] : lmax;
     float sum = 0.f, my_s = 0.f;
     int my_id = 0;
     for (int j = 0; j < k; j++) {
-        // largest s, lowest id on ties (ids grow with i)
-        float bv = -INFINITY;
-        int bi = 0x7fffffff;
+        unsigned long long m = lmax;
 #pragma unroll
-        for (int i = 0; i < PER; i++) {
-            const int e = lane + 32 * i;
-            if (e < E && (s[i] > bv || (s[i] == bv && e < bi))) { bv = s[i]; bi = e; }
-        }
         for (int o = 16; o > 0; o >>= 1) {
-            const float ov = __shfl_xor_sync(0xffffffffu, bv, o);
-            const int oi = __shfl_xor_sync(0xffffffffu, bi, o);
-            if (ov > bv || (ov == bv && oi < bi)) { bv = ov; bi = oi; }
+            const unsigned long long om = __shfl_xor_sync(0xffffffffu, m, o);
+            m = om > m ? om : m;
         }
+        const int bi = static_cast<int>(~static_cast<uint32_t>(m));
+        const float bv = __uint_as_float(static_cast<uint32_t>(m >> 32));
         if ((bi & 31) == lane) {
+            lmax = 0ull;
 #pragma unroll
-            for (int i = 0; i < PER; i++)
-                if (lane + 32 * i == bi) s[i] = -INFINITY;
+            for (int i = 0; i < PER; i++) {
+                if (i == (bi >> 5)) key[i] = 0ull;
+                lmax = key[i] > lmax ? key[i] : lmax;
+            }
         }
         if (lane == j) { my_s = bv; my_id = bi; }
         sum = sum + bv;
@@ -266,8 +272,10 @@ __global__ void __launch_bounds__(RD_WARPS * 32) router_decode(RouterDecodeArgs 
     }
 #pragma unroll
     for (int t = 0; t < RD_TMAX; t++) {
-        const float v = warp_sum(acc[t], 32);
-        if (lane == 0 && t < a.T) s_part[el][kq][t] = v;
+        if (t < a.T) {                                       // uniform: only the tokens present
+            const float v = warp_sum(acc[t], 32);
+            if (lane == 0) s_part[el][kq][t] = v;
+        }
     }
     __syncthreads();
     // quarters in a fixed order
