@@ -609,14 +609,23 @@ __global__ void __launch_bounds__(G_THREADS, 1) tc_grouped_gemm(const __grid_con
                 g_fence_before();
                 __syncwarp();
                 if (lane == 0) g_arrive(g_smem(&acc_empty[bi]));
+                // the step's kGroups scales of this row are adjacent: one 4- or 8-byte load per matrix
+                const int grp0 = T.kbase / 128 + ks * C::kGroups;
+                using SV = typename std::conditional<C::kGroups == 4, uint2, uint32_t>::type;
+                const SV sv0 = *reinterpret_cast<const SV*>(sc0 + grp0);
+                SV sv1{};
+                if (GU) sv1 = *reinterpret_cast<const SV*>(sc1 + grp0);
+                const uint32_t* s0w = reinterpret_cast<const uint32_t*>(&sv0);
+                const uint32_t* s1w = reinterpret_cast<const uint32_t*>(&sv1);
 #pragma unroll
                 for (int gi = 0; gi < C::kGroups; gi++) {
-                    const int grp = T.kbase / 128 + ks * C::kGroups + gi;
-                    const float s0 = __bfloat162float(sc0[grp]);
-                    const float s1 = GU ? __bfloat162float(sc1[grp]) : 0.f;
+                    const int grp = grp0 + gi;
+                    const float s0 = __uint_as_float((s0w[gi >> 1] >> (16 * (gi & 1))) << 16);
+                    const float s1 = GU ? __uint_as_float((s1w[gi >> 1] >> (16 * (gi & 1))) << 16) : 0.f;
 #pragma unroll
                     for (int j = 0; j < C::kNMax; j++) {
-                        const float zj = j < T.nval ? zs[j * zst + grp] : 0.f;
+                        if (j >= T.nval) break;                  // uniform: the tokens of this tile only
+                        const float zj = zs[j * zst + grp];
                         const float vg = fmaf(float(int(g[gi][3 * j])), 65536.f,
                                               fmaf(float(int(g[gi][3 * j + 1])), 256.f, float(int(g[gi][3 * j + 2])))) - zj;
                         tg[j] = fmaf(s0, vg, tg[j]);
