@@ -341,7 +341,7 @@ def main():
     pk, pk_kind = peaks()
     # DRAM bytes (read + write) of one gate/up tcgen05_grouped_gemm launch, from the ncu captures summarised
     # under profiles/ for the current kernel; workloads without a capture report null
-    traffic = {"decode_int4_T8": 395251456, "prefill_int4_T2048": 2484627008}.get(wl.name)
+    traffic = {"decode_int4_T8": 395251456, "prefill_int4_T2048": 2472866648}.get(wl.name)
     decode = T <= 64
     if decode:
         kbytes = touched * gateup_bytes_per_expert(wl) + T * wl.H * 2

@@ -690,7 +690,7 @@ __global__ void __launch_bounds__(G_THREADS, 1) tc_grouped_gemm(const __grid_con
                 g_ld16(acc0 + c, g);
                 if (GU) g_ld16(acc0 + C::kUpCol + c, u);
                 g_ld_wait();
-                if (ksplit > 1) {
+                if (FMT == MOE_FMT_BF16 && ksplit > 1) {
                     // split-K: raw fp32 sums of this K slice; the tile's last slice (or a kernel) finishes the rows
 #pragma unroll
                     for (int j = 0; j < 16; j++) {
@@ -722,7 +722,7 @@ __global__ void __launch_bounds__(G_THREADS, 1) tc_grouped_gemm(const __grid_con
             g_fence_before();
             __syncwarp();
             if (lane == 0) g_arrive(g_smem(&acc_empty[buf]));
-            if (ksplit > 1 && a.tile_cnt) {
+            if (FMT == MOE_FMT_BF16 && ksplit > 1 && a.tile_cnt) {
                 // Per (tile, quarter of its rows): the epilogue warp that writes the last K slice of
                 // its 32 rows sums all slices in slice order and writes the bf16 rows (E = 1: no
                 // routing weight on gate/up, the slot weight on down).  Warps count separately, so
