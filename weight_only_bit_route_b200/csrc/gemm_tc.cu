@@ -788,15 +788,22 @@ __global__ void __launch_bounds__(G_THREADS, 1) tc_grouped_gemm(const __grid_con
                 if (!g_wait_w(g_smem(&pk_full[s]), (pc / NPK) & 1, &s_abort)) { ok = false; break; }
                 const uint8_t* st = pk + s * C::kPkStageBytes;
                 uint32_t o[kNBuf][16];
-                auto unpack = [&](auto uc) {
+                uint4 raw[2][2];                                // packed chunks, loaded one piece ahead
+                auto load = [&](auto uc) {
                     // piece u: matrix m, 16-byte chunks c0 and c0 + 1 of the row, in TMA box c0 / 8
                     constexpr int u = decltype(uc)::value, m = u / kPpm, c0 = 2 * (u % kPpm);
                     const uint8_t* wt = st + m * C::kMatBytes + (c0 / 8) * (G_BM * 128);
-                    const uint4 w0 = *reinterpret_cast<const uint4*>(wt + g_swz(r, c0 % 8));
-                    const uint4 w1 = *reinterpret_cast<const uint4*>(wt + g_swz(r, c0 % 8 + 1));
-                    g_dq_int4_i8<0>(w0, o[u % kNBuf]);
-                    g_dq_int4_i8<8>(w1, o[u % kNBuf]);
+                    raw[u & 1][0] = *reinterpret_cast<const uint4*>(wt + g_swz(r, c0 % 8));
+                    raw[u & 1][1] = *reinterpret_cast<const uint4*>(wt + g_swz(r, c0 % 8 + 1));
                 };
+                auto unpack = [&](auto uc) {
+                    constexpr int u = decltype(uc)::value;
+                    g_dq_int4_i8<0>(raw[u & 1][0], o[u % kNBuf]);
+                    g_dq_int4_i8<8>(raw[u & 1][1], o[u % kNBuf]);
+                    if constexpr (u + 2 < kPieces) load(std::integral_constant<int, u + 2>{});
+                };
+                load(std::integral_constant<int, 0>{});
+                if constexpr (kPieces > 1) load(std::integral_constant<int, 1>{});
                 unpack(std::integral_constant<int, 0>{});
                 const int sa = pc % C::kAStages;
                 if (pc >= uint32_t(C::kAStages) && !g_wait_w(g_smem(&done[(pc - C::kAStages) % G_DONE]),
