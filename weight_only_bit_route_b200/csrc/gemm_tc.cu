@@ -33,7 +33,8 @@
 //               (8-bit int4: warps 2 and 3 take alternate steps).
 // The three single-issue roles run warp-uniform loops and elect one lane to
 // issue, which keeps the instruction operands in uniform registers.  The MMA
-// pipeline steps in K = 128 and commits once per step, to one barrier of a
+// pipeline steps in K = 128 (8-bit path: K = 256 for gate/up, 512 for down)
+// and commits once per step, to one barrier of a
 // ring of 16 ("stage done"): a tcgen05.commit costs as much issue time as
 // several MMAs, so every role that waits for a step to finish (the activation
 // producer, the dequantisation warps, the BF16 weight producer, the small-
@@ -47,7 +48,9 @@
 //               (int4: q*s rounded once) or f16 pairs (NVFP4: e2m1 * e4m3,
 //               exact) in registers and writes them to tensor memory with
 //               tcgen05.st; the MMA reads its A operand from there.  The
-//               dequantised weights never pass through shared memory.
+//               dequantised weights never pass through shared memory.  On
+//               the 8-bit path the warps only unpack nibbles into bytes, in
+//               two groups of four that take alternate weight stages.
 // BF16 weights (the shared expert) need no dequantisation: the MMA reads the
 // TMA-staged weight tile from shared memory directly.
 //
