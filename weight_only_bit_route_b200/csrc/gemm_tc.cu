@@ -584,12 +584,9 @@ __global__ void __launch_bounds__(G_THREADS, 1) tc_grouped_gemm(const __grid_con
             const int rbase = T.ebase + T.n0;
             const bool live = lane < T.nval;
             const int b = t % NSC;
-            // the row factors are needed after the last step: issue their loads now
-            float rowf = 1.f;
-            if (live) {
-                rowf = a.act_scale[rbase + lane];
-                if (!GU && a.topk_w) rowf *= a.topk_w[a.row_slot[rbase + lane]];
-            }
+            // the row factor (2^-c, times the routing weight on down, folded by the pre-pass)
+            // is needed after the last step: issue its load now
+            const float rowf = live ? a.act_scale[rbase + lane] : 1.f;
             if (!g_wait(g_smem(&sc_full[b]), (t / NSC) & 1, &s_abort, 64)) { ok = false; break; }
             const __nv_bfloat16* sc0 = reinterpret_cast<const __nv_bfloat16*>(scbuf + b * sc_buf_bytes) + r * ngroups;
             const __nv_bfloat16* sc1 = sc0 + G_BM * ngroups;
@@ -675,7 +672,8 @@ __global__ void __launch_bounds__(G_THREADS, 1) tc_grouped_gemm(const __grid_con
                 const int nn = c + (lane & 15);
                 if (nn < T.nval) {
                     if (FMT == MOE_FMT_NVFP4) v = a.act_scale[rbase + nn];
-                    if (!GU && a.topk_w) v *= a.topk_w[a.row_slot[rbase + nn]];
+                    // NVFP4: the pre-pass folded the routing weight into the row scale
+                    if (!GU && a.topk_w && FMT != MOE_FMT_NVFP4) v *= a.topk_w[a.row_slot[rbase + nn]];
                 }
                 return v;
             };
@@ -935,8 +933,8 @@ __global__ void __launch_bounds__(G_THREADS, 1) tc_grouped_gemm(const __grid_con
 // ---------------------------------------------------------------------------
 __global__ void __launch_bounds__(256) g_prep(const __nv_bfloat16* __restrict__ src, int in_dim,
                                               const int32_t* __restrict__ row_slot, int top_k, int by_token,
-                                              int rows, int mode, uint16_t* __restrict__ dst,
-                                              float* __restrict__ scale) {
+                                              int rows, int mode, const float* __restrict__ row_w,
+                                              uint16_t* __restrict__ dst, float* __restrict__ scale) {
     asm volatile("griddepcontrol.wait;" ::: "memory");
     const int row = (blockIdx.x * blockDim.x + threadIdx.x) >> 5, lane = threadIdx.x & 31;
     if (row >= rows) return;
@@ -976,7 +974,8 @@ __global__ void __launch_bounds__(256) g_prep(const __nv_bfloat16* __restrict__ 
             h[3] = __floats2half2_rn(bf16_lo(v.w) * down, bf16_hi(v.w) * down);
             d[i] = *reinterpret_cast<uint4*>(h);
         }
-        if (lane == 0) scale[row] = ldexpf(1.f, e);
+        // mode 2 row scale, times the down projection's routing weight when given (exact: 2^e * w)
+        if (lane == 0) scale[row] = row_w ? ldexpf(1.f, e) * row_w[row_slot[row]] : ldexpf(1.f, e);
     }
 }
 
@@ -985,13 +984,16 @@ __global__ void __launch_bounds__(256) g_prep(const __nv_bfloat16* __restrict__ 
 // [2^21, 2^22), written as signed digits X = 65536 d2 + 256 d1 + d0 in int8
 // rows 3 row (d2), 3 row + 1 (d1), 3 row + 2 (d0) of dst, in the K order
 // 0, 2, 4, 6, 1, 3, 5, 7 of every 8 (the order of the unpacked weight bytes);
-// scale[row] = 2^-c; zsum[row][g] (row stride zst) = 8 * sum of X over group
-// g, the u - 8 offset of the weights.
+// scale[row] = 2^-c, times row_w[row_slot[row]] when row_w is given (the
+// down projection's routing weight; a power of two times w is exact);
+// zsum[row][g] (row stride zst) = 8 * sum of X over group g, the u - 8 offset
+// of the weights.
 constexpr int G_PREP_I8_THREADS = 128;
 __global__ void __launch_bounds__(G_PREP_I8_THREADS) g_prep_i8(const __nv_bfloat16* __restrict__ src, int in_dim,
                                                                const int32_t* __restrict__ row_slot, int top_k,
-                                                               int by_token, uint8_t* __restrict__ dst,
-                                                               float* __restrict__ scale, float* __restrict__ zsum) {
+                                                               int by_token, const float* __restrict__ row_w,
+                                                               uint8_t* __restrict__ dst, float* __restrict__ scale,
+                                                               float* __restrict__ zsum) {
     __shared__ float s_max[G_PREP_I8_THREADS / 32];
     asm volatile("griddepcontrol.wait;" ::: "memory");
     const int row = blockIdx.x, tid = threadIdx.x, lane = tid & 31;
@@ -1041,7 +1043,7 @@ __global__ void __launch_bounds__(G_PREP_I8_THREADS) g_prep_i8(const __nv_bfloat
         for (int o = 8; o > 0; o >>= 1) zs += __shfl_xor_sync(0xffffffffu, zs, o);
         if ((lane & 15) == 0 && i < n16) zsum[size_t(row) * zst + i / 16] = 8.f * float(zs);
     }
-    if (tid == 0) scale[row] = 1.f / fc;
+    if (tid == 0) scale[row] = row_w ? (1.f / fc) * row_w[row_slot[row]] : 1.f / fc;
 }
 
 // ---------------------------------------------------------------------------
@@ -1157,14 +1159,17 @@ int launch_grouped_gemm(const GemvProblem& p, bool gateup, int rows, const GemmB
     if (!buf.act_ready || nv || i8) {
         if (!buf.act_buf || (nv && !buf.scale_buf)) return MOE_ERR_WORKSPACE;
         if (i8) {
+            const float* row_w = gateup ? nullptr : p.topk_w;
             if (launch_pdl(g_prep_i8, dim3(rows), dim3(G_PREP_I8_THREADS), 0, s, p.act, in, p.row_slot, p.top_k,
-                           p.act_by_token, reinterpret_cast<uint8_t*>(buf.act_buf), buf.scale_buf, buf.zbuf) != cudaSuccess)
+                           p.act_by_token, row_w, reinterpret_cast<uint8_t*>(buf.act_buf), buf.scale_buf,
+                           buf.zbuf) != cudaSuccess)
                 return MOE_ERR_CUDA;
         } else {
             const int mode = nv ? 2 : (i4 ? 1 : 0);
+            const float* row_w = (nv && !gateup) ? p.topk_w : nullptr;     // folded into the NVFP4 row scale
             if (launch_pdl(g_prep, dim3((rows * 32 + 255) / 256), dim3(256), 0, s, p.act, in, p.row_slot, p.top_k,
-                           p.act_by_token, rows, mode, reinterpret_cast<uint16_t*>(buf.act_buf), buf.scale_buf) !=
-                cudaSuccess)
+                           p.act_by_token, rows, mode, row_w, reinterpret_cast<uint16_t*>(buf.act_buf),
+                           buf.scale_buf) != cudaSuccess)
                 return MOE_ERR_CUDA;
         }
         bsrc = buf.act_buf;
