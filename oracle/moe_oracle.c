@@ -551,7 +551,9 @@ void oracle_grouped_down(const uint16_t* h_in, int64_t F, int64_t H,
 }
 
 /* Combine: y[t] = shared[t] + sum_j y_perm[slot_row[t*k + j]] (fp64).
- * y_perm: bf16 bits [T*k, H]; shared: bf16 bits [T, H] or NULL. */
+ * y_perm: bf16 bits [T*k, H]; shared: bf16 bits [T, H] or NULL.
+ * A slot whose row is negative was dropped by the bucketing (its expert id
+ * was out of range) and contributes nothing. */
 void oracle_combine(const uint16_t* y_perm, const int32_t* slot_row, int64_t T, int k,
                     int64_t H, const uint16_t* shared, double* y) {
     for (int64_t t = 0; t < T; t++)
@@ -559,6 +561,7 @@ void oracle_combine(const uint16_t* y_perm, const int32_t* slot_row, int64_t T, 
             double acc = shared ? (double)oracle_bf16_to_f32(shared[t * H + hh]) : 0.0;
             for (int j = 0; j < k; j++) {
                 int32_t r = slot_row[t * k + j];
+                if (r < 0) continue;
                 acc += (double)oracle_bf16_to_f32(y_perm[(int64_t)r * H + hh]);
             }
             y[t * H + hh] = acc;
