@@ -4,14 +4,19 @@ One step = one pass of the whole layer (router, bucketing, grouped gate/up +
 SwiGLU, grouped down with routing weights, BF16 shared expert, combine) over
 one batch of synthetic tokens, through the library's C ABI.
 
-    python bench.py [--gpus N] [--steps K] [--warmup W] [--config C] [--impl reference]
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--config C] [--per-config 2,3,4]
+                    [--impl reference]
 
-Default workload: decode-shaped layer, int4 g128 W4A16, T = 8 tokens, hidden
-4096, 352 experts of width 1536, top-8, BF16 shared expert.  Weights are bf16
-N(0, 0.02^2) drawn on the GPU and converted by the library's quantiser;
-activations bf16 N(0, 1); router fp32 N(0, 1/4096).  L2 is flushed (256 MB
-write) before every timed step; each step is timed with CUDA events on the
-launching stream and the flush is outside the events.
+Headline workload (the line's value): decode-shaped layer, int4 g128 W4A16,
+T = 8 tokens, hidden 4096, 352 experts of width 1536, top-8, BF16 shared
+expert.  The other workloads (NVFP4 decode, int4 prefill T = 2048, NVFP4
+prefill T = 8192 with Zipf-skewed routing) go into `per_config` on the same
+line, each with its layer time (mean, median, p10, p90), its dominant-kernel
+roofline, its whole-layer roofline and the time of each step through its own
+C-ABI call.  Weights are bf16 N(0, 0.02^2) drawn on the GPU and converted by
+the library's quantisers; activations bf16 N(0, 1); router fp32 N(0, 1/4096).
+L2 is flushed (256 MB write) before every timed call; each call is timed with
+CUDA events on the launching stream and the flush is outside the events.
 
 Under torchrun every rank runs an independent replica on its own GPU (the
 layer has no cross-GPU exchange on this path); the step time is the maximum
@@ -131,30 +136,39 @@ def build_layer(moe, wl, seed=0, device="cuda"):
 # ---------------------------------------------------------------------------
 
 class ClockSampler:
-    """Samples SM clock, power and clock-event reasons through NVML in a
-    background thread while the timed region runs (read-only queries)."""
+    """Samples SM clock and clock-event reasons through NVML (read-only
+    queries): a background thread every `period_s` while the sampler is open,
+    plus a synchronous sample whenever mark() is called (before and after
+    every timed loop), so that short timed regions still get samples."""
 
     REASONS = {"hw_slowdown": 0x8, "sw_thermal_slowdown": 0x20, "hw_thermal_slowdown": 0x40,
                "sw_power_cap": 0x4}
 
-    def __init__(self, gpu_index, period_s=0.01):
+    def __init__(self, gpu_index, period_s=0.005):
         self.gpu, self.period = gpu_index, period_s
         self.samples, self.reasons, self.max_mhz = [], set(), None
+        self.handle = None
+        self.error = None
+
+    def _sample(self):
+        import pynvml
+        self.samples.append(float(pynvml.nvmlDeviceGetClockInfo(self.handle, pynvml.NVML_CLOCK_SM)))
+        try:
+            r = pynvml.nvmlDeviceGetCurrentClocksEventReasons(self.handle)
+        except Exception:
+            r = pynvml.nvmlDeviceGetCurrentClocksThrottleReasons(self.handle)
+        for name, bit in self.REASONS.items():
+            if r & bit:
+                self.reasons.add(name)
 
     def _run(self):
-        import pynvml
-        h = pynvml.nvmlDeviceGetHandleByIndex(self.gpu)
-        self.max_mhz = float(pynvml.nvmlDeviceGetMaxClockInfo(h, pynvml.NVML_CLOCK_SM))
         while not self.stop.is_set():
-            self.samples.append(float(pynvml.nvmlDeviceGetClockInfo(h, pynvml.NVML_CLOCK_SM)))
-            try:
-                r = pynvml.nvmlDeviceGetCurrentClocksEventReasons(h)
-            except Exception:
-                r = pynvml.nvmlDeviceGetCurrentClocksThrottleReasons(h)
-            for name, bit in self.REASONS.items():
-                if r & bit:
-                    self.reasons.add(name)
+            self._sample()
             self.stop.wait(self.period)
+
+    def mark(self):
+        if self.handle is not None:
+            self._sample()
 
     def __enter__(self):
         import threading
@@ -163,13 +177,17 @@ class ClockSampler:
         try:
             import pynvml
             pynvml.nvmlInit()
+            gpu = self.gpu
             vis = os.environ.get("CUDA_VISIBLE_DEVICES")
             if vis:
-                self.gpu = int(vis.split(",")[self.gpu])
+                gpu = int(vis.split(",")[self.gpu])
+            self.handle = pynvml.nvmlDeviceGetHandleByIndex(gpu)
+            self.max_mhz = float(pynvml.nvmlDeviceGetMaxClockInfo(self.handle, pynvml.NVML_CLOCK_SM))
             self.thread = threading.Thread(target=self._run, daemon=True)
             self.thread.start()
         except Exception as e:   # no NVML: report no samples
             self.error = str(e)
+            self.handle = None
         return self
 
     def __exit__(self, *a):
@@ -179,7 +197,8 @@ class ClockSampler:
 
     def summary(self):
         if not self.samples:
-            return {"sm_mhz": None, "sm_max_mhz": self.max_mhz, "reasons": [], "samples": 0}
+            return {"sm_mhz": None, "sm_max_mhz": self.max_mhz, "reasons": [], "samples": 0,
+                    "error": self.error}
         return {"sm_mhz": float(np.median(self.samples)), "sm_max_mhz": self.max_mhz,
                 "reasons": sorted(self.reasons), "samples": len(self.samples)}
 
@@ -248,15 +267,153 @@ def cpu_baseline(wl, moe, x, layer, budget_s=20.0):
 
 
 # ---------------------------------------------------------------------------
-# main
+# measurement
 # ---------------------------------------------------------------------------
+
+# DRAM bytes (read + write) per launch of the dominant kernel, from one-pass ncu
+# captures of that kernel (summarised under profiles/), keyed by workload and by
+# a hash of the GEMM's sources at the time of the capture: a figure whose
+# kernel has changed since is reported as null.
+TRAFFIC = {}
+
+
+def gemm_source_hash():
+    import hashlib
+    h = hashlib.sha256()
+    for f in ("gemm_tc.cu", "tc_ptx.cuh", "moe_internal.cuh"):
+        h.update(open(os.path.join(ROOT, "weight_only_bit_route_b200", "csrc", f), "rb").read())
+    return h.hexdigest()[:16]
+
+
+def _pcts(ms):
+    a = np.asarray(ms, np.float64)
+    return {"mean": round(float(a.mean()), 5), "median": round(float(np.median(a)), 5),
+            "p10": round(float(np.percentile(a, 10)), 5), "p90": round(float(np.percentile(a, 90)), 5)}
+
+
+def time_calls(fn, steps, flush, stream, clk, warmup=3):
+    """CUDA-event times (ms) of `steps` calls of fn on `stream`, L2 flushed
+    before each call outside the events."""
+    for _ in range(warmup):
+        flush.zero_()
+        fn()
+    torch.cuda.synchronize()
+    evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(steps)]
+    clk.mark()
+    for i in range(steps):
+        flush.zero_()
+        evs[i][0].record(stream)
+        fn()
+        evs[i][1].record(stream)
+    torch.cuda.synchronize()
+    clk.mark()
+    return [a.elapsed_time(b) for a, b in evs]
+
+
+def step_times(moe, wl, x, layer, ws, steps, flush, stream, clk):
+    """Median time of each step through its own C-ABI call (a1..a6)."""
+    T, k = x.shape[0], wl.k
+    R = T * k
+    ids, tw = moe.route_topk(x, layer.router_w, layer.router_bias, k, ws)
+    off, rs, sr = moe.permute(ids, wl.E, ws)
+    h = torch.empty(R, wl.F, dtype=torch.bfloat16, device="cuda")
+    yp = torch.empty(R, wl.H, dtype=torch.bfloat16, device="cuda")
+    y = torch.empty_like(x)
+    out = {}
+    med = lambda v: round(float(np.median(v)), 5)
+    out["a1_router"] = med(time_calls(lambda: moe.route_topk(x, layer.router_w, layer.router_bias, k, ws),
+                                      steps, flush, stream, clk))
+    out["a2_bucketing"] = med(time_calls(lambda: moe.permute(ids, wl.E, ws), steps, flush, stream, clk))
+    out["a3_gateup_swiglu"] = med(time_calls(
+        lambda: moe.grouped_swiglu(x, off, rs, k, layer.gate, layer.up, R, ws, out=h), steps, flush, stream, clk))
+    out["a4_down"] = med(time_calls(lambda: moe.grouped_down(h, off, rs, tw.view(-1), layer.down, ws, out=yp),
+                                    steps, flush, stream, clk))
+    ys = None
+    if layer.shared:
+        so = torch.tensor([0, T], dtype=torch.int32, device="cuda")
+        srs = torch.arange(T, dtype=torch.int32, device="cuda") * k
+        hs = torch.empty(T, wl.F, dtype=torch.bfloat16, device="cuda")
+        ys = torch.empty_like(x)
+
+        def shared():
+            moe.grouped_swiglu(x, so, srs, k, layer.shared[0], layer.shared[1], T, ws, out=hs)
+            moe.grouped_down(hs, so, srs, None, layer.shared[2], ws, out=ys)
+        out["a5_shared_expert"] = med(time_calls(shared, steps, flush, stream, clk))
+    out["a6_combine"] = med(time_calls(lambda: moe.unpermute_combine(yp, sr, T, k, ys, out=y),
+                                       steps, flush, stream, clk))
+    return out
+
+
+def measure(moe, wl, x, layer, args, flush, stream, clk, pk, pk_kind, per_step=True):
+    """Layer timing (+ dominant-kernel roofline and per-step times) of one workload."""
+    T = wl.T
+    ws = moe.workspace(T, wl.H, wl.E, wl.F, wl.k)
+    y = torch.empty_like(x)
+    entry = moe.layer_decode if T <= 64 else moe.layer_forward
+    step = lambda: entry(x, layer, ws, out=y)
+    for _ in range(max(3, args.warmup)):
+        flush.zero_()
+        step()
+    torch.cuda.synchronize()
+    status = moe.read_status(ws)
+    if status != 0:
+        raise RuntimeError(f"device status {status} after warm-up")
+    ids, _ = moe.route_topk(x, layer.router_w, layer.router_bias, wl.k, ws)
+    touched = int(torch.unique(ids).numel())
+    torch.cuda.synchronize()
+    launches0 = moe.launch_count()
+    ms_list = time_calls(step, args.steps, flush, stream, clk, warmup=0)
+    launches = moe.launch_count() - launches0
+    # dominant kernel: grouped gate/up (+ SwiGLU) through its own C-ABI call
+    off, rs, sr = moe.permute(ids, wl.E, ws)
+    R = T * wl.k
+    h = torch.empty(R, wl.F, dtype=torch.bfloat16, device="cuda")
+    k_ms = float(np.mean(time_calls(lambda: moe.grouped_swiglu(x, off, rs, wl.k, layer.gate, layer.up, R, ws, out=h),
+                                    args.steps, flush, stream, clk)))
+    if moe.read_status(ws) != 0:
+        raise RuntimeError("device status set during timing")
+    ms = float(np.mean(ms_list))
+    decode = T <= 64
+    traffic = TRAFFIC.get((wl.name, gemm_source_hash()))
+    lbytes, lflops = layer_bytes(wl, touched), layer_flops(wl)
+    kernel_name = "tc_grouped_gemm gate/up+SwiGLU (with its activation pre-pass)"
+    if decode:
+        kbytes = touched * gateup_bytes_per_expert(wl) + T * wl.H * 2
+        achieved = kbytes / (k_ms * 1e-3) / 1e9
+        roof = {"bound": "hbm", "achieved": round(achieved, 1), "peak": pk["hbm_gbs"], "unit": "GB/s",
+                "frac": round(achieved / pk["hbm_gbs"], 4), "traffic": traffic, "kernel": kernel_name,
+                "algorithmic_bytes": kbytes, "kernel_ms": round(k_ms, 5), "peak_source": f"{pk_kind} hbm_gbs"}
+        layer_roof = {"bound": "hbm", "algorithmic_bytes": lbytes,
+                      "achieved_gbs": round(lbytes / (ms * 1e-3) / 1e9, 1),
+                      "frac": round(lbytes / (ms * 1e-3) / 1e9 / pk["hbm_gbs"], 4)}
+    else:
+        kflops = 2 * 2 * wl.F * wl.H * R
+        achieved = kflops / (k_ms * 1e-3) / 1e12
+        roof = {"bound": "tensor", "achieved": round(achieved, 1), "peak": pk["bf16_tflops"], "unit": "TFLOP/s",
+                "frac": round(achieved / pk["bf16_tflops"], 4), "traffic": traffic, "kernel": kernel_name,
+                "algorithmic_flops": kflops, "kernel_ms": round(k_ms, 5), "peak_source": f"{pk_kind} bf16_tflops"}
+        tf = lflops / (ms * 1e-3) / 1e12
+        layer_roof = {"bound": "tensor", "algorithmic_flops": lflops, "achieved_tflops": round(tf, 1),
+                      "frac_burst": round(tf / pk["bf16_tflops"], 4),
+                      "frac_sustained": round(tf / pk.get("bf16_tflops_sustained", pk["bf16_tflops"]), 4),
+                      "algorithmic_bytes": lbytes,
+                      "hbm_frac": round(lbytes / (ms * 1e-3) / 1e9 / pk["hbm_gbs"], 4)}
+    res = {"workload": describe(wl), "T": T, "format": wl.fmt, "touched_experts": touched,
+           "tokens_per_s": round(T / (ms * 1e-3), 1), "layer_ms": _pcts(ms_list),
+           "roofline": roof, "layer_roofline": layer_roof, "gpu_launches_per_step": launches / args.steps}
+    if per_step:
+        res["steps_ms"] = step_times(moe, wl, x, layer, ws, args.steps, flush, stream, clk)
+    return res, ms, ms_list, touched, launches, ws, entry
+
 
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
     ap.add_argument("--steps", type=int, default=200)
     ap.add_argument("--warmup", type=int, default=10)
-    ap.add_argument("--config", type=int, default=1)
+    ap.add_argument("--config", type=int, default=1, help="the headline workload")
+    ap.add_argument("--per-config", default="2,3,4",
+                    help="other workloads measured into per_config (comma list, or 'none')")
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
     args = ap.parse_args()
@@ -265,6 +422,8 @@ def main():
     world = int(os.environ.get("WORLD_SIZE", "1"))
     local_rank = int(os.environ.get("LOCAL_RANK", "0"))
     wl = syn.WORKLOADS[args.config]
+    others = [] if args.per_config == "none" else [int(c) for c in args.per_config.split(",") if c.strip()]
+    others = [c for c in others if c != args.config]
 
     if args.impl == "reference":
         run_reference(args, wl, rank, world)
@@ -278,108 +437,61 @@ def main():
         dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
     from weight_only_bit_route_b200 import moe
 
-    x, layer = build_layer(moe, wl)
-    T = wl.T
-    ws = moe.workspace(T, wl.H, wl.E, wl.F, wl.k)
-    y = torch.empty_like(x)
-    entry = moe.layer_decode if T <= 64 else moe.layer_forward
+    # weights: one int4 and one NVFP4 bank set (the workloads of a format share their weights)
+    layers = {}
+
+    def layer_for(w):
+        if w.fmt not in layers:
+            layers[w.fmt] = build_layer(moe, w)[1]
+        lay = layers[w.fmt]
+        b = syn.gen_bias(w)
+        lay.router_bias = None if b is None else torch.from_numpy(b).cuda()
+        return lay
+
+    def x_for(w):
+        return torch.from_numpy(syn.gen_x(w).view(np.int16)).cuda().view(torch.bfloat16)
+
     flush = torch.empty(256 * 1024 * 1024, dtype=torch.uint8, device="cuda")
     stream = torch.cuda.current_stream()
-
-    def step():
-        entry(x, layer, ws, out=y)
-
-    for _ in range(max(3, args.warmup)):
-        flush.zero_()
-        step()
-    torch.cuda.synchronize()
-    status = moe.read_status(ws)
-    if status != 0:
-        raise RuntimeError(f"device status {status} after warm-up")
-
-    # routing facts for the algorithmic byte count
-    ids, _ = moe.route_topk(x, layer.router_w, layer.router_bias, wl.k, ws)
-    touched = int(torch.unique(ids).numel())
-
-    evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(args.steps)]
-    if dist:
-        dist.barrier()
-    torch.cuda.synchronize()
-    launches0 = moe.launch_count()
-    with ClockSampler(local_rank) as clk:
-        for i in range(args.steps):
-            flush.zero_()
-            evs[i][0].record(stream)
-            step()
-            evs[i][1].record(stream)
-        torch.cuda.synchronize()
-    launches = moe.launch_count() - launches0      # the library's own kernels in the timed region
-    if dist:
-        dist.barrier()
-    step_ms = [a.elapsed_time(b) for a, b in evs]
-    ms = float(np.mean(step_ms))
-    if dist:
-        t = torch.tensor([ms], device="cuda")
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        ms = float(t.item())
-    value = world * T / (ms * 1e-3)
-
-    # dominant kernel: grouped gate/up (+SwiGLU) through its own C-ABI call
-    off, rs, sr = moe.permute(ids, wl.E, ws)
-    R = T * wl.k
-    h = torch.empty(R, wl.F, dtype=torch.bfloat16, device="cuda")
-    for _ in range(3):
-        moe.grouped_swiglu(x, off, rs, wl.k, layer.gate, layer.up, R, ws, out=h)
-    kev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(args.steps)]
-    for i in range(args.steps):
-        flush.zero_()
-        kev[i][0].record(stream)
-        moe.grouped_swiglu(x, off, rs, wl.k, layer.gate, layer.up, R, ws, out=h)
-        kev[i][1].record(stream)
-    torch.cuda.synchronize()
-    k_ms = float(np.mean([a.elapsed_time(b) for a, b in kev]))
     pk, pk_kind = peaks()
-    # DRAM bytes (read + write) of one gate/up tcgen05_grouped_gemm launch, from the ncu captures summarised
-    # under profiles/ for the current kernel; workloads without a capture report null
-    traffic = {"decode_int4_T8": 395251456, "prefill_int4_T2048": 2472866648}.get(wl.name)
-    decode = T <= 64
-    if decode:
-        kbytes = touched * gateup_bytes_per_expert(wl) + T * wl.H * 2
-        achieved = kbytes / (k_ms * 1e-3) / 1e9
-        roof = {"bound": "hbm", "achieved": round(achieved, 1), "peak": pk["hbm_gbs"], "unit": "GB/s",
-                "frac": round(achieved / pk["hbm_gbs"], 4), "traffic": traffic,
-                "kernel": "tc_grouped_gemm gate/up+SwiGLU (with its activation gather)", "algorithmic_bytes": kbytes,
-                "kernel_ms": round(k_ms, 5), "peak_source": f"{pk_kind} hbm_gbs"}
-    else:
-        kflops = 2 * 2 * wl.F * wl.H * R
-        achieved = kflops / (k_ms * 1e-3) / 1e12
-        peak = pk["bf16_tflops"]
-        roof = {"bound": "tensor", "achieved": round(achieved, 1), "peak": peak, "unit": "TFLOP/s",
-                "frac": round(achieved / peak, 4), "traffic": traffic,
-                "kernel": "tc_grouped_gemm gate/up+SwiGLU (with its activation gather)",
-                "algorithmic_flops": kflops, "kernel_ms": round(k_ms, 5), "peak_source": f"{pk_kind} bf16_tflops"}
-
-    # end to end through the public API with host buffers
-    xh = x.cpu().pin_memory()
-    yh = torch.empty_like(xh).pin_memory()
-    xd = torch.empty_like(x)
-    eev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(args.steps)]
-    for i in range(args.steps + 3):
-        flush.zero_()
-        j = i - 3
-        if j >= 0:
-            eev[j][0].record(stream)
-        xd.copy_(xh, non_blocking=True)
-        entry(xd, layer, ws, out=y)
-        yh.copy_(y, non_blocking=True)
-        if j >= 0:
-            eev[j][1].record(stream)
-    torch.cuda.synchronize()
-    e_ms = float(np.mean([a.elapsed_time(b) for a, b in eev]))
+    T = wl.T
+    x = x_for(wl)
+    layer = layer_for(wl)
     if dist:
-        t = torch.tensor([e_ms], device="cuda")
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        e_ms = float(t.item())
+        dist.barrier()
+    torch.cuda.synchronize()
+    with ClockSampler(local_rank) as clk:
+        head, ms, ms_list, touched, launches, ws, entry = measure(moe, wl, x, layer, args, flush, stream, clk,
+                                                                  pk, pk_kind)
+        if dist:
+            t = torch.tensor([ms], device="cuda")
+            dist.all_reduce(t, op=dist.ReduceOp.MAX)
+            ms = float(t.item())
+        value = world * T / (ms * 1e-3)
+
+        # end to end through the public API with host buffers
+        y = torch.empty_like(x)
+        xh = x.cpu().pin_memory()
+        yh = torch.empty_like(xh).pin_memory()
+        xd = torch.empty_like(x)
+
+        def e2e_step():
+            xd.copy_(xh, non_blocking=True)
+            entry(xd, layer, ws, out=y)
+            yh.copy_(y, non_blocking=True)
+        e_ms = float(np.mean(time_calls(e2e_step, args.steps, flush, stream, clk)))
+        if dist:
+            t = torch.tensor([e_ms], device="cuda")
+            dist.all_reduce(t, op=dist.ReduceOp.MAX)
+            e_ms = float(t.item())
+
+        per_config = {}
+        for c in others:
+            w2 = syn.WORKLOADS[c]
+            res = measure(moe, w2, x_for(w2), layer_for(w2), args, flush, stream, clk, pk, pk_kind)[0]
+            per_config[str(c)] = res
+            torch.cuda.empty_cache()
+        layer = layer_for(wl)          # restore the headline workload's bias for the CPU leg
 
     line = {
         "metric": METRIC, "value": round(value, 1), "unit": UNIT, "n_gpus": world, "steps": args.steps,
@@ -391,13 +503,16 @@ def main():
                    "l2": "flushed before every step (256 MB write, outside the events)",
                    "parallelism": f"replicas x{world}" if world > 1 else "single GPU",
                    "algorithmic_bytes_per_step": layer_bytes(wl, touched),
-                   "algorithmic_flops_per_step": layer_flops(wl),
-                   "hbm_frac_whole_layer": round(layer_bytes(wl, touched) / (ms * 1e-3) / 1e9 / pk["hbm_gbs"], 4)},
-        "roofline": roof,
+                   "algorithmic_flops_per_step": layer_flops(wl)},
+        "layer_ms": head["layer_ms"],
+        "roofline": head["roofline"],
+        "layer_roofline": head["layer_roofline"],
+        "steps_ms": head.get("steps_ms"),
         "e2e": {"value": round(world * T / (e_ms * 1e-3), 1), "unit": UNIT,
-                "h2d_bytes_per_step": int(x.numel() * 2), "d2h_bytes_per_step": int(y.numel() * 2)},
+                "h2d_bytes_per_step": int(x.numel() * 2), "d2h_bytes_per_step": int(x.numel() * 2)},
         "gpu_launches": launches,
         "clocks": clk.summary(),
+        "per_config": per_config,
     }
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         line["cpu_baseline"] = cpu_baseline(wl, moe, x, layer)

@@ -68,7 +68,10 @@ typedef enum {
     MOE_ERR_CUDA = -3,        /* a CUDA call or kernel launch failed          */
     MOE_ERR_TIMEOUT = -4,     /* device status: a bounded wait ran out        */
     MOE_ERR_WORKSPACE = -5,   /* workspace missing or too small               */
-    MOE_ERR_DEVICE_INDEX = -6 /* device status: an index was out of range     */
+    MOE_ERR_DEVICE_INDEX = -6,/* device status: an index was out of range     */
+    MOE_ERR_NONFINITE = -7    /* device status: an activation row held an inf
+                                 or NaN where the kernel needs a finite row
+                                 maximum; that row's outputs are NaN        */
 } moe_status;
 
 typedef enum { MOE_FMT_INT4_G128 = 0, MOE_FMT_NVFP4 = 1, MOE_FMT_BF16 = 2 } moe_wfmt;
@@ -111,8 +114,22 @@ size_t moe_workspace_bytes(int T, int H, int E, int F, int top_k);
 int moe_workspace_init(void* ws, size_t ws_bytes, moe_stream_t stream);
 
 /* Synchronise `stream`, copy the workspace's device status word to
- * *status_out (MOE_OK or a negative moe_status), and clear it. */
+ * *status_out (MOE_OK or a negative moe_status; the first condition recorded
+ * wins), and clear it.  When it was not MOE_OK, the arrival counters of the
+ * control block are cleared too (a kernel that stopped early may have left
+ * them set), so the workspace serves the next call. */
 int moe_read_status(void* ws, moe_stream_t stream, int32_t* status_out);
+
+/* Bound, in nanoseconds, on each device-side wait of the tensor-core kernels
+ * and the fused router when they run with this workspace (stream-ordered: a
+ * one-thread kernel writes words 4-5 of the control block).  0 restores the
+ * default of about 2 s, which a zero-filled workspace starts with.  A wait
+ * that runs out records MOE_ERR_TIMEOUT, the kernel stops issuing work,
+ * waits (bounded by the default) for the copies and MMAs it has in flight,
+ * releases its tensor memory and returns; its outputs are then undefined.
+ * For failure testing: a bound shorter than the kernels' normal waits makes
+ * every call time out.  The pages have no counterpart to this call. */
+int moe_set_wait_limit(void* ws, uint64_t limit_ns, moe_stream_t stream);
 
 /* Static description of a status code. */
 const char* moe_status_string(int status);
@@ -141,8 +158,12 @@ int moe_route_topk(const void* x, int T, int H, const float* router_w,
                    const float* router_bias, int E, int top_k, int32_t* topk_ids,
                    float* topk_w, void* ws, size_t ws_bytes, moe_stream_t stream);
 
-/* Token -> expert bucketing: a stable counting sort of the R = T*top_k slots
- * (slot = t*top_k + j) by expert id.
+/* Token -> expert bucketing ("Step 5 Preview: 92 narrow layers...", The
+ * shape: each token goes to its 8 routed experts, whose weights sit in the
+ * fused [E, out, in] banks of "Step-5-Preview-Int4-g128", Tensor layout, so
+ * each expert's tokens are gathered into one contiguous block of rows): a
+ * stable counting sort of the R = T*top_k slots (slot = t*top_k + j) by
+ * expert id.
  * topk_ids: int32 [T, top_k], each in [0, E) (an id outside sets the device
  * status MOE_ERR_DEVICE_INDEX and is dropped);
  * expert_offsets: int32 [E+1] (out), exclusive prefix sum of per-expert counts;
@@ -168,12 +189,17 @@ int moe_permute(const int32_t* topk_ids, int T, int top_k, int E,
  * stream capture.  All calls share the array and each call overwrites it:
  * calls that may overlap on the GPU (different streams with no ordering
  * between them) race.  An expert id outside [0, E) is dropped and its slot_row
- * entry is -1.  The paper has no counterpart to this call. */
+ * entry is -1; that condition is not reported (no caller can read the static
+ * array's status word), and row_slot past expert_offsets[E] is left
+ * unwritten.  The paper has no counterpart to this call. */
 int moe_permute_noalloc(const int32_t* topk_ids, int T, int top_k, int E,
                         int32_t* expert_offsets, int32_t* row_slot, int32_t* slot_row,
                         moe_stream_t stream);
 
-/* Grouped gate/up projection with fused SwiGLU, weights dequantised in-kernel:
+/* Grouped gate/up projection with fused SwiGLU, weights dequantised in-kernel
+ * ("Step 5 Preview: 92 narrow layers...", The shape: routed SwiGLU experts of
+ * width 1536 at hidden 4096; weights as "Step-5-Preview-Int4-g128", Recipe /
+ * Tensor layout, or "Step-5-Preview-NVFP4-Local", Format):
  * for each expert e and row r in [expert_offsets[e], expert_offsets[e+1]),
  * with token t = row_slot[r] / top_k:
  *     h_perm[r, f] = bf16( silu(g) * u ),  g = x[t] . Wg[e,f,:],  u = x[t] . Wu[e,f,:]
@@ -198,7 +224,12 @@ int moe_grouped_w4a16_swiglu(const void* x, int T, int H,
                              float swiglu_limit, void* h_perm,
                              void* ws, size_t ws_bytes, moe_stream_t stream);
 
-/* Grouped down projection with the routing weight fused:
+/* Grouped down projection with the routing weight fused ("Step 5 Preview:
+ * 92 narrow layers...", The shape: the down projection of each routed SwiGLU
+ * expert, [E, 4096, 1536] in the banks of "Step-5-Preview-Int4-g128", Tensor
+ * layout / "Step-5-Preview-NVFP4-Local", Format; the token's output weighs
+ * each routed expert by its renormalised sigmoid score, "Step-5-Preview-Spark",
+ * At a glance):
  *     y_perm[r, :] = bf16( topk_w[row_slot[r]] * (h_perm[r] . Wd[e]^T) )
  * for rows r of expert e (fp32 accumulation).  h_perm: bf16 [rows, F];
  * topk_w: fp32 [rows] indexed by slot, or NULL for weight 1;
@@ -216,7 +247,9 @@ int moe_grouped_w4a16_down(const void* h_perm, const int32_t* expert_offsets,
                            const moe_qweight* down, void* y_perm,
                            void* ws, size_t ws_bytes, moe_stream_t stream);
 
-/* Unpermute and combine:
+/* Unpermute and combine ("Step 5 Preview: 92 narrow layers...", The shape:
+ * a token's output is its shared expert plus its 8 routed experts; the
+ * routing weight was applied by the down projection):
  *     y[t, :] = bf16( shared_out[t, :] + sum_{j<top_k} y_perm[slot_row[t*top_k + j], :] )
  * summed in fp32 in the order shared, j = 0..top_k-1.  y_perm: bf16 [T*top_k, H];
  * shared_out: bf16 [T, H] or NULL; y: bf16 [T, H] (out). */
@@ -226,7 +259,13 @@ int moe_unpermute_combine(const void* y_perm, const int32_t* slot_row, int T,
 
 /* The whole layer for decode-sized batches (1 <= T <= 64): router, bucketing,
  * gate/up + SwiGLU, down with routing weights, shared expert and combine, on
- * device with no host synchronisation.  x: bf16 [T, H]; y: bf16 [T, H] (out). */
+ * device with no host synchronisation ("Step-5-Preview-Spark", At a glance and
+ * How it was made: the decode path of the layer, 8 routed experts plus one
+ * shared per token; "Step 5 Preview: 92 narrow layers...", The shape).
+ * x: bf16 [T, H]; y: bf16 [T, H] (out).  The shared expert runs on a
+ * per-device side stream that the caller's stream forks to and joins; calls
+ * from several host threads are safe with separate workspaces (their
+ * shared-expert work is serialised on that side stream). */
 int moe_layer_decode(const void* x, int T, const moe_layer* L, void* y,
                      void* ws, size_t ws_bytes, moe_stream_t stream);
 

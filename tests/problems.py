@@ -62,7 +62,12 @@ def build(cfg, mode="quantised", T=None, seed=0, experts=None, shared=None, chec
     P.ids, P.w, P.scores = oracle.route(P.x, P.Wr, P.bias, wl.k, want_scores=True)
     P.check_tokens = np.arange(P.T, dtype=np.int32) if check_tokens is None else np.asarray(check_tokens, np.int32)
     if experts is None:
-        experts = sorted(set(P.ids[P.check_tokens].ravel().tolist()))
+        ex = set(P.ids[P.check_tokens].ravel().tolist())
+        # a near-tied token may select its (k+1)-th expert on the GPU: give that expert weights too
+        nt = P.check_tokens[near_tie_tokens(P.scores[P.check_tokens], wl.k)]
+        for t in nt:
+            ex.update(np.argsort(-P.scores[t], kind="stable")[:wl.k + 2].tolist())
+        experts = sorted(ex)
     P.experts = experts
     P.banks = {}
     for which in ("gate", "up", "down"):
@@ -121,3 +126,69 @@ def near_tie_tokens(scores, k, eps=1e-5):
     s = -np.sort(-scores, axis=1)[:, :k + 1]
     gaps = s[:, :-1] - s[:, 1:]
     return np.nonzero(np.min(gaps, axis=1) <= eps)[0]
+
+
+def tile_edge_tokens(ids, E, k, nheavy=12, nmaxes=(64, 128, 256), nlight=0):
+    """Tokens whose routed rows sit at both edges of every n-tile of the
+    nheavy most loaded experts (and the nlight least loaded non-empty ones),
+    for the balanced row partitions of the grouped GEMM at each tile height
+    in nmaxes (n rows in ceil(n / nmax) tiles of ceil(n / ntile) rows)."""
+    off, rs, _ = oracle.permute(ids, E)
+    cnt = np.diff(off)
+    order = np.argsort(-cnt, kind="stable")
+    chosen = list(order[:nheavy])
+    if nlight:
+        chosen += [e for e in order[::-1] if cnt[e] > 0][:nlight]
+    rows = set()
+    for e in chosen:
+        n = int(cnt[e])
+        for nm in nmaxes:
+            nt = -(-n // nm)
+            per = -(-n // nt)
+            for i in range(nt):
+                a = i * per
+                b = min(n, a + per) - 1
+                rows.update((int(off[e] + a), int(off[e] + b)))
+    return sorted(set(int(rs[r]) // k for r in rows))
+
+
+# ---- comparisons ------------------------------------------------------------
+
+def check_ids(ids_gpu, P, tokens):
+    """Exact ids outside near ties; valid selections inside.  Returns the
+    near-tie tokens found among `tokens`."""
+    k = P.wl.k
+    nt = set(near_tie_tokens(P.scores[tokens], k).tolist())
+    flipped = []
+    for i, t in enumerate(tokens):
+        if i in nt:
+            s = P.scores[t]
+            kth = -np.sort(-s)[k - 1]
+            sel = ids_gpu[i]
+            assert len(set(sel.tolist())) == k
+            assert np.all(s[sel] >= kth - 1e-5), (t, sel)
+            if not np.array_equal(sel, P.ids[t]):
+                flipped.append(int(t))
+        else:
+            assert np.array_equal(ids_gpu[i], P.ids[t]), (t, ids_gpu[i], P.ids[t])
+    return nt, flipped
+
+
+def layer_check(P, y_gpu, tokens, ids_gpu, w_gpu):
+    """Every listed token against the oracle.  ids_gpu / w_gpu: the GPU's routing
+    of those tokens.  A near-tied token is recomputed in the oracle with the
+    GPU's ids and weights (either selection is a valid top-k), so its output is
+    checked too."""
+    nt, flipped = check_ids(ids_gpu, P, tokens)
+    ids = P.ids.copy()
+    w = P.w.copy()
+    for i in nt:
+        ids[tokens[i]] = ids_gpu[i]
+        w[tokens[i]] = w_gpu[i]
+    ref = oracle.moe_forward(P.x, ids, w, P.banks["gate"], P.banks["up"], P.banks["down"],
+                             shared=P.shared, tokens=tokens)
+    got = oracle.bf16_to_f32(y_gpu[tokens]).astype(np.float64)
+    tol = layer_tolerance(ref)
+    err = np.abs(got - ref)
+    assert np.all(err <= tol), f"max err {err.max()} (tol scale {1e-2 * np.max(np.abs(ref))})"
+    return len(nt), len(flipped), float(err.max() / np.max(np.abs(ref)))

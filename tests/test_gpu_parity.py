@@ -7,7 +7,8 @@ whose oracle top-8 has a near tie (adjacent scores within 1e-5; the pages
 note that a 352-expert top-8 router flips near-tied choices under tiny
 summation-order changes, "Step-5-Preview-Spark", Quality) accept either
 selection: their GPU ids must be a valid top-8 within 1e-5 of the oracle's
-scores, and they are counted and excluded from the element-wise output check.
+scores, they are counted, and their layer output is compared with the oracle
+recomputed with the GPU's ids and weights.
 """
 import numpy as np
 import pytest
@@ -17,8 +18,8 @@ import oracle
 from weight_only_bit_route_b200 import moe
 from weight_only_bit_route_b200 import synthetic as syn
 
-from problems import (bf16_bits, build, dev, dev_bf16, device_bank, device_layer, layer_tolerance,
-                      near_tie_tokens)
+from problems import (bf16_bits, build, check_ids, dev, dev_bf16, device_bank, device_layer, layer_check,
+                      layer_tolerance, tile_edge_tokens)
 
 pytestmark = pytest.mark.gpu
 
@@ -31,26 +32,6 @@ def _cuda():
 
 def _ws(T, wl):
     return moe.workspace(T, wl.H, wl.E, wl.F, wl.k)
-
-
-def _check_ids(ids_gpu, P, tokens):
-    """Exact ids outside near ties; valid selections inside.  Returns the
-    near-tie tokens found among `tokens`."""
-    k = P.wl.k
-    nt = set(near_tie_tokens(P.scores[tokens], k).tolist())
-    flipped = []
-    for i, t in enumerate(tokens):
-        if i in nt:
-            s = P.scores[t]
-            kth = -np.sort(-s)[k - 1]
-            sel = ids_gpu[i]
-            assert len(set(sel.tolist())) == k
-            assert np.all(s[sel] >= kth - 1e-5), (t, sel)
-            if not np.array_equal(sel, P.ids[t]):
-                flipped.append(int(t))
-        else:
-            assert np.array_equal(ids_gpu[i], P.ids[t]), (t, ids_gpu[i], P.ids[t])
-    return nt, flipped
 
 
 # ---------------------------------------------------------------------------
@@ -114,7 +95,7 @@ def test_route_topk(cfg, T):
     ids, w = moe.route_topk(dev_bf16(x), dev(Wr), None if b is None else dev(b), wl.k, ws)
     torch.cuda.synchronize()
     ids, w = ids.cpu().numpy(), w.cpu().numpy()
-    nt, flipped = _check_ids(ids, P, np.arange(T))
+    nt, flipped = check_ids(ids, P, np.arange(T))
     ok = np.array([i not in nt for i in range(T)])
     assert np.allclose(w[ok], w_ref[ok], rtol=2e-5, atol=1e-7)
     assert np.all(np.abs(w.sum(1) - 1) < 1e-5)
@@ -242,10 +223,10 @@ def test_layer_streaming_gemv_path(fmt):
     ws = _ws(P.T, wl)
     x = dev_bf16(P.x)
     y = moe.layer_decode(x, L, ws)
-    ids, _ = moe.route_topk(x, L.router_w, L.router_bias, wl.k, ws)
+    ids, w = moe.route_topk(x, L.router_w, L.router_bias, wl.k, ws)
     torch.cuda.synchronize()
     assert moe.read_status(ws) == 0
-    _layer_check(P, bf16_bits(y), np.arange(P.T, dtype=np.int32), ids.cpu().numpy())
+    layer_check(P, bf16_bits(y), np.arange(P.T, dtype=np.int32), ids.cpu().numpy(), w.cpu().numpy())
 
 
 def _mid(fmt, T):
@@ -264,10 +245,10 @@ def test_layer_down_width_not_multiple_of_512(fmt):
     ws = _ws(P.T, wl)
     x = dev_bf16(P.x)
     y = moe.layer_decode(x, L, ws)
-    ids, _ = moe.route_topk(x, L.router_w, L.router_bias, wl.k, ws)
+    ids, w = moe.route_topk(x, L.router_w, L.router_bias, wl.k, ws)
     torch.cuda.synchronize()
     assert moe.read_status(ws) == 0
-    _layer_check(P, bf16_bits(y), np.arange(P.T, dtype=np.int32), ids.cpu().numpy())
+    layer_check(P, bf16_bits(y), np.arange(P.T, dtype=np.int32), ids.cpu().numpy(), w.cpu().numpy())
 
 
 @pytest.mark.parametrize("T", [5, 300])
@@ -314,18 +295,6 @@ def bf16_ulp_arr(v):
 # whole layer
 # ---------------------------------------------------------------------------
 
-def _layer_check(P, y_gpu, tokens, ids_gpu):
-    nt, flipped = _check_ids(ids_gpu, P, tokens)
-    keep = np.array([i for i in range(len(tokens)) if i not in nt], np.int64)
-    ref = oracle.moe_forward(P.x, P.ids, P.w, P.banks["gate"], P.banks["up"], P.banks["down"],
-                             shared=P.shared, tokens=tokens[keep])
-    got = oracle.bf16_to_f32(y_gpu[tokens[keep]]).astype(np.float64)
-    tol = layer_tolerance(ref)
-    err = np.abs(got - ref)
-    assert np.all(err <= tol), f"max err {err.max()} (tol scale {1e-2 * np.max(np.abs(ref))})"
-    return len(nt), len(flipped), float(err.max() / np.max(np.abs(ref)))
-
-
 @pytest.mark.parametrize("cfg", [0, 1, 2])
 def test_layer_decode(cfg):
     P = build(cfg, "quantised" if cfg == 0 else "random")
@@ -334,28 +303,37 @@ def test_layer_decode(cfg):
     ws = _ws(P.T, wl)
     x = dev_bf16(P.x)
     y = moe.layer_decode(x, L, ws)
-    ids, _ = moe.route_topk(x, L.router_w, L.router_bias, wl.k, ws)
+    ids, w = moe.route_topk(x, L.router_w, L.router_bias, wl.k, ws)
     torch.cuda.synchronize()
     assert moe.read_status(ws) == 0
-    n_nt, n_flip, rel = _layer_check(P, bf16_bits(y), P.check_tokens, ids.cpu().numpy())
+    n_nt, n_flip, rel = layer_check(P, bf16_bits(y), P.check_tokens, ids.cpu().numpy(), w.cpu().numpy())
     print(f"cfg {cfg}: near-tie {n_nt}, flipped {n_flip}, max rel err {rel:.2e}")
 
 
 @pytest.mark.parametrize("cfg", [3, 4])
 def test_layer_forward_sampled(cfg):
+    """Full-size prefill layers, checked on the tokens whose rows sit at both
+    edges of every n-tile of the 12 most loaded experts (for the grouped GEMM's
+    balanced partitions at tile heights 64, 128 and 256), the first and last
+    token and 14 random ones; on the uniform workload also the 12 least loaded
+    experts' edges."""
     wl = syn.WORKLOADS[cfg]
     rng = np.random.default_rng(cfg)
-    tokens = np.sort(np.concatenate([[0, wl.T - 1], rng.choice(np.arange(1, wl.T - 1), 14, replace=False)])).astype(np.int32)
+    x_np = syn.gen_x(wl)
+    ids_o, _ = oracle.route(x_np, syn.gen_router(wl), syn.gen_bias(wl), wl.k)
+    edges = tile_edge_tokens(ids_o, wl.E, wl.k, nlight=0 if wl.skew else 12)
+    extra = [0, wl.T - 1] + rng.choice(np.arange(1, wl.T - 1), 14, replace=False).tolist()
+    tokens = np.array(sorted(set(edges) | set(extra)), np.int32)
     P = build(cfg, "random", check_tokens=tokens)
     L = device_layer(moe, P)
     ws = _ws(P.T, wl)
     x = dev_bf16(P.x)
     y = moe.layer_forward(x, L, ws)
-    ids, _ = moe.route_topk(x, L.router_w, L.router_bias, wl.k, ws)
+    ids, w = moe.route_topk(x, L.router_w, L.router_bias, wl.k, ws)
     torch.cuda.synchronize()
     assert moe.read_status(ws) == 0
-    n_nt, n_flip, rel = _layer_check(P, bf16_bits(y), tokens, ids.cpu().numpy()[tokens])
-    print(f"cfg {cfg}: near-tie {n_nt}, flipped {n_flip}, max rel err {rel:.2e}")
+    n_nt, n_flip, rel = layer_check(P, bf16_bits(y), tokens, ids.cpu().numpy()[tokens], w.cpu().numpy()[tokens])
+    print(f"cfg {cfg}: {len(tokens)} tokens checked, near-tie {n_nt}, flipped {n_flip}, max rel err {rel:.2e}")
 
 
 @pytest.mark.parametrize("fmt", ["int4", "nvfp4"])
@@ -369,12 +347,37 @@ def test_layer_forward_gemm_path_all_tokens(fmt):
     ws = _ws(P.T, wl)
     x = dev_bf16(P.x)
     y = moe.layer_forward(x, L, ws)
-    ids, _ = moe.route_topk(x, L.router_w, L.router_bias, wl.k, ws)
+    ids, w = moe.route_topk(x, L.router_w, L.router_bias, wl.k, ws)
     torch.cuda.synchronize()
     assert moe.read_status(ws) == 0
     tokens = np.arange(P.T, dtype=np.int32)
-    n_nt, n_flip, rel = _layer_check(P, bf16_bits(y), tokens, ids.cpu().numpy())
+    n_nt, n_flip, rel = layer_check(P, bf16_bits(y), tokens, ids.cpu().numpy(), w.cpu().numpy())
     print(f"{fmt}: near-tie {n_nt}, flipped {n_flip}, max rel err {rel:.2e}")
+
+
+def _wide(fmt, T):
+    # F = 512: with E = 32 both int4 projections can take the 8-bit GEMM (down K = F is a multiple of 512)
+    base = syn.WORKLOADS[0]
+    return syn.Workload(f"wide_{fmt}_T{T}", T, 1024, 32, 512, base.k, fmt, False, base.router_std, False)
+
+
+@pytest.mark.parametrize("T", [64, 65])
+def test_layer_int4_path_crossover(T):
+    """64 tokens make 512 routed rows, the most the 8-bit int4 GEMM takes;
+    65 tokens (520 rows) run the 16-bit int4 GEMM.  Every token of both
+    layers against the oracle, shared expert included."""
+    wl = _wide("int4", T)
+    P = build(wl, "quantised", shared=True)
+    L = device_layer(moe, P)
+    ws = _ws(P.T, wl)
+    x = dev_bf16(P.x)
+    y = moe.layer_forward(x, L, ws)
+    ids, w = moe.route_topk(x, L.router_w, L.router_bias, wl.k, ws)
+    torch.cuda.synchronize()
+    assert moe.read_status(ws) == 0
+    tokens = np.arange(P.T, dtype=np.int32)
+    n_nt, n_flip, rel = layer_check(P, bf16_bits(y), tokens, ids.cpu().numpy(), w.cpu().numpy())
+    print(f"T={T}: near-tie {n_nt}, flipped {n_flip}, max rel err {rel:.2e}")
 
 
 def test_layer_zero_input_is_zero():

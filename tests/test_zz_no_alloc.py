@@ -10,6 +10,7 @@ import numpy as np
 import pytest
 import torch
 
+import oracle
 from weight_only_bit_route_b200 import moe
 
 pytestmark = pytest.mark.gpu
@@ -33,6 +34,11 @@ def test_permute_noalloc_matches_workspace_permute():
         assert torch.equal(off, off2)
         assert torch.equal(rs, rs2)
         assert torch.equal(sr, sr2)
+        # and against the oracle's bucketing directly
+        o_off, o_rs, o_sr = oracle.permute(ids_np, E)
+        assert np.array_equal(off2.cpu().numpy(), o_off)
+        assert np.array_equal(rs2.cpu().numpy(), o_rs)
+        assert np.array_equal(sr2.cpu().numpy(), o_sr)
 
 
 def test_permute_noalloc_rejects_oversize():

@@ -116,10 +116,15 @@ int layer_checks(const void* x, int T, const moe_layer* L, void* y, void* ws, si
 }
 
 // A non-blocking stream per device for the shared expert, with fork/join
-// events, created on first use.
+// events, created on first use.  A layer call holds `call` from its fork
+// record until its stream's wait on the join event is enqueued, so calls
+// from several host threads cannot interleave their records on the shared
+// events (their shared-expert work then runs one after another on the side
+// stream).
 struct SideStream {
     cudaStream_t s = nullptr;
     cudaEvent_t fork = nullptr, join = nullptr;
+    std::mutex call;
 };
 int side_stream(SideStream** out) {
     static std::mutex mu;
@@ -164,8 +169,10 @@ int layer_run(const void* x, int T, const moe_layer* L, void* y, void* ws, cudaS
     // for it before the combine.  Its own routing (offsets {0, T}, row i at
     // slot i * top_k) comes first on that stream.
     SideStream* side = nullptr;
+    std::unique_lock<std::mutex> side_lock;
     if (has_sh) {
         MOE_TRY(side_stream(&side));
+        side_lock = std::unique_lock<std::mutex>(side->call);
         if (cudaEventRecord(side->fork, s) != cudaSuccess || cudaStreamWaitEvent(side->s, side->fork, 0) != cudaSuccess)
             return MOE_ERR_CUDA;
         GemvProblem sg{};
@@ -268,8 +275,18 @@ int moe_read_status(void* ws, moe_stream_t stream, int32_t* status_out) {
     if (cudaMemcpyAsync(&v, ws, 4, cudaMemcpyDeviceToHost, cs(stream)) != cudaSuccess) return MOE_ERR_CUDA;
     if (cudaStreamSynchronize(cs(stream)) != cudaSuccess) return MOE_ERR_CUDA;
     *status_out = v;
-    if (v != 0 && cudaMemsetAsync(ws, 0, 4, cs(stream)) != cudaSuccess) return MOE_ERR_CUDA;
+    if (v != 0) {
+        // a kernel that stopped early may have left its arrival counters (router word 1,
+        // split-K words 16..255) non-zero: clear them with the status word
+        if (cudaMemsetAsync(ws, 0, 8, cs(stream)) != cudaSuccess) return MOE_ERR_CUDA;
+        if (cudaMemsetAsync(at<int32_t>(ws, 64), 0, kStepScratch - 64, cs(stream)) != cudaSuccess) return MOE_ERR_CUDA;
+    }
     return MOE_OK;
+}
+
+int moe_set_wait_limit(void* ws, uint64_t limit_ns, moe_stream_t stream) {
+    if (!ws || (reinterpret_cast<uintptr_t>(ws) & 255u)) return MOE_ERR_WORKSPACE;
+    return launch_set_u64(at<unsigned long long>(ws, 16), limit_ns, cs(stream));
 }
 
 uint64_t moe_launch_count(void) { return moe::g_launches.load(std::memory_order_relaxed); }
@@ -283,6 +300,7 @@ const char* moe_status_string(int status) {
         case MOE_ERR_TIMEOUT: return "device wait timed out";
         case MOE_ERR_WORKSPACE: return "workspace missing, misaligned or too small";
         case MOE_ERR_DEVICE_INDEX: return "index out of range on device";
+        case MOE_ERR_NONFINITE: return "non-finite activation on device";
     }
     return "unknown status";
 }

@@ -69,4 +69,13 @@ int launch_shared_routing(int T, int k, int32_t* sh_offsets, int32_t* sh_rowslot
     return cudaGetLastError() == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
 }
 
+// One 64-bit word of the workspace control block (moe_set_wait_limit).
+__global__ void set_u64_kernel(unsigned long long* dst, unsigned long long v) { *dst = v; }
+
+int launch_set_u64(unsigned long long* dst, unsigned long long v, cudaStream_t s) {
+    set_u64_kernel<<<1, 1, 0, s>>>(dst, v);
+    count_launch();
+    return cudaGetLastError() == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
+}
+
 }  // namespace moe

@@ -245,7 +245,7 @@ __global__ void __launch_bounds__(G_THREADS, 1) tc_grouped_gemm(const __grid_con
     __shared__ int s_prefix[kMaxE];
     __shared__ int s_wsum[G_THREADS / 32], s_wt[G_THREADS / 32];
     __shared__ int s_nact, s_total;
-    __shared__ volatile int s_abort;
+    __shared__ volatile GAbort s_ab;
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int MT = a.out_dim / G_BM;
@@ -285,13 +285,15 @@ __global__ void __launch_bounds__(G_THREADS, 1) tc_grouped_gemm(const __grid_con
             asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(g_smem(&acc_empty[s])), "r"(G_EPI_WARPS));
         asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(g_smem(&drain)), "r"(C::kI8 ? 2 : 1));
         asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
-        s_abort = 0;
+        s_ab.flag = 0;
+        s_ab.limit_ns = G_WAIT_NS;
     }
     if (warp == 2) {
         asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], 512;" ::"r"(g_smem(&s_tmem)));
         asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;");
     }
     asm volatile("griddepcontrol.wait;" ::: "memory");
+    if (tid == 0) s_ab.limit_ns = g_limit_from(a.status);   // published by the __syncthreads below
 
     // tile list: active experts and the prefix sum of their tile counts
     {
@@ -361,19 +363,19 @@ __global__ void __launch_bounds__(G_THREADS, 1) tc_grouped_gemm(const __grid_con
     };
     auto fail = [&]() {
         set_status(a.status, MOE_ERR_TIMEOUT);
-        s_abort = 1;
+        s_ab.flag = 1;
     };
 
     if (warp == 0) {
         // ---------------- weight producer (whole warp, one lane issues) ----------------
         uint32_t pc = 0;
         int t = 0;
-        for (int tile = blockIdx.x; tile < ntiles && !s_abort; tile += gridDim.x) {
+        for (int tile = blockIdx.x; tile < ntiles && !g_aborted(&s_ab); tile += gridDim.x) {
             const GTile T = tile_of(tile);
             const int row0 = T.e * a.out_dim + T.m0;
             if (C::kInt4) {
                 const int b = t % NSC;
-                if (t >= NSC && !g_wait_w(g_smem(&sc_empty[b]), ((t / NSC) - 1) & 1, &s_abort, 64)) { fail(); break; }
+                if (t >= NSC && !g_wait_w(g_smem(&sc_empty[b]), ((t / NSC) - 1) & 1, &s_ab, 64)) { fail(); break; }
                 const uint32_t bar = g_smem(&sc_full[b]);
                 uint8_t* dst = scbuf + b * sc_buf_bytes;
                 const uint32_t zbytes = C::kI8 ? uint32_t(T.nval * zst * 4) : 0u;
@@ -391,9 +393,9 @@ __global__ void __launch_bounds__(G_THREADS, 1) tc_grouped_gemm(const __grid_con
             for (int ps = 0; ps < NPS; ps++, pc++) {
                 const int s = pc % NPK;
                 // 4-bit stages are freed by the dequantisation warps, BF16 ones by the MMA step
-                if (pc >= NPK && !(C::kTmemA ? g_wait_w(g_smem(&pk_empty[s]), ((pc / NPK) - 1) & 1, &s_abort, 32)
+                if (pc >= NPK && !(C::kTmemA ? g_wait_w(g_smem(&pk_empty[s]), ((pc / NPK) - 1) & 1, &s_ab, 32)
                                              : g_wait_w(g_smem(&done[(pc - NPK) % G_DONE]), ((pc - NPK) / G_DONE) & 1,
-                                                        &s_abort, 32))) {
+                                                        &s_ab, 32))) {
                     ok = false;
                     break;
                 }
@@ -439,7 +441,7 @@ __global__ void __launch_bounds__(G_THREADS, 1) tc_grouped_gemm(const __grid_con
     } else if (warp == 1) {
         // ---------------- activation producer (whole warp, one lane issues) ----------------
         uint32_t bc = 0;
-        for (int tile = blockIdx.x; tile < ntiles && !s_abort; tile += gridDim.x) {
+        for (int tile = blockIdx.x; tile < ntiles && !g_aborted(&s_ab); tile += gridDim.x) {
             const GTile T = tile_of(tile);
             const int row0 = (C::kI8 ? 3 : 1) * (T.ebase + T.n0);      // i8: three digit rows per token
             const CUtensorMap* map = &a.tm_b[C::kI8 ? 0 : T.bn / 16 - 1];
@@ -447,7 +449,7 @@ __global__ void __launch_bounds__(G_THREADS, 1) tc_grouped_gemm(const __grid_con
             for (int ks = 0; ks < KS; ks++, bc++) {
                 const int s = bc % C::kBStages;
                 if (bc >= uint32_t(C::kBStages) && !g_wait_w(g_smem(&done[(bc - C::kBStages) % G_DONE]),
-                                                             ((bc - C::kBStages) / G_DONE) & 1, &s_abort, 32)) {
+                                                             ((bc - C::kBStages) / G_DONE) & 1, &s_ab, 32)) {
                     ok = false;
                     break;
                 }
@@ -494,12 +496,12 @@ __global__ void __launch_bounds__(G_THREADS, 1) tc_grouped_gemm(const __grid_con
         const uint32_t n_iss = C::kI8 ? 2u : 1u, iss = uint32_t(warp - 2);
         uint32_t bc = 0, ac = 0, pc = 0;
         int t = 0;
-        for (int tile = blockIdx.x; tile < ntiles && !s_abort; tile += gridDim.x, t++) {
+        for (int tile = blockIdx.x; tile < ntiles && !g_aborted(&s_ab); tile += gridDim.x, t++) {
             const GTile T = tile_of(tile);
             const uint32_t idesc = C::kI8 ? g_idesc_i8(T.bn) : g_idesc(T.bn, C::kMmaF16);
             const int buf = t & 1;
             uint32_t d = tmem + buf * 128;
-            if (!C::kI8 && t >= 2 && !g_wait_w(g_smem(&acc_empty[buf]), ((t >> 1) - 1) & 1, &s_abort)) {
+            if (!C::kI8 && t >= 2 && !g_wait_w(g_smem(&acc_empty[buf]), ((t >> 1) - 1) & 1, &s_ab)) {
                 fail();
                 break;
             }
@@ -512,18 +514,18 @@ __global__ void __launch_bounds__(G_THREADS, 1) tc_grouped_gemm(const __grid_con
                     continue;
                 }
                 const int sb = bc % C::kBStages, sa = ac % C::kAStages;
-                if (!g_wait_w(g_smem(&b_full[sb]), (bc / C::kBStages) & 1, &s_abort)) { ok = false; break; }
+                if (!g_wait_w(g_smem(&b_full[sb]), (bc / C::kBStages) & 1, &s_ab)) { ok = false; break; }
                 if (C::kI8) g_fence_proxy_async();      // B was written through the generic proxy
                 if (C::kTmemA) {
-                    if (!g_wait_w(g_smem(&a_full[sa]), (ac / C::kAStages) & 1, &s_abort)) { ok = false; break; }
+                    if (!g_wait_w(g_smem(&a_full[sa]), (ac / C::kAStages) & 1, &s_ab)) { ok = false; break; }
                 } else {
-                    if (!g_wait_w(g_smem(&pk_full[pc % NPK]), (pc / NPK) & 1, &s_abort)) { ok = false; break; }
+                    if (!g_wait_w(g_smem(&pk_full[pc % NPK]), (pc / NPK) & 1, &s_ab)) { ok = false; break; }
                 }
                 if (C::kI8) {
                     // every step into the next accumulator buffer, freed by the epilogue
                     const int bi = bc % C::kAccBufs;
                     if (bc >= uint32_t(C::kAccBufs) &&
-                        !g_wait_w(g_smem(&acc_empty[bi]), ((bc / C::kAccBufs) - 1) & 1, &s_abort)) { ok = false; break; }
+                        !g_wait_w(g_smem(&acc_empty[bi]), ((bc / C::kAccBufs) - 1) & 1, &s_ab)) { ok = false; break; }
                     d = tmem + bi * C::kAccCols;
                 }
                 g_fence_after();
@@ -578,7 +580,7 @@ __global__ void __launch_bounds__(G_THREADS, 1) tc_grouped_gemm(const __grid_con
         uint32_t ac = 0;
         int t = 0;
         bool ok = true;
-        for (int tile = blockIdx.x; tile < ntiles && ok && !s_abort; tile += gridDim.x, t++) {
+        for (int tile = blockIdx.x; tile < ntiles && ok && !g_aborted(&s_ab); tile += gridDim.x, t++) {
             const GTile T = tile_of(tile);
             const int f = T.m0 + r;
             const int rbase = T.ebase + T.n0;
@@ -587,7 +589,7 @@ __global__ void __launch_bounds__(G_THREADS, 1) tc_grouped_gemm(const __grid_con
             // the row factor (2^-c, times the routing weight on down, folded by the pre-pass)
             // is needed after the last step: issue its load now
             const float rowf = live ? a.act_scale[rbase + lane] : 1.f;
-            if (!g_wait(g_smem(&sc_full[b]), (t / NSC) & 1, &s_abort, 64)) { ok = false; break; }
+            if (!g_wait_w(g_smem(&sc_full[b]), (t / NSC) & 1, &s_ab, 64)) { ok = false; break; }
             const __nv_bfloat16* sc0 = reinterpret_cast<const __nv_bfloat16*>(scbuf + b * sc_buf_bytes) + r * ngroups;
             const __nv_bfloat16* sc1 = sc0 + G_BM * ngroups;
             const float* zs = reinterpret_cast<const float*>(scbuf + b * sc_buf_bytes + C::kNMat * sc_mat_bytes);
@@ -596,7 +598,7 @@ __global__ void __launch_bounds__(G_THREADS, 1) tc_grouped_gemm(const __grid_con
             for (int j = 0; j < C::kNMax; j++) tg[j] = tu[j] = 0.f;
             for (int ks = 0; ks < KS; ks++, ac++) {
                 const int bi = ac % C::kAccBufs;
-                if (!g_wait(g_smem(&done[ac % G_DONE]), (ac / G_DONE) & 1, &s_abort)) { ok = false; break; }
+                if (!g_wait_w(g_smem(&done[ac % G_DONE]), (ac / G_DONE) & 1, &s_ab)) { ok = false; break; }
                 g_fence_after();
                 uint32_t g[C::kGroups][16], u[C::kGroups][16];
                 const uint32_t ab = tmem + lane_addr + bi * C::kAccCols;
@@ -661,7 +663,7 @@ __global__ void __launch_bounds__(G_THREADS, 1) tc_grouped_gemm(const __grid_con
         const int q = warp & 3;
         const uint32_t lane_addr = uint32_t(q * 32) << 16;
         int t = 0;
-        for (int tile = blockIdx.x; tile < ntiles && !s_abort; tile += gridDim.x, t++) {
+        for (int tile = blockIdx.x; tile < ntiles && !g_aborted(&s_ab); tile += gridDim.x, t++) {
             const GTile T = tile_of(tile);
             const int buf = t & 1;
             const int rbase = T.ebase + T.n0;
@@ -680,7 +682,7 @@ __global__ void __launch_bounds__(G_THREADS, 1) tc_grouped_gemm(const __grid_con
             float rowf0 = row_factor(0);
             float gsc = 1.f, usc = 1.f;
             if (FMT == MOE_FMT_NVFP4) { gsc = a.g0[T.e]; if (GU) usc = a.g1[T.e]; }
-            if (!g_wait(g_smem(&acc_full[buf]), (t >> 1) & 1, &s_abort, 128)) { fail(); break; }
+            if (!g_wait_w(g_smem(&acc_full[buf]), (t >> 1) & 1, &s_ab, 128)) { fail(); break; }
             g_fence_after();
             const int f = T.m0 + q * 32 + lane;
             const int fo = a.perm_out ? ((f & ~7) | ((f & 7) < 4 ? 2 * (f & 7) : 2 * (f & 7) - 7)) : f;
@@ -782,11 +784,11 @@ __global__ void __launch_bounds__(G_THREADS, 1) tc_grouped_gemm(const __grid_con
         const uint32_t lane_addr = uint32_t(q * 32) << 16;
         uint32_t pc = 0;
         bool ok = true;
-        for (int tile = blockIdx.x; tile < ntiles && ok && !s_abort; tile += gridDim.x) {
+        for (int tile = blockIdx.x; tile < ntiles && ok && !g_aborted(&s_ab); tile += gridDim.x) {
             for (int ps = 0; ps < NPS; ps++, pc++) {
                 if (int(pc & 1) != grp) continue;
                 const int s = pc % NPK;
-                if (!g_wait_w(g_smem(&pk_full[s]), (pc / NPK) & 1, &s_abort)) { ok = false; break; }
+                if (!g_wait_w(g_smem(&pk_full[s]), (pc / NPK) & 1, &s_ab)) { ok = false; break; }
                 const uint8_t* st = pk + s * C::kPkStageBytes;
                 uint32_t o[kNBuf][16];
                 uint4 raw[2][2];                                // packed chunks, loaded one piece ahead
@@ -808,7 +810,7 @@ __global__ void __launch_bounds__(G_THREADS, 1) tc_grouped_gemm(const __grid_con
                 unpack(std::integral_constant<int, 0>{});
                 const int sa = pc % C::kAStages;
                 if (pc >= uint32_t(C::kAStages) && !g_wait_w(g_smem(&done[(pc - C::kAStages) % G_DONE]),
-                                                             ((pc - C::kAStages) / G_DONE) & 1, &s_abort)) {
+                                                             ((pc - C::kAStages) / G_DONE) & 1, &s_ab)) {
                     ok = false;
                     break;
                 }
@@ -846,16 +848,16 @@ __global__ void __launch_bounds__(G_THREADS, 1) tc_grouped_gemm(const __grid_con
         uint32_t pc = 0;
         int t = 0;
         bool ok = true;
-        for (int tile = blockIdx.x; tile < ntiles && ok && !s_abort; tile += gridDim.x, t++) {
+        for (int tile = blockIdx.x; tile < ntiles && ok && !g_aborted(&s_ab); tile += gridDim.x, t++) {
             const uint8_t* scrow = nullptr;
             if (FMT == MOE_FMT_INT4_G128) {
                 const int b = t % NSC;
-                if (!g_wait(g_smem(&sc_full[b]), (t / NSC) & 1, &s_abort)) { ok = false; break; }
+                if (!g_wait_w(g_smem(&sc_full[b]), (t / NSC) & 1, &s_ab)) { ok = false; break; }
                 scrow = scbuf + b * sc_buf_bytes + (GU ? hsel * sc_mat_bytes : 0) + r * ngroups * 2;
             }
             for (int ps = 0; ps < NPS && ok; ps++, pc++) {
                 const int s = pc % NPK;
-                if (!g_wait(g_smem(&pk_full[s]), (pc / NPK) & 1, &s_abort)) { ok = false; break; }
+                if (!g_wait_w(g_smem(&pk_full[s]), (pc / NPK) & 1, &s_ab)) { ok = false; break; }
                 const uint8_t* st = pk + s * C::kPkStageBytes;
                 const uint8_t* wt = st + (GU ? hsel * C::kMatBytes : 0);
                 uint32_t scw = 0;                      // int4: bf16 scales of groups 2ps (low) and 2ps+1 (high)
@@ -890,8 +892,8 @@ __global__ void __launch_bounds__(G_THREADS, 1) tc_grouped_gemm(const __grid_con
                     if (l == 0) {
                         const uint32_t acn = pc * C::kAPerPk + j;    // A stage index in this CTA's stream
                         sa = acn % C::kAStages;
-                        if (acn >= uint32_t(C::kAStages) && !g_wait(g_smem(&done[(acn - C::kAStages) % G_DONE]),
-                                                                      ((acn - C::kAStages) / G_DONE) & 1, &s_abort)) {
+                        if (acn >= uint32_t(C::kAStages) && !g_wait_w(g_smem(&done[(acn - C::kAStages) % G_DONE]),
+                                                                      ((acn - C::kAStages) / G_DONE) & 1, &s_ab)) {
                             ok = false;
                             return;
                         }
@@ -987,13 +989,16 @@ __global__ void __launch_bounds__(256) g_prep(const __nv_bfloat16* __restrict__ 
 // scale[row] = 2^-c, times row_w[row_slot[row]] when row_w is given (the
 // down projection's routing weight; a power of two times w is exact);
 // zsum[row][g] (row stride zst) = 8 * sum of X over group g, the u - 8 offset
-// of the weights.
+// of the weights.  A row holding an infinity or a NaN has no fixed point: it
+// records MOE_ERR_NONFINITE and gets a NaN row factor, so its outputs are NaN
+// (as a floating-point product with that row would be) instead of finite
+// values made from meaningless digits.
 constexpr int G_PREP_I8_THREADS = 128;
 __global__ void __launch_bounds__(G_PREP_I8_THREADS) g_prep_i8(const __nv_bfloat16* __restrict__ src, int in_dim,
                                                                const int32_t* __restrict__ row_slot, int top_k,
                                                                int by_token, const float* __restrict__ row_w,
                                                                uint8_t* __restrict__ dst, float* __restrict__ scale,
-                                                               float* __restrict__ zsum) {
+                                                               float* __restrict__ zsum, int32_t* status) {
     __shared__ float s_max[G_PREP_I8_THREADS / 32];
     asm volatile("griddepcontrol.wait;" ::: "memory");
     const int row = blockIdx.x, tid = threadIdx.x, lane = tid & 31;
@@ -1010,9 +1015,10 @@ __global__ void __launch_bounds__(G_PREP_I8_THREADS) g_prep_i8(const __nv_bfloat
     if (lane == 0) s_max[tid >> 5] = amax;
     __syncthreads();
     amax = fmaxf(fmaxf(s_max[0], s_max[1]), fmaxf(s_max[2], s_max[3]));
+    const bool finite = isfinite(amax);                 // amax is NaN or inf when any element is
     int ex = 0;
-    frexpf(amax, &ex);                                  // amax < 2^ex
-    const int c = amax > 0.f ? min(22 - ex, 126) : 0;   // |x| 2^c < 2^22
+    if (finite) frexpf(amax, &ex);                      // amax < 2^ex
+    const int c = (finite && amax > 0.f) ? min(22 - ex, 126) : 0;   // |x| 2^c < 2^22
     const float fc = ldexpf(1.f, c);                    // a power of two: x * fc is exact
     uint8_t* d8 = dst + size_t(row) * 3 * in_dim;
     // 16 pieces of 8 make a group of 128: lanes 0-15 and 16-31 hold one group each
@@ -1026,7 +1032,7 @@ __global__ void __launch_bounds__(G_PREP_I8_THREADS) g_prep_i8(const __nv_bfloat
             uint32_t p2[2] = {0u, 0u}, p1[2] = {0u, 0u}, p0[2] = {0u, 0u};
 #pragma unroll
             for (int e = 0; e < 8; e++) {
-                const int X = __float2int_rn(xs[e] * fc);
+                const int X = finite ? __float2int_rn(xs[e] * fc) : 0;
                 zs += X;
                 const int d0 = ((X + 128) & 255) - 128;          // signed digits in [-128, 127]
                 const int X1 = (X - d0) >> 8;
@@ -1043,7 +1049,14 @@ __global__ void __launch_bounds__(G_PREP_I8_THREADS) g_prep_i8(const __nv_bfloat
         for (int o = 8; o > 0; o >>= 1) zs += __shfl_xor_sync(0xffffffffu, zs, o);
         if ((lane & 15) == 0 && i < n16) zsum[size_t(row) * zst + i / 16] = 8.f * float(zs);
     }
-    if (tid == 0) scale[row] = row_w ? (1.f / fc) * row_w[row_slot[row]] : 1.f / fc;
+    if (tid == 0) {
+        if (finite) {
+            scale[row] = row_w ? (1.f / fc) * row_w[row_slot[row]] : 1.f / fc;
+        } else {
+            scale[row] = __int_as_float(0x7fc00000);        // quiet NaN
+            set_status(status, MOE_ERR_NONFINITE);
+        }
+    }
 }
 
 // ---------------------------------------------------------------------------
@@ -1162,7 +1175,7 @@ int launch_grouped_gemm(const GemvProblem& p, bool gateup, int rows, const GemmB
             const float* row_w = gateup ? nullptr : p.topk_w;
             if (launch_pdl(g_prep_i8, dim3(rows), dim3(G_PREP_I8_THREADS), 0, s, p.act, in, p.row_slot, p.top_k,
                            p.act_by_token, row_w, reinterpret_cast<uint8_t*>(buf.act_buf), buf.scale_buf,
-                           buf.zbuf) != cudaSuccess)
+                           buf.zbuf, p.status) != cudaSuccess)
                 return MOE_ERR_CUDA;
         } else {
             const int mode = nv ? 2 : (i4 ? 1 : 0);

@@ -19,8 +19,10 @@ constexpr int kMaxDecodeT = 64;
 // ---------------------------------------------------------------------------
 // Workspace layout.  Every region starts on a 256-byte boundary.
 // ctrl (1 KB): [0] status word, [1] router arrival counter, [2] quantiser
-//              amax (float bits), [3..15] reserved, [16..255] split-K tile
-//              arrival counters (left at zero by every call).
+//              amax (float bits), [3] reserved, [4..5] bound on every
+//              device wait in ns (uint64, 0 = the default of about 2 s),
+//              [6..15] reserved, [16..255] split-K tile arrival counters
+//              (left at zero by every call that completes).
 // ---------------------------------------------------------------------------
 struct WsLayout {
     size_t ctrl, logits, wsplit, hist, offsets, row_slot, slot_row, ids, tw;
@@ -208,6 +210,8 @@ int launch_quant_nvfp4(const __nv_bfloat16* w, int64_t rows, int64_t cols, uint8
 
 int launch_shared_routing(int T, int k, int32_t* sh_offsets, int32_t* sh_rowslot,
                           cudaStream_t s);
+// Writes one 64-bit word of device memory in stream order.
+int launch_set_u64(unsigned long long* dst, unsigned long long v, cudaStream_t s);
 
 // Activation operand of the tcgen05 grouped GEMM.  Unless act_ready, a
 // pre-pass gathers the problem's rows (row r reads activation row

@@ -189,6 +189,14 @@ __global__ void __launch_bounds__(256) router_topk(
 // last CTA is found with an arrival counter in the workspace (no waiting);
 // it leaves the counter at zero for the next call.
 // ---------------------------------------------------------------------------
+constexpr unsigned long long kRouterWaitNs = 2000000000ull;   // default bound of a wait
+// Bound on the fused router's wait: words 4-5 of the workspace control block
+// (moe_set_wait_limit), 0 = the default.  Read after griddepcontrol.wait.
+__device__ __forceinline__ unsigned long long router_wait_limit(const int32_t* status) {
+    if (!status) return kRouterWaitNs;
+    const unsigned long long v = *reinterpret_cast<const volatile unsigned long long*>(status + 4);
+    return v ? v : kRouterWaitNs;
+}
 constexpr int RD_WARPS = 8;          // 2 experts x 4 quarters of H per CTA
 constexpr int RD_EPC = 2;            // experts per CTA
 constexpr int RD_TMAX = 16;          // tokens (kRouterDecodeMaxT)
@@ -225,7 +233,8 @@ __global__ void __launch_bounds__(RD_WARPS * 32) router_decode(RouterDecodeArgs 
 #pragma unroll
     for (int q = 0; q < 8; q++)
         wv[q] = (q < nq) ? __ldg(reinterpret_cast<const float4*>(wq + q * 128 + lane * 4)) : make_float4(0, 0, 0, 0);
-    {   // activations landed (bounded wait)
+    {   // activations landed (bounded wait; the bound comes from the workspace control block)
+        const unsigned long long limit = router_wait_limit(a.status);
         uint32_t ok = 0;
         unsigned long long t_start, t_now;
         asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t_start));
@@ -233,7 +242,18 @@ __global__ void __launch_bounds__(RD_WARPS * 32) router_decode(RouterDecodeArgs 
             asm volatile("{ .reg .pred p; mbarrier.try_wait.parity.shared::cta.b64 p, [%1], 0; selp.u32 %0, 1, 0, p; }"
                          : "=r"(ok) : "r"(bar_a) : "memory");
             asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t_now));
-            if (!ok && t_now - t_start > 2000000000ull) { set_status(a.status, MOE_ERR_TIMEOUT); break; }
+            if (!ok && t_now - t_start > limit) {
+                set_status(a.status, MOE_ERR_TIMEOUT);
+                // the copy is still in flight: wait for it (at most the default bound) before this
+                // CTA's shared memory is read or released
+                while (!ok) {
+                    asm volatile("{ .reg .pred p; mbarrier.try_wait.parity.shared::cta.b64 p, [%1], 0; selp.u32 %0, 1, 0, p; }"
+                                 : "=r"(ok) : "r"(bar_a) : "memory");
+                    asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t_now));
+                    if (t_now - t_start > kRouterWaitNs) break;
+                }
+                break;
+            }
         }
     }
     float acc[RD_TMAX];

@@ -47,7 +47,7 @@ __global__ void __launch_bounds__(RT_THREADS, 1) router_tc(const __grid_constant
     extern __shared__ __align__(1024) uint8_t smem[];
     __shared__ __align__(8) uint64_t full[RT_STAGES], empty[RT_STAGES], acc_full[2], acc_empty[2], done;
     __shared__ uint32_t s_tmem;
-    __shared__ volatile int s_abort;
+    __shared__ volatile GAbort s_ab;
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int m0 = blockIdx.x * RT_M, n0 = blockIdx.y * RT_BN;
     const int KB = a.H / 64;
@@ -63,13 +63,15 @@ __global__ void __launch_bounds__(RT_THREADS, 1) router_tc(const __grid_constant
         }
         asm volatile("mbarrier.init.shared::cta.b64 [%0], 1;" ::"r"(g_smem(&done)));
         asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
-        s_abort = 0;
+        s_ab.flag = 0;
+        s_ab.limit_ns = G_WAIT_NS;
     }
     if (warp == 0) {
         asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], 128;" ::"r"(g_smem(&s_tmem)));
         asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;");
     }
     asm volatile("griddepcontrol.wait;" ::: "memory");
+    if (threadIdx.x == 0) s_ab.limit_ns = g_limit_from(a.status);
     g_fence_before();
     __syncthreads();
     g_fence_after();
@@ -77,15 +79,15 @@ __global__ void __launch_bounds__(RT_THREADS, 1) router_tc(const __grid_constant
     uint8_t* ring = smem + ((1024u - (g_smem(smem) & 1023u)) & 1023u);
     auto fail = [&]() {
         set_status(a.status, MOE_ERR_TIMEOUT);
-        s_abort = 1;
+        s_ab.flag = 1;
     };
 
     if (warp == 4) {
         // TMA producer: three weight planes (rows p*E + m0 ...) and 64 token rows per stage
         int kb = 0;
-        for (; kb < KB && !s_abort; kb++) {
+        for (; kb < KB && !g_aborted(&s_ab); kb++) {
             const int s = kb % RT_STAGES;
-            if (kb >= RT_STAGES && !g_wait_w(g_smem(&empty[s]), ((kb / RT_STAGES) - 1) & 1, &s_abort, 32)) {
+            if (kb >= RT_STAGES && !g_wait_w(g_smem(&empty[s]), ((kb / RT_STAGES) - 1) & 1, &s_ab, 32)) {
                 fail();
                 break;
             }
@@ -105,13 +107,13 @@ __global__ void __launch_bounds__(RT_THREADS, 1) router_tc(const __grid_constant
     } else if (warp == 5) {
         // MMA issuer: stage kb accumulates (from zero) into buffer kb & 1
         const uint32_t idesc = g_idesc(RT_BN, false, RT_M);
-        for (int kb = 0; kb < KB && !s_abort; kb++) {
+        for (int kb = 0; kb < KB && !g_aborted(&s_ab); kb++) {
             const int s = kb % RT_STAGES, b = kb & 1;
-            if (kb >= 2 && !g_wait_w(g_smem(&acc_empty[b]), ((kb >> 1) - 1) & 1, &s_abort)) {
+            if (kb >= 2 && !g_wait_w(g_smem(&acc_empty[b]), ((kb >> 1) - 1) & 1, &s_ab)) {
                 fail();
                 break;
             }
-            if (!g_wait_w(g_smem(&full[s]), (kb / RT_STAGES) & 1, &s_abort)) {
+            if (!g_wait_w(g_smem(&full[s]), (kb / RT_STAGES) & 1, &s_ab)) {
                 fail();
                 break;
             }
@@ -145,7 +147,7 @@ __global__ void __launch_bounds__(RT_THREADS, 1) router_tc(const __grid_constant
         bool ok = true;
         for (int kb = 0; kb < KB; kb++) {
             const int b = kb & 1;
-            if (!g_wait(g_smem(&acc_full[b]), (kb >> 1) & 1, &s_abort, 32)) {
+            if (!g_wait_w(g_smem(&acc_full[b]), (kb >> 1) & 1, &s_ab, 32)) {
                 ok = false;
                 break;
             }

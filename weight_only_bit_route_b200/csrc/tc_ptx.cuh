@@ -12,7 +12,23 @@
 
 namespace moe {
 
-constexpr unsigned long long G_WAIT_NS = 2000000000ull;   // bound on every device-side wait
+constexpr unsigned long long G_WAIT_NS = 2000000000ull;   // default bound on every device-side wait
+
+// Per-CTA abort state of the warp-specialised kernels: the flag a role sets
+// when one of its waits runs out (the other roles then stop issuing work),
+// and the bound on each wait, read from the workspace control block (words
+// 4-5, 0 = the default G_WAIT_NS; moe_set_wait_limit writes it).
+struct GAbort {
+    int flag;
+    unsigned long long limit_ns;
+};
+// The configured wait bound (status = the control block, may be null).  Read
+// it after griddepcontrol.wait: the word may come from the previous kernel.
+__device__ __forceinline__ unsigned long long g_limit_from(const int32_t* status) {
+    if (!status) return G_WAIT_NS;
+    const unsigned long long v = *reinterpret_cast<const volatile unsigned long long*>(status + 4);
+    return v ? v : G_WAIT_NS;
+}
 
 // ---------------------------------------------------------------------------
 // PTX helpers
@@ -29,24 +45,28 @@ __device__ __forceinline__ bool g_try(uint32_t bar, uint32_t parity) {
                  : "=r"(ok) : "r"(bar), "r"(parity) : "memory");
     return ok != 0;
 }
-// Bounded wait: false after about 2 s, or as soon as another role has aborted.
-// Roles off the critical path back off with a short sleep between polls so
-// that they leave issue slots to the dequantisation warps.
-__device__ __forceinline__ bool g_wait(uint32_t bar, uint32_t parity, volatile int* abort_flag, int sleep_ns = 0) {
+// Bounded wait: false once the configured bound has passed, or as soon as
+// another role has aborted.  Roles off the critical path back off with a
+// short sleep between polls so that they leave issue slots to the
+// dequantisation warps.
+__device__ __forceinline__ bool g_wait(uint32_t bar, uint32_t parity, volatile GAbort* ab, int sleep_ns = 0) {
     if (g_try(bar, parity)) return true;
     const unsigned long long t0 = g_timer();
     while (true) {
         if (sleep_ns) __nanosleep(sleep_ns);
         if (g_try(bar, parity)) return true;
-        if (*abort_flag || g_timer() - t0 > G_WAIT_NS) return false;
+        if (ab->flag || g_timer() - t0 > ab->limit_ns) return false;
     }
 }
 // Warp-wide bounded wait: every lane observes the phase (so whichever lane
-// is elected to issue has acquired it); the outcome is warp-uniform.
-__device__ __forceinline__ bool g_wait_w(uint32_t bar, uint32_t parity, volatile int* abort_flag, int sleep_ns = 0) {
-    const bool ok = g_wait(bar, parity, abort_flag, sleep_ns);
+// is elected to issue has acquired it); the outcome is warp-uniform, so the
+// warp stays converged for the .sync.aligned instructions that follow.
+__device__ __forceinline__ bool g_wait_w(uint32_t bar, uint32_t parity, volatile GAbort* ab, int sleep_ns = 0) {
+    const bool ok = g_wait(bar, parity, ab, sleep_ns);
     return __all_sync(0xffffffffu, ok);
 }
+// Warp-uniform test of the abort flag (loop conditions of whole-warp roles).
+__device__ __forceinline__ bool g_aborted(volatile GAbort* ab) { return __any_sync(0xffffffffu, ab->flag != 0); }
 // Bounded wait that ignores the abort flag (draining work already in flight).
 __device__ __forceinline__ void g_drain_wait(uint32_t bar, uint32_t parity) {
     const unsigned long long t0 = g_timer();

@@ -22,7 +22,7 @@ lib = ctypes.CDLL(LIB_PATH)
 
 FMT_INT4_G128, FMT_NVFP4, FMT_BF16 = 0, 1, 2
 STATUS = {0: "MOE_OK", -1: "MOE_ERR_INVALID_ARG", -2: "MOE_ERR_UNSUPPORTED", -3: "MOE_ERR_CUDA",
-          -4: "MOE_ERR_TIMEOUT", -5: "MOE_ERR_WORKSPACE", -6: "MOE_ERR_DEVICE_INDEX"}
+          -4: "MOE_ERR_TIMEOUT", -5: "MOE_ERR_WORKSPACE", -6: "MOE_ERR_DEVICE_INDEX", -7: "MOE_ERR_NONFINITE"}
 
 _P = ctypes.c_void_p
 _I = ctypes.c_int
@@ -54,6 +54,7 @@ def _sig(name, res, args):
 _sig("moe_workspace_bytes", _SZ, [_I, _I, _I, _I, _I])
 _sig("moe_workspace_init", _I, [_P, _SZ, _P])
 _sig("moe_read_status", _I, [_P, _P, ctypes.POINTER(ctypes.c_int32)])
+_sig("moe_set_wait_limit", _I, [_P, ctypes.c_uint64, _P])
 _sig("moe_status_string", ctypes.c_char_p, [_I])
 _sig("moe_launch_count", ctypes.c_uint64, [])
 _sig("moe_route_topk", _I, [_P, _I, _I, _P, _P, _I, _I, _P, _P, _P, _SZ, _P])
@@ -159,6 +160,11 @@ def read_status(ws):
     v = ctypes.c_int32(0)
     _check("moe_read_status", lib.moe_read_status(_ptr(ws), _stream(), ctypes.byref(v)))
     return int(v.value)
+
+
+def set_wait_limit(ws, limit_ns):
+    """Bound on each device wait of the kernels using this workspace (0 = default)."""
+    _check("moe_set_wait_limit", lib.moe_set_wait_limit(_ptr(ws), int(limit_ns), _stream()))
 
 
 def route_topk(x, router_w, router_bias, top_k, ws):
