@@ -61,6 +61,10 @@ def lib():
         L.oracle_grouped_down.restype = None
         L.oracle_combine.argtypes = [P, P, I64, I, I64, P, P]
         L.oracle_combine.restype = None
+        L.oracle_csf_encode.argtypes = [P, I64, I64, I64, P, P, P]
+        L.oracle_csf_encode.restype = I64
+        L.oracle_csf_decode.argtypes = [P, P, P, I64, I64, I64, P]
+        L.oracle_csf_decode.restype = None
         _lib = L
     return _lib
 
@@ -282,3 +286,25 @@ def combine(y_perm_bits, slot_row, T, k, shared_bits=None):
     sh = None if shared_bits is None else _c(shared_bits, np.uint16)
     lib().oracle_combine(_p(yp), _p(_c(slot_row, np.int32)), T, k, H, _p(sh), _p(y))
     return y
+
+
+def csf_encode(scales):
+    """E4M3 scale bytes uint8 [E, R, C] -> (fixed uint8 [E, R/16, 16*(1+C/2)],
+    exceptions uint32 [n], starts int64 [E+1]) in the compressed scale format."""
+    sc = _c(scales, np.uint8)
+    E, R, C = sc.shape
+    assert R % 16 == 0 and C % 2 == 0
+    fixed = np.empty((E, R // 16, 16 * (1 + C // 2)), np.uint8)
+    starts = np.empty(E + 1, np.int64)
+    n = lib().oracle_csf_encode(_p(sc), E, R, C, _p(fixed), _p(starts), None)
+    exc = np.empty(n, np.uint32)
+    lib().oracle_csf_encode(_p(sc), E, R, C, _p(fixed), _p(starts), _p(exc))
+    return fixed, exc, starts
+
+
+def csf_decode(fixed, exceptions, starts, R, C):
+    fixed = _c(fixed, np.uint8)
+    E = fixed.shape[0]
+    out = np.empty((E, R, C), np.uint8)
+    lib().oracle_csf_decode(_p(fixed), _p(_c(exceptions, np.uint32)), _p(_c(starts, np.int64)), E, R, C, _p(out))
+    return out

@@ -20,6 +20,11 @@
  *   [Art]   "Step 5 Preview: 92 narrow layers, and a sparse indexer that scores
  *           blocks of 8": The shape (8 routed experts per token plus one shared
  *           expert, each a SwiGLU of width 1536).
+ *   [CSF]   "Step-5-Preview-NVFP4-Local", Format (the compressed scale format:
+ *           per 16-row slab 16 row bases then 4-bit codes, low nibble first;
+ *           exceptions (row*C + col) | byte << 24 grouped by expert, row-major;
+ *           starts [E+1]; a row's base is the lowest value whose 16-value
+ *           window covers the most of its bytes, 0..240) and Size.
  *
  * Readings where the pages are silent (each listed in the design notes):
  *   - int4: divisor 7 with clamp [-8, 7]; ratios r_i = (24 + i) / 40, i = 0..16;
@@ -34,6 +39,9 @@
  *     (fp32); top-k by s, ties to the lower expert id, listed by descending s;
  *     weights s / sum(selected s) (fp32).
  *   - Layer: no routed scaling factor, no shared-expert gate, SwiGLU limit off.
+ *   - CSF: the 4-bit code stored at an exception's position is 0 (the
+ *     decoder replaces that byte, so any code would do; 0 is the plainest);
+ *     the rows of a slab follow one another, each C/2 bytes.
  *
  * Floating point: quantiser decisions are taken in fp32 (the precision the
  * CUDA library's own quantiser uses, so codes agree bit for bit); dequantised
@@ -566,4 +574,86 @@ void oracle_combine(const uint16_t* y_perm, const int32_t* slot_row, int64_t T, 
             }
             y[t * H + hh] = acc;
         }
+}
+
+
+/* ------------------------------------------------------------------------ */
+/* Compressed scale format (CSF)  [CSF] Format                               */
+/* ------------------------------------------------------------------------ */
+
+/* Base of one row of n scale bytes: the lowest b in 0..240 whose window
+ * [b, b + 15] holds the most of the row's bytes. */
+static int csf_row_base(const uint8_t* row, int64_t n) {
+    int64_t hist[256];
+    memset(hist, 0, sizeof(hist));
+    for (int64_t i = 0; i < n; i++) hist[row[i]]++;
+    int best = 0;
+    int64_t best_cnt = -1;
+    for (int b = 0; b <= 240; b++) {
+        int64_t cnt = 0;
+        for (int v = b; v < b + 16; v++) cnt += hist[v];
+        if (cnt > best_cnt) { best_cnt = cnt; best = b; }      /* strict: the lowest base wins ties */
+    }
+    return best;
+}
+
+/* Encode scales u8 [E, R, C] (R % 16 == 0, C even).
+ * fixed: u8 [E, R/16, 16 * (1 + C/2)]: per slab of 16 rows, the 16 row bases,
+ *        then the rows' codes in row order, C/2 bytes each, column 2j in the
+ *        low nibble of byte j and column 2j + 1 in its high nibble;
+ * starts: int64 [E + 1], expert e owns exceptions[starts[e] .. starts[e+1]);
+ * exceptions: uint32 [n] (may be NULL to count only), (row * C + col) | byte << 24
+ *        for every byte outside its row's window, in (expert, row, col) order.
+ * Returns n, the number of exceptions. */
+int64_t oracle_csf_encode(const uint8_t* scales, int64_t E, int64_t R, int64_t C,
+                          uint8_t* fixed, int64_t* starts, uint32_t* exceptions) {
+    int64_t slab = 16 * (1 + C / 2);
+    int64_t n = 0;
+    for (int64_t e = 0; e < E; e++) {
+        starts[e] = n;
+        for (int64_t r = 0; r < R; r++) {
+            const uint8_t* row = scales + (e * R + r) * C;
+            int base = csf_row_base(row, C);
+            uint8_t* sl = fixed + (e * (R / 16) + r / 16) * slab;
+            sl[r % 16] = (uint8_t)base;
+            uint8_t* codes = sl + 16 + (r % 16) * (C / 2);
+            for (int64_t j = 0; j < C / 2; j++) codes[j] = 0;
+            for (int64_t c = 0; c < C; c++) {
+                int v = row[c];
+                int code = 0;
+                if (v >= base && v <= base + 15) {
+                    code = v - base;
+                } else {
+                    if (exceptions) exceptions[n] = (uint32_t)(r * C + c) | ((uint32_t)v << 24);
+                    n++;
+                }
+                codes[c / 2] |= (uint8_t)(code << (4 * (c % 2)));
+            }
+        }
+    }
+    starts[E] = n;
+    return n;
+}
+
+/* Decode back to scales u8 [E, R, C]: base + code, then each exception of
+ * expert e replaces the byte at its position. */
+void oracle_csf_decode(const uint8_t* fixed, const uint32_t* exceptions, const int64_t* starts,
+                       int64_t E, int64_t R, int64_t C, uint8_t* scales) {
+    int64_t slab = 16 * (1 + C / 2);
+    for (int64_t e = 0; e < E; e++) {
+        for (int64_t r = 0; r < R; r++) {
+            const uint8_t* sl = fixed + (e * (R / 16) + r / 16) * slab;
+            int base = sl[r % 16];
+            const uint8_t* codes = sl + 16 + (r % 16) * (C / 2);
+            for (int64_t c = 0; c < C; c++) {
+                int code = (codes[c / 2] >> (4 * (c % 2))) & 0xF;
+                scales[(e * R + r) * C + c] = (uint8_t)(base + code);
+            }
+        }
+        for (int64_t i = starts[e]; i < starts[e + 1]; i++) {
+            uint32_t x = exceptions[i];
+            int64_t pos = (int64_t)(x & 0xFFFFFFu);
+            scales[e * R * C + pos] = (uint8_t)(x >> 24);
+        }
+    }
 }
