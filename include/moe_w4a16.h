@@ -127,9 +127,20 @@ int moe_read_status(void* ws, moe_stream_t stream, int32_t* status_out);
  * that runs out records MOE_ERR_TIMEOUT, the kernel stops issuing work,
  * waits (bounded by the default) for the copies and MMAs it has in flight,
  * releases its tensor memory and returns; its outputs are then undefined.
- * For failure testing: a bound shorter than the kernels' normal waits makes
- * every call time out.  The pages have no counterpart to this call. */
+ * A wait polls with mbarrier try_wait, which may itself suspend until the
+ * barrier completes, so a wait that the hardware completes within that
+ * suspension never times out, however short the bound.  The pages have no
+ * counterpart to this call. */
 int moe_set_wait_limit(void* ws, uint64_t limit_ns, moe_stream_t stream);
+
+/* Failure testing: while `hold` is non-zero (word 6 of the control block,
+ * stream-ordered), the MMA warp of every tensor-core GEMM launched with this
+ * workspace first waits on a barrier that nothing completes, so that wait
+ * runs out after the configured bound (moe_set_wait_limit) with the kernel's
+ * copies in flight, and the kernel takes its abort path (MOE_ERR_TIMEOUT,
+ * drain, return).  No other call is affected.  hold = 0 ends it.  The pages
+ * have no counterpart to this call. */
+int moe_set_wait_hold(void* ws, int hold, moe_stream_t stream);
 
 /* Static description of a status code. */
 const char* moe_status_string(int status);
@@ -296,6 +307,50 @@ int moe_quantize_int4_g128(const void* w, int64_t rows, int64_t cols, int32_t* p
 int moe_quantize_nvfp4(const void* w, int64_t rows, int64_t cols, uint8_t* packed,
                        uint8_t* scales, float* global_scale, void* ws, size_t ws_bytes,
                        moe_stream_t stream);
+
+/* ---------------------------------------------------------------------- */
+/* Compressed scale format of the NVFP4 block scales                       */
+/* ---------------------------------------------------------------------- */
+
+/* CSF ("Step-5-Preview-NVFP4-Local", Format): a scale tensor u8 [E, R, C]
+ * (one E4M3 byte per 16 weights; gate/up R = 1536, C = 256, down R = 4096,
+ * C = 96) is stored as
+ *   fixed       u8 [E, R/16, 16 * (1 + C/2)]: per slab of 16 rows the 16 row
+ *               bases, then each row's 4-bit codes (C/2 bytes per row, in row
+ *               order; column 2j in the low nibble of byte j);
+ *   exceptions  u32 [n]: (row * C + col) | byte << 24, grouped by expert and
+ *               row-major within an expert (row counts from 0 in each expert);
+ *   starts      i64 [E + 1]: expert e owns exceptions[starts[e], starts[e+1]).
+ * A byte is its row's base plus its code unless an exception replaces it.  A
+ * row's base is the lowest value 0..240 whose window [base, base + 15] holds
+ * the most of the row's bytes; the code at an exception's position is 0.
+ * Requirements: R % 16 == 0, C even, R * C < 2^24, 1 <= E <= 1024. */
+
+/* Expand CSF planes into scale bytes u8 [E, R, C] (scales, out), e.g. one
+ * layer's scales into scratch before the layer runs ("The b12x loader ...
+ * expands one MoE layer's scales into shared scratch", Size).  expert_offsets:
+ * int32 [E+1] of a routing (moe_permute), or NULL; when given, only experts
+ * with at least one routed row are expanded and the other experts' bytes are
+ * left as they were.  exceptions and starts are both given or both NULL (no
+ * exceptions); an exception whose position is R * C or more is ignored.
+ * Two kernels (expansion, then the exceptions), stream-ordered. */
+int moe_csf_decode(const uint8_t* fixed, const uint32_t* exceptions, const int64_t* starts,
+                   int E, int R, int C, const int32_t* expert_offsets, uint8_t* scales,
+                   moe_stream_t stream);
+
+/* Workspace bytes moe_csf_encode needs for E experts of R rows (0 if invalid). */
+size_t moe_csf_encode_workspace_bytes(int E, int R);
+
+/* Encode scale bytes u8 [E, R, C] into CSF (offline step).  Always writes
+ * fixed and starts (device memory); with exceptions non-NULL it also writes
+ * the exceptions, at most exceptions_capacity of them (a larger count records
+ * MOE_ERR_DEVICE_INDEX in the workspace status word).  To size the
+ * exceptions, call once with exceptions = NULL and read starts[E].
+ * ws: moe_csf_encode_workspace_bytes(E, R) bytes, 256-byte aligned, its first
+ * 1024 bytes zero-filled (moe_workspace_init). */
+int moe_csf_encode(const uint8_t* scales, int E, int R, int C, uint8_t* fixed, int64_t* starts,
+                   uint32_t* exceptions, int64_t exceptions_capacity, void* ws, size_t ws_bytes,
+                   moe_stream_t stream);
 
 #ifdef __cplusplus
 }

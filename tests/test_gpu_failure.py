@@ -1,11 +1,11 @@
 """Failure handling on the GPU, without faulting it.
 
-1. Bounded waits: with the workspace's wait bound set to 1 ns, every wait of
-   the tensor-core kernels and the fused router that does not succeed at once
-   runs out.  The call must record MOE_ERR_TIMEOUT, the kernels must stop,
-   drain what they have in flight and return (the context stays usable), and
-   after the default bound is restored the same workspace must give the
-   oracle's result.
+1. Bounded waits: with the workspace's hold set, the MMA warp of each
+   tensor-core GEMM waits on a barrier nothing completes; with the wait bound
+   at 1 ms that wait runs out.  The call must record MOE_ERR_TIMEOUT, the
+   kernels must stop, drain the copies they have in flight and return (the
+   context stays usable), and once the hold and the bound are cleared the same
+   workspace must give the oracle's result.
 2. A non-finite activation row on the 8-bit int4 path records
    MOE_ERR_NONFINITE and yields NaN for that token's rows only.
 """
@@ -37,10 +37,12 @@ def test_wait_limit_runs_out_then_recovers():
     L = device_layer(moe, P)
     ws = moe.workspace(P.T, wl.H, wl.E, wl.F, wl.k)
     x = dev_bf16(P.x)
-    moe.set_wait_limit(ws, 1)
+    moe.set_wait_limit(ws, 1_000_000)             # 1 ms
+    moe.set_wait_hold(ws, 1)
     moe.layer_decode(x, L, ws)
     torch.cuda.synchronize()                       # the kernels returned
     assert moe.read_status(ws) == MOE_ERR_TIMEOUT
+    moe.set_wait_hold(ws, 0)
     moe.set_wait_limit(ws, 0)
     for _ in range(2):                             # the workspace serves later calls
         y = moe.layer_decode(x, L, ws)

@@ -289,6 +289,11 @@ int moe_set_wait_limit(void* ws, uint64_t limit_ns, moe_stream_t stream) {
     return launch_set_u64(at<unsigned long long>(ws, 16), limit_ns, cs(stream));
 }
 
+int moe_set_wait_hold(void* ws, int hold, moe_stream_t stream) {
+    if (!ws || (reinterpret_cast<uintptr_t>(ws) & 255u)) return MOE_ERR_WORKSPACE;
+    return launch_set_u32(at<uint32_t>(ws, 24), hold ? 1u : 0u, cs(stream));
+}
+
 uint64_t moe_launch_count(void) { return moe::g_launches.load(std::memory_order_relaxed); }
 
 const char* moe_status_string(int status) {
@@ -426,6 +431,32 @@ int moe_layer_forward(const void* x, int T, const moe_layer* L, void* y, void* w
     MOE_TRY(layer_checks(x, T, L, y, ws, ws_bytes));
     if (T == 0) return MOE_OK;
     return layer_run(x, T, L, y, ws, cs(stream));
+}
+
+int moe_csf_decode(const uint8_t* fixed, const uint32_t* exceptions, const int64_t* starts, int E, int R, int C,
+                   const int32_t* expert_offsets, uint8_t* scales, moe_stream_t stream) {
+    if (E <= 0 || R <= 0 || C <= 0) return MOE_ERR_INVALID_ARG;
+    if (E > kMaxE || R % 16 || C % 2 || int64_t(R) * C >= (int64_t(1) << 24)) return MOE_ERR_UNSUPPORTED;
+    if (!fixed || !scales || (!exceptions) != (!starts)) return MOE_ERR_INVALID_ARG;
+    return launch_csf_decode(fixed, exceptions, starts, E, R, C, expert_offsets, scales, cs(stream));
+}
+
+size_t moe_csf_encode_workspace_bytes(int E, int R) {
+    if (E <= 0 || R <= 0 || E > kMaxE) return 0;
+    return kStepScratch + csf_encode_scratch(E, R);
+}
+
+int moe_csf_encode(const uint8_t* scales, int E, int R, int C, uint8_t* fixed, int64_t* starts,
+                   uint32_t* exceptions, int64_t exceptions_capacity, void* ws, size_t ws_bytes,
+                   moe_stream_t stream) {
+    if (E <= 0 || R <= 0 || C <= 0 || exceptions_capacity < 0) return MOE_ERR_INVALID_ARG;
+    if (E > kMaxE || R % 16 || C % 2 || int64_t(R) * C >= (int64_t(1) << 24)) return MOE_ERR_UNSUPPORTED;
+    if (!scales || !fixed || !starts) return MOE_ERR_INVALID_ARG;
+    MOE_TRY(check_ws(ws, ws_bytes, kStepScratch + csf_encode_scratch(E, R)));
+    int32_t* rowcnt = at<int32_t>(ws, kStepScratch);
+    int64_t* tot = at<int64_t>(ws, kStepScratch + align256(size_t(E) * R * 4));
+    return launch_csf_encode(scales, E, R, C, fixed, starts, exceptions, exceptions_capacity, rowcnt, tot,
+                             at<int32_t>(ws, 0), cs(stream));
 }
 
 int moe_quantize_int4_g128(const void* w, int64_t rows, int64_t cols, int32_t* packed, void* scales,

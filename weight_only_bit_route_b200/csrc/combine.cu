@@ -78,4 +78,13 @@ int launch_set_u64(unsigned long long* dst, unsigned long long v, cudaStream_t s
     return cudaGetLastError() == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
 }
 
+// One 32-bit word of the workspace control block (moe_set_wait_hold).
+__global__ void set_u32_kernel(uint32_t* dst, uint32_t v) { *dst = v; }
+
+int launch_set_u32(uint32_t* dst, uint32_t v, cudaStream_t s) {
+    set_u32_kernel<<<1, 1, 0, s>>>(dst, v);
+    count_launch();
+    return cudaGetLastError() == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
+}
+
 }  // namespace moe

@@ -240,6 +240,8 @@ __global__ void __launch_bounds__(G_THREADS, 1) tc_grouped_gemm(const __grid_con
     __shared__ __align__(8) uint64_t b_full[C::kBStages], a_full[C::kAStages], done[G_DONE];
     __shared__ __align__(8) uint64_t sc_full[G_SC_MAX], sc_empty[G_SC_MAX];
     __shared__ __align__(8) uint64_t acc_full[2], acc_empty[C::kAccBufs], drain;
+    __shared__ __align__(8) uint64_t hold_bar;        // failure testing: a barrier nothing completes
+    __shared__ int s_hold;
     __shared__ uint32_t s_tmem;
     __shared__ int s_active[kMaxE];
     __shared__ int s_prefix[kMaxE];
@@ -284,6 +286,7 @@ __global__ void __launch_bounds__(G_THREADS, 1) tc_grouped_gemm(const __grid_con
         for (int s = 0; s < C::kAccBufs; s++)
             asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(g_smem(&acc_empty[s])), "r"(G_EPI_WARPS));
         asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(g_smem(&drain)), "r"(C::kI8 ? 2 : 1));
+        asm volatile("mbarrier.init.shared::cta.b64 [%0], 1;" ::"r"(g_smem(&hold_bar)));
         asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
         s_ab.flag = 0;
         s_ab.limit_ns = G_WAIT_NS;
@@ -293,7 +296,10 @@ __global__ void __launch_bounds__(G_THREADS, 1) tc_grouped_gemm(const __grid_con
         asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;");
     }
     asm volatile("griddepcontrol.wait;" ::: "memory");
-    if (tid == 0) s_ab.limit_ns = g_limit_from(a.status);   // published by the __syncthreads below
+    if (tid == 0) {                                   // published by the __syncthreads below
+        s_ab.limit_ns = g_limit_from(a.status);
+        s_hold = g_hold_from(a.status);
+    }
 
     // tile list: active experts and the prefix sum of their tile counts
     {
@@ -494,6 +500,9 @@ __global__ void __launch_bounds__(G_THREADS, 1) tc_grouped_gemm(const __grid_con
         // cannot keep up with the weight stream (each step costs it about a
         // thousand cycles of serial work around eight or sixteen MMAs).
         const uint32_t n_iss = C::kI8 ? 2u : 1u, iss = uint32_t(warp - 2);
+        // failure testing (moe_set_wait_hold): wait for a barrier that nothing completes, so the
+        // bound runs out while the producers have copies in flight and the kernel takes its abort path
+        if (s_hold && !g_wait_w(g_smem(&hold_bar), 0, &s_ab)) fail();
         uint32_t bc = 0, ac = 0, pc = 0;
         int t = 0;
         for (int tile = blockIdx.x; tile < ntiles && !g_aborted(&s_ab); tile += gridDim.x, t++) {

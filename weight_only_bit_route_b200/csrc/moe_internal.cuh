@@ -21,8 +21,10 @@ constexpr int kMaxDecodeT = 64;
 // ctrl (1 KB): [0] status word, [1] router arrival counter, [2] quantiser
 //              amax (float bits), [3] reserved, [4..5] bound on every
 //              device wait in ns (uint64, 0 = the default of about 2 s),
-//              [6..15] reserved, [16..255] split-K tile arrival counters
-//              (left at zero by every call that completes).
+//              [6] failure-testing hold (non-zero: each tensor-core GEMM
+//              first waits on a barrier nothing completes), [7..15]
+//              reserved, [16..255] split-K tile arrival counters (left at
+//              zero by every call that completes).
 // ---------------------------------------------------------------------------
 struct WsLayout {
     size_t ctrl, logits, wsplit, hist, offsets, row_slot, slot_row, ids, tw;
@@ -210,8 +212,17 @@ int launch_quant_nvfp4(const __nv_bfloat16* w, int64_t rows, int64_t cols, uint8
 
 int launch_shared_routing(int T, int k, int32_t* sh_offsets, int32_t* sh_rowslot,
                           cudaStream_t s);
+// Compressed scale format (csf.cu).
+int launch_csf_decode(const uint8_t* fixed, const uint32_t* exc, const int64_t* starts, int E, int R, int C,
+                      const int32_t* offsets, uint8_t* out, cudaStream_t s);
+int launch_csf_encode(const uint8_t* sc, int E, int R, int C, uint8_t* fixed, int64_t* starts, uint32_t* exc,
+                      int64_t capacity, int32_t* rowcnt, int64_t* tot, int32_t* status, cudaStream_t s);
+inline size_t csf_encode_scratch(int E, int R) { return align256(size_t(E) * R * 4) + align256(size_t(E) * 8); }
+
 // Writes one 64-bit word of device memory in stream order.
 int launch_set_u64(unsigned long long* dst, unsigned long long v, cudaStream_t s);
+// Writes one 32-bit word of device memory in stream order.
+int launch_set_u32(uint32_t* dst, uint32_t v, cudaStream_t s);
 
 // Activation operand of the tcgen05 grouped GEMM.  Unless act_ready, a
 // pre-pass gathers the problem's rows (row r reads activation row

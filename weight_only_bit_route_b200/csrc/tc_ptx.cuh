@@ -30,6 +30,11 @@ __device__ __forceinline__ unsigned long long g_limit_from(const int32_t* status
     return v ? v : G_WAIT_NS;
 }
 
+// Failure-testing hold: word 6 of the control block (moe_set_wait_hold).
+__device__ __forceinline__ int g_hold_from(const int32_t* status) {
+    return status ? *reinterpret_cast<const volatile int32_t*>(status + 6) : 0;
+}
+
 // ---------------------------------------------------------------------------
 // PTX helpers
 // ---------------------------------------------------------------------------

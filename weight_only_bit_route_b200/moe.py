@@ -55,6 +55,7 @@ _sig("moe_workspace_bytes", _SZ, [_I, _I, _I, _I, _I])
 _sig("moe_workspace_init", _I, [_P, _SZ, _P])
 _sig("moe_read_status", _I, [_P, _P, ctypes.POINTER(ctypes.c_int32)])
 _sig("moe_set_wait_limit", _I, [_P, ctypes.c_uint64, _P])
+_sig("moe_set_wait_hold", _I, [_P, _I, _P])
 _sig("moe_status_string", ctypes.c_char_p, [_I])
 _sig("moe_launch_count", ctypes.c_uint64, [])
 _sig("moe_route_topk", _I, [_P, _I, _I, _P, _P, _I, _I, _P, _P, _P, _SZ, _P])
@@ -67,6 +68,9 @@ _sig("moe_layer_decode", _I, [_P, _I, _P, _P, _P, _SZ, _P])
 _sig("moe_layer_forward", _I, [_P, _I, _P, _P, _P, _SZ, _P])
 _sig("moe_quantize_int4_g128", _I, [_P, _I64, _I64, _P, _P, _P])
 _sig("moe_quantize_nvfp4", _I, [_P, _I64, _I64, _P, _P, _P, _P, _SZ, _P])
+_sig("moe_csf_decode", _I, [_P, _P, _P, _I, _I, _I, _P, _P, _P])
+_sig("moe_csf_encode_workspace_bytes", _SZ, [_I, _I])
+_sig("moe_csf_encode", _I, [_P, _I, _I, _I, _P, _P, _P, _I64, _P, _SZ, _P])
 
 
 def declared_functions():
@@ -167,6 +171,11 @@ def set_wait_limit(ws, limit_ns):
     _check("moe_set_wait_limit", lib.moe_set_wait_limit(_ptr(ws), int(limit_ns), _stream()))
 
 
+def set_wait_hold(ws, hold):
+    """Failure testing: the tensor-core GEMMs using this workspace first wait on a barrier nothing completes."""
+    _check("moe_set_wait_hold", lib.moe_set_wait_hold(_ptr(ws), int(bool(hold)), _stream()))
+
+
 def route_topk(x, router_w, router_bias, top_k, ws):
     T, H = x.shape
     E = router_w.shape[0]
@@ -264,3 +273,35 @@ def quantize_nvfp4(w, ws, global_out=None):
            lib.moe_quantize_nvfp4(_ptr(w), rows, cols, _ptr(packed), _ptr(scales), _ptr(g), _ptr(ws),
                                   ws.numel(), _stream()))
     return packed, scales, g
+
+
+def csf_encode(scales):
+    """Scale bytes uint8 [E, R, C] (device) -> CSF planes (fixed uint8
+    [E, R/16, 16*(1+C/2)], exceptions uint32 [n] as int32 storage, starts int64 [E+1])."""
+    E, R, C = scales.shape
+    n = int(lib.moe_csf_encode_workspace_bytes(E, R))
+    if n == 0:
+        raise MoEError("moe_csf_encode_workspace_bytes", -2)
+    ws = torch.empty(n, dtype=torch.uint8, device=scales.device)
+    _check("moe_workspace_init", lib.moe_workspace_init(_ptr(ws), n, _stream()))
+    fixed = torch.empty(E, R // 16, 16 * (1 + C // 2), dtype=torch.uint8, device=scales.device)
+    starts = torch.empty(E + 1, dtype=torch.int64, device=scales.device)
+    _check("moe_csf_encode", lib.moe_csf_encode(_ptr(scales), E, R, C, _ptr(fixed), _ptr(starts), None, 0,
+                                                _ptr(ws), n, _stream()))
+    count = int(starts[E].item())
+    exc = torch.empty(max(count, 1), dtype=torch.int32, device=scales.device)
+    _check("moe_csf_encode", lib.moe_csf_encode(_ptr(scales), E, R, C, _ptr(fixed), _ptr(starts), _ptr(exc), count,
+                                                _ptr(ws), n, _stream()))
+    st = read_status(ws)
+    if st != 0:
+        raise MoEError("moe_csf_encode (device)", st)
+    return fixed, exc[:count], starts
+
+
+def csf_decode(fixed, exceptions, starts, R, C, expert_offsets=None, out=None):
+    E = fixed.shape[0]
+    sc = out if out is not None else torch.empty(E, R, C, dtype=torch.uint8, device=fixed.device)
+    exc = exceptions if exceptions.numel() else torch.zeros(1, dtype=torch.int32, device=fixed.device)
+    _check("moe_csf_decode", lib.moe_csf_decode(_ptr(fixed), _ptr(exc), _ptr(starts), E, R, C, _ptr(expert_offsets),
+                                                _ptr(sc), _stream()))
+    return sc
