@@ -78,7 +78,6 @@ GemmBuffers gemm_buffers(void* base, int rows, int in_dim, bool act_ready, bool 
     b.zbuf = reinterpret_cast<float*>(p + align256(size_t(rows) * 4));
     b.act_buf = p + align256(size_t(rows) * 4) + align256(size_t(rows) * zsum_stride(in_dim) * 4);
     b.act_ready = act_ready;
-    b.perm_out = 0;
     b.i8 = i8;
     return b;
 }
@@ -207,7 +206,6 @@ int layer_run(const void* x, int T, const moe_layer* L, void* y, void* ws, cudaS
         MOE_TRY(launch_permute(ids, T, k, E, offsets, row_slot, slot_row, at<int32_t>(ws, W.hist), status, s));
     }
     const bool routed_gemm = gemm_shape_ok(H, F) && gemm_shape_ok(F, H);
-    const bool int4 = L->gate.fmt == MOE_FMT_INT4_G128;
 
     GemvProblem gu{};
     gu.act = xb; gu.act_by_token = 1; gu.top_k = k; gu.offsets = offsets; gu.row_slot = row_slot;
@@ -220,22 +218,19 @@ int layer_run(const void* x, int T, const moe_layer* L, void* y, void* ws, cudaS
     dn.E = E; dn.topk_w = tw; dn.fmt = L->down.fmt; dn.out_dim = H; dn.in_dim = F;
     dn.p0 = L->down.packed; dn.s0 = L->down.scales; dn.g0 = L->down.global_scale;
     dn.out = y_perm; dn.status = status;
-    // routed experts: both projections on one path (the int4 GEMM hands h to
-    // the down GEMM in its pair order)
+    // routed experts: both projections on one path
     const bool i8 = routed_gemm && i8_int4(gu, R);
     if (routed_gemm) {
         // 16-bit gate/up activation rows are gathered into the y_perm region,
         // free until the down projection writes it
         GemmBuffers gb = gemm_buffers(prep, R, H, false, i8);
         if (!i8) gb.act_buf = y_perm;
-        gb.perm_out = int4 && !i8;
         MOE_TRY(launch_grouped_gemm(gu, true, R, gb, s));
     } else {
         MOE_TRY(launch_stream_gemv(gu, nullptr, true, T, prep, s, true));
     }
     if (routed_gemm) {
-        // int4 h is already in the pair order unless the 8-bit path made it
-        GemmBuffers db = gemm_buffers(prep, R, F, int4 && !i8, i8);
+        GemmBuffers db = gemm_buffers(prep, R, F, false, i8);
         MOE_TRY(launch_grouped_gemm(dn, false, R, db, s));
     } else {
         MOE_TRY(launch_stream_gemv(dn, nullptr, false, R, prep, s, true));

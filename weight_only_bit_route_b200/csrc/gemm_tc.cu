@@ -136,7 +136,7 @@ struct GCfg {
     static constexpr int kAPerPk = kPkK / kSK;                      // A stages per weight stage (2, or 1 for i8)
     static constexpr int kChunkCols = 16;                           // 16-bit paths: TMEM columns of one packed chunk
     static constexpr int kDqArrivals = kI8 ? G_DQ_WARPS / 2 : G_DQ_WARPS;  // warps that fill one stage
-    static constexpr bool kMmaF16 = FMT == MOE_FMT_NVFP4;
+    static constexpr bool kMmaF16 = FMT == MOE_FMT_NVFP4 || FMT == MOE_FMT_INT4_G128;   // f16 operands
 };
 
 constexpr int G_DONE = 16;                                          // "stage done" barrier ring
@@ -162,7 +162,7 @@ struct GArgs {
     float* partial;                  // split-K: fp32 partial sums [ksplit][nmat][rows][out_dim]
     const float* zsum;               // 8-bit int4: 8 * sum of the row's fixed-point values per group [rows][zst]
     const uint8_t* bdig;             // 8-bit int4: the digit rows [3 rows][in]
-    int E, out_dim, in_dim, perm_out;
+    int E, out_dim, in_dim;
     int ksplit, rows;                // K slices per (m-tile, n-tile); activation rows of the problem
     int* tile_cnt;                   // split-K: zeroed arrival counters, four per (m-tile, n-tile); the last
                                      // epilogue warp of each quarter sums the slices (else a kernel does)
@@ -175,21 +175,47 @@ struct GArgs {
 // bf16/f16 pairs.  int4: pair order within each 8, sc = bf16 scale bits.
 // NVFP4: natural order, sc = two E4M3 bytes (K 0-15, K 16-31 of the chunk).
 // ---------------------------------------------------------------------------
-__device__ __forceinline__ void g_dq_int4(const uint4 w, uint32_t sc, uint32_t (&o)[16]) {
-    const __nv_bfloat162 s2 = __bfloat162bfloat162(__ushort_as_bfloat16(static_cast<unsigned short>(sc)));
-    const __nv_bfloat162 off = __floats2bfloat162_rn(136.f, 136.f);
+__device__ __forceinline__ void g_dq_int4(const uint4 w, uint32_t s2, uint32_t s16, uint32_t (&o)[16]) {
+    // s2 = {s', s'} and s16 = {s'/16, s'/16} in f16, s' = the group scale times the row's power of
+    // two.  A mask puts nibbles (p, p+4) of a word into the mantissas of 1024.0 (p even, values
+    // 1024 + u) or of 1024.0 with the nibble four bits up (p odd, 1024 + 16 u): subtracting 1032 or
+    // 1152 gives q or 16 q exactly, and one multiply by s' or s'/16 gives q s' exactly (at most
+    // 11 significant bits, in f16's normal range by the choice of the row's power of two).
+    const __half2 hs = *reinterpret_cast<const __half2*>(&s2);
+    const __half2 hs16 = *reinterpret_cast<const __half2*>(&s16);
+    const __half2 off0 = __floats2half2_rn(1032.f, 1032.f), off1 = __floats2half2_rn(1152.f, 1152.f);
     const uint32_t ws[4] = {w.x, w.y, w.z, w.w};
 #pragma unroll
     for (int j = 0; j < 4; j++) {
-#pragma unroll
-        for (int p = 0; p < 4; p++) {
-            // nibbles (p, p+4) -> bf16 {128+u}; minus 136 gives q exactly; times s rounds once
-            uint32_t v = ((ws[j] >> (4 * p)) & 0x000F000Fu) | 0x43004300u;
-            __nv_bfloat162 h = *reinterpret_cast<__nv_bfloat162*>(&v);
-            h = __hmul2(__hsub2(h, off), s2);
-            o[j * 4 + p] = *reinterpret_cast<uint32_t*>(&h);
-        }
+        const uint32_t t = ws[j] >> 8;
+        uint32_t v0 = (ws[j] & 0x000F000Fu) | 0x64006400u;      // nibbles 0, 4
+        uint32_t v1 = (ws[j] & 0x00F000F0u) | 0x64006400u;      // nibbles 1, 5 (x 16)
+        uint32_t v2 = (t & 0x000F000Fu) | 0x64006400u;          // nibbles 2, 6
+        uint32_t v3 = (t & 0x00F000F0u) | 0x64006400u;          // nibbles 3, 7 (x 16)
+        __half2 h0 = __hmul2(__hsub2(*reinterpret_cast<__half2*>(&v0), off0), hs);
+        __half2 h1 = __hmul2(__hsub2(*reinterpret_cast<__half2*>(&v1), off1), hs16);
+        __half2 h2 = __hmul2(__hsub2(*reinterpret_cast<__half2*>(&v2), off0), hs);
+        __half2 h3 = __hmul2(__hsub2(*reinterpret_cast<__half2*>(&v3), off1), hs16);
+        o[j * 4 + 0] = *reinterpret_cast<uint32_t*>(&h0);
+        o[j * 4 + 1] = *reinterpret_cast<uint32_t*>(&h1);
+        o[j * 4 + 2] = *reinterpret_cast<uint32_t*>(&h2);
+        o[j * 4 + 3] = *reinterpret_cast<uint32_t*>(&h3);
     }
+}
+// The power of two k that puts a row's largest int4 group scale m in [2^11, 2^12): then every
+// q s 2^k (|q| <= 8) stays below 2^15 and is exact in f16 down to scales 2^25 below m.
+__device__ __forceinline__ int g_int4_row_shift(float m) {
+    if (!(m > 0.f)) return 0;
+    int e = 0;
+    frexpf(m, &e);                                       // m = f 2^e, f in [0.5, 1)
+    return min(60, max(-24, 12 - e));
+}
+// the f16 pair {s 2^k, s 2^k} and {s 2^k / 16, ...} of a bf16 group scale
+__device__ __forceinline__ void g_int4_scale_pair(uint32_t sbf16, float fk, uint32_t& s2, uint32_t& s16) {
+    const float sv = __uint_as_float(sbf16 << 16) * fk;
+    __half2 a = __float2half2_rn(sv), b = __float2half2_rn(sv * 0.0625f);
+    s2 = *reinterpret_cast<uint32_t*>(&a);
+    s16 = *reinterpret_cast<uint32_t*>(&b);
 }
 __device__ __forceinline__ void g_dq_nvfp4(const uint4 w, uint32_t sc2, uint32_t (&o)[16]) {
     const uint32_t ws[4] = {w.x, w.y, w.z, w.w};
@@ -197,10 +223,11 @@ __device__ __forceinline__ void g_dq_nvfp4(const uint4 w, uint32_t sc2, uint32_t
     for (int j = 0; j < 4; j++) {
         uint32_t sv = g_e4m3_f16x2((sc2 >> (8 * (j >> 1))) & 0xffu);
         const __half2 s2 = *reinterpret_cast<__half2*>(&sv);
+        uint32_t hv[4];
+        g_e2m1x8_f16x2(ws[j], hv);                       // the word's four bytes, no shifts
 #pragma unroll
         for (int b = 0; b < 4; b++) {
-            uint32_t hv = g_e2m1x2_f16x2((ws[j] >> (8 * b)) & 0xffu);
-            __half2 h = __hmul2(*reinterpret_cast<__half2*>(&hv), s2);       // exact
+            __half2 h = __hmul2(*reinterpret_cast<__half2*>(&hv[b]), s2);       // exact
             o[j * 4 + b] = *reinterpret_cast<uint32_t*>(&h);
         }
     }
@@ -682,19 +709,36 @@ __global__ void __launch_bounds__(G_THREADS, 1) tc_grouped_gemm(const __grid_con
                 float v = 1.f;
                 const int nn = c + (lane & 15);
                 if (nn < T.nval) {
-                    if (FMT == MOE_FMT_NVFP4) v = a.act_scale[rbase + nn];
-                    // NVFP4: the pre-pass folded the routing weight into the row scale
-                    if (!GU && a.topk_w && FMT != MOE_FMT_NVFP4) v *= a.topk_w[a.row_slot[rbase + nn]];
+                    if (C::kMmaF16) v = a.act_scale[rbase + nn];
+                    // 4-bit formats: the pre-pass folded the routing weight into the row scale
+                    if (!GU && a.topk_w && !C::kMmaF16) v *= a.topk_w[a.row_slot[rbase + nn]];
                 }
                 return v;
             };
             float rowf0 = row_factor(0);
             float gsc = 1.f, usc = 1.f;
             if (FMT == MOE_FMT_NVFP4) { gsc = a.g0[T.e]; if (GU) usc = a.g1[T.e]; }
+            if (FMT == MOE_FMT_INT4_G128) {
+                // undo the dequantisation's power of two of this weight row (gate and up separately)
+                const int row = T.e * a.out_dim + T.m0 + q * 32 + lane;
+                const int ng2 = a.in_dim / 256;                   // bf16 scale pairs per row
+                float mg = 0.f, mu = 0.f;
+                const uint32_t* s0r = reinterpret_cast<const uint32_t*>(a.sc0) + size_t(row) * ng2;
+                const uint32_t* s1r = reinterpret_cast<const uint32_t*>(a.sc1) + size_t(row) * ng2;
+                for (int g2 = 0; g2 < ng2; g2++) {
+                    const uint32_t v = __ldg(s0r + g2);
+                    mg = fmaxf(mg, fmaxf(fabsf(bf16_lo(v)), fabsf(bf16_hi(v))));
+                    if (GU) {
+                        const uint32_t w = __ldg(s1r + g2);
+                        mu = fmaxf(mu, fmaxf(fabsf(bf16_lo(w)), fabsf(bf16_hi(w))));
+                    }
+                }
+                gsc = ldexpf(1.f, -g_int4_row_shift(mg));
+                if (GU) usc = ldexpf(1.f, -g_int4_row_shift(mu));
+            }
             if (!g_wait_w(g_smem(&acc_full[buf]), (t >> 1) & 1, &s_ab, 128)) { fail(); break; }
             g_fence_after();
             const int f = T.m0 + q * 32 + lane;
-            const int fo = a.perm_out ? ((f & ~7) | ((f & 7) < 4 ? 2 * (f & 7) : 2 * (f & 7) - 7)) : f;
             const uint32_t acc0 = tmem + lane_addr + buf * 128;
             for (int c = 0; c < T.bn; c += 16) {
                 const float rowf = c == 0 ? rowf0 : row_factor(c);
@@ -727,7 +771,7 @@ __global__ void __launch_bounds__(G_THREADS, 1) tc_grouped_gemm(const __grid_con
                         } else {
                             v = __uint_as_float(g[j]) * gsc * fj;
                         }
-                        a.out[size_t(rbase + c + j) * a.out_dim + fo] = __float2bfloat16_rn(v);
+                        a.out[size_t(rbase + c + j) * a.out_dim + f] = __float2bfloat16_rn(v);
                     }
                 }
             }
@@ -859,10 +903,17 @@ __global__ void __launch_bounds__(G_THREADS, 1) tc_grouped_gemm(const __grid_con
         bool ok = true;
         for (int tile = blockIdx.x; tile < ntiles && ok && !g_aborted(&s_ab); tile += gridDim.x, t++) {
             const uint8_t* scrow = nullptr;
+            float fk = 1.f;                             // int4: 2^k of this weight row (the epilogue undoes it)
             if (FMT == MOE_FMT_INT4_G128) {
                 const int b = t % NSC;
                 if (!g_wait_w(g_smem(&sc_full[b]), (t / NSC) & 1, &s_ab)) { ok = false; break; }
                 scrow = scbuf + b * sc_buf_bytes + (GU ? hsel * sc_mat_bytes : 0) + r * ngroups * 2;
+                float m = 0.f;
+                for (int g2 = 0; g2 < ngroups / 2; g2++) {
+                    const uint32_t v = reinterpret_cast<const uint32_t*>(scrow)[g2];
+                    m = fmaxf(m, fmaxf(fabsf(bf16_lo(v)), fabsf(bf16_hi(v))));
+                }
+                fk = ldexpf(1.f, g_int4_row_shift(m));
             }
             for (int ps = 0; ps < NPS && ok; ps++, pc++) {
                 const int s = pc % NPK;
@@ -876,6 +927,11 @@ __global__ void __launch_bounds__(G_THREADS, 1) tc_grouped_gemm(const __grid_con
                     nsc = *reinterpret_cast<const uint4*>(st + C::kNMat * C::kMatBytes + (GU ? hsel * C::kNvScBytes : 0) +
                                                           r * 16);
                 const uint32_t nscw[4] = {nsc.x, nsc.y, nsc.z, nsc.w};
+                uint32_t s2[2] = {0u, 0u}, s16[2] = {0u, 0u};   // int4: f16 scale pairs of the two groups
+                if (FMT == MOE_FMT_INT4_G128) {
+                    g_int4_scale_pair(scw & 0xffffu, fk, s2[0], s16[0]);
+                    g_int4_scale_pair(scw >> 16, fk, s2[1], s16[1]);
+                }
                 // Four register buffers in rotation: a buffer is rewritten three
                 // chunks after its tensor-memory store was issued, so the store
                 // has read it by then and the dequantisation does not stall.
@@ -885,9 +941,9 @@ __global__ void __launch_bounds__(G_THREADS, 1) tc_grouped_gemm(const __grid_con
                     constexpr int i = decltype(ic)::value, j = i / kPer, l = i % kPer;
                     const int c = (8 / C::kAPerPk) * j + (GU ? l : kPer * hsel + l);
                     const uint4 w = *reinterpret_cast<const uint4*>(wt + g_swz(r, c));
-                    if (FMT == MOE_FMT_INT4_G128) {
-                        g_dq_int4(w, scw >> (16 * j), o[i % kNBuf]);
-                    } else {
+                    if constexpr (FMT == MOE_FMT_INT4_G128) {
+                        g_dq_int4(w, s2[j], s16[j], o[i % kNBuf]);
+                    } else if constexpr (FMT == MOE_FMT_NVFP4) {
                         // the two E4M3 scales of chunk c are bytes 2c and 2c+1
                         const uint32_t sw = GU ? nscw[2 * j + (l >> 1)] : (hsel ? nscw[2 * j + 1] : nscw[2 * j]);
                         g_dq_nvfp4(w, sw >> (16 * (GU ? (l & 1) : l)), o[i % kNBuf]);
@@ -938,9 +994,15 @@ __global__ void __launch_bounds__(G_THREADS, 1) tc_grouped_gemm(const __grid_con
 // ---------------------------------------------------------------------------
 // Activation pre-pass: gather the GEMM's rows (row r reads activation row
 // row_slot[r] / top_k when by_token, else row r) into the operand order:
-//   mode 0: bf16 copy;  mode 1: bf16, pair order 0,4,1,5,2,6,3,7 in every 8;
-//   mode 2: f16 times 2^-e (e >= 0 least with |x| * 2^-e <= 16384), row scale 2^e.
-// One warp per row.
+//   mode 0: bf16 copy (BF16 weights);
+//   mode 2: f16 times 2^-e in natural order (NVFP4 weights);
+//   mode 3: f16 times 2^-e, pairs (0,4) (1,5) (2,6) (3,7) in every 8 (int4
+//           weights, the order of their dequantised pairs);
+// with e the exponent that puts the row's largest |x| 2^-e in [2^13, 2^14):
+// every bf16 value becomes an f16 exactly (bf16 has 8 significant bits, f16
+// 11) unless it is 2^27 below the row's largest.  The row scale 2^e (times
+// row_w[row_slot[row]] when given: the down projection's routing weight, a
+// power of two times w being exact) goes to scale[row].  One warp per row.
 // ---------------------------------------------------------------------------
 __global__ void __launch_bounds__(256) g_prep(const __nv_bfloat16* __restrict__ src, int in_dim,
                                               const int32_t* __restrict__ row_slot, int top_k, int by_token,
@@ -955,39 +1017,39 @@ __global__ void __launch_bounds__(256) g_prep(const __nv_bfloat16* __restrict__ 
     const int n16 = in_dim / 8;
     if (mode == 0) {
         for (int i = lane; i < n16; i += 32) d[i] = s[i];
-    } else if (mode == 1) {
-        for (int i = lane; i < n16; i += 32) {
-            const uint4 v = s[i];
-            uint4 o;
-            o.x = __byte_perm(v.x, v.z, 0x5410);   // (x0, x4)
-            o.y = __byte_perm(v.x, v.z, 0x7632);   // (x1, x5)
-            o.z = __byte_perm(v.y, v.w, 0x5410);   // (x2, x6)
-            o.w = __byte_perm(v.y, v.w, 0x7632);   // (x3, x7)
-            d[i] = o;
-        }
-    } else {
-        float amax = 0.f;
-        for (int i = lane; i < n16; i += 32) {
-            const uint4 v = s[i];
-            amax = fmaxf(amax, fmaxf(fmaxf(fabsf(bf16_lo(v.x)), fabsf(bf16_hi(v.x))), fmaxf(fabsf(bf16_lo(v.y)), fabsf(bf16_hi(v.y)))));
-            amax = fmaxf(amax, fmaxf(fmaxf(fabsf(bf16_lo(v.z)), fabsf(bf16_hi(v.z))), fmaxf(fabsf(bf16_lo(v.w)), fabsf(bf16_hi(v.w)))));
-        }
-        for (int o = 16; o > 0; o >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, o));
-        int e = 0;
-        while (e < 126 && ldexpf(amax, -e) > 16384.f) e++;
-        const float down = ldexpf(1.f, -e);
-        for (int i = lane; i < n16; i += 32) {
-            const uint4 v = s[i];
-            __half2 h[4];
-            h[0] = __floats2half2_rn(bf16_lo(v.x) * down, bf16_hi(v.x) * down);
-            h[1] = __floats2half2_rn(bf16_lo(v.y) * down, bf16_hi(v.y) * down);
-            h[2] = __floats2half2_rn(bf16_lo(v.z) * down, bf16_hi(v.z) * down);
-            h[3] = __floats2half2_rn(bf16_lo(v.w) * down, bf16_hi(v.w) * down);
-            d[i] = *reinterpret_cast<uint4*>(h);
-        }
-        // mode 2 row scale, times the down projection's routing weight when given (exact: 2^e * w)
-        if (lane == 0) scale[row] = row_w ? ldexpf(1.f, e) * row_w[row_slot[row]] : ldexpf(1.f, e);
+        return;
     }
+    float amax = 0.f;
+    for (int i = lane; i < n16; i += 32) {
+        const uint4 v = s[i];
+        amax = fmaxf(amax, fmaxf(fmaxf(fabsf(bf16_lo(v.x)), fabsf(bf16_hi(v.x))), fmaxf(fabsf(bf16_lo(v.y)), fabsf(bf16_hi(v.y)))));
+        amax = fmaxf(amax, fmaxf(fmaxf(fabsf(bf16_lo(v.z)), fabsf(bf16_hi(v.z))), fmaxf(fabsf(bf16_lo(v.w)), fabsf(bf16_hi(v.w)))));
+    }
+    for (int o = 16; o > 0; o >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, o));
+    int e = 0;
+    if (amax > 0.f && isfinite(amax)) {
+        frexpf(amax, &e);                       // amax = f 2^ex, f in [0.5, 1): amax 2^-(ex-14) in [2^13, 2^14)
+        e = max(e - 14, -100);
+    }
+    const float down = ldexpf(1.f, -e);
+    for (int i = lane; i < n16; i += 32) {
+        const uint4 v = s[i];
+        __half2 h[4];
+        h[0] = __floats2half2_rn(bf16_lo(v.x) * down, bf16_hi(v.x) * down);
+        h[1] = __floats2half2_rn(bf16_lo(v.y) * down, bf16_hi(v.y) * down);
+        h[2] = __floats2half2_rn(bf16_lo(v.z) * down, bf16_hi(v.z) * down);
+        h[3] = __floats2half2_rn(bf16_lo(v.w) * down, bf16_hi(v.w) * down);
+        uint4 o = *reinterpret_cast<uint4*>(h);
+        if (mode == 3) {                        // (x0 x1)(x2 x3)(x4 x5)(x6 x7) -> (x0 x4)(x1 x5)(x2 x6)(x3 x7)
+            const uint4 n = o;
+            o.x = __byte_perm(n.x, n.z, 0x5410);
+            o.y = __byte_perm(n.x, n.z, 0x7632);
+            o.z = __byte_perm(n.y, n.w, 0x5410);
+            o.w = __byte_perm(n.y, n.w, 0x7632);
+        }
+        d[i] = o;
+    }
+    if (lane == 0) scale[row] = row_w ? ldexpf(1.f, e) * row_w[row_slot[row]] : ldexpf(1.f, e);
 }
 
 // 8-bit int4 pre-pass: one CTA of 128 threads per GEMM row (gathered like
@@ -1173,13 +1235,13 @@ int launch_grouped_gemm(const GemvProblem& p, bool gateup, int rows, const GemmB
     const bool nv = p.fmt == MOE_FMT_NVFP4, i4 = p.fmt == MOE_FMT_INT4_G128;
     // the 8-bit down GEMM steps in K = 512; other widths take the 16-bit int4 path
     const bool i8 = i4 && buf.i8 && (gateup || in % 512 == 0);
-    if (i8 && (!buf.zbuf || !buf.scale_buf || !buf.act_buf || buf.perm_out || ksplit > 1)) return MOE_ERR_UNSUPPORTED;
+    if (i8 && (!buf.zbuf || !buf.scale_buf || !buf.act_buf || ksplit > 1)) return MOE_ERR_UNSUPPORTED;
     // activation operand rows [rows, in]: bf16 (f16 for NVFP4) in the kernel's order; 8-bit int4: three
     // int8 digit rows per row
     const void* bsrc = p.act;
     const float* ascale = nullptr;
-    if (!buf.act_ready || nv || i8) {
-        if (!buf.act_buf || (nv && !buf.scale_buf)) return MOE_ERR_WORKSPACE;
+    if (!buf.act_ready || nv || i4) {
+        if (!buf.act_buf || ((nv || i4) && !buf.scale_buf)) return MOE_ERR_WORKSPACE;
         if (i8) {
             const float* row_w = gateup ? nullptr : p.topk_w;
             if (launch_pdl(g_prep_i8, dim3(rows), dim3(G_PREP_I8_THREADS), 0, s, p.act, in, p.row_slot, p.top_k,
@@ -1187,8 +1249,8 @@ int launch_grouped_gemm(const GemvProblem& p, bool gateup, int rows, const GemmB
                            buf.zbuf, p.status) != cudaSuccess)
                 return MOE_ERR_CUDA;
         } else {
-            const int mode = nv ? 2 : (i4 ? 1 : 0);
-            const float* row_w = (nv && !gateup) ? p.topk_w : nullptr;     // folded into the NVFP4 row scale
+            const int mode = nv ? 2 : (i4 ? 3 : 0);
+            const float* row_w = ((nv || i4) && !gateup) ? p.topk_w : nullptr;   // folded into the row scale
             if (launch_pdl(g_prep, dim3((rows * 32 + 255) / 256), dim3(256), 0, s, p.act, in, p.row_slot, p.top_k,
                            p.act_by_token, rows, mode, row_w, reinterpret_cast<uint16_t*>(buf.act_buf),
                            buf.scale_buf) != cudaSuccess)
@@ -1230,7 +1292,6 @@ int launch_grouped_gemm(const GemvProblem& p, bool gateup, int rows, const GemmB
     a.E = E;
     a.out_dim = out;
     a.in_dim = in;
-    a.perm_out = buf.perm_out;
     a.ksplit = ksplit;
     a.partial = buf.partial;
     a.rows = rows;

@@ -224,20 +224,18 @@ int launch_set_u64(unsigned long long* dst, unsigned long long v, cudaStream_t s
 // Writes one 32-bit word of device memory in stream order.
 int launch_set_u32(uint32_t* dst, uint32_t v, cudaStream_t s);
 
-// Activation operand of the tcgen05 grouped GEMM.  Unless act_ready, a
-// pre-pass gathers the problem's rows (row r reads activation row
-// row_slot[r] / top_k when act_by_token, else row r) into act_buf
-// ([rows, in] 16-bit) in the kernel's operand order: bf16 pairs reordered
-// 0,4,1,5,2,6,3,7 in every 8 for int4, f16 with a power-of-two row scale
-// (scale_buf, [rows] fp32) for NVFP4, a plain copy for BF16.  act_ready: the
-// activation rows are already in that order (row r is row r; int4 h written
-// with perm_out, or BF16 rows that need no gather); NVFP4 always runs the
-// pre-pass.  perm_out (gate/up): write h columns in the int4 pair order.
+// Activation operand of the tcgen05 grouped GEMM.  A pre-pass gathers the
+// problem's rows (row r reads activation row row_slot[r] / top_k when
+// act_by_token, else row r) into act_buf ([rows, in] 16-bit) in the kernel's
+// operand order: f16 with a power-of-two row scale (scale_buf, [rows] fp32)
+// for the 4-bit formats (int4: its pairs (0,4) (1,5) (2,6) (3,7) in every 8),
+// a plain copy for BF16; the 8-bit int4 path writes three int8 digit rows
+// per row instead.  act_ready (BF16 only): the rows are already in place
+// (row r is row r), no pre-pass runs.
 struct GemmBuffers {
     void* act_buf;
     float* scale_buf;
     int act_ready;
-    int perm_out;
     int ksplit;          // > 1: split K into this many slices (BF16 only); fp32 partial sums go to partial
     float* partial;      // split_bytes(...) bytes
     int i8;              // int4 on the 8-bit MMA with per-group accumulation (small batches)

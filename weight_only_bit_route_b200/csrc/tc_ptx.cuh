@@ -161,6 +161,13 @@ __device__ __forceinline__ uint32_t g_e2m1x2_f16x2(uint32_t byte) {
     asm("{ .reg .b8 t; cvt.u8.u32 t, %1; cvt.rn.f16x2.e2m1x2 %0, t; }" : "=r"(h) : "r"(byte));
     return h;
 }
+// The four bytes of a word, each a pair of E2M1 codes (low nibble first), as four f16 pairs.
+__device__ __forceinline__ void g_e2m1x8_f16x2(uint32_t w, uint32_t (&h)[4]) {
+    asm("{ .reg .b8 b0, b1, b2, b3; mov.b32 {b0, b1, b2, b3}, %4;\n"
+        " cvt.rn.f16x2.e2m1x2 %0, b0; cvt.rn.f16x2.e2m1x2 %1, b1;\n"
+        " cvt.rn.f16x2.e2m1x2 %2, b2; cvt.rn.f16x2.e2m1x2 %3, b3; }"
+        : "=r"(h[0]), "=r"(h[1]), "=r"(h[2]), "=r"(h[3]) : "r"(w));
+}
 __device__ __forceinline__ uint32_t g_e4m3_f16x2(uint32_t byte) {          // {s, s} in f16
     uint32_t h;
     asm("{ .reg .b16 t; cvt.u16.u32 t, %1; cvt.rn.f16x2.e4m3x2 %0, t; }" : "=r"(h) : "r"(byte | (byte << 8)));
