@@ -61,6 +61,14 @@ def lib():
         L.oracle_grouped_down.restype = None
         L.oracle_combine.argtypes = [P, P, I64, I, I64, P, P]
         L.oracle_combine.restype = None
+        L.oracle_act_quant_nvfp4.argtypes = [P, I64, I64, P, P, P, P]
+        L.oracle_act_quant_nvfp4.restype = None
+        L.oracle_grouped_swiglu_w4a4.argtypes = [P, I64, I64, I, P, P, P, P, P, P, I64, P]
+        L.oracle_grouped_swiglu_w4a4.restype = None
+        L.oracle_grouped_down_w4a4.argtypes = [P, I64, I64, P, P, P, P, P, P, I64, P]
+        L.oracle_grouped_down_w4a4.restype = None
+        L.oracle_moe_forward_w4a4.argtypes = [P, I64, I64, I64, I, P, P, P, P, P, P, P, P, P, P, P, I64, P]
+        L.oracle_moe_forward_w4a4.restype = I
         L.oracle_csf_encode.argtypes = [P, I64, I64, I64, P, P, P]
         L.oracle_csf_encode.restype = I64
         L.oracle_csf_decode.argtypes = [P, P, P, I64, I64, I64, P]
@@ -308,3 +316,66 @@ def csf_decode(fixed, exceptions, starts, R, C):
     out = np.empty((E, R, C), np.uint8)
     lib().oracle_csf_decode(_p(fixed), _p(_c(exceptions, np.uint32)), _p(_c(starts, np.int64)), E, R, C, _p(out))
     return out
+
+
+def act_quant_nvfp4(x_bits, g):
+    """bf16 bits [rows, cols], global fp32 per row (scalar or [rows]) ->
+    (packed uint8 [rows, cols/2], scales uint8 [rows, cols/16], dequantised fp32 [rows, cols])."""
+    x = _c(x_bits, np.uint16)
+    rows, cols = x.shape
+    gg = _c(np.broadcast_to(np.asarray(g, np.float32), (rows,)), np.float32)
+    packed = np.empty((rows, cols // 2), np.uint8)
+    scales = np.empty((rows, cols // 16), np.uint8)
+    xq = np.empty((rows, cols), np.float32)
+    lib().oracle_act_quant_nvfp4(_p(x), rows, cols, _p(gg), _p(packed), _p(scales), _p(xq))
+    return packed, scales, xq
+
+
+def grouped_swiglu_w4a4(x_bits, offsets, row_slot, k, gate, up, in_scale, rows):
+    x = _c(x_bits, np.uint16)
+    H = x.shape[1]
+    F = gate.out
+    rows = _c(rows, np.int32)
+    h = np.empty((rows.shape[0], F), np.float64)
+    g, u = gate._struct(), up._struct()
+    lib().oracle_grouped_swiglu_w4a4(_p(x), H, F, k, _p(_c(offsets, np.int32)), _p(_c(row_slot, np.int32)),
+                                     ctypes.addressof(g), ctypes.addressof(u), _p(_c(in_scale, np.float32)),
+                                     _p(rows), rows.shape[0], _p(h))
+    return h
+
+
+def grouped_down_w4a4(h_bits, offsets, row_slot, topk_w, down, in_scale, rows):
+    hb = _c(h_bits, np.uint16)
+    F = hb.shape[1]
+    H = down.out
+    rows = _c(rows, np.int32)
+    y = np.empty((rows.shape[0], H), np.float64)
+    d = down._struct()
+    tw = None if topk_w is None else _c(topk_w, np.float32)
+    lib().oracle_grouped_down_w4a4(_p(hb), F, H, _p(_c(offsets, np.int32)), _p(_c(row_slot, np.int32)), _p(tw),
+                                   ctypes.addressof(d), _p(_c(in_scale, np.float32)), _p(rows), rows.shape[0], _p(y))
+    return y
+
+
+def moe_forward_w4a4(x_bits, ids, topk_w, gate, up, down, in_gu, in_dn, shared=None, tokens=None):
+    """fp64 W4A4 layer output for the listed tokens (default: all) -> float64 [n, H]."""
+    x = _c(x_bits, np.uint16)
+    T, H = x.shape
+    ids = _c(ids, np.int32)
+    w = _c(topk_w, np.float32)
+    k = ids.shape[1]
+    F = gate.out
+    if tokens is None:
+        tokens = np.arange(T, dtype=np.int32)
+    tok = _c(tokens, np.int32)
+    n = tok.shape[0]
+    y = np.empty((n, H), np.float64)
+    sg, su, sd = (shared if shared is not None else (None, None, None))
+    structs = [b._struct() if b is not None else None for b in (gate, up, down, sg, su, sd)]
+    refs = [ctypes.addressof(s) if s is not None else None for s in structs]
+    rc = lib().oracle_moe_forward_w4a4(_p(x), T, H, F, k, _p(ids), _p(w), refs[0], refs[1], refs[2],
+                                       _p(_c(in_gu, np.float32)), _p(_c(in_dn, np.float32)), refs[3], refs[4],
+                                       refs[5], _p(tok), n, _p(y))
+    if rc != 0:
+        raise ValueError("expert id out of range")
+    return y

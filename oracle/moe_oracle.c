@@ -39,6 +39,13 @@
  *     (fp32); top-k by s, ties to the lower expert id, listed by descending s;
  *     weights s / sum(selected s) (fp32).
  *   - Layer: no routed scaling factor, no shared-expert gate, SwiGLU limit off.
+ *   - NVFP4 W4A4 (layers 3-87, quant_algo NVFP4 with an input_scale): the
+ *     activation entering a projection is quantised like a weight row, per
+ *     16 elements, with the expert's input_scale as its global scale (a static
+ *     value, so large blocks saturate at 448 x 6); gate and up read the same
+ *     activation, quantised once with the gate's input_scale; the down
+ *     projection's input is h rounded to bf16 (the activations between the
+ *     projections are bf16), then quantised with the down input_scale.
  *   - CSF: the 4-bit code stored at an exception's position is 0 (the
  *     decoder replaces that byte, so any code would do; 0 is the plainest);
  *     the rows of a slab follow one another, each C/2 bytes.
@@ -656,4 +663,197 @@ void oracle_csf_decode(const uint8_t* fixed, const uint32_t* exceptions, const i
             scales[e * R * C + pos] = (uint8_t)(x >> 24);
         }
     }
+}
+
+
+/* ------------------------------------------------------------------------ */
+/* NVFP4 W4A4  [NVFP4] Modifications items 2-3 (quant_algo NVFP4 with an     */
+/* input_scale for layers 3-87; group size 16)                              */
+/* ------------------------------------------------------------------------ */
+
+/* Quantise one activation row of n bf16 values (n % 16 == 0) with global g:
+ * per block sb = e4m3_rne_sat(amax_b / (6 g)), codes e2m1_rne_sat(x / (e4m3(sb) g));
+ * returns the dequantised values e2m1 x e4m3 x g in xq (fp32, one rounding),
+ * and (optionally) the packed codes [n/2] and block scales [n/16]. */
+static void act_quant_row(const float* x, int64_t n, float g, float* xq, uint8_t* packed, uint8_t* scales) {
+    for (int64_t b = 0; b < n / FP4_BLOCK; b++) {
+        const float* xb = x + b * FP4_BLOCK;
+        float amax_b = 0.0f;
+        for (int j = 0; j < FP4_BLOCK; j++) {
+            float a = fabsf(xb[j]);
+            if (a > amax_b) amax_b = a;
+        }
+        uint8_t sb = 0;
+        if (g > 0.0f) sb = oracle_e4m3_encode_nonneg(amax_b / (6.0f * g));
+        float eff = oracle_e4m3_decode(sb) * g;
+        if (scales) scales[b] = sb;
+        for (int j = 0; j < FP4_BLOCK; j++) {
+            uint8_t code = (eff > 0.0f) ? oracle_e2m1_encode(xb[j] / eff) : 0;
+            xq[b * FP4_BLOCK + j] = (oracle_e2m1_decode(code) * oracle_e4m3_decode(sb)) * g;
+            if (packed) {
+                int64_t c = b * FP4_BLOCK + j;
+                if (c % 2 == 0) packed[c / 2] = code;
+                else packed[c / 2] = (uint8_t)(packed[c / 2] | (code << 4));
+            }
+        }
+    }
+}
+
+/* Activation quantiser: bf16 rows [rows, cols], row r with global g[r]
+ * -> packed u8 [rows, cols/2] (even element in the low nibble), scales u8
+ * E4M3 [rows, cols/16], and the dequantised values fp32 [rows, cols]
+ * (any output may be NULL). */
+void oracle_act_quant_nvfp4(const uint16_t* x, int64_t rows, int64_t cols, const float* g,
+                            uint8_t* packed, uint8_t* scales, float* xq) {
+    #pragma omp parallel for schedule(static)
+    for (int64_t r = 0; r < rows; r++) {
+        float* xf = (float*)malloc(sizeof(float) * cols);
+        float* q = (float*)malloc(sizeof(float) * cols);
+        for (int64_t c = 0; c < cols; c++) xf[c] = oracle_bf16_to_f32(x[r * cols + c]);
+        act_quant_row(xf, cols, g[r], q, packed ? packed + r * (cols / 2) : NULL,
+                      scales ? scales + r * (cols / FP4_BLOCK) : NULL);
+        if (xq) memcpy(xq + r * cols, q, sizeof(float) * cols);
+        free(xf);
+        free(q);
+    }
+}
+
+/* W4A4 gate/up + SwiGLU over bucketed rows: for row r of expert e (token
+ * t = row_slot[r] / k), xq = x[t] quantised with in_scale[e], then
+ * h[r] = silu(Wg[e] xq) * (Wu[e] xq) in fp64.  h is [n, F]. */
+void oracle_grouped_swiglu_w4a4(const uint16_t* x, int64_t H, int64_t F, int k,
+                                const int32_t* offsets, const int32_t* row_slot,
+                                const oracle_bank* gate, const oracle_bank* up, const float* in_scale,
+                                const int32_t* rows, int64_t n, double* h) {
+    int64_t E = gate->E;
+    float* wg = (float*)malloc(sizeof(float) * F * H);
+    float* wu = (float*)malloc(sizeof(float) * F * H);
+    float* xf = (float*)malloc(sizeof(float) * H);
+    float* xq = (float*)malloc(sizeof(float) * H);
+    for (int64_t e = 0; e < E; e++) {
+        int any = 0;
+        for (int64_t i = 0; i < n; i++)
+            if (rows[i] >= offsets[e] && rows[i] < offsets[e + 1]) any = 1;
+        if (!any) continue;
+        oracle_dequant_expert(gate, (int)e, wg);
+        oracle_dequant_expert(up, (int)e, wu);
+        for (int64_t i = 0; i < n; i++) {
+            int32_t r = rows[i];
+            if (r < offsets[e] || r >= offsets[e + 1]) continue;
+            int64_t t = row_slot[r] / k;
+            for (int64_t hh = 0; hh < H; hh++) xf[hh] = oracle_bf16_to_f32(x[t * H + hh]);
+            act_quant_row(xf, H, in_scale[e], xq, NULL, NULL);
+            #pragma omp parallel for schedule(static)
+            for (int64_t f = 0; f < F; f++) {
+                double g = 0.0, u = 0.0;
+                for (int64_t hh = 0; hh < H; hh++) {
+                    g += (double)wg[f * H + hh] * (double)xq[hh];
+                    u += (double)wu[f * H + hh] * (double)xq[hh];
+                }
+                h[i * F + f] = silu(g) * u;
+            }
+        }
+    }
+    free(wg); free(wu); free(xf); free(xq);
+}
+
+/* W4A4 down projection: for row r of expert e, hq = h_in[r] (bf16) quantised
+ * with in_scale[e]; y[r] = w[row_slot[r]] * (Wd[e] hq) (w = 1 if topk_w is NULL). */
+void oracle_grouped_down_w4a4(const uint16_t* h_in, int64_t F, int64_t H,
+                              const int32_t* offsets, const int32_t* row_slot,
+                              const float* topk_w, const oracle_bank* down, const float* in_scale,
+                              const int32_t* rows, int64_t n, double* y) {
+    int64_t E = down->E;
+    float* wd = (float*)malloc(sizeof(float) * H * F);
+    float* hf = (float*)malloc(sizeof(float) * F);
+    float* hq = (float*)malloc(sizeof(float) * F);
+    for (int64_t e = 0; e < E; e++) {
+        int any = 0;
+        for (int64_t i = 0; i < n; i++)
+            if (rows[i] >= offsets[e] && rows[i] < offsets[e + 1]) any = 1;
+        if (!any) continue;
+        oracle_dequant_expert(down, (int)e, wd);
+        for (int64_t i = 0; i < n; i++) {
+            int32_t r = rows[i];
+            if (r < offsets[e] || r >= offsets[e + 1]) continue;
+            double wt = topk_w ? (double)topk_w[row_slot[r]] : 1.0;
+            for (int64_t f = 0; f < F; f++) hf[f] = oracle_bf16_to_f32(h_in[(int64_t)r * F + f]);
+            act_quant_row(hf, F, in_scale[e], hq, NULL, NULL);
+            #pragma omp parallel for schedule(static)
+            for (int64_t hh = 0; hh < H; hh++) {
+                double acc = 0.0;
+                for (int64_t f = 0; f < F; f++) acc += (double)wd[hh * F + f] * (double)hq[f];
+                y[i * H + hh] = wt * acc;
+            }
+        }
+    }
+    free(wd); free(hf); free(hq);
+}
+
+/* W4A4 layer forward for the listed tokens: as oracle_moe_forward, with each
+ * routed expert's input quantised (in_gu[e] for gate/up, in_dn[e] for down,
+ * the down input being h rounded to bf16).  The shared expert is BF16 and
+ * reads x unquantised.  Returns 0, or -1 on an out-of-range id. */
+int oracle_moe_forward_w4a4(const uint16_t* x, int64_t T, int64_t H, int64_t F, int k,
+                            const int32_t* ids, const float* topk_w,
+                            const oracle_bank* gate, const oracle_bank* up, const oracle_bank* down,
+                            const float* in_gu, const float* in_dn,
+                            const oracle_bank* sh_gate, const oracle_bank* sh_up, const oracle_bank* sh_down,
+                            const int32_t* tok, int64_t n, double* y) {
+    int64_t E = gate->E;
+    for (int64_t i = 0; i < n; i++)
+        for (int64_t j = 0; j < k; j++) {
+            int32_t e = ids[tok[i] * k + j];
+            if (e < 0 || e >= E) return -1;
+        }
+    /* routed part through the per-step definitions, one (token, slot) row at a time */
+    memset(y, 0, sizeof(double) * n * H);
+    double* hrow = (double*)malloc(sizeof(double) * F);
+    uint16_t* hb = (uint16_t*)malloc(sizeof(uint16_t) * F);
+    double* yrow = (double*)malloc(sizeof(double) * H);
+    for (int64_t i = 0; i < n; i++) {
+        for (int64_t j = 0; j < k; j++) {
+            int32_t e = ids[tok[i] * k + j];
+            /* a one-row problem: expert e owns row 0, which holds slot tok[i]*k + j of token tok[i] */
+            int32_t* off = (int32_t*)calloc(E + 1, sizeof(int32_t));
+            for (int64_t q = e + 1; q <= E; q++) off[q] = 1;
+            int32_t slot = (int32_t)(tok[i] * k + j);
+            int32_t row0 = 0;
+            oracle_grouped_swiglu_w4a4(x, H, F, k, off, &slot, gate, up, in_gu, &row0, 1, hrow);
+            for (int64_t f = 0; f < F; f++) hb[f] = oracle_f32_to_bf16((float)hrow[f]);
+            oracle_grouped_down_w4a4(hb, F, H, off, &slot, topk_w, down, in_dn, &row0, 1, yrow);
+            for (int64_t hh = 0; hh < H; hh++) y[i * H + hh] += yrow[hh];
+            free(off);
+        }
+    }
+    if (sh_gate) {                           /* shared expert: BF16 weights, x unquantised, weight 1 */
+        float* wg = (float*)malloc(sizeof(float) * F * H);
+        float* wu = (float*)malloc(sizeof(float) * F * H);
+        float* wd = (float*)malloc(sizeof(float) * H * F);
+        oracle_dequant_expert(sh_gate, 0, wg);
+        oracle_dequant_expert(sh_up, 0, wu);
+        oracle_dequant_expert(sh_down, 0, wd);
+        for (int64_t i = 0; i < n; i++) {
+            const uint16_t* xt = x + (int64_t)tok[i] * H;
+            #pragma omp parallel for schedule(static)
+            for (int64_t f = 0; f < F; f++) {
+                double g = 0.0, u = 0.0;
+                for (int64_t hh = 0; hh < H; hh++) {
+                    double xv = (double)oracle_bf16_to_f32(xt[hh]);
+                    g += (double)wg[f * H + hh] * xv;
+                    u += (double)wu[f * H + hh] * xv;
+                }
+                hrow[f] = silu(g) * u;
+            }
+            #pragma omp parallel for schedule(static)
+            for (int64_t hh = 0; hh < H; hh++) {
+                double acc = 0.0;
+                for (int64_t f = 0; f < F; f++) acc += (double)wd[hh * F + f] * hrow[f];
+                y[i * H + hh] += acc;
+            }
+        }
+        free(wg); free(wu); free(wd);
+    }
+    free(hrow); free(hb); free(yrow);
+    return 0;
 }
