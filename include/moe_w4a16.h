@@ -22,6 +22,14 @@
  *       [E, out, in/2], two E2M1 codes per byte, even element in the low nibble;
  *       scales: uint8 E4M3 [E, out, in/16]; global_scale: fp32 [E]
  *       (weight_scale_2).  w = e2m1(code) * e4m3(scale) * global_scale[e].
+ *       With input_scale (W4A4, layers 3-87 of the pages' model): the
+ *       activation entering the projection is quantised to NVFP4 on the fly,
+ *       per 16 elements, with the expert's input_scale as its global scale
+ *       (block scale e4m3_rne_sat(amax / (6 g)), codes e2m1_rne_sat(x / (e4m3 g))),
+ *       and the product runs on the quantised values.  Gate and up read the
+ *       same activation, quantised once with gate.input_scale (up.input_scale
+ *       must be NULL or the same pointer); the down projection's input is h
+ *       rounded to bf16, quantised with down.input_scale.
  *   MOE_FMT_BF16 -- plain bf16 [E, out, in] (used for the shared expert).
  *
  * Conventions for every entry point:
@@ -85,6 +93,11 @@ typedef struct {
     const void* packed;       /* INT4: int32[E,out,in/8]; NVFP4: u8[E,out,in/2]; BF16: bf16[E,out,in] */
     const void* scales;       /* INT4: bf16[E,out,in/128]; NVFP4: u8 E4M3[E,out,in/16]; BF16: NULL   */
     const float* global_scale;/* NVFP4: fp32[E]; otherwise NULL                    */
+    const float* input_scale; /* NVFP4 W4A4: fp32[E], the activation global scale of
+                                 each expert (quant_algo NVFP4 with an input_scale,
+                                 "Step-5-Preview-NVFP4-Local", Modifications); NULL:
+                                 W4A16 (activations stay bf16).  Only NVFP4 banks
+                                 on the tensor-core GEMM take it.               */
 } moe_qweight;
 
 /* A whole MoE layer.  sh_gate/sh_up/sh_down: MOE_FMT_BF16 banks with
@@ -288,6 +301,16 @@ int moe_layer_forward(const void* x, int T, const moe_layer* L, void* y,
 /* ---------------------------------------------------------------------- */
 /* Weight conversion (offline step, not on the hot path)                   */
 /* ---------------------------------------------------------------------- */
+
+/* NVFP4 activation quantiser (W4A4 inputs, "Step-5-Preview-NVFP4-Local",
+ * Modifications: quant_algo NVFP4, group size 16, with an input_scale): row r
+ * of x (bf16 [rows, cols], cols % 16 == 0) with global g[r] (device fp32
+ * [rows]): scales[r, b] = e4m3_rne_sat(amax_b / (6 g[r])), codes
+ * e2m1_rne_sat(x / (e4m3(scale) g[r])); packed: u8 [rows, cols/2] (even
+ * element in the low nibble), scales: u8 [rows, cols/16] (out).  The layer
+ * paths quantise the same way inside their activation pre-pass. */
+int moe_quantize_nvfp4_act(const void* x, int64_t rows, int64_t cols, const float* g,
+                           uint8_t* packed, uint8_t* scales, moe_stream_t stream);
 
 /* int4 symmetric g128 quantiser ("Step-5-Preview-Int4-g128", Recipe): per row
  * and group of 128, the scale is bf16((r * amax) / 7) for the clip ratio r in

@@ -355,6 +355,26 @@ def test_layer_forward_gemm_path_all_tokens(fmt):
     print(f"{fmt}: near-tie {n_nt}, flipped {n_flip}, max rel err {rel:.2e}")
 
 
+@pytest.mark.parametrize("fmt", ["int4", "nvfp4"])
+def test_layer_wide_gateup_tiles(fmt):
+    """8 experts and 200 tokens (1600 routed rows, about 200 per expert): the
+    gate/up GEMM takes tiles of up to 128 token rows (a single accumulator
+    buffer), the shared expert too.  Every token against the oracle."""
+    base = syn.WORKLOADS[0]
+    wl = syn.Workload(f"wide_tiles_{fmt}_T200", 200, base.H, 8, base.F, base.k, fmt, False, base.router_std, False)
+    P = build(wl, "quantised", shared=True)
+    L = device_layer(moe, P)
+    ws = _ws(P.T, wl)
+    x = dev_bf16(P.x)
+    y = moe.layer_forward(x, L, ws)
+    ids, w = moe.route_topk(x, L.router_w, L.router_bias, wl.k, ws)
+    torch.cuda.synchronize()
+    assert moe.read_status(ws) == 0
+    tokens = np.arange(P.T, dtype=np.int32)
+    n_nt, n_flip, rel = layer_check(P, bf16_bits(y), tokens, ids.cpu().numpy(), w.cpu().numpy())
+    print(f"{fmt}: near-tie {n_nt}, flipped {n_flip}, max rel err {rel:.2e}")
+
+
 def _wide(fmt, T):
     # F = 512: with E = 32 both int4 projections can take the 8-bit GEMM (down K = F is a multiple of 512)
     base = syn.WORKLOADS[0]

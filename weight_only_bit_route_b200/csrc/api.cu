@@ -28,6 +28,7 @@ int check_dims(int T, int H, int E, int F, int k) {
 
 int check_bank(const moe_qweight* b, int E, int out, int in) {
     if (!b) return MOE_ERR_INVALID_ARG;
+    if (b->input_scale && b->fmt != MOE_FMT_NVFP4) return MOE_ERR_UNSUPPORTED;   // W4A4 is NVFP4 only
     if (b->fmt != MOE_FMT_INT4_G128 && b->fmt != MOE_FMT_NVFP4 && b->fmt != MOE_FMT_BF16)
         return MOE_ERR_UNSUPPORTED;
     if (b->num_experts != E || b->out_dim != out || b->in_dim != in) return MOE_ERR_INVALID_ARG;
@@ -59,7 +60,10 @@ bool gemm_shape_ok(int in_dim, int out_dim) { return in_dim % 256 == 0 && out_di
 
 int run_problem(const GemvProblem& p, bool gateup, int rows, int act_rows, void* prep, const GemmBuffers& gb,
                 float* partial, cudaStream_t s) {
-    if (!gemm_shape_ok(p.in_dim, p.out_dim)) return launch_stream_gemv(p, nullptr, gateup, act_rows, prep, s, true);
+    if (!gemm_shape_ok(p.in_dim, p.out_dim)) {
+        if (p.in_scale) return MOE_ERR_UNSUPPORTED;     // W4A4 runs on the GEMM only
+        return launch_stream_gemv(p, nullptr, gateup, act_rows, prep, s, true);
+    }
     GemmBuffers b = gb;
     b.ksplit = shared_ksplit(p.E, p.fmt, gateup, rows, p.in_dim);
     b.partial = partial;
@@ -102,6 +106,10 @@ int layer_checks(const void* x, int T, const moe_layer* L, void* y, void* ws, si
     MOE_TRY(check_bank(&L->up, L->E, L->F, L->H));
     MOE_TRY(check_bank(&L->down, L->E, L->H, L->F));
     if (L->gate.fmt == MOE_FMT_BF16 || L->gate.fmt != L->up.fmt || L->gate.fmt != L->down.fmt)
+        return MOE_ERR_UNSUPPORTED;
+    // gate and up share one quantised activation (the gate's input scale)
+    if (L->up.input_scale && L->up.input_scale != L->gate.input_scale) return MOE_ERR_UNSUPPORTED;
+    if ((L->gate.input_scale || L->down.input_scale) && !(gemm_shape_ok(L->H, L->F) && gemm_shape_ok(L->F, L->H)))
         return MOE_ERR_UNSUPPORTED;
     const bool has_sh = L->sh_gate.packed || L->sh_up.packed || L->sh_down.packed;
     if (has_sh) {
@@ -212,12 +220,12 @@ int layer_run(const void* x, int T, const moe_layer* L, void* y, void* ws, cudaS
     gu.E = E; gu.topk_w = nullptr; gu.fmt = L->gate.fmt; gu.out_dim = F; gu.in_dim = H;
     gu.p0 = L->gate.packed; gu.s0 = L->gate.scales; gu.g0 = L->gate.global_scale;
     gu.p1 = L->up.packed; gu.s1 = L->up.scales; gu.g1 = L->up.global_scale;
-    gu.out = h_perm; gu.status = status;
+    gu.out = h_perm; gu.status = status; gu.in_scale = L->gate.input_scale;
     GemvProblem dn{};
     dn.act = h_perm; dn.act_by_token = 0; dn.top_k = k; dn.offsets = offsets; dn.row_slot = row_slot;
     dn.E = E; dn.topk_w = tw; dn.fmt = L->down.fmt; dn.out_dim = H; dn.in_dim = F;
     dn.p0 = L->down.packed; dn.s0 = L->down.scales; dn.g0 = L->down.global_scale;
-    dn.out = y_perm; dn.status = status;
+    dn.out = y_perm; dn.status = status; dn.in_scale = L->down.input_scale;
     // routed experts: both projections on one path
     const bool i8 = routed_gemm && i8_int4(gu, R);
     if (routed_gemm) {
@@ -359,6 +367,7 @@ int moe_grouped_w4a16_swiglu(const void* x, int T, int H, const int32_t* expert_
     MOE_TRY(check_bank(gate, E, F, H));
     MOE_TRY(check_bank(up, E, F, H));
     if (gate->fmt != up->fmt || F % 128) return MOE_ERR_UNSUPPORTED;
+    if (up->input_scale && up->input_scale != gate->input_scale) return MOE_ERR_UNSUPPORTED;
     if (T == 0) return MOE_OK;
     if (!x || !al16(x) || !expert_offsets || !row_slot || !h_perm || !al16(h_perm)) return MOE_ERR_INVALID_ARG;
     // rows present: T * top_k routed slots, or T for a single shared expert
@@ -371,6 +380,7 @@ int moe_grouped_w4a16_swiglu(const void* x, int T, int H, const int32_t* expert_
     p.p0 = gate->packed; p.s0 = gate->scales; p.g0 = gate->global_scale;
     p.p1 = up->packed; p.s1 = up->scales; p.g1 = up->global_scale;
     p.out = reinterpret_cast<__nv_bfloat16*>(h_perm); p.status = at<int32_t>(ws, 0);
+    p.in_scale = gate->input_scale;
     void* prep = at<void>(ws, kStepScratch + align256(size_t(E + 2) * 16));
     return run_problem(p, true, rows, T, prep, gemm_buffers(prep, rows, H, false, i8_int4(p, rows)),
                        step_partial(ws, E, rows, H), cs(stream));
@@ -394,6 +404,7 @@ int moe_grouped_w4a16_down(const void* h_perm, const int32_t* expert_offsets, co
     p.fmt = down->fmt; p.out_dim = H; p.in_dim = F;
     p.p0 = down->packed; p.s0 = down->scales; p.g0 = down->global_scale;
     p.out = reinterpret_cast<__nv_bfloat16*>(y_perm); p.status = at<int32_t>(ws, 0);
+    p.in_scale = down->input_scale;
     void* prep = at<void>(ws, kStepScratch + align256(size_t(E + 2) * 16));
     // BF16 rows are read in place (row r is activation row r)
     return run_problem(p, false, rows, rows, prep,
@@ -462,6 +473,16 @@ int moe_quantize_int4_g128(const void* w, int64_t rows, int64_t cols, int32_t* p
     if (!w || !packed || !scales || !al16(w) || !al16(packed)) return MOE_ERR_INVALID_ARG;
     return launch_quant_int4(reinterpret_cast<const __nv_bfloat16*>(w), rows, cols, packed,
                              reinterpret_cast<__nv_bfloat16*>(scales), cs(stream));
+}
+
+int moe_quantize_nvfp4_act(const void* x, int64_t rows, int64_t cols, const float* g, uint8_t* packed,
+                           uint8_t* scales, moe_stream_t stream) {
+    if (rows < 0 || cols < 0) return MOE_ERR_INVALID_ARG;
+    if (cols % 16) return MOE_ERR_UNSUPPORTED;
+    if (rows == 0 || cols == 0) return MOE_OK;
+    if (!x || !g || !packed || !scales) return MOE_ERR_INVALID_ARG;
+    return launch_quant_nvfp4_act(reinterpret_cast<const __nv_bfloat16*>(x), rows, cols, g, packed, scales,
+                                  cs(stream));
 }
 
 int moe_quantize_nvfp4(const void* w, int64_t rows, int64_t cols, uint8_t* packed, uint8_t* scales,

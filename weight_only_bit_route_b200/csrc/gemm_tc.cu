@@ -76,6 +76,7 @@
 #include <type_traits>
 
 #include "moe_internal.cuh"
+#include "nvfp4_block.cuh"
 #include "tc_ptx.cuh"
 
 namespace moe {
@@ -100,23 +101,28 @@ constexpr int G_EPI_WARPS = 4;
 // format value.
 constexpr int FMT_INT4_I8 = 3;
 
-template <int FMT, bool GU>
+// W (wide): gate/up tiles of up to 128 token rows instead of 64, for batches
+// whose experts hold many rows: each dequantised weight then serves twice the
+// tokens.  The 4-bit formats keep a single accumulator buffer of 256 columns
+// (gate, up) and two A stages; BF16 (no A stages) keeps two buffers.
+template <int FMT, bool GU, bool W = false>
 struct GCfg {
     static constexpr bool kI8 = FMT == FMT_INT4_I8;
     static constexpr bool kInt4 = FMT == MOE_FMT_INT4_G128 || kI8;
     static constexpr bool kTmemA = FMT != MOE_FMT_BF16;
+    static constexpr bool kWide = W && GU && !kI8;
     static constexpr int kNMat = GU ? 2 : 1;
-    static constexpr int kNMax = kI8 ? 5 : (GU ? 64 : 128);        // token rows per tile
-    static constexpr int kUpCol = 64;                               // 16-bit paths: up accumulator within a buffer
+    static constexpr int kNMax = kI8 ? 5 : (GU ? (kWide ? 128 : 64) : 128);   // token rows per tile
+    static constexpr int kUpCol = kWide ? 128 : 64;                 // 16-bit paths: up accumulator within a buffer
     // K per MMA step: 8-bit down steps are K = 512, so that the per-step fixed cost of the
     // issuer and the unpack warps covers 32 KB of weights, as a gate/up step does
     static constexpr int kSK = kI8 ? (GU ? 256 : 512) : 128;
     static constexpr int kGroups = kSK / 128;                       // i8: scale groups per MMA stage
-    static constexpr int kAccCols = kI8 ? kGroups * kNMat * 16 : 128;   // one accumulator buffer
+    static constexpr int kAccCols = kI8 ? kGroups * kNMat * 16 : (kWide ? 256 : 128);   // one accumulator buffer
     // Tensor memory: accumulators in [0, kABase), A stages in [kABase, 512).  The
     // 8-bit path keeps few small accumulators and gives the A ring the room
     // (its dequantise -> MMA -> free cycle is long against a step).
-    static constexpr int kAccBufs = kI8 ? 128 / kAccCols : 256 / kAccCols;
+    static constexpr int kAccBufs = kI8 ? 128 / kAccCols : (kWide && kTmemA ? 1 : (kWide ? 2 : 256 / kAccCols));
     static constexpr int kABase = kAccBufs * kAccCols;
     static constexpr int kMmaK = kI8 ? 32 : 16;                     // K per MMA instruction
     static constexpr int kPkK = kTmemA ? (kI8 ? kSK : 256) : 128;   // K per weight stage
@@ -129,14 +135,16 @@ struct GCfg {
     static constexpr int kBAtom = (kI8 ? 16 : kNMax) * 128;         // 128 bytes of K for every B row
     static constexpr int kBAtoms = kI8 ? kSK / 128 : 2;             // 128-byte K slices per B stage
     static constexpr int kBStageBytes = kBAtoms * kBAtom;
-    static constexpr int kBStages = kI8 ? (GU ? 6 : 4) : 4;         // i8 stages are small; cover the copy latency
+    // i8 stages are small: cover the copy latency; wide stages are large: fit shared memory
+    static constexpr int kBStages = kI8 ? (GU ? 6 : 4) : (kWide ? (kTmemA ? 3 : 2) : 4);
     static constexpr int kAColsK = kI8 ? kSK / 4 : 64;              // TMEM columns of one matrix's A stage
     static constexpr int kAStageCols = kNMat * kAColsK;
-    static constexpr int kAStages = (512 - kABase) / kAStageCols;
+    static constexpr int kAStages = kTmemA ? (512 - kABase) / kAStageCols : 1;   // (BF16: none used)
     static constexpr int kAPerPk = kPkK / kSK;                      // A stages per weight stage (2, or 1 for i8)
     static constexpr int kChunkCols = 16;                           // 16-bit paths: TMEM columns of one packed chunk
     static constexpr int kDqArrivals = kI8 ? G_DQ_WARPS / 2 : G_DQ_WARPS;  // warps that fill one stage
     static constexpr bool kMmaF16 = FMT == MOE_FMT_NVFP4 || FMT == MOE_FMT_INT4_G128;   // f16 operands
+    static_assert(kABase <= 512 && (!kTmemA || kAStages >= 2), "tensor memory layout");
 };
 
 constexpr int G_DONE = 16;                                          // "stage done" barrier ring
@@ -259,14 +267,14 @@ __device__ __forceinline__ void g_static_for(F&& f) {
     }
 }
 
-template <int FMT, bool GU>
+template <int FMT, bool GU, bool W>
 __global__ void __launch_bounds__(G_THREADS, 1) tc_grouped_gemm(const __grid_constant__ GArgs a) {
-    using C = GCfg<FMT, GU>;
+    using C = GCfg<FMT, GU, W>;
     extern __shared__ __align__(1024) uint8_t smem[];
     __shared__ __align__(8) uint64_t pk_full[C::kPkMax], pk_empty[C::kPkMax];
     __shared__ __align__(8) uint64_t b_full[C::kBStages], a_full[C::kAStages], done[G_DONE];
     __shared__ __align__(8) uint64_t sc_full[G_SC_MAX], sc_empty[G_SC_MAX];
-    __shared__ __align__(8) uint64_t acc_full[2], acc_empty[C::kAccBufs], drain;
+    __shared__ __align__(8) uint64_t acc_full[2], acc_empty[2], drain;
     __shared__ __align__(8) uint64_t hold_bar;        // failure testing: a barrier nothing completes
     __shared__ int s_hold;
     __shared__ uint32_t s_tmem;
@@ -308,7 +316,7 @@ __global__ void __launch_bounds__(G_THREADS, 1) tc_grouped_gemm(const __grid_con
             asm volatile("mbarrier.init.shared::cta.b64 [%0], 1;" ::"r"(g_smem(&sc_full[s])));
             asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(g_smem(&sc_empty[s])), "r"(C::kScStages));
         }
-        for (int s = 0; s < 2; s++)
+        for (int s = 0; s < 2; s++)          // (at most two buffers on the 16-bit paths)
             asm volatile("mbarrier.init.shared::cta.b64 [%0], 1;" ::"r"(g_smem(&acc_full[s])));
         for (int s = 0; s < C::kAccBufs; s++)
             asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(g_smem(&acc_empty[s])), "r"(G_EPI_WARPS));
@@ -388,8 +396,17 @@ __global__ void __launch_bounds__(G_THREADS, 1) tc_grouped_gemm(const __grid_con
         t.kbase = t.ks * kc;
         const int mn = local / ksplit;
         t.mn = mn;
-        t.m0 = (mn / ntile) * G_BM;
-        t.n0 = (mn % ntile) * per;
+        // Blocks of BN n-tiles x all MT m-tiles, about one wave of the grid: inside a block the
+        // n-tiles of an m-tile are adjacent (CTAs running together share the weight tile through
+        // L2) and every n-tile's activation rows are read by all MT m-tiles within the same wave,
+        // so both operands come from DRAM about once per block instead of the activations once
+        // per m-tile.
+        const int BN = max(1, int(gridDim.x) / MT);
+        const int blk = mn / (MT * BN);
+        const int bnb = min(BN, ntile - blk * BN);               // n-tiles in this block
+        const int idx = mn - blk * MT * BN;
+        t.m0 = (idx / bnb) * G_BM;
+        t.n0 = (blk * BN + idx % bnb) * per;
         t.nval = min(per, n_e - t.n0);
         t.bn = (t.nval + 15) & ~15;
         return t;
@@ -535,9 +552,10 @@ __global__ void __launch_bounds__(G_THREADS, 1) tc_grouped_gemm(const __grid_con
         for (int tile = blockIdx.x; tile < ntiles && !g_aborted(&s_ab); tile += gridDim.x, t++) {
             const GTile T = tile_of(tile);
             const uint32_t idesc = C::kI8 ? g_idesc_i8(T.bn) : g_idesc(T.bn, C::kMmaF16);
-            const int buf = t & 1;
-            uint32_t d = tmem + buf * 128;
-            if (!C::kI8 && t >= 2 && !g_wait_w(g_smem(&acc_empty[buf]), ((t >> 1) - 1) & 1, &s_ab)) {
+            const int buf = C::kI8 ? 0 : t % C::kAccBufs;
+            uint32_t d = tmem + buf * C::kAccCols;
+            if (!C::kI8 && t >= C::kAccBufs &&
+                !g_wait_w(g_smem(&acc_empty[buf]), ((t / C::kAccBufs) - 1) & 1, &s_ab)) {
                 fail();
                 break;
             }
@@ -701,7 +719,7 @@ __global__ void __launch_bounds__(G_THREADS, 1) tc_grouped_gemm(const __grid_con
         int t = 0;
         for (int tile = blockIdx.x; tile < ntiles && !g_aborted(&s_ab); tile += gridDim.x, t++) {
             const GTile T = tile_of(tile);
-            const int buf = t & 1;
+            const int buf = t % C::kAccBufs;
             const int rbase = T.ebase + T.n0;
             // the factor of row c + j (activation row scale, routing weight) sits in lane j;
             // the loads of the first 16 rows' factors and of the global scales go out before the wait
@@ -736,10 +754,10 @@ __global__ void __launch_bounds__(G_THREADS, 1) tc_grouped_gemm(const __grid_con
                 gsc = ldexpf(1.f, -g_int4_row_shift(mg));
                 if (GU) usc = ldexpf(1.f, -g_int4_row_shift(mu));
             }
-            if (!g_wait_w(g_smem(&acc_full[buf]), (t >> 1) & 1, &s_ab, 128)) { fail(); break; }
+            if (!g_wait_w(g_smem(&acc_full[buf]), (t / C::kAccBufs) & 1, &s_ab, 128)) { fail(); break; }
             g_fence_after();
             const int f = T.m0 + q * 32 + lane;
-            const uint32_t acc0 = tmem + lane_addr + buf * 128;
+            const uint32_t acc0 = tmem + lane_addr + buf * C::kAccCols;
             for (int c = 0; c < T.bn; c += 16) {
                 const float rowf = c == 0 ? rowf0 : row_factor(c);
                 uint32_t g[16], u[16];
@@ -1007,7 +1025,9 @@ __global__ void __launch_bounds__(G_THREADS, 1) tc_grouped_gemm(const __grid_con
 __global__ void __launch_bounds__(256) g_prep(const __nv_bfloat16* __restrict__ src, int in_dim,
                                               const int32_t* __restrict__ row_slot, int top_k, int by_token,
                                               int rows, int mode, const float* __restrict__ row_w,
-                                              uint16_t* __restrict__ dst, float* __restrict__ scale) {
+                                              uint16_t* __restrict__ dst, float* __restrict__ scale,
+                                              const int32_t* __restrict__ offsets, int E,
+                                              const float* __restrict__ in_scale) {
     asm volatile("griddepcontrol.wait;" ::: "memory");
     const int row = (blockIdx.x * blockDim.x + threadIdx.x) >> 5, lane = threadIdx.x & 31;
     if (row >= rows) return;
@@ -1017,6 +1037,38 @@ __global__ void __launch_bounds__(256) g_prep(const __nv_bfloat16* __restrict__ 
     const int n16 = in_dim / 8;
     if (mode == 0) {
         for (int i = lane; i < n16; i += 32) d[i] = s[i];
+        return;
+    }
+    if (mode == 4) {
+        // NVFP4 W4A4: the row's expert (the last e with offsets[e] <= row) gives the global scale
+        int lo = 0, hi = E - 1;
+        while (lo < hi) {
+            const int mid = (lo + hi + 1) >> 1;
+            if (offsets[mid] <= row) lo = mid; else hi = mid - 1;
+        }
+        const float g = in_scale[lo];
+        for (int b = lane; b < in_dim / 16; b += 32) {       // a block of 16 per lane and step
+            const uint4 v0 = s[2 * b], v1 = s[2 * b + 1];
+            const float xf[16] = {bf16_lo(v0.x), bf16_hi(v0.x), bf16_lo(v0.y), bf16_hi(v0.y),
+                                  bf16_lo(v0.z), bf16_hi(v0.z), bf16_lo(v0.w), bf16_hi(v0.w),
+                                  bf16_lo(v1.x), bf16_hi(v1.x), bf16_lo(v1.y), bf16_hi(v1.y),
+                                  bf16_lo(v1.z), bf16_hi(v1.z), bf16_lo(v1.w), bf16_hi(v1.w)};
+            uint32_t bytes[8];
+            const uint32_t sb = nv_quant_block16(xf, g, bytes);
+            // e2m1 x e4m3 in f16 (exact: at most 6 significant bits, 2^-10 .. 2688)
+            uint32_t sv = g_e4m3_f16x2(sb);
+            const __half2 s2 = *reinterpret_cast<__half2*>(&sv);
+            uint32_t o[8];
+#pragma unroll
+            for (int j = 0; j < 8; j++) {
+                uint32_t hv = g_e2m1x2_f16x2(bytes[j]);
+                __half2 h = __hmul2(*reinterpret_cast<__half2*>(&hv), s2);
+                o[j] = *reinterpret_cast<uint32_t*>(&h);
+            }
+            d[2 * b] = make_uint4(o[0], o[1], o[2], o[3]);
+            d[2 * b + 1] = make_uint4(o[4], o[5], o[6], o[7]);
+        }
+        if (lane == 0) scale[row] = row_w ? g * row_w[row_slot[row]] : g;
         return;
     }
     float amax = 0.f;
@@ -1174,18 +1226,18 @@ __global__ void __launch_bounds__(256) g_splitk_finish(const float* __restrict__
 // ---------------------------------------------------------------------------
 // Host side
 // ---------------------------------------------------------------------------
-template <int FMT, bool GU>
+template <int FMT, bool GU, bool W>
 static size_t g_smem_bytes(int in_dim, int npk, int nsc) {
-    using C = GCfg<FMT, GU>;
+    using C = GCfg<FMT, GU, W>;
     size_t b = size_t(npk) * C::kPkStageBytes + size_t(C::kBStages) * C::kBStageBytes + 1024;
     if (C::kInt4) b += size_t(nsc) * (C::kNMat * G_BM * (in_dim / 128) * 2 + (C::kI8 ? C::kNMax * (((in_dim / 128) + 3) & ~3) * 4 : 0));
     return b;
 }
 
-template <int FMT, bool GU>
+template <int FMT, bool GU, bool W = false>
 static int g_launch(const GArgs& a, cudaStream_t s) {
-    using C = GCfg<FMT, GU>;
-    auto k = tc_grouped_gemm<FMT, GU>;
+    using C = GCfg<FMT, GU, W>;
+    auto k = tc_grouped_gemm<FMT, GU, W>;
     int dev = 0, sms = 0, optin = 0;
     if (cudaGetDevice(&dev) != cudaSuccess) return MOE_ERR_CUDA;
     if (cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) return MOE_ERR_CUDA;
@@ -1201,13 +1253,13 @@ static int g_launch(const GArgs& a, cudaStream_t s) {
     int npk = C::kPkMax, nsc = 2;
     for (; npk >= 2; npk--) {
         nsc = C::kInt4 ? std::min(G_SC_MAX, std::max(2, (npk + nps - 1) / nps + 1)) : 2;
-        if (g_smem_bytes<FMT, GU>(a.in_dim, npk, nsc) <= room) break;
+        if (g_smem_bytes<FMT, GU, W>(a.in_dim, npk, nsc) <= room) break;
     }
     if (npk < 2) return MOE_ERR_UNSUPPORTED;
     GArgs args = a;
     args.npk = npk;
     args.nsc = nsc;
-    const size_t smem = g_smem_bytes<FMT, GU>(a.in_dim, npk, nsc);
+    const size_t smem = g_smem_bytes<FMT, GU, W>(a.in_dim, npk, nsc);
     if (cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem)) != cudaSuccess)
         return MOE_ERR_CUDA;
     return launch_pdl(k, dim3(sms), dim3(G_THREADS), smem, s, args) == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
@@ -1228,6 +1280,7 @@ int launch_grouped_gemm(const GemvProblem& p, bool gateup, int rows, const GemmB
     if (p.fmt == MOE_FMT_INT4_G128 &&
         ((reinterpret_cast<uintptr_t>(p.s0) & 15u) || (gateup && (reinterpret_cast<uintptr_t>(p.s1) & 15u))))
         return MOE_ERR_INVALID_ARG;
+    if (p.in_scale && p.fmt != MOE_FMT_NVFP4) return MOE_ERR_UNSUPPORTED;
     if (rows <= 0) return MOE_OK;
     G_TRY(g_encoder());
 
@@ -1249,11 +1302,12 @@ int launch_grouped_gemm(const GemvProblem& p, bool gateup, int rows, const GemmB
                            buf.zbuf, p.status) != cudaSuccess)
                 return MOE_ERR_CUDA;
         } else {
-            const int mode = nv ? 2 : (i4 ? 3 : 0);
+            const bool w4a4 = nv && p.in_scale;
+            const int mode = w4a4 ? 4 : (nv ? 2 : (i4 ? 3 : 0));
             const float* row_w = ((nv || i4) && !gateup) ? p.topk_w : nullptr;   // folded into the row scale
             if (launch_pdl(g_prep, dim3((rows * 32 + 255) / 256), dim3(256), 0, s, p.act, in, p.row_slot, p.top_k,
                            p.act_by_token, rows, mode, row_w, reinterpret_cast<uint16_t*>(buf.act_buf),
-                           buf.scale_buf) != cudaSuccess)
+                           buf.scale_buf, p.offsets, p.E, p.in_scale) != cudaSuccess)
                 return MOE_ERR_CUDA;
         }
         bsrc = buf.act_buf;
@@ -1301,10 +1355,15 @@ int launch_grouped_gemm(const GemvProblem& p, bool gateup, int rows, const GemmB
     if (ksplit > 1 && ksplit <= G_KSPLIT_MAX && buf.tile_cnt && 4 * (out / G_BM) * ntile_max <= kTileCounters)
         a.tile_cnt = buf.tile_cnt;
 
+    // wide gate/up tiles (128 token rows) once the experts average more than 64 rows
+    const bool wide = gateup && ksplit == 1 && rows > 64 * E;
     if (i8) return gateup ? g_launch<FMT_INT4_I8, true>(a, s) : g_launch<FMT_INT4_I8, false>(a, s);
-    if (i4) return gateup ? g_launch<MOE_FMT_INT4_G128, true>(a, s) : g_launch<MOE_FMT_INT4_G128, false>(a, s);
-    if (nv) return gateup ? g_launch<MOE_FMT_NVFP4, true>(a, s) : g_launch<MOE_FMT_NVFP4, false>(a, s);
-    const int rc = gateup ? g_launch<MOE_FMT_BF16, true>(a, s) : g_launch<MOE_FMT_BF16, false>(a, s);
+    if (i4) return gateup ? (wide ? g_launch<MOE_FMT_INT4_G128, true, true>(a, s) : g_launch<MOE_FMT_INT4_G128, true>(a, s))
+                          : g_launch<MOE_FMT_INT4_G128, false>(a, s);
+    if (nv) return gateup ? (wide ? g_launch<MOE_FMT_NVFP4, true, true>(a, s) : g_launch<MOE_FMT_NVFP4, true>(a, s))
+                          : g_launch<MOE_FMT_NVFP4, false>(a, s);
+    const int rc = gateup ? (wide ? g_launch<MOE_FMT_BF16, true, true>(a, s) : g_launch<MOE_FMT_BF16, true>(a, s))
+                          : g_launch<MOE_FMT_BF16, false>(a, s);
     if (rc != MOE_OK) return rc;
     if (ksplit > 1 && !a.tile_cnt) {
         const size_t n4 = size_t(rows) * out / 4;

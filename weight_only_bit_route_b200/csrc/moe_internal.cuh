@@ -194,6 +194,7 @@ struct GemvProblem {
     const void* p1; const void* s1; const float* g1;   // up (gate/up only)
     __nv_bfloat16* out;        // [rows, out_dim]
     int32_t* status;
+    const float* in_scale;     // NVFP4 W4A4: activation global scale by expert [E] (nullable)
 };
 
 // Streaming grouped GEMV (decode): routed bank plus an optional BF16 shared
@@ -207,6 +208,8 @@ int launch_combine(const __nv_bfloat16* y_perm, const int32_t* slot_row, int T, 
 
 int launch_quant_int4(const __nv_bfloat16* w, int64_t rows, int64_t cols, int32_t* packed,
                       __nv_bfloat16* scales, cudaStream_t s);
+int launch_quant_nvfp4_act(const __nv_bfloat16* x, int64_t rows, int64_t cols, const float* g, uint8_t* packed,
+                           uint8_t* scales, cudaStream_t s);
 int launch_quant_nvfp4(const __nv_bfloat16* w, int64_t rows, int64_t cols, uint8_t* packed,
                        uint8_t* scales, float* global, uint32_t* amax_slot, cudaStream_t s);
 
@@ -228,7 +231,9 @@ int launch_set_u32(uint32_t* dst, uint32_t v, cudaStream_t s);
 // problem's rows (row r reads activation row row_slot[r] / top_k when
 // act_by_token, else row r) into act_buf ([rows, in] 16-bit) in the kernel's
 // operand order: f16 with a power-of-two row scale (scale_buf, [rows] fp32)
-// for the 4-bit formats (int4: its pairs (0,4) (1,5) (2,6) (3,7) in every 8),
+// for the 4-bit formats (int4: its pairs (0,4) (1,5) (2,6) (3,7) in every 8;
+// NVFP4 W4A4: the NVFP4-quantised values e2m1 x e4m3, exact in f16, with the
+// expert's input scale as the row scale),
 // a plain copy for BF16; the 8-bit int4 path writes three int8 digit rows
 // per row instead.  act_ready (BF16 only): the rows are already in place
 // (row r is row r), no pre-pass runs.

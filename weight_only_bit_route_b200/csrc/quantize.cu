@@ -12,6 +12,7 @@
 // block scale = E4M3(amax_block / (6 * global)); code = E2M1(w / (E4M3 * global)),
 // both conversions round to nearest even and saturate (hardware cvt).
 #include "moe_internal.cuh"
+#include "nvfp4_block.cuh"
 
 namespace moe {
 
@@ -76,24 +77,6 @@ __global__ void amax_kernel(const __nv_bfloat16* __restrict__ w, long long n, ui
     if ((threadIdx.x & 31) == 0) atomicMax(slot, __float_as_uint(m));   // m >= 0: bit order = value order
 }
 
-__device__ __forceinline__ uint32_t f32_to_e4m3_rn_sat(float v) {
-    uint16_t r;
-    asm("cvt.rn.satfinite.e4m3x2.f32 %0, %1, %2;" : "=h"(r) : "f"(0.f), "f"(v));
-    return r & 0xffu;
-}
-
-__device__ __forceinline__ float e4m3_val(uint32_t b) {
-    uint32_t h;
-    asm("{ .reg .b16 t; cvt.u16.u32 t, %1; cvt.rn.f16x2.e4m3x2 %0, t; }" : "=r"(h) : "r"(b));
-    return __half2float(__ushort_as_half(uint16_t(h & 0xffffu)));
-}
-
-__device__ __forceinline__ uint32_t f32x2_to_e2m1x2(float lo, float hi) {
-    uint16_t r;
-    asm("{ .reg .b8 t; cvt.rn.satfinite.e2m1x2.f32 t, %1, %2; cvt.u16.u8 %0, t; }" : "=h"(r) : "f"(hi), "f"(lo));
-    return r & 0xffu;
-}
-
 // one thread per block of 16
 __global__ void quant_nvfp4_kernel(const __nv_bfloat16* __restrict__ w, long long rows, long long cols,
                                    const uint32_t* __restrict__ amax_slot, uint8_t* __restrict__ packed,
@@ -107,27 +90,44 @@ __global__ void quant_nvfp4_kernel(const __nv_bfloat16* __restrict__ w, long lon
     const long long r = bidx / nb, b = bidx % nb;
     const __nv_bfloat16* src = w + r * cols + b * 16;
     float wf[16];
-    float amax_b = 0.f;
-    for (int i = 0; i < 16; i++) {
-        wf[i] = __bfloat162float(src[i]);
-        amax_b = fmaxf(amax_b, fabsf(wf[i]));
-    }
-    uint32_t sb = 0;
-    if (g > 0.f) sb = f32_to_e4m3_rn_sat(__fdiv_rn(amax_b, __fmul_rn(6.0f, g)));
-    scales[r * nb + b] = uint8_t(sb);
-    const float eff = __fmul_rn(e4m3_val(sb), g);
+    for (int i = 0; i < 16; i++) wf[i] = __bfloat162float(src[i]);
+    uint32_t bytes[8];
+    scales[r * nb + b] = uint8_t(nv_quant_block16(wf, g, bytes));
     uint8_t* dst = packed + r * (cols / 2) + b * 8;
-    for (int j = 0; j < 8; j++) {
-        uint32_t byte = 0;
-        if (eff > 0.f) byte = f32x2_to_e2m1x2(__fdiv_rn(wf[2 * j], eff), __fdiv_rn(wf[2 * j + 1], eff));
-        dst[j] = uint8_t(byte);
-    }
+    for (int j = 0; j < 8; j++) dst[j] = uint8_t(bytes[j]);
+}
+
+// Activations ("Step-5-Preview-NVFP4-Local", Modifications: quant_algo NVFP4
+// with an input_scale): row r quantised with its own global g[r]; one thread
+// per block of 16.
+__global__ void quant_nvfp4_act_kernel(const __nv_bfloat16* __restrict__ x, long long rows, long long cols,
+                                       const float* __restrict__ g, uint8_t* __restrict__ packed,
+                                       uint8_t* __restrict__ scales) {
+    const long long nb = cols / 16;
+    const long long bidx = (long long)blockIdx.x * blockDim.x + threadIdx.x;
+    if (bidx >= rows * nb) return;
+    const long long r = bidx / nb, b = bidx % nb;
+    const __nv_bfloat16* src = x + r * cols + b * 16;
+    float xf[16];
+    for (int i = 0; i < 16; i++) xf[i] = __bfloat162float(src[i]);
+    uint32_t bytes[8];
+    scales[r * nb + b] = uint8_t(nv_quant_block16(xf, g[r], bytes));
+    uint8_t* dst = packed + r * (cols / 2) + b * 8;
+    for (int j = 0; j < 8; j++) dst[j] = uint8_t(bytes[j]);
 }
 
 int launch_quant_int4(const __nv_bfloat16* w, int64_t rows, int64_t cols, int32_t* packed,
                       __nv_bfloat16* scales, cudaStream_t s) {
     const long long n = rows * (cols / 128);
     quant_int4_kernel<<<int((n + 127) / 128), 128, 0, s>>>(w, rows, cols, packed, scales);
+    count_launch();
+    return cudaGetLastError() == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
+}
+
+int launch_quant_nvfp4_act(const __nv_bfloat16* x, int64_t rows, int64_t cols, const float* g, uint8_t* packed,
+                           uint8_t* scales, cudaStream_t s) {
+    const long long nb = rows * (cols / 16);
+    quant_nvfp4_act_kernel<<<int((nb + 255) / 256), 256, 0, s>>>(x, rows, cols, g, packed, scales);
     count_launch();
     return cudaGetLastError() == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
 }

@@ -33,7 +33,8 @@ _SZ = ctypes.c_size_t
 
 class QWeight(ctypes.Structure):
     _fields_ = [("fmt", ctypes.c_int32), ("num_experts", ctypes.c_int32), ("out_dim", ctypes.c_int32),
-                ("in_dim", ctypes.c_int32), ("packed", _P), ("scales", _P), ("global_scale", _P)]
+                ("in_dim", ctypes.c_int32), ("packed", _P), ("scales", _P), ("global_scale", _P),
+                ("input_scale", _P)]
 
 
 class Layer(ctypes.Structure):
@@ -68,6 +69,7 @@ _sig("moe_layer_decode", _I, [_P, _I, _P, _P, _P, _SZ, _P])
 _sig("moe_layer_forward", _I, [_P, _I, _P, _P, _P, _SZ, _P])
 _sig("moe_quantize_int4_g128", _I, [_P, _I64, _I64, _P, _P, _P])
 _sig("moe_quantize_nvfp4", _I, [_P, _I64, _I64, _P, _P, _P, _P, _SZ, _P])
+_sig("moe_quantize_nvfp4_act", _I, [_P, _I64, _I64, _P, _P, _P, _P])
 _sig("moe_csf_decode", _I, [_P, _P, _P, _I, _I, _I, _P, _P, _P])
 _sig("moe_csf_encode_workspace_bytes", _SZ, [_I, _I])
 _sig("moe_csf_encode", _I, [_P, _I, _I, _I, _P, _P, _P, _I64, _P, _SZ, _P])
@@ -107,8 +109,9 @@ class Bank:
     bf16:  packed bf16 [E,out,in]
     """
 
-    def __init__(self, fmt, packed, scales=None, global_scale=None, out_dim=None, in_dim=None):
+    def __init__(self, fmt, packed, scales=None, global_scale=None, out_dim=None, in_dim=None, input_scale=None):
         self.fmt, self.packed, self.scales, self.global_scale = fmt, packed, scales, global_scale
+        self.input_scale = input_scale       # NVFP4 W4A4: activation global scale by expert, fp32 [E]
         self.E = packed.shape[0]
         self.out_dim = packed.shape[1] if out_dim is None else out_dim
         mult = {FMT_INT4_G128: 8, FMT_NVFP4: 2, FMT_BF16: 1}[fmt]
@@ -116,11 +119,11 @@ class Bank:
 
     def struct(self):
         return QWeight(self.fmt, self.E, self.out_dim, self.in_dim, _ptr(self.packed),
-                       _ptr(self.scales), _ptr(self.global_scale))
+                       _ptr(self.scales), _ptr(self.global_scale), _ptr(self.input_scale))
 
 
 def _empty_qweight():
-    return QWeight(0, 0, 0, 0, None, None, None)
+    return QWeight(0, 0, 0, 0, None, None, None, None)
 
 
 class MoELayer:
@@ -305,3 +308,14 @@ def csf_decode(fixed, exceptions, starts, R, C, expert_offsets=None, out=None):
     _check("moe_csf_decode", lib.moe_csf_decode(_ptr(fixed), _ptr(exc), _ptr(starts), E, R, C, _ptr(expert_offsets),
                                                 _ptr(sc), _stream()))
     return sc
+
+
+def quantize_nvfp4_act(x, g):
+    """Activations bf16 [rows, cols] with per-row globals g fp32 [rows] (device) ->
+    (packed uint8 [rows, cols/2], scales uint8 [rows, cols/16])."""
+    rows, cols = x.shape
+    packed = torch.empty(rows, cols // 2, dtype=torch.uint8, device=x.device)
+    scales = torch.empty(rows, cols // 16, dtype=torch.uint8, device=x.device)
+    _check("moe_quantize_nvfp4_act",
+           lib.moe_quantize_nvfp4_act(_ptr(x), rows, cols, _ptr(g), _ptr(packed), _ptr(scales), _stream()))
+    return packed, scales
