@@ -39,6 +39,8 @@ from weight_only_bit_route_b200 import synthetic as syn  # noqa: E402
 
 METRIC = "MoE-layer tokens/s on 1 B200; % of HBM peak (decode) / BF16 tensor peak (prefill)"
 UNIT = "tokens/s"
+W4A4_IN_GATEUP = 4.5 / 2688.0       # activation global scales of the W4A4 runs (amax / (6 * 448))
+W4A4_IN_DOWN = 8.0 / 2688.0
 PEAKS_FALLBACK = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 
 
@@ -344,7 +346,7 @@ def step_times(moe, wl, x, layer, ws, steps, flush, stream, clk):
     return out
 
 
-def measure(moe, wl, x, layer, args, flush, stream, clk, pk, pk_kind, per_step=True):
+def measure(moe, wl, x, layer, args, flush, stream, clk, pk, pk_kind, per_step=True, fp4=False):
     """Layer timing (+ dominant-kernel roofline and per-step times) of one workload."""
     T = wl.T
     ws = moe.workspace(T, wl.H, wl.E, wl.F, wl.k)
@@ -389,9 +391,13 @@ def measure(moe, wl, x, layer, args, flush, stream, clk, pk, pk_kind, per_step=T
     else:
         kflops = 2 * 2 * wl.F * wl.H * R
         achieved = kflops / (k_ms * 1e-3) / 1e12
-        roof = {"bound": "tensor", "achieved": round(achieved, 1), "peak": pk["bf16_tflops"], "unit": "TFLOP/s",
-                "frac": round(achieved / pk["bf16_tflops"], 4), "traffic": traffic, "kernel": kernel_name,
-                "algorithmic_flops": kflops, "kernel_ms": round(k_ms, 5), "peak_source": f"{pk_kind} bf16_tflops"}
+        # W4A4 runs on the FP4 tensor cores: its peak is the measured BF16 one times the nominal
+        # dense ratio FP4 / BF16 (9 / 2.25 PFLOP/s)
+        kpeak = pk["bf16_tflops"] * (4.0 if fp4 else 1.0)
+        roof = {"bound": "tensor", "achieved": round(achieved, 1), "peak": round(kpeak, 1), "unit": "TFLOP/s",
+                "frac": round(achieved / kpeak, 4), "traffic": traffic, "kernel": kernel_name,
+                "algorithmic_flops": kflops, "kernel_ms": round(k_ms, 5),
+                "peak_source": f"{pk_kind} bf16_tflops" + (" x 4 (FP4 / BF16 nominal dense ratio)" if fp4 else "")}
         tf = lflops / (ms * 1e-3) / 1e12
         layer_roof = {"bound": "tensor", "algorithmic_flops": lflops, "achieved_tflops": round(tf, 1),
                       "frac_burst": round(tf / pk["bf16_tflops"], 4),
@@ -412,8 +418,9 @@ def main():
     ap.add_argument("--steps", type=int, default=200)
     ap.add_argument("--warmup", type=int, default=10)
     ap.add_argument("--config", type=int, default=1, help="the headline workload")
-    ap.add_argument("--per-config", default="2,3,4",
-                    help="other workloads measured into per_config (comma list, or 'none')")
+    ap.add_argument("--per-config", default="2,3,4,2w,4w",
+                    help="other workloads measured into per_config (comma list; a trailing 'w' runs an NVFP4 "
+                         "workload as W4A4, activations quantised on the fly; or 'none')")
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
     args = ap.parse_args()
@@ -422,8 +429,8 @@ def main():
     world = int(os.environ.get("WORLD_SIZE", "1"))
     local_rank = int(os.environ.get("LOCAL_RANK", "0"))
     wl = syn.WORKLOADS[args.config]
-    others = [] if args.per_config == "none" else [int(c) for c in args.per_config.split(",") if c.strip()]
-    others = [c for c in others if c != args.config]
+    others = [] if args.per_config == "none" else [c.strip() for c in args.per_config.split(",") if c.strip()]
+    others = [c for c in others if c != str(args.config)]
 
     if args.impl == "reference":
         run_reference(args, wl, rank, world)
@@ -487,9 +494,21 @@ def main():
 
         per_config = {}
         for c in others:
-            w2 = syn.WORKLOADS[c]
-            res = measure(moe, w2, x_for(w2), layer_for(w2), args, flush, stream, clk, pk, pk_kind)[0]
-            per_config[str(c)] = res
+            w4a4 = c.endswith("w")
+            w2 = syn.WORKLOADS[int(c.rstrip("w"))]
+            lay = layer_for(w2)
+            if w4a4:
+                if w2.fmt != "nvfp4":
+                    continue
+                # static activation scales standing in for calibrated ones: the inputs' typical
+                # amax / (6 * 448) (x ~ N(0, 1) over 4096 elements; h of these weights stays below ~8)
+                lay.gate.input_scale = torch.full((w2.E,), W4A4_IN_GATEUP, dtype=torch.float32, device="cuda")
+                lay.down.input_scale = torch.full((w2.E,), W4A4_IN_DOWN, dtype=torch.float32, device="cuda")
+            res = measure(moe, w2, x_for(w2), lay, args, flush, stream, clk, pk, pk_kind, fp4=w4a4)[0]
+            if w4a4:
+                res["workload"] += " (W4A4: NVFP4 activations, static input scales)"
+                lay.gate.input_scale = lay.down.input_scale = None
+            per_config[c] = res
             torch.cuda.empty_cache()
         layer = layer_for(wl)          # restore the headline workload's bias for the CPU leg
 

@@ -100,6 +100,13 @@ constexpr int G_EPI_WARPS = 4;
 // the per-weight work, and the accumulation itself is exact.  Internal
 // format value.
 constexpr int FMT_INT4_I8 = 3;
+// NVFP4 W4A4 on the block-scaled FP4 tensor cores: weights and activations
+// both E2M1 with E4M3 scales per 16, tcgen05.mma.kind::mxf4nvf4 with
+// scale_vec::4X.  A (weights) and B (the quantised activations) are read from
+// shared memory as stored, K = 64 per instruction; the scale factors go to
+// tensor memory by tcgen05.cp.  Internal format value.
+constexpr int FMT_NVFP4_A4 = 4;
+constexpr int G_SF_RING = 4;                 // A4: scale-factor slots (shared and tensor memory)
 
 // W (wide): gate/up tiles of up to 128 token rows instead of 64, for batches
 // whose experts hold many rows: each dequantised weight then serves twice the
@@ -108,43 +115,52 @@ constexpr int FMT_INT4_I8 = 3;
 template <int FMT, bool GU, bool W = false>
 struct GCfg {
     static constexpr bool kI8 = FMT == FMT_INT4_I8;
+    static constexpr bool kA4 = FMT == FMT_NVFP4_A4;
     static constexpr bool kInt4 = FMT == MOE_FMT_INT4_G128 || kI8;
-    static constexpr bool kTmemA = FMT != MOE_FMT_BF16;
+    static constexpr bool kTmemA = FMT != MOE_FMT_BF16 && !kA4;     // A dequantised into tensor memory
+    static constexpr bool kPacked = kTmemA || kA4;                    // 4-bit weight stages (128 B = K 256 per row)
     static constexpr bool kWide = W && GU && !kI8;
     static constexpr int kNMat = GU ? 2 : 1;
     static constexpr int kNMax = kI8 ? 5 : (GU ? (kWide ? 128 : 64) : 128);   // token rows per tile
     static constexpr int kUpCol = kWide ? 128 : 64;                 // 16-bit paths: up accumulator within a buffer
     // K per MMA step: 8-bit down steps are K = 512, so that the per-step fixed cost of the
     // issuer and the unpack warps covers 32 KB of weights, as a gate/up step does
-    static constexpr int kSK = kI8 ? (GU ? 256 : 512) : 128;
+    static constexpr int kSK = kI8 ? (GU ? 256 : 512) : (kA4 ? 256 : 128);
     static constexpr int kGroups = kSK / 128;                       // i8: scale groups per MMA stage
     static constexpr int kAccCols = kI8 ? kGroups * kNMat * 16 : (kWide ? 256 : 128);   // one accumulator buffer
     // Tensor memory: accumulators in [0, kABase), A stages in [kABase, 512).  The
     // 8-bit path keeps few small accumulators and gives the A ring the room
     // (its dequantise -> MMA -> free cycle is long against a step).
-    static constexpr int kAccBufs = kI8 ? 128 / kAccCols : (kWide && kTmemA ? 1 : (kWide ? 2 : 256 / kAccCols));
+    static constexpr int kAccBufs = kI8 ? 128 / kAccCols : (kWide && kPacked ? 1 : (kWide ? 2 : 256 / kAccCols));
     static constexpr int kABase = kAccBufs * kAccCols;
-    static constexpr int kMmaK = kI8 ? 32 : 16;                     // K per MMA instruction
-    static constexpr int kPkK = kTmemA ? (kI8 ? kSK : 256) : 128;   // K per weight stage
-    static constexpr int kBoxes = kTmemA ? kPkK / 256 : 2;          // 128-byte-wide TMA boxes per matrix and stage
-    static constexpr int kMatBytes = kTmemA ? G_BM * kPkK / 2 : G_BM * 256;   // one matrix of a weight stage
-    static constexpr int kNvScBytes = FMT == MOE_FMT_NVFP4 ? G_BM * 16 : 0;
+    static constexpr int kMmaK = kI8 ? 32 : (kA4 ? 64 : 16);        // K per MMA instruction
+    static constexpr int kPkK = kPacked ? (kI8 ? kSK : 256) : 128;  // K per weight stage
+    static constexpr int kBoxes = kPacked ? kPkK / 256 : 2;         // 128-byte-wide TMA boxes per matrix and stage
+    static constexpr int kMatBytes = kPacked ? G_BM * kPkK / 2 : G_BM * 256;   // one matrix of a weight stage
+    static constexpr int kNvScBytes = (FMT == MOE_FMT_NVFP4 || kA4) ? G_BM * 16 : 0;
     static constexpr int kPkStageBytes = kNMat * (kMatBytes + kNvScBytes);
     static constexpr int kPkMax = 12;                               // weight stages: as many as fit, up to this
     static constexpr int kScStages = kI8 ? G_EPI_WARPS : G_DQ_WARPS;     // readers of the int4 scale buffer
     static constexpr int kBAtom = (kI8 ? 16 : kNMax) * 128;         // 128 bytes of K for every B row
-    static constexpr int kBAtoms = kI8 ? kSK / 128 : 2;             // 128-byte K slices per B stage
-    static constexpr int kBStageBytes = kBAtoms * kBAtom;
+    static constexpr int kBAtoms = kI8 ? kSK / 128 : (kA4 ? 1 : 2); // 128-byte K slices per B stage
+    static constexpr int kBScBytes = kA4 ? kNMax * 16 : 0;          // A4: the B rows' raw scale factors
+    static constexpr int kBStageBytes = kBAtoms * kBAtom + kBScBytes;
+    // A4: per step the scale factors of kNMat weight tiles and the B tile, as 4 chunks (K 64 each)
+    // of 512 bytes apiece in shared memory, and 4 tensor-memory columns per chunk
+    static constexpr int kSfChunks = kA4 ? (kNMat + 1) * 4 : 0;
+    static constexpr int kSfSlotBytes = kSfChunks * 512;
+    static constexpr int kSfSlotCols = kSfChunks * 4;
     // i8 stages are small: cover the copy latency; wide stages are large: fit shared memory
     static constexpr int kBStages = kI8 ? (GU ? 6 : 4) : (kWide ? (kTmemA ? 3 : 2) : 4);
     static constexpr int kAColsK = kI8 ? kSK / 4 : 64;              // TMEM columns of one matrix's A stage
     static constexpr int kAStageCols = kNMat * kAColsK;
-    static constexpr int kAStages = kTmemA ? (512 - kABase) / kAStageCols : 1;   // (BF16: none used)
+    static constexpr int kAStages = kTmemA ? (512 - kABase) / kAStageCols : 1;   // (BF16, A4: none used)
     static constexpr int kAPerPk = kPkK / kSK;                      // A stages per weight stage (2, or 1 for i8)
     static constexpr int kChunkCols = 16;                           // 16-bit paths: TMEM columns of one packed chunk
     static constexpr int kDqArrivals = kI8 ? G_DQ_WARPS / 2 : G_DQ_WARPS;  // warps that fill one stage
     static constexpr bool kMmaF16 = FMT == MOE_FMT_NVFP4 || FMT == MOE_FMT_INT4_G128;   // f16 operands
     static_assert(kABase <= 512 && (!kTmemA || kAStages >= 2), "tensor memory layout");
+    static_assert(!kA4 || kABase + G_SF_RING * kSfSlotCols <= 512, "A4 scale-factor ring");
 };
 
 constexpr int G_DONE = 16;                                          // "stage done" barrier ring
@@ -157,6 +173,7 @@ struct GArgs {
     CUtensorMap tm_p0, tm_p1;        // packed (or BF16) weights of gate (or down) and up
     CUtensorMap tm_s0, tm_s1;        // NVFP4 block scales
     CUtensorMap tm_b[G_NB_MAPS];     // activation operand rows, box height 16*(i+1)
+    CUtensorMap tm_bs[G_NB_MAPS];    // A4: the activation rows' scale factors, box height 16*(i+1)
     const uint8_t* sc0;              // int4 scales (bf16), bulk-copied per tile
     const uint8_t* sc1;
     const float* g0;                 // NVFP4 per-expert global scales
@@ -276,6 +293,7 @@ __global__ void __launch_bounds__(G_THREADS, 1) tc_grouped_gemm(const __grid_con
     __shared__ __align__(8) uint64_t sc_full[G_SC_MAX], sc_empty[G_SC_MAX];
     __shared__ __align__(8) uint64_t acc_full[2], acc_empty[2], drain;
     __shared__ __align__(8) uint64_t hold_bar;        // failure testing: a barrier nothing completes
+    __shared__ __align__(8) uint64_t sf_full[G_SF_RING];   // A4: a step's scale-factor chunks are in place
     __shared__ int s_hold;
     __shared__ uint32_t s_tmem;
     __shared__ int s_active[kMaxE];
@@ -322,6 +340,8 @@ __global__ void __launch_bounds__(G_THREADS, 1) tc_grouped_gemm(const __grid_con
             asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(g_smem(&acc_empty[s])), "r"(G_EPI_WARPS));
         asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(g_smem(&drain)), "r"(C::kI8 ? 2 : 1));
         asm volatile("mbarrier.init.shared::cta.b64 [%0], 1;" ::"r"(g_smem(&hold_bar)));
+        for (int s = 0; s < G_SF_RING; s++)       // A4: one arrival per scale-factor warp
+            asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(g_smem(&sf_full[s])), "r"(4));
         asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
         s_ab.flag = 0;
         s_ab.limit_ns = G_WAIT_NS;
@@ -378,6 +398,7 @@ __global__ void __launch_bounds__(G_THREADS, 1) tc_grouped_gemm(const __grid_con
     uint8_t* pk = smem + ((1024u - (g_smem(smem) & 1023u)) & 1023u);
     uint8_t* bring = pk + NPK * C::kPkStageBytes;
     uint8_t* scbuf = bring + C::kBStages * C::kBStageBytes;         // int4: NSC buffers of sc_buf_bytes
+    uint8_t* sfring = scbuf;                                        // A4: G_SF_RING slots of kSfSlotBytes (no int4 buffers)
 
     auto tile_of = [&](int tile) {
         int lo = 0, hi = nact - 1;
@@ -443,6 +464,7 @@ __global__ void __launch_bounds__(G_THREADS, 1) tc_grouped_gemm(const __grid_con
             for (int ps = 0; ps < NPS; ps++, pc++) {
                 const int s = pc % NPK;
                 // 4-bit stages are freed by the dequantisation warps, BF16 ones by the MMA step
+                // (A4 stages too: the MMA reads them from shared memory)
                 if (pc >= NPK && !(C::kTmemA ? g_wait_w(g_smem(&pk_empty[s]), ((pc / NPK) - 1) & 1, &s_ab, 32)
                                              : g_wait_w(g_smem(&done[(pc - NPK) % G_DONE]), ((pc - NPK) / G_DONE) & 1,
                                                         &s_ab, 32))) {
@@ -453,7 +475,7 @@ __global__ void __launch_bounds__(G_THREADS, 1) tc_grouped_gemm(const __grid_con
                 const uint32_t st = g_smem(pk + s * C::kPkStageBytes);
                 if (g_elect()) {
                     g_expect(bar, C::kPkStageBytes);
-                    if (C::kTmemA) {
+                    if (C::kPacked) {
                         // 4-bit: 128 bytes of each row = K 256 per box, kBoxes boxes side by side
 #pragma unroll
                         for (int h = 0; h < C::kBoxes; h++) {
@@ -461,7 +483,7 @@ __global__ void __launch_bounds__(G_THREADS, 1) tc_grouped_gemm(const __grid_con
                             g_tma2d(st + h * (G_BM * 128), &a.tm_p0, x, row0, bar);
                             if (GU) g_tma2d(st + C::kMatBytes + h * (G_BM * 128), &a.tm_p1, x, row0, bar);
                         }
-                        if (FMT == MOE_FMT_NVFP4) {
+                        if (FMT == MOE_FMT_NVFP4 || C::kA4) {
                             const uint32_t ss = st + C::kNMat * C::kMatBytes;
                             g_tma2d(ss, &a.tm_s0, T.kbase / 16 + ps * 16, row0, bar);
                             if (GU) g_tma2d(ss + C::kNvScBytes, &a.tm_s1, T.kbase / 16 + ps * 16, row0, bar);
@@ -524,9 +546,16 @@ __global__ void __launch_bounds__(G_THREADS, 1) tc_grouped_gemm(const __grid_con
                     continue;
                 }
                 if (g_elect()) {
-                    g_expect(bar, uint32_t(T.bn) * 256u);
-                    g_tma2d(st, map, T.kbase + ks * C::kSK, row0, bar);
-                    g_tma2d(st + C::kBAtom, map, T.kbase + ks * C::kSK + 64, row0, bar);
+                    if constexpr (C::kA4) {
+                        // K 256 of packed E2M1 (128 bytes per row, swizzled) and the rows' 16 scale bytes
+                        g_expect(bar, uint32_t(T.bn) * (128u + 16u));
+                        g_tma2d(st, map, (T.kbase + ks * C::kSK) / 2, row0, bar);
+                        g_tma2d(st + C::kBAtom, &a.tm_bs[T.bn / 16 - 1], (T.kbase + ks * C::kSK) / 16, row0, bar);
+                    } else {
+                        g_expect(bar, uint32_t(T.bn) * 256u);
+                        g_tma2d(st, map, T.kbase + ks * C::kSK, row0, bar);
+                        g_tma2d(st + C::kBAtom, map, T.kbase + ks * C::kSK + 64, row0, bar);
+                    }
                 }
                 __syncwarp();
             }
@@ -575,6 +604,10 @@ __global__ void __launch_bounds__(G_THREADS, 1) tc_grouped_gemm(const __grid_con
                 } else {
                     if (!g_wait_w(g_smem(&pk_full[pc % NPK]), (pc / NPK) & 1, &s_ab)) { ok = false; break; }
                 }
+                if (C::kA4 && !g_wait_w(g_smem(&sf_full[bc % G_SF_RING]), (bc / G_SF_RING) & 1, &s_ab)) {
+                    ok = false;
+                    break;
+                }
                 if (C::kI8) {
                     // every step into the next accumulator buffer, freed by the epilogue
                     const int bi = bc % C::kAccBufs;
@@ -586,7 +619,27 @@ __global__ void __launch_bounds__(G_THREADS, 1) tc_grouped_gemm(const __grid_con
                 const uint32_t b0 = g_smem(bring + sb * C::kBStageBytes);
                 const uint32_t at = tmem + C::kABase + sa * C::kAStageCols;
                 const uint32_t a0 = g_smem(pk + (pc % NPK) * C::kPkStageBytes);
-                if (g_elect()) {
+                if constexpr (C::kA4) {
+                    // scale factors of this step into tensor-memory slot bc % G_SF_RING (A chunks of each
+                    // matrix, then B's), then per K 64 one block-scaled MMA per matrix
+                    const uint32_t slot = tmem + C::kABase + (bc % G_SF_RING) * C::kSfSlotCols;
+                    const uint32_t sfs = g_smem(sfring + (bc % G_SF_RING) * C::kSfSlotBytes);
+                    const uint32_t idesc4 = g_idesc_mxf4(T.bn);
+                    if (g_elect()) {
+#pragma unroll
+                        for (int c = 0; c < C::kSfChunks; c++) g_cp_sf(slot + 4 * c, g_desc_sf(sfs + c * 512));
+#pragma unroll
+                        for (int k = 0; k < 4; k++) {
+                            const uint64_t bd = g_desc(b0 + k * 32);
+                            const uint32_t acc = (k > 0 || ks > 0) ? 1u : 0u;
+                            const uint32_t sfb = slot + C::kNMat * 16 + 4 * k;
+                            g_mma_mxf4(d, g_desc(a0 + k * 32), bd, idesc4, acc, slot + 4 * k, sfb);
+                            if (GU) g_mma_mxf4(d + C::kUpCol, g_desc(a0 + C::kMatBytes + k * 32), bd, idesc4, acc,
+                                               slot + 16 + 4 * k, sfb);
+                        }
+                        g_commit(g_smem(&done[bc % G_DONE]));
+                    }
+                } else if (g_elect()) {
 #pragma unroll
                     for (int k = 0; k < C::kSK / C::kMmaK; k++) {
                         const uint64_t bd = g_desc(b0 + (k >> 2) * C::kBAtom + (k & 3) * 32);
@@ -727,15 +780,15 @@ __global__ void __launch_bounds__(G_THREADS, 1) tc_grouped_gemm(const __grid_con
                 float v = 1.f;
                 const int nn = c + (lane & 15);
                 if (nn < T.nval) {
-                    if (C::kMmaF16) v = a.act_scale[rbase + nn];
+                    if (C::kMmaF16 || C::kA4) v = a.act_scale[rbase + nn];
                     // 4-bit formats: the pre-pass folded the routing weight into the row scale
-                    if (!GU && a.topk_w && !C::kMmaF16) v *= a.topk_w[a.row_slot[rbase + nn]];
+                    if (!GU && a.topk_w && !(C::kMmaF16 || C::kA4)) v *= a.topk_w[a.row_slot[rbase + nn]];
                 }
                 return v;
             };
             float rowf0 = row_factor(0);
             float gsc = 1.f, usc = 1.f;
-            if (FMT == MOE_FMT_NVFP4) { gsc = a.g0[T.e]; if (GU) usc = a.g1[T.e]; }
+            if (FMT == MOE_FMT_NVFP4 || C::kA4) { gsc = a.g0[T.e]; if (GU) usc = a.g1[T.e]; }
             if (FMT == MOE_FMT_INT4_G128) {
                 // undo the dequantisation's power of two of this weight row (gate and up separately)
                 const int row = T.e * a.out_dim + T.m0 + q * 32 + lane;
@@ -838,6 +891,47 @@ __global__ void __launch_bounds__(G_THREADS, 1) tc_grouped_gemm(const __grid_con
                 }
             }
         }
+    } else if (warp >= 8 && warp < 12 && C::kA4) {
+        // ---------------- A4: scale factors into the MMA's chunk layout ----------------
+        // Thread (warp w, lane l) takes row r = 32 (w % 4) + l of the step's weight tiles and of
+        // its B tile.  A chunk (K 64: four 16-element blocks) of 128 rows is 512 bytes with the
+        // four factors of row 32 m1 + m0 at 16 m0 + 4 m1; the factors of one chunk are one word
+        // of the row's 16 raw bytes.  Rows past the tile's token rows read as zero.
+        const int q = warp & 3;
+        const int r = q * 32 + lane;
+        const uint32_t at = 16u * uint32_t(r & 31) + 4u * uint32_t(r >> 5);
+        uint32_t bc = 0;
+        bool ok = true;
+        for (int tile = blockIdx.x; tile < ntiles && ok && !g_aborted(&s_ab); tile += gridDim.x) {
+            const GTile T = tile_of(tile);
+            for (int ks = 0; ks < KS; ks++, bc++) {
+                if (!g_wait_w(g_smem(&pk_full[bc % NPK]), (bc / NPK) & 1, &s_ab) ||
+                    !g_wait_w(g_smem(&b_full[bc % C::kBStages]), (bc / C::kBStages) & 1, &s_ab) ||
+                    (bc >= uint32_t(G_SF_RING) && !g_wait_w(g_smem(&done[(bc - G_SF_RING) % G_DONE]),
+                                                            ((bc - G_SF_RING) / G_DONE) & 1, &s_ab))) {
+                    ok = false;
+                    break;
+                }
+                const uint8_t* wsc = pk + (bc % NPK) * C::kPkStageBytes + C::kNMat * C::kMatBytes;
+                const uint8_t* bsc = bring + (bc % C::kBStages) * C::kBStageBytes + C::kBAtom;
+                uint8_t* slot = sfring + (bc % G_SF_RING) * C::kSfSlotBytes;
+#pragma unroll
+                for (int m = 0; m < C::kNMat; m++) {
+                    const uint4 v = *reinterpret_cast<const uint4*>(wsc + m * C::kNvScBytes + r * 16);
+                    const uint32_t w4[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+                    for (int c = 0; c < 4; c++) *reinterpret_cast<uint32_t*>(slot + (m * 4 + c) * 512 + at) = w4[c];
+                }
+                const uint4 v = r < T.bn ? *reinterpret_cast<const uint4*>(bsc + r * 16) : make_uint4(0, 0, 0, 0);
+                const uint32_t w4[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+                for (int c = 0; c < 4; c++) *reinterpret_cast<uint32_t*>(slot + (C::kNMat * 4 + c) * 512 + at) = w4[c];
+                g_fence_proxy_async();                  // generic stores, read by tcgen05.cp
+                __syncwarp();
+                if (lane == 0) g_arrive(g_smem(&sf_full[bc % G_SF_RING]));
+            }
+        }
+        if (!ok) fail();
     } else if (warp >= 8 && C::kI8) {
         // ---------------- 8-bit int4 unpacking ----------------
         // Two groups of four warps take alternate weight stages; a warp unpacks
@@ -1016,6 +1110,9 @@ __global__ void __launch_bounds__(G_THREADS, 1) tc_grouped_gemm(const __grid_con
 //   mode 2: f16 times 2^-e in natural order (NVFP4 weights);
 //   mode 3: f16 times 2^-e, pairs (0,4) (1,5) (2,6) (3,7) in every 8 (int4
 //           weights, the order of their dequantised pairs);
+//   mode 5: NVFP4 W4A4 activations: each row quantised with its expert's
+//           input scale g (the row's expert found in offsets), codes and
+//           block scales as stored, row scale g;
 // with e the exponent that puts the row's largest |x| 2^-e in [2^13, 2^14):
 // every bf16 value becomes an f16 exactly (bf16 has 8 significant bits, f16
 // 11) unless it is 2^27 below the row's largest.  The row scale 2^e (times
@@ -1027,7 +1124,7 @@ __global__ void __launch_bounds__(256) g_prep(const __nv_bfloat16* __restrict__ 
                                               int rows, int mode, const float* __restrict__ row_w,
                                               uint16_t* __restrict__ dst, float* __restrict__ scale,
                                               const int32_t* __restrict__ offsets, int E,
-                                              const float* __restrict__ in_scale) {
+                                              const float* __restrict__ in_scale, size_t sc_off) {
     asm volatile("griddepcontrol.wait;" ::: "memory");
     const int row = (blockIdx.x * blockDim.x + threadIdx.x) >> 5, lane = threadIdx.x & 31;
     if (row >= rows) return;
@@ -1039,34 +1136,27 @@ __global__ void __launch_bounds__(256) g_prep(const __nv_bfloat16* __restrict__ 
         for (int i = lane; i < n16; i += 32) d[i] = s[i];
         return;
     }
-    if (mode == 4) {
-        // NVFP4 W4A4: the row's expert (the last e with offsets[e] <= row) gives the global scale
+    if (mode == 5) {
+        // NVFP4 W4A4 on the FP4 tensor cores: the codes (two per byte, even element low) and the
+        // E4M3 block scales as stored, [rows, in / 2] then [rows, in / 16] (dst + sc_off bytes)
         int lo = 0, hi = E - 1;
         while (lo < hi) {
             const int mid = (lo + hi + 1) >> 1;
             if (offsets[mid] <= row) lo = mid; else hi = mid - 1;
         }
         const float g = in_scale[lo];
-        for (int b = lane; b < in_dim / 16; b += 32) {       // a block of 16 per lane and step
+        uint8_t* d8 = reinterpret_cast<uint8_t*>(dst) + size_t(row) * (in_dim / 2);
+        uint8_t* sc8 = reinterpret_cast<uint8_t*>(dst) + sc_off + size_t(row) * (in_dim / 16);
+        for (int b = lane; b < in_dim / 16; b += 32) {
             const uint4 v0 = s[2 * b], v1 = s[2 * b + 1];
             const float xf[16] = {bf16_lo(v0.x), bf16_hi(v0.x), bf16_lo(v0.y), bf16_hi(v0.y),
                                   bf16_lo(v0.z), bf16_hi(v0.z), bf16_lo(v0.w), bf16_hi(v0.w),
                                   bf16_lo(v1.x), bf16_hi(v1.x), bf16_lo(v1.y), bf16_hi(v1.y),
                                   bf16_lo(v1.z), bf16_hi(v1.z), bf16_lo(v1.w), bf16_hi(v1.w)};
             uint32_t bytes[8];
-            const uint32_t sb = nv_quant_block16(xf, g, bytes);
-            // e2m1 x e4m3 in f16 (exact: at most 6 significant bits, 2^-10 .. 2688)
-            uint32_t sv = g_e4m3_f16x2(sb);
-            const __half2 s2 = *reinterpret_cast<__half2*>(&sv);
-            uint32_t o[8];
-#pragma unroll
-            for (int j = 0; j < 8; j++) {
-                uint32_t hv = g_e2m1x2_f16x2(bytes[j]);
-                __half2 h = __hmul2(*reinterpret_cast<__half2*>(&hv), s2);
-                o[j] = *reinterpret_cast<uint32_t*>(&h);
-            }
-            d[2 * b] = make_uint4(o[0], o[1], o[2], o[3]);
-            d[2 * b + 1] = make_uint4(o[4], o[5], o[6], o[7]);
+            sc8[b] = uint8_t(nv_quant_block16(xf, g, bytes));
+            *reinterpret_cast<uint2*>(d8 + 8 * b) = make_uint2(bytes[0] | (bytes[1] << 8) | (bytes[2] << 16) | (bytes[3] << 24),
+                                                              bytes[4] | (bytes[5] << 8) | (bytes[6] << 16) | (bytes[7] << 24));
         }
         if (lane == 0) scale[row] = row_w ? g * row_w[row_slot[row]] : g;
         return;
@@ -1231,6 +1321,7 @@ static size_t g_smem_bytes(int in_dim, int npk, int nsc) {
     using C = GCfg<FMT, GU, W>;
     size_t b = size_t(npk) * C::kPkStageBytes + size_t(C::kBStages) * C::kBStageBytes + 1024;
     if (C::kInt4) b += size_t(nsc) * (C::kNMat * G_BM * (in_dim / 128) * 2 + (C::kI8 ? C::kNMax * (((in_dim / 128) + 3) & ~3) * 4 : 0));
+    if (C::kA4) b += size_t(G_SF_RING) * C::kSfSlotBytes;
     return b;
 }
 
@@ -1286,6 +1377,8 @@ int launch_grouped_gemm(const GemvProblem& p, bool gateup, int rows, const GemmB
 
     const int in = p.in_dim, out = p.out_dim, E = p.E;
     const bool nv = p.fmt == MOE_FMT_NVFP4, i4 = p.fmt == MOE_FMT_INT4_G128;
+    const bool a4 = nv && p.in_scale != nullptr;                      // W4A4 on the FP4 tensor cores
+    const size_t a4_sc_off = align256(size_t(rows) * (in / 2));     // A4: scale bytes after the codes
     // the 8-bit down GEMM steps in K = 512; other widths take the 16-bit int4 path
     const bool i8 = i4 && buf.i8 && (gateup || in % 512 == 0);
     if (i8 && (!buf.zbuf || !buf.scale_buf || !buf.act_buf || ksplit > 1)) return MOE_ERR_UNSUPPORTED;
@@ -1302,12 +1395,11 @@ int launch_grouped_gemm(const GemvProblem& p, bool gateup, int rows, const GemmB
                            buf.zbuf, p.status) != cudaSuccess)
                 return MOE_ERR_CUDA;
         } else {
-            const bool w4a4 = nv && p.in_scale;
-            const int mode = w4a4 ? 4 : (nv ? 2 : (i4 ? 3 : 0));
+            const int mode = a4 ? 5 : (nv ? 2 : (i4 ? 3 : 0));
             const float* row_w = ((nv || i4) && !gateup) ? p.topk_w : nullptr;   // folded into the row scale
             if (launch_pdl(g_prep, dim3((rows * 32 + 255) / 256), dim3(256), 0, s, p.act, in, p.row_slot, p.top_k,
                            p.act_by_token, rows, mode, row_w, reinterpret_cast<uint16_t*>(buf.act_buf),
-                           buf.scale_buf, p.offsets, p.E, p.in_scale) != cudaSuccess)
+                           buf.scale_buf, p.offsets, p.E, p.in_scale, a4_sc_off) != cudaSuccess)
                 return MOE_ERR_CUDA;
         }
         bsrc = buf.act_buf;
@@ -1328,11 +1420,20 @@ int launch_grouped_gemm(const GemvProblem& p, bool gateup, int rows, const GemmB
         G_TRY(g_map(&a.tm_s0, false, p.s0, in / 16, wrows, uint64_t(in) / 16, 16, 128, false));
         if (gateup) G_TRY(g_map(&a.tm_s1, false, p.s1, in / 16, wrows, uint64_t(in) / 16, 16, 128, false));
     }
-    if (i8)
+    if (i8) {
         a.bdig = static_cast<const uint8_t*>(bsrc);
-    else
+    } else if (a4) {
+        const uint8_t* codes = static_cast<const uint8_t*>(bsrc);
+        for (int i = 0; i < G_NB_MAPS; i++) {
+            G_TRY(g_map(&a.tm_b[i], false, codes, in / 2, uint64_t(rows), uint64_t(in) / 2, 128, uint32_t(16 * (i + 1)),
+                        true));
+            G_TRY(g_map(&a.tm_bs[i], false, codes + a4_sc_off, in / 16, uint64_t(rows), uint64_t(in) / 16, 16,
+                        uint32_t(16 * (i + 1)), false));
+        }
+    } else {
         for (int i = 0; i < G_NB_MAPS; i++)
             G_TRY(g_map(&a.tm_b[i], true, bsrc, in, uint64_t(rows), uint64_t(in) * 2, 64, uint32_t(16 * (i + 1)), true));
+    }
     a.sc0 = reinterpret_cast<const uint8_t*>(p.s0);
     a.sc1 = reinterpret_cast<const uint8_t*>(p.s1);
     a.g0 = p.g0;
@@ -1360,6 +1461,8 @@ int launch_grouped_gemm(const GemvProblem& p, bool gateup, int rows, const GemmB
     if (i8) return gateup ? g_launch<FMT_INT4_I8, true>(a, s) : g_launch<FMT_INT4_I8, false>(a, s);
     if (i4) return gateup ? (wide ? g_launch<MOE_FMT_INT4_G128, true, true>(a, s) : g_launch<MOE_FMT_INT4_G128, true>(a, s))
                           : g_launch<MOE_FMT_INT4_G128, false>(a, s);
+    if (a4) return gateup ? (wide ? g_launch<FMT_NVFP4_A4, true, true>(a, s) : g_launch<FMT_NVFP4_A4, true>(a, s))
+                          : g_launch<FMT_NVFP4_A4, false>(a, s);
     if (nv) return gateup ? (wide ? g_launch<MOE_FMT_NVFP4, true, true>(a, s) : g_launch<MOE_FMT_NVFP4, true>(a, s))
                           : g_launch<MOE_FMT_NVFP4, false>(a, s);
     const int rc = gateup ? (wide ? g_launch<MOE_FMT_BF16, true, true>(a, s) : g_launch<MOE_FMT_BF16, true>(a, s))

@@ -127,6 +127,30 @@ __device__ __forceinline__ void g_mma_ts_i8(uint32_t d, uint32_t a_tmem, uint64_
     asm volatile("{ .reg .pred p; setp.ne.b32 p, %4, 0; tcgen05.mma.cta_group::1.kind::i8 [%0], [%1], %2, %3, p; }"
                  ::"r"(d), "r"(a_tmem), "l"(b), "r"(idesc), "r"(acc) : "memory");
 }
+// kind::mxf4nvf4 block-scaled instruction descriptor: A and B E2M1 (format 1), UE4M3 scale
+// factors (scale format 0, factor ids 0), K-major, M = 128, N = n, dense K = 64
+__device__ __forceinline__ uint32_t g_idesc_mxf4(int n, int m = 128) {
+    return (1u << 7) | (1u << 10) | (uint32_t(n >> 3) << 17) | (uint32_t(m >> 4) << 24);
+}
+// D (+)= A (E2M1, shared memory) x B (E2M1, shared memory), each 16-element block scaled by its
+// E4M3 factor from tensor memory (sfa: the A rows' four factors of this K 64, sfb: B's)
+__device__ __forceinline__ void g_mma_mxf4(uint32_t d, uint64_t a, uint64_t b, uint32_t idesc, uint32_t acc,
+                                           uint32_t sfa, uint32_t sfb) {
+    asm volatile("{ .reg .pred p; setp.ne.b32 p, %4, 0;\n"
+                 "tcgen05.mma.cta_group::1.kind::mxf4nvf4.block_scale.scale_vec::4X [%0], %1, %2, %3, [%5], [%6], p; }"
+                 ::"r"(d), "l"(a), "l"(b), "r"(idesc), "r"(acc), "r"(sfa), "r"(sfb) : "memory");
+}
+// Shared-memory descriptor of a 32-row x 16-byte scale-factor chunk (rows 16 bytes apart, no
+// swizzle: 8-row core matrices 128 bytes apart)
+__device__ __forceinline__ uint64_t g_desc_sf(uint32_t saddr) {
+    return uint64_t((saddr >> 4) & 0x3FFF) | (uint64_t(128 >> 4) << 16) | (uint64_t(128 >> 4) << 32) |
+           (uint64_t(1) << 46);
+}
+// Copy one scale-factor chunk into four tensor-memory columns, broadcast to the four lane
+// quarters: lane 32 q + m0 then holds the factors of rows m0, m0 + 32, m0 + 64, m0 + 96
+__device__ __forceinline__ void g_cp_sf(uint32_t taddr, uint64_t sdesc) {
+    asm volatile("tcgen05.cp.cta_group::1.32x128b.warpx4 [%0], %1;" ::"r"(taddr), "l"(sdesc) : "memory");
+}
 __device__ __forceinline__ void g_commit(uint32_t bar) {
     asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(bar) : "memory");
 }
