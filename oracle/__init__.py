@@ -31,6 +31,10 @@ def lib():
         L.oracle_bf16_to_f32.restype = F
         L.oracle_f32_to_bf16.argtypes = [F]
         L.oracle_f32_to_bf16.restype = ctypes.c_uint16
+        L.oracle_f16_to_f32.argtypes = [ctypes.c_uint16]
+        L.oracle_f16_to_f32.restype = F
+        L.oracle_set_x_f16.argtypes = [I]
+        L.oracle_set_x_f16.restype = None
         L.oracle_e2m1_decode.argtypes = [ctypes.c_uint8]
         L.oracle_e2m1_decode.restype = F
         L.oracle_e2m1_encode.argtypes = [F]
@@ -123,6 +127,22 @@ class Bank:
 def bf16_to_f32(bits):
     bits = np.asarray(bits, dtype=np.uint16)
     return (bits.astype(np.uint32) << 16).view(np.float32)
+
+
+def f16_to_f32(bits):
+    return lib().oracle_f16_to_f32(int(bits))
+
+
+class x_f16:
+    """Context: the layer's input activations x are fp16 bits instead of bf16
+    (route, moe_forward, grouped_swiglu and the W4A4 gate/up read x that way)."""
+
+    def __enter__(self):
+        lib().oracle_set_x_f16(1)
+        return self
+
+    def __exit__(self, *a):
+        lib().oracle_set_x_f16(0)
 
 
 def f32_to_bf16_scalar(v):

@@ -76,6 +76,23 @@ float oracle_bf16_to_f32(uint16_t b) {
     return f;
 }
 
+/* IEEE binary16 -> fp32 (exact): 1 sign, 5 exponent (bias 15), 10 mantissa bits. */
+float oracle_f16_to_f32(uint16_t h) {
+    int s = (h >> 15) & 1, e = (h >> 10) & 31, m = h & 1023;
+    float v;
+    if (e == 0) v = ldexpf((float)m, -24);                         /* subnormal: m 2^-24 */
+    else if (e == 31) v = m ? NAN : INFINITY;
+    else v = ldexpf(1.0f + (float)m / 1024.0f, e - 15);
+    return s ? -v : v;
+}
+
+/* The layer's input activations are bf16 by default; fp16 when set ("Step-5-
+ * Preview-Spark", Quality: the release runs activations in fp16).  Only the
+ * readers of the input x follow this; intermediates are given as bf16. */
+static int g_x_f16 = 0;
+void oracle_set_x_f16(int on) { g_x_f16 = on; }
+static float x_to_f32(uint16_t v);
+
 /* Round-to-nearest-even to bf16 (finite inputs). */
 uint16_t oracle_f32_to_bf16(float f) {
     uint32_t u;
@@ -87,6 +104,8 @@ uint16_t oracle_f32_to_bf16(float f) {
     u += 0x7fffu + lsb;
     return (uint16_t)(u >> 16);
 }
+
+static float x_to_f32(uint16_t v) { return g_x_f16 ? oracle_f16_to_f32(v) : oracle_bf16_to_f32(v); }
 
 /* ------------------------------------------------------------------------ */
 /* E2M1 and E4M3 (the two NVFP4 element types)                               */
@@ -362,7 +381,7 @@ void oracle_route(const uint16_t* x, int64_t T, int64_t H, const float* Wr,
         for (int64_t e = 0; e < E; e++) {
             float l = 0.0f;
             for (int64_t h = 0; h < H; h++)
-                l = l + oracle_bf16_to_f32(x[t * H + h]) * Wr[e * H + h];
+                l = l + x_to_f32(x[t * H + h]) * Wr[e * H + h];
             if (bias) l = l + bias[e];
             s[e] = 1.0f / (1.0f + expf(-l));
             if (scores) scores[t * E + e] = s[e];
@@ -441,7 +460,7 @@ int oracle_moe_forward(const uint16_t* x, int64_t T, int64_t H, int64_t F, int k
     double* xd = (double*)malloc(sizeof(double) * n * H);
     for (int64_t i = 0; i < n; i++)
         for (int64_t h = 0; h < H; h++)
-            xd[i * H + h] = (double)oracle_bf16_to_f32(x[tok[i] * H + h]);
+            xd[i * H + h] = (double)x_to_f32(x[tok[i] * H + h]);
     memset(y, 0, sizeof(double) * n * H);
 
     float* wg = (float*)malloc(sizeof(float) * F * H);
@@ -522,7 +541,7 @@ void oracle_grouped_swiglu(const uint16_t* x, int64_t H, int64_t F, int k,
             for (int64_t f = 0; f < F; f++) {
                 double g = 0.0, u = 0.0;
                 for (int64_t hh = 0; hh < H; hh++) {
-                    double xv = (double)oracle_bf16_to_f32(x[t * H + hh]);
+                    double xv = (double)x_to_f32(x[t * H + hh]);
                     g += (double)wg[f * H + hh] * xv;
                     u += (double)wu[f * H + hh] * xv;
                 }
@@ -741,7 +760,7 @@ void oracle_grouped_swiglu_w4a4(const uint16_t* x, int64_t H, int64_t F, int k,
             int32_t r = rows[i];
             if (r < offsets[e] || r >= offsets[e + 1]) continue;
             int64_t t = row_slot[r] / k;
-            for (int64_t hh = 0; hh < H; hh++) xf[hh] = oracle_bf16_to_f32(x[t * H + hh]);
+            for (int64_t hh = 0; hh < H; hh++) xf[hh] = x_to_f32(x[t * H + hh]);
             act_quant_row(xf, H, in_scale[e], xq, NULL, NULL);
             #pragma omp parallel for schedule(static)
             for (int64_t f = 0; f < F; f++) {
@@ -839,7 +858,7 @@ int oracle_moe_forward_w4a4(const uint16_t* x, int64_t T, int64_t H, int64_t F, 
             for (int64_t f = 0; f < F; f++) {
                 double g = 0.0, u = 0.0;
                 for (int64_t hh = 0; hh < H; hh++) {
-                    double xv = (double)oracle_bf16_to_f32(xt[hh]);
+                    double xv = (double)x_to_f32(xt[hh]);
                     g += (double)wg[f * H + hh] * xv;
                     u += (double)wu[f * H + hh] * xv;
                 }
