@@ -287,6 +287,12 @@ def gemm_source_hash():
     return h.hexdigest()[:16]
 
 
+def oracle_free_f16(wl, seed=0):
+    """The workload's activations drawn in fp32 and rounded to fp16 (not through bf16)."""
+    rng = np.random.Generator(np.random.PCG64(np.random.SeedSequence(seed).spawn(9)[0]))
+    return rng.standard_normal((wl.T, wl.H), dtype=np.float32).astype(np.float16)
+
+
 def _pcts(ms):
     a = np.asarray(ms, np.float64)
     return {"mean": round(float(a.mean()), 5), "median": round(float(np.median(a)), 5),
@@ -360,7 +366,10 @@ def measure(moe, wl, x, layer, args, flush, stream, clk, pk, pk_kind, per_step=T
     status = moe.read_status(ws)
     if status != 0:
         raise RuntimeError(f"device status {status} after warm-up")
-    ids, _ = moe.route_topk(x, layer.router_w, layer.router_bias, wl.k, ws)
+    # the step-level calls take bf16 activations: an fp16 layer's routing facts and dominant-kernel
+    # time come from the same values rounded to bf16
+    xb = x if x.dtype == torch.bfloat16 else x.to(torch.bfloat16)
+    ids, _ = moe.route_topk(xb, layer.router_w, layer.router_bias, wl.k, ws)
     touched = int(torch.unique(ids).numel())
     torch.cuda.synchronize()
     launches0 = moe.launch_count()
@@ -370,7 +379,7 @@ def measure(moe, wl, x, layer, args, flush, stream, clk, pk, pk_kind, per_step=T
     off, rs, sr = moe.permute(ids, wl.E, ws)
     R = T * wl.k
     h = torch.empty(R, wl.F, dtype=torch.bfloat16, device="cuda")
-    k_ms = float(np.mean(time_calls(lambda: moe.grouped_swiglu(x, off, rs, wl.k, layer.gate, layer.up, R, ws, out=h),
+    k_ms = float(np.mean(time_calls(lambda: moe.grouped_swiglu(xb, off, rs, wl.k, layer.gate, layer.up, R, ws, out=h),
                                     args.steps, flush, stream, clk)))
     if moe.read_status(ws) != 0:
         raise RuntimeError("device status set during timing")
@@ -418,9 +427,10 @@ def main():
     ap.add_argument("--steps", type=int, default=200)
     ap.add_argument("--warmup", type=int, default=10)
     ap.add_argument("--config", type=int, default=1, help="the headline workload")
-    ap.add_argument("--per-config", default="2,3,4,2w,4w",
+    ap.add_argument("--per-config", default="2,3,4,2w,4w,1h",
                     help="other workloads measured into per_config (comma list; a trailing 'w' runs an NVFP4 "
-                         "workload as W4A4, activations quantised on the fly; or 'none')")
+                         "workload as W4A4, activations quantised on the fly; a trailing 'h' runs it with fp16 "
+                         "activations; or 'none')")
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
     args = ap.parse_args()
@@ -495,8 +505,14 @@ def main():
         per_config = {}
         for c in others:
             w4a4 = c.endswith("w")
-            w2 = syn.WORKLOADS[int(c.rstrip("w"))]
+            f16 = c.endswith("h")
+            w2 = syn.WORKLOADS[int(c.rstrip("wh"))]
             lay = layer_for(w2)
+            x2 = x_for(w2)
+            if f16:
+                # fp16 activations: the same draw as fp16 values
+                x2 = torch.from_numpy(oracle_free_f16(w2)).cuda()
+                lay.act_f16 = True
             if w4a4:
                 if w2.fmt != "nvfp4":
                     continue
@@ -504,10 +520,13 @@ def main():
                 # amax / (6 * 448) (x ~ N(0, 1) over 4096 elements; h of these weights stays below ~8)
                 lay.gate.input_scale = torch.full((w2.E,), W4A4_IN_GATEUP, dtype=torch.float32, device="cuda")
                 lay.down.input_scale = torch.full((w2.E,), W4A4_IN_DOWN, dtype=torch.float32, device="cuda")
-            res = measure(moe, w2, x_for(w2), lay, args, flush, stream, clk, pk, pk_kind, fp4=w4a4)[0]
+            res = measure(moe, w2, x2, lay, args, flush, stream, clk, pk, pk_kind, fp4=w4a4, per_step=not f16)[0]
             if w4a4:
                 res["workload"] += " (W4A4: NVFP4 activations, static input scales)"
                 lay.gate.input_scale = lay.down.input_scale = None
+            if f16:
+                res["workload"] += " (fp16 activations)"
+                lay.act_f16 = False
             per_config[c] = res
             torch.cuda.empty_cache()
         layer = layer_for(wl)          # restore the headline workload's bias for the CPU leg

@@ -104,7 +104,16 @@ typedef struct {
  * num_experts = 1, or all three with packed = NULL for no shared expert.
  * router_w: fp32 [E, H]; router_bias: fp32 [E] added to the logits before
  * the sigmoid, or NULL.  swiglu_limit must be 0 (the pages give no value or
- * definition for a SwiGLU limit, so none is applied). */
+ * definition for a SwiGLU limit, so none is applied).
+ * act_f16: 0 = x and y are bf16; 1 = x and y are IEEE fp16 ("Step-5-Preview-
+ * Spark", At a glance and Quality: the release runs activations in fp16, since
+ * bf16 rounding of the routing input changed far more top-8 sets).  The router
+ * and the routed experts read the fp16 x exactly; the BF16 shared expert reads x
+ * rounded to bf16 (its MMA takes bf16 operands); the intermediates h and
+ * y_perm stay bf16.  Requires the routed banks in a 4-bit format with both
+ * projections on the tensor-core GEMM (H and F multiples of 256); from 64
+ * tokens the router logits run on the fp32 SIMT kernel (the tensor-core router
+ * splits bf16 operands). */
 typedef struct {
     moe_qweight gate, up, down;
     moe_qweight sh_gate, sh_up, sh_down;
@@ -112,6 +121,7 @@ typedef struct {
     const float* router_bias;
     int32_t E, H, F, top_k;
     float swiglu_limit;
+    int32_t act_f16;
 } moe_layer;
 
 /* ---------------------------------------------------------------------- */

@@ -88,7 +88,8 @@ float oracle_f16_to_f32(uint16_t h) {
 
 /* The layer's input activations are bf16 by default; fp16 when set ("Step-5-
  * Preview-Spark", Quality: the release runs activations in fp16).  Only the
- * readers of the input x follow this; intermediates are given as bf16. */
+ * readers of the input x follow this; intermediates are given as bf16.  The
+ * BF16 shared expert computes in bf16, so it reads x rounded to bf16. */
 static int g_x_f16 = 0;
 void oracle_set_x_f16(int on) { g_x_f16 = on; }
 static float x_to_f32(uint16_t v);
@@ -461,6 +462,10 @@ int oracle_moe_forward(const uint16_t* x, int64_t T, int64_t H, int64_t F, int k
     for (int64_t i = 0; i < n; i++)
         for (int64_t h = 0; h < H; h++)
             xd[i * H + h] = (double)x_to_f32(x[tok[i] * H + h]);
+    /* the BF16 shared expert computes in bf16: with fp16 inputs it reads x rounded to bf16 */
+    double* xs = (double*)malloc(sizeof(double) * n * H);
+    for (int64_t i = 0; i < n * H; i++)
+        xs[i] = g_x_f16 ? (double)oracle_bf16_to_f32(oracle_f32_to_bf16((float)xd[i])) : xd[i];
     memset(y, 0, sizeof(double) * n * H);
 
     float* wg = (float*)malloc(sizeof(float) * F * H);
@@ -489,7 +494,7 @@ int oracle_moe_forward(const uint16_t* x, int64_t T, int64_t H, int64_t F, int k
             double wt;
             if (who[p] < 0) { i = -1 - who[p]; slot = -1; wt = 1.0; }
             else { i = who[p] / k; slot = who[p] % k; wt = (double)topk_w[tok[i] * k + slot]; }
-            const double* xi = xd + i * H;
+            const double* xi = (shared ? xs : xd) + i * H;
             #pragma omp parallel for schedule(static)
             for (int64_t f = 0; f < F; f++) {
                 double g = 0.0, u = 0.0;
@@ -507,7 +512,7 @@ int oracle_moe_forward(const uint16_t* x, int64_t T, int64_t H, int64_t F, int k
             }
         }
     }
-    free(xd); free(wg); free(wu); free(wd); free(hbuf); free(who);
+    free(xd); free(xs); free(wg); free(wu); free(wd); free(hbuf); free(who);
     return 0;
 }
 
@@ -858,7 +863,9 @@ int oracle_moe_forward_w4a4(const uint16_t* x, int64_t T, int64_t H, int64_t F, 
             for (int64_t f = 0; f < F; f++) {
                 double g = 0.0, u = 0.0;
                 for (int64_t hh = 0; hh < H; hh++) {
-                    double xv = (double)x_to_f32(xt[hh]);
+                    float xf32 = x_to_f32(xt[hh]);
+                    /* the BF16 shared expert: x rounded to bf16 when x is fp16 */
+                    double xv = g_x_f16 ? (double)oracle_bf16_to_f32(oracle_f32_to_bf16(xf32)) : (double)xf32;
                     g += (double)wg[f * H + hh] * xv;
                     u += (double)wu[f * H + hh] * xv;
                 }

@@ -107,6 +107,7 @@ int layer_checks(const void* x, int T, const moe_layer* L, void* y, void* ws, si
     MOE_TRY(check_bank(&L->down, L->E, L->H, L->F));
     if (L->gate.fmt == MOE_FMT_BF16 || L->gate.fmt != L->up.fmt || L->gate.fmt != L->down.fmt)
         return MOE_ERR_UNSUPPORTED;
+    if (L->act_f16 && !(gemm_shape_ok(L->H, L->F) && gemm_shape_ok(L->F, L->H))) return MOE_ERR_UNSUPPORTED;
     // gate and up share one quantised activation (the gate's input scale)
     if (L->up.input_scale && L->up.input_scale != L->gate.input_scale) return MOE_ERR_UNSUPPORTED;
     if ((L->gate.input_scale || L->down.input_scale) && !(gemm_shape_ok(L->H, L->F) && gemm_shape_ok(L->F, L->H)))
@@ -165,6 +166,7 @@ int layer_run(const void* x, int T, const moe_layer* L, void* y, void* ws, cudaS
     const __nv_bfloat16* xb = reinterpret_cast<const __nv_bfloat16*>(x);
 
     const bool has_sh = L->sh_gate.packed != nullptr;
+    const int x_f16 = L->act_f16 ? 1 : 0;
     int32_t* sh_off = at<int32_t>(ws, W.sh_offsets);
     int32_t* sh_rs = at<int32_t>(ws, W.sh_rowslot);
     int32_t* counter = status + 1;
@@ -182,8 +184,15 @@ int layer_run(const void* x, int T, const moe_layer* L, void* y, void* ws, cudaS
         side_lock = std::unique_lock<std::mutex>(side->call);
         if (cudaEventRecord(side->fork, s) != cudaSuccess || cudaStreamWaitEvent(side->s, side->fork, 0) != cudaSuccess)
             return MOE_ERR_CUDA;
+        // fp16 mode: the BF16 shared expert reads x rounded to bf16, staged in its output region (the
+        // down projection overwrites it only after the gate/up projection has read it)
+        const __nv_bfloat16* xs = xb;
+        if (x_f16) {
+            MOE_TRY(launch_f16_to_bf16(reinterpret_cast<const __half*>(x), ys, size_t(T) * H, side->s));
+            xs = ys;
+        }
         GemvProblem sg{};
-        sg.act = xb; sg.act_by_token = 1; sg.top_k = k; sg.offsets = sh_off; sg.row_slot = sh_rs;
+        sg.act = xs; sg.act_by_token = 1; sg.top_k = k; sg.offsets = sh_off; sg.row_slot = sh_rs;
         sg.E = 1; sg.fmt = MOE_FMT_BF16; sg.out_dim = F; sg.in_dim = H;
         sg.p0 = L->sh_gate.packed; sg.p1 = L->sh_up.packed; sg.out = h_sh; sg.status = status;
         GemvProblem sd{};
@@ -206,11 +215,11 @@ int layer_run(const void* x, int T, const moe_layer* L, void* y, void* ws, cudaS
         ra.x = xb; ra.T = T; ra.H = H; ra.Wr = L->router_w; ra.bias = L->router_bias; ra.E = E; ra.k = k;
         ra.logits = at<float>(ws, W.logits); ra.ids = ids; ra.w = tw; ra.counter = counter; ra.status = status;
         ra.offsets = offsets; ra.row_slot = row_slot; ra.slot_row = slot_row;
-        ra.sh_offsets = nullptr; ra.sh_rowslot = nullptr;
+        ra.sh_offsets = nullptr; ra.sh_rowslot = nullptr; ra.x_f16 = x_f16;
         MOE_TRY(launch_route_decode(ra, s));
     } else {
         MOE_TRY(launch_route(xb, T, H, L->router_w, L->router_bias, E, k, ids, tw, at<float>(ws, W.logits),
-                             at<__nv_bfloat16>(ws, W.wsplit), status, counter, s));
+                             at<__nv_bfloat16>(ws, W.wsplit), status, counter, s, x_f16));
         MOE_TRY(launch_permute(ids, T, k, E, offsets, row_slot, slot_row, at<int32_t>(ws, W.hist), status, s));
     }
     const bool routed_gemm = gemm_shape_ok(H, F) && gemm_shape_ok(F, H);
@@ -220,7 +229,7 @@ int layer_run(const void* x, int T, const moe_layer* L, void* y, void* ws, cudaS
     gu.E = E; gu.topk_w = nullptr; gu.fmt = L->gate.fmt; gu.out_dim = F; gu.in_dim = H;
     gu.p0 = L->gate.packed; gu.s0 = L->gate.scales; gu.g0 = L->gate.global_scale;
     gu.p1 = L->up.packed; gu.s1 = L->up.scales; gu.g1 = L->up.global_scale;
-    gu.out = h_perm; gu.status = status; gu.in_scale = L->gate.input_scale;
+    gu.out = h_perm; gu.status = status; gu.in_scale = L->gate.input_scale; gu.act_f16 = x_f16;
     GemvProblem dn{};
     dn.act = h_perm; dn.act_by_token = 0; dn.top_k = k; dn.offsets = offsets; dn.row_slot = row_slot;
     dn.E = E; dn.topk_w = tw; dn.fmt = L->down.fmt; dn.out_dim = H; dn.in_dim = F;
@@ -248,7 +257,7 @@ int layer_run(const void* x, int T, const moe_layer* L, void* y, void* ws, cudaS
     // after a join with the side stream the combine starts only when both inputs are complete (no
     // early launch of a dependent grid across an event wait)
     return launch_combine(y_perm, slot_row, T, k, H, has_sh ? ys : nullptr,
-                          reinterpret_cast<__nv_bfloat16*>(y), s, !has_sh);
+                          reinterpret_cast<__nv_bfloat16*>(y), s, !has_sh, x_f16);
 }
 
 }  // namespace

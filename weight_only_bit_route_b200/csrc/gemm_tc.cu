@@ -1119,6 +1119,7 @@ __global__ void __launch_bounds__(G_THREADS, 1) tc_grouped_gemm(const __grid_con
 // row_w[row_slot[row]] when given: the down projection's routing weight, a
 // power of two times w being exact) goes to scale[row].  One warp per row.
 // ---------------------------------------------------------------------------
+template <bool F16>
 __global__ void __launch_bounds__(256) g_prep(const __nv_bfloat16* __restrict__ src, int in_dim,
                                               const int32_t* __restrict__ row_slot, int top_k, int by_token,
                                               int rows, int mode, const float* __restrict__ row_w,
@@ -1149,10 +1150,10 @@ __global__ void __launch_bounds__(256) g_prep(const __nv_bfloat16* __restrict__ 
         uint8_t* sc8 = reinterpret_cast<uint8_t*>(dst) + sc_off + size_t(row) * (in_dim / 16);
         for (int b = lane; b < in_dim / 16; b += 32) {
             const uint4 v0 = s[2 * b], v1 = s[2 * b + 1];
-            const float xf[16] = {bf16_lo(v0.x), bf16_hi(v0.x), bf16_lo(v0.y), bf16_hi(v0.y),
-                                  bf16_lo(v0.z), bf16_hi(v0.z), bf16_lo(v0.w), bf16_hi(v0.w),
-                                  bf16_lo(v1.x), bf16_hi(v1.x), bf16_lo(v1.y), bf16_hi(v1.y),
-                                  bf16_lo(v1.z), bf16_hi(v1.z), bf16_lo(v1.w), bf16_hi(v1.w)};
+            const float xf[16] = {act_lo<F16>(v0.x), act_hi<F16>(v0.x), act_lo<F16>(v0.y), act_hi<F16>(v0.y),
+                                  act_lo<F16>(v0.z), act_hi<F16>(v0.z), act_lo<F16>(v0.w), act_hi<F16>(v0.w),
+                                  act_lo<F16>(v1.x), act_hi<F16>(v1.x), act_lo<F16>(v1.y), act_hi<F16>(v1.y),
+                                  act_lo<F16>(v1.z), act_hi<F16>(v1.z), act_lo<F16>(v1.w), act_hi<F16>(v1.w)};
             uint32_t bytes[8];
             sc8[b] = uint8_t(nv_quant_block16(xf, g, bytes));
             *reinterpret_cast<uint2*>(d8 + 8 * b) = make_uint2(bytes[0] | (bytes[1] << 8) | (bytes[2] << 16) | (bytes[3] << 24),
@@ -1164,8 +1165,8 @@ __global__ void __launch_bounds__(256) g_prep(const __nv_bfloat16* __restrict__ 
     float amax = 0.f;
     for (int i = lane; i < n16; i += 32) {
         const uint4 v = s[i];
-        amax = fmaxf(amax, fmaxf(fmaxf(fabsf(bf16_lo(v.x)), fabsf(bf16_hi(v.x))), fmaxf(fabsf(bf16_lo(v.y)), fabsf(bf16_hi(v.y)))));
-        amax = fmaxf(amax, fmaxf(fmaxf(fabsf(bf16_lo(v.z)), fabsf(bf16_hi(v.z))), fmaxf(fabsf(bf16_lo(v.w)), fabsf(bf16_hi(v.w)))));
+        amax = fmaxf(amax, fmaxf(fmaxf(fabsf(act_lo<F16>(v.x)), fabsf(act_hi<F16>(v.x))), fmaxf(fabsf(act_lo<F16>(v.y)), fabsf(act_hi<F16>(v.y)))));
+        amax = fmaxf(amax, fmaxf(fmaxf(fabsf(act_lo<F16>(v.z)), fabsf(act_hi<F16>(v.z))), fmaxf(fabsf(act_lo<F16>(v.w)), fabsf(act_hi<F16>(v.w)))));
     }
     for (int o = 16; o > 0; o >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, o));
     int e = 0;
@@ -1177,10 +1178,10 @@ __global__ void __launch_bounds__(256) g_prep(const __nv_bfloat16* __restrict__ 
     for (int i = lane; i < n16; i += 32) {
         const uint4 v = s[i];
         __half2 h[4];
-        h[0] = __floats2half2_rn(bf16_lo(v.x) * down, bf16_hi(v.x) * down);
-        h[1] = __floats2half2_rn(bf16_lo(v.y) * down, bf16_hi(v.y) * down);
-        h[2] = __floats2half2_rn(bf16_lo(v.z) * down, bf16_hi(v.z) * down);
-        h[3] = __floats2half2_rn(bf16_lo(v.w) * down, bf16_hi(v.w) * down);
+        h[0] = __floats2half2_rn(act_lo<F16>(v.x) * down, act_hi<F16>(v.x) * down);
+        h[1] = __floats2half2_rn(act_lo<F16>(v.y) * down, act_hi<F16>(v.y) * down);
+        h[2] = __floats2half2_rn(act_lo<F16>(v.z) * down, act_hi<F16>(v.z) * down);
+        h[3] = __floats2half2_rn(act_lo<F16>(v.w) * down, act_hi<F16>(v.w) * down);
         uint4 o = *reinterpret_cast<uint4*>(h);
         if (mode == 3) {                        // (x0 x1)(x2 x3)(x4 x5)(x6 x7) -> (x0 x4)(x1 x5)(x2 x6)(x3 x7)
             const uint4 n = o;
@@ -1207,6 +1208,7 @@ __global__ void __launch_bounds__(256) g_prep(const __nv_bfloat16* __restrict__ 
 // (as a floating-point product with that row would be) instead of finite
 // values made from meaningless digits.
 constexpr int G_PREP_I8_THREADS = 128;
+template <bool F16>
 __global__ void __launch_bounds__(G_PREP_I8_THREADS) g_prep_i8(const __nv_bfloat16* __restrict__ src, int in_dim,
                                                                const int32_t* __restrict__ row_slot, int top_k,
                                                                int by_token, const float* __restrict__ row_w,
@@ -1221,8 +1223,8 @@ __global__ void __launch_bounds__(G_PREP_I8_THREADS) g_prep_i8(const __nv_bfloat
     float amax = 0.f;
     for (int i = tid; i < n16; i += G_PREP_I8_THREADS) {
         const uint4 v = s[i];
-        amax = fmaxf(amax, fmaxf(fmaxf(fabsf(bf16_lo(v.x)), fabsf(bf16_hi(v.x))), fmaxf(fabsf(bf16_lo(v.y)), fabsf(bf16_hi(v.y)))));
-        amax = fmaxf(amax, fmaxf(fmaxf(fabsf(bf16_lo(v.z)), fabsf(bf16_hi(v.z))), fmaxf(fabsf(bf16_lo(v.w)), fabsf(bf16_hi(v.w)))));
+        amax = fmaxf(amax, fmaxf(fmaxf(fabsf(act_lo<F16>(v.x)), fabsf(act_hi<F16>(v.x))), fmaxf(fabsf(act_lo<F16>(v.y)), fabsf(act_hi<F16>(v.y)))));
+        amax = fmaxf(amax, fmaxf(fmaxf(fabsf(act_lo<F16>(v.z)), fabsf(act_hi<F16>(v.z))), fmaxf(fabsf(act_lo<F16>(v.w)), fabsf(act_hi<F16>(v.w)))));
     }
     for (int o = 16; o > 0; o >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, o));
     if (lane == 0) s_max[tid >> 5] = amax;
@@ -1240,8 +1242,8 @@ __global__ void __launch_bounds__(G_PREP_I8_THREADS) g_prep_i8(const __nv_bfloat
         int zs = 0;
         if (i < n16) {
             const uint4 v = s[i];
-            const float xs[8] = {bf16_lo(v.x), bf16_lo(v.y), bf16_lo(v.z), bf16_lo(v.w),
-                                 bf16_hi(v.x), bf16_hi(v.y), bf16_hi(v.z), bf16_hi(v.w)};
+            const float xs[8] = {act_lo<F16>(v.x), act_lo<F16>(v.y), act_lo<F16>(v.z), act_lo<F16>(v.w),
+                                 act_hi<F16>(v.x), act_hi<F16>(v.y), act_hi<F16>(v.z), act_hi<F16>(v.w)};
             uint32_t p2[2] = {0u, 0u}, p1[2] = {0u, 0u}, p0[2] = {0u, 0u};
 #pragma unroll
             for (int e = 0; e < 8; e++) {
@@ -1372,6 +1374,8 @@ int launch_grouped_gemm(const GemvProblem& p, bool gateup, int rows, const GemmB
         ((reinterpret_cast<uintptr_t>(p.s0) & 15u) || (gateup && (reinterpret_cast<uintptr_t>(p.s1) & 15u))))
         return MOE_ERR_INVALID_ARG;
     if (p.in_scale && p.fmt != MOE_FMT_NVFP4) return MOE_ERR_UNSUPPORTED;
+    // fp16 activations enter through the pre-pass: the 4-bit formats only (BF16 reads its rows as they are)
+    if (p.act_f16 && p.fmt == MOE_FMT_BF16) return MOE_ERR_UNSUPPORTED;
     if (rows <= 0) return MOE_OK;
     G_TRY(g_encoder());
 
@@ -1390,14 +1394,16 @@ int launch_grouped_gemm(const GemvProblem& p, bool gateup, int rows, const GemmB
         if (!buf.act_buf || ((nv || i4) && !buf.scale_buf)) return MOE_ERR_WORKSPACE;
         if (i8) {
             const float* row_w = gateup ? nullptr : p.topk_w;
-            if (launch_pdl(g_prep_i8, dim3(rows), dim3(G_PREP_I8_THREADS), 0, s, p.act, in, p.row_slot, p.top_k,
+            if (launch_pdl(p.act_f16 ? g_prep_i8<true> : g_prep_i8<false>, dim3(rows), dim3(G_PREP_I8_THREADS), 0, s,
+                           p.act, in, p.row_slot, p.top_k,
                            p.act_by_token, row_w, reinterpret_cast<uint8_t*>(buf.act_buf), buf.scale_buf,
                            buf.zbuf, p.status) != cudaSuccess)
                 return MOE_ERR_CUDA;
         } else {
             const int mode = a4 ? 5 : (nv ? 2 : (i4 ? 3 : 0));
             const float* row_w = ((nv || i4) && !gateup) ? p.topk_w : nullptr;   // folded into the row scale
-            if (launch_pdl(g_prep, dim3((rows * 32 + 255) / 256), dim3(256), 0, s, p.act, in, p.row_slot, p.top_k,
+            if (launch_pdl(p.act_f16 ? g_prep<true> : g_prep<false>, dim3((rows * 32 + 255) / 256), dim3(256), 0, s,
+                           p.act, in, p.row_slot, p.top_k,
                            p.act_by_token, rows, mode, row_w, reinterpret_cast<uint16_t*>(buf.act_buf),
                            buf.scale_buf, p.offsets, p.E, p.in_scale, a4_sc_off) != cudaSuccess)
                 return MOE_ERR_CUDA;

@@ -3,6 +3,7 @@
 #pragma once
 
 #include <cuda_bf16.h>
+#include <cuda_fp16.h>
 #include <cuda_runtime.h>
 #include <stdint.h>
 
@@ -44,6 +45,17 @@ __device__ __forceinline__ void set_status(int32_t* status, int32_t code) {
 
 __device__ __forceinline__ float bf16_lo(uint32_t v) { return __uint_as_float(v << 16); }
 __device__ __forceinline__ float bf16_hi(uint32_t v) { return __uint_as_float(v & 0xffff0000u); }
+// The layer's input activations: bf16, or fp16 in the fp16 activation mode (both exact in fp32).
+template <bool F16>
+__device__ __forceinline__ float act_lo(uint32_t v) {
+    if constexpr (F16) return __half2float(__ushort_as_half(static_cast<unsigned short>(v & 0xffffu)));
+    else return bf16_lo(v);
+}
+template <bool F16>
+__device__ __forceinline__ float act_hi(uint32_t v) {
+    if constexpr (F16) return __half2float(__ushort_as_half(static_cast<unsigned short>(v >> 16)));
+    else return bf16_hi(v);
+}
 
 __device__ __forceinline__ float warp_sum(float v, int width) {
     for (int o = width / 2; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
@@ -160,13 +172,14 @@ constexpr int kRouterTcMinT = 64;      // from this many tokens the router logit
 // planes: 3 * E * H bf16 of scratch for the tensor-core logits (used when T >= 64).
 int launch_route(const __nv_bfloat16* x, int T, int H, const float* Wr, const float* bias,
                  int E, int k, int32_t* ids, float* w, float* logits, __nv_bfloat16* planes,
-                 int32_t* status, int32_t* counter, cudaStream_t s);
+                 int32_t* status, int32_t* counter, cudaStream_t s, int x_f16 = 0);
 // Router logits l = x Wr^T (fp32) on the tensor cores (Wr split into three bf16 planes).
 int launch_router_logits_tc(const __nv_bfloat16* x, int T, int H, const float* Wr, int E, float* logits,
                             __nv_bfloat16* planes, int32_t* status, cudaStream_t s);
 
 struct RouterDecodeArgs {
     const __nv_bfloat16* x; int T, H; const float* Wr; const float* bias; int E, k;
+    int x_f16;                                                  // x holds fp16 values (fp16 activation mode)
     float* logits; int32_t* ids; float* w;
     int32_t* counter; int32_t* status;
     int32_t* offsets; int32_t* row_slot; int32_t* slot_row;     // bucketing (nullable: skip)
@@ -195,6 +208,7 @@ struct GemvProblem {
     __nv_bfloat16* out;        // [rows, out_dim]
     int32_t* status;
     const float* in_scale;     // NVFP4 W4A4: activation global scale by expert [E] (nullable)
+    int act_f16;               // act holds fp16 values (fp16 activation mode; 4-bit formats on the GEMM)
 };
 
 // Streaming grouped GEMV (decode): routed bank plus an optional BF16 shared
@@ -204,7 +218,11 @@ int launch_stream_gemv(const GemvProblem& routed, const GemvProblem* shared, boo
                        void* prep_ws, cudaStream_t s, bool pdl);
 
 int launch_combine(const __nv_bfloat16* y_perm, const int32_t* slot_row, int T, int k, int H,
-                   const __nv_bfloat16* shared_out, __nv_bfloat16* y, cudaStream_t s, bool pdl = true);
+                   const __nv_bfloat16* shared_out, __nv_bfloat16* y, cudaStream_t s, bool pdl = true,
+                   int y_f16 = 0);
+// fp16 -> bf16 (round to nearest even), n elements, n % 8 == 0: the BF16 shared expert's input
+// in the fp16 activation mode.
+int launch_f16_to_bf16(const __half* src, __nv_bfloat16* dst, size_t n, cudaStream_t s);
 
 int launch_quant_int4(const __nv_bfloat16* w, int64_t rows, int64_t cols, int32_t* packed,
                       __nv_bfloat16* scales, cudaStream_t s);

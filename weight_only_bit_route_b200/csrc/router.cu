@@ -19,7 +19,7 @@ namespace moe {
 // ---------------------------------------------------------------------------
 // Logits, few tokens: warp per expert, NT tokens per pass.
 // ---------------------------------------------------------------------------
-template <int NT>
+template <int NT, bool F16>
 __global__ void __launch_bounds__(256) router_logits_rows(
         const __nv_bfloat16* __restrict__ x, int T, int H, const float* __restrict__ Wr, int E,
         float* __restrict__ logits) {
@@ -40,10 +40,10 @@ __global__ void __launch_bounds__(256) router_logits_rows(
             if (t0 + i < T) {
                 const uint4 xv = __ldg(reinterpret_cast<const uint4*>(x + size_t(t0 + i) * H + h));
                 float a = acc[i];
-                a = fmaf(bf16_lo(xv.x), w0.x, a); a = fmaf(bf16_hi(xv.x), w0.y, a);
-                a = fmaf(bf16_lo(xv.y), w0.z, a); a = fmaf(bf16_hi(xv.y), w0.w, a);
-                a = fmaf(bf16_lo(xv.z), w1.x, a); a = fmaf(bf16_hi(xv.z), w1.y, a);
-                a = fmaf(bf16_lo(xv.w), w1.z, a); a = fmaf(bf16_hi(xv.w), w1.w, a);
+                a = fmaf(act_lo<F16>(xv.x), w0.x, a); a = fmaf(act_hi<F16>(xv.x), w0.y, a);
+                a = fmaf(act_lo<F16>(xv.y), w0.z, a); a = fmaf(act_hi<F16>(xv.y), w0.w, a);
+                a = fmaf(act_lo<F16>(xv.z), w1.x, a); a = fmaf(act_hi<F16>(xv.z), w1.y, a);
+                a = fmaf(act_lo<F16>(xv.w), w1.z, a); a = fmaf(act_hi<F16>(xv.w), w1.w, a);
                 acc[i] = a;
             }
         }
@@ -61,6 +61,7 @@ __global__ void __launch_bounds__(256) router_logits_rows(
 // ---------------------------------------------------------------------------
 constexpr int RT_BM = 64, RT_BN = 64, RT_BK = 32;
 
+template <bool F16>
 __global__ void __launch_bounds__(256) router_logits_tiled(
         const __nv_bfloat16* __restrict__ x, int T, int H, const float* __restrict__ Wr, int E,
         float* __restrict__ logits) {
@@ -76,10 +77,10 @@ __global__ void __launch_bounds__(256) router_logits_tiled(
             int r = tid / 4, c = (tid % 4) * 8;
             uint4 v = make_uint4(0, 0, 0, 0);
             if (m0 + r < T) v = __ldg(reinterpret_cast<const uint4*>(x + size_t(m0 + r) * H + k0 + c));
-            xs[c + 0][r] = bf16_lo(v.x); xs[c + 1][r] = bf16_hi(v.x);
-            xs[c + 2][r] = bf16_lo(v.y); xs[c + 3][r] = bf16_hi(v.y);
-            xs[c + 4][r] = bf16_lo(v.z); xs[c + 5][r] = bf16_hi(v.z);
-            xs[c + 6][r] = bf16_lo(v.w); xs[c + 7][r] = bf16_hi(v.w);
+            xs[c + 0][r] = act_lo<F16>(v.x); xs[c + 1][r] = act_hi<F16>(v.x);
+            xs[c + 2][r] = act_lo<F16>(v.y); xs[c + 3][r] = act_hi<F16>(v.y);
+            xs[c + 4][r] = act_lo<F16>(v.z); xs[c + 5][r] = act_hi<F16>(v.z);
+            xs[c + 6][r] = act_lo<F16>(v.w); xs[c + 7][r] = act_hi<F16>(v.w);
         }
         // Wr tile: 64 experts x 32 k fp32; each thread loads 8 (two float4)
         {
@@ -201,6 +202,7 @@ constexpr int RD_WARPS = 8;          // 2 experts x 4 quarters of H per CTA
 constexpr int RD_EPC = 2;            // experts per CTA
 constexpr int RD_TMAX = 16;          // tokens (kRouterDecodeMaxT)
 
+template <bool F16>
 __global__ void __launch_bounds__(RD_WARPS * 32) router_decode(RouterDecodeArgs a) {
     extern __shared__ __align__(16) uint8_t rsm[];
     __shared__ int s_last;
@@ -268,8 +270,8 @@ __global__ void __launch_bounds__(RD_WARPS * 32) router_decode(RouterDecodeArgs 
                 if (t < a.T) {
                     const uint2 xv = *reinterpret_cast<const uint2*>(xs + t * a.H + h);
                     float v = acc[t];
-                    v = fmaf(bf16_lo(xv.x), wv[q].x, v); v = fmaf(bf16_hi(xv.x), wv[q].y, v);
-                    v = fmaf(bf16_lo(xv.y), wv[q].z, v); v = fmaf(bf16_hi(xv.y), wv[q].w, v);
+                    v = fmaf(act_lo<F16>(xv.x), wv[q].x, v); v = fmaf(act_hi<F16>(xv.x), wv[q].y, v);
+                    v = fmaf(act_lo<F16>(xv.y), wv[q].z, v); v = fmaf(act_hi<F16>(xv.y), wv[q].w, v);
                     acc[t] = v;
                 }
             }
@@ -284,8 +286,8 @@ __global__ void __launch_bounds__(RD_WARPS * 32) router_decode(RouterDecodeArgs 
             if (t < a.T) {
                 const uint2 xv = *reinterpret_cast<const uint2*>(xs + t * a.H + h);
                 float v = acc[t];
-                v = fmaf(bf16_lo(xv.x), w4.x, v); v = fmaf(bf16_hi(xv.x), w4.y, v);
-                v = fmaf(bf16_lo(xv.y), w4.z, v); v = fmaf(bf16_hi(xv.y), w4.w, v);
+                v = fmaf(act_lo<F16>(xv.x), w4.x, v); v = fmaf(act_hi<F16>(xv.x), w4.y, v);
+                v = fmaf(act_lo<F16>(xv.y), w4.z, v); v = fmaf(act_hi<F16>(xv.y), w4.w, v);
                 acc[t] = v;
             }
         }
@@ -380,44 +382,44 @@ __global__ void __launch_bounds__(RD_WARPS * 32) router_decode(RouterDecodeArgs 
 
 int launch_route_decode(const RouterDecodeArgs& a, cudaStream_t s) {
     const size_t smem = std::max<size_t>(size_t(a.T) * a.H * 2, size_t(a.E) * 4);
-    static size_t smem_set = 0;
-    if (smem > 48 * 1024 && smem > smem_set) {
-        if (cudaFuncSetAttribute(router_decode, cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem)) != cudaSuccess)
-            return MOE_ERR_UNSUPPORTED;
-        smem_set = smem;
-    }
     if (a.T > RD_TMAX || a.H % 512) return MOE_ERR_UNSUPPORTED;
-    return launch_pdl(router_decode, dim3((a.E + RD_EPC - 1) / RD_EPC), dim3(RD_WARPS * 32), smem, s, a) == cudaSuccess
+    auto k = a.x_f16 ? router_decode<true> : router_decode<false>;
+    if (smem > 48 * 1024 &&
+        cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem)) != cudaSuccess)
+        return MOE_ERR_UNSUPPORTED;
+    return launch_pdl(k, dim3((a.E + RD_EPC - 1) / RD_EPC), dim3(RD_WARPS * 32), smem, s, a) == cudaSuccess
                ? MOE_OK : MOE_ERR_CUDA;
 }
 
 int launch_route(const __nv_bfloat16* x, int T, int H, const float* Wr, const float* bias,
                  int E, int k, int32_t* ids, float* w, float* logits, __nv_bfloat16* planes,
-                 int32_t* status, int32_t* counter, cudaStream_t s) {
+                 int32_t* status, int32_t* counter, cudaStream_t s, int x_f16) {
     if (T <= kRouterDecodeMaxT && counter && router_decode_ok(H)) {
         RouterDecodeArgs a{};
         a.x = x; a.T = T; a.H = H; a.Wr = Wr; a.bias = bias; a.E = E; a.k = k;
-        a.logits = logits; a.ids = ids; a.w = w; a.counter = counter; a.status = status;
+        a.logits = logits; a.ids = ids; a.w = w; a.counter = counter; a.status = status; a.x_f16 = x_f16;
         return launch_route_decode(a, s);
     }
+    auto rows8 = x_f16 ? router_logits_rows<8, true> : router_logits_rows<8, false>;
+    auto tiled = x_f16 ? router_logits_tiled<true> : router_logits_tiled<false>;
     if (T <= 32) {
         dim3 block(256);
         int epb = 8;
         if (T <= 8) {
             dim3 grid((E + epb - 1) / epb, 1);
-            router_logits_rows<8><<<grid, block, 0, s>>>(x, T, H, Wr, E, logits);
+            rows8<<<grid, block, 0, s>>>(x, T, H, Wr, E, logits);
             count_launch();
         } else {
             dim3 grid((E + epb - 1) / epb, (T + 7) / 8);
-            router_logits_rows<8><<<grid, block, 0, s>>>(x, T, H, Wr, E, logits);
+            rows8<<<grid, block, 0, s>>>(x, T, H, Wr, E, logits);
             count_launch();
         }
-    } else if (T >= kRouterTcMinT && planes) {
+    } else if (T >= kRouterTcMinT && planes && !x_f16) {     // (bf16 planes: x must be bf16)
         const int rc = launch_router_logits_tc(x, T, H, Wr, E, logits, planes, status, s);
         if (rc != MOE_OK) return rc;
     } else {
         dim3 grid((E + RT_BN - 1) / RT_BN, (T + RT_BM - 1) / RT_BM);
-        router_logits_tiled<<<grid, 256, 0, s>>>(x, T, H, Wr, E, logits);
+        tiled<<<grid, 256, 0, s>>>(x, T, H, Wr, E, logits);
         count_launch();
     }
     router_topk<<<(T + 7) / 8, 256, 0, s>>>(logits, bias, T, E, k, ids, w);

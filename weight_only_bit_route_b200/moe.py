@@ -42,7 +42,7 @@ class Layer(ctypes.Structure):
                 ("sh_gate", QWeight), ("sh_up", QWeight), ("sh_down", QWeight),
                 ("router_w", _P), ("router_bias", _P),
                 ("E", ctypes.c_int32), ("H", ctypes.c_int32), ("F", ctypes.c_int32),
-                ("top_k", ctypes.c_int32), ("swiglu_limit", ctypes.c_float)]
+                ("top_k", ctypes.c_int32), ("swiglu_limit", ctypes.c_float), ("act_f16", ctypes.c_int32)]
 
 
 def _sig(name, res, args):
@@ -127,7 +127,8 @@ def _empty_qweight():
 
 
 class MoELayer:
-    def __init__(self, gate, up, down, router_w, top_k=8, router_bias=None, shared=None):
+    def __init__(self, gate, up, down, router_w, top_k=8, router_bias=None, shared=None, act_f16=False):
+        self.act_f16 = act_f16               # x and y in fp16 instead of bf16
         self.gate, self.up, self.down = gate, up, down
         self.shared = shared
         self.router_w, self.router_bias = router_w, router_bias
@@ -142,7 +143,7 @@ class MoELayer:
                      sh[1].struct() if sh else _empty_qweight(),
                      sh[2].struct() if sh else _empty_qweight(),
                      _ptr(self.router_w), _ptr(self.router_bias),
-                     self.E, self.H, self.F, self.top_k, 0.0)
+                     self.E, self.H, self.F, self.top_k, 0.0, 1 if self.act_f16 else 0)
 
 
 def workspace_bytes(T, H, E, F, top_k):
