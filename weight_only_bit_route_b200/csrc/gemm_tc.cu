@@ -160,6 +160,11 @@ struct GCfg {
     static constexpr int kDqArrivals = kI8 ? G_DQ_WARPS / 2 : G_DQ_WARPS;  // warps that fill one stage
     static constexpr bool kMmaF16 = FMT == MOE_FMT_NVFP4 || FMT == MOE_FMT_INT4_G128;   // f16 operands
     static_assert(kABase <= 512 && (!kTmemA || kAStages >= 2), "tensor memory layout");
+    // the 8-bit path's two MMA issuers take alternate steps: even B and accumulator rings give each
+    // the slots it alone waits on, so it sees every phase of them in order; an issuer's accumulator
+    // wait covers the other issuer's A stages as long as there are no more buffers than A stages
+    static_assert(!kI8 || (kBStages % 2 == 0 && kAccBufs % 2 == 0 && kAccBufs <= kAStages),
+                  "8-bit rings");
     static_assert(!kA4 || kABase + G_SF_RING * kSfSlotCols <= 512, "A4 scale-factor ring");
 };
 
@@ -172,7 +177,7 @@ constexpr int G_NB_MAPS = 8;                                        // box heigh
 struct GArgs {
     CUtensorMap tm_p0, tm_p1;        // packed (or BF16) weights of gate (or down) and up
     CUtensorMap tm_s0, tm_s1;        // NVFP4 block scales
-    CUtensorMap tm_b[G_NB_MAPS];     // activation operand rows, box height 16*(i+1)
+    CUtensorMap tm_b[G_NB_MAPS];     // activation operand rows, box height 16*(i+1) (8-bit int4: [0], digit rows)
     CUtensorMap tm_bs[G_NB_MAPS];    // A4: the activation rows' scale factors, box height 16*(i+1)
     const uint8_t* sc0;              // int4 scales (bf16), bulk-copied per tile
     const uint8_t* sc1;
@@ -186,7 +191,6 @@ struct GArgs {
     int32_t* status;
     float* partial;                  // split-K: fp32 partial sums [ksplit][nmat][rows][out_dim]
     const float* zsum;               // 8-bit int4: 8 * sum of the row's fixed-point values per group [rows][zst]
-    const uint8_t* bdig;             // 8-bit int4: the digit rows [3 rows][in]
     int E, out_dim, in_dim;
     int ksplit, rows;                // K slices per (m-tile, n-tile); activation rows of the problem
     int* tile_cnt;                   // split-K: zeroed arrival counters, four per (m-tile, n-tile); the last
@@ -273,6 +277,10 @@ __device__ __forceinline__ void g_dq_int4_i8(const uint4 w, uint32_t (&o)[16]) {
 
 struct GTile { int e, m0, n0, nval, bn, ebase, ks, kbase, mn; };
 
+// Bytes of the per-expert tile table at the start of the dynamic shared memory (16 per expert),
+// rounded so the stage rings after it stay 1024-byte aligned.
+__host__ __device__ inline uint32_t g_tbl_bytes(int E) { return (uint32_t(E) * 16u + 1023u) & ~1023u; }
+
 // ---------------------------------------------------------------------------
 // Kernel
 // ---------------------------------------------------------------------------
@@ -296,8 +304,6 @@ __global__ void __launch_bounds__(G_THREADS, 1) tc_grouped_gemm(const __grid_con
     __shared__ __align__(8) uint64_t sf_full[G_SF_RING];   // A4: a step's scale-factor chunks are in place
     __shared__ int s_hold;
     __shared__ uint32_t s_tmem;
-    __shared__ int s_active[kMaxE];
-    __shared__ int s_prefix[kMaxE];
     __shared__ int s_wsum[G_THREADS / 32], s_wt[G_THREADS / 32];
     __shared__ int s_nact, s_total;
     __shared__ volatile GAbort s_ab;
@@ -325,7 +331,7 @@ __global__ void __launch_bounds__(G_THREADS, 1) tc_grouped_gemm(const __grid_con
                 asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(g_smem(&pk_empty[s])), "r"(C::kDqArrivals));
         }
         for (int s = 0; s < C::kBStages; s++)   // i8: one asynchronous arrival per lane of the copying warp
-            asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(g_smem(&b_full[s])), "r"(C::kI8 ? 32 : 1));
+            asm volatile("mbarrier.init.shared::cta.b64 [%0], 1;" ::"r"(g_smem(&b_full[s])));
         for (int s = 0; s < C::kAStages; s++)
             asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(g_smem(&a_full[s])), "r"(C::kDqArrivals));
         for (int s = 0; s < G_DONE; s++)
@@ -356,14 +362,19 @@ __global__ void __launch_bounds__(G_THREADS, 1) tc_grouped_gemm(const __grid_con
         s_hold = g_hold_from(a.status);
     }
 
-    // tile list: active experts and the prefix sum of their tile counts
+    // Tile list: per active expert {expert, first tile, first row, rows}, in dynamic shared memory
+    // ahead of the stage rings (every role looks a tile up here, with no global load)
+    uint8_t* dbase = smem + ((1024u - (g_smem(smem) & 1023u)) & 1023u);
+    int4* tbl = reinterpret_cast<int4*>(dbase);
     {
         constexpr int PER = kMaxE / G_THREADS;
-        int cnt[PER], nt[PER], local = 0, ltiles = 0;
+        int cnt[PER], nt[PER], eb[PER], ne[PER], local = 0, ltiles = 0;
 #pragma unroll
         for (int i = 0; i < PER; i++) {
             const int e = tid * PER + i;
-            const int n = (e < a.E) ? a.offsets[e + 1] - a.offsets[e] : 0;
+            eb[i] = (e < a.E) ? a.offsets[e] : 0;
+            const int n = (e < a.E) ? a.offsets[e + 1] - eb[i] : 0;
+            ne[i] = n;
             cnt[i] = n > 0;
             nt[i] = n > 0 ? ((n + C::kNMax - 1) / C::kNMax) * MT * ksplit : 0;
             local += cnt[i];
@@ -387,7 +398,7 @@ __global__ void __launch_bounds__(G_THREADS, 1) tc_grouped_gemm(const __grid_con
         int pos = base + v - local, tpos = tbase + w - ltiles;
 #pragma unroll
         for (int i = 0; i < PER; i++)
-            if (cnt[i]) { s_active[pos] = tid * PER + i; s_prefix[pos] = tpos; pos++; tpos += nt[i]; }
+            if (cnt[i]) { tbl[pos] = make_int4(tid * PER + i, tpos, eb[i], ne[i]); pos++; tpos += nt[i]; }
         if (tid == 0) { s_nact = tot; s_total = ttot; }
         __syncthreads();
     }
@@ -395,7 +406,7 @@ __global__ void __launch_bounds__(G_THREADS, 1) tc_grouped_gemm(const __grid_con
 
     const uint32_t tmem = s_tmem;
     const int ntiles = s_total, nact = s_nact;
-    uint8_t* pk = smem + ((1024u - (g_smem(smem) & 1023u)) & 1023u);
+    uint8_t* pk = dbase + g_tbl_bytes(a.E);
     uint8_t* bring = pk + NPK * C::kPkStageBytes;
     uint8_t* scbuf = bring + C::kBStages * C::kBStageBytes;         // int4: NSC buffers of sc_buf_bytes
     uint8_t* sfring = scbuf;                                        // A4: G_SF_RING slots of kSfSlotBytes (no int4 buffers)
@@ -404,13 +415,14 @@ __global__ void __launch_bounds__(G_THREADS, 1) tc_grouped_gemm(const __grid_con
         int lo = 0, hi = nact - 1;
         while (lo < hi) {
             const int mid = (lo + hi + 1) >> 1;
-            if (s_prefix[mid] <= tile) lo = mid; else hi = mid - 1;
+            if (tbl[mid].y <= tile) lo = mid; else hi = mid - 1;
         }
+        const int4 te = tbl[lo];
         GTile t;
-        t.e = s_active[lo];
-        const int local = tile - s_prefix[lo];
-        t.ebase = a.offsets[t.e];
-        const int n_e = a.offsets[t.e + 1] - t.ebase;
+        t.e = te.x;
+        const int local = tile - te.y;
+        t.ebase = te.z;
+        const int n_e = te.w;
         const int ntile = (n_e + C::kNMax - 1) / C::kNMax;
         const int per = (n_e + ntile - 1) / ntile;                  // balanced rows per n-tile
         t.ks = local % ksplit;                                      // K slice fastest
@@ -527,26 +539,15 @@ __global__ void __launch_bounds__(G_THREADS, 1) tc_grouped_gemm(const __grid_con
                 }
                 const uint32_t bar = g_smem(&b_full[s]);
                 const uint32_t st = g_smem(bring + s * C::kBStageBytes);
-                if (C::kI8) {
-                    // lane: digit row n = lane / 2 of the tile and the 128-byte K slices h, h + 2, ... of the
-                    // stage, each as eight 16-byte chunks at their 128-byte-swizzled places; rows past the end
-                    // read as zero
-                    const int n = lane >> 1;
-                    const int grow = row0 + n;
-                    const bool in_rows = grow < 3 * a.rows;
-                    const uint8_t* src = a.bdig + size_t(in_rows ? grow : 0) * in_dim + T.kbase + ks * C::kSK;
-#pragma unroll
-                    for (int h = lane & 1; h < C::kBAtoms; h += 2) {
-                        const uint32_t dst = st + h * C::kBAtom + n * 128;
-#pragma unroll
-                        for (int c = 0; c < 8; c++)
-                            g_cp16(dst + ((c ^ (n & 7)) << 4), src + h * 128 + c * 16, in_rows ? 16u : 0u);
-                    }
-                    g_cp_arrive(bar);
-                    continue;
-                }
                 if (g_elect()) {
-                    if constexpr (C::kA4) {
+                    if constexpr (C::kI8) {
+                        // 16 digit rows (128-byte swizzled) per 128-byte K slice of the step; rows past the
+                        // problem's last read as zero
+                        g_expect(bar, uint32_t(C::kBStageBytes));
+#pragma unroll
+                        for (int h = 0; h < C::kBAtoms; h++)
+                            g_tma2d(st + h * C::kBAtom, map, T.kbase + ks * C::kSK + h * 128, row0, bar);
+                    } else if constexpr (C::kA4) {
                         // K 256 of packed E2M1 (128 bytes per row, swizzled) and the rows' 16 scale bytes
                         g_expect(bar, uint32_t(T.bn) * (128u + 16u));
                         g_tma2d(st, map, (T.kbase + ks * C::kSK) / 2, row0, bar);
@@ -597,8 +598,18 @@ __global__ void __launch_bounds__(G_THREADS, 1) tc_grouped_gemm(const __grid_con
                     continue;
                 }
                 const int sb = bc % C::kBStages, sa = ac % C::kAStages;
+                if (C::kI8) {
+                    // every step into the next accumulator buffer, freed by the epilogue.  This wait comes
+                    // first: the two issuers take alternate steps and the A ring is odd, so the step that
+                    // last filled A stage sa (ac - kAStages) was the other issuer's; the release of step
+                    // bc - kAccBufs means the epilogue, which goes in order, has seen every earlier step,
+                    // so that fill has landed and the parity wait on a_full below cannot pass a phase early
+                    const int bi = bc % C::kAccBufs;
+                    if (bc >= uint32_t(C::kAccBufs) &&
+                        !g_wait_w(g_smem(&acc_empty[bi]), ((bc / C::kAccBufs) - 1) & 1, &s_ab)) { ok = false; break; }
+                    d = tmem + bi * C::kAccCols;
+                }
                 if (!g_wait_w(g_smem(&b_full[sb]), (bc / C::kBStages) & 1, &s_ab)) { ok = false; break; }
-                if (C::kI8) g_fence_proxy_async();      // B was written through the generic proxy
                 if (C::kTmemA) {
                     if (!g_wait_w(g_smem(&a_full[sa]), (ac / C::kAStages) & 1, &s_ab)) { ok = false; break; }
                 } else {
@@ -607,13 +618,6 @@ __global__ void __launch_bounds__(G_THREADS, 1) tc_grouped_gemm(const __grid_con
                 if (C::kA4 && !g_wait_w(g_smem(&sf_full[bc % G_SF_RING]), (bc / G_SF_RING) & 1, &s_ab)) {
                     ok = false;
                     break;
-                }
-                if (C::kI8) {
-                    // every step into the next accumulator buffer, freed by the epilogue
-                    const int bi = bc % C::kAccBufs;
-                    if (bc >= uint32_t(C::kAccBufs) &&
-                        !g_wait_w(g_smem(&acc_empty[bi]), ((bc / C::kAccBufs) - 1) & 1, &s_ab)) { ok = false; break; }
-                    d = tmem + bi * C::kAccCols;
                 }
                 g_fence_after();
                 const uint32_t b0 = g_smem(bring + sb * C::kBStageBytes);
@@ -953,7 +957,20 @@ __global__ void __launch_bounds__(G_THREADS, 1) tc_grouped_gemm(const __grid_con
             for (int ps = 0; ps < NPS; ps++, pc++) {
                 if (int(pc & 1) != grp) continue;
                 const int s = pc % NPK;
-                if (!g_wait_w(g_smem(&pk_full[s]), (pc / NPK) & 1, &s_ab)) { ok = false; break; }
+                // A stage sa is free once the MMA of step pc - kAStages has completed.  A parity wait
+                // only tells a phase from the one before it, so a wait on pk_full[s] must come after the
+                // stage's previous fill (step pc - NPK) has landed.  With an even ring that step was
+                // this group's own; with an odd one it was the other group's, and the release of A stage
+                // sa (every step up to pc - kAStages unpacked, NPK >= kAStages) comes first.
+                const int sa = pc % C::kAStages;
+                auto a_free = [&]() {
+                    return pc < uint32_t(C::kAStages) ||
+                           g_wait_w(g_smem(&done[(pc - C::kAStages) % G_DONE]), ((pc - C::kAStages) / G_DONE) & 1, &s_ab);
+                };
+                if (((NPK & 1) && !a_free()) || !g_wait_w(g_smem(&pk_full[s]), (pc / NPK) & 1, &s_ab)) {
+                    ok = false;
+                    break;
+                }
                 const uint8_t* st = pk + s * C::kPkStageBytes;
                 uint32_t o[kNBuf][16];
                 uint4 raw[2][2];                                // packed chunks, loaded one piece ahead
@@ -973,9 +990,7 @@ __global__ void __launch_bounds__(G_THREADS, 1) tc_grouped_gemm(const __grid_con
                 load(std::integral_constant<int, 0>{});
                 if constexpr (kPieces > 1) load(std::integral_constant<int, 1>{});
                 unpack(std::integral_constant<int, 0>{});
-                const int sa = pc % C::kAStages;
-                if (pc >= uint32_t(C::kAStages) && !g_wait_w(g_smem(&done[(pc - C::kAStages) % G_DONE]),
-                                                             ((pc - C::kAStages) / G_DONE) & 1, &s_ab)) {
+                if (!(NPK & 1) && !a_free()) {
                     ok = false;
                     break;
                 }
@@ -1319,9 +1334,9 @@ __global__ void __launch_bounds__(256) g_splitk_finish(const float* __restrict__
 // Host side
 // ---------------------------------------------------------------------------
 template <int FMT, bool GU, bool W>
-static size_t g_smem_bytes(int in_dim, int npk, int nsc) {
+static size_t g_smem_bytes(int in_dim, int npk, int nsc, int E) {
     using C = GCfg<FMT, GU, W>;
-    size_t b = size_t(npk) * C::kPkStageBytes + size_t(C::kBStages) * C::kBStageBytes + 1024;
+    size_t b = g_tbl_bytes(E) + size_t(npk) * C::kPkStageBytes + size_t(C::kBStages) * C::kBStageBytes + 1024;
     if (C::kInt4) b += size_t(nsc) * (C::kNMat * G_BM * (in_dim / 128) * 2 + (C::kI8 ? C::kNMax * (((in_dim / 128) + 3) & ~3) * 4 : 0));
     if (C::kA4) b += size_t(G_SF_RING) * C::kSfSlotBytes;
     return b;
@@ -1346,13 +1361,13 @@ static int g_launch(const GArgs& a, cudaStream_t s) {
     int npk = C::kPkMax, nsc = 2;
     for (; npk >= 2; npk--) {
         nsc = C::kInt4 ? std::min(G_SC_MAX, std::max(2, (npk + nps - 1) / nps + 1)) : 2;
-        if (g_smem_bytes<FMT, GU, W>(a.in_dim, npk, nsc) <= room) break;
+        if (g_smem_bytes<FMT, GU, W>(a.in_dim, npk, nsc, a.E) <= room) break;
     }
     if (npk < 2) return MOE_ERR_UNSUPPORTED;
     GArgs args = a;
     args.npk = npk;
     args.nsc = nsc;
-    const size_t smem = g_smem_bytes<FMT, GU, W>(a.in_dim, npk, nsc);
+    const size_t smem = g_smem_bytes<FMT, GU, W>(a.in_dim, npk, nsc, a.E);
     if (cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem)) != cudaSuccess)
         return MOE_ERR_CUDA;
     return launch_pdl(k, dim3(sms), dim3(G_THREADS), smem, s, args) == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
@@ -1427,7 +1442,8 @@ int launch_grouped_gemm(const GemvProblem& p, bool gateup, int rows, const GemmB
         if (gateup) G_TRY(g_map(&a.tm_s1, false, p.s1, in / 16, wrows, uint64_t(in) / 16, 16, 128, false));
     }
     if (i8) {
-        a.bdig = static_cast<const uint8_t*>(bsrc);
+        // three digit rows per activation row, 16 rows and 128 bytes of K per box
+        G_TRY(g_map(&a.tm_b[0], false, bsrc, in, uint64_t(rows) * 3, uint64_t(in), 128, 16, true));
     } else if (a4) {
         const uint8_t* codes = static_cast<const uint8_t*>(bsrc);
         for (int i = 0; i < G_NB_MAPS; i++) {

@@ -123,19 +123,26 @@ __global__ void __launch_bounds__(256) router_logits_tiled(
 // score) above the complement of its id (so equal scores prefer the lower id);
 // 0 marks an empty or taken slot.  A lane keeps the largest of its keys; a pick
 // is one warp-wide maximum, after which only the lane that owned the winner
-// rescans its keys.
+// rescans its keys.  STAGED: lrow and bias are in shared memory (bias not
+// null), and the ids also go to ids_s.
 // ---------------------------------------------------------------------------
-template <int PER>
+template <int PER, bool STAGED = false>
 __device__ __forceinline__ void topk_warp(const float* __restrict__ lrow, const float* __restrict__ bias, int E,
-                                          int k, int32_t* __restrict__ ids, float* __restrict__ wout, int lane) {
+                                          int k, int32_t* __restrict__ ids, float* __restrict__ wout, int lane,
+                                          int32_t* ids_s = nullptr) {
     unsigned long long key[PER];
 #pragma unroll
     for (int i = 0; i < PER; i++) {
         const int e = lane + 32 * i;
         key[i] = 0ull;
         if (e < E) {
-            float l = __ldcg(lrow + e);       // written by other CTAs of the fused router
-            if (bias) l = l + bias[e];
+            float l;
+            if constexpr (STAGED) {
+                l = lrow[e] + bias[e];
+            } else {
+                l = lrow[e];
+                if (bias) l = l + bias[e];
+            }
             const float v = 1.0f / (1.0f + expf(-l));
             key[i] = (static_cast<unsigned long long>(__float_as_uint(v)) << 32) | static_cast<uint32_t>(~e);
         }
@@ -168,6 +175,7 @@ __device__ __forceinline__ void topk_warp(const float* __restrict__ lrow, const 
     if (lane < k) {
         ids[lane] = my_id;
         wout[lane] = my_s / sum;
+        if constexpr (STAGED) ids_s[lane] = my_id;
     }
 }
 
@@ -313,9 +321,37 @@ __global__ void __launch_bounds__(RD_WARPS * 32) router_decode(RouterDecodeArgs 
     __syncthreads();
     if (!s_last) return;
     __threadfence();
+    // Every token's logits (written by the other CTAs: read at L2) and the bias into shared memory,
+    // each thread's loads all issued before its stores, so the tail waits for one round of loads
+    float* lg = reinterpret_cast<float*>(rsm);               // [T][E] (x staging is no longer needed)
+    float* bs = lg + a.T * a.E;                              // [E]
+    int32_t* ids_s = reinterpret_cast<int32_t*>(bs + a.E);   // [T][k]
+    int32_t* cnt = ids_s + a.T * a.k;                        // [E]
+    {
+        constexpr int LPT = 16;
+        const int n = a.T * a.E, nb = n + a.E;
+        for (int i0 = 0; i0 < nb; i0 += LPT * RD_WARPS * 32) {
+            float v[LPT];
+#pragma unroll
+            for (int j = 0; j < LPT; j++) {
+                const int i = i0 + j * RD_WARPS * 32 + threadIdx.x;
+                v[j] = i < n ? __ldcg(a.logits + i) : (i < nb && a.bias ? a.bias[i - n] : 0.f);
+            }
+#pragma unroll
+            for (int j = 0; j < LPT; j++) {
+                const int i = i0 + j * RD_WARPS * 32 + threadIdx.x;
+                if (i < nb) lg[i] = v[j];
+            }
+        }
+    }
+    __syncthreads();
     for (int t = warp; t < a.T; t += RD_WARPS) {
-        if (a.E <= 384) topk_warp<12>(a.logits + size_t(t) * a.E, a.bias, a.E, a.k, a.ids + size_t(t) * a.k, a.w + size_t(t) * a.k, lane);
-        else topk_warp<kMaxE / 32>(a.logits + size_t(t) * a.E, a.bias, a.E, a.k, a.ids + size_t(t) * a.k, a.w + size_t(t) * a.k, lane);
+        if (a.E <= 384)
+            topk_warp<12, true>(lg + t * a.E, bs, a.E, a.k, a.ids + size_t(t) * a.k, a.w + size_t(t) * a.k, lane,
+                                ids_s + t * a.k);
+        else
+            topk_warp<kMaxE / 32, true>(lg + t * a.E, bs, a.E, a.k, a.ids + size_t(t) * a.k, a.w + size_t(t) * a.k,
+                                        lane, ids_s + t * a.k);
     }
     if (threadIdx.x == 0) *a.counter = 0;
     if (a.sh_offsets) {
@@ -323,15 +359,14 @@ __global__ void __launch_bounds__(RD_WARPS * 32) router_decode(RouterDecodeArgs 
         for (int i = threadIdx.x; i < a.T; i += blockDim.x) a.sh_rowslot[i] = i * a.k;
     }
     if (!a.offsets) return;
-    __syncthreads();                       // ids of every token written (by this CTA)
-    // stable counting sort of the R <= 128 slots by expert id
-    int32_t* cnt = reinterpret_cast<int32_t*>(rsm);          // [E] (x staging is no longer needed)
+    __syncthreads();                       // ids of every token in ids_s
+    // stable counting sort of the R <= T * k slots by expert id
     __shared__ int s_wsum[RD_WARPS];
     const int R = a.T * a.k;
     for (int i = threadIdx.x; i < a.E; i += blockDim.x) cnt[i] = 0;
     __syncthreads();
     for (int sl = threadIdx.x; sl < R; sl += blockDim.x) {
-        const int id = a.ids[sl];
+        const int id = ids_s[sl];
         if (id >= 0 && id < a.E) atomicAdd(&cnt[id], 1);
         else set_status(a.status, MOE_ERR_DEVICE_INDEX);
     }
@@ -363,7 +398,7 @@ __global__ void __launch_bounds__(RD_WARPS * 32) router_decode(RouterDecodeArgs 
         const unsigned lt = (1u << lane) - 1u;
         for (int s0 = 0; s0 < R; s0 += 32) {
             const int sl = s0 + lane;
-            const int id = (sl < R) ? a.ids[sl] : -1;
+            const int id = (sl < R) ? ids_s[sl] : -1;
             const bool ok = id >= 0 && id < a.E;
             const unsigned act = __ballot_sync(0xffffffffu, ok);
             const unsigned peers = __match_any_sync(0xffffffffu, ok ? id : -1) & act;
@@ -381,7 +416,8 @@ __global__ void __launch_bounds__(RD_WARPS * 32) router_decode(RouterDecodeArgs 
 }
 
 int launch_route_decode(const RouterDecodeArgs& a, cudaStream_t s) {
-    const size_t smem = std::max<size_t>(size_t(a.T) * a.H * 2, size_t(a.E) * 4);
+    // x staging, then (the last CTA) logits, bias, ids and the bucket counters
+    const size_t smem = std::max<size_t>(size_t(a.T) * a.H * 2, (size_t(a.T) * a.E + 2 * size_t(a.E) + size_t(a.T) * a.k) * 4);
     if (a.T > RD_TMAX || a.H % 512) return MOE_ERR_UNSUPPORTED;
     auto k = a.x_f16 ? router_decode<true> : router_decode<false>;
     if (smem > 48 * 1024 &&

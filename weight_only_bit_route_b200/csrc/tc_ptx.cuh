@@ -169,15 +169,6 @@ __device__ __forceinline__ void g_st16(uint32_t taddr, const uint32_t (&v)[16]) 
                    "r"(v[8]), "r"(v[9]), "r"(v[10]), "r"(v[11]), "r"(v[12]), "r"(v[13]), "r"(v[14]), "r"(v[15])
                  : "memory");
 }
-// 16-byte global -> shared copy outside the tensor-copy engine (zero fill past
-// src_size), and an mbarrier arrival (counted against the expected arrivals)
-// once every such copy of the calling thread has landed.
-__device__ __forceinline__ void g_cp16(uint32_t dst, const void* src, uint32_t src_size) {
-    asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(dst), "l"(src), "r"(src_size) : "memory");
-}
-__device__ __forceinline__ void g_cp_arrive(uint32_t bar) {
-    asm volatile("cp.async.mbarrier.arrive.noinc.shared::cta.b64 [%0];" ::"r"(bar) : "memory");
-}
 __device__ __forceinline__ void g_fence_proxy_async() { asm volatile("fence.proxy.async.shared::cta;" ::: "memory"); }
 __device__ __forceinline__ void g_st_wait() { asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory"); }
 __device__ __forceinline__ uint32_t g_e2m1x2_f16x2(uint32_t byte) {
