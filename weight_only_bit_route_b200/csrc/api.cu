@@ -150,6 +150,10 @@ int side_stream(SideStream** out) {
     return MOE_OK;
 }
 
+// SMs the BF16 shared expert's GEMMs may take at decode sizes (T <= 16): its 38 MB stream in
+// about the time the router and the first pre-pass take on the other SMs.
+constexpr int kSharedDecodeCtas = 32;
+
 int layer_run(const void* x, int T, const moe_layer* L, void* y, void* ws, cudaStream_t s) {
     const int H = L->H, E = L->E, F = L->F, k = L->top_k;
     const WsLayout W = ws_layout(T, H, E, F, k);
@@ -175,8 +179,11 @@ int layer_run(const void* x, int T, const moe_layer* L, void* y, void* ws, cudaS
 
     // The shared expert needs x only: it runs on a side stream while the
     // router, the bucketing and the routed experts run on `s`, and `s` waits
-    // for it before the combine.  Its own routing (offsets {0, T}, row i at
-    // slot i * top_k) comes first on that stream.
+    // for it before the combine.  The router is launched first (it starts the
+    // critical path); the shared expert's own routing (offsets {0, T}, row i at
+    // slot i * top_k) comes first on its stream.  At decode sizes its GEMMs take
+    // at most kSharedDecodeCtas SMs and no early launch, so the router's CTAs
+    // find SMs free beside them and no waiting CTA holds an SM.
     SideStream* side = nullptr;
     std::unique_lock<std::mutex> side_lock;
     if (has_sh) {
@@ -184,6 +191,23 @@ int layer_run(const void* x, int T, const moe_layer* L, void* y, void* ws, cudaS
         side_lock = std::unique_lock<std::mutex>(side->call);
         if (cudaEventRecord(side->fork, s) != cudaSuccess || cudaStreamWaitEvent(side->s, side->fork, 0) != cudaSuccess)
             return MOE_ERR_CUDA;
+    }
+
+    if (T <= kRouterDecodeMaxT && router_decode_ok(H)) {
+        // router, top-k and bucketing in one launch
+        RouterDecodeArgs ra{};
+        ra.x = xb; ra.T = T; ra.H = H; ra.Wr = L->router_w; ra.bias = L->router_bias; ra.E = E; ra.k = k;
+        ra.logits = at<float>(ws, W.logits); ra.ids = ids; ra.w = tw; ra.counter = counter; ra.status = status;
+        ra.offsets = offsets; ra.row_slot = row_slot; ra.slot_row = slot_row;
+        ra.sh_offsets = nullptr; ra.sh_rowslot = nullptr; ra.x_f16 = x_f16;
+        MOE_TRY(launch_route_decode(ra, s));
+    } else {
+        MOE_TRY(launch_route(xb, T, H, L->router_w, L->router_bias, E, k, ids, tw, at<float>(ws, W.logits),
+                             at<__nv_bfloat16>(ws, W.wsplit), status, counter, s, x_f16));
+        MOE_TRY(launch_permute(ids, T, k, E, offsets, row_slot, slot_row, at<int32_t>(ws, W.hist), status, s));
+    }
+
+    if (has_sh) {
         // fp16 mode: the BF16 shared expert reads x rounded to bf16, staged in its output region (the
         // down projection overwrites it only after the gate/up projection has read it)
         const __nv_bfloat16* xs = xb;
@@ -202,25 +226,16 @@ int layer_run(const void* x, int T, const moe_layer* L, void* y, void* ws, cudaS
         // the shared expert reads x and its own h directly (identity routing, natural order)
         GemmBuffers direct{};
         direct.act_ready = 1;
+        direct.max_expert_rows = T;
+        if (T <= kRouterDecodeMaxT) {
+            direct.max_ctas = kSharedDecodeCtas;
+            direct.no_pdl = 1;
+        }
         float* shpart = at<float>(ws, W.shpart);
         MOE_TRY(launch_shared_routing(T, k, sh_off, sh_rs, side->s));
         MOE_TRY(run_problem(sg, true, T, T, nullptr, direct, shpart, side->s));
         MOE_TRY(run_problem(sd, false, T, T, nullptr, direct, shpart, side->s));
         if (cudaEventRecord(side->join, side->s) != cudaSuccess) return MOE_ERR_CUDA;
-    }
-
-    if (T <= kRouterDecodeMaxT && router_decode_ok(H)) {
-        // router, top-k and bucketing in one launch
-        RouterDecodeArgs ra{};
-        ra.x = xb; ra.T = T; ra.H = H; ra.Wr = L->router_w; ra.bias = L->router_bias; ra.E = E; ra.k = k;
-        ra.logits = at<float>(ws, W.logits); ra.ids = ids; ra.w = tw; ra.counter = counter; ra.status = status;
-        ra.offsets = offsets; ra.row_slot = row_slot; ra.slot_row = slot_row;
-        ra.sh_offsets = nullptr; ra.sh_rowslot = nullptr; ra.x_f16 = x_f16;
-        MOE_TRY(launch_route_decode(ra, s));
-    } else {
-        MOE_TRY(launch_route(xb, T, H, L->router_w, L->router_bias, E, k, ids, tw, at<float>(ws, W.logits),
-                             at<__nv_bfloat16>(ws, W.wsplit), status, counter, s, x_f16));
-        MOE_TRY(launch_permute(ids, T, k, E, offsets, row_slot, slot_row, at<int32_t>(ws, W.hist), status, s));
     }
     const bool routed_gemm = gemm_shape_ok(H, F) && gemm_shape_ok(F, H);
 
@@ -241,6 +256,8 @@ int layer_run(const void* x, int T, const moe_layer* L, void* y, void* ws, cudaS
         // 16-bit gate/up activation rows are gathered into the y_perm region,
         // free until the down projection writes it
         GemmBuffers gb = gemm_buffers(prep, R, H, false, i8);
+        gb.sched = status + 8;             // tiles handed out as CTAs get SMs (the shared expert may hold some)
+        gb.max_expert_rows = T;            // a token routes to an expert at most once
         if (!i8) gb.act_buf = y_perm;
         MOE_TRY(launch_grouped_gemm(gu, true, R, gb, s));
     } else {
@@ -248,6 +265,8 @@ int layer_run(const void* x, int T, const moe_layer* L, void* y, void* ws, cudaS
     }
     if (routed_gemm) {
         GemmBuffers db = gemm_buffers(prep, R, F, false, i8);
+        db.sched = status + 8;
+        db.max_expert_rows = T;
         MOE_TRY(launch_grouped_gemm(dn, false, R, db, s));
     } else {
         MOE_TRY(launch_stream_gemv(dn, nullptr, false, R, prep, s, true));
@@ -288,9 +307,10 @@ int moe_read_status(void* ws, moe_stream_t stream, int32_t* status_out) {
     if (cudaStreamSynchronize(cs(stream)) != cudaSuccess) return MOE_ERR_CUDA;
     *status_out = v;
     if (v != 0) {
-        // a kernel that stopped early may have left its arrival counters (router word 1,
-        // split-K words 16..255) non-zero: clear them with the status word
+        // a kernel that stopped early may have left its arrival counters (router word 1, tile
+        // scheduler words 8-9, split-K words 16..255) non-zero: clear them with the status word
         if (cudaMemsetAsync(ws, 0, 8, cs(stream)) != cudaSuccess) return MOE_ERR_CUDA;
+        if (cudaMemsetAsync(at<int32_t>(ws, 32), 0, 8, cs(stream)) != cudaSuccess) return MOE_ERR_CUDA;
         if (cudaMemsetAsync(at<int32_t>(ws, 64), 0, kStepScratch - 64, cs(stream)) != cudaSuccess) return MOE_ERR_CUDA;
     }
     return MOE_OK;
@@ -391,8 +411,10 @@ int moe_grouped_w4a16_swiglu(const void* x, int T, int H, const int32_t* expert_
     p.out = reinterpret_cast<__nv_bfloat16*>(h_perm); p.status = at<int32_t>(ws, 0);
     p.in_scale = gate->input_scale;
     void* prep = at<void>(ws, kStepScratch + align256(size_t(E + 2) * 16));
-    return run_problem(p, true, rows, T, prep, gemm_buffers(prep, rows, H, false, i8_int4(p, rows)),
-                       step_partial(ws, E, rows, H), cs(stream));
+    GemmBuffers b = gemm_buffers(prep, rows, H, false, i8_int4(p, rows));
+    b.sched = p.status + 8;
+    b.max_expert_rows = T;
+    return run_problem(p, true, rows, T, prep, b, step_partial(ws, E, rows, H), cs(stream));
 }
 
 int moe_grouped_w4a16_down(const void* h_perm, const int32_t* expert_offsets, const int32_t* row_slot,
@@ -416,9 +438,10 @@ int moe_grouped_w4a16_down(const void* h_perm, const int32_t* expert_offsets, co
     p.in_scale = down->input_scale;
     void* prep = at<void>(ws, kStepScratch + align256(size_t(E + 2) * 16));
     // BF16 rows are read in place (row r is activation row r)
-    return run_problem(p, false, rows, rows, prep,
-                       gemm_buffers(prep, rows, F, down->fmt == MOE_FMT_BF16, i8_int4(p, rows)),
-                       step_partial(ws, E, rows, F), cs(stream));
+    GemmBuffers b = gemm_buffers(prep, rows, F, down->fmt == MOE_FMT_BF16, i8_int4(p, rows));
+    b.sched = p.status + 8;
+    b.max_expert_rows = rows;
+    return run_problem(p, false, rows, rows, prep, b, step_partial(ws, E, rows, F), cs(stream));
 }
 
 int moe_unpermute_combine(const void* y_perm, const int32_t* slot_row, int T, int top_k, int H,

@@ -72,7 +72,9 @@
 #include <cuda_fp16.h>
 
 #include <algorithm>
+#include <atomic>
 #include <cstring>
+#include <mutex>
 #include <type_traits>
 
 #include "moe_internal.cuh"
@@ -108,20 +110,25 @@ constexpr int FMT_INT4_I8 = 3;
 constexpr int FMT_NVFP4_A4 = 4;
 constexpr int G_SF_RING = 4;                 // A4: scale-factor slots (shared and tensor memory)
 
-// W (wide): gate/up tiles of up to 128 token rows instead of 64, for batches
-// whose experts hold many rows: each dequantised weight then serves twice the
-// tokens.  The 4-bit formats keep a single accumulator buffer of 256 columns
-// (gate, up) and two A stages; BF16 (no A stages) keeps two buffers.
-template <int FMT, bool GU, bool W = false>
+// NW: tile width class.  1 (wide): gate/up tiles of up to 128 token rows
+// instead of 64, for batches whose experts hold many rows: each dequantised
+// weight then serves twice the tokens.  The 4-bit formats keep a single
+// accumulator buffer of 256 columns (gate, up) and two A stages; BF16 (no A
+// stages) keeps two buffers.  2 (narrow, BF16 and NVFP4 16-bit): at most 16
+// token rows per tile, for decode batches (an expert holds at most one row per
+// token): the activation stages shrink to 2 KB per K 64, and shared memory
+// goes to weight stages in flight instead.
+template <int FMT, bool GU, int NW = 0>
 struct GCfg {
     static constexpr bool kI8 = FMT == FMT_INT4_I8;
     static constexpr bool kA4 = FMT == FMT_NVFP4_A4;
     static constexpr bool kInt4 = FMT == MOE_FMT_INT4_G128 || kI8;
     static constexpr bool kTmemA = FMT != MOE_FMT_BF16 && !kA4;     // A dequantised into tensor memory
     static constexpr bool kPacked = kTmemA || kA4;                    // 4-bit weight stages (128 B = K 256 per row)
-    static constexpr bool kWide = W && GU && !kI8;
+    static constexpr bool kWide = NW == 1 && GU && !kI8;
+    static constexpr bool kNarrow = NW == 2 && !kI8;
     static constexpr int kNMat = GU ? 2 : 1;
-    static constexpr int kNMax = kI8 ? 5 : (GU ? (kWide ? 128 : 64) : 128);   // token rows per tile
+    static constexpr int kNMax = kI8 ? 5 : (kNarrow ? 16 : (GU ? (kWide ? 128 : 64) : 128));   // token rows per tile
     static constexpr int kUpCol = kWide ? 128 : 64;                 // 16-bit paths: up accumulator within a buffer
     // K per MMA step: 8-bit down steps are K = 512, so that the per-step fixed cost of the
     // issuer and the unpack warps covers 32 KB of weights, as a gate/up step does
@@ -151,7 +158,7 @@ struct GCfg {
     static constexpr int kSfSlotBytes = kSfChunks * 512;
     static constexpr int kSfSlotCols = kSfChunks * 4;
     // i8 stages are small: cover the copy latency; wide stages are large: fit shared memory
-    static constexpr int kBStages = kI8 ? (GU ? 6 : 4) : (kWide ? (kTmemA ? 3 : 2) : 4);
+    static constexpr int kBStages = kI8 ? (GU ? 6 : 4) : (kWide ? (kTmemA ? 3 : 2) : (kNarrow ? 6 : 4));
     static constexpr int kAColsK = kI8 ? kSK / 4 : 64;              // TMEM columns of one matrix's A stage
     static constexpr int kAStageCols = kNMat * kAColsK;
     static constexpr int kAStages = kTmemA ? (512 - kABase) / kAStageCols : 1;   // (BF16, A4: none used)
@@ -159,6 +166,9 @@ struct GCfg {
     static constexpr int kChunkCols = 16;                           // 16-bit paths: TMEM columns of one packed chunk
     static constexpr int kDqArrivals = kI8 ? G_DQ_WARPS / 2 : G_DQ_WARPS;  // warps that fill one stage
     static constexpr bool kMmaF16 = FMT == MOE_FMT_NVFP4 || FMT == MOE_FMT_INT4_G128;   // f16 operands
+    // warps that read the tile queue: activation producer, MMA issuer(s), epilogue, and the
+    // scale-factor (A4) or dequantisation / unpacking warps
+    static constexpr int kQReaders = 1 + (kI8 ? 2 : 1) + G_EPI_WARPS + (kA4 ? 4 : (kTmemA ? G_DQ_WARPS : 0));
     static_assert(kABase <= 512 && (!kTmemA || kAStages >= 2), "tensor memory layout");
     // the 8-bit path's two MMA issuers take alternate steps: even B and accumulator rings give each
     // the slots it alone waits on, so it sees every phase of them in order; an issuer's accumulator
@@ -169,6 +179,7 @@ struct GCfg {
 };
 
 constexpr int G_DONE = 16;                                          // "stage done" barrier ring
+constexpr int G_TQ = 16;                                            // tile queue: tile ids the producer hands out
 constexpr int G_SC_MAX = 8;                                         // int4 scale buffers (one tile each)
 constexpr int G_KSPLIT_MAX = 8;                                     // split-K slices summed inside the GEMM
 
@@ -195,6 +206,8 @@ struct GArgs {
     int ksplit, rows;                // K slices per (m-tile, n-tile); activation rows of the problem
     int* tile_cnt;                   // split-K: zeroed arrival counters, four per (m-tile, n-tile); the last
                                      // epilogue warp of each quarter sums the slices (else a kernel does)
+    int* sched;                      // null: tile blockIdx.x + i * gridDim.x; else {next, done}: tiles handed out by
+                                     // an atomic counter, zero on entry, left at zero by the last CTA
     int npk;                         // weight stages in the shared-memory ring (2 .. kPkMax)
     int nsc;                         // int4 scale buffers (2 .. G_SC_MAX)
 };
@@ -292,9 +305,9 @@ __device__ __forceinline__ void g_static_for(F&& f) {
     }
 }
 
-template <int FMT, bool GU, bool W>
+template <int FMT, bool GU, int NW>
 __global__ void __launch_bounds__(G_THREADS, 1) tc_grouped_gemm(const __grid_constant__ GArgs a) {
-    using C = GCfg<FMT, GU, W>;
+    using C = GCfg<FMT, GU, NW>;
     extern __shared__ __align__(1024) uint8_t smem[];
     __shared__ __align__(8) uint64_t pk_full[C::kPkMax], pk_empty[C::kPkMax];
     __shared__ __align__(8) uint64_t b_full[C::kBStages], a_full[C::kAStages], done[G_DONE];
@@ -302,6 +315,9 @@ __global__ void __launch_bounds__(G_THREADS, 1) tc_grouped_gemm(const __grid_con
     __shared__ __align__(8) uint64_t acc_full[2], acc_empty[2], drain;
     __shared__ __align__(8) uint64_t hold_bar;        // failure testing: a barrier nothing completes
     __shared__ __align__(8) uint64_t sf_full[G_SF_RING];   // A4: a step's scale-factor chunks are in place
+    __shared__ __align__(8) uint64_t tq_full[G_TQ], tq_empty[G_TQ];   // tile queue
+    __shared__ int s_tq[G_TQ];
+    __shared__ int s_first;
     __shared__ int s_hold;
     __shared__ uint32_t s_tmem;
     __shared__ int s_wsum[G_THREADS / 32], s_wt[G_THREADS / 32];
@@ -348,6 +364,10 @@ __global__ void __launch_bounds__(G_THREADS, 1) tc_grouped_gemm(const __grid_con
         asm volatile("mbarrier.init.shared::cta.b64 [%0], 1;" ::"r"(g_smem(&hold_bar)));
         for (int s = 0; s < G_SF_RING; s++)       // A4: one arrival per scale-factor warp
             asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(g_smem(&sf_full[s])), "r"(4));
+        for (int s = 0; s < G_TQ; s++) {
+            asm volatile("mbarrier.init.shared::cta.b64 [%0], 1;" ::"r"(g_smem(&tq_full[s])));
+            asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(g_smem(&tq_empty[s])), "r"(C::kQReaders));
+        }
         asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
         s_ab.flag = 0;
         s_ab.limit_ns = G_WAIT_NS;
@@ -367,6 +387,9 @@ __global__ void __launch_bounds__(G_THREADS, 1) tc_grouped_gemm(const __grid_con
     uint8_t* dbase = smem + ((1024u - (g_smem(smem) & 1023u)) & 1023u);
     int4* tbl = reinterpret_cast<int4*>(dbase);
     {
+        // this CTA's first tile: asked for now, its latency hidden behind the scan below
+        int first = int(blockIdx.x);
+        if (tid == 0 && a.sched) first = atomicAdd(a.sched, 1);
         constexpr int PER = kMaxE / G_THREADS;
         int cnt[PER], nt[PER], eb[PER], ne[PER], local = 0, ltiles = 0;
 #pragma unroll
@@ -399,7 +422,7 @@ __global__ void __launch_bounds__(G_THREADS, 1) tc_grouped_gemm(const __grid_con
 #pragma unroll
         for (int i = 0; i < PER; i++)
             if (cnt[i]) { tbl[pos] = make_int4(tid * PER + i, tpos, eb[i], ne[i]); pos++; tpos += nt[i]; }
-        if (tid == 0) { s_nact = tot; s_total = ttot; }
+        if (tid == 0) { s_nact = tot; s_total = ttot; s_first = first; }
         __syncthreads();
     }
     asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
@@ -448,12 +471,47 @@ __global__ void __launch_bounds__(G_THREADS, 1) tc_grouped_gemm(const __grid_con
         set_status(a.status, MOE_ERR_TIMEOUT);
         s_ab.flag = 1;
     };
+    // Tile queue: warp 0 publishes, in order, every tile it starts and finally a value >= ntiles;
+    // the other roles take the same sequence.  A reader sees every phase of each slot in order (it
+    // took the slot's previous entry itself), and warp 0 reuses a slot only after all readers have
+    // taken its previous entry.  A wait that runs out ends the reader's loop (>= ntiles).
+    auto q_take = [&](uint32_t& qi) -> int {
+        const uint32_t slot = qi % G_TQ;
+        if (!g_wait_w(g_smem(&tq_full[slot]), (qi / G_TQ) & 1, &s_ab)) {
+            fail();
+            return ntiles;
+        }
+        const int v = *reinterpret_cast<volatile int*>(&s_tq[slot]);
+        __syncwarp();
+        if (lane == 0) g_arrive(g_smem(&tq_empty[slot]));
+        qi++;
+        return v;
+    };
 
     if (warp == 0) {
         // ---------------- weight producer (whole warp, one lane issues) ----------------
-        uint32_t pc = 0;
+        uint32_t pc = 0, qi = 0;
         int t = 0;
-        for (int tile = blockIdx.x; tile < ntiles && !g_aborted(&s_ab); tile += gridDim.x) {
+        int tile = s_first;
+        while (!g_aborted(&s_ab)) {
+            // hand the tile (or the end, >= ntiles) to the other roles
+            {
+                const uint32_t slot = qi % G_TQ;
+                if (qi >= G_TQ && !g_wait_w(g_smem(&tq_empty[slot]), ((qi / G_TQ) - 1) & 1, &s_ab, 32)) {
+                    fail();
+                    break;
+                }
+                if (lane == 0) {
+                    s_tq[slot] = tile;
+                    g_arrive(g_smem(&tq_full[slot]));
+                }
+                __syncwarp();
+                qi++;
+            }
+            if (tile >= ntiles) break;
+            // the next tile's id: asked for now, read when this tile's copies are issued
+            int nxt = 0;
+            if (lane == 0 && a.sched) nxt = atomicAdd(a.sched, 1);
             const GTile T = tile_of(tile);
             const int row0 = T.e * a.out_dim + T.m0;
             if (C::kInt4) {
@@ -513,6 +571,13 @@ __global__ void __launch_bounds__(G_THREADS, 1) tc_grouped_gemm(const __grid_con
                 __syncwarp();
             }
             if (!ok) { fail(); break; }
+            tile = a.sched ? __shfl_sync(0xffffffffu, nxt, 0) : tile + int(gridDim.x);
+        }
+        // the scheduler's counters: every CTA asks once past the end; the last one to do so
+        // leaves both at zero for the next launch
+        if (a.sched && lane == 0 && tile >= ntiles && atomicAdd(a.sched + 1, 1) == int(gridDim.x) - 1) {
+            a.sched[0] = 0;
+            a.sched[1] = 0;
         }
         // drain: every copy issued has landed before the CTA exits
         if (lane == 0) {
@@ -525,7 +590,8 @@ __global__ void __launch_bounds__(G_THREADS, 1) tc_grouped_gemm(const __grid_con
     } else if (warp == 1) {
         // ---------------- activation producer (whole warp, one lane issues) ----------------
         uint32_t bc = 0;
-        for (int tile = blockIdx.x; tile < ntiles && !g_aborted(&s_ab); tile += gridDim.x) {
+        uint32_t qi = 0;
+        for (int tile = q_take(qi); tile < ntiles && !g_aborted(&s_ab); tile = q_take(qi)) {
             const GTile T = tile_of(tile);
             const int row0 = (C::kI8 ? 3 : 1) * (T.ebase + T.n0);      // i8: three digit rows per token
             const CUtensorMap* map = &a.tm_b[C::kI8 ? 0 : T.bn / 16 - 1];
@@ -579,7 +645,8 @@ __global__ void __launch_bounds__(G_THREADS, 1) tc_grouped_gemm(const __grid_con
         if (s_hold && !g_wait_w(g_smem(&hold_bar), 0, &s_ab)) fail();
         uint32_t bc = 0, ac = 0, pc = 0;
         int t = 0;
-        for (int tile = blockIdx.x; tile < ntiles && !g_aborted(&s_ab); tile += gridDim.x, t++) {
+        uint32_t qi = 0;
+        for (int tile = q_take(qi); tile < ntiles && !g_aborted(&s_ab); tile = q_take(qi), t++) {
             const GTile T = tile_of(tile);
             const uint32_t idesc = C::kI8 ? g_idesc_i8(T.bn) : g_idesc(T.bn, C::kMmaF16);
             const int buf = C::kI8 ? 0 : t % C::kAccBufs;
@@ -691,7 +758,8 @@ __global__ void __launch_bounds__(G_THREADS, 1) tc_grouped_gemm(const __grid_con
         uint32_t ac = 0;
         int t = 0;
         bool ok = true;
-        for (int tile = blockIdx.x; tile < ntiles && ok && !g_aborted(&s_ab); tile += gridDim.x, t++) {
+        uint32_t qi = 0;
+        for (int tile = q_take(qi); tile < ntiles && ok && !g_aborted(&s_ab); tile = q_take(qi), t++) {
             const GTile T = tile_of(tile);
             const int f = T.m0 + r;
             const int rbase = T.ebase + T.n0;
@@ -774,7 +842,8 @@ __global__ void __launch_bounds__(G_THREADS, 1) tc_grouped_gemm(const __grid_con
         const int q = warp & 3;
         const uint32_t lane_addr = uint32_t(q * 32) << 16;
         int t = 0;
-        for (int tile = blockIdx.x; tile < ntiles && !g_aborted(&s_ab); tile += gridDim.x, t++) {
+        uint32_t qi = 0;
+        for (int tile = q_take(qi); tile < ntiles && !g_aborted(&s_ab); tile = q_take(qi), t++) {
             const GTile T = tile_of(tile);
             const int buf = t % C::kAccBufs;
             const int rbase = T.ebase + T.n0;
@@ -906,7 +975,8 @@ __global__ void __launch_bounds__(G_THREADS, 1) tc_grouped_gemm(const __grid_con
         const uint32_t at = 16u * uint32_t(r & 31) + 4u * uint32_t(r >> 5);
         uint32_t bc = 0;
         bool ok = true;
-        for (int tile = blockIdx.x; tile < ntiles && ok && !g_aborted(&s_ab); tile += gridDim.x) {
+        uint32_t qi = 0;
+        for (int tile = q_take(qi); tile < ntiles && ok && !g_aborted(&s_ab); tile = q_take(qi)) {
             const GTile T = tile_of(tile);
             for (int ks = 0; ks < KS; ks++, bc++) {
                 if (!g_wait_w(g_smem(&pk_full[bc % NPK]), (bc / NPK) & 1, &s_ab) ||
@@ -953,7 +1023,8 @@ __global__ void __launch_bounds__(G_THREADS, 1) tc_grouped_gemm(const __grid_con
         const uint32_t lane_addr = uint32_t(q * 32) << 16;
         uint32_t pc = 0;
         bool ok = true;
-        for (int tile = blockIdx.x; tile < ntiles && ok && !g_aborted(&s_ab); tile += gridDim.x) {
+        uint32_t qi = 0;
+        for (int tile = q_take(qi); tile < ntiles && ok && !g_aborted(&s_ab); tile = q_take(qi)) {
             for (int ps = 0; ps < NPS; ps++, pc++) {
                 if (int(pc & 1) != grp) continue;
                 const int s = pc % NPK;
@@ -1028,7 +1099,8 @@ __global__ void __launch_bounds__(G_THREADS, 1) tc_grouped_gemm(const __grid_con
         uint32_t pc = 0;
         int t = 0;
         bool ok = true;
-        for (int tile = blockIdx.x; tile < ntiles && ok && !g_aborted(&s_ab); tile += gridDim.x, t++) {
+        uint32_t qi = 0;
+        for (int tile = q_take(qi); tile < ntiles && ok && !g_aborted(&s_ab); tile = q_take(qi), t++) {
             const uint8_t* scrow = nullptr;
             float fk = 1.f;                             // int4: 2^k of this weight row (the epilogue undoes it)
             if (FMT == MOE_FMT_INT4_G128) {
@@ -1333,44 +1405,72 @@ __global__ void __launch_bounds__(256) g_splitk_finish(const float* __restrict__
 // ---------------------------------------------------------------------------
 // Host side
 // ---------------------------------------------------------------------------
-template <int FMT, bool GU, bool W>
+template <int FMT, bool GU, int NW>
 static size_t g_smem_bytes(int in_dim, int npk, int nsc, int E) {
-    using C = GCfg<FMT, GU, W>;
+    using C = GCfg<FMT, GU, NW>;
     size_t b = g_tbl_bytes(E) + size_t(npk) * C::kPkStageBytes + size_t(C::kBStages) * C::kBStageBytes + 1024;
     if (C::kInt4) b += size_t(nsc) * (C::kNMat * G_BM * (in_dim / 128) * 2 + (C::kI8 ? C::kNMax * (((in_dim / 128) + 3) & ~3) * 4 : 0));
     if (C::kA4) b += size_t(G_SF_RING) * C::kSfSlotBytes;
     return b;
 }
 
-template <int FMT, bool GU, bool W = false>
-static int g_launch(const GArgs& a, cudaStream_t s) {
-    using C = GCfg<FMT, GU, W>;
-    auto k = tc_grouped_gemm<FMT, GU, W>;
-    int dev = 0, sms = 0, optin = 0;
-    if (cudaGetDevice(&dev) != cudaSuccess) return MOE_ERR_CUDA;
-    if (cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) return MOE_ERR_CUDA;
-    if (cudaDeviceGetAttribute(&optin, cudaDevAttrMaxSharedMemoryPerBlockOptin, dev) != cudaSuccess) return MOE_ERR_CUDA;
-    cudaFuncAttributes fa{};
-    if (cudaFuncGetAttributes(&fa, k) != cudaSuccess) return MOE_ERR_CUDA;
+template <int FMT, bool GU, int NW = 0>
+static int g_launch(const GArgs& a, cudaStream_t s, int max_ctas, bool pdl) {
+    using C = GCfg<FMT, GU, NW>;
+    auto k = tc_grouped_gemm<FMT, GU, NW>;
+    // per device: SM count, the opt-in shared memory left beside the kernel's static shared memory,
+    // and the dynamic shared memory size granted so far (read once; raised only when a call needs more)
+    struct DevInfo {
+        std::once_flag once;
+        int sms = 0;
+        size_t room = 0;
+        std::atomic<size_t> granted{0};
+        int rc = MOE_ERR_CUDA;
+    };
+    static DevInfo info[64];
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return MOE_ERR_CUDA;
+    DevInfo& di = info[dev];
+    std::call_once(di.once, [&] {
+        int optin = 0;
+        cudaFuncAttributes fa{};
+        if (cudaDeviceGetAttribute(&di.sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess ||
+            cudaDeviceGetAttribute(&optin, cudaDevAttrMaxSharedMemoryPerBlockOptin, dev) != cudaSuccess ||
+            cudaFuncGetAttributes(&fa, k) != cudaSuccess)
+            return;
+        di.room = size_t(optin) - std::min(size_t(optin), fa.sharedSizeBytes);
+        di.rc = MOE_OK;
+    });
+    if (di.rc != MOE_OK) return di.rc;
+    const int sms = di.sms;
     // The weight stream wants as many bytes in flight as shared memory holds.
     // The producer runs ahead by whole tiles only as far as free int4 scale
     // buffers allow, so those cover the ring's reach: one per tile it spans,
     // plus the tile being consumed.
-    const size_t room = size_t(optin) - std::min(size_t(optin), fa.sharedSizeBytes);
+    const size_t room = di.room;
     const int nps = std::max(1, (a.in_dim / a.ksplit) / C::kPkK);            // weight stages per tile
     int npk = C::kPkMax, nsc = 2;
     for (; npk >= 2; npk--) {
         nsc = C::kInt4 ? std::min(G_SC_MAX, std::max(2, (npk + nps - 1) / nps + 1)) : 2;
-        if (g_smem_bytes<FMT, GU, W>(a.in_dim, npk, nsc, a.E) <= room) break;
+        if (g_smem_bytes<FMT, GU, NW>(a.in_dim, npk, nsc, a.E) <= room) break;
     }
     if (npk < 2) return MOE_ERR_UNSUPPORTED;
     GArgs args = a;
     args.npk = npk;
     args.nsc = nsc;
-    const size_t smem = g_smem_bytes<FMT, GU, W>(a.in_dim, npk, nsc, a.E);
-    if (cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem)) != cudaSuccess)
-        return MOE_ERR_CUDA;
-    return launch_pdl(k, dim3(sms), dim3(G_THREADS), smem, s, args) == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
+    const size_t smem = g_smem_bytes<FMT, GU, NW>(a.in_dim, npk, nsc, a.E);
+    if (smem > di.granted.load(std::memory_order_acquire)) {
+        if (cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem)) != cudaSuccess)
+            return MOE_ERR_CUDA;
+        size_t cur = di.granted.load(std::memory_order_acquire);
+        while (cur < smem && !di.granted.compare_exchange_weak(cur, smem, std::memory_order_acq_rel)) {
+        }
+    }
+    const int grid = max_ctas > 0 ? std::min(sms, max_ctas) : sms;
+    if (pdl) return launch_pdl(k, dim3(grid), dim3(G_THREADS), smem, s, args) == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
+    k<<<grid, G_THREADS, smem, s>>>(args);
+    count_launch();
+    return cudaGetLastError() == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
 }
 
 #define G_TRY(x)                       \
@@ -1441,19 +1541,21 @@ int launch_grouped_gemm(const GemvProblem& p, bool gateup, int rows, const GemmB
         G_TRY(g_map(&a.tm_s0, false, p.s0, in / 16, wrows, uint64_t(in) / 16, 16, 128, false));
         if (gateup) G_TRY(g_map(&a.tm_s1, false, p.s1, in / 16, wrows, uint64_t(in) / 16, 16, 128, false));
     }
+    // a tile holds at most min(rows, 128) token rows: only the box heights up to that are encoded
+    const int nb_maps = std::min(G_NB_MAPS, (std::min(rows, 128) + 15) / 16);
     if (i8) {
         // three digit rows per activation row, 16 rows and 128 bytes of K per box
         G_TRY(g_map(&a.tm_b[0], false, bsrc, in, uint64_t(rows) * 3, uint64_t(in), 128, 16, true));
     } else if (a4) {
         const uint8_t* codes = static_cast<const uint8_t*>(bsrc);
-        for (int i = 0; i < G_NB_MAPS; i++) {
+        for (int i = 0; i < nb_maps; i++) {
             G_TRY(g_map(&a.tm_b[i], false, codes, in / 2, uint64_t(rows), uint64_t(in) / 2, 128, uint32_t(16 * (i + 1)),
                         true));
             G_TRY(g_map(&a.tm_bs[i], false, codes + a4_sc_off, in / 16, uint64_t(rows), uint64_t(in) / 16, 16,
                         uint32_t(16 * (i + 1)), false));
         }
     } else {
-        for (int i = 0; i < G_NB_MAPS; i++)
+        for (int i = 0; i < nb_maps; i++)
             G_TRY(g_map(&a.tm_b[i], true, bsrc, in, uint64_t(rows), uint64_t(in) * 2, 64, uint32_t(16 * (i + 1)), true));
     }
     a.sc0 = reinterpret_cast<const uint8_t*>(p.s0);
@@ -1473,22 +1575,32 @@ int launch_grouped_gemm(const GemvProblem& p, bool gateup, int rows, const GemmB
     a.partial = buf.partial;
     a.rows = rows;
     a.zsum = buf.zbuf;
+    a.sched = buf.sched;
+    // wide gate/up tiles (128 token rows) once the experts average more than 64 rows; narrow ones
+    // (16) when no expert can hold more than 16 rows (BF16 and the NVFP4 16-bit path)
+    const bool wide = gateup && ksplit == 1 && rows > 64 * E;
+    const bool narrow = !wide && (p.fmt == MOE_FMT_BF16 || (nv && !a4)) && buf.max_expert_rows > 0 &&
+                        buf.max_expert_rows <= 16;
+    const int mc = buf.max_ctas;
+    const bool pdl = !buf.no_pdl;
     // split-K tiles finish in the GEMM when their counters fit the workspace's control block
-    const int ntile_max = (rows + (gateup ? 63 : 127)) / (gateup ? 64 : 128);
+    const int nmax = narrow ? 16 : (gateup ? 64 : 128);
+    const int ntile_max = (rows + nmax - 1) / nmax;
     if (ksplit > 1 && ksplit <= G_KSPLIT_MAX && buf.tile_cnt && 4 * (out / G_BM) * ntile_max <= kTileCounters)
         a.tile_cnt = buf.tile_cnt;
-
-    // wide gate/up tiles (128 token rows) once the experts average more than 64 rows
-    const bool wide = gateup && ksplit == 1 && rows > 64 * E;
-    if (i8) return gateup ? g_launch<FMT_INT4_I8, true>(a, s) : g_launch<FMT_INT4_I8, false>(a, s);
-    if (i4) return gateup ? (wide ? g_launch<MOE_FMT_INT4_G128, true, true>(a, s) : g_launch<MOE_FMT_INT4_G128, true>(a, s))
-                          : g_launch<MOE_FMT_INT4_G128, false>(a, s);
-    if (a4) return gateup ? (wide ? g_launch<FMT_NVFP4_A4, true, true>(a, s) : g_launch<FMT_NVFP4_A4, true>(a, s))
-                          : g_launch<FMT_NVFP4_A4, false>(a, s);
-    if (nv) return gateup ? (wide ? g_launch<MOE_FMT_NVFP4, true, true>(a, s) : g_launch<MOE_FMT_NVFP4, true>(a, s))
-                          : g_launch<MOE_FMT_NVFP4, false>(a, s);
-    const int rc = gateup ? (wide ? g_launch<MOE_FMT_BF16, true, true>(a, s) : g_launch<MOE_FMT_BF16, true>(a, s))
-                          : g_launch<MOE_FMT_BF16, false>(a, s);
+    if (i8) return gateup ? g_launch<FMT_INT4_I8, true>(a, s, mc, pdl) : g_launch<FMT_INT4_I8, false>(a, s, mc, pdl);
+    if (i4) return gateup ? (wide ? g_launch<MOE_FMT_INT4_G128, true, 1>(a, s, mc, pdl) : g_launch<MOE_FMT_INT4_G128, true>(a, s, mc, pdl))
+                          : g_launch<MOE_FMT_INT4_G128, false>(a, s, mc, pdl);
+    if (a4) return gateup ? (wide ? g_launch<FMT_NVFP4_A4, true, 1>(a, s, mc, pdl) : g_launch<FMT_NVFP4_A4, true>(a, s, mc, pdl))
+                          : g_launch<FMT_NVFP4_A4, false>(a, s, mc, pdl);
+    if (nv) {
+        if (narrow) return gateup ? g_launch<MOE_FMT_NVFP4, true, 2>(a, s, mc, pdl) : g_launch<MOE_FMT_NVFP4, false, 2>(a, s, mc, pdl);
+        return gateup ? (wide ? g_launch<MOE_FMT_NVFP4, true, 1>(a, s, mc, pdl) : g_launch<MOE_FMT_NVFP4, true>(a, s, mc, pdl))
+                      : g_launch<MOE_FMT_NVFP4, false>(a, s, mc, pdl);
+    }
+    const int rc = narrow ? (gateup ? g_launch<MOE_FMT_BF16, true, 2>(a, s, mc, pdl) : g_launch<MOE_FMT_BF16, false, 2>(a, s, mc, pdl))
+                          : gateup ? (wide ? g_launch<MOE_FMT_BF16, true, 1>(a, s, mc, pdl) : g_launch<MOE_FMT_BF16, true>(a, s, mc, pdl))
+                                   : g_launch<MOE_FMT_BF16, false>(a, s, mc, pdl);
     if (rc != MOE_OK) return rc;
     if (ksplit > 1 && !a.tile_cnt) {
         const size_t n4 = size_t(rows) * out / 4;

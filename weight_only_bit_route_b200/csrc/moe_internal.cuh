@@ -23,9 +23,11 @@ constexpr int kMaxDecodeT = 64;
 //              amax (float bits), [3] reserved, [4..5] bound on every
 //              device wait in ns (uint64, 0 = the default of about 2 s),
 //              [6] failure-testing hold (non-zero: each tensor-core GEMM
-//              first waits on a barrier nothing completes), [7..15]
-//              reserved, [16..255] split-K tile arrival counters (left at
-//              zero by every call that completes).
+//              first waits on a barrier nothing completes), [7] reserved,
+//              [8..9] the routed GEMMs' tile scheduler (next tile, CTAs
+//              done), [10..15] reserved, [16..255] split-K tile arrival
+//              counters (counters are left at zero by every call that
+//              completes).
 // ---------------------------------------------------------------------------
 struct WsLayout {
     size_t ctrl, logits, wsplit, hist, offsets, row_slot, slot_row, ids, tw;
@@ -264,6 +266,11 @@ struct GemmBuffers {
     int i8;              // int4 on the 8-bit MMA with per-group accumulation (small batches)
     float* zbuf;         // i8: 8 * group sums of the fixed-point rows [rows][zsum_stride(in)]
     int* tile_cnt;       // split-K: kTileCounters zeroed ints (the control block's [16..255])
+    int max_ctas;        // > 0: at most this many CTAs (a side-stream problem leaves the other SMs free)
+    int no_pdl;          // launch without programmatic dependent launch (its CTAs hold no SM while waiting)
+    int* sched;          // tensor-core GEMM: {next, done} tile counters (zero), or null for a static tile order;
+                         // problems that may run at the same time need their own
+    int max_expert_rows; // > 0: no expert holds more rows than this (the batch's token count); 0: unknown
 };
 constexpr int kTileCounters = 240;
 
