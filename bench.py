@@ -373,7 +373,17 @@ def measure(moe, wl, x, layer, args, flush, stream, clk, pk, pk_kind, per_step=T
     touched = int(torch.unique(ids).numel())
     torch.cuda.synchronize()
     launches0 = moe.launch_count()
-    ms_list = time_calls(step, args.steps, flush, stream, clk, warmup=0)
+    eager_list = time_calls(step, args.steps, flush, stream, clk, warmup=0)
+    eager_launches = moe.launch_count() - launches0
+    # the same call recorded once as a CUDA graph (moe_layer_graph_*) and replayed: the layer's
+    # kernels without the host's per-call launch work
+    graph = moe.LayerGraph(x, layer, ws, out=y)
+    for _ in range(3):
+        flush.zero_()
+        graph.launch()
+    torch.cuda.synchronize()
+    launches0 = moe.launch_count()
+    ms_list = time_calls(graph.launch, args.steps, flush, stream, clk, warmup=0)
     launches = moe.launch_count() - launches0
     # dominant kernel: grouped gate/up (+ SwiGLU) through its own C-ABI call
     off, rs, sr = moe.permute(ids, wl.E, ws)
@@ -413,12 +423,15 @@ def measure(moe, wl, x, layer, args, flush, stream, clk, pk, pk_kind, per_step=T
                       "frac_sustained": round(tf / pk.get("bf16_tflops_sustained", pk["bf16_tflops"]), 4),
                       "algorithmic_bytes": lbytes,
                       "hbm_frac": round(lbytes / (ms * 1e-3) / 1e9 / pk["hbm_gbs"], 4)}
+    e_ms = float(np.mean(eager_list))
     res = {"workload": describe(wl), "T": T, "format": wl.fmt, "touched_experts": touched,
            "tokens_per_s": round(T / (ms * 1e-3), 1), "layer_ms": _pcts(ms_list),
-           "roofline": roof, "layer_roofline": layer_roof, "gpu_launches_per_step": launches / args.steps}
+           "roofline": roof, "layer_roofline": layer_roof, "gpu_launches_per_step": launches / args.steps,
+           "eager": {"tokens_per_s": round(T / (e_ms * 1e-3), 1), "layer_ms": _pcts(eager_list),
+                     "gpu_launches_per_step": eager_launches / args.steps}}
     if per_step:
         res["steps_ms"] = step_times(moe, wl, x, layer, ws, args.steps, flush, stream, clk)
-    return res, ms, ms_list, touched, launches, ws, entry
+    return res, ms, ms_list, touched, launches, ws, graph
 
 
 def main():
@@ -478,7 +491,7 @@ def main():
         dist.barrier()
     torch.cuda.synchronize()
     with ClockSampler(local_rank) as clk:
-        head, ms, ms_list, touched, launches, ws, entry = measure(moe, wl, x, layer, args, flush, stream, clk,
+        head, ms, ms_list, touched, launches, ws, graph = measure(moe, wl, x, layer, args, flush, stream, clk,
                                                                   pk, pk_kind)
         if dist:
             t = torch.tensor([ms], device="cuda")
@@ -486,16 +499,15 @@ def main():
             ms = float(t.item())
         value = world * T / (ms * 1e-3)
 
-        # end to end through the public API with host buffers
-        y = torch.empty_like(x)
+        # end to end through the public API with host buffers: each step copies its tokens into the
+        # recorded layer's input, replays the layer and copies the output back
         xh = x.cpu().pin_memory()
         yh = torch.empty_like(xh).pin_memory()
-        xd = torch.empty_like(x)
 
         def e2e_step():
-            xd.copy_(xh, non_blocking=True)
-            entry(xd, layer, ws, out=y)
-            yh.copy_(y, non_blocking=True)
+            graph.x.copy_(xh, non_blocking=True)
+            graph.launch()
+            yh.copy_(graph.y, non_blocking=True)
         e_ms = float(np.mean(time_calls(e2e_step, args.steps, flush, stream, clk)))
         if dist:
             t = torch.tensor([e_ms], device="cuda")
@@ -543,6 +555,7 @@ def main():
                    "algorithmic_bytes_per_step": layer_bytes(wl, touched),
                    "algorithmic_flops_per_step": layer_flops(wl)},
         "layer_ms": head["layer_ms"],
+        "eager": head["eager"],
         "roofline": head["roofline"],
         "layer_roofline": head["layer_roofline"],
         "steps_ms": head.get("steps_ms"),

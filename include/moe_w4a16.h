@@ -308,6 +308,24 @@ int moe_layer_decode(const void* x, int T, const moe_layer* L, void* y,
 int moe_layer_forward(const void* x, int T, const moe_layer* L, void* y,
                       void* ws, size_t ws_bytes, moe_stream_t stream);
 
+/* A layer call recorded once as a CUDA graph and replayed: the same kernels
+ * as moe_layer_forward(x, T, L, y, ws, ws_bytes, .) with these exact
+ * pointers, without the host's per-call launch work (argument checks, tensor
+ * map encoding, about ten kernel launches).  The graph reads x and the banks
+ * and writes y and ws at every launch, so the caller refills x in place
+ * between launches and keeps every buffer (and the banks' contents, which may
+ * change) alive until moe_layer_graph_destroy.  One launch at a time per
+ * workspace.  create: checks as moe_layer_forward, records on a private
+ * stream (the caller's stream is not touched), returns the handle in *out
+ * (NULL on error).  launch: enqueues one layer on `stream`.  The recording
+ * uses the per-device side stream of the shared expert, so create must not
+ * overlap a layer call of another host thread on the same device. */
+typedef struct moe_layer_graph_s* moe_layer_graph_t;
+int moe_layer_graph_create(const void* x, int T, const moe_layer* L, void* y,
+                           void* ws, size_t ws_bytes, moe_layer_graph_t* out);
+int moe_layer_graph_launch(moe_layer_graph_t graph, moe_stream_t stream);
+int moe_layer_graph_destroy(moe_layer_graph_t graph);
+
 /* ---------------------------------------------------------------------- */
 /* Weight conversion (offline step, not on the hot path)                   */
 /* ---------------------------------------------------------------------- */

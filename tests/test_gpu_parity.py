@@ -453,6 +453,32 @@ def test_layer_decode_repeated_calls(cfg):
     assert not differ, f"calls (index, tokens) that differ from the first: {differ[:8]}"
 
 
+@pytest.mark.parametrize("cfg", [0, 1, 2])
+def test_layer_graph_matches_eager(cfg):
+    """The recorded layer (moe_layer_graph_*) replays the eager call bit for bit: three launches
+    with x refilled in place between them, each against moe_layer_decode on the same input; each
+    replay adds the recorded kernels to the launch count."""
+    P = build(cfg, "random" if cfg else "quantised")
+    L = device_layer(moe, P)
+    ws_g, ws_e = _ws(P.T, P.wl), _ws(P.T, P.wl)
+    x = dev_bf16(P.x)
+    g = moe.LayerGraph(x, L, ws_g)
+    n0 = moe.launch_count()
+    g.launch()
+    torch.cuda.synchronize()
+    per_launch = moe.launch_count() - n0
+    assert per_launch >= 5
+    for seed in (None, 11, 12):
+        if seed is not None:
+            x.copy_(dev_bf16(syn.gen_x(P.wl, seed=seed, T=P.T)))
+            g.launch()
+        ref = moe.layer_decode(x.clone(), L, ws_e)
+        torch.cuda.synchronize()
+        assert torch.equal(g.y, ref)
+    assert moe.read_status(ws_g) == 0 and moe.read_status(ws_e) == 0
+    g.close()
+
+
 def test_layer_T0_is_noop():
     P = build(0, "quantised")
     L = device_layer(moe, P)

@@ -4,6 +4,7 @@
 #include <algorithm>
 #include <atomic>
 #include <mutex>
+#include <vector>
 
 #include "moe_internal.cuh"
 
@@ -179,11 +180,13 @@ int layer_run(const void* x, int T, const moe_layer* L, void* y, void* ws, cudaS
 
     // The shared expert needs x only: it runs on a side stream while the
     // router, the bucketing and the routed experts run on `s`, and `s` waits
-    // for it before the combine.  The router is launched first (it starts the
-    // critical path); the shared expert's own routing (offsets {0, T}, row i at
-    // slot i * top_k) comes first on its stream.  At decode sizes its GEMMs take
-    // at most kSharedDecodeCtas SMs and no early launch, so the router's CTAs
-    // find SMs free beside them and no waiting CTA holds an SM.
+    // for it before the combine.  The routed chain is launched first (it is
+    // the critical path, and the host's launch work for the shared expert would
+    // otherwise delay it); the shared expert's own routing (offsets {0, T}, row
+    // i at slot i * top_k) comes first on its stream.  At decode sizes its GEMMs
+    // take at most kSharedDecodeCtas SMs and no early launch, so that no waiting
+    // CTA holds an SM; the routed GEMMs hand out their tiles dynamically around
+    // them.
     SideStream* side = nullptr;
     std::unique_lock<std::mutex> side_lock;
     if (has_sh) {
@@ -207,36 +210,6 @@ int layer_run(const void* x, int T, const moe_layer* L, void* y, void* ws, cudaS
         MOE_TRY(launch_permute(ids, T, k, E, offsets, row_slot, slot_row, at<int32_t>(ws, W.hist), status, s));
     }
 
-    if (has_sh) {
-        // fp16 mode: the BF16 shared expert reads x rounded to bf16, staged in its output region (the
-        // down projection overwrites it only after the gate/up projection has read it)
-        const __nv_bfloat16* xs = xb;
-        if (x_f16) {
-            MOE_TRY(launch_f16_to_bf16(reinterpret_cast<const __half*>(x), ys, size_t(T) * H, side->s));
-            xs = ys;
-        }
-        GemvProblem sg{};
-        sg.act = xs; sg.act_by_token = 1; sg.top_k = k; sg.offsets = sh_off; sg.row_slot = sh_rs;
-        sg.E = 1; sg.fmt = MOE_FMT_BF16; sg.out_dim = F; sg.in_dim = H;
-        sg.p0 = L->sh_gate.packed; sg.p1 = L->sh_up.packed; sg.out = h_sh; sg.status = status;
-        GemvProblem sd{};
-        sd.act = h_sh; sd.act_by_token = 0; sd.top_k = k; sd.offsets = sh_off; sd.row_slot = sh_rs;
-        sd.E = 1; sd.fmt = MOE_FMT_BF16; sd.out_dim = H; sd.in_dim = F;
-        sd.p0 = L->sh_down.packed; sd.out = ys; sd.status = status;
-        // the shared expert reads x and its own h directly (identity routing, natural order)
-        GemmBuffers direct{};
-        direct.act_ready = 1;
-        direct.max_expert_rows = T;
-        if (T <= kRouterDecodeMaxT) {
-            direct.max_ctas = kSharedDecodeCtas;
-            direct.no_pdl = 1;
-        }
-        float* shpart = at<float>(ws, W.shpart);
-        MOE_TRY(launch_shared_routing(T, k, sh_off, sh_rs, side->s));
-        MOE_TRY(run_problem(sg, true, T, T, nullptr, direct, shpart, side->s));
-        MOE_TRY(run_problem(sd, false, T, T, nullptr, direct, shpart, side->s));
-        if (cudaEventRecord(side->join, side->s) != cudaSuccess) return MOE_ERR_CUDA;
-    }
     const bool routed_gemm = gemm_shape_ok(H, F) && gemm_shape_ok(F, H);
 
     GemvProblem gu{};
@@ -270,6 +243,36 @@ int layer_run(const void* x, int T, const moe_layer* L, void* y, void* ws, cudaS
         MOE_TRY(launch_grouped_gemm(dn, false, R, db, s));
     } else {
         MOE_TRY(launch_stream_gemv(dn, nullptr, false, R, prep, s, true));
+    }
+    if (has_sh) {
+        // fp16 mode: the BF16 shared expert reads x rounded to bf16, staged in its output region (the
+        // down projection overwrites it only after the gate/up projection has read it)
+        const __nv_bfloat16* xs = xb;
+        if (x_f16) {
+            MOE_TRY(launch_f16_to_bf16(reinterpret_cast<const __half*>(x), ys, size_t(T) * H, side->s));
+            xs = ys;
+        }
+        GemvProblem sg{};
+        sg.act = xs; sg.act_by_token = 1; sg.top_k = k; sg.offsets = sh_off; sg.row_slot = sh_rs;
+        sg.E = 1; sg.fmt = MOE_FMT_BF16; sg.out_dim = F; sg.in_dim = H;
+        sg.p0 = L->sh_gate.packed; sg.p1 = L->sh_up.packed; sg.out = h_sh; sg.status = status;
+        GemvProblem sd{};
+        sd.act = h_sh; sd.act_by_token = 0; sd.top_k = k; sd.offsets = sh_off; sd.row_slot = sh_rs;
+        sd.E = 1; sd.fmt = MOE_FMT_BF16; sd.out_dim = H; sd.in_dim = F;
+        sd.p0 = L->sh_down.packed; sd.out = ys; sd.status = status;
+        // the shared expert reads x and its own h directly (identity routing, natural order)
+        GemmBuffers direct{};
+        direct.act_ready = 1;
+        direct.max_expert_rows = T;
+        if (T <= kRouterDecodeMaxT) {
+            direct.max_ctas = kSharedDecodeCtas;
+            direct.no_pdl = 1;
+        }
+        float* shpart = at<float>(ws, W.shpart);
+        MOE_TRY(launch_shared_routing(T, k, sh_off, sh_rs, side->s));
+        MOE_TRY(run_problem(sg, true, T, T, nullptr, direct, shpart, side->s));
+        MOE_TRY(run_problem(sd, false, T, T, nullptr, direct, shpart, side->s));
+        if (cudaEventRecord(side->join, side->s) != cudaSuccess) return MOE_ERR_CUDA;
     }
     if (has_sh && cudaStreamWaitEvent(s, side->join, 0) != cudaSuccess) return MOE_ERR_CUDA;
 
@@ -469,6 +472,77 @@ int moe_layer_forward(const void* x, int T, const moe_layer* L, void* y, void* w
     MOE_TRY(layer_checks(x, T, L, y, ws, ws_bytes));
     if (T == 0) return MOE_OK;
     return layer_run(x, T, L, y, ws, cs(stream));
+}
+
+}  // extern "C"
+
+struct moe_layer_graph_s {
+    cudaGraphExec_t exec = nullptr;
+    uint64_t kernels = 0;             // kernel nodes: added to the launch count at every replay
+};
+
+extern "C" {
+
+int moe_layer_graph_create(const void* x, int T, const moe_layer* L, void* y, void* ws, size_t ws_bytes,
+                           moe_layer_graph_t* out) {
+    if (!out) return MOE_ERR_INVALID_ARG;
+    *out = nullptr;
+    MOE_TRY(layer_checks(x, T, L, y, ws, ws_bytes));
+    if (T == 0) return MOE_ERR_INVALID_ARG;
+    if (L->sh_gate.packed) {                 // the side stream and its events exist before the recording
+        SideStream* side = nullptr;
+        MOE_TRY(side_stream(&side));
+    }
+    cudaStream_t cap = nullptr;
+    if (cudaStreamCreateWithFlags(&cap, cudaStreamNonBlocking) != cudaSuccess) return MOE_ERR_CUDA;
+    cudaGraph_t graph = nullptr;
+    int rc = MOE_OK;
+    if (cudaStreamBeginCapture(cap, cudaStreamCaptureModeRelaxed) != cudaSuccess) {
+        rc = MOE_ERR_CUDA;
+    } else {
+        rc = layer_run(x, T, L, y, ws, cap);
+        // the capture is ended whatever happened inside it
+        if (cudaStreamEndCapture(cap, &graph) != cudaSuccess && rc == MOE_OK) rc = MOE_ERR_CUDA;
+    }
+    moe_layer_graph_s* g = nullptr;
+    if (rc == MOE_OK) {
+        g = new moe_layer_graph_s();
+        size_t n = 0;
+        if (cudaGraphGetNodes(graph, nullptr, &n) != cudaSuccess) rc = MOE_ERR_CUDA;
+        std::vector<cudaGraphNode_t> nodes(n);
+        if (rc == MOE_OK && n && cudaGraphGetNodes(graph, nodes.data(), &n) != cudaSuccess) rc = MOE_ERR_CUDA;
+        for (size_t i = 0; rc == MOE_OK && i < n; i++) {
+            cudaGraphNodeType t;
+            if (cudaGraphNodeGetType(nodes[i], &t) != cudaSuccess) rc = MOE_ERR_CUDA;
+            else if (t == cudaGraphNodeTypeKernel) g->kernels++;
+        }
+        if (rc == MOE_OK && cudaGraphInstantiate(&g->exec, graph, 0) != cudaSuccess) rc = MOE_ERR_CUDA;
+    }
+    if (graph) cudaGraphDestroy(graph);
+    cudaStreamDestroy(cap);
+    // the launches recorded above ran nothing: they are counted when the graph is launched
+    if (rc != MOE_OK) {
+        cudaGetLastError();
+        delete g;
+        return rc;
+    }
+    moe::g_launches.fetch_sub(g->kernels, std::memory_order_relaxed);
+    *out = g;
+    return MOE_OK;
+}
+
+int moe_layer_graph_launch(moe_layer_graph_t graph, moe_stream_t stream) {
+    if (!graph || !graph->exec) return MOE_ERR_INVALID_ARG;
+    if (cudaGraphLaunch(graph->exec, cs(stream)) != cudaSuccess) return MOE_ERR_CUDA;
+    moe::g_launches.fetch_add(graph->kernels, std::memory_order_relaxed);
+    return MOE_OK;
+}
+
+int moe_layer_graph_destroy(moe_layer_graph_t graph) {
+    if (!graph) return MOE_OK;
+    const int rc = (graph->exec && cudaGraphExecDestroy(graph->exec) != cudaSuccess) ? MOE_ERR_CUDA : MOE_OK;
+    delete graph;
+    return rc;
 }
 
 int moe_csf_decode(const uint8_t* fixed, const uint32_t* exceptions, const int64_t* starts, int E, int R, int C,

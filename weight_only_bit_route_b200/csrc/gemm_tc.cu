@@ -1303,16 +1303,32 @@ __global__ void __launch_bounds__(G_PREP_I8_THREADS) g_prep_i8(const __nv_bfloat
                                                                float* __restrict__ zsum, int32_t* status) {
     __shared__ float s_max[G_PREP_I8_THREADS / 32];
     asm volatile("griddepcontrol.wait;" ::: "memory");
+    // the GEMM that reads these rows may be placed on free SMs now; it waits for this grid
+    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
     const int row = blockIdx.x, tid = threadIdx.x, lane = tid & 31;
-    const int srow = by_token ? row_slot[row] / top_k : row;
+    const int slot = (by_token || row_w) ? row_slot[row] : 0;
+    // the row's routing weight (down): its load goes out with the row's, it is used last
+    const float rw = (tid == 0 && row_w) ? row_w[slot] : 1.f;
+    const int srow = by_token ? slot / top_k : row;
     const uint4* s = reinterpret_cast<const uint4*>(src + size_t(srow) * in_dim);
     const int n16 = in_dim / 8, zst = ((in_dim / 128) + 3) & ~3;
-    float amax = 0.f;
-    for (int i = tid; i < n16; i += G_PREP_I8_THREADS) {
-        const uint4 v = s[i];
-        amax = fmaxf(amax, fmaxf(fmaxf(fabsf(act_lo<F16>(v.x)), fabsf(act_hi<F16>(v.x))), fmaxf(fabsf(act_lo<F16>(v.y)), fabsf(act_hi<F16>(v.y)))));
-        amax = fmaxf(amax, fmaxf(fmaxf(fabsf(act_lo<F16>(v.z)), fabsf(act_hi<F16>(v.z))), fmaxf(fabsf(act_lo<F16>(v.w)), fabsf(act_hi<F16>(v.w)))));
+    // the row stays in registers between the two passes (up to kPrepRegs chunks per thread;
+    // wider rows read the rest again)
+    constexpr int kPrepRegs = 4;
+    uint4 v[kPrepRegs];
+#pragma unroll
+    for (int j = 0; j < kPrepRegs; j++) {
+        const int i = tid + j * G_PREP_I8_THREADS;
+        v[j] = i < n16 ? s[i] : make_uint4(0, 0, 0, 0);
     }
+    float amax = 0.f;
+    auto fold = [&](const uint4 w) {
+        amax = fmaxf(amax, fmaxf(fmaxf(fabsf(act_lo<F16>(w.x)), fabsf(act_hi<F16>(w.x))), fmaxf(fabsf(act_lo<F16>(w.y)), fabsf(act_hi<F16>(w.y)))));
+        amax = fmaxf(amax, fmaxf(fmaxf(fabsf(act_lo<F16>(w.z)), fabsf(act_hi<F16>(w.z))), fmaxf(fabsf(act_lo<F16>(w.w)), fabsf(act_hi<F16>(w.w)))));
+    };
+#pragma unroll
+    for (int j = 0; j < kPrepRegs; j++) fold(v[j]);
+    for (int i = tid + kPrepRegs * G_PREP_I8_THREADS; i < n16; i += G_PREP_I8_THREADS) fold(s[i]);
     for (int o = 16; o > 0; o >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, o));
     if (lane == 0) s_max[tid >> 5] = amax;
     __syncthreads();
@@ -1324,13 +1340,11 @@ __global__ void __launch_bounds__(G_PREP_I8_THREADS) g_prep_i8(const __nv_bfloat
     const float fc = ldexpf(1.f, c);                    // a power of two: x * fc is exact
     uint8_t* d8 = dst + size_t(row) * 3 * in_dim;
     // 16 pieces of 8 make a group of 128: lanes 0-15 and 16-31 hold one group each
-    for (int i0 = 0; i0 < n16; i0 += G_PREP_I8_THREADS) {
-        const int i = i0 + tid;
+    auto emit = [&](const int i, const uint4 w) {
         int zs = 0;
         if (i < n16) {
-            const uint4 v = s[i];
-            const float xs[8] = {act_lo<F16>(v.x), act_lo<F16>(v.y), act_lo<F16>(v.z), act_lo<F16>(v.w),
-                                 act_hi<F16>(v.x), act_hi<F16>(v.y), act_hi<F16>(v.z), act_hi<F16>(v.w)};
+            const float xs[8] = {act_lo<F16>(w.x), act_lo<F16>(w.y), act_lo<F16>(w.z), act_lo<F16>(w.w),
+                                 act_hi<F16>(w.x), act_hi<F16>(w.y), act_hi<F16>(w.z), act_hi<F16>(w.w)};
             uint32_t p2[2] = {0u, 0u}, p1[2] = {0u, 0u}, p0[2] = {0u, 0u};
 #pragma unroll
             for (int e = 0; e < 8; e++) {
@@ -1350,10 +1364,17 @@ __global__ void __launch_bounds__(G_PREP_I8_THREADS) g_prep_i8(const __nv_bfloat
         }
         for (int o = 8; o > 0; o >>= 1) zs += __shfl_xor_sync(0xffffffffu, zs, o);
         if ((lane & 15) == 0 && i < n16) zsum[size_t(row) * zst + i / 16] = 8.f * float(zs);
+    };
+#pragma unroll
+    for (int j = 0; j < kPrepRegs; j++)
+        if (j * G_PREP_I8_THREADS < n16) emit(tid + j * G_PREP_I8_THREADS, v[j]);     // uniform condition
+    for (int i0 = kPrepRegs * G_PREP_I8_THREADS; i0 < n16; i0 += G_PREP_I8_THREADS) {
+        const int i = i0 + tid;
+        emit(i, i < n16 ? s[i] : make_uint4(0, 0, 0, 0));
     }
     if (tid == 0) {
         if (finite) {
-            scale[row] = row_w ? (1.f / fc) * row_w[row_slot[row]] : 1.f / fc;
+            scale[row] = (1.f / fc) * rw;
         } else {
             scale[row] = __int_as_float(0x7fc00000);        // quiet NaN
             set_status(status, MOE_ERR_NONFINITE);

@@ -123,8 +123,9 @@ __global__ void __launch_bounds__(256) router_logits_tiled(
 // score) above the complement of its id (so equal scores prefer the lower id);
 // 0 marks an empty or taken slot.  A lane keeps the largest of its keys; a pick
 // is one warp-wide maximum, after which only the lane that owned the winner
-// rescans its keys.  STAGED: lrow and bias are in shared memory (bias not
-// null), and the ids also go to ids_s.
+// rescans its keys.  STAGED: lrow holds the scores s themselves (sigmoid of
+// the biased logits, computed where the logits were), in shared memory, and
+// the ids also go to ids_s.
 // ---------------------------------------------------------------------------
 template <int PER, bool STAGED = false>
 __device__ __forceinline__ void topk_warp(const float* __restrict__ lrow, const float* __restrict__ bias, int E,
@@ -136,14 +137,14 @@ __device__ __forceinline__ void topk_warp(const float* __restrict__ lrow, const 
         const int e = lane + 32 * i;
         key[i] = 0ull;
         if (e < E) {
-            float l;
+            float v;
             if constexpr (STAGED) {
-                l = lrow[e] + bias[e];
+                v = lrow[e];
             } else {
-                l = lrow[e];
+                float l = lrow[e];
                 if (bias) l = l + bias[e];
+                v = 1.0f / (1.0f + expf(-l));
             }
-            const float v = 1.0f / (1.0f + expf(-l));
             key[i] = (static_cast<unsigned long long>(__float_as_uint(v)) << 32) | static_cast<uint32_t>(~e);
         }
     }
@@ -190,13 +191,14 @@ __global__ void __launch_bounds__(256) router_topk(
 }
 
 // ---------------------------------------------------------------------------
-// Fused decode router (T <= 16): logits, then the last CTA to finish does the
-// top-k of every token, the stable bucketing of the T*k slots and the shared
-// expert's routing.  Each warp owns one router row (16 KB at H = 4096) and
-// multiplies it with every token's activations, staged once per CTA in shared
-// memory; the router weights are read once in total across ~90 CTAs.  The
-// last CTA is found with an arrival counter in the workspace (no waiting);
-// it leaves the counter at zero for the next call.
+// Fused decode router (T <= 16).  Each CTA takes two experts, a warp per
+// quarter of H of one of them, against every token's activations (staged once
+// per CTA in shared memory), and writes the two experts' scores
+// s = sigmoid(l + b); the router weights are read once in total.  The last CTA
+// to finish (an arrival counter in the workspace, no waiting; it leaves the
+// counter at zero for the next call) stages all scores in shared memory and
+// does the top-k of every token, the stable bucketing of the T*k slots and
+// the shared expert's routing.
 // ---------------------------------------------------------------------------
 constexpr unsigned long long kRouterWaitNs = 2000000000ull;   // default bound of a wait
 // Bound on the fused router's wait: words 4-5 of the workspace control block
@@ -308,50 +310,57 @@ __global__ void __launch_bounds__(RD_WARPS * 32) router_decode(RouterDecodeArgs 
         }
     }
     __syncthreads();
-    // quarters in a fixed order
+    // quarters in a fixed order; the CTA's experts' scores s = sigmoid(l + b) go out (into the
+    // logits region) for the last CTA's selection
     for (int i = threadIdx.x; i < RD_EPC * a.T; i += blockDim.x) {
         const int ee = i / a.T, t = i % a.T, eg = blockIdx.x * RD_EPC + ee;
-        if (eg < a.E)
-            a.logits[size_t(t) * a.E + eg] = ((s_part[ee][0][t] + s_part[ee][1][t]) + s_part[ee][2][t]) + s_part[ee][3][t];
+        if (eg < a.E) {
+            float l = ((s_part[ee][0][t] + s_part[ee][1][t]) + s_part[ee][2][t]) + s_part[ee][3][t];
+            if (a.bias) l = l + a.bias[eg];
+            a.logits[size_t(t) * a.E + eg] = 1.0f / (1.0f + expf(-l));
+        }
     }
-    // last CTA to arrive continues
-    __threadfence();
+    // last CTA to arrive continues: the CTA's stores are ordered before its arrival by the barrier
+    // and thread 0's release fence; the last CTA acquires everyone's before it reads them
     __syncthreads();
-    if (threadIdx.x == 0) s_last = (atomicAdd(a.counter, 1) == int(gridDim.x) - 1);
+    if (threadIdx.x == 0) {
+        asm volatile("fence.acq_rel.gpu;" ::: "memory");
+        const int last = atomicAdd(a.counter, 1) == int(gridDim.x) - 1;
+        if (last) asm volatile("fence.acq_rel.gpu;" ::: "memory");
+        s_last = last;
+    }
     __syncthreads();
     if (!s_last) return;
-    __threadfence();
-    // Every token's logits (written by the other CTAs: read at L2) and the bias into shared memory,
-    // each thread's loads all issued before its stores, so the tail waits for one round of loads
+    // Every token's scores (written by the other CTAs: read at L2) into shared memory, each
+    // thread's loads all issued before its stores, so the tail waits for one round of loads
     float* lg = reinterpret_cast<float*>(rsm);               // [T][E] (x staging is no longer needed)
-    float* bs = lg + a.T * a.E;                              // [E]
-    int32_t* ids_s = reinterpret_cast<int32_t*>(bs + a.E);   // [T][k]
+    int32_t* ids_s = reinterpret_cast<int32_t*>(lg + a.T * a.E);   // [T][k]
     int32_t* cnt = ids_s + a.T * a.k;                        // [E]
     {
         constexpr int LPT = 16;
-        const int n = a.T * a.E, nb = n + a.E;
-        for (int i0 = 0; i0 < nb; i0 += LPT * RD_WARPS * 32) {
+        const int n = a.T * a.E;
+        for (int i0 = 0; i0 < n; i0 += LPT * RD_WARPS * 32) {
             float v[LPT];
 #pragma unroll
             for (int j = 0; j < LPT; j++) {
                 const int i = i0 + j * RD_WARPS * 32 + threadIdx.x;
-                v[j] = i < n ? __ldcg(a.logits + i) : (i < nb && a.bias ? a.bias[i - n] : 0.f);
+                v[j] = i < n ? __ldcg(a.logits + i) : 0.f;
             }
 #pragma unroll
             for (int j = 0; j < LPT; j++) {
                 const int i = i0 + j * RD_WARPS * 32 + threadIdx.x;
-                if (i < nb) lg[i] = v[j];
+                if (i < n) lg[i] = v[j];
             }
         }
     }
     __syncthreads();
     for (int t = warp; t < a.T; t += RD_WARPS) {
         if (a.E <= 384)
-            topk_warp<12, true>(lg + t * a.E, bs, a.E, a.k, a.ids + size_t(t) * a.k, a.w + size_t(t) * a.k, lane,
-                                ids_s + t * a.k);
+            topk_warp<12, true>(lg + t * a.E, nullptr, a.E, a.k, a.ids + size_t(t) * a.k, a.w + size_t(t) * a.k,
+                                lane, ids_s + t * a.k);
         else
-            topk_warp<kMaxE / 32, true>(lg + t * a.E, bs, a.E, a.k, a.ids + size_t(t) * a.k, a.w + size_t(t) * a.k,
-                                        lane, ids_s + t * a.k);
+            topk_warp<kMaxE / 32, true>(lg + t * a.E, nullptr, a.E, a.k, a.ids + size_t(t) * a.k,
+                                        a.w + size_t(t) * a.k, lane, ids_s + t * a.k);
     }
     if (threadIdx.x == 0) *a.counter = 0;
     if (a.sh_offsets) {
@@ -416,8 +425,8 @@ __global__ void __launch_bounds__(RD_WARPS * 32) router_decode(RouterDecodeArgs 
 }
 
 int launch_route_decode(const RouterDecodeArgs& a, cudaStream_t s) {
-    // x staging, then (the last CTA) logits, bias, ids and the bucket counters
-    const size_t smem = std::max<size_t>(size_t(a.T) * a.H * 2, (size_t(a.T) * a.E + 2 * size_t(a.E) + size_t(a.T) * a.k) * 4);
+    // x staging, then (the last CTA) scores, ids and the bucket counters
+    const size_t smem = std::max<size_t>(size_t(a.T) * a.H * 2, (size_t(a.T) * a.E + size_t(a.E) + size_t(a.T) * a.k) * 4);
     if (a.T > RD_TMAX || a.H % 512) return MOE_ERR_UNSUPPORTED;
     auto k = a.x_f16 ? router_decode<true> : router_decode<false>;
     if (smem > 48 * 1024 &&

@@ -67,6 +67,9 @@ _sig("moe_grouped_w4a16_down", _I, [_P, _P, _P, _P, _I, _P, _P, _P, _SZ, _P])
 _sig("moe_unpermute_combine", _I, [_P, _P, _I, _I, _I, _P, _P, _P])
 _sig("moe_layer_decode", _I, [_P, _I, _P, _P, _P, _SZ, _P])
 _sig("moe_layer_forward", _I, [_P, _I, _P, _P, _P, _SZ, _P])
+_sig("moe_layer_graph_create", _I, [_P, _I, _P, _P, _P, _SZ, ctypes.POINTER(_P)])
+_sig("moe_layer_graph_launch", _I, [_P, _P])
+_sig("moe_layer_graph_destroy", _I, [_P])
 _sig("moe_quantize_int4_g128", _I, [_P, _I64, _I64, _P, _P, _P])
 _sig("moe_quantize_nvfp4", _I, [_P, _I64, _I64, _P, _P, _P, _P, _SZ, _P])
 _sig("moe_quantize_nvfp4_act", _I, [_P, _I64, _I64, _P, _P, _P, _P])
@@ -248,6 +251,36 @@ def layer_decode(x, layer, ws, out=None):
     _check("moe_layer_decode", lib.moe_layer_decode(_ptr(x), T, ctypes.byref(L), _ptr(y), _ptr(ws),
                                                     ws.numel(), _stream()))
     return y
+
+
+class LayerGraph:
+    """One layer call (moe_layer_forward on these exact tensors) recorded as a CUDA graph;
+    launch() replays it on the current stream.  x is read and out written in place at every
+    launch; the tensors and the layer's banks are held until the graph is released."""
+
+    def __init__(self, x, layer, ws, out=None):
+        self.x, self.layer, self.ws = x, layer, ws
+        self.y = out if out is not None else torch.empty_like(x)
+        self._L = layer.struct()
+        h = _P()
+        _check("moe_layer_graph_create", lib.moe_layer_graph_create(
+            _ptr(x), x.shape[0], ctypes.byref(self._L), _ptr(self.y), _ptr(ws), ws.numel(), ctypes.byref(h)))
+        self._h = h
+
+    def launch(self):
+        _check("moe_layer_graph_launch", lib.moe_layer_graph_launch(self._h, _stream()))
+        return self.y
+
+    def close(self):
+        if getattr(self, "_h", None) is not None and self._h.value:
+            lib.moe_layer_graph_destroy(self._h)
+        self._h = None
+
+    def __del__(self):
+        try:
+            self.close()
+        except Exception:
+            pass
 
 
 def layer_forward(x, layer, ws, out=None):
