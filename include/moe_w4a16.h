@@ -243,14 +243,15 @@ int moe_permute_noalloc(const int32_t* topk_ids, int T, int top_k, int E,
  * and row_slot[i] = i * top_k.  rows = T*top_k (T for E = 1).  With H a
  * multiple of 256 and F of 128 the call runs the tcgen05 grouped GEMM: int4
  * banks with E > 1 and rows <= 512 on the 8-bit tensor-core path (x as three
- * 8-bit digits of a per-row 24-bit fixed point, exact integer sums per scale
- * group), everything else on the 16-bit one; other shapes stream the weights
- * with a GEMV.
+ * 8-bit digits of a 24-bit fixed point with an exponent per row and scale
+ * group, exact integer sums per scale group), everything else on the 16-bit
+ * one; other shapes stream the weights with a GEMV.
  * ws (256-byte aligned): at least 1024 + a(16*(E+2)) + max(a(rows*H/8) +
- * a(2*rows*H), a(4*rows) + a(rows*H/32) + a(c*rows*H)) bytes, c = 3 for
- * rows <= 512 and 2 above, plus a(8*k*rows*F) for a BF16 bank with E = 1 and
- * rows <= 64 (split-K partial sums, k = 8 halved while H is not a multiple of
- * 128*k); a() rounds up to a multiple of 256.  moe_workspace_bytes(T, H, E, F,
+ * a(2*rows*H), a(4*rows) + a(8*rows*z) + a(c*rows*H)) bytes, z = H/128
+ * rounded up to a multiple of 4, c = 3 for rows <= 512 and 2 above, plus
+ * a(8*k*rows*F) for a BF16 bank with E = 1 and rows <= 64 (split-K partial
+ * sums, k = 4 halved while H is not a multiple of 128*k); a() rounds up to a
+ * multiple of 256.  moe_workspace_bytes(T, H, E, F,
  * top_k) is always enough. */
 int moe_grouped_w4a16_swiglu(const void* x, int T, int H,
                              const int32_t* expert_offsets, const int32_t* row_slot,
@@ -271,10 +272,10 @@ int moe_grouped_w4a16_swiglu(const void* x, int T, int H,
  * gate/up call's rule with the roles of H and F exchanged (F a multiple of
  * 256, H of 128 for the GEMM).
  * ws (256-byte aligned): at least 1024 + a(16*(E+2)) + max(a(rows*F/8) +
- * a(2*rows*F), a(4*rows) + a(rows*F/32) + a(c*rows*F)) bytes, c = 3 for
- * rows <= 512 and 2 above, plus a(4*k*rows*H) for a BF16 bank with E = 1 and
- * rows <= 64 (k = 4 halved while F is not a multiple of 128*k); a() rounds up
- * to a multiple of 256.  moe_workspace_bytes(T, H, E, F, top_k) with
+ * a(2*rows*F), a(4*rows) + a(8*rows*z) + a(c*rows*F)) bytes, z = F/128
+ * rounded up to a multiple of 4, c = 3 for rows <= 512 and 2 above, plus
+ * a(4*k*rows*H) for a BF16 bank with E = 1 and rows <= 64 (k = 2 halved while
+ * F is not a multiple of 128*k); a() rounds up to a multiple of 256.  moe_workspace_bytes(T, H, E, F, top_k) with
  * rows = T*top_k is always enough. */
 int moe_grouped_w4a16_down(const void* h_perm, const int32_t* expert_offsets,
                            const int32_t* row_slot, const float* topk_w, int rows,

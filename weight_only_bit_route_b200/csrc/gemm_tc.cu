@@ -201,13 +201,18 @@ struct GArgs {
     __nv_bfloat16* out;
     int32_t* status;
     float* partial;                  // split-K: fp32 partial sums [ksplit][nmat][rows][out_dim]
-    const float* zsum;               // 8-bit int4: 8 * sum of the row's fixed-point values per group [rows][zst]
+    const float* zsum;               // 8-bit int4: per row, 8 * sum of the fixed-point values of each group, then each
+                                     // group's 2^-c: [rows][2 * zst]
     int E, out_dim, in_dim;
     int ksplit, rows;                // K slices per (m-tile, n-tile); activation rows of the problem
     int* tile_cnt;                   // split-K: zeroed arrival counters, four per (m-tile, n-tile); the last
                                      // epilogue warp of each quarter sums the slices (else a kernel does)
     int* sched;                      // null: tile blockIdx.x + i * gridDim.x; else {next, done}: tiles handed out by
                                      // an atomic counter, zero on entry, left at zero by the last CTA
+    int early;                       // the kernel before is this GEMM's pre-pass, which lets it start once that has
+                                     // waited for its own predecessor: only the roles that read the pre-pass's
+                                     // output (activation producer, epilogue) wait for it; the tile list and the
+                                     // weight stream start at once
     int npk;                         // weight stages in the shared-memory ring (2 .. kPkMax)
     int nsc;                         // int4 scale buffers (2 .. G_SC_MAX)
 };
@@ -336,7 +341,7 @@ __global__ void __launch_bounds__(G_THREADS, 1) tc_grouped_gemm(const __grid_con
     const int zst = ((ngroups + 3) & ~3);                           // i8: group-sum row stride
     // one scale buffer: the int4 scales of the tile's rows (per matrix), then
     // (i8) the group sums of the tile's tokens
-    const uint32_t sc_buf_bytes = C::kNMat * sc_mat_bytes + (C::kI8 ? uint32_t(C::kNMax * zst * 4) : 0u);
+    const uint32_t sc_buf_bytes = C::kNMat * sc_mat_bytes + (C::kI8 ? uint32_t(C::kNMax * 2 * zst * 4) : 0u);
     const uint32_t NPK = uint32_t(a.npk);                          // weight stages in the ring
     const int NSC = a.nsc;                                          // int4 scale buffers, one tile each
 
@@ -353,7 +358,7 @@ __global__ void __launch_bounds__(G_THREADS, 1) tc_grouped_gemm(const __grid_con
         for (int s = 0; s < G_DONE; s++)
             asm volatile("mbarrier.init.shared::cta.b64 [%0], 1;" ::"r"(g_smem(&done[s])));
         for (int s = 0; s < a.nsc; s++) {
-            asm volatile("mbarrier.init.shared::cta.b64 [%0], 1;" ::"r"(g_smem(&sc_full[s])));
+            asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(g_smem(&sc_full[s])), "r"(C::kI8 ? 2 : 1));
             asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(g_smem(&sc_empty[s])), "r"(C::kScStages));
         }
         for (int s = 0; s < 2; s++)          // (at most two buffers on the 16-bit paths)
@@ -376,7 +381,7 @@ __global__ void __launch_bounds__(G_THREADS, 1) tc_grouped_gemm(const __grid_con
         asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], 512;" ::"r"(g_smem(&s_tmem)));
         asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;");
     }
-    asm volatile("griddepcontrol.wait;" ::: "memory");
+    if (!a.early) asm volatile("griddepcontrol.wait;" ::: "memory");
     if (tid == 0) {                                   // published by the __syncthreads below
         s_ab.limit_ns = g_limit_from(a.status);
         s_hold = g_hold_from(a.status);
@@ -519,13 +524,10 @@ __global__ void __launch_bounds__(G_THREADS, 1) tc_grouped_gemm(const __grid_con
                 if (t >= NSC && !g_wait_w(g_smem(&sc_empty[b]), ((t / NSC) - 1) & 1, &s_ab, 64)) { fail(); break; }
                 const uint32_t bar = g_smem(&sc_full[b]);
                 uint8_t* dst = scbuf + b * sc_buf_bytes;
-                const uint32_t zbytes = C::kI8 ? uint32_t(T.nval * zst * 4) : 0u;
-                if (g_elect()) {
-                    g_expect(bar, sc_mat_bytes * C::kNMat + zbytes);
+                if (g_elect()) {         // (8-bit: the tokens' group sums come from the activation producer)
+                    g_expect(bar, sc_mat_bytes * C::kNMat);
                     g_bulk(g_smem(dst), a.sc0 + size_t(row0) * ngroups * 2, sc_mat_bytes, bar);
                     if (GU) g_bulk(g_smem(dst + sc_mat_bytes), a.sc1 + size_t(row0) * ngroups * 2, sc_mat_bytes, bar);
-                    if (C::kI8)
-                        g_bulk(g_smem(dst + C::kNMat * sc_mat_bytes), a.zsum + size_t(T.ebase + T.n0) * zst, zbytes, bar);
                 }
                 __syncwarp();
             }
@@ -589,13 +591,35 @@ __global__ void __launch_bounds__(G_THREADS, 1) tc_grouped_gemm(const __grid_con
         __syncwarp();
     } else if (warp == 1) {
         // ---------------- activation producer (whole warp, one lane issues) ----------------
+        // The activation rows come from the kernel before (the pre-pass): with an early start the
+        // weight stream has been running since the prologue, and this role waits for them here.
+        if (a.early) asm volatile("griddepcontrol.wait;" ::: "memory");
         uint32_t bc = 0;
         uint32_t qi = 0;
-        for (int tile = q_take(qi); tile < ntiles && !g_aborted(&s_ab); tile = q_take(qi)) {
+        int t = 0;
+        bool ok = true;
+        for (int tile = q_take(qi); tile < ntiles && ok && !g_aborted(&s_ab); tile = q_take(qi), t++) {
             const GTile T = tile_of(tile);
             const int row0 = (C::kI8 ? 3 : 1) * (T.ebase + T.n0);      // i8: three digit rows per token
             const CUtensorMap* map = &a.tm_b[C::kI8 ? 0 : T.bn / 16 - 1];
-            bool ok = true;
+            if constexpr (C::kI8) {
+                // the tile's tokens' group sums and factors, into the tile's scale buffer beside the
+                // weight scales that warp 0 copies (sc_full takes both arrivals)
+                const int b = t % NSC;
+                if (t >= NSC && !g_wait_w(g_smem(&sc_empty[b]), ((t / NSC) - 1) & 1, &s_ab, 64)) {
+                    fail();
+                    ok = false;
+                    break;
+                }
+                const uint32_t bar = g_smem(&sc_full[b]);
+                const uint32_t zbytes = uint32_t(T.nval * 2 * zst * 4);
+                if (g_elect()) {
+                    g_expect(bar, zbytes);
+                    g_bulk(g_smem(scbuf + b * sc_buf_bytes + C::kNMat * sc_mat_bytes),
+                           a.zsum + size_t(T.ebase + T.n0) * 2 * zst, zbytes, bar);
+                }
+                __syncwarp();
+            }
             for (int ks = 0; ks < KS; ks++, bc++) {
                 const int s = bc % C::kBStages;
                 if (bc >= uint32_t(C::kBStages) && !g_wait_w(g_smem(&done[(bc - C::kBStages) % G_DONE]),
@@ -752,6 +776,7 @@ __global__ void __launch_bounds__(G_THREADS, 1) tc_grouped_gemm(const __grid_con
         // j < kNMax also holds token j's row factor.  A step holds kGroups scale
         // groups, each in its own 16 accumulator columns (gate, then up); token
         // j's digit sums are columns 3j (d2), 3j+1 (d1), 3j+2 (d0) of a group.
+        if (a.early) asm volatile("griddepcontrol.wait;" ::: "memory");   // the pre-pass's row factors and sums
         const int q = warp & 3;
         const uint32_t lane_addr = uint32_t(q * 32) << 16;
         const int r = q * 32 + lane;
@@ -765,8 +790,8 @@ __global__ void __launch_bounds__(G_THREADS, 1) tc_grouped_gemm(const __grid_con
             const int rbase = T.ebase + T.n0;
             const bool live = lane < T.nval;
             const int b = t % NSC;
-            // the row factor (2^-c, times the routing weight on down, folded by the pre-pass)
-            // is needed after the last step: issue its load now
+            // the row factor (the routing weight on down, 1 on gate/up) is needed after the last
+            // step: issue its load now
             const float rowf = live ? a.act_scale[rbase + lane] : 1.f;
             if (!g_wait_w(g_smem(&sc_full[b]), (t / NSC) & 1, &s_ab, 64)) { ok = false; break; }
             const __nv_bfloat16* sc0 = reinterpret_cast<const __nv_bfloat16*>(scbuf + b * sc_buf_bytes) + r * ngroups;
@@ -806,14 +831,15 @@ __global__ void __launch_bounds__(G_THREADS, 1) tc_grouped_gemm(const __grid_con
 #pragma unroll
                     for (int j = 0; j < C::kNMax; j++) {
                         if (j >= T.nval) break;                  // uniform: the tokens of this tile only
-                        const float zj = zs[j * zst + grp];
+                        // the group's sum of u X less 8 sum X, times 2^-c of the group (exact), times the scale
+                        const float zj = zs[j * 2 * zst + grp], fj = zs[j * 2 * zst + zst + grp];
                         const float vg = fmaf(float(int(g[gi][3 * j])), 65536.f,
                                               fmaf(float(int(g[gi][3 * j + 1])), 256.f, float(int(g[gi][3 * j + 2])))) - zj;
-                        tg[j] = fmaf(s0, vg, tg[j]);
+                        tg[j] = fmaf(s0, vg * fj, tg[j]);
                         if (GU) {
                             const float vu = fmaf(float(int(u[gi][3 * j])), 65536.f,
                                                   fmaf(float(int(u[gi][3 * j + 1])), 256.f, float(int(u[gi][3 * j + 2])))) - zj;
-                            tu[j] = fmaf(s1, vu, tu[j]);
+                            tu[j] = fmaf(s1, vu * fj, tu[j]);
                         }
                     }
                 }
@@ -839,6 +865,7 @@ __global__ void __launch_bounds__(G_THREADS, 1) tc_grouped_gemm(const __grid_con
         if (!ok) fail();
     } else if (warp >= 4 && warp < 8) {
         // ---------------- epilogue ----------------
+        if (a.early) asm volatile("griddepcontrol.wait;" ::: "memory");   // the pre-pass's row factors
         const int q = warp & 3;
         const uint32_t lane_addr = uint32_t(q * 32) << 16;
         int t = 0;
@@ -1214,6 +1241,8 @@ __global__ void __launch_bounds__(256) g_prep(const __nv_bfloat16* __restrict__ 
                                               const int32_t* __restrict__ offsets, int E,
                                               const float* __restrict__ in_scale, size_t sc_off) {
     asm volatile("griddepcontrol.wait;" ::: "memory");
+    // the GEMM that reads these rows may start now (its weight stream needs nothing from here)
+    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
     const int row = (blockIdx.x * blockDim.x + threadIdx.x) >> 5, lane = threadIdx.x & 31;
     if (row >= rows) return;
     const int srow = by_token ? row_slot[row] / top_k : row;
@@ -1283,37 +1312,38 @@ __global__ void __launch_bounds__(256) g_prep(const __nv_bfloat16* __restrict__ 
 }
 
 // 8-bit int4 pre-pass: one CTA of 128 threads per GEMM row (gathered like
-// g_prep).  X = rint(x * 2^c), c the row's exponent that puts max |X| in
-// [2^21, 2^22), written as signed digits X = 65536 d2 + 256 d1 + d0 in int8
-// rows 3 row (d2), 3 row + 1 (d1), 3 row + 2 (d0) of dst, in the K order
-// 0, 2, 4, 6, 1, 3, 5, 7 of every 8 (the order of the unpacked weight bytes);
-// scale[row] = 2^-c, times row_w[row_slot[row]] when row_w is given (the
-// down projection's routing weight; a power of two times w is exact);
-// zsum[row][g] (row stride zst) = 8 * sum of X over group g, the u - 8 offset
-// of the weights.  A row holding an infinity or a NaN has no fixed point: it
-// records MOE_ERR_NONFINITE and gets a NaN row factor, so its outputs are NaN
-// (as a floating-point product with that row would be) instead of finite
-// values made from meaningless digits.
+// g_prep).  Per scale group g of 128 elements, X = rint(x * 2^c), c the
+// group's exponent that puts its max |X| in [2^21, 2^22), written as signed
+// digits X = 65536 d2 + 256 d1 + d0 in int8 rows 3 row (d2), 3 row + 1 (d1),
+// 3 row + 2 (d0) of dst, in the K order 0, 2, 4, 6, 1, 3, 5, 7 of every 8
+// (the order of the unpacked weight bytes).  zf[row] holds two arrays of zst
+// floats: [g] = 8 * sum of X over group g (the u - 8 offset of the weights),
+// then [zst + g] = 2^-c of group g.  scale[row] = row_w[row_slot[row]] when
+// row_w is given (the down projection's routing weight), else 1.  A group
+// holding an infinity or a NaN has no fixed point: it records
+// MOE_ERR_NONFINITE and gets a NaN factor, so its token's outputs are NaN (as
+// a floating-point product with that row would be) instead of finite values
+// made from meaningless digits.  The 16 threads of a half warp hold a group
+// (8 elements each), so every exponent comes from a half-warp reduction.
 constexpr int G_PREP_I8_THREADS = 128;
 template <bool F16>
 __global__ void __launch_bounds__(G_PREP_I8_THREADS) g_prep_i8(const __nv_bfloat16* __restrict__ src, int in_dim,
                                                                const int32_t* __restrict__ row_slot, int top_k,
                                                                int by_token, const float* __restrict__ row_w,
                                                                uint8_t* __restrict__ dst, float* __restrict__ scale,
-                                                               float* __restrict__ zsum, int32_t* status) {
-    __shared__ float s_max[G_PREP_I8_THREADS / 32];
+                                                               float* __restrict__ zf, int32_t* status) {
     asm volatile("griddepcontrol.wait;" ::: "memory");
     // the GEMM that reads these rows may be placed on free SMs now; it waits for this grid
     asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
     const int row = blockIdx.x, tid = threadIdx.x, lane = tid & 31;
     const int slot = (by_token || row_w) ? row_slot[row] : 0;
-    // the row's routing weight (down): its load goes out with the row's, it is used last
-    const float rw = (tid == 0 && row_w) ? row_w[slot] : 1.f;
+    const float rw = (tid == 0 && row_w) ? row_w[slot] : 1.f;   // used last: its load goes out first
     const int srow = by_token ? slot / top_k : row;
     const uint4* s = reinterpret_cast<const uint4*>(src + size_t(srow) * in_dim);
     const int n16 = in_dim / 8, zst = ((in_dim / 128) + 3) & ~3;
-    // the row stays in registers between the two passes (up to kPrepRegs chunks per thread;
-    // wider rows read the rest again)
+    float* zrow = zf + size_t(row) * 2 * zst;
+    uint8_t* d8 = dst + size_t(row) * 3 * in_dim;
+    // every chunk's load goes out before any is used (up to kPrepRegs chunks per thread)
     constexpr int kPrepRegs = 4;
     uint4 v[kPrepRegs];
 #pragma unroll
@@ -1321,30 +1351,21 @@ __global__ void __launch_bounds__(G_PREP_I8_THREADS) g_prep_i8(const __nv_bfloat
         const int i = tid + j * G_PREP_I8_THREADS;
         v[j] = i < n16 ? s[i] : make_uint4(0, 0, 0, 0);
     }
-    float amax = 0.f;
-    auto fold = [&](const uint4 w) {
-        amax = fmaxf(amax, fmaxf(fmaxf(fabsf(act_lo<F16>(w.x)), fabsf(act_hi<F16>(w.x))), fmaxf(fabsf(act_lo<F16>(w.y)), fabsf(act_hi<F16>(w.y)))));
-        amax = fmaxf(amax, fmaxf(fmaxf(fabsf(act_lo<F16>(w.z)), fabsf(act_hi<F16>(w.z))), fmaxf(fabsf(act_lo<F16>(w.w)), fabsf(act_hi<F16>(w.w)))));
-    };
-#pragma unroll
-    for (int j = 0; j < kPrepRegs; j++) fold(v[j]);
-    for (int i = tid + kPrepRegs * G_PREP_I8_THREADS; i < n16; i += G_PREP_I8_THREADS) fold(s[i]);
-    for (int o = 16; o > 0; o >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, o));
-    if (lane == 0) s_max[tid >> 5] = amax;
-    __syncthreads();
-    amax = fmaxf(fmaxf(s_max[0], s_max[1]), fmaxf(s_max[2], s_max[3]));
-    const bool finite = isfinite(amax);                 // amax is NaN or inf when any element is
-    int ex = 0;
-    if (finite) frexpf(amax, &ex);                      // amax < 2^ex
-    const int c = (finite && amax > 0.f) ? min(22 - ex, 126) : 0;   // |x| 2^c < 2^22
-    const float fc = ldexpf(1.f, c);                    // a power of two: x * fc is exact
-    uint8_t* d8 = dst + size_t(row) * 3 * in_dim;
-    // 16 pieces of 8 make a group of 128: lanes 0-15 and 16-31 hold one group each
+    bool bad = false;
     auto emit = [&](const int i, const uint4 w) {
+        const float xs[8] = {act_lo<F16>(w.x), act_lo<F16>(w.y), act_lo<F16>(w.z), act_lo<F16>(w.w),
+                             act_hi<F16>(w.x), act_hi<F16>(w.y), act_hi<F16>(w.z), act_hi<F16>(w.w)};
+        float amax = 0.f;
+#pragma unroll
+        for (int e = 0; e < 8; e++) amax = fmaxf(amax, fabsf(xs[e]));
+        for (int o = 8; o > 0; o >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, o));
+        const bool finite = isfinite(amax);             // amax is NaN or inf when any element is
+        int ex = 0;
+        if (finite) frexpf(amax, &ex);                  // amax < 2^ex
+        const int c = (finite && amax > 0.f) ? min(22 - ex, 126) : 0;   // |x| 2^c < 2^22
+        const float fc = ldexpf(1.f, c);                // a power of two: x * fc is exact
         int zs = 0;
         if (i < n16) {
-            const float xs[8] = {act_lo<F16>(w.x), act_lo<F16>(w.y), act_lo<F16>(w.z), act_lo<F16>(w.w),
-                                 act_hi<F16>(w.x), act_hi<F16>(w.y), act_hi<F16>(w.z), act_hi<F16>(w.w)};
             uint32_t p2[2] = {0u, 0u}, p1[2] = {0u, 0u}, p0[2] = {0u, 0u};
 #pragma unroll
             for (int e = 0; e < 8; e++) {
@@ -1363,7 +1384,11 @@ __global__ void __launch_bounds__(G_PREP_I8_THREADS) g_prep_i8(const __nv_bfloat
             *reinterpret_cast<uint2*>(d8 + 2 * size_t(in_dim) + size_t(i) * 8) = make_uint2(p0[0], p0[1]);
         }
         for (int o = 8; o > 0; o >>= 1) zs += __shfl_xor_sync(0xffffffffu, zs, o);
-        if ((lane & 15) == 0 && i < n16) zsum[size_t(row) * zst + i / 16] = 8.f * float(zs);
+        if ((lane & 15) == 0 && i < n16) {
+            zrow[i / 16] = 8.f * float(zs);
+            zrow[zst + i / 16] = finite ? 1.f / fc : __int_as_float(0x7fc00000);   // quiet NaN
+            bad = bad || !finite;
+        }
     };
 #pragma unroll
     for (int j = 0; j < kPrepRegs; j++)
@@ -1372,14 +1397,8 @@ __global__ void __launch_bounds__(G_PREP_I8_THREADS) g_prep_i8(const __nv_bfloat
         const int i = i0 + tid;
         emit(i, i < n16 ? s[i] : make_uint4(0, 0, 0, 0));
     }
-    if (tid == 0) {
-        if (finite) {
-            scale[row] = (1.f / fc) * rw;
-        } else {
-            scale[row] = __int_as_float(0x7fc00000);        // quiet NaN
-            set_status(status, MOE_ERR_NONFINITE);
-        }
-    }
+    if (bad) set_status(status, MOE_ERR_NONFINITE);
+    if (tid == 0) scale[row] = rw;
 }
 
 // ---------------------------------------------------------------------------
@@ -1526,6 +1545,7 @@ int launch_grouped_gemm(const GemvProblem& p, bool gateup, int rows, const GemmB
     // int8 digit rows per row
     const void* bsrc = p.act;
     const float* ascale = nullptr;
+    bool prep_launched = false;
     if (!buf.act_ready || nv || i4) {
         if (!buf.act_buf || ((nv || i4) && !buf.scale_buf)) return MOE_ERR_WORKSPACE;
         if (i8) {
@@ -1546,6 +1566,7 @@ int launch_grouped_gemm(const GemvProblem& p, bool gateup, int rows, const GemmB
         }
         bsrc = buf.act_buf;
         ascale = buf.scale_buf;
+        prep_launched = true;
     }
 
     GArgs a;
@@ -1597,6 +1618,7 @@ int launch_grouped_gemm(const GemvProblem& p, bool gateup, int rows, const GemmB
     a.rows = rows;
     a.zsum = buf.zbuf;
     a.sched = buf.sched;
+    a.early = prep_launched ? 1 : 0;
     // wide gate/up tiles (128 token rows) once the experts average more than 64 rows; narrow ones
     // (16) when no expert can hold more than 16 rows (BF16 and the NVFP4 16-bit path)
     const bool wide = gateup && ksplit == 1 && rows > 64 * E;

@@ -84,11 +84,11 @@ constexpr int kI8Int4MaxRows = 512;
 // Row stride (floats) of the 8-bit int4 group sums: in/128 rounded up to a
 // multiple of 4, so that a tile's rows are one 16-byte aligned block.
 inline int zsum_stride(int in_dim) { return ((in_dim / 128) + 3) & ~3; }
-// GEMM pre-pass output: row scales [rows] fp32, group sums [rows][zsum_stride] fp32,
-// then the gathered rows: 16-bit [rows][in], or three int8 digit rows per row
-// when the 8-bit int4 GEMM can take the problem.
+// GEMM pre-pass output: row scales [rows] fp32, group sums and group factors
+// [rows][2 * zsum_stride] fp32, then the gathered rows: 16-bit [rows][in], or
+// three int8 digit rows per row when the 8-bit int4 GEMM can take the problem.
 inline size_t gemm_prep_bytes(int rows, int in_dim) {
-    return align256(size_t(rows) * 4) + align256(size_t(rows) * zsum_stride(in_dim) * 4) +
+    return align256(size_t(rows) * 4) + align256(size_t(rows) * 2 * zsum_stride(in_dim) * 4) +
            align256(size_t(rows) * in_dim * (rows <= kI8Int4MaxRows ? 3 : 2));
 }
 // Step-level scratch of a grouped call: tile metadata, then the pre-pass of
@@ -98,10 +98,11 @@ inline size_t grouped_scratch(int E, int act_rows, int in_dim) {
 }
 
 // The BF16 shared expert at a small batch has few (m, n) tiles (12 for gate/up,
-// 32 for down); split K so that the weight stream spreads over the GPU.
+// 32 for down); split K so that the weight stream spreads over more SMs (48 and
+// 64 tiles: at decode sizes it runs beside the routed chain on at most 64 SMs).
 inline int shared_ksplit(int E, int fmt, bool gateup, int rows, int in_dim) {
     if (E != 1 || fmt != MOE_FMT_BF16 || rows > 64) return 1;
-    int ks = gateup ? 8 : 4;
+    int ks = gateup ? 4 : 2;
     while (ks > 1 && in_dim % (ks * 128)) ks >>= 1;
     return ks;
 }
