@@ -392,7 +392,8 @@ __global__ void __launch_bounds__(G_THREADS, 1) tc_grouped_gemm(const __grid_con
     uint8_t* dbase = smem + ((1024u - (g_smem(smem) & 1023u)) & 1023u);
     int4* tbl = reinterpret_cast<int4*>(dbase);
     {
-        // this CTA's first tile: asked for now, its latency hidden behind the scan below
+        // this CTA's first tile: asked for now, its latency partly hidden behind the scan below (a CTA
+        // that gets its SM late, behind another kernel, then holds no tile meanwhile)
         int first = int(blockIdx.x);
         if (tid == 0 && a.sched) first = atomicAdd(a.sched, 1);
         constexpr int PER = kMaxE / G_THREADS;
@@ -497,31 +498,31 @@ __global__ void __launch_bounds__(G_THREADS, 1) tc_grouped_gemm(const __grid_con
         // ---------------- weight producer (whole warp, one lane issues) ----------------
         uint32_t pc = 0, qi = 0;
         int t = 0;
-        int tile = s_first;
-        while (!g_aborted(&s_ab)) {
-            // hand the tile (or the end, >= ntiles) to the other roles
-            {
-                const uint32_t slot = qi % G_TQ;
-                if (qi >= G_TQ && !g_wait_w(g_smem(&tq_empty[slot]), ((qi / G_TQ) - 1) & 1, &s_ab, 32)) {
-                    fail();
-                    break;
-                }
-                if (lane == 0) {
-                    s_tq[slot] = tile;
-                    g_arrive(g_smem(&tq_full[slot]));
-                }
-                __syncwarp();
-                qi++;
+        // hand a tile (or the end, >= ntiles) to the other roles
+        auto publish = [&](int tile) -> bool {
+            const uint32_t slot = qi % G_TQ;
+            if (qi >= G_TQ && !g_wait_w(g_smem(&tq_empty[slot]), ((qi / G_TQ) - 1) & 1, &s_ab, 32)) {
+                fail();
+                return false;
             }
-            if (tile >= ntiles) break;
-            // the next tile's id: asked for now, read when this tile's copies are issued
-            int nxt = 0;
-            if (lane == 0 && a.sched) nxt = atomicAdd(a.sched, 1);
+            if (lane == 0) {
+                s_tq[slot] = tile;
+                g_arrive(g_smem(&tq_full[slot]));
+            }
+            __syncwarp();
+            qi++;
+            return true;
+        };
+        // the tile's scales and weight stages
+        auto produce = [&](int tile) -> bool {
             const GTile T = tile_of(tile);
             const int row0 = T.e * a.out_dim + T.m0;
             if (C::kInt4) {
                 const int b = t % NSC;
-                if (t >= NSC && !g_wait_w(g_smem(&sc_empty[b]), ((t / NSC) - 1) & 1, &s_ab, 64)) { fail(); break; }
+                if (t >= NSC && !g_wait_w(g_smem(&sc_empty[b]), ((t / NSC) - 1) & 1, &s_ab, 64)) {
+                    fail();
+                    return false;
+                }
                 const uint32_t bar = g_smem(&sc_full[b]);
                 uint8_t* dst = scbuf + b * sc_buf_bytes;
                 if (g_elect()) {         // (8-bit: the tokens' group sums come from the activation producer)
@@ -532,7 +533,6 @@ __global__ void __launch_bounds__(G_THREADS, 1) tc_grouped_gemm(const __grid_con
                 __syncwarp();
             }
             t++;
-            bool ok = true;
             for (int ps = 0; ps < NPS; ps++, pc++) {
                 const int s = pc % NPK;
                 // 4-bit stages are freed by the dequantisation warps, BF16 ones by the MMA step
@@ -540,8 +540,8 @@ __global__ void __launch_bounds__(G_THREADS, 1) tc_grouped_gemm(const __grid_con
                 if (pc >= NPK && !(C::kTmemA ? g_wait_w(g_smem(&pk_empty[s]), ((pc / NPK) - 1) & 1, &s_ab, 32)
                                              : g_wait_w(g_smem(&done[(pc - NPK) % G_DONE]), ((pc - NPK) / G_DONE) & 1,
                                                         &s_ab, 32))) {
-                    ok = false;
-                    break;
+                    fail();
+                    return false;
                 }
                 const uint32_t bar = g_smem(&pk_full[s]);
                 const uint32_t st = g_smem(pk + s * C::kPkStageBytes);
@@ -572,12 +572,30 @@ __global__ void __launch_bounds__(G_THREADS, 1) tc_grouped_gemm(const __grid_con
                 }
                 __syncwarp();
             }
-            if (!ok) { fail(); break; }
-            tile = a.sched ? __shfl_sync(0xffffffffu, nxt, 0) : tile + int(gridDim.x);
+            return true;
+        };
+        // Dynamic order: lane 0 asks for a tile id one tile before the id is needed, into one of two
+        // registers that the two halves of the loop below take turns with: an atomic under a full
+        // weight stream takes microseconds (its reply queues behind this SM's incoming copies), and a
+        // pending value must never be moved between registers, which would wait for it at once.
+        int tile = s_first, fa = 0, fb = 0;
+        if (lane == 0 && a.sched && tile < ntiles) fa = atomicAdd(a.sched, 1);
+        while (!g_aborted(&s_ab)) {
+            if (!publish(tile) || tile >= ntiles) break;
+            if (lane == 0 && a.sched) fb = atomicAdd(a.sched, 1);
+            if (!produce(tile)) break;
+            tile = a.sched ? __shfl_sync(0xffffffffu, fa, 0) : tile + int(gridDim.x);
+            if (g_aborted(&s_ab) || !publish(tile) || tile >= ntiles) break;
+            if (lane == 0 && a.sched) fa = atomicAdd(a.sched, 1);
+            if (!produce(tile)) break;
+            tile = a.sched ? __shfl_sync(0xffffffffu, fb, 0) : tile + int(gridDim.x);
         }
-        // the scheduler's counters: every CTA asks once past the end; the last one to do so
-        // leaves both at zero for the next launch
-        if (a.sched && lane == 0 && tile >= ntiles && atomicAdd(a.sched + 1, 1) == int(gridDim.x) - 1) {
+        // the scheduler's counters: a CTA stops at its first id past the end, with one id after it
+        // in flight; once that is back it counts itself done, and the last CTA to do so leaves both
+        // counters at zero for the next launch.  (Reading fa and fb makes the lane wait for the one
+        // in flight, so it is performed before the count; ids are never negative.)
+        if (a.sched && lane == 0 && tile >= ntiles &&
+            atomicAdd(a.sched + 1, (fa | fb) < 0 ? 2 : 1) == int(gridDim.x) - 1) {
             a.sched[0] = 0;
             a.sched[1] = 0;
         }
