@@ -276,7 +276,14 @@ def cpu_baseline(wl, moe, x, layer, budget_s=20.0):
 # captures of that kernel (summarised under profiles/), keyed by workload and by
 # a hash of the GEMM's sources at the time of the capture: a figure whose
 # kernel has changed since is reported as null.
-TRAFFIC = {}
+# DRAM bytes (read + write) of one launch of the dominant kernel, from one ncu capture of the bench's own
+# command (`ncu --metrics dram__bytes_read.sum,dram__bytes_write.sum,... -k regex:tc_grouped_gemm -s 0 -c 2`, and
+# the launch list of workload 2; profiles/), keyed by workload and by the hash of the GEMM's sources at the time:
+# a later change to the kernel drops the entry (reported as null).
+TRAFFIC = {
+    ("decode_int4_T8", "5baaf88a128019c7"): 390211840 + 3336448,
+    ("decode_nvfp4_T8", "5baaf88a128019c7"): 425676544 + 576256,
+}
 
 
 def gemm_source_hash():
@@ -395,7 +402,7 @@ def measure(moe, wl, x, layer, args, flush, stream, clk, pk, pk_kind, per_step=T
         raise RuntimeError("device status set during timing")
     ms = float(np.mean(ms_list))
     decode = T <= 64
-    traffic = TRAFFIC.get((wl.name, gemm_source_hash()))
+    traffic = None if fp4 else TRAFFIC.get((wl.name, gemm_source_hash()))    # (W4A4 runs another kernel)
     lbytes, lflops = layer_bytes(wl, touched), layer_flops(wl)
     kernel_name = "tc_grouped_gemm gate/up+SwiGLU (with its activation pre-pass)"
     if decode:
