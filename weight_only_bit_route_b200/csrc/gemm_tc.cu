@@ -322,6 +322,7 @@ __global__ void __launch_bounds__(G_THREADS, 1) tc_grouped_gemm(const __grid_con
     __shared__ __align__(8) uint64_t sf_full[G_SF_RING];   // A4: a step's scale-factor chunks are in place
     __shared__ __align__(8) uint64_t tq_full[G_TQ], tq_empty[G_TQ];   // tile queue
     __shared__ int s_tq[G_TQ];
+    __shared__ GTile s_tqt[G_TQ];                    // the queued tiles' coordinates (computed once, by warp 0)
     __shared__ int s_first;
     __shared__ int s_hold;
     __shared__ uint32_t s_tmem;
@@ -452,6 +453,17 @@ __global__ void __launch_bounds__(G_THREADS, 1) tc_grouped_gemm(const __grid_con
         const int local = tile - te.y;
         t.ebase = te.z;
         const int n_e = te.w;
+        if (ksplit == 1 && n_e <= C::kNMax) {
+            // one n-tile, no K slices (every decode tile): the m-tile is the position, no divisions
+            t.ks = 0;
+            t.kbase = 0;
+            t.mn = local;
+            t.m0 = local * G_BM;
+            t.n0 = 0;
+            t.nval = n_e;
+            t.bn = (n_e + 15) & ~15;
+            return t;
+        }
         const int ntile = (n_e + C::kNMax - 1) / C::kNMax;
         const int per = (n_e + ntile - 1) / ntile;                  // balanced rows per n-tile
         t.ks = local % ksplit;                                      // K slice fastest
@@ -481,13 +493,14 @@ __global__ void __launch_bounds__(G_THREADS, 1) tc_grouped_gemm(const __grid_con
     // the other roles take the same sequence.  A reader sees every phase of each slot in order (it
     // took the slot's previous entry itself), and warp 0 reuses a slot only after all readers have
     // taken its previous entry.  A wait that runs out ends the reader's loop (>= ntiles).
-    auto q_take = [&](uint32_t& qi) -> int {
+    auto q_take = [&](uint32_t& qi, GTile& T) -> int {
         const uint32_t slot = qi % G_TQ;
         if (!g_wait_w(g_smem(&tq_full[slot]), (qi / G_TQ) & 1, &s_ab)) {
             fail();
             return ntiles;
         }
         const int v = *reinterpret_cast<volatile int*>(&s_tq[slot]);
+        if (v < ntiles) T = s_tqt[slot];
         __syncwarp();
         if (lane == 0) g_arrive(g_smem(&tq_empty[slot]));
         qi++;
@@ -499,13 +512,14 @@ __global__ void __launch_bounds__(G_THREADS, 1) tc_grouped_gemm(const __grid_con
         uint32_t pc = 0, qi = 0;
         int t = 0;
         // hand a tile (or the end, >= ntiles) to the other roles
-        auto publish = [&](int tile) -> bool {
+        auto publish = [&](int tile, const GTile& T) -> bool {
             const uint32_t slot = qi % G_TQ;
             if (qi >= G_TQ && !g_wait_w(g_smem(&tq_empty[slot]), ((qi / G_TQ) - 1) & 1, &s_ab, 32)) {
                 fail();
                 return false;
             }
             if (lane == 0) {
+                if (tile < ntiles) s_tqt[slot] = T;
                 s_tq[slot] = tile;
                 g_arrive(g_smem(&tq_full[slot]));
             }
@@ -514,8 +528,7 @@ __global__ void __launch_bounds__(G_THREADS, 1) tc_grouped_gemm(const __grid_con
             return true;
         };
         // the tile's scales and weight stages
-        auto produce = [&](int tile) -> bool {
-            const GTile T = tile_of(tile);
+        auto produce = [&](const GTile& T) -> bool {
             const int row0 = T.e * a.out_dim + T.m0;
             if (C::kInt4) {
                 const int b = t % NSC;
@@ -580,14 +593,17 @@ __global__ void __launch_bounds__(G_THREADS, 1) tc_grouped_gemm(const __grid_con
         // pending value must never be moved between registers, which would wait for it at once.
         int tile = s_first, fa = 0, fb = 0;
         if (lane == 0 && a.sched && tile < ntiles) fa = atomicAdd(a.sched, 1);
+        GTile T{};
         while (!g_aborted(&s_ab)) {
-            if (!publish(tile) || tile >= ntiles) break;
+            if (tile < ntiles) T = tile_of(tile);
+            if (!publish(tile, T) || tile >= ntiles) break;
             if (lane == 0 && a.sched) fb = atomicAdd(a.sched, 1);
-            if (!produce(tile)) break;
+            if (!produce(T)) break;
             tile = a.sched ? __shfl_sync(0xffffffffu, fa, 0) : tile + int(gridDim.x);
-            if (g_aborted(&s_ab) || !publish(tile) || tile >= ntiles) break;
+            if (tile < ntiles) T = tile_of(tile);
+            if (g_aborted(&s_ab) || !publish(tile, T) || tile >= ntiles) break;
             if (lane == 0 && a.sched) fa = atomicAdd(a.sched, 1);
-            if (!produce(tile)) break;
+            if (!produce(T)) break;
             tile = a.sched ? __shfl_sync(0xffffffffu, fb, 0) : tile + int(gridDim.x);
         }
         // the scheduler's counters: a CTA stops at its first id past the end, with one id after it
@@ -616,8 +632,8 @@ __global__ void __launch_bounds__(G_THREADS, 1) tc_grouped_gemm(const __grid_con
         uint32_t qi = 0;
         int t = 0;
         bool ok = true;
-        for (int tile = q_take(qi); tile < ntiles && ok && !g_aborted(&s_ab); tile = q_take(qi), t++) {
-            const GTile T = tile_of(tile);
+        GTile T{};
+        for (int tile = q_take(qi, T); tile < ntiles && ok && !g_aborted(&s_ab); tile = q_take(qi, T), t++) {
             const int row0 = (C::kI8 ? 3 : 1) * (T.ebase + T.n0);      // i8: three digit rows per token
             const CUtensorMap* map = &a.tm_b[C::kI8 ? 0 : T.bn / 16 - 1];
             if constexpr (C::kI8) {
@@ -688,8 +704,8 @@ __global__ void __launch_bounds__(G_THREADS, 1) tc_grouped_gemm(const __grid_con
         uint32_t bc = 0, ac = 0, pc = 0;
         int t = 0;
         uint32_t qi = 0;
-        for (int tile = q_take(qi); tile < ntiles && !g_aborted(&s_ab); tile = q_take(qi), t++) {
-            const GTile T = tile_of(tile);
+        GTile T{};
+        for (int tile = q_take(qi, T); tile < ntiles && !g_aborted(&s_ab); tile = q_take(qi, T), t++) {
             const uint32_t idesc = C::kI8 ? g_idesc_i8(T.bn) : g_idesc(T.bn, C::kMmaF16);
             const int buf = C::kI8 ? 0 : t % C::kAccBufs;
             uint32_t d = tmem + buf * C::kAccCols;
@@ -802,8 +818,8 @@ __global__ void __launch_bounds__(G_THREADS, 1) tc_grouped_gemm(const __grid_con
         int t = 0;
         bool ok = true;
         uint32_t qi = 0;
-        for (int tile = q_take(qi); tile < ntiles && ok && !g_aborted(&s_ab); tile = q_take(qi), t++) {
-            const GTile T = tile_of(tile);
+        GTile T{};
+        for (int tile = q_take(qi, T); tile < ntiles && ok && !g_aborted(&s_ab); tile = q_take(qi, T), t++) {
             const int f = T.m0 + r;
             const int rbase = T.ebase + T.n0;
             const bool live = lane < T.nval;
@@ -888,8 +904,8 @@ __global__ void __launch_bounds__(G_THREADS, 1) tc_grouped_gemm(const __grid_con
         const uint32_t lane_addr = uint32_t(q * 32) << 16;
         int t = 0;
         uint32_t qi = 0;
-        for (int tile = q_take(qi); tile < ntiles && !g_aborted(&s_ab); tile = q_take(qi), t++) {
-            const GTile T = tile_of(tile);
+        GTile T{};
+        for (int tile = q_take(qi, T); tile < ntiles && !g_aborted(&s_ab); tile = q_take(qi, T), t++) {
             const int buf = t % C::kAccBufs;
             const int rbase = T.ebase + T.n0;
             // the factor of row c + j (activation row scale, routing weight) sits in lane j;
@@ -1021,8 +1037,8 @@ __global__ void __launch_bounds__(G_THREADS, 1) tc_grouped_gemm(const __grid_con
         uint32_t bc = 0;
         bool ok = true;
         uint32_t qi = 0;
-        for (int tile = q_take(qi); tile < ntiles && ok && !g_aborted(&s_ab); tile = q_take(qi)) {
-            const GTile T = tile_of(tile);
+        GTile T{};
+        for (int tile = q_take(qi, T); tile < ntiles && ok && !g_aborted(&s_ab); tile = q_take(qi, T)) {
             for (int ks = 0; ks < KS; ks++, bc++) {
                 if (!g_wait_w(g_smem(&pk_full[bc % NPK]), (bc / NPK) & 1, &s_ab) ||
                     !g_wait_w(g_smem(&b_full[bc % C::kBStages]), (bc / C::kBStages) & 1, &s_ab) ||
@@ -1069,7 +1085,8 @@ __global__ void __launch_bounds__(G_THREADS, 1) tc_grouped_gemm(const __grid_con
         uint32_t pc = 0;
         bool ok = true;
         uint32_t qi = 0;
-        for (int tile = q_take(qi); tile < ntiles && ok && !g_aborted(&s_ab); tile = q_take(qi)) {
+        GTile Tq{};
+        for (int tile = q_take(qi, Tq); tile < ntiles && ok && !g_aborted(&s_ab); tile = q_take(qi, Tq)) {
             for (int ps = 0; ps < NPS; ps++, pc++) {
                 if (int(pc & 1) != grp) continue;
                 const int s = pc % NPK;
@@ -1145,7 +1162,8 @@ __global__ void __launch_bounds__(G_THREADS, 1) tc_grouped_gemm(const __grid_con
         int t = 0;
         bool ok = true;
         uint32_t qi = 0;
-        for (int tile = q_take(qi); tile < ntiles && ok && !g_aborted(&s_ab); tile = q_take(qi), t++) {
+        GTile Tq{};
+        for (int tile = q_take(qi, Tq); tile < ntiles && ok && !g_aborted(&s_ab); tile = q_take(qi, Tq), t++) {
             const uint8_t* scrow = nullptr;
             float fk = 1.f;                             // int4: 2^k of this weight row (the epilogue undoes it)
             if (FMT == MOE_FMT_INT4_G128) {
