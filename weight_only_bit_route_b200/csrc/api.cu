@@ -81,7 +81,7 @@ GemmBuffers gemm_buffers(void* base, int rows, int in_dim, bool act_ready, bool 
     GemmBuffers b{};
     b.scale_buf = reinterpret_cast<float*>(p);
     b.zbuf = reinterpret_cast<float*>(p + align256(size_t(rows) * 4));
-    b.act_buf = p + align256(size_t(rows) * 4) + align256(size_t(rows) * 2 * zsum_stride(in_dim) * 4);
+    b.act_buf = p + align256(size_t(rows) * 4) + align256(size_t(rows) * zrow_floats(in_dim) * 4);
     b.act_ready = act_ready;
     b.i8 = i8;
     return b;

@@ -201,8 +201,8 @@ struct GArgs {
     __nv_bfloat16* out;
     int32_t* status;
     float* partial;                  // split-K: fp32 partial sums [ksplit][nmat][rows][out_dim]
-    const float* zsum;               // 8-bit int4: per row, 8 * sum of the fixed-point values of each group, then each
-                                     // group's 2^-c: [rows][2 * zst]
+    const float* zsum;               // 8-bit int4: per row, 8 * sum of the fixed-point values of each group, each
+                                     // group's 2^-c, the row factor: [rows][2 * zst + 4]
     int E, out_dim, in_dim;
     int ksplit, rows;                // K slices per (m-tile, n-tile); activation rows of the problem
     int* tile_cnt;                   // split-K: zeroed arrival counters, four per (m-tile, n-tile); the last
@@ -339,10 +339,11 @@ __global__ void __launch_bounds__(G_THREADS, 1) tc_grouped_gemm(const __grid_con
     const int NPS = kc / C::kPkK;                                   // weight stages per tile
     const int ngroups = in_dim / 128;
     const uint32_t sc_mat_bytes = uint32_t(G_BM * ngroups * 2);
-    const int zst = ((ngroups + 3) & ~3);                           // i8: group-sum row stride
+    const int zst = ((ngroups + 3) & ~3);                           // i8: groups per row record, rounded to 4
+    const int zrs = 2 * zst + 4;                                    // i8: row record (floats)
     // one scale buffer: the int4 scales of the tile's rows (per matrix), then
     // (i8) the group sums of the tile's tokens
-    const uint32_t sc_buf_bytes = C::kNMat * sc_mat_bytes + (C::kI8 ? uint32_t(C::kNMax * 2 * zst * 4) : 0u);
+    const uint32_t sc_buf_bytes = C::kNMat * sc_mat_bytes + (C::kI8 ? uint32_t(C::kNMax * zrs * 4) : 0u);
     const uint32_t NPK = uint32_t(a.npk);                          // weight stages in the ring
     const int NSC = a.nsc;                                          // int4 scale buffers, one tile each
 
@@ -646,11 +647,11 @@ __global__ void __launch_bounds__(G_THREADS, 1) tc_grouped_gemm(const __grid_con
                     break;
                 }
                 const uint32_t bar = g_smem(&sc_full[b]);
-                const uint32_t zbytes = uint32_t(T.nval * 2 * zst * 4);
+                const uint32_t zbytes = uint32_t(T.nval * zrs * 4);
                 if (g_elect()) {
                     g_expect(bar, zbytes);
                     g_bulk(g_smem(scbuf + b * sc_buf_bytes + C::kNMat * sc_mat_bytes),
-                           a.zsum + size_t(T.ebase + T.n0) * 2 * zst, zbytes, bar);
+                           a.zsum + size_t(T.ebase + T.n0) * zrs, zbytes, bar);
                 }
                 __syncwarp();
             }
@@ -824,13 +825,13 @@ __global__ void __launch_bounds__(G_THREADS, 1) tc_grouped_gemm(const __grid_con
             const int rbase = T.ebase + T.n0;
             const bool live = lane < T.nval;
             const int b = t % NSC;
-            // the row factor (the routing weight on down, 1 on gate/up) is needed after the last
-            // step: issue its load now
-            const float rowf = live ? a.act_scale[rbase + lane] : 1.f;
             if (!g_wait_w(g_smem(&sc_full[b]), (t / NSC) & 1, &s_ab, 64)) { ok = false; break; }
             const __nv_bfloat16* sc0 = reinterpret_cast<const __nv_bfloat16*>(scbuf + b * sc_buf_bytes) + r * ngroups;
             const __nv_bfloat16* sc1 = sc0 + G_BM * ngroups;
             const float* zs = reinterpret_cast<const float*>(scbuf + b * sc_buf_bytes + C::kNMat * sc_mat_bytes);
+            // the token's row factor (the routing weight on down, 1 on gate/up) travels in its row record
+            // (a global load from an SM under a full weight stream would take microseconds)
+            const float rowf = live ? zs[lane * zrs + 2 * zst] : 1.f;
             float tg[C::kNMax], tu[C::kNMax];
 #pragma unroll
             for (int j = 0; j < C::kNMax; j++) tg[j] = tu[j] = 0.f;
@@ -866,7 +867,7 @@ __global__ void __launch_bounds__(G_THREADS, 1) tc_grouped_gemm(const __grid_con
                     for (int j = 0; j < C::kNMax; j++) {
                         if (j >= T.nval) break;                  // uniform: the tokens of this tile only
                         // the group's sum of u X less 8 sum X, times 2^-c of the group (exact), times the scale
-                        const float zj = zs[j * 2 * zst + grp], fj = zs[j * 2 * zst + zst + grp];
+                        const float zj = zs[j * zrs + grp], fj = zs[j * zrs + zst + grp];
                         const float vg = fmaf(float(int(g[gi][3 * j])), 65536.f,
                                               fmaf(float(int(g[gi][3 * j + 1])), 256.f, float(int(g[gi][3 * j + 2])))) - zj;
                         tg[j] = fmaf(s0, vg * fj, tg[j]);
@@ -1352,10 +1353,11 @@ __global__ void __launch_bounds__(256) g_prep(const __nv_bfloat16* __restrict__ 
 // group's exponent that puts its max |X| in [2^21, 2^22), written as signed
 // digits X = 65536 d2 + 256 d1 + d0 in int8 rows 3 row (d2), 3 row + 1 (d1),
 // 3 row + 2 (d0) of dst, in the K order 0, 2, 4, 6, 1, 3, 5, 7 of every 8
-// (the order of the unpacked weight bytes).  zf[row] holds two arrays of zst
+// (the order of the unpacked weight bytes).  zf[row] is a record of 2 zst + 4
 // floats: [g] = 8 * sum of X over group g (the u - 8 offset of the weights),
-// then [zst + g] = 2^-c of group g.  scale[row] = row_w[row_slot[row]] when
-// row_w is given (the down projection's routing weight), else 1.  A group
+// [zst + g] = 2^-c of group g, [2 zst] = the row factor: row_w[row_slot[row]]
+// when row_w is given (the down projection's routing weight), else 1 (also in
+// scale[row]).  A group
 // holding an infinity or a NaN has no fixed point: it records
 // MOE_ERR_NONFINITE and gets a NaN factor, so its token's outputs are NaN (as
 // a floating-point product with that row would be) instead of finite values
@@ -1377,7 +1379,7 @@ __global__ void __launch_bounds__(G_PREP_I8_THREADS) g_prep_i8(const __nv_bfloat
     const int srow = by_token ? slot / top_k : row;
     const uint4* s = reinterpret_cast<const uint4*>(src + size_t(srow) * in_dim);
     const int n16 = in_dim / 8, zst = ((in_dim / 128) + 3) & ~3;
-    float* zrow = zf + size_t(row) * 2 * zst;
+    float* zrow = zf + size_t(row) * (2 * zst + 4);
     uint8_t* d8 = dst + size_t(row) * 3 * in_dim;
     // every chunk's load goes out before any is used (up to kPrepRegs chunks per thread)
     constexpr int kPrepRegs = 4;
@@ -1434,7 +1436,10 @@ __global__ void __launch_bounds__(G_PREP_I8_THREADS) g_prep_i8(const __nv_bfloat
         emit(i, i < n16 ? s[i] : make_uint4(0, 0, 0, 0));
     }
     if (bad) set_status(status, MOE_ERR_NONFINITE);
-    if (tid == 0) scale[row] = rw;
+    if (tid == 0) {
+        scale[row] = rw;
+        zrow[2 * zst] = rw;                              // the row factor, also in the row record
+    }
 }
 
 // ---------------------------------------------------------------------------

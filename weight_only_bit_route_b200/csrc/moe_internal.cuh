@@ -84,11 +84,13 @@ constexpr int kI8Int4MaxRows = 512;
 // Row stride (floats) of the 8-bit int4 group sums: in/128 rounded up to a
 // multiple of 4, so that a tile's rows are one 16-byte aligned block.
 inline int zsum_stride(int in_dim) { return ((in_dim / 128) + 3) & ~3; }
-// GEMM pre-pass output: row scales [rows] fp32, group sums and group factors
-// [rows][2 * zsum_stride] fp32, then the gathered rows: 16-bit [rows][in], or
+// 8-bit int4 row record (floats): group sums [zst], group factors [zst], the row factor, padding to 16 bytes
+inline int zrow_floats(int in_dim) { return 2 * zsum_stride(in_dim) + 4; }
+// GEMM pre-pass output: row scales [rows] fp32, the 8-bit path's row records
+// [rows][zrow_floats] fp32, then the gathered rows: 16-bit [rows][in], or
 // three int8 digit rows per row when the 8-bit int4 GEMM can take the problem.
 inline size_t gemm_prep_bytes(int rows, int in_dim) {
-    return align256(size_t(rows) * 4) + align256(size_t(rows) * 2 * zsum_stride(in_dim) * 4) +
+    return align256(size_t(rows) * 4) + align256(size_t(rows) * zrow_floats(in_dim) * 4) +
            align256(size_t(rows) * in_dim * (rows <= kI8Int4MaxRows ? 3 : 2));
 }
 // Step-level scratch of a grouped call: tile metadata, then the pre-pass of
@@ -265,7 +267,7 @@ struct GemmBuffers {
     int ksplit;          // > 1: split K into this many slices (BF16 only); fp32 partial sums go to partial
     float* partial;      // split_bytes(...) bytes
     int i8;              // int4 on the 8-bit MMA with per-group accumulation (small batches)
-    float* zbuf;         // i8: 8 * group sums of the fixed-point rows [rows][zsum_stride(in)]
+    float* zbuf;         // i8: row records [rows][zrow_floats(in)] (group sums, group factors, row factor)
     int* tile_cnt;       // split-K: kTileCounters zeroed ints (the control block's [16..255])
     int max_ctas;        // > 0: at most this many CTAs (a side-stream problem leaves the other SMs free)
     int no_pdl;          // launch without programmatic dependent launch (its CTAs hold no SM while waiting)
