@@ -276,13 +276,13 @@ def cpu_baseline(wl, moe, x, layer, budget_s=20.0):
 # captures of that kernel (summarised under profiles/), keyed by workload and by
 # a hash of the GEMM's sources at the time of the capture: a figure whose
 # kernel has changed since is reported as null.
-# DRAM bytes (read + write) of one launch of the dominant kernel, from one ncu capture of the bench's own
-# command (`ncu --metrics dram__bytes_read.sum,dram__bytes_write.sum,... -k regex:tc_grouped_gemm -s 0 -c 2`, and
-# the launch list of workload 2; profiles/), keyed by workload and by the hash of the GEMM's sources at the time:
-# a later change to the kernel drops the entry (reported as null).
+# DRAM bytes (read + write) of one launch of the dominant kernel, from the launch lists of the bench's own
+# command with `--metrics gpu__time_duration.sum,dram__bytes_read.sum,dram__bytes_write.sum` (profiles/), keyed
+# by workload and by the hash of the GEMM's sources at the time: a later change to the kernel drops the entry
+# (reported as null).
 TRAFFIC = {
-    ("decode_int4_T8", "5baaf88a128019c7"): 390211840 + 3336448,
-    ("decode_nvfp4_T8", "5baaf88a128019c7"): 425676544 + 576256,
+    ("decode_int4_T8", "6b3d2137b6c5e087"): 390216960 + 591616,
+    ("decode_nvfp4_T8", "6b3d2137b6c5e087"): 425606912 + 201216,
 }
 
 
