@@ -247,7 +247,7 @@ int moe_permute_noalloc(const int32_t* topk_ids, int T, int top_k, int E,
  * group, exact integer sums per scale group), everything else on the 16-bit
  * one; other shapes stream the weights with a GEMV.
  * ws (256-byte aligned): at least 1024 + a(16*(E+2)) + max(a(rows*H/8) +
- * a(2*rows*H), a(4*rows) + a(8*rows*z) + a(c*rows*H)) bytes, z = H/128
+ * a(2*rows*H), a(4*rows) + a(rows*(8*z+16)) + a(c*rows*H)) bytes, z = H/128
  * rounded up to a multiple of 4, c = 3 for rows <= 512 and 2 above, plus
  * a(8*k*rows*F) for a BF16 bank with E = 1 and rows <= 64 (split-K partial
  * sums, k = 4 halved while H is not a multiple of 128*k); a() rounds up to a
@@ -272,7 +272,7 @@ int moe_grouped_w4a16_swiglu(const void* x, int T, int H,
  * gate/up call's rule with the roles of H and F exchanged (F a multiple of
  * 256, H of 128 for the GEMM).
  * ws (256-byte aligned): at least 1024 + a(16*(E+2)) + max(a(rows*F/8) +
- * a(2*rows*F), a(4*rows) + a(8*rows*z) + a(c*rows*F)) bytes, z = F/128
+ * a(2*rows*F), a(4*rows) + a(rows*(8*z+16)) + a(c*rows*F)) bytes, z = F/128
  * rounded up to a multiple of 4, c = 3 for rows <= 512 and 2 above, plus
  * a(4*k*rows*H) for a BF16 bank with E = 1 and rows <= 64 (k = 2 halved while
  * F is not a multiple of 128*k); a() rounds up to a multiple of 256.  moe_workspace_bytes(T, H, E, F, top_k) with
