@@ -1,0 +1,135 @@
+"""Expert-parallel layer (weight_only_bit_route_b200/ep.py) on two CPU ranks over gloo.
+
+Each rank owns half of the routed experts and routes its own tokens; the steps run in the oracle (an injected
+step set: the collectives and the bookkeeping around them are what is tested here, the steps' kernels are
+tested on the GPU).  Bars: each rank's output is bit-identical to the same steps run on one process with every
+expert local, and within the layer tolerance of the oracle's fp64 layer.
+"""
+import os
+import socket
+
+import numpy as np
+import pytest
+import torch
+import torch.multiprocessing as mp
+
+
+def _free_port():
+    with socket.socket() as s:
+        s.bind(("127.0.0.1", 0))
+        return s.getsockname()[1]
+
+
+def _bits(t):
+    return t.contiguous().view(torch.int16).numpy().view(np.uint16)
+
+
+def _from_bits(b):
+    return torch.from_numpy(np.ascontiguousarray(b).view(np.int16)).view(torch.bfloat16)
+
+
+def _to_bf16(v):
+    u = np.asarray(v, np.float32).view(np.uint32).astype(np.uint64)
+    return ((u + 0x7fff + ((u >> 16) & 1)) >> 16).astype(np.uint16)
+
+
+class RefOps:
+    """The layer's steps in the oracle, with the GPU path's roundings (h and the expert outputs to bf16)."""
+
+    def __init__(self, oracle, P, e0, e1):
+        self.o, self.P, self.k = oracle, P, P.wl.k
+        self.e_local = e1 - e0
+        sl = slice(e0, e1)
+        self.banks = {w: oracle.Bank(b.fmt, b.packed[sl], b.scales[sl],
+                                     None if b.global_scale is None else b.global_scale[sl])
+                      for w, b in P.banks.items()}
+
+    def route(self, x):
+        ids, w = self.o.route(_bits(x), self.P.Wr, self.P.bias, self.k)
+        return torch.from_numpy(ids), torch.from_numpy(w)
+
+    def group(self, owner, world):
+        off, rs, sr = self.o.permute(owner.numpy(), world)
+        return torch.from_numpy(off), torch.from_numpy(rs), torch.from_numpy(sr)
+
+    def experts(self, xr, er, wr):
+        R = xr.shape[0]
+        if R == 0:
+            return torch.empty_like(xr)
+        off, rs, sr = self.o.permute(er.numpy().reshape(R, 1), self.e_local)
+        rows = np.arange(R, dtype=np.int32)
+        h = self.o.grouped_swiglu(_bits(xr), off, rs, 1, self.banks["gate"], self.banks["up"], rows)
+        yp = _to_bf16(self.o.grouped_down(_to_bf16(h), off, rs, wr.numpy(), self.banks["down"], rows))
+        return _from_bits(yp[sr])
+
+    def shared_expert(self, x):
+        if self.P.shared is None:
+            return None
+        T = x.shape[0]
+        so = np.array([0, T], np.int32)
+        srs = (np.arange(T) * self.k).astype(np.int32)
+        rows = np.arange(T, dtype=np.int32)
+        hs = self.o.grouped_swiglu(_bits(x), so, srs, self.k, self.P.shared[0], self.P.shared[1], rows)
+        return _from_bits(_to_bf16(self.o.grouped_down(_to_bf16(hs), so, srs, None, self.P.shared[2], rows)))
+
+    def combine(self, y_back, slot_pos, T, shared_out):
+        sh = None if shared_out is None else _bits(shared_out)
+        return _from_bits(_to_bf16(self.o.combine(_bits(y_back), slot_pos.numpy(), T, self.k, sh)))
+
+
+def _worker(rank, world, port, results):
+    import sys
+    root = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+    sys.path[:0] = [root, os.path.join(root, "tests")]
+    import torch.distributed as dist
+    import oracle
+    from problems import build, layer_tolerance
+    from weight_only_bit_route_b200 import ep
+    from weight_only_bit_route_b200 import synthetic as syn
+
+    dist.init_process_group("gloo", rank=rank, world_size=world, init_method=f"tcp://127.0.0.1:{port}")
+    try:
+        wl = syn.WORKLOADS[0]
+        P = build(0, "random", experts=list(range(wl.E)), shared=True)
+        x = _from_bits(syn.gen_x(wl, seed=100 + rank, T=13 if rank else 16))    # ragged: 16 and 13 tokens
+        e_per = wl.E // world
+        ops = RefOps(oracle, P, rank * e_per, (rank + 1) * e_per)
+        layer = ep.ExpertParallelMoE(ops.banks["gate"], ops.banks["up"], ops.banks["down"], P.Wr, top_k=wl.k,
+                                     max_tokens=16, ops=ops)
+        y = _bits(layer.forward(x))
+        # the same steps on one process, every expert local
+        full = RefOps(oracle, P, 0, wl.E)
+        ids, w = full.route(x)
+        T = x.shape[0]
+        off, rs, sr = full.group(torch.zeros(T, wl.k, dtype=torch.int32), 1)
+        ys = full.experts(x.index_select(0, rs.to(torch.int64) // wl.k), ids.view(-1)[rs.to(torch.int64)],
+                          w.view(-1)[rs.to(torch.int64)])
+        y1 = _bits(full.combine(ys, sr, T, full.shared_expert(x)))
+        ref = oracle.moe_forward(_bits(x), ids.numpy(), w.numpy(), P.banks["gate"], P.banks["up"], P.banks["down"],
+                                 shared=P.shared)
+        got = oracle.bf16_to_f32(y).astype(np.float64)
+        ok_tol = bool(np.all(np.abs(got - ref) <= layer_tolerance(ref)))
+        results.put((rank, bool(np.array_equal(y, y1)), ok_tol, int(T)))
+    finally:
+        dist.destroy_process_group()
+
+
+def test_expert_parallel_two_ranks_gloo():
+    ctx = mp.get_context("spawn")
+    results = ctx.Queue()
+    port = _free_port()
+    procs = [ctx.Process(target=_worker, args=(r, 2, port, results)) for r in range(2)]
+    for p in procs:
+        p.start()
+    for p in procs:
+        p.join(timeout=300)
+    codes = [p.exitcode for p in procs]
+    for p in procs:
+        if p.is_alive():
+            p.kill()
+    assert codes == [0, 0], f"rank exit codes {codes}"
+    got = sorted(results.get(timeout=5) for _ in range(2))
+    assert [g[3] for g in got] == [16, 13]
+    for rank, same, within, _ in got:
+        assert same, f"rank {rank}: the expert-parallel result differs from the one-process composition"
+        assert within, f"rank {rank}: outside the layer tolerance of the oracle"

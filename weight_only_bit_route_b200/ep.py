@@ -1,0 +1,132 @@
+"""Expert-parallel MoE layer: one process per GPU, the routed experts split across the ranks.
+
+The layer of "Step 5 Preview: 92 narrow layers, and a sparse indexer that scores blocks of 8" (The shape: 352
+routed experts, top-8, one shared expert per token), split the way the DEP8 deployment of the same page (15
+October) splits it: every rank keeps its own tokens (data parallel), the router and the shared expert are
+replicated, and rank r owns the routed experts [r * E / N, (r + 1) * E / N).  Per call on each rank:
+
+    1. route the rank's tokens (moe_route_topk);
+    2. group the T * top_k slots by owning rank (moe_permute with the ranks as the buckets);
+    3. all-to-all: each slot's token row, its expert (local to the owner) and its routing weight go to the owner;
+    4. the owner runs its experts on the rows it received, as a batch of single-slot tokens (moe_permute by local
+       expert, moe_grouped_w4a16_swiglu, moe_grouped_w4a16_down with the weight by row, moe_unpermute_combine with
+       top_k = 1, which puts the rows back in the order received);
+    5. all-to-all back, into the order the slots were sent;
+    6. the shared expert on the rank's own tokens, and moe_unpermute_combine with the inverse of step 2's grouping
+       (slot -> position in the returned rows): y[t] = shared[t] + sum_j of token t's returned rows.
+
+Every step of the layer runs in the library's kernels; this module marshals arguments and moves rows between
+ranks with torch.distributed (NCCL over NVLink on GPUs, gloo on CPU).  The collective is the stock all-to-all:
+rows cross the fabric once each way, and no multicast of any kind is used.  Each row's result is independent of
+which other rows share its tile, so on one rank the layer reproduces moe_layer_decode bit for bit.
+
+The split sizes of an all-to-all are host values, so each call reads the per-rank slot counts back to the host
+once (after step 2) and the returned counts once (after the counts' exchange).
+"""
+import torch
+import torch.distributed as dist
+
+from . import moe
+
+
+class CudaOps:
+    """The layer's steps on this rank's GPU, through the C ABI."""
+
+    def __init__(self, gate, up, down, router_w, router_bias, top_k, shared, max_tokens, world):
+        self.gate, self.up, self.down = gate, up, down
+        self.router_w, self.router_bias, self.k, self.shared = router_w, router_bias, top_k, shared
+        E, H = router_w.shape
+        F, e_local = gate.out_dim, gate.E
+        # route + owner grouping of up to max_tokens tokens; the experts of up to world * max_tokens * k rows.
+        # (moe_workspace_bytes sizes a whole layer, which needs top_k <= E: the owner grouping, with the ranks
+        # as its buckets, and the shared expert, E = 1, take a layer of top_k experts, which covers them.)
+        dev = router_w.device
+        self.ws_route = moe.workspace(max_tokens, H, E, F, top_k, device=dev)
+        self.ws_owner = moe.workspace(max_tokens, 128, max(world, top_k), 128, top_k, device=dev)
+        rows = max(world, 1) * max_tokens * top_k
+        self.ws_experts = moe.workspace(rows, H, e_local, F, 1, device=dev)
+        self.ws_shared = moe.workspace(max_tokens, H, top_k, F, top_k, device=dev) if shared else None
+
+    def route(self, x):
+        return moe.route_topk(x, self.router_w, self.router_bias, self.k, self.ws_route)
+
+    def group(self, owner, world):
+        return moe.permute(owner, world, self.ws_owner)
+
+    def experts(self, xr, er, wr):
+        R = xr.shape[0]
+        if R == 0:
+            return torch.empty_like(xr)
+        off, rs, sr = moe.permute(er.view(R, 1), self.gate.E, self.ws_experts)
+        h = moe.grouped_swiglu(xr, off, rs, 1, self.gate, self.up, R, self.ws_experts)
+        yp = moe.grouped_down(h, off, rs, wr, self.down, self.ws_experts)
+        return moe.unpermute_combine(yp, sr, R, 1)
+
+    def shared_expert(self, x):
+        if not self.shared:
+            return None
+        T = x.shape[0]
+        so = torch.tensor([0, T], dtype=torch.int32, device=x.device)
+        srs = torch.arange(T, dtype=torch.int32, device=x.device) * self.k
+        hs = moe.grouped_swiglu(x, so, srs, self.k, self.shared[0], self.shared[1], T, self.ws_shared)
+        return moe.grouped_down(hs, so, srs, None, self.shared[2], self.ws_shared)
+
+    def combine(self, y_back, slot_pos, T, shared_out):
+        return moe.unpermute_combine(y_back, slot_pos, T, self.k, shared_out)
+
+
+class ExpertParallelMoE:
+    """The routed experts [rank * E / world, (rank + 1) * E / world) of a layer on this rank.
+
+    gate, up, down: this rank's experts only (moe.Bank with E / world experts); router_w (fp32 [E, H]),
+    router_bias and shared (a (gate, up, down) tuple of E = 1 BF16 banks, or None) are the whole layer's,
+    replicated.  max_tokens bounds the tokens of one call on any rank.  ops replaces the step implementations
+    (tests run the collectives on CPU ranks with reference steps); by default the steps are the library's
+    kernels on this rank's GPU."""
+
+    def __init__(self, gate, up, down, router_w, top_k=8, router_bias=None, shared=None, group=None,
+                 max_tokens=64, ops=None):
+        self.group = group
+        self.world = dist.get_world_size(group)
+        self.rank = dist.get_rank(group)
+        E = router_w.shape[0]
+        if E % self.world or gate.E * self.world != E:
+            raise ValueError(f"{E} experts do not split into {self.world} ranks of {gate.E}")
+        self.E, self.e_per_rank, self.k, self.max_tokens = E, gate.E, top_k, max_tokens
+        self.ops = ops if ops is not None else CudaOps(gate, up, down, router_w, router_bias, top_k, shared,
+                                                       max_tokens, self.world)
+
+    def _a2a(self, out, inp, out_split, in_split):
+        dist.all_to_all_single(out, inp, out_split, in_split, group=self.group)
+
+    def forward(self, x):
+        """x: bf16 [T, H] (this rank's tokens, T <= max_tokens) -> y: bf16 [T, H]."""
+        T, H = x.shape
+        k, world = self.k, self.world
+        if T > self.max_tokens:
+            raise ValueError(f"T = {T} exceeds max_tokens = {self.max_tokens}")
+        dev = x.device
+        ids, w = self.ops.route(x)                                     # [T, k] expert ids, weights
+        owner = torch.div(ids, self.e_per_rank, rounding_mode="floor").to(torch.int32)
+        off, order, slot_pos = self.ops.group(owner, world)          # slots by owner; slot -> send position
+        send_counts = (off[1:] - off[:-1]).to(torch.int64)
+        recv_counts = torch.empty_like(send_counts)
+        self._a2a(recv_counts, send_counts, None, None)
+        sc, rc = send_counts.tolist(), recv_counts.tolist()
+        R = int(sum(rc))
+        order_l = order.to(torch.int64)
+        # rows travel as bytes, expert and weight bits as one int32 pair per row
+        send_x = x.index_select(0, torch.div(order_l, k, rounding_mode="floor")).contiguous()
+        meta = torch.stack([ids.view(-1).index_select(0, order_l) - owner.view(-1).index_select(0, order_l)
+                            * self.e_per_rank,
+                            w.view(-1).index_select(0, order_l).view(torch.int32)], dim=1).contiguous()
+        recv_x = torch.empty(R, H, dtype=x.dtype, device=dev)
+        recv_meta = torch.empty(R, 2, dtype=torch.int32, device=dev)
+        self._a2a(recv_x.view(torch.uint8), send_x.view(torch.uint8), rc, sc)
+        self._a2a(recv_meta, meta, rc, sc)
+        er = recv_meta[:, 0].contiguous()
+        wr = recv_meta[:, 1].contiguous().view(torch.float32)
+        y_recv = self.ops.experts(recv_x, er, wr)                    # [R, H], received order
+        y_back = torch.empty(T * k, H, dtype=x.dtype, device=dev)
+        self._a2a(y_back.view(torch.uint8), y_recv.contiguous().view(torch.uint8), sc, rc)
+        return self.ops.combine(y_back, slot_pos, T, self.ops.shared_expert(x))
