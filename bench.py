@@ -278,19 +278,24 @@ def cpu_baseline(wl, moe, x, layer, budget_s=20.0):
 # kernel has changed since is reported as null.
 # DRAM bytes (read + write) of one launch of the dominant kernel, from the launch lists of the bench's own
 # command with `--metrics gpu__time_duration.sum,dram__bytes_read.sum,dram__bytes_write.sum` (profiles/), keyed
-# by workload and by the hash of the GEMM's sources at the time: a later change to the kernel drops the entry
+# by workload and by the hash of the GEMM's code (comments aside) at the time: a later change to the kernel drops the entry
 # (reported as null).
 TRAFFIC = {
-    ("decode_int4_T8", "6b3d2137b6c5e087"): 390216960 + 591616,
-    ("decode_nvfp4_T8", "6b3d2137b6c5e087"): 425606912 + 201216,
+    ("decode_int4_T8", "94e237ba6c42a308"): 390216960 + 591616,
+    ("decode_nvfp4_T8", "94e237ba6c42a308"): 425606912 + 201216,
 }
 
 
 def gemm_source_hash():
+    """Hash of the GEMM's code with comments and blank space removed (a comment edit keeps the kernel)."""
     import hashlib
+    import re
     h = hashlib.sha256()
     for f in ("gemm_tc.cu", "tc_ptx.cuh", "moe_internal.cuh"):
-        h.update(open(os.path.join(ROOT, "weight_only_bit_route_b200", "csrc", f), "rb").read())
+        src = open(os.path.join(ROOT, "weight_only_bit_route_b200", "csrc", f)).read()
+        src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+        src = re.sub(r"//[^\n]*", "", src)
+        h.update(re.sub(r"\s+", "", src).encode())
     return h.hexdigest()[:16]
 
 

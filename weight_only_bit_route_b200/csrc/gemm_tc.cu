@@ -1,19 +1,21 @@
-// Prefill-shaped grouped GEMM on the 5th-generation tensor cores (tcgen05).
+// Grouped GEMM on the 5th-generation tensor cores (tcgen05), every batch size.
 //
 // Per expert e with n_e routed rows, gate/up computes
 //     G = X_e Wg_e^T, U = X_e Wu_e^T, h = bf16(silu(G) * U)      (K = H)
 // and down computes
 //     Y = w * (Hp_e Wd_e^T)                                         (K = F)
-// with the 4-bit weights dequantised inside the kernel
+// with the 4-bit weights turned into MMA operands inside the kernel
 // ("Step-5-Preview-Int4-g128", Recipe; "Step-5-Preview-NVFP4-Local", Format).
 //
 // Tiles are swapped: weights are the M = 128 operand and tokens the N operand,
 // because an expert sees few tokens (about 47 at 2048 tokens).  A tile is
-// (expert, m-tile of 128 weight rows, n-tile of up to 128 (gate/up) or 256
-// (down) rows).  The n-tiles of one m-tile are adjacent in the tile order, so
-// CTAs running side by side share the weight tile through L2.  A persistent
-// CTA per SM walks the tile list, which it builds on the device from
-// expert_offsets.
+// (expert, m-tile of 128 weight rows, n-tile of token rows: up to 64 for
+// gate/up and 128 for down, 128 for "wide" gate/up tiles, 16 for "narrow"
+// decode tiles, 5 tokens on the 8-bit path).  A persistent CTA per SM builds
+// the tile list on the device from expert_offsets; warp 0 takes the CTA's
+// tiles (in a blocked order, or from an atomic counter when the launch hands
+// tiles out dynamically), computes their coordinates once and queues them for
+// the other roles.
 //
 // Warp roles inside a CTA (16 warps):
 //   warp 0      TMA producer of the weight stream: per stage, 2D tensor
@@ -22,49 +24,51 @@
 //               plus the NVFP4 block scales of those rows.  int4 scales are
 //               one bulk copy per tile, since all groups of the tile's rows
 //               are contiguous.
-//   warp 1      producer of the activation operand: per K = 128 stage, two
-//               TMA boxes of the tile's rows x 64 elements, 128-byte swizzled (the
-//               K-major layout the MMA descriptors read); the box height comes
-//               from one of several tensor maps, matching the tile's rows.  The
-//               8-bit int4 path copies its small stages (16 rows x 256 bytes)
-//               with per-lane 16-byte asynchronous copies instead, which do not
-//               queue behind the weight stream in the tensor-copy engine.
+//   warp 1      producer of the activation operand: per stage, TMA boxes of
+//               the tile's rows, 128-byte swizzled (the K-major layout the MMA
+//               descriptors read); the box height comes from one of several
+//               tensor maps, matching the tile's rows (8-bit path: 16 digit
+//               rows per box, and the tile's row records by bulk copy).
 //   warp 2      allocates tensor memory and issues tcgen05.mma from one lane
 //               (8-bit int4: warps 2 and 3 take alternate steps).
-// The three single-issue roles run warp-uniform loops and elect one lane to
-// issue, which keeps the instruction operands in uniform registers.  The MMA
-// pipeline steps in K = 128 (8-bit path: K = 256 for gate/up, 512 for down)
-// and commits once per step, to one barrier of a
-// ring of 16 ("stage done"): a tcgen05.commit costs as much issue time as
-// several MMAs, so every role that waits for a step to finish (the activation
-// producer, the dequantisation warps, the BF16 weight producer, the small-
-// batch epilogue) waits on that one barrier.  No waiter can fall 16 steps
-// behind, which keeps the ring's phases unambiguous.
+// The single-issue roles run warp-uniform loops and elect one lane to issue,
+// which keeps the instruction operands in uniform registers.  The MMA
+// pipeline steps in K = 128 (8-bit path: K = 256 for gate/up, 512 for down;
+// W4A4: 256) and commits once per step, to one barrier of a ring of 16
+// ("stage done"): a tcgen05.commit costs as much issue time as several MMAs,
+// so every role that waits for a step to finish (the activation producer, the
+// dequantisation warps, the BF16 weight producer, the small-batch epilogue)
+// waits on that one barrier.  A parity wait only tells a phase from the one
+// before it: every waiter either sees all phases of a barrier in order or
+// first waits for something that orders it after the previous phase.
 //   warps 4-7   epilogue: tcgen05.ld of the accumulators, SwiGLU or the
 //               routing weight, bf16 stores.  Warp w reads TMEM lanes
 //               32*(w%4) to 32*(w%4)+31.
-//   warps 8-15  dequantisation (4-bit formats).  Each thread owns one weight
-//               row of the tile.  It turns packed weights into bf16 pairs
-//               (int4: q*s rounded once) or f16 pairs (NVFP4: e2m1 * e4m3,
-//               exact) in registers and writes them to tensor memory with
-//               tcgen05.st; the MMA reads its A operand from there.  The
-//               dequantised weights never pass through shared memory.  On
-//               the 8-bit path the warps only unpack nibbles into bytes, in
-//               two groups of four that take alternate weight stages.
+//   warps 8-15  dequantisation (16-bit paths).  Each thread owns one weight
+//               row of the tile.  It turns packed weights into exact f16
+//               pairs in registers (int4: q s 2^k with a power of two per
+//               weight row; NVFP4: e2m1 * e4m3) and writes them to tensor
+//               memory with tcgen05.st; the MMA reads its A operand from
+//               there, so dequantised weights never pass through shared
+//               memory.  On the 8-bit path the warps only unpack nibbles into
+//               bytes, in two groups of four that take alternate weight
+//               stages.  On the W4A4 path warps 8-11 arrange the block scale
+//               factors for tcgen05.cp and the MMA reads both operands from
+//               shared memory.
 // BF16 weights (the shared expert) need no dequantisation: the MMA reads the
 // TMA-staged weight tile from shared memory directly.
 //
-// Tensor memory (512 columns): two accumulator buffers in [0, 256), so the
-// epilogue of one tile overlaps the main loop of the next (buffer b at
-// 128*b; gate/up keeps gate at +0 and up at +64), A stages in [256, 512).
-// The 8-bit path accumulates per step: its small accumulator buffers take
+// Tensor memory (512 columns): accumulator buffers first (two of 128 columns
+// on the 16-bit paths, so the epilogue of one tile overlaps the main loop of
+// the next; gate at +0 and up at +64 or +128), A stages after them.  The
+// 8-bit path accumulates per step: its small accumulator buffers take
 // [0, 128) and the A stages [128, 512).
 //
-// int4 pairs: one mask turns the nibbles (j, j+4) of a packed word into one
-// bf16 pair, so the A operand holds the K elements of each group of 8 in the
-// order 0,4,1,5,2,6,3,7.  The activation operand is stored in the same order,
-// by a pre-pass or by the gate/up epilogue writing h that way.  A dot product
-// does not depend on the order of its terms.
+// int4 words: one mask per nibble pair places the nibbles (j, j+4) of a packed
+// word into one f16 pair, so the A operand holds the K elements of each group
+// of 8 in the order 0,4,1,5,2,6,3,7 (8-bit path: 0,2,4,6,1,3,5,7); the
+// activation pre-pass stores its rows in the same order.  A dot product does
+// not depend on the order of its terms.
 //
 // Every wait is bounded (about 2 s).  On expiry the kernel records
 // MOE_ERR_TIMEOUT and stops issuing work.  It then waits, again bounded, for
