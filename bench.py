@@ -272,14 +272,10 @@ def cpu_baseline(wl, moe, x, layer, budget_s=20.0):
 # measurement
 # ---------------------------------------------------------------------------
 
-# DRAM bytes (read + write) per launch of the dominant kernel, from one-pass ncu
-# captures of that kernel (summarised under profiles/), keyed by workload and by
-# a hash of the GEMM's sources at the time of the capture: a figure whose
-# kernel has changed since is reported as null.
 # DRAM bytes (read + write) of one launch of the dominant kernel, from the launch lists of the bench's own
-# command with `--metrics gpu__time_duration.sum,dram__bytes_read.sum,dram__bytes_write.sum` (profiles/), keyed
-# by workload and by the hash of the GEMM's code (comments aside) at the time: a later change to the kernel drops the entry
-# (reported as null).
+# command with `--metrics gpu__time_duration.sum,dram__bytes_read.sum,dram__bytes_write.sum` (summarised under
+# profiles/), keyed by workload and by the hash of the GEMM's code (comments aside) at the time of the capture:
+# a figure whose kernel has changed since is reported as null.
 TRAFFIC = {
     ("decode_int4_T8", "94e237ba6c42a308"): 390216960 + 591616,
     ("decode_nvfp4_T8", "94e237ba6c42a308"): 425606912 + 201216,
