@@ -133,3 +133,27 @@ def test_expert_parallel_two_ranks_gloo():
     for rank, same, within, _ in got:
         assert same, f"rank {rank}: the expert-parallel result differs from the one-process composition"
         assert within, f"rank {rank}: outside the layer tolerance of the oracle"
+
+
+def test_expert_parallel_argument_checks():
+    """Experts that do not split evenly over the ranks, and batches above max_tokens, are refused."""
+    import torch.distributed as dist
+    from weight_only_bit_route_b200 import ep
+
+    class _Bank:
+        def __init__(self, E):
+            self.E = E
+
+    class _Ops:
+        pass
+
+    dist.init_process_group("gloo", rank=0, world_size=1, init_method=f"tcp://127.0.0.1:{_free_port()}")
+    try:
+        router_w = torch.zeros(8, 128)
+        with pytest.raises(ValueError):
+            ep.ExpertParallelMoE(_Bank(4), _Bank(4), _Bank(4), router_w, top_k=2, ops=_Ops())
+        layer = ep.ExpertParallelMoE(_Bank(8), _Bank(8), _Bank(8), router_w, top_k=2, max_tokens=4, ops=_Ops())
+        with pytest.raises(ValueError):
+            layer.forward(torch.zeros(5, 128, dtype=torch.bfloat16))
+    finally:
+        dist.destroy_process_group()
