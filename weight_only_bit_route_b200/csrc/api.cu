@@ -75,7 +75,8 @@ int run_problem(const GemvProblem& p, bool gateup, int rows, int act_rows, void*
 // The step-level calls' scratch: the GEMV or GEMM pre-pass of rows rows, then
 // the shared expert's split-K partial sums.
 // GEMM pre-pass layout in a scratch region of gemm_prep_bytes(rows, in_dim):
-// row scales [rows], group sums [rows][in / 128] (8-bit int4), gathered rows.
+// row scales [rows], row records [rows][zrow_floats(in_dim)] (8-bit int4),
+// gathered rows.
 GemmBuffers gemm_buffers(void* base, int rows, int in_dim, bool act_ready, bool i8) {
     uint8_t* p = reinterpret_cast<uint8_t*>(base);
     GemmBuffers b{};
