@@ -1,6 +1,6 @@
-"""Expert-parallel layer (weight_only_bit_route_b200/ep.py) on two CPU ranks over gloo.
+"""Expert-parallel layer (weight_only_bit_route_b200/ep.py) on two and four CPU ranks over gloo.
 
-Each rank owns half of the routed experts and routes its own tokens; the steps run in the oracle (an injected
+Each rank owns an equal share of the routed experts and routes its own tokens; the steps run in the oracle (an injected
 step set: the collectives and the bookkeeping around them are what is tested here, the steps' kernels are
 tested on the GPU).  Bars: each rank's output is bit-identical to the same steps run on one process with every
 expert local, and within the layer tolerance of the oracle's fp64 layer.
@@ -77,7 +77,7 @@ class RefOps:
         return _from_bits(_to_bf16(self.o.combine(_bits(y_back), slot_pos.numpy(), T, self.k, sh)))
 
 
-def _worker(rank, world, port, results):
+def _worker(rank, world, counts, port, results):
     import sys
     root = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
     sys.path[:0] = [root, os.path.join(root, "tests")]
@@ -91,7 +91,7 @@ def _worker(rank, world, port, results):
     try:
         wl = syn.WORKLOADS[0]
         P = build(0, "random", experts=list(range(wl.E)), shared=True)
-        x = _from_bits(syn.gen_x(wl, seed=100 + rank, T=13 if rank else 16))    # ragged: 16 and 13 tokens
+        x = _from_bits(syn.gen_x(wl, seed=100 + rank, T=counts[rank]))
         e_per = wl.E // world
         ops = RefOps(oracle, P, rank * e_per, (rank + 1) * e_per)
         layer = ep.ExpertParallelMoE(ops.banks["gate"], ops.banks["up"], ops.banks["down"], P.Wr, top_k=wl.k,
@@ -101,6 +101,7 @@ def _worker(rank, world, port, results):
         full = RefOps(oracle, P, 0, wl.E)
         ids, w = full.route(x)
         T = x.shape[0]
+        assert y.shape == (T, wl.H)
         off, rs, sr = full.group(torch.zeros(T, wl.k, dtype=torch.int32), 1)
         ys = full.experts(x.index_select(0, rs.to(torch.int64) // wl.k), ids.view(-1)[rs.to(torch.int64)],
                           w.view(-1)[rs.to(torch.int64)])
@@ -108,17 +109,20 @@ def _worker(rank, world, port, results):
         ref = oracle.moe_forward(_bits(x), ids.numpy(), w.numpy(), P.banks["gate"], P.banks["up"], P.banks["down"],
                                  shared=P.shared)
         got = oracle.bf16_to_f32(y).astype(np.float64)
-        ok_tol = bool(np.all(np.abs(got - ref) <= layer_tolerance(ref)))
+        ok_tol = T == 0 or bool(np.all(np.abs(got - ref) <= layer_tolerance(ref)))
         results.put((rank, bool(np.array_equal(y, y1)), ok_tol, int(T)))
     finally:
         dist.destroy_process_group()
 
 
-def test_expert_parallel_two_ranks_gloo():
+@pytest.mark.parametrize("counts", [(16, 13), (16, 13, 0, 5)], ids=["two_ranks_ragged", "four_ranks_one_empty"])
+def test_expert_parallel_gloo(counts):
+    """Ragged token counts; on four ranks one rank has no tokens and still takes part in every exchange."""
+    world = len(counts)
     ctx = mp.get_context("spawn")
     results = ctx.Queue()
     port = _free_port()
-    procs = [ctx.Process(target=_worker, args=(r, 2, port, results)) for r in range(2)]
+    procs = [ctx.Process(target=_worker, args=(r, world, counts, port, results)) for r in range(world)]
     for p in procs:
         p.start()
     for p in procs:
@@ -127,9 +131,9 @@ def test_expert_parallel_two_ranks_gloo():
     for p in procs:
         if p.is_alive():
             p.kill()
-    assert codes == [0, 0], f"rank exit codes {codes}"
-    got = sorted(results.get(timeout=5) for _ in range(2))
-    assert [g[3] for g in got] == [16, 13]
+    assert codes == [0] * world, f"rank exit codes {codes}"
+    got = sorted(results.get(timeout=5) for _ in range(world))
+    assert [g[3] for g in got] == list(counts)
     for rank, same, within, _ in got:
         assert same, f"rank {rank}: the expert-parallel result differs from the one-process composition"
         assert within, f"rank {rank}: outside the layer tolerance of the oracle"
