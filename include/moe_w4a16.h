@@ -170,7 +170,9 @@ const char* moe_status_string(int status);
 
 /* Number of kernels this library has launched in this process since it was
  * loaded (a host-side count of successful launch calls, over every stream
- * and device).  For measurement; no part of the layer's arithmetic. */
+ * and device).  Launches recorded by moe_layer_graph_create are not counted;
+ * each moe_layer_graph_launch adds the graph's kernels.  For measurement; no
+ * part of the layer's arithmetic. */
 uint64_t moe_launch_count(void);
 
 /* ---------------------------------------------------------------------- */

@@ -288,8 +288,12 @@ int layer_run(const void* x, int T, const moe_layer* L, void* y, void* ws, cudaS
 namespace moe {
 namespace {
 std::atomic<uint64_t> g_launches{0};
+thread_local uint64_t t_launches = 0;      // this thread's share, so a recording can take back its own
 }
-void count_launch() { g_launches.fetch_add(1, std::memory_order_relaxed); }
+void count_launch() {
+    g_launches.fetch_add(1, std::memory_order_relaxed);
+    t_launches++;
+}
 }  // namespace moe
 
 extern "C" {
@@ -496,6 +500,7 @@ int moe_layer_graph_create(const void* x, int T, const moe_layer* L, void* y, vo
     }
     cudaStream_t cap = nullptr;
     if (cudaStreamCreateWithFlags(&cap, cudaStreamNonBlocking) != cudaSuccess) return MOE_ERR_CUDA;
+    const uint64_t counted_before = moe::t_launches;
     cudaGraph_t graph = nullptr;
     int rc = MOE_OK;
     if (cudaStreamBeginCapture(cap, cudaStreamCaptureModeRelaxed) != cudaSuccess) {
@@ -521,13 +526,15 @@ int moe_layer_graph_create(const void* x, int T, const moe_layer* L, void* y, vo
     }
     if (graph) cudaGraphDestroy(graph);
     cudaStreamDestroy(cap);
-    // the launches recorded above ran nothing: they are counted when the graph is launched
+    // the launches recorded above ran nothing, whether or not the recording succeeded: take them back (the
+    // graph's kernels are counted when it is launched)
+    moe::g_launches.fetch_sub(moe::t_launches - counted_before, std::memory_order_relaxed);
+    moe::t_launches = counted_before;
     if (rc != MOE_OK) {
         cudaGetLastError();
         delete g;
         return rc;
     }
-    moe::g_launches.fetch_sub(g->kernels, std::memory_order_relaxed);
     *out = g;
     return MOE_OK;
 }
