@@ -5,6 +5,7 @@ step set: the collectives and the bookkeeping around them are what is tested her
 tested on the GPU).  Bars: each rank's output is bit-identical to the same steps run on one process with every
 expert local, and within the layer tolerance of the oracle's fp64 layer.
 """
+import datetime
 import os
 import socket
 
@@ -137,6 +138,115 @@ def test_expert_parallel_gloo(counts):
     for rank, same, within, _ in got:
         assert same, f"rank {rank}: the expert-parallel result differs from the one-process composition"
         assert within, f"rank {rank}: outside the layer tolerance of the oracle"
+
+
+def _refusal_worker(rank, world, port, results):
+    import sys
+    root = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+    sys.path[:0] = [root, os.path.join(root, "tests")]
+    import torch.distributed as dist
+    import oracle
+    from problems import build
+    from weight_only_bit_route_b200 import ep
+    from weight_only_bit_route_b200 import synthetic as syn
+
+    dist.init_process_group("gloo", rank=rank, world_size=world, init_method=f"tcp://127.0.0.1:{port}",
+                            timeout=datetime.timedelta(seconds=60))
+    try:
+        wl = syn.WORKLOADS[0]
+        P = build(0, "random", experts=list(range(wl.E)), shared=False)
+        e_per = wl.E // world
+        ops = RefOps(oracle, P, rank * e_per, (rank + 1) * e_per)
+        layer = ep.ExpertParallelMoE(ops.banks["gate"], ops.banks["up"], ops.banks["down"], P.Wr, top_k=wl.k,
+                                     max_tokens=8, ops=ops)
+        # rank 1's batch is one token too many: both ranks must raise, neither may wait for the other
+        x = _from_bits(syn.gen_x(wl, seed=200 + rank, T=9 if rank == 1 else 4))
+        try:
+            layer.forward(x)
+            raised = ""
+        except ValueError as e:
+            raised = str(e)
+        # the group is still in step: a valid call afterwards completes on both ranks
+        y = layer.forward(x[:3].contiguous())
+        results.put((rank, raised, tuple(y.shape)))
+    finally:
+        dist.destroy_process_group()
+
+
+def test_expert_parallel_refusal_reaches_every_rank():
+    """A batch above max_tokens on one rank makes every rank raise ValueError after the counts' exchange (no rank
+    is left in a collective), and the next call runs normally."""
+    ctx = mp.get_context("spawn")
+    results = ctx.Queue()
+    port = _free_port()
+    procs = [ctx.Process(target=_refusal_worker, args=(r, 2, port, results)) for r in range(2)]
+    for p in procs:
+        p.start()
+    for p in procs:
+        p.join(timeout=300)
+    codes = [p.exitcode for p in procs]
+    for p in procs:
+        if p.is_alive():
+            p.kill()
+    assert codes == [0, 0], f"rank exit codes {codes}"
+    got = sorted(results.get(timeout=5) for _ in range(2))
+    assert "refused" in got[0][1], got[0]
+    assert "exceeds max_tokens" in got[1][1], got[1]
+    assert [g[2] for g in got] == [(3, 1024), (3, 1024)]
+
+
+def _leaver_worker(rank, world, port, results):
+    import sys
+    import time
+    root = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+    sys.path[:0] = [root, os.path.join(root, "tests")]
+    import torch.distributed as dist
+    import oracle
+    from problems import build
+    from weight_only_bit_route_b200 import ep
+    from weight_only_bit_route_b200 import synthetic as syn
+
+    dist.init_process_group("gloo", rank=rank, world_size=world, init_method=f"tcp://127.0.0.1:{port}",
+                            timeout=datetime.timedelta(seconds=10))
+    if rank == 1:
+        # this rank leaves between calls, with nothing in flight
+        dist.destroy_process_group()
+        return
+    wl = syn.WORKLOADS[0]
+    P = build(0, "random", experts=list(range(wl.E)), shared=False)
+    e_per = wl.E // world
+    ops = RefOps(oracle, P, 0, e_per)
+    layer = ep.ExpertParallelMoE(ops.banks["gate"], ops.banks["up"], ops.banks["down"], P.Wr, top_k=wl.k,
+                                 max_tokens=8, ops=ops)
+    t0 = time.monotonic()
+    try:
+        layer.forward(_from_bits(syn.gen_x(wl, seed=300, T=4)))
+        err = ""
+    except Exception as e:                  # the backend's error type differs between versions
+        err = type(e).__name__
+    results.put((rank, err, time.monotonic() - t0))
+
+
+def test_expert_parallel_rank_that_left():
+    """A rank that leaves the group between calls: the other rank's next call ends with an error from its first
+    collective, within the group's timeout, instead of waiting for ever."""
+    ctx = mp.get_context("spawn")
+    results = ctx.Queue()
+    port = _free_port()
+    procs = [ctx.Process(target=_leaver_worker, args=(r, 2, port, results)) for r in range(2)]
+    for p in procs:
+        p.start()
+    for p in procs:
+        p.join(timeout=120)
+    codes = [p.exitcode for p in procs]
+    for p in procs:
+        if p.is_alive():
+            p.kill()
+    assert codes == [0, 0], f"rank exit codes {codes}"
+    rank, err, secs = results.get(timeout=5)
+    assert rank == 0 and err, "the remaining rank's call did not fail"
+    assert err != "ValueError", "the call failed before its first collective"
+    assert secs < 60
 
 
 def test_expert_parallel_argument_checks():

@@ -21,7 +21,9 @@ rows cross the fabric once each way, and no multicast of any kind is used.  Each
 which other rows share its tile, so on one rank the layer reproduces moe_layer_decode bit for bit.
 
 The split sizes of an all-to-all are host values, so each call reads the per-rank slot counts back to the host
-once (after step 2) and the returned counts once (after the counts' exchange).
+once (after step 2) and the returned counts once (after the counts' exchange).  A rank whose batch is above
+max_tokens still takes part in the counts' exchange (with counts of -1), and then every rank raises ValueError, so
+an oversized batch on one rank ends the call on all of them instead of leaving the others in a collective.
 """
 import torch
 import torch.distributed as dist
@@ -103,16 +105,24 @@ class ExpertParallelMoE:
         """x: bf16 [T, H] (this rank's tokens, T <= max_tokens) -> y: bf16 [T, H]."""
         T, H = x.shape
         k, world = self.k, self.world
-        if T > self.max_tokens:
-            raise ValueError(f"T = {T} exceeds max_tokens = {self.max_tokens}")
         dev = x.device
-        ids, w = self.ops.route(x)                                     # [T, k] expert ids, weights
-        owner = torch.div(ids, self.e_per_rank, rounding_mode="floor").to(torch.int32)
-        off, order, slot_pos = self.ops.group(owner, world)          # slots by owner; slot -> send position
-        send_counts = (off[1:] - off[:-1]).to(torch.int64)
+        # A batch above max_tokens is refused on every rank: the refusing rank sends counts of -1 in the counts'
+        # exchange (which every rank takes), and every rank raises after it, so none is left waiting for a peer.
+        refused = T > self.max_tokens
+        if refused:
+            send_counts = torch.full((world,), -1, dtype=torch.int64, device=dev)
+        else:
+            ids, w = self.ops.route(x)                                 # [T, k] expert ids, weights
+            owner = torch.div(ids, self.e_per_rank, rounding_mode="floor").to(torch.int32)
+            off, order, slot_pos = self.ops.group(owner, world)      # slots by owner; slot -> send position
+            send_counts = (off[1:] - off[:-1]).to(torch.int64)
         recv_counts = torch.empty_like(send_counts)
         self._a2a(recv_counts, send_counts, None, None)
         sc, rc = send_counts.tolist(), recv_counts.tolist()
+        if refused:
+            raise ValueError(f"T = {T} exceeds max_tokens = {self.max_tokens}")
+        if min(rc) < 0:
+            raise ValueError(f"rank(s) {[r for r in range(world) if rc[r] < 0]} refused a batch above max_tokens")
         R = int(sum(rc))
         order_l = order.to(torch.int64)
         # rows travel as bytes, expert and weight bits as one int32 pair per row
