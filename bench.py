@@ -265,7 +265,29 @@ def cpu_baseline(wl, moe, x, layer, budget_s=20.0):
     cores = len(os.sched_getaffinity(0)) if hasattr(os, "sched_getaffinity") else os.cpu_count()
     return {"value": round(done / dt, 3), "unit": UNIT, "cores": cores, "kind": "oracle",
             "sample": f"first {n} of the workload's {T} tokens, router -> combine (oracle fp64 layer, "
-                      f"OpenMP on {cores} threads), {passes} passes, {dt:.2f} s"}
+                      f"OpenMP on {cores} threads), {passes} passes, {dt:.2f} s",
+            "single_thread": oracle_single_thread(oracle, sample[:1], Wr, bias, wl.k, (gate, up, down), sh,
+                                                  min(8.0, budget_s / 2)),
+            "host_threads": os.cpu_count()}
+
+
+def oracle_single_thread(oracle, sample, Wr, bias, k, banks, sh, budget_s):
+    """The oracle's layer forward on one OpenMP thread: passes over a one-token sample until budget_s has gone."""
+    oracle.set_threads(1)
+    try:
+        passes = 0
+        t0 = time.perf_counter()
+        while True:
+            ids, w = oracle.route(sample, Wr, bias, k)
+            oracle.moe_forward(sample, ids, w, *banks, shared=sh)
+            passes += 1
+            dt = time.perf_counter() - t0
+            if dt >= budget_s:
+                break
+    finally:
+        oracle.set_threads(0)
+    return {"value": round(passes * sample.shape[0] / dt, 3), "unit": UNIT, "cores": 1,
+            "sample": f"{sample.shape[0]} token, router -> combine on one thread, {passes} passes, {dt:.2f} s"}
 
 
 # ---------------------------------------------------------------------------
@@ -632,7 +654,9 @@ def run_reference(args, wl, rank, world):
     value = n / (ms * 1e-3)
     cores = len(os.sched_getaffinity(0)) if hasattr(os, "sched_getaffinity") else os.cpu_count()
     cb = {"value": round(value, 3), "unit": UNIT, "cores": cores, "kind": "oracle",
-          "sample": f"{n} of the workload's {wl.T} tokens per step, router -> combine, OpenMP on {cores} threads"}
+          "sample": f"{n} of the workload's {wl.T} tokens per step, router -> combine, OpenMP on {cores} threads",
+          "single_thread": oracle_single_thread(oracle, sample[:1], Wr, bias, wl.k, banks, sh, 5.0),
+          "host_threads": os.cpu_count()}
     print(json.dumps({
         "impl": "reference", "metric": METRIC, "value": round(value, 3), "unit": UNIT, "n_gpus": world,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms, 3), "higher_is_better": True,

@@ -35,6 +35,8 @@ def lib():
         L.oracle_f16_to_f32.restype = F
         L.oracle_set_x_f16.argtypes = [I]
         L.oracle_set_x_f16.restype = None
+        L.oracle_set_threads.argtypes = [I]
+        L.oracle_set_threads.restype = I
         L.oracle_e2m1_decode.argtypes = [ctypes.c_uint8]
         L.oracle_e2m1_decode.restype = F
         L.oracle_e2m1_encode.argtypes = [F]
@@ -143,6 +145,12 @@ class x_f16:
 
     def __exit__(self, *a):
         lib().oracle_set_x_f16(0)
+
+
+def set_threads(n):
+    """OpenMP threads of later oracle calls (n <= 0: one per host core); returns the count in effect.
+    For timing only: results do not depend on it."""
+    return int(lib().oracle_set_threads(int(n)))
 
 
 def f32_to_bf16_scalar(v):

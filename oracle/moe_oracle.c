@@ -64,6 +64,9 @@
 #include <stdint.h>
 #include <stdlib.h>
 #include <string.h>
+#ifdef _OPENMP
+#include <omp.h>
+#endif
 
 /* ------------------------------------------------------------------------ */
 /* bf16 <-> fp32                                                             */
@@ -92,6 +95,21 @@ float oracle_f16_to_f32(uint16_t h) {
  * BF16 shared expert computes in bf16, so it reads x rounded to bf16. */
 static int g_x_f16 = 0;
 void oracle_set_x_f16(int on) { g_x_f16 = on; }
+
+/* Thread control for timing, no part of the arithmetic: every parallel loop
+ * here gives each item (a row, an expert, a group) to one thread and no loop
+ * reduces across threads, so results do not depend on the count.  n > 0 sets
+ * the OpenMP thread count of later calls, n <= 0 restores one thread per host
+ * core; returns the count in effect. */
+int oracle_set_threads(int n) {
+#ifdef _OPENMP
+    omp_set_num_threads(n > 0 ? n : omp_get_num_procs());
+    return omp_get_max_threads();
+#else
+    (void)n;
+    return 1;
+#endif
+}
 static float x_to_f32(uint16_t v);
 
 /* Round-to-nearest-even to bf16 (finite inputs). */

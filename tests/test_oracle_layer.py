@@ -191,6 +191,24 @@ def test_layer_token_independence():
     assert not np.array_equal(y2[t0 + 1:], y[t0 + 1:])
 
 
+def test_layer_thread_count_independence():
+    """The thread count is timing control only: one thread and one per host core give bit-identical scores, ids,
+    weights and layer outputs (each parallel item is computed by one thread, and no loop reduces across threads)."""
+    wl = syn.WORKLOADS[0]
+    x, Wr, banks, sh = _tiny_problem(wl, "nvfp4", True)
+    outs = []
+    try:
+        for n in (1, 0):
+            oracle.set_threads(n)
+            ids, w, sc = oracle.route(x, Wr, None, 8, want_scores=True)
+            y = oracle.moe_forward(x, ids, w, banks["gate"], banks["up"], banks["down"], shared=sh)
+            outs.append((ids, w, sc, y))
+    finally:
+        oracle.set_threads(0)
+    for a, b in zip(*outs):
+        assert np.array_equal(a, b)
+
+
 def test_zipf_workload_histogram():
     """The skewed workload leaves some experts empty and a few with > 1500 rows
     at T = 8192 (checked on the full token set)."""
