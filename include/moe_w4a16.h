@@ -215,9 +215,9 @@ int moe_permute(const int32_t* topk_ids, int T, int top_k, int E,
  * inside another runtime's fixed memory plan (an engine that reserves the GPU's
  * memory up front and hands out no extra buffers), or cannot afford the
  * device-wide synchronisation that an allocation can cause in the middle of a
- * step; they cannot supply the workspace moe_permute needs.  This call computes exactly what moe_permute
- * computes (same arguments and outputs, minus the workspace) and allocates
- * nothing: its scratch is a file-scope device array of about 64 KB that every
+ * step; they cannot supply the workspace moe_permute needs.  This call
+ * computes exactly what moe_permute computes (same arguments and outputs,
+ * minus the workspace) and allocates nothing: its scratch is a file-scope device array of about 64 KB that every
  * GPU loading the library keeps until the process exits.
  * Limits: T*top_k <= 65536 and E <= 1024; larger sizes return
  * MOE_ERR_UNSUPPORTED.  The first call on a device looks up the array's device
@@ -227,7 +227,7 @@ int moe_permute(const int32_t* topk_ids, int T, int top_k, int E,
  * between them) race.  An expert id outside [0, E) is dropped and its slot_row
  * entry is -1; that condition is not reported (no caller can read the static
  * array's status word), and row_slot past expert_offsets[E] is left
- * unwritten.  The paper has no counterpart to this call. */
+ * unwritten.  The model pages describe no counterpart to this call. */
 int moe_permute_noalloc(const int32_t* topk_ids, int T, int top_k, int E,
                         int32_t* expert_offsets, int32_t* row_slot, int32_t* slot_row,
                         moe_stream_t stream);
