@@ -83,6 +83,24 @@ def test_layer_argument_errors():
     assert L.moe_layer_decode(None, 8, ctypes.byref(_layer()), FAKE, FAKE, 1 << 34, None) == -1
 
 
+def test_layer_graph_argument_errors():
+    """The recorded layer's calls refuse bad arguments before any CUDA call, and leave the handle empty."""
+    L = moe.lib
+    h = P(0x1234)
+
+    def create(lay, T=8, ws=FAKE, wsb=1 << 34, out=True):
+        h.value = 0x1234
+        return L.moe_layer_graph_create(FAKE, T, ctypes.byref(lay), FAKE, ws, wsb, ctypes.byref(h) if out else None)
+
+    assert create(_layer(), out=False) == -1
+    assert create(_layer(), T=0) == -1 and not h.value                 # nothing to record
+    assert create(_layer(swiglu_limit=7.0)) == -2 and not h.value
+    assert create(_layer(gate=_bank(0, 351, 1536, 4096))) == -1 and not h.value
+    assert create(_layer(), ws=None) == -5 and not h.value
+    assert L.moe_layer_graph_launch(None, None) == -1
+    assert L.moe_layer_graph_destroy(None) == 0
+
+
 def test_step_argument_errors():
     L = moe.lib
     g = _bank(0, 352, 1536, 4096)
