@@ -618,8 +618,6 @@ def run_reference(args, wl, rank, world):
     ids, w = oracle.route(sample, Wr, bias, wl.k)
     experts = sorted(set(ids.ravel().tolist()))
 
-    class _W:
-        pass
     fmt = oracle.FMT_INT4 if wl.fmt == "int4" else oracle.FMT_NVFP4
     banks = []
     for which in ("gate", "up", "down"):
@@ -642,8 +640,9 @@ def run_reference(args, wl, rank, world):
     sh = None
     if wl.shared:
         sh = tuple(oracle.Bank(oracle.FMT_BF16, syn.gen_shared(wl, w)[None]) for w in ("gate", "up", "down"))
-    for _ in range(args.warmup):
-        pass   # the oracle has no warm-up state; skip untimed passes to bound the run time
+    for _ in range(args.warmup):                     # untimed passes of the same sample
+        ids, w = oracle.route(sample, Wr, bias, wl.k)
+        oracle.moe_forward(sample, ids, w, *banks, shared=sh)
     times = []
     for _ in range(args.steps):
         t0 = time.perf_counter()
