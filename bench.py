@@ -25,7 +25,6 @@ over ranks and `value` sums all ranks' tokens.
 import argparse
 import json
 import os
-import subprocess
 import sys
 import time
 

@@ -3,8 +3,6 @@ and rejects bad arguments on the host before launching anything (no GPU
 needed: every call below returns during argument validation)."""
 import ctypes
 
-import pytest
-
 from weight_only_bit_route_b200 import moe
 
 P = ctypes.c_void_p

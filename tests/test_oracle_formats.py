@@ -9,7 +9,6 @@ Recipe).
 import math
 
 import numpy as np
-import pytest
 import torch
 
 import oracle

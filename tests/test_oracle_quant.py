@@ -9,7 +9,6 @@ quantiser's output; independent decoder).
 import os
 
 import numpy as np
-import pytest
 import torch
 
 import oracle
