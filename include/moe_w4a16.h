@@ -307,18 +307,23 @@ int moe_layer_decode(const void* x, int T, const moe_layer* L, void* y,
                      void* ws, size_t ws_bytes, moe_stream_t stream);
 
 /* The whole layer for any T >= 1 (prefill-sized batches use the tcgen05
- * grouped GEMM).  Same arguments and result as moe_layer_decode. */
+ * grouped GEMM; "Step-5-Preview-Spark", Serving on 4 x DGX Spark, which
+ * reports prefill and decode separately).  Same arguments and result as
+ * moe_layer_decode; T = 0 does nothing and returns 0. */
 int moe_layer_forward(const void* x, int T, const moe_layer* L, void* y,
                       void* ws, size_t ws_bytes, moe_stream_t stream);
 
-/* A layer call recorded once as a CUDA graph and replayed: the same kernels
+/* A layer call recorded once as a CUDA graph and replayed (no page has a
+ * counterpart: it removes the host's launch work from a decode step, which
+ * on this path is a large share of the layer's time): the same kernels
  * as moe_layer_forward(x, T, L, y, ws, ws_bytes, .) with these exact
  * pointers, without the host's per-call launch work (argument checks, tensor
  * map encoding, about ten kernel launches).  The graph reads x and the banks
  * and writes y and ws at every launch, so the caller refills x in place
  * between launches and keeps every buffer (and the banks' contents, which may
  * change) alive until moe_layer_graph_destroy.  One launch at a time per
- * workspace.  create: checks as moe_layer_forward, records on a private
+ * workspace.  create: checks as moe_layer_forward and refuses T = 0 (nothing
+ * to record), records on a private
  * stream (the caller's stream is not touched), returns the handle in *out
  * (NULL on error).  launch: enqueues one layer on `stream`.  The recording
  * uses the per-device side stream of the shared expert, so create must not
@@ -381,8 +386,8 @@ int moe_quantize_nvfp4(const void* w, int64_t rows, int64_t cols, uint8_t* packe
  * Requirements: R % 16 == 0, C even, R * C < 2^24, 1 <= E <= 1024. */
 
 /* Expand CSF planes into scale bytes u8 [E, R, C] (scales, out), e.g. one
- * layer's scales into scratch before the layer runs ("The b12x loader ...
- * expands one MoE layer's scales into shared scratch", Size).  expert_offsets:
+ * layer's scales into scratch before the layer runs, which is how the page's
+ * loader uses the format ("Step-5-Preview-NVFP4-Local", Size).  expert_offsets:
  * int32 [E+1] of a routing (moe_permute), or NULL; when given, only experts
  * with at least one routed row are expanded and the other experts' bytes are
  * left as they were.  exceptions and starts are both given or both NULL (no
@@ -395,7 +400,9 @@ int moe_csf_decode(const uint8_t* fixed, const uint32_t* exceptions, const int64
 /* Workspace bytes moe_csf_encode needs for E experts of R rows (0 if invalid). */
 size_t moe_csf_encode_workspace_bytes(int E, int R);
 
-/* Encode scale bytes u8 [E, R, C] into CSF (offline step).  Always writes
+/* Encode scale bytes u8 [E, R, C] into CSF ("Step-5-Preview-NVFP4-Local",
+ * Format: per 16 rows a slab of row bases and 4-bit codes, exceptions where
+ * a byte is not base + code; an offline step).  Always writes
  * fixed and starts (device memory); with exceptions non-NULL it also writes
  * the exceptions, at most exceptions_capacity of them (a larger count records
  * MOE_ERR_DEVICE_INDEX in the workspace status word).  To size the
