@@ -377,12 +377,14 @@ int moe_quantize_nvfp4(const void* w, int64_t rows, int64_t cols, uint8_t* packe
  *   fixed       u8 [E, R/16, 16 * (1 + C/2)]: per slab of 16 rows the 16 row
  *               bases, then each row's 4-bit codes (C/2 bytes per row, in row
  *               order; column 2j in the low nibble of byte j);
- *   exceptions  u32 [n]: (row * C + col) | byte << 24, grouped by expert and
- *               row-major within an expert (row counts from 0 in each expert);
- *   starts      i64 [E + 1]: expert e owns exceptions[starts[e], starts[e+1]).
- * A byte is its row's base plus its code unless an exception replaces it.  A
- * row's base is the lowest value 0..240 whose window [base, base + 15] holds
- * the most of the row's bytes; the code at an exception's position is 0.
+ *   exceptions  u32 [n]: (row * C + col) | byte << 24 (row counts from 0 in
+ *               each expert); expert 0's entries first, then expert 1's and
+ *               so on, each expert's in increasing position;
+ *   starts      i64 [E + 1]: expert e's entries are exceptions[starts[e],
+ *               starts[e+1]).
+ * Decoding: byte = base(row) + code, or the stored byte of an exception.  A
+ * row's base is the smallest b in 0..240 that puts the largest number of the
+ * row's bytes inside [b, b + 15]; the code stored under an exception is 0.
  * Requirements: R % 16 == 0, C even, R * C < 2^24, 1 <= E <= 1024. */
 
 /* Expand CSF planes into scale bytes u8 [E, R, C] (scales, out), e.g. one

@@ -15,16 +15,18 @@
  *           Format (one E4M3 byte per 16 weights, [E, R, C]; dequant =
  *           E2M1 value x E4M3 block scale x weight_scale_2; nibble order
  *           "low nibble first" stated there for the CSF codes).
- *   [Spark] "Step-5-Preview-Spark": At a glance (hidden 4096, 352 routed
- *           experts, top-8, sigmoid router, 1 shared expert).
+ *   [Spark] "Step-5-Preview-Spark": At a glance (hidden 4096; a sigmoid
+ *           router keeps 8 of 352 routed experts; one shared expert).
  *   [Art]   "Step 5 Preview: 92 narrow layers, and a sparse indexer that scores
- *           blocks of 8": The shape (8 routed experts per token plus one shared
- *           expert, each a SwiGLU of width 1536).
+ *           blocks of 8": The shape (each token goes to 8 routed SwiGLU experts
+ *           and to a shared one, all of width 1536).
  *   [CSF]   "Step-5-Preview-NVFP4-Local", Format (the compressed scale format:
- *           per 16-row slab 16 row bases then 4-bit codes, low nibble first;
- *           exceptions (row*C + col) | byte << 24 grouped by expert, row-major;
- *           starts [E+1]; a row's base is the lowest value whose 16-value
- *           window covers the most of its bytes, 0..240) and Size.
+ *           each slab of 16 rows holds their 16 bases and then their 4-bit
+ *           codes, the lower nibble of a byte first; exceptions are
+ *           (row*C + col) | byte << 24, expert by expert in increasing
+ *           position; starts [E+1]; a row's base, in 0..240, is the start of
+ *           the 16-value window holding the largest share of its bytes) and
+ *           Size.
  *
  * Readings where the pages are silent (each listed in the design notes):
  *   - int4: divisor 7 with clamp [-8, 7]; ratios r_i = (24 + i) / 40, i = 0..16;
@@ -197,7 +199,7 @@ uint8_t oracle_e4m3_encode_nonneg(float v) {
 #define I4_GROUP 128
 #define I4_NRATIO 17
 
-/* The 17 evenly spaced clip ratios in [0.60, 1.00]: (24 + i) / 40. */
+/* Clip ratio i of the search, i = 0..16: (24 + i) / 40, evenly spaced from 0.60 to 1.00. */
 static float clip_ratio(int i) { return (float)(24 + i) / 40.0f; }
 
 static int32_t rne_clamp_q(float w, float s) {
@@ -630,8 +632,8 @@ void oracle_combine(const uint16_t* y_perm, const int32_t* slot_row, int64_t T, 
 /* Compressed scale format (CSF)  [CSF] Format                               */
 /* ------------------------------------------------------------------------ */
 
-/* Base of one row of n scale bytes: the lowest b in 0..240 whose window
- * [b, b + 15] holds the most of the row's bytes. */
+/* Base of one row of n scale bytes: the smallest b in 0..240 that puts the
+ * largest number of the row's bytes inside [b, b + 15]. */
 static int csf_row_base(const uint8_t* row, int64_t n) {
     int64_t hist[256];
     memset(hist, 0, sizeof(hist));
@@ -650,7 +652,7 @@ static int csf_row_base(const uint8_t* row, int64_t n) {
  * fixed: u8 [E, R/16, 16 * (1 + C/2)]: per slab of 16 rows, the 16 row bases,
  *        then the rows' codes in row order, C/2 bytes each, column 2j in the
  *        low nibble of byte j and column 2j + 1 in its high nibble;
- * starts: int64 [E + 1], expert e owns exceptions[starts[e] .. starts[e+1]);
+ * starts: int64 [E + 1], expert e's entries are exceptions[starts[e] .. starts[e+1]);
  * exceptions: uint32 [n] (may be NULL to count only), (row * C + col) | byte << 24
  *        for every byte outside its row's window, in (expert, row, col) order.
  * Returns n, the number of exceptions. */

@@ -4,8 +4,8 @@ Bars: bit-exact for integer work (routing ids outside near ties, the
 permutation, quantised codes and scales); layer outputs within
 |gpu - oracle| <= 1e-2 * max|oracle| + one bf16 ulp per element.  Tokens
 whose oracle top-8 has a near tie (adjacent scores within 1e-5; the pages
-note that a 352-expert top-8 router flips near-tied choices under tiny
-summation-order changes, "Step-5-Preview-Spark", Quality) accept either
+report that merely reordering the sums can change which of two nearly equal
+experts the top-8 keeps, "Step-5-Preview-Spark", Quality) accept either
 selection: their GPU ids must be a valid top-8 within 1e-5 of the oracle's
 scores, they are counted, and their layer output is compared with the oracle
 recomputed with the GPU's ids and weights.

@@ -1,13 +1,13 @@
 """Pins for the oracle's compressed scale format (CSF) encoder and decoder.
 
-"Step-5-Preview-NVFP4-Local", Format: fixed U8 [E, R/16, 16 * (1 + C/2)] (per
-16-row slab: 16 row bases, then each row's 4-bit codes, low nibble first),
-exceptions U32 (row * C + col) | byte << 24 grouped by expert and row-major,
-starts I64 [E + 1]; a byte is base + code unless an exception replaces it; a
-row's base is the lowest value 0..240 whose 16-value window covers the most of
-the row's bytes.  Size: the CSF planes of layers 3-87 take 51.44 % of the raw
-block scales.  Fidelity: every CSF tensor decodes, with an independent
-decoder, to the bytes it encodes.
+"Step-5-Preview-NVFP4-Local", Format: fixed U8 [E, R/16, 16 * (1 + C/2)] (each
+slab of 16 rows: their bases, then their 4-bit codes, lower nibble first),
+exceptions U32 (row * C + col) | byte << 24, expert by expert in increasing
+position, starts I64 [E + 1]; a byte is base + code unless an exception
+replaces it; a row's base is the smallest value in 0..240 whose 16-value window
+holds the largest number of the row's bytes.  Size: the CSF planes of layers 3-87 take 51.44 % of the raw
+block scales.  Fidelity: a second decoder, written separately, recovers from
+each CSF tensor exactly the scale bytes it was made from.
 """
 import os
 
@@ -101,7 +101,7 @@ def test_roundtrip_and_independent_decoder():
 def test_nvfp4_scales_roundtrip_and_per_expert_form():
     """Block scales from the NVFP4 quantiser at the gate/up (C = 256) and down
     (C = 96) widths; one expert encoded alone equals its slice of the fused
-    encoding (fixed[e] with exceptions[starts[e]:starts[e+1]])."""
+    encoding (its slab rows, and its span of the exceptions as starts delimits it)."""
     wl = syn.WORKLOADS[0]
     for which, R, C in (("gate", 64, 256), ("down", 32, 96)):
         mats = []

@@ -1,6 +1,6 @@
 """Pins for the oracle's quantisers and dequantisers.
 
-int4: "Step-5-Preview-Int4-g128", Recipe (RTN, 17 clip ratios in [0.60, 1.00],
+int4: "Step-5-Preview-Int4-g128", Recipe (RTN, seventeen clip ratios from 0.60 to 1.00,
 bf16 scales, error table) and Tensor layout.  NVFP4:
 "Step-5-Preview-NVFP4-Local", Modifications item 2, Format, Layers 88-90
 (NVFP4 weight NMSE) and Fidelity (packed matrices decode exactly to the

@@ -5,12 +5,14 @@
 //   fixed       u8  [E, R/16, 16 * (1 + C/2)]: per slab of 16 rows, the 16 row
 //               bases, then the rows' 4-bit codes in row order (C/2 bytes per
 //               row, column 2j in the low nibble of byte j, 2j + 1 in the high);
-//   exceptions  u32 [n]: (row * C + col) | byte << 24, grouped by expert,
-//               row-major within an expert;
-//   starts      i64 [E + 1]: expert e owns exceptions[starts[e], starts[e+1]).
-// A byte is its row's base plus its code unless an exception replaces it.  A
-// row's base is the lowest value 0..240 whose window [base, base + 15] holds
-// the most of the row's bytes; the code stored where an exception sits is 0.
+//   exceptions  u32 [n]: (row * C + col) | byte << 24; expert 0's entries
+//               first, then expert 1's and so on, each expert's in increasing
+//               position;
+//   starts      i64 [E + 1]: expert e's entries are exceptions[starts[e],
+//               starts[e+1]).
+// Decoding: byte = base(row) + code, or the stored byte of an exception.  A
+// row's base is the smallest b in 0..240 that puts the largest number of the
+// row's bytes inside [b, b + 15]; the code stored under an exception is 0.
 //
 // Decode (the serving-time step: one layer's scales are expanded into scratch
 // before the layer runs, or only the experts a batch routes to):

@@ -1,5 +1,5 @@
-// Sigmoid top-k router ("Step-5-Preview-Spark", At a glance: 352 routed
-// experts, top-8, sigmoid router).
+// Sigmoid top-k router ("Step-5-Preview-Spark", At a glance: a sigmoid router
+// keeps 8 of the 352 routed experts per token).
 //
 //   l[t,e] = sum_h x[t,h] * Wr[e,h] (+ bias[e])   fp32
 //   s      = 1 / (1 + exp(-l))                     fp32

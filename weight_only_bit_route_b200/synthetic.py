@@ -38,8 +38,8 @@ class Workload:
     skew_coef: float = 0.85
 
 
-# Step-5-Preview's MoE layer: hidden 4096, 352 routed experts, top-8, sigmoid
-# router, one shared expert, SwiGLU width 1536 (Step-5-Preview-Spark, At a
+# Step-5-Preview's MoE layer: hidden 4096, a sigmoid router keeping 8 of 352
+# routed experts, one shared expert, SwiGLU width 1536 (Step-5-Preview-Spark, At a
 # glance; "Step 5 Preview: 92 narrow layers...", The shape).
 WORKLOADS = {
     0: Workload("tiny_int4_T16_H1024_E32_F256", 16, 1024, 32, 256, 8, "int4", False,
