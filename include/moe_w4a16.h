@@ -374,9 +374,9 @@ int moe_quantize_nvfp4(const void* w, int64_t rows, int64_t cols, uint8_t* packe
 /* CSF ("Step-5-Preview-NVFP4-Local", Format): a scale tensor u8 [E, R, C]
  * (one E4M3 byte per 16 weights; gate/up R = 1536, C = 256, down R = 4096,
  * C = 96) is stored as
- *   fixed       u8 [E, R/16, 16 * (1 + C/2)]: per slab of 16 rows the 16 row
- *               bases, then each row's 4-bit codes (C/2 bytes per row, in row
- *               order; column 2j in the low nibble of byte j);
+ *   fixed       u8 [E, R/16, 16 * (1 + C/2)]: a slab of 16 rows is their 16
+ *               bases followed by their 4-bit codes (C/2 bytes per row, rows
+ *               in order; column 2j in the low nibble of byte j);
  *   exceptions  u32 [n]: (row * C + col) | byte << 24 (row counts from 0 in
  *               each expert); expert 0's entries first, then expert 1's and
  *               so on, each expert's in increasing position;
