@@ -463,6 +463,46 @@ def measure(moe, wl, x, layer, args, flush, stream, clk, pk, pk_kind, per_step=T
     return res, ms, ms_list, touched, launches, ws, graph
 
 
+def measure_csf(moe, wl, x, layer, steps, flush, stream, clk, pk, pk_kind):
+    """CSF scale expansion ("Step-5-Preview-NVFP4-Local", Format and Size) of the layer's NVFP4 block scales,
+    encoded once here: all experts of the three projections (one layer's scales before it runs) and only the
+    experts this workload routes to.  HBM-bound: the algorithmic bytes are the planes read (fixed, the
+    exceptions, starts) plus the scale bytes written, for the experts expanded."""
+    banks = (layer.gate, layer.up, layer.down)
+    planes = []
+    for bank in banks:
+        _, R, C = bank.scales.shape
+        f, e, s = moe.csf_encode(bank.scales)
+        planes.append((f, e, s, R, C, torch.empty_like(bank.scales)))
+    ws = moe.workspace(wl.T, wl.H, wl.E, wl.F, wl.k)
+    ids, _ = moe.route_topk(x, layer.router_w, layer.router_bias, wl.k, ws)
+    off, _, _ = moe.permute(ids, wl.E, ws)
+
+    def expand(offsets):
+        for f, e, s, R, C, out in planes:
+            moe.csf_decode(f, e, s, R, C, expert_offsets=offsets, out=out)
+
+    expand(None)
+    torch.cuda.synchronize()
+    exact = all(torch.equal(p[5], b.scales) for p, b in zip(planes, banks))
+    live = (off[1:] > off[:-1]).cpu().numpy()
+    bytes_all, bytes_routed = 0, 0
+    for f, e, s, R, C, out in planes:
+        st = s.cpu().numpy()
+        per_e = f[0].numel() + R * C + 16                      # fixed slab + scales written + starts pair
+        exc_e = (st[1:] - st[:-1]) * 4
+        bytes_all += int(f.shape[0] * per_e + exc_e.sum())
+        bytes_routed += int(live.sum() * per_e + exc_e[live].sum())
+    res = {"exact": bool(exact), "experts_routed": int(live.sum()), "kernel": "csf_expand + csf_patch, x3 projections",
+           "peak": pk["hbm_gbs"], "unit": "GB/s", "peak_source": f"{pk_kind} hbm_gbs"}
+    for name, offsets, nbytes in (("all_experts", None, bytes_all), ("routed_experts", off, bytes_routed)):
+        ms = float(np.mean(time_calls(lambda: expand(offsets), steps, flush, stream, clk)))
+        gbs = nbytes / (ms * 1e-3) / 1e9
+        res[name] = {"ms": round(ms, 5), "algorithmic_bytes": nbytes, "achieved": round(gbs, 1),
+                     "frac": round(gbs / pk["hbm_gbs"], 4)}
+    return res
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -562,6 +602,12 @@ def main():
                 lay.gate.input_scale = torch.full((w2.E,), W4A4_IN_GATEUP, dtype=torch.float32, device="cuda")
                 lay.down.input_scale = torch.full((w2.E,), W4A4_IN_DOWN, dtype=torch.float32, device="cuda")
             res = measure(moe, w2, x2, lay, args, flush, stream, clk, pk, pk_kind, fp4=w4a4, per_step=not f16)[0]
+            if c == "2":
+                # the scales of this NVFP4 layer through the compressed scale format's expansion
+                try:
+                    res["csf"] = measure_csf(moe, w2, x2, lay, args.steps, flush, stream, clk, pk, pk_kind)
+                except Exception as err:             # recorded, so that the rest of the line still prints
+                    res["csf"] = {"error": f"{type(err).__name__}: {err}"[:300]}
             if w4a4:
                 res["workload"] += " (W4A4: NVFP4 activations, static input scales)"
                 lay.gate.input_scale = lay.down.input_scale = None
