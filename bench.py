@@ -503,6 +503,39 @@ def measure_csf(moe, wl, x, layer, steps, flush, stream, clk, pk, pk_kind):
     return res
 
 
+def measure_ep_one_rank(moe, wl, x, layer, steps, flush, stream, clk):
+    """The expert-parallel layer (weight_only_bit_route_b200/ep.py) as a one-rank NCCL group: every step in the
+    library's kernels and the rows through NCCL's all-to-all, which on one rank is a local copy.  Its time
+    against the fused layer's is the cost of the split's bookkeeping (the host reads of the split sizes, the
+    exchanges, the per-rank grouping); its output must equal the fused layer's bit for bit."""
+    import datetime
+    import socket
+
+    import torch.distributed as dist
+
+    from weight_only_bit_route_b200 import ep
+    with socket.socket() as sk:
+        sk.bind(("127.0.0.1", 0))
+        port = sk.getsockname()[1]
+    dist.init_process_group("nccl", rank=0, world_size=1, init_method=f"tcp://127.0.0.1:{port}",
+                            timeout=datetime.timedelta(seconds=60))
+    try:
+        lay = ep.ExpertParallelMoE(layer.gate, layer.up, layer.down, layer.router_w, top_k=wl.k,
+                                   router_bias=layer.router_bias, shared=layer.shared, max_tokens=wl.T)
+        ws = moe.workspace(wl.T, wl.H, wl.E, wl.F, wl.k)
+        y_ref = moe.layer_decode(x, layer, ws)
+        y = lay.forward(x)
+        torch.cuda.synchronize()
+        exact = bool(torch.equal(y, y_ref))
+        ms_list = time_calls(lambda: lay.forward(x), steps, flush, stream, clk)
+        torch.cuda.synchronize()
+        return {"world": 1, "exact_vs_fused_layer": exact, "layer_ms": _pcts(ms_list),
+                "tokens_per_s": round(wl.T / (float(np.mean(ms_list)) * 1e-3), 1),
+                "note": "one rank: the all-to-all moves rows within this GPU; several GPUs are not measured"}
+    finally:
+        dist.destroy_process_group()
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -640,6 +673,13 @@ def main():
         "clocks": clk.summary(),
         "per_config": per_config,
     }
+    if world == 1 and T <= 64:
+        # the expert-parallel split of the same layer, on one rank (recorded, so that an error cannot drop the line)
+        try:
+            line["expert_parallel"] = measure_ep_one_rank(moe, wl, x, layer, min(args.steps, 50), flush, stream,
+                                                          ClockSampler(local_rank))
+        except Exception as err:
+            line["expert_parallel"] = {"error": f"{type(err).__name__}: {err}"[:300]}
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         line["cpu_baseline"] = cpu_baseline(wl, moe, x, layer)
     if rank == 0:
