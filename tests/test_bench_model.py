@@ -8,6 +8,8 @@ checked against things other than its own formulas:
   scale per 16 inputs, an fp32 weight_scale_2), counted by hand below;
 - the FLOPs are the layer's matrix products counted by brute force on a tiny layer (one multiply-add per weight
   and routed row), and the full-size figure is the same count written out.
+- the CSF leg's bytes are the encoded planes and the expanded scales of the experts it expands, counted from the
+  oracle's encoding of a tiny layer.
 """
 import dataclasses
 
@@ -80,3 +82,54 @@ def test_prefill_flops_by_hand():
     assert bench.layer_flops(syn.WORKLOADS[3]) == T * per_token
     # the gate/up call alone: 2 projections x 2 FLOPs x F x H per routed row, 8T rows
     assert 2 * 2 * F * H * k * T == 412_316_860_416
+
+
+def test_csf_expansion_bytes(monkeypatch):
+    """The bench's CSF leg counts, per expert expanded, its fixed slab bytes, its exceptions (4 bytes each), its
+    pair of starts and the scale bytes it writes.  Run on a tiny layer with the oracle's encoder and decoder
+    standing in for the library (the accounting, not the kernels, is under test)."""
+    import types
+
+    import torch
+
+    rng = np.random.default_rng(5)
+    E, R, C, k = 6, 32, 64, 2
+    wl = dataclasses.replace(syn.WORKLOADS[0], T=3, E=E, k=k)
+    banks = [types.SimpleNamespace(scales=torch.from_numpy(rng.integers(0x30, 0x50, size=(E, R, C), dtype=np.uint8)))
+             for _ in range(3)]
+    layer = types.SimpleNamespace(gate=banks[0], up=banks[1], down=banks[2], router_w=None, router_bias=None)
+    ids = torch.tensor([[0, 2], [2, 5], [0, 5]], dtype=torch.int32)            # experts 0, 2, 5 routed
+
+    def csf_encode(sc):
+        f, e, s = oracle.csf_encode(sc.numpy())
+        return torch.from_numpy(f), torch.from_numpy(e.view(np.int32)), torch.from_numpy(s)
+
+    def csf_decode(f, e, s, R_, C_, expert_offsets=None, out=None):
+        full = torch.from_numpy(oracle.csf_decode(f.numpy(), e.numpy().view(np.uint32), s.numpy(), R_, C_))
+        o = None if expert_offsets is None else expert_offsets.numpy()
+        for ee in range(f.shape[0]):
+            if o is None or o[ee + 1] > o[ee]:
+                out[ee].copy_(full[ee])
+        return out
+
+    def permute(ids_, E_, ws):
+        off, rs, sr = oracle.permute(ids_.numpy(), E_)
+        return torch.from_numpy(off), torch.from_numpy(rs), torch.from_numpy(sr)
+
+    fake = types.SimpleNamespace(csf_encode=csf_encode, csf_decode=csf_decode, permute=permute,
+                                 route_topk=lambda *a: (ids, None), workspace=lambda *a: None)
+    monkeypatch.setattr(bench, "time_calls", lambda fn, steps, *a, **kw: [fn() or 1.0 for _ in range(steps)])
+    monkeypatch.setattr(torch.cuda, "synchronize", lambda: None)
+    res = bench.measure_csf(fake, wl, None, layer, 2, None, None, None, {"hbm_gbs": 1000.0}, "test")
+    assert res["exact"] and res["experts_routed"] == 3
+    want_all, want_routed = 0, 0
+    for b in banks:
+        f, e, s = oracle.csf_encode(b.scales.numpy())
+        n_exc = np.diff(s)
+        per = [f[x].nbytes + 4 * int(n_exc[x]) + 16 + R * C for x in range(E)]
+        want_all += sum(per)
+        want_routed += per[0] + per[2] + per[5]
+    assert res["all_experts"]["algorithmic_bytes"] == want_all
+    assert res["routed_experts"]["algorithmic_bytes"] == want_routed
+    # 1 ms per call: achieved GB/s is bytes / 1e6
+    assert res["all_experts"]["achieved"] == round(want_all / 1e6, 1)
