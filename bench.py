@@ -503,11 +503,12 @@ def measure_csf(moe, wl, x, layer, steps, flush, stream, clk, pk, pk_kind):
     return res
 
 
-def measure_ep_one_rank(moe, wl, x, layer, steps, flush, stream, clk):
+def measure_ep_one_rank(moe, wl, x, layer, steps, flush, stream, clk, backend="nccl", ops=None):
     """The expert-parallel layer (weight_only_bit_route_b200/ep.py) as a one-rank NCCL group: every step in the
     library's kernels and the rows through NCCL's all-to-all, which on one rank is a local copy.  Its time
     against the fused layer's is the cost of the split's bookkeeping (the host reads of the split sizes, the
-    exchanges, the per-rank grouping); its output must equal the fused layer's bit for bit."""
+    exchanges, the per-rank grouping); its output must equal the fused layer's bit for bit.  backend and ops
+    exist for a CPU test of this function (gloo, the oracle's steps)."""
     import datetime
     import socket
 
@@ -517,11 +518,11 @@ def measure_ep_one_rank(moe, wl, x, layer, steps, flush, stream, clk):
     with socket.socket() as sk:
         sk.bind(("127.0.0.1", 0))
         port = sk.getsockname()[1]
-    dist.init_process_group("nccl", rank=0, world_size=1, init_method=f"tcp://127.0.0.1:{port}",
+    dist.init_process_group(backend, rank=0, world_size=1, init_method=f"tcp://127.0.0.1:{port}",
                             timeout=datetime.timedelta(seconds=60))
     try:
         lay = ep.ExpertParallelMoE(layer.gate, layer.up, layer.down, layer.router_w, top_k=wl.k,
-                                   router_bias=layer.router_bias, shared=layer.shared, max_tokens=wl.T)
+                                   router_bias=layer.router_bias, shared=layer.shared, max_tokens=wl.T, ops=ops)
         ws = moe.workspace(wl.T, wl.H, wl.E, wl.F, wl.k)
         y_ref = moe.layer_decode(x, layer, ws)
         y = lay.forward(x)

@@ -271,3 +271,48 @@ def test_expert_parallel_argument_checks():
             layer.forward(torch.zeros(5, 128, dtype=torch.bfloat16))
     finally:
         dist.destroy_process_group()
+
+
+def test_bench_expert_parallel_leg_runs_on_cpu(monkeypatch):
+    """bench.py's one-rank expert-parallel leg, run over gloo with the oracle's steps (its GPU run uses NCCL and
+    the library): it initialises and releases its group, times the calls and compares with the fused layer,
+    here the same steps composed on one process, bit for bit."""
+    import bench
+    import oracle
+    from problems import build
+    from weight_only_bit_route_b200 import synthetic as syn
+
+    wl = syn.WORKLOADS[0]
+    P = build(0, "random", experts=list(range(wl.E)), shared=True)
+    ops = RefOps(oracle, P, 0, wl.E)
+    x = _from_bits(syn.gen_x(wl, seed=7, T=5))
+
+    def fused(x_, layer_, ws_):
+        T = x_.shape[0]
+        ids, w = ops.route(x_)
+        off, rs, sr = ops.group(torch.zeros(T, wl.k, dtype=torch.int32), 1)
+        rows = rs.to(torch.int64)
+        ys = ops.experts(x_.index_select(0, rows // wl.k), ids.view(-1)[rows], w.view(-1)[rows])
+        return ops.combine(ys, sr, T, ops.shared_expert(x_))
+
+    class _Bank:
+        E = wl.E
+
+    layer = type("L", (), {"gate": _Bank(), "up": _Bank(), "down": _Bank(), "router_w": torch.from_numpy(P.Wr),
+                           "router_bias": None, "shared": None})()
+    fake = type("M", (), {"workspace": staticmethod(lambda *a: None), "layer_decode": staticmethod(fused)})
+    def one_ms_each(fn, steps, *a, **kw):
+        out = []
+        for _ in range(steps):
+            fn()
+            out.append(1.0)
+        return out
+
+    monkeypatch.setattr(bench, "time_calls", one_ms_each)
+    monkeypatch.setattr(torch.cuda, "synchronize", lambda: None)
+    wl5 = syn.Workload(wl.name, 5, wl.H, wl.E, wl.F, wl.k, wl.fmt, True, wl.router_std, False)
+    res = bench.measure_ep_one_rank(fake, wl5, x, layer, 2, None, None, None, backend="gloo", ops=ops)
+    assert res["exact_vs_fused_layer"] is True
+    assert res["world"] == 1 and res["tokens_per_s"] > 0
+    import torch.distributed as dist
+    assert not dist.is_initialized()
