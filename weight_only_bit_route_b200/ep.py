@@ -7,7 +7,8 @@ replicated, and rank r owns the routed experts [r * E / N, (r + 1) * E / N).  Pe
 
     1. route the rank's tokens (moe_route_topk);
     2. group the T * top_k slots by owning rank (moe_permute with the ranks as the buckets);
-    3. all-to-all: each slot's token row, its expert (local to the owner) and its routing weight go to the owner;
+    3. all-to-all: each slot's token row, its expert (local to the owner) and its routing weight go to the owner,
+       as one record per slot;
     4. the owner runs its experts on the rows it received, as a batch of single-slot tokens (moe_permute by local
        expert, moe_grouped_w4a16_swiglu, moe_grouped_w4a16_down with the weight by row, moe_unpermute_combine with
        top_k = 1, which puts the rows back in the order received);
@@ -126,15 +127,19 @@ class ExpertParallelMoE:
             raise ValueError(f"rank(s) {[r for r in range(world) if rc[r] < 0]} refused a batch above max_tokens")
         R = int(sum(rc))
         order_l = order.to(torch.int64)
-        # rows travel as bytes, expert and weight bits as one int32 pair per row
-        send_x = x.index_select(0, torch.div(order_l, k, rounding_mode="floor")).contiguous()
+        # one exchange for rows and their metadata: each record is the token row's bytes followed by the
+        # slot's local expert and routing weight bits (an int32 pair)
+        nb = H * x.element_size()
         meta = torch.stack([ids.view(-1).index_select(0, order_l) - owner.view(-1).index_select(0, order_l)
                             * self.e_per_rank,
-                            w.view(-1).index_select(0, order_l).view(torch.int32)], dim=1).contiguous()
-        recv_x = torch.empty(R, H, dtype=x.dtype, device=dev)
-        recv_meta = torch.empty(R, 2, dtype=torch.int32, device=dev)
-        self._a2a(recv_x.view(torch.uint8), send_x.view(torch.uint8), rc, sc)
-        self._a2a(recv_meta, meta, rc, sc)
+                            w.view(-1).index_select(0, order_l).view(torch.int32)], dim=1)
+        send = torch.empty(order_l.numel(), nb + 8, dtype=torch.uint8, device=dev)
+        send[:, :nb] = x.index_select(0, torch.div(order_l, k, rounding_mode="floor")).view(torch.uint8)
+        send[:, nb:] = meta.contiguous().view(torch.uint8)
+        recv = torch.empty(R, nb + 8, dtype=torch.uint8, device=dev)
+        self._a2a(recv, send, rc, sc)
+        recv_x = recv[:, :nb].contiguous().view(x.dtype)
+        recv_meta = recv[:, nb:].contiguous().view(torch.int32)
         er = recv_meta[:, 0].contiguous()
         wr = recv_meta[:, 1].contiguous().view(torch.float32)
         y_recv = self.ops.experts(recv_x, er, wr)                    # [R, H], received order
