@@ -17,10 +17,11 @@ replicated, and rank r owns the routed experts [r * E / N, (r + 1) * E / N).  Pe
        (slot -> position in the returned rows): y[t] = shared[t] + sum_j of token t's returned rows.
 
 Every step of the layer runs in the library's kernels; this module marshals arguments and moves rows between
-ranks with torch.distributed (NCCL over NVLink on GPUs, gloo on CPU).  The send buffer is gathered, and the
-(expert, weight) pairs packed, with torch indexing: data movement for the exchange, no arithmetic of the layer.  The collective is the stock all-to-all:
-rows cross the fabric once each way, and no multicast of any kind is used.  Each row's result is independent of
-which other rows share its tile, so on one rank the layer reproduces moe_layer_decode bit for bit.
+ranks with torch.distributed (NCCL over NVLink on GPUs, gloo on CPU).  The send records are gathered, and the
+(expert, weight) pairs appended, with torch indexing: data movement for the exchange, no arithmetic of the
+layer.  The collective is the stock all-to-all: rows cross the fabric once each way, and no multicast of any
+kind is used.  Each row's result is independent of which other rows share its tile, so on one rank the layer
+reproduces moe_layer_decode bit for bit.
 
 The split sizes of an all-to-all are host values, so each call reads the per-rank slot counts back to the host
 once (after step 2) and the returned counts once (after the counts' exchange).  A rank whose batch is above
