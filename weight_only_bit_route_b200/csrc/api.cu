@@ -190,11 +190,22 @@ int layer_run(const void* x, int T, const moe_layer* L, void* y, void* ws, cudaS
     // them.
     SideStream* side = nullptr;
     std::unique_lock<std::mutex> side_lock;
+    // An error return after the fork still joins the side stream back into `s` (and so into a recording
+    // in progress), before the lock is released; the normal path joins explicitly and disarms it.
+    struct JoinOnExit {
+        SideStream* side = nullptr;
+        cudaStream_t s = nullptr;
+        ~JoinOnExit() {
+            if (side && cudaEventRecord(side->join, side->s) == cudaSuccess) cudaStreamWaitEvent(s, side->join, 0);
+        }
+    } join_on_exit;
     if (has_sh) {
         MOE_TRY(side_stream(&side));
         side_lock = std::unique_lock<std::mutex>(side->call);
         if (cudaEventRecord(side->fork, s) != cudaSuccess || cudaStreamWaitEvent(side->s, side->fork, 0) != cudaSuccess)
             return MOE_ERR_CUDA;
+        join_on_exit.side = side;
+        join_on_exit.s = s;
     }
 
     if (T <= kRouterDecodeMaxT && router_decode_ok(H)) {
@@ -273,6 +284,7 @@ int layer_run(const void* x, int T, const moe_layer* L, void* y, void* ws, cudaS
         MOE_TRY(launch_shared_routing(T, k, sh_off, sh_rs, side->s));
         MOE_TRY(run_problem(sg, true, T, T, nullptr, direct, shpart, side->s));
         MOE_TRY(run_problem(sd, false, T, T, nullptr, direct, shpart, side->s));
+        join_on_exit.side = nullptr;
         if (cudaEventRecord(side->join, side->s) != cudaSuccess) return MOE_ERR_CUDA;
     }
     if (has_sh && cudaStreamWaitEvent(s, side->join, 0) != cudaSuccess) return MOE_ERR_CUDA;
