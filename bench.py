@@ -13,7 +13,10 @@ expert.  The other workloads (NVFP4 decode, int4 prefill T = 2048, NVFP4
 prefill T = 8192 with Zipf-skewed routing) go into `per_config` on the same
 line, each with its layer time (mean, median, p10, p90), its dominant-kernel
 roofline, its whole-layer roofline and the time of each step through its own
-C-ABI call.  Weights are bf16 N(0, 0.02^2) drawn on the GPU and converted by
+C-ABI call; the NVFP4 decode workload also carries the CSF expansion of its
+layer's scales (`csf`).  With one process, `expert_parallel` times the same
+layer split by experts over a one-rank NCCL group.  Weights are bf16
+N(0, 0.02^2) drawn on the GPU and converted by
 the library's quantisers; activations bf16 N(0, 1); router fp32 N(0, 1/4096).
 L2 is flushed (256 MB write) before every timed call; each call is timed with
 CUDA events on the launching stream and the flush is outside the events.
