@@ -34,6 +34,7 @@
 #include <cuda_fp16.h>
 
 #include <algorithm>
+#include <mutex>
 
 #include "moe_internal.cuh"
 
@@ -848,20 +849,32 @@ static cudaError_t launch_ex(K kern, dim3 grid, dim3 block, size_t smem, cudaStr
 
 template <int FMT>
 static cudaError_t launch_sv(const SvArgs& a, size_t smem, cudaStream_t s, bool pdl) {
-    static int sms = 0;
-    static size_t smem_set = 0;
+    // per device (a kernel's shared memory limit is a per-device attribute): the SM count, read once, and
+    // the dynamic shared memory granted so far, raised under a lock when a call needs more
+    struct Dev {
+        std::once_flag once;
+        int sms = 0;
+        std::mutex mu;
+        size_t granted = 0;
+    };
+    static Dev devs[64];
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return cudaErrorInvalidDevice;
+    Dev& d = devs[dev];
+    std::call_once(d.once, [&] {
+        if (cudaDeviceGetAttribute(&d.sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) d.sms = 0;
+    });
+    if (d.sms <= 0) return cudaErrorInvalidDevice;
     auto k = stream_gemv<FMT>;
-    if (sms == 0) {
-        int dev = 0;
-        cudaGetDevice(&dev);
-        cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+    {
+        std::lock_guard<std::mutex> lock(d.mu);
+        if (smem > d.granted) {
+            cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem));
+            if (e != cudaSuccess) return e;
+            d.granted = smem;
+        }
     }
-    if (smem > smem_set) {
-        cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem));
-        if (e != cudaSuccess) return e;
-        smem_set = smem;
-    }
-    return launch_ex(k, dim3(sms), dim3(SV_THREADS), smem, s, pdl, a);
+    return launch_ex(k, dim3(d.sms), dim3(SV_THREADS), smem, s, pdl, a);
 }
 
 int launch_stream_gemv(const GemvProblem& routed, const GemvProblem* shared, bool gateup, int act_rows,
