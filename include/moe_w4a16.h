@@ -56,6 +56,11 @@
  *     the layer entries the whole of moe_workspace_bytes().  A workspace of
  *     moe_workspace_bytes(T, H, E, F, top_k) bytes serves every call at those
  *     sizes.  Calls that share a workspace must not run concurrently.
+ *   - Host threads: calls from several threads are safe when they use separate
+ *     workspaces (moe_permute_noalloc excepted: its calls share one scratch
+ *     array).  The library's launch-time state (per-device kernel attributes,
+ *     the shared expert's side stream) is taken under locks; no lock is held
+ *     while the GPU is waited on.
  */
 #ifndef MOE_W4A16_H
 #define MOE_W4A16_H

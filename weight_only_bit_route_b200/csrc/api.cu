@@ -59,6 +59,16 @@ int check_ws(void* ws, size_t ws_bytes, size_t need) {
 // stream spreads over the GPU; partial is split_bytes() of scratch for that.
 bool gemm_shape_ok(int in_dim, int out_dim) { return in_dim % 256 == 0 && out_dim % 128 == 0; }
 
+// The grouped GEMM raises its kernel's shared-memory attribute the first time a launch needs more; two host
+// threads doing that at once for one kernel could leave the smaller value set last.  Every grouped GEMM
+// launch of this library is therefore made under one process-wide lock (host launch work only: nothing
+// waits on the GPU while it is held).
+int grouped_gemm(const GemvProblem& p, bool gateup, int rows, const GemmBuffers& b, cudaStream_t s) {
+    static std::mutex mu;
+    std::lock_guard<std::mutex> lock(mu);
+    return launch_grouped_gemm(p, gateup, rows, b, s);
+}
+
 int run_problem(const GemvProblem& p, bool gateup, int rows, int act_rows, void* prep, const GemmBuffers& gb,
                 float* partial, cudaStream_t s) {
     if (!gemm_shape_ok(p.in_dim, p.out_dim)) {
@@ -69,7 +79,7 @@ int run_problem(const GemvProblem& p, bool gateup, int rows, int act_rows, void*
     b.ksplit = shared_ksplit(p.E, p.fmt, gateup, rows, p.in_dim);
     b.partial = partial;
     b.tile_cnt = p.status + 16;            // the control block's split-K counters
-    return launch_grouped_gemm(p, gateup, rows, b, s);
+    return grouped_gemm(p, gateup, rows, b, s);
 }
 
 // The step-level calls' scratch: the GEMV or GEMM pre-pass of rows rows, then
@@ -244,7 +254,7 @@ int layer_run(const void* x, int T, const moe_layer* L, void* y, void* ws, cudaS
         gb.sched = status + 8;             // tiles handed out as CTAs get SMs (the shared expert may hold some)
         gb.max_expert_rows = T;            // a token routes to an expert at most once
         if (!i8) gb.act_buf = y_perm;
-        MOE_TRY(launch_grouped_gemm(gu, true, R, gb, s));
+        MOE_TRY(grouped_gemm(gu, true, R, gb, s));
     } else {
         MOE_TRY(launch_stream_gemv(gu, nullptr, true, T, prep, s, true));
     }
@@ -252,7 +262,7 @@ int layer_run(const void* x, int T, const moe_layer* L, void* y, void* ws, cudaS
         GemmBuffers db = gemm_buffers(prep, R, F, false, i8);
         db.sched = status + 8;
         db.max_expert_rows = T;
-        MOE_TRY(launch_grouped_gemm(dn, false, R, db, s));
+        MOE_TRY(grouped_gemm(dn, false, R, db, s));
     } else {
         MOE_TRY(launch_stream_gemv(dn, nullptr, false, R, prep, s, true));
     }
