@@ -11,6 +11,7 @@
 // GEMM above) and a warp-per-token kernel for the sigmoid, selection and
 // renormalisation.
 #include <algorithm>
+#include <mutex>
 
 #include "moe_internal.cuh"
 
@@ -429,6 +430,10 @@ int launch_route_decode(const RouterDecodeArgs& a, cudaStream_t s) {
     const size_t smem = std::max<size_t>(size_t(a.T) * a.H * 2, (size_t(a.T) * a.E + size_t(a.E) + size_t(a.T) * a.k) * 4);
     if (a.T > RD_TMAX || a.H % 512) return MOE_ERR_UNSUPPORTED;
     auto k = a.x_f16 ? router_decode<true> : router_decode<false>;
+    // the attribute is set to this call's size and the launch follows under one lock, so that another host
+    // thread cannot lower it in between
+    static std::mutex mu;
+    std::lock_guard<std::mutex> lock(mu);
     if (smem > 48 * 1024 &&
         cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem)) != cudaSuccess)
         return MOE_ERR_UNSUPPORTED;
