@@ -28,7 +28,7 @@
  *           the 16-value window holding the largest share of its bytes) and
  *           Size.
  *
- * Readings where the pages are silent (each listed in the design notes):
+ * Readings where the pages are silent:
  *   - int4: divisor 7 with clamp [-8, 7]; ratios r_i = (24 + i) / 40, i = 0..16;
  *     candidate scale bf16_rne((r_i * amax) / 7) in fp32; rounding error
  *     sum (q*s - w)^2 accumulated in fp32 in index order; ties keep the larger

@@ -7,8 +7,8 @@ largest |x| in [2^13, 2^14); then every bf16 element within 2^27 of that largest
 the scaling.  The NVFP4 weights: an e2m1 value times an E4M3 block scale is an f16 value exactly (at most 5
 significant bits, magnitudes from 2^-10 to 2688).
 
-(These are the readings "int4 products on the 16-bit tensor cores" in the design notes; the kernel itself is
-compared with the oracle by the GPU parity tests.)
+(These are the exactness readings the 16-bit path is built on; the kernel itself is compared with the oracle by
+the GPU parity tests.)
 """
 import numpy as np
 

@@ -10,8 +10,8 @@ per digit the s32 sums A_i = sum(u * d_i) with u = q + 8 the stored nibble, and 
 - the recombination equals sum(q * X) exactly;
 - X = x * 2^c exactly for every element with |x| >= M * 2^-13, and |X - x * 2^c| <= M * 2^-22 * 2^c otherwise.
 
-(This is the reading "int4 products on the 8-bit tensor cores" in the design notes; the kernel itself is compared
-with the oracle by the GPU parity tests.)
+(This is the exactness reading the 8-bit path is built on; the kernel itself is compared with the oracle by the
+GPU parity tests.)
 """
 import numpy as np
 
