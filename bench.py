@@ -638,13 +638,17 @@ def main():
                 # amax / (6 * 448) (x ~ N(0, 1) over 4096 elements; h of these weights stays below ~8)
                 lay.gate.input_scale = torch.full((w2.E,), W4A4_IN_GATEUP, dtype=torch.float32, device="cuda")
                 lay.down.input_scale = torch.full((w2.E,), W4A4_IN_DOWN, dtype=torch.float32, device="cuda")
-            res = measure(moe, w2, x2, lay, args, flush, stream, clk, pk, pk_kind, fp4=w4a4, per_step=not f16)[0]
-            if c == "2":
-                # the scales of this NVFP4 layer through the compressed scale format's expansion
-                try:
-                    res["csf"] = measure_csf(moe, w2, x2, lay, args.steps, flush, stream, clk, pk, pk_kind)
-                except Exception as err:             # recorded, so that the rest of the line still prints
-                    res["csf"] = {"error": f"{type(err).__name__}: {err}"[:300]}
+            try:
+                res = measure(moe, w2, x2, lay, args, flush, stream, clk, pk, pk_kind, fp4=w4a4,
+                              per_step=not f16)[0]
+                if c == "2":
+                    # the scales of this NVFP4 layer through the compressed scale format's expansion
+                    try:
+                        res["csf"] = measure_csf(moe, w2, x2, lay, args.steps, flush, stream, clk, pk, pk_kind)
+                    except Exception as err:         # recorded, so that the rest of the line still prints
+                        res["csf"] = {"error": f"{type(err).__name__}: {err}"[:300]}
+            except Exception as err:                 # one workload's failure is recorded, not fatal to the line
+                res = {"workload": describe(w2), "error": f"{type(err).__name__}: {err}"[:300]}
             if w4a4:
                 res["workload"] += " (W4A4: NVFP4 activations, static input scales)"
                 lay.gate.input_scale = lay.down.input_scale = None
