@@ -481,45 +481,6 @@ def test_layer_graph_matches_eager(cfg):
     g.close()
 
 
-def test_layer_decode_from_two_host_threads():
-    """Two host threads call moe_layer_decode at the same time, each on its own stream and workspace (the
-    library releases the interpreter lock during a call; the shared expert's side stream is one per device,
-    taken under a lock from its fork to its join): every call reproduces the one-thread result bit for bit."""
-    import threading
-    P = build(1, "random")
-    L = device_layer(moe, P)
-    x = dev_bf16(P.x)
-    ref = moe.layer_decode(x, L, _ws(P.T, P.wl)).clone()
-    torch.cuda.synchronize()
-    outs, errors = [[], []], []
-
-    def worker(i):
-        try:
-            s = torch.cuda.Stream()
-            with torch.cuda.stream(s):
-                ws = _ws(P.T, P.wl)
-                for _ in range(20):
-                    outs[i].append(moe.layer_decode(x, L, ws))
-                if moe.read_status(ws) != 0:
-                    errors.append(f"thread {i}: device status set")
-            s.synchronize()
-        except Exception as e:          # reported below, in the test's own thread
-            errors.append(f"thread {i}: {e!r}")
-
-    threads = [threading.Thread(target=worker, args=(i,)) for i in range(2)]
-    for t in threads:
-        t.start()
-    for t in threads:
-        t.join(timeout=300)
-    assert not any(t.is_alive() for t in threads), "a layer call did not return"
-    assert not errors, errors
-    torch.cuda.synchronize()
-    for i in range(2):
-        assert len(outs[i]) == 20
-        bad = [j for j, y in enumerate(outs[i]) if not torch.equal(y, ref)]
-        assert not bad, f"thread {i}: calls {bad} differ from the one-thread result"
-
-
 def test_layer_T0_is_noop():
     P = build(0, "quantised")
     L = device_layer(moe, P)
