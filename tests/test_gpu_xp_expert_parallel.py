@@ -1,5 +1,5 @@
 """Expert-parallel layer on one GPU (a one-rank NCCL group): every step in the library's kernels, the rows through
-the NCCL all-to-all.  With one rank every expert is local, and each row's result does not depend on the rows
+the NCCL all-to-all (collected after the single-GPU parity suites).  With one rank every expert is local, and each row's result does not depend on the rows
 that share its tile, so the layer must reproduce moe_layer_decode bit for bit."""
 import socket
 
