@@ -4,6 +4,7 @@ failing under `-x` cannot keep the rest from running.
 - The compressed scale format at the size the benchmark expands: all 352 experts of one projection at the pages'
   shapes ("Step-5-Preview-NVFP4-Local", Format and Size), against the oracle's planes and the input bytes.
 - Layer calls from two host threads at once, each on its own stream and workspace: bit-identical to one thread.
+- Recording a layer as a graph launches nothing, so it adds nothing to the library's launch count.
 """
 import numpy as np
 import pytest
@@ -95,3 +96,22 @@ def test_layer_decode_from_two_host_threads():
         assert len(outs[i]) == 20
         bad = [j for j, y in enumerate(outs[i]) if not torch.equal(y, ref)]
         assert not bad, f"thread {i}: calls {bad} differ from the one-thread result"
+
+
+def test_graph_recording_adds_no_launches():
+    """moe_layer_graph_create records the layer's launches without running them: the launch count is the same
+    before and after it, and one replay adds the recorded kernels (nine for the decode layer with a shared
+    expert)."""
+    P = build(1, "random")
+    L = device_layer(moe, P)
+    x = dev_bf16(P.x)
+    ws = _ws(P.T, P.wl)
+    torch.cuda.synchronize()
+    n_rec = moe.launch_count()
+    g = moe.LayerGraph(x, L, ws)
+    assert moe.launch_count() == n_rec
+    g.launch()
+    torch.cuda.synchronize()
+    assert moe.launch_count() - n_rec == 9
+    assert moe.read_status(ws) == 0
+    g.close()
